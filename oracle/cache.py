@@ -1,0 +1,88 @@
+"""LRU refinement cache (oracle; test infrastructure).
+
+StrataFlux caches fetched precision on the GPU and reuses it across decode
+steps (arXiv 2611.08363 abstract; rag-lover.com explainer, TL;DR and 解説
+sections).  The pages give no policy, so this module takes an LRU reading.
+One cache per weight matrix holds up to C units (a unit is one input
+column's refinement bits).  At step t, given the ascending selected set S:
+
+C1  hits H = S ∩ cached; misses M = S \\ H.
+C2  every hit gets last_use = t.
+C3  slots for misses come first from free slots, lowest slot index first,
+    then from victims: cached units not in S, ordered by (last_use
+    ascending, unit ascending).
+C4  misses take those slots in ascending unit order until none are left; the
+    misses left over form the bypass set: fetched for this step only, never
+    cached.
+C5  every inserted unit gets last_use = t; then t advances by one.
+C6  for weights the correction always uses all of S (every fetch completes
+    before use), so the GEMV result does not depend on cache state; what is
+    compared is the hit / miss / bypass sets and the slot each unit lands in.
+
+``preload`` fills an empty cache with the given units in slots 0, 1, ...
+with last_use = -1 (older than any step), and counts nothing.
+"""
+
+from __future__ import annotations
+
+
+class LRUCache:
+    def __init__(self, num_units: int, capacity: int):
+        if capacity < 0 or num_units < 0:
+            raise ValueError("negative size")
+        self.num_units = num_units
+        self.capacity = capacity
+        self.slot_of: dict[int, int] = {}
+        self.last_use: dict[int, int] = {}
+        self.free: list[int] = list(range(capacity))
+        self.t = 0
+        self.hits = self.misses = self.bypass = 0
+
+    def preload(self, units) -> None:
+        units = list(units)
+        if self.slot_of or len(units) > self.capacity or len(set(units)) != len(units):
+            raise ValueError("preload needs an empty cache and at most C distinct units")
+        for u in units:
+            if not 0 <= u < self.num_units:
+                raise ValueError("unit out of range")
+            slot = self.free.pop(0)
+            self.slot_of[u] = slot
+            self.last_use[u] = -1
+
+    def step(self, S) -> dict:
+        S = [int(u) for u in S]
+        if S != sorted(set(S)):
+            raise ValueError("S must be strictly ascending")
+        t = self.t
+        in_S = set(S)
+        H = [u for u in S if u in self.slot_of]                       # C1
+        M = [u for u in S if u not in self.slot_of]
+        for u in H:                                                    # C2
+            self.last_use[u] = t
+        victims = sorted((u for u in self.slot_of if u not in in_S),  # C3
+                         key=lambda u: (self.last_use[u], u))
+        free_sorted = sorted(self.free)
+        avail = [("free", s, None) for s in free_sorted] + [("victim", self.slot_of[v], v) for v in victims]
+        inserted, bypass = [], []
+        for i, u in enumerate(M):                                      # C4
+            if i >= len(avail):
+                bypass.append(u)
+                continue
+            kind, slot, old = avail[i]
+            if kind == "victim":
+                del self.slot_of[old]
+                del self.last_use[old]
+            else:
+                self.free.remove(slot)
+            self.slot_of[u] = slot
+            self.last_use[u] = t                                       # C5
+            inserted.append((u, slot))
+        self.t = t + 1
+        self.hits += len(H)
+        self.misses += len(M)
+        self.bypass += len(bypass)
+        return dict(hits=H, misses=M, bypass=bypass, inserted=inserted)
+
+    def snapshot(self) -> dict[int, int]:
+        """unit -> slot for every cached unit."""
+        return dict(self.slot_of)
