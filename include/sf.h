@@ -1,0 +1,273 @@
+/*
+ * sf.h -- selective precision streaming for low-bit LLM decoding (StrataFlux),
+ * the data-parallel hot path, as a C ABI.
+ *
+ * The method ("StrataFlux: Memory-Hierarchy-Native Low-Bit LLM Inference",
+ * arXiv 2611.08363, abstract; rag-lover.com explainer, sections TL;DR and
+ * 解説) keeps low-bit weights and KV resident on the GPU and streams only the
+ * extra low-order bits ("nested refinement") of the weight columns with the
+ * largest input activations and of the tokens with the largest attention
+ * weight as seen through the low-bit keys.  Fetched refinements are cached
+ * on the GPU and reused across decode steps; misses come from pinned host
+ * memory on a side stream, overlapped with compute.
+ *
+ * Conventions for every entry point
+ *  - Returns sf_status; SF_OK is 0.  On any other value nothing was enqueued
+ *    and sf_last_error() gives a message for the calling thread.  No C++
+ *    exception crosses this boundary.
+ *  - Device buffers are owned by the caller, stay owned by the caller, and
+ *    must stay valid until the work enqueued on the given stream completes.
+ *    Handles (sf_refine_cache) own their internals and free them in *_destroy.
+ *  - Work is asynchronous on the given CUDA stream (NULL = legacy default
+ *    stream) unless stated otherwise.  Shapes are checked on the host;
+ *    data-dependent errors found on the device are reported through device
+ *    outputs as stated per call.
+ *  - bf16 and fp16 values are passed as their 16-bit patterns (uint16_t).
+ *  - Packed codes are little-endian bitstreams in uint32 words: a stream's
+ *    bit t is bit (t mod 32) of word t/32, and code j of a b-bit stream
+ *    occupies stream bits [b*j, b*j + b).
+ */
+#ifndef SF_H
+#define SF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sf_stream_t; /* a cudaStream_t */
+
+typedef enum sf_status {
+  SF_OK = 0,
+  SF_EINVAL = 1,    /* an argument or shape is outside the contract */
+  SF_ENOMEM = 2,    /* a library-owned allocation failed */
+  SF_ECUDA = 3,     /* a CUDA runtime call failed (message has the CUDA error) */
+  SF_ETIMEOUT = 4,  /* a bounded wait expired */
+  SF_ENOTIMPL = 5   /* combination not implemented */
+} sf_status;
+
+/* Refinement-code layouts of sf_quantize_nested. */
+#define SF_REF_BY_COLUMN 0 /* weights: ref [K][N*b_f/32], one column per row of words */
+#define SF_REF_BY_ROW 1    /* KV:      ref [N][K*b_f/32], same layout as resident codes */
+
+/* Library version string (static storage). */
+const char* sf_version(void);
+
+/* Name of a status code (static storage). */
+const char* sf_status_string(sf_status s);
+
+/* Copy the calling thread's last error message into buf (always
+ * NUL-terminated when len > 0).  Returns the full message length. */
+size_t sf_last_error(char* buf, size_t len);
+
+/*
+ * sf_quantize_nested -- nested min-max quantization of a row-major fp32
+ * matrix W[N][K] with groups of G consecutive inputs along K.
+ *
+ * Source: nested refinement, rag-lover.com explainer (解説): the fetched bits
+ * subdivide between resident levels; bit widths from the arXiv abstract.
+ * Definition (the pages give no formula; this is the reading the library
+ * fixes, identical to the oracle's):
+ *   lo, hi = min, max of the group (fp32);
+ *   s = fp16_RNE(min(fp32((hi - lo) / (2^b - 1)), 65504)), s = 1 if it is 0;
+ *   z = clamp(rint(-lo / s), 0, 2^b - 1)  (fp32 division, ties to even);
+ *   q = clamp(rint(w / s) + z, 0, 2^b - 1), b = b_r + b_f;
+ *   resident code q >> b_f, refinement code q & (2^b_f - 1).
+ * Outputs (device, caller-allocated):
+ *   res_codes  uint32 [N][K*b_r/32], row i = bitstream of its K resident codes;
+ *   ref_codes  layout SF_REF_BY_COLUMN: uint32 [K][N*b_f/32], row j = bitstream
+ *              of column j's N refinement codes (one column = one contiguous
+ *              transfer unit); SF_REF_BY_ROW: uint32 [N][K*b_f/32];
+ *   scale,zero fp16 [K/G][N] (zero is an exact small integer, +0 for zero).
+ * Constraints: b_r in {2,3}, b_f in {1,2}, b_r + b_f <= 4, G % 32 == 0,
+ *   K % G == 0, N >= 1; SF_REF_BY_COLUMN also needs N % 32 == 0.
+ *   W must be finite (non-finite input gives unspecified codes).
+ */
+sf_status sf_quantize_nested(const float* W, int N, int K, int G, int b_r, int b_f, int layout,
+                             uint32_t* res_codes, uint32_t* ref_codes, uint16_t* scale,
+                             uint16_t* zero, sf_stream_t stream);
+
+/*
+ * sf_select_topk -- channel selection by activation magnitude.
+ *
+ * Source: rag-lover.com explainer (解説): weights are refined where the input
+ * activation is large.  Per batch row the k channels with the largest |x|
+ * (exact bf16 magnitudes, +0 == -0) are chosen, ties to the lower channel
+ * index; the result is the union over the B rows in ascending order.
+ *   x       device bf16 [B][K];
+ *   idx_out device int32, capacity B*k, receives the ascending union;
+ *   n_out   device int32 scalar, receives its length, or -1 if x holds a
+ *           NaN or Inf (idx_out is then unspecified).
+ * Constraints: 1 <= B <= 16, 1 <= K <= 65536, 0 <= k <= K.
+ */
+sf_status sf_select_topk(const uint16_t* x, int B, int K, int k, int32_t* idx_out,
+                         int32_t* n_out, sf_stream_t stream);
+
+/* A quantized weight matrix as produced by sf_quantize_nested (views, not
+ * owned).  ref may be NULL; when non-NULL it is the complete refinement store
+ * [K][N*b_f/32] resident in device memory. */
+typedef struct sf_qweight {
+  const uint32_t* res;   /* [N][K*b_r/32] */
+  const uint16_t* scale; /* fp16 [K/G][N] */
+  const uint16_t* zero;  /* fp16 [K/G][N] */
+  const uint32_t* ref;   /* [K][N*b_f/32] or NULL */
+  int N, K, G, b_r, b_f;
+} sf_qweight;
+
+/* ---- refinement cache (one per weight matrix) -------------------------- */
+
+typedef struct sf_refine_cache sf_refine_cache;
+
+typedef struct sf_cache_stats {
+  int64_t steps;     /* prefetch steps taken */
+  int64_t hits;      /* selected units found in the cache */
+  int64_t misses;    /* selected units not found (bypass included) */
+  int64_t bypass;    /* misses fetched for one step only (no slot left) */
+  int64_t h2d_bytes; /* bytes moved from host memory for misses */
+} sf_cache_stats;
+
+/*
+ * sf_refine_cache_create -- an LRU cache of refinement units in device memory.
+ *
+ * Source: reuse of fetched precision across decode steps (arXiv abstract;
+ * rag-lover.com explainer, TL;DR and 解説).  Policy (reading fixed by the
+ * library): at each step with ascending selection S, hits H = S ∩ cached;
+ * misses take free slots (lowest index first), then the slots of cached units
+ * not in S ordered by (last use, unit), in ascending unit order; misses left
+ * without a slot are the bypass set (fetched for this step only); every unit
+ * used this step gets last use = this step.
+ *   num_units   units addressable (K for a weight matrix);
+ *   unit_bytes  bytes per unit (N*b_f/8 for a weight column), a multiple of 16;
+ *   capacity    cache slots, 0 <= capacity <= num_units;
+ *   max_select  largest selection a prefetch will see (B*k), >= 1;
+ *   host_master host copy of all units, [num_units][unit_bytes], 16-byte
+ *               aligned.  It must stay valid and unchanged until destroy.  If it
+ *               is not page-locked the cache page-locks it (and unlocks it in
+ *               destroy); either way the device reads it directly over the
+ *               host link.
+ *   device      CUDA device ordinal the cache lives on.
+ * Allocates device memory for capacity + max_select unit rows plus small
+ * index arrays.  Returns SF_ENOMEM / SF_ECUDA on allocation failure.
+ */
+sf_status sf_refine_cache_create(sf_refine_cache** out, int num_units, size_t unit_bytes,
+                                 int capacity, int max_select, const void* host_master,
+                                 int device);
+
+/* Fill an empty cache with n distinct units (device int32, ascending,
+ * n <= capacity) in slots 0..n-1 with last use older than any step.  Counts
+ * nothing in the statistics.  Enqueued on stream. */
+sf_status sf_refine_cache_preload(sf_refine_cache* c, const int32_t* units, int n,
+                                  sf_stream_t stream);
+
+/*
+ * sf_refine_cache_prefetch -- one cache step for the selection (idx, n) that
+ * `producer` writes: resolve hits / misses / bypass, assign slots, and copy
+ * every missed unit from host memory into its slot (or bypass row).  The work
+ * runs on `side` after the producer's work so far; the next sf_gemv_refine
+ * given this cache makes its own stream wait for it.  Issuing the prefetch of
+ * a later layer before the GEMV of the current one overlaps the transfer with
+ * compute (fetch lead, rag-lover.com explainer 解説).
+ *   idx  device int32 ascending unit indices (length *n <= max_select; a
+ *        negative *n counts as 0).
+ * The GEMV that consumes this step must be enqueued before the next
+ * prefetch on the same cache; the library orders the two streams.
+ */
+sf_status sf_refine_cache_prefetch(sf_refine_cache* c, const int32_t* idx, const int32_t* n,
+                                   sf_stream_t producer, sf_stream_t side);
+
+/* Copy the last step's sets to host arrays (each of capacity max_select):
+ * hits, misses (bypass included) and bypass, ascending; counts[3] receives
+ * their lengths.  Synchronizes with the last prefetch.  If that prefetch was
+ * captured into a CUDA graph, the caller must first synchronize the stream
+ * the graph was launched on (the same holds for _slots, _stats, _reset). */
+sf_status sf_refine_cache_sets(sf_refine_cache* c, int32_t* hits, int32_t* misses,
+                               int32_t* bypass, int32_t counts[3]);
+
+/* Copy the unit held by each slot to host slot_units[capacity] (-1 = free).
+ * Synchronizes with the last prefetch. */
+sf_status sf_refine_cache_slots(sf_refine_cache* c, int32_t* slot_units);
+
+/* Cumulative statistics since create/reset.  Synchronizes. */
+sf_status sf_refine_cache_stats(sf_refine_cache* c, sf_cache_stats* out);
+
+/* Empty the cache and zero the statistics.  Synchronizes. */
+sf_status sf_refine_cache_reset(sf_refine_cache* c);
+
+/* Free everything the cache owns.  Synchronizes.  NULL is accepted. */
+sf_status sf_refine_cache_destroy(sf_refine_cache* c);
+
+/*
+ * sf_gemv_refine -- refined decode GEMV, y[b][i] = sum_j x[b][j] w_eff[i][j].
+ *
+ * Source: rag-lover.com explainer (解説): columns picked by activation
+ * magnitude use resident + refinement bits, all others the resident code
+ * dequantized at the midpoint of its refinement interval.  Equivalently
+ *   y = W_res x + sum_{j in S} x_j s_{g(j)} (q_f - m_f),  m_f = (2^b_f - 1)/2.
+ *   W      quantized weights; x device bf16 [B][K]; y device fp32 [B][N].
+ *   idx,n  the selection S (device, as written by sf_select_topk).
+ *   c      non-NULL: refinements come from the cache's last prefetch, which
+ *          must have been given this same (idx, n);
+ *          NULL and W->ref non-NULL: refinements read from W->ref directly;
+ *          NULL and W->ref NULL: resident-only GEMV (idx, n ignored).
+ * Constraints: 1 <= B <= 16, b_r in {2,3}, b_f in {1,2}, G % 32 == 0,
+ *   K % G == 0, K <= 32768, N % 32 == 0.
+ * Accuracy: |y - exact| <= 2e-3 * sum_j |w_eff[i][j] x[b][j]| per output.
+ */
+sf_status sf_gemv_refine(const sf_qweight* W, const uint16_t* x, int B, const int32_t* idx,
+                         const int32_t* n, sf_refine_cache* c, float* y, sf_stream_t stream);
+
+/* ---- refined decode attention ----------------------------------------- */
+
+/* Quantized K and V (views).  Rows are token-heads ordered [Hkv][T], each
+ * quantized as one group of d values with sf_quantize_nested(layout
+ * SF_REF_BY_ROW): *_res [Hkv*T][d*b_r/32], *_ref [Hkv*T][d*b_f/32],
+ * *_scale/*_zero fp16 [Hkv*T]. */
+typedef struct sf_qkv {
+  const uint32_t *k_res, *k_ref, *v_res, *v_ref;
+  const uint16_t *k_scale, *k_zero, *v_scale, *v_zero;
+  int b_r, b_f;
+} sf_qkv;
+
+/* Workspace bytes sf_attn_decode_refine needs for these sizes. */
+sf_status sf_attn_workspace_size(int Hq, int Hkv, int d, int T, int k_tokens, size_t* bytes);
+
+/*
+ * sf_attn_decode_refine -- one decode step of attention over low-bit K/V with
+ * the most-attended tokens refined.
+ *
+ * Source: rag-lover.com explainer (解説): KV refinement is chosen by the
+ * attention weight computed from the low-bit keys.  Definition:
+ *   query head h reads KV head h / (Hq/Hkv);
+ *   key of token t for head h: kappa = fp64(s_t * sum_d q[h][d]*(c[t][d]*2^b_f
+ *   + m_f - z_t)) computed exactly (c = resident key code); per head the
+ *   k_tokens largest keys are selected (ties to the lower token index); the
+ *   union over the heads of a KV group is refined in both K and V; the output
+ *   is softmax attention over all T tokens with refined (full-code) K/V for the
+ *   union and resident K/V elsewhere.
+ *   q        device bf16 [Hq][d];
+ *   sel_out  device int32 [Hkv][(Hq/Hkv)*k_tokens]: per KV head the ascending
+ *            union; sel_n device int32 [Hkv] its lengths;
+ *   out      device fp32 [Hq][d];
+ *   workspace device scratch of at least sf_attn_workspace_size bytes (caller
+ *            owned, contents need not be initialised, not read afterwards).
+ * Exact selection needs, per query head, the binary exponents of its nonzero
+ * q entries to span at most 53 - 9 - (b_r + b_f) - log2(d) = 33 binades (so
+ * every key is exact in fp64).  When a head of KV group g violates it, the
+ * selection still runs on the fp64 keys (then possibly not exact) and
+ * sel_n[g] is written as -1 - (union length) to report it.
+ * Constraints: d == 128, Hq % Hkv == 0, Hq/Hkv <= 8, 1 <= T, 0 <= k_tokens
+ *   <= min(T, 4096), b_r == 2, b_f == 2.
+ * Accuracy: max |out - exact| <= 2e-3.
+ */
+sf_status sf_attn_decode_refine(const uint16_t* q, int Hq, int Hkv, int d, int T,
+                                const sf_qkv* kv, int k_tokens, int32_t* sel_out,
+                                int32_t* sel_n, float* out, void* workspace, size_t ws_bytes,
+                                sf_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SF_H */

@@ -1,0 +1,307 @@
+"""Python binding of libsf, the StrataFlux selective-precision-streaming hot
+path for B200 (sm_100a).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels
+of ``libsf.so``.  PyTorch provides device memory and the current CUDA stream.
+The functions mirror the C ABI declared in ``include/sf.h``:
+
+  quantize_nested, select_topk, gemv_refine, attn_decode_refine,
+  attn_workspace_size, RefineCache (sf_refine_cache_*).
+
+Importing fails loudly when the library has not been built (``build()`` in
+``quantized_gemv_kv_b200.build``); there is no CPU fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsf.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m quantized_gemv_kv_b200.build` "
+                      "(nvcc, sm_100a); there is no fallback path")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+SF_OK, SF_EINVAL, SF_ENOMEM, SF_ECUDA, SF_ETIMEOUT, SF_ENOTIMPL = range(6)
+SF_REF_BY_COLUMN, SF_REF_BY_ROW = 0, 1
+_LAYOUTS = {"by_column": SF_REF_BY_COLUMN, "by_row": SF_REF_BY_ROW}
+
+_p = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+
+
+class SfError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_lib.sf_status_string(status).decode()}: {msg}")
+        self.status = status
+
+
+class _QWeight(ctypes.Structure):
+    _fields_ = [("res", _p), ("scale", _p), ("zero", _p), ("ref", _p),
+                ("N", _i), ("K", _i), ("G", _i), ("b_r", _i), ("b_f", _i)]
+
+
+class _QKV(ctypes.Structure):
+    _fields_ = [("k_res", _p), ("k_ref", _p), ("v_res", _p), ("v_ref", _p),
+                ("k_scale", _p), ("k_zero", _p), ("v_scale", _p), ("v_zero", _p),
+                ("b_r", _i), ("b_f", _i)]
+
+
+class CacheStats(ctypes.Structure):
+    _fields_ = [("steps", ctypes.c_int64), ("hits", ctypes.c_int64), ("misses", ctypes.c_int64),
+                ("bypass", ctypes.c_int64), ("h2d_bytes", ctypes.c_int64)]
+
+
+_SIGS = {
+    "sf_version": ([], ctypes.c_char_p),
+    "sf_status_string": ([_i], ctypes.c_char_p),
+    "sf_last_error": ([ctypes.c_char_p, _sz], _sz),
+    "sf_quantize_nested": ([_p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p], _i),
+    "sf_select_topk": ([_p, _i, _i, _i, _p, _p, _p], _i),
+    "sf_refine_cache_create": ([ctypes.POINTER(_p), _i, _sz, _i, _i, _p, _i], _i),
+    "sf_refine_cache_preload": ([_p, _p, _i, _p], _i),
+    "sf_refine_cache_prefetch": ([_p, _p, _p, _p, _p], _i),
+    "sf_refine_cache_sets": ([_p, _p, _p, _p, _p], _i),
+    "sf_refine_cache_slots": ([_p, _p], _i),
+    "sf_refine_cache_stats": ([_p, ctypes.POINTER(CacheStats)], _i),
+    "sf_refine_cache_reset": ([_p], _i),
+    "sf_refine_cache_destroy": ([_p], _i),
+    "sf_gemv_refine": ([ctypes.POINTER(_QWeight), _p, _i, _p, _p, _p, _p, _p], _i),
+    "sf_attn_workspace_size": ([_i, _i, _i, _i, _i, ctypes.POINTER(_sz)], _i),
+    "sf_attn_decode_refine": ([_p, _i, _i, _i, _i, ctypes.POINTER(_QKV), _i, _p, _p, _p, _p, _sz, _p], _i),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+EXPORTED = tuple(_SIGS)
+
+
+def version() -> str:
+    return _lib.sf_version().decode()
+
+
+def _check(status: int) -> None:
+    if status != SF_OK:
+        buf = ctypes.create_string_buffer(1024)
+        _lib.sf_last_error(buf, len(buf))
+        raise SfError(status, buf.value.decode(errors="replace"))
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libsf must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream: torch.cuda.Stream | None = None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _dev(t: torch.Tensor, name: str) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+# ---- quantization ------------------------------------------------------------
+
+@dataclass
+class QWeight:
+    """Packed nested-quantized matrix (see ``sf_quantize_nested``)."""
+    res: torch.Tensor      # int32 [N][K*b_r/32] (uint32 words)
+    ref: torch.Tensor      # int32 [K][N*b_f/32] (by_column) or [N][K*b_f/32] (by_row)
+    scale: torch.Tensor    # float16 [K/G][N]
+    zero: torch.Tensor     # float16 [K/G][N]
+    N: int
+    K: int
+    G: int
+    b_r: int
+    b_f: int
+    layout: str = "by_column"
+
+    def c_struct(self, with_ref: bool = False) -> _QWeight:
+        return _QWeight(_ptr(self.res), _ptr(self.scale), _ptr(self.zero),
+                        _ptr(self.ref) if with_ref else None, self.N, self.K, self.G, self.b_r, self.b_f)
+
+
+def quantize_nested(W: torch.Tensor, G: int, b_r: int, b_f: int, layout: str = "by_column",
+                    stream: torch.cuda.Stream | None = None) -> QWeight:
+    """Nested min-max group quantization of fp32 W[N][K] on the device."""
+    _dev(W, "W")
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise ValueError("W must be a 2-D float32 tensor")
+    N, K = W.shape
+    dev = W.device
+    res = torch.empty((N, K * b_r // 32), dtype=torch.int32, device=dev)
+    if layout == "by_column":
+        ref = torch.empty((K, N * b_f // 32), dtype=torch.int32, device=dev)
+    else:
+        ref = torch.empty((N, K * b_f // 32), dtype=torch.int32, device=dev)
+    scale = torch.empty((K // G, N), dtype=torch.float16, device=dev)
+    zero = torch.empty((K // G, N), dtype=torch.float16, device=dev)
+    _check(_lib.sf_quantize_nested(_ptr(W), N, K, G, b_r, b_f, _LAYOUTS[layout], _ptr(res), _ptr(ref),
+                                   _ptr(scale), _ptr(zero), _stream(stream)))
+    return QWeight(res, ref, scale, zero, N, K, G, b_r, b_f, layout)
+
+
+# ---- selection ---------------------------------------------------------------
+
+def select_topk(x: torch.Tensor, k: int, idx_out: torch.Tensor | None = None, n_out: torch.Tensor | None = None,
+                stream: torch.cuda.Stream | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Top-k channels by |x| per row of bf16 x[B][K], union ascending.
+    Returns (idx int32 [B*k] buffer, n int32 [1] device scalar)."""
+    _dev(x, "x")
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    B, K = x.shape
+    if idx_out is None:
+        idx_out = torch.empty(max(B * k, 1), dtype=torch.int32, device=x.device)
+    if n_out is None:
+        n_out = torch.empty(1, dtype=torch.int32, device=x.device)
+    _check(_lib.sf_select_topk(_ptr(x), B, K, k, _ptr(idx_out), _ptr(n_out), _stream(stream)))
+    return idx_out, n_out
+
+
+# ---- refinement cache ----------------------------------------------------------
+
+class RefineCache:
+    """LRU refinement cache in device memory fed from a host master copy
+    (``sf_refine_cache_*``).  ``host_master`` is a CPU uint8/int32 tensor of
+    num_units * unit_bytes bytes; it is kept alive by this object."""
+
+    def __init__(self, num_units: int, unit_bytes: int, capacity: int, max_select: int,
+                 host_master: torch.Tensor, device: int | None = None):
+        if host_master.is_cuda or not host_master.is_contiguous():
+            raise ValueError("host_master must be a contiguous CPU tensor")
+        if host_master.numel() * host_master.element_size() < num_units * unit_bytes:
+            raise ValueError("host_master is smaller than num_units * unit_bytes")
+        self._master = host_master
+        self.num_units, self.unit_bytes, self.capacity, self.max_select = num_units, unit_bytes, capacity, max_select
+        self.device = torch.cuda.current_device() if device is None else device
+        h = _p()
+        _check(_lib.sf_refine_cache_create(ctypes.byref(h), num_units, unit_bytes, capacity, max_select,
+                                           host_master.data_ptr(), self.device))
+        self._h = h
+
+    @property
+    def handle(self) -> int:
+        return self._h.value
+
+    def preload(self, units: torch.Tensor, stream: torch.cuda.Stream | None = None) -> None:
+        _dev(units, "units")
+        _check(_lib.sf_refine_cache_preload(self._h, _ptr(units), units.numel(), _stream(stream)))
+
+    def prefetch(self, idx: torch.Tensor, n: torch.Tensor, producer: torch.cuda.Stream | None = None,
+                 side: torch.cuda.Stream | None = None) -> None:
+        _check(_lib.sf_refine_cache_prefetch(self._h, _ptr(idx), _ptr(n), _stream(producer),
+                                             _stream(side if side is not None else producer)))
+
+    def sets(self) -> dict:
+        import numpy as np
+        h = np.zeros(self.max_select, np.int32)
+        m = np.zeros(self.max_select, np.int32)
+        b = np.zeros(self.max_select, np.int32)
+        c = np.zeros(3, np.int32)
+        _check(_lib.sf_refine_cache_sets(self._h, h.ctypes.data, m.ctypes.data, b.ctypes.data, c.ctypes.data))
+        return dict(hits=h[:c[0]].tolist(), misses=m[:c[1]].tolist(), bypass=b[:c[2]].tolist())
+
+    def slots(self) -> list[int]:
+        import numpy as np
+        s = np.zeros(max(self.capacity, 1), np.int32)
+        _check(_lib.sf_refine_cache_slots(self._h, s.ctypes.data))
+        return s[:self.capacity].tolist()
+
+    def stats(self) -> CacheStats:
+        st = CacheStats()
+        _check(_lib.sf_refine_cache_stats(self._h, ctypes.byref(st)))
+        return st
+
+    def reset(self) -> None:
+        _check(_lib.sf_refine_cache_reset(self._h))
+
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None and self._h.value:
+            _check(_lib.sf_refine_cache_destroy(self._h))
+            self._h = _p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+# ---- GEMV ----------------------------------------------------------------------
+
+def gemv_refine(W: QWeight, x: torch.Tensor, idx: torch.Tensor | None = None, n: torch.Tensor | None = None,
+                cache: RefineCache | None = None, use_ref_store: bool = False, y: torch.Tensor | None = None,
+                stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """Refined decode GEMV y[B][N] (fp32).  Refinements come from ``cache``,
+    else from W.ref when ``use_ref_store``, else none (resident-only)."""
+    _dev(x, "x")
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    B = x.shape[0]
+    if y is None:
+        y = torch.empty((B, W.N), dtype=torch.float32, device=x.device)
+    qw = W.c_struct(with_ref=use_ref_store and cache is None)
+    _check(_lib.sf_gemv_refine(ctypes.byref(qw), _ptr(x), B, _ptr(idx), _ptr(n),
+                               cache.handle if cache is not None else None, _ptr(y), _stream(stream)))
+    return y
+
+
+# ---- attention -----------------------------------------------------------------
+
+@dataclass
+class QKV:
+    """Quantized K and V, rows = token-heads [Hkv][T] (layout by_row, G = d)."""
+    k: QWeight
+    v: QWeight
+
+    def c_struct(self) -> _QKV:
+        return _QKV(_ptr(self.k.res), _ptr(self.k.ref), _ptr(self.v.res), _ptr(self.v.ref),
+                    _ptr(self.k.scale), _ptr(self.k.zero), _ptr(self.v.scale), _ptr(self.v.zero),
+                    self.k.b_r, self.k.b_f)
+
+
+def attn_workspace_size(Hq: int, Hkv: int, d: int, T: int, k_tokens: int) -> int:
+    out = _sz()
+    _check(_lib.sf_attn_workspace_size(Hq, Hkv, d, T, k_tokens, ctypes.byref(out)))
+    return out.value
+
+
+def attn_decode_refine(q: torch.Tensor, kv: QKV, Hkv: int, T: int, k_tokens: int,
+                       workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                       sel_out: torch.Tensor | None = None, sel_n: torch.Tensor | None = None,
+                       stream: torch.cuda.Stream | None = None):
+    """Refined decode attention.  Returns (out fp32 [Hq][d], sel int32
+    [Hkv][Hq/Hkv*k], sel_n int32 [Hkv])."""
+    _dev(q, "q")
+    Hq, d = q.shape
+    grp = Hq // Hkv
+    dev = q.device
+    if workspace is None:
+        workspace = torch.empty(attn_workspace_size(Hq, Hkv, d, T, k_tokens), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty((Hq, d), dtype=torch.float32, device=dev)
+    if sel_out is None:
+        sel_out = torch.empty((Hkv, max(grp * k_tokens, 1)), dtype=torch.int32, device=dev)
+    if sel_n is None:
+        sel_n = torch.empty(Hkv, dtype=torch.int32, device=dev)
+    s = kv.c_struct()
+    _check(_lib.sf_attn_decode_refine(_ptr(q), Hq, Hkv, d, T, ctypes.byref(s), k_tokens, _ptr(sel_out),
+                                      _ptr(sel_n), _ptr(out), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out, sel_out, sel_n

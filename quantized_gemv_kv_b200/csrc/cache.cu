@@ -1,0 +1,488 @@
+// Refinement cache: an LRU set of refinement units (weight columns) kept in
+// device memory and refilled from a host-resident master copy.
+//
+// StrataFlux reuses fetched precision across decode steps and hides transfer
+// behind compute (arXiv 2611.08363 abstract; rag-lover.com explainer, 解説:
+// fetch lead and caching).  Everything that decides hits, misses, slots and
+// the LRU order runs on the device in one CTA (no host round trip), so a
+// step can be enqueued ahead of time and captured in a CUDA graph.  Misses
+// are copied by a gather kernel that reads the page-locked, device-mapped
+// host master directly over the host link, on a side stream.
+//
+// LRU bookkeeping: `order` lists the cached units from least to most
+// recently used, ties (units touched in the same step) in ascending unit
+// order.  A step removes the hits from it, takes victims from its front,
+// and appends the units touched this step (hits and inserted misses) in
+// ascending order -- which keeps it sorted by (last use, unit) without
+// storing the last-use stamps.  Slots are never freed except by reset, so
+// the free slots are always the suffix [occupied, capacity).
+#include <algorithm>
+#include <cstring>
+#include <vector>
+
+#include "block_scan.cuh"
+#include "sf_internal.h"
+
+namespace {
+
+constexpr int kIndexThreads = 1024;
+constexpr int kGatherThreads = 128;
+
+enum Meta { kOcc = 0, kStep, kHits, kMisses, kBypass, kGather, kMetaCount };
+enum Stat { kStSteps = 0, kStHits, kStMisses, kStBypass, kStBytes, kStatCount };
+
+// One cache step.  S = idx[0..n) ascending.
+__global__ void __launch_bounds__(kIndexThreads)
+cache_index_kernel(const int32_t* __restrict__ S, const int32_t* __restrict__ n_ptr, int max_select, int capacity,
+                   int64_t unit_bytes, int32_t* __restrict__ unit_slot, int32_t* __restrict__ slot_unit,
+                   int32_t* __restrict__ order, int32_t* __restrict__ order_tmp, int32_t* __restrict__ row_of,
+                   int32_t* __restrict__ hits_out, int32_t* __restrict__ misses_out, int32_t* __restrict__ bypass_out,
+                   int32_t* __restrict__ victim_unit, int32_t* __restrict__ victim_slot,
+                   int32_t* __restrict__ gather_unit, int32_t* __restrict__ gather_row, int32_t* __restrict__ meta,
+                   int64_t* __restrict__ stats) {
+  extern __shared__ uint8_t slot_hit[];  // [capacity]
+  __shared__ int scratch[33];
+  const int tid = threadIdx.x;
+  int n = *n_ptr;
+  n = n < 0 ? 0 : (n > max_select ? max_select : n);
+  const int occ = meta[kOcc];
+
+  for (int i = tid; i < capacity; i += kIndexThreads) slot_hit[i] = 0;
+  __syncthreads();
+
+  // 1. hits and misses of S, in ascending order (ordered scan over chunks)
+  const int chunk = (n + kIndexThreads - 1) / kIndexThreads;
+  const int p0 = min(n, tid * chunk), p1 = min(n, p0 + chunk);
+  int h = 0;
+  for (int p = p0; p < p1; ++p) {
+    const int sl = unit_slot[S[p]];
+    if (sl >= 0) { ++h; slot_hit[sl] = 1; }
+  }
+  int H;
+  const int h_before = sfd::block_exclusive_scan(h, scratch, &H);
+  {
+    int hh = h_before, mm = p0 - h_before;
+    for (int p = p0; p < p1; ++p) {
+      const int u = S[p];
+      if (unit_slot[u] >= 0) hits_out[hh++] = u; else misses_out[mm++] = u;
+    }
+  }
+  const int mi = n - H;
+  const int avail = capacity - H;
+  const int ins = min(mi, avail);
+  const int use_free = min(ins, capacity - occ);
+  const int v = ins - use_free;
+
+  // 2. LRU order without the hits; its first v entries are the victims
+  const int ochunk = (occ + kIndexThreads - 1) / kIndexThreads;
+  const int o0 = min(occ, tid * ochunk), o1 = min(occ, o0 + ochunk);
+  int keep = 0;
+  for (int i = o0; i < o1; ++i) keep += !slot_hit[unit_slot[order[i]]];
+  int F;
+  int fpos = sfd::block_exclusive_scan(keep, scratch, &F);
+  for (int i = o0; i < o1; ++i) {
+    const int u = order[i];
+    const int sl = unit_slot[u];
+    if (slot_hit[sl]) continue;
+    if (fpos < v) { victim_unit[fpos] = u; victim_slot[fpos] = sl; }
+    else order_tmp[fpos - v] = u;
+    ++fpos;
+  }
+  __syncthreads();
+
+  // 3. place the misses: free slots first, then victims, then bypass rows
+  for (int r = tid; r < mi; r += kIndexThreads) {
+    const int u = misses_out[r];
+    int row;
+    if (r < use_free) {
+      row = occ + r;
+    } else if (r < ins) {
+      row = victim_slot[r - use_free];
+      unit_slot[victim_unit[r - use_free]] = -1;
+    } else {
+      row = capacity + (r - ins);
+      bypass_out[r - ins] = u;
+    }
+    if (r < ins) { unit_slot[u] = row; slot_unit[row] = u; }
+    gather_unit[r] = u;
+    gather_row[r] = row;
+  }
+  __syncthreads();
+
+  // 4. row of every selected position; 5. append touched units to the order
+  int touched = 0;
+  {
+    int mm = p0 - h_before;
+    for (int p = p0; p < p1; ++p) {
+      const int u = S[p];
+      // a unit is a hit iff it is not in the miss list; misses are ranked mm
+      // in ascending order, so compare with the miss list entry at rank mm
+      const bool is_miss = (mm < mi) && (misses_out[mm] == u);
+      if (is_miss) {
+        row_of[p] = gather_row[mm];
+        if (mm < ins) ++touched;
+        ++mm;
+      } else {
+        row_of[p] = unit_slot[u];
+        ++touched;
+      }
+    }
+  }
+  int T_all;
+  int tpos = sfd::block_exclusive_scan(touched, scratch, &T_all);
+  const int base = (occ - H) - v;
+  {
+    int mm = p0 - h_before;
+    for (int p = p0; p < p1; ++p) {
+      const int u = S[p];
+      const bool is_miss = (mm < mi) && (misses_out[mm] == u);
+      bool t_here = true;
+      if (is_miss) { t_here = mm < ins; ++mm; }
+      if (t_here) order_tmp[base + tpos++] = u;
+    }
+  }
+  __syncthreads();
+  const int new_occ = occ + use_free;
+  for (int i = tid; i < new_occ; i += kIndexThreads) order[i] = order_tmp[i];
+  if (tid == 0) {
+    meta[kOcc] = new_occ;
+    meta[kStep] += 1;
+    meta[kHits] = H;
+    meta[kMisses] = mi;
+    meta[kBypass] = mi - ins;
+    meta[kGather] = mi;
+    stats[kStSteps] += 1;
+    stats[kStHits] += H;
+    stats[kStMisses] += mi;
+    stats[kStBypass] += mi - ins;
+    stats[kStBytes] += static_cast<int64_t>(mi) * unit_bytes;
+  }
+}
+
+// Copy every missed unit from the device-mapped host master into its row.
+__global__ void __launch_bounds__(kGatherThreads)
+cache_gather_kernel(const uint4* __restrict__ master, uint4* __restrict__ rows, const int32_t* __restrict__ gather_unit,
+                    const int32_t* __restrict__ gather_row, const int32_t* __restrict__ meta, int unit_vec) {
+  const int n = meta[kGather];
+  for (int e = blockIdx.x; e < n; e += gridDim.x) {
+    const uint4* src = master + static_cast<size_t>(gather_unit[e]) * unit_vec;
+    uint4* dst = rows + static_cast<size_t>(gather_row[e]) * unit_vec;
+    for (int w = threadIdx.x; w < unit_vec; w += kGatherThreads) dst[w] = src[w];
+  }
+}
+
+// Preload: units[i] goes to slot i; copies its bytes too.
+__global__ void cache_preload_kernel(const int32_t* __restrict__ units, int n, const uint4* __restrict__ master,
+                                     uint4* __restrict__ rows, int unit_vec, int32_t* __restrict__ unit_slot,
+                                     int32_t* __restrict__ slot_unit, int32_t* __restrict__ order,
+                                     int32_t* __restrict__ meta) {
+  for (int e = blockIdx.x; e < n; e += gridDim.x) {
+    const int u = units[e];
+    if (threadIdx.x == 0) {
+      unit_slot[u] = e;
+      slot_unit[e] = u;
+      order[e] = u;
+    }
+    const uint4* src = master + static_cast<size_t>(u) * unit_vec;
+    uint4* dst = rows + static_cast<size_t>(e) * unit_vec;
+    for (int w = threadIdx.x; w < unit_vec; w += blockDim.x) dst[w] = src[w];
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) meta[kOcc] = n;
+}
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    cudaGetDevice(&prev);
+    if (prev != dev) cudaSetDevice(dev);
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (prev >= 0 && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+unsigned long long capture_id(cudaStream_t s) {
+  cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+  unsigned long long id = 0;
+  if (cudaStreamGetCaptureInfo(s, &st, &id) != cudaSuccess) return 0;
+  return st == cudaStreamCaptureStatusActive ? id : 0;
+}
+
+}  // namespace
+
+struct sf_refine_cache {
+  int device = 0;
+  int num_units = 0;
+  size_t unit_bytes = 0;
+  int capacity = 0;
+  int max_select = 0;
+  const void* host_master = nullptr;
+  const void* master_dev = nullptr;
+  bool registered_here = false;
+  uint32_t* rows = nullptr;
+  int32_t* ints = nullptr;  // one allocation for every int32 array below
+  int32_t *unit_slot = nullptr, *slot_unit = nullptr, *order = nullptr, *order_tmp = nullptr, *row_of = nullptr,
+          *hits = nullptr, *misses = nullptr, *bypass = nullptr, *victim_unit = nullptr, *victim_slot = nullptr,
+          *gather_unit = nullptr, *gather_row = nullptr, *meta = nullptr;
+  int64_t* stats = nullptr;
+  cudaEvent_t ev_idx = nullptr, ev_ready = nullptr, ev_used = nullptr;
+  cudaStream_t aux = nullptr;
+  bool ready_pending = false, used_pending = false;
+  unsigned long long ready_capture = 0, used_capture = 0;
+};
+
+namespace {
+
+sf_status cache_free(sf_refine_cache* c) {
+  if (!c) return SF_OK;
+  DeviceGuard g(c->device);
+  if (c->aux) cudaStreamSynchronize(c->aux);
+  if (c->ev_ready) cudaEventSynchronize(c->ev_ready);
+  if (c->ev_used) cudaEventSynchronize(c->ev_used);
+  if (c->rows) cudaFree(c->rows);
+  if (c->ints) cudaFree(c->ints);
+  if (c->stats) cudaFree(c->stats);
+  if (c->ev_idx) cudaEventDestroy(c->ev_idx);
+  if (c->ev_ready) cudaEventDestroy(c->ev_ready);
+  if (c->ev_used) cudaEventDestroy(c->ev_used);
+  if (c->aux) cudaStreamDestroy(c->aux);
+  if (c->registered_here) cudaHostUnregister(const_cast<void*>(c->host_master));
+  delete c;
+  return SF_OK;
+}
+
+sf_status cache_clear(sf_refine_cache* c, cudaStream_t s) {
+  SF_CHECK_CUDA(cudaMemsetAsync(c->unit_slot, 0xFF, sizeof(int32_t) * c->num_units, s));
+  SF_CHECK_CUDA(cudaMemsetAsync(c->slot_unit, 0xFF, sizeof(int32_t) * std::max(c->capacity, 1), s));
+  SF_CHECK_CUDA(cudaMemsetAsync(c->meta, 0, sizeof(int32_t) * kMetaCount, s));
+  SF_CHECK_CUDA(cudaMemsetAsync(c->stats, 0, sizeof(int64_t) * kStatCount, s));
+  return SF_OK;
+}
+
+// Host wait for the last prefetch.  Once it has completed, later GEMVs need
+// not wait for it on the device any more (so a GEMV captured into a graph
+// after this point may consume an eager prefetch).
+// A prefetch captured into a graph has no event to wait on from the host:
+// the caller synchronizes the stream the graph was launched on first.
+sf_status wait_ready(sf_refine_cache* c) {
+  if (c->ready_pending) {
+    if (c->ready_capture == 0) SF_CHECK_CUDA(cudaEventSynchronize(c->ev_ready));
+    c->ready_pending = false;
+  }
+  SF_CHECK_CUDA(cudaStreamSynchronize(c->aux));
+  return SF_OK;
+}
+
+}  // namespace
+
+namespace sf {
+
+sf_status cache_view_for_gemv(sf_refine_cache* c, cudaStream_t stream, CacheView* v) {
+  if (c->ready_pending) {
+    const unsigned long long cid = capture_id(stream);
+    SF_REQUIRE(cid == c->ready_capture,
+               "sf_gemv_refine: the cache's last prefetch and this GEMV must both be inside the same stream "
+               "capture, or both outside one");
+    SF_CHECK_CUDA(cudaStreamWaitEvent(stream, c->ev_ready, 0));
+  }
+  v->rows = c->rows;
+  v->row_of = c->row_of;
+  v->unit_words = static_cast<int>(c->unit_bytes / 4);
+  return SF_OK;
+}
+
+sf_status cache_mark_used(sf_refine_cache* c, cudaStream_t stream) {
+  SF_CHECK_CUDA(cudaEventRecord(c->ev_used, stream));
+  c->used_pending = true;
+  c->used_capture = capture_id(stream);
+  return SF_OK;
+}
+
+}  // namespace sf
+
+extern "C" {
+
+sf_status sf_refine_cache_create(sf_refine_cache** out, int num_units, size_t unit_bytes, int capacity,
+                                 int max_select, const void* host_master, int device) {
+  SF_REQUIRE(out && host_master, "sf_refine_cache_create: null pointer");
+  *out = nullptr;
+  SF_REQUIRE(num_units >= 1, "sf_refine_cache_create: num_units must be >= 1");
+  SF_REQUIRE(unit_bytes >= 16 && unit_bytes % 16 == 0, "sf_refine_cache_create: unit_bytes must be a positive multiple of 16");
+  SF_REQUIRE(capacity >= 0 && capacity <= num_units && capacity <= 65536,
+             "sf_refine_cache_create: capacity must be in [0, min(num_units, 65536)]");
+  SF_REQUIRE(max_select >= 1 && max_select <= 1 << 20, "sf_refine_cache_create: max_select out of range");
+  SF_REQUIRE(sf::aligned(host_master, 16), "sf_refine_cache_create: host_master must be 16-byte aligned");
+  DeviceGuard g(device);
+  auto* c = new sf_refine_cache();
+  c->device = device;
+  c->num_units = num_units;
+  c->unit_bytes = unit_bytes;
+  c->capacity = capacity;
+  c->max_select = max_select;
+  c->host_master = host_master;
+  const size_t master_bytes = static_cast<size_t>(num_units) * unit_bytes;
+
+  cudaPointerAttributes attr{};
+  cudaError_t e = cudaPointerGetAttributes(&attr, host_master);
+  if (e != cudaSuccess) cudaGetLastError();
+  if (e != cudaSuccess || attr.type == cudaMemoryTypeUnregistered) {
+    e = cudaHostRegister(const_cast<void*>(host_master), master_bytes, cudaHostRegisterMapped);
+    if (e != cudaSuccess) { cache_free(c); return sf::cuda_fail(e, "cudaHostRegister(host_master)"); }
+    c->registered_here = true;
+  } else if (attr.type != cudaMemoryTypeHost) {
+    cache_free(c);
+    return sf::fail(SF_EINVAL, "sf_refine_cache_create: host_master must be host memory");
+  }
+  void* dptr = nullptr;
+  e = cudaHostGetDevicePointer(&dptr, const_cast<void*>(host_master), 0);
+  if (e != cudaSuccess) { cache_free(c); return sf::cuda_fail(e, "cudaHostGetDevicePointer(host_master)"); }
+  c->master_dev = dptr;
+
+  const size_t rows_bytes = (static_cast<size_t>(capacity) + max_select) * unit_bytes;
+  e = cudaMalloc(&c->rows, rows_bytes);
+  if (e != cudaSuccess) { cache_free(c); return sf::fail(SF_ENOMEM, "sf_refine_cache_create: cudaMalloc rows: %s", cudaGetErrorString(e)); }
+  const size_t cap1 = std::max(capacity, 1);
+  const size_t n_ints = static_cast<size_t>(num_units) + 3 * cap1 + 8 * static_cast<size_t>(max_select) + kMetaCount;
+  e = cudaMalloc(&c->ints, n_ints * sizeof(int32_t));
+  if (e != cudaSuccess) { cache_free(c); return sf::fail(SF_ENOMEM, "sf_refine_cache_create: cudaMalloc index: %s", cudaGetErrorString(e)); }
+  e = cudaMalloc(&c->stats, kStatCount * sizeof(int64_t));
+  if (e != cudaSuccess) { cache_free(c); return sf::fail(SF_ENOMEM, "sf_refine_cache_create: cudaMalloc stats: %s", cudaGetErrorString(e)); }
+  int32_t* p = c->ints;
+  c->unit_slot = p; p += num_units;
+  c->slot_unit = p; p += cap1;
+  c->order = p; p += cap1;
+  c->order_tmp = p; p += cap1;
+  c->row_of = p; p += max_select;
+  c->hits = p; p += max_select;
+  c->misses = p; p += max_select;
+  c->bypass = p; p += max_select;
+  c->victim_unit = p; p += max_select;
+  c->victim_slot = p; p += max_select;
+  c->gather_unit = p; p += max_select;
+  c->gather_row = p; p += max_select;
+  c->meta = p;
+  if ((e = cudaEventCreateWithFlags(&c->ev_idx, cudaEventDisableTiming)) != cudaSuccess ||
+      (e = cudaEventCreateWithFlags(&c->ev_ready, cudaEventDisableTiming)) != cudaSuccess ||
+      (e = cudaEventCreateWithFlags(&c->ev_used, cudaEventDisableTiming)) != cudaSuccess ||
+      (e = cudaStreamCreateWithFlags(&c->aux, cudaStreamNonBlocking)) != cudaSuccess) {
+    cache_free(c);
+    return sf::cuda_fail(e, "sf_refine_cache_create: events/stream");
+  }
+  sf_status st = cache_clear(c, c->aux);
+  if (st == SF_OK) {
+    e = cudaStreamSynchronize(c->aux);
+    if (e != cudaSuccess) st = sf::cuda_fail(e, "sf_refine_cache_create: init");
+  }
+  if (st != SF_OK) { cache_free(c); return st; }
+  *out = c;
+  return SF_OK;
+}
+
+sf_status sf_refine_cache_preload(sf_refine_cache* c, const int32_t* units, int n, sf_stream_t stream) {
+  SF_REQUIRE(c, "sf_refine_cache_preload: null cache");
+  SF_REQUIRE(n >= 0 && n <= c->capacity, "sf_refine_cache_preload: n must be in [0, capacity]");
+  SF_REQUIRE(n == 0 || units, "sf_refine_cache_preload: null units");
+  DeviceGuard g(c->device);
+  if (n == 0) return SF_OK;
+  cudaStream_t s = sf::as_cuda(stream);
+  const int grid = std::min(n, 4 * sf::sm_count());
+  cache_preload_kernel<<<grid, kGatherThreads, 0, s>>>(units, n, static_cast<const uint4*>(c->master_dev),
+                                                        reinterpret_cast<uint4*>(c->rows),
+                                                        static_cast<int>(c->unit_bytes / 16), c->unit_slot,
+                                                        c->slot_unit, c->order, c->meta);
+  return sf::check_launch("cache_preload_kernel");
+}
+
+sf_status sf_refine_cache_prefetch(sf_refine_cache* c, const int32_t* idx, const int32_t* n, sf_stream_t producer,
+                                   sf_stream_t side) {
+  SF_REQUIRE(c && idx && n, "sf_refine_cache_prefetch: null pointer");
+  DeviceGuard g(c->device);
+  cudaStream_t ps = sf::as_cuda(producer), ss = sf::as_cuda(side);
+  const unsigned long long cid = capture_id(ss);
+  SF_REQUIRE(capture_id(ps) == cid, "sf_refine_cache_prefetch: producer and side stream capture states differ");
+  SF_CHECK_CUDA(cudaEventRecord(c->ev_idx, ps));
+  SF_CHECK_CUDA(cudaStreamWaitEvent(ss, c->ev_idx, 0));
+  // the previous step's GEMV must have read the rows before they change
+  if (c->used_pending && c->used_capture == cid) SF_CHECK_CUDA(cudaStreamWaitEvent(ss, c->ev_used, 0));
+  const size_t smem = std::max(c->capacity, 1);
+  cache_index_kernel<<<1, kIndexThreads, smem, ss>>>(
+      idx, n, c->max_select, c->capacity, static_cast<int64_t>(c->unit_bytes), c->unit_slot, c->slot_unit, c->order,
+      c->order_tmp, c->row_of, c->hits, c->misses, c->bypass, c->victim_unit, c->victim_slot, c->gather_unit,
+      c->gather_row, c->meta, c->stats);
+  sf_status st = sf::check_launch("cache_index_kernel");
+  if (st != SF_OK) return st;
+  const int grid = std::min(c->max_select, 2 * sf::sm_count());
+  cache_gather_kernel<<<grid, kGatherThreads, 0, ss>>>(static_cast<const uint4*>(c->master_dev),
+                                                       reinterpret_cast<uint4*>(c->rows), c->gather_unit,
+                                                       c->gather_row, c->meta, static_cast<int>(c->unit_bytes / 16));
+  st = sf::check_launch("cache_gather_kernel");
+  if (st != SF_OK) return st;
+  SF_CHECK_CUDA(cudaEventRecord(c->ev_ready, ss));
+  c->ready_pending = true;
+  c->ready_capture = cid;
+  c->used_pending = false;
+  return SF_OK;
+}
+
+sf_status sf_refine_cache_sets(sf_refine_cache* c, int32_t* hits, int32_t* misses, int32_t* bypass,
+                               int32_t counts[3]) {
+  SF_REQUIRE(c && counts, "sf_refine_cache_sets: null pointer");
+  DeviceGuard g(c->device);
+  sf_status st = wait_ready(c);
+  if (st != SF_OK) return st;
+  int32_t meta[kMetaCount];
+  SF_CHECK_CUDA(cudaMemcpy(meta, c->meta, sizeof(meta), cudaMemcpyDeviceToHost));
+  counts[0] = meta[kHits];
+  counts[1] = meta[kMisses];
+  counts[2] = meta[kBypass];
+  if (hits && meta[kHits]) SF_CHECK_CUDA(cudaMemcpy(hits, c->hits, sizeof(int32_t) * meta[kHits], cudaMemcpyDeviceToHost));
+  if (misses && meta[kMisses])
+    SF_CHECK_CUDA(cudaMemcpy(misses, c->misses, sizeof(int32_t) * meta[kMisses], cudaMemcpyDeviceToHost));
+  if (bypass && meta[kBypass])
+    SF_CHECK_CUDA(cudaMemcpy(bypass, c->bypass, sizeof(int32_t) * meta[kBypass], cudaMemcpyDeviceToHost));
+  return SF_OK;
+}
+
+sf_status sf_refine_cache_slots(sf_refine_cache* c, int32_t* slot_units) {
+  SF_REQUIRE(c && slot_units, "sf_refine_cache_slots: null pointer");
+  DeviceGuard g(c->device);
+  sf_status st = wait_ready(c);
+  if (st != SF_OK) return st;
+  if (c->capacity)
+    SF_CHECK_CUDA(cudaMemcpy(slot_units, c->slot_unit, sizeof(int32_t) * c->capacity, cudaMemcpyDeviceToHost));
+  return SF_OK;
+}
+
+sf_status sf_refine_cache_stats(sf_refine_cache* c, sf_cache_stats* out) {
+  SF_REQUIRE(c && out, "sf_refine_cache_stats: null pointer");
+  DeviceGuard g(c->device);
+  sf_status st = wait_ready(c);
+  if (st != SF_OK) return st;
+  int64_t s[kStatCount];
+  SF_CHECK_CUDA(cudaMemcpy(s, c->stats, sizeof(s), cudaMemcpyDeviceToHost));
+  out->steps = s[kStSteps];
+  out->hits = s[kStHits];
+  out->misses = s[kStMisses];
+  out->bypass = s[kStBypass];
+  out->h2d_bytes = s[kStBytes];
+  return SF_OK;
+}
+
+sf_status sf_refine_cache_reset(sf_refine_cache* c) {
+  SF_REQUIRE(c, "sf_refine_cache_reset: null cache");
+  DeviceGuard g(c->device);
+  sf_status st = wait_ready(c);
+  if (st != SF_OK) return st;
+  if (c->used_pending) SF_CHECK_CUDA(cudaEventSynchronize(c->ev_used));
+  st = cache_clear(c, c->aux);
+  if (st != SF_OK) return st;
+  SF_CHECK_CUDA(cudaStreamSynchronize(c->aux));
+  c->ready_pending = c->used_pending = false;
+  return SF_OK;
+}
+
+sf_status sf_refine_cache_destroy(sf_refine_cache* c) { return cache_free(c); }
+
+}  // extern "C"

@@ -1,0 +1,184 @@
+// sf_select_topk: top-k input channels by |x| per batch row, union over rows.
+//
+// |x| of a bf16 value is its 15 low bits read as an unsigned integer (sign
+// dropped, so +0 and -0 tie and larger magnitudes give larger keys), which
+// makes the selection exact integer work.  One CTA of 1024 threads; each of
+// the B rows owns a contiguous slice of the threads and all rows advance
+// together through a two-pass radix select (8 high bits, then 7 low bits)
+// that finds the k-th largest key tau.  Keys above tau are taken; keys equal
+// to tau are taken in ascending channel order until k are chosen (an ordered
+// scan), which is the "ties to the lower index" rule.  A final ordered
+// compaction writes the union in ascending order.
+#include "block_scan.cuh"
+#include "sf_internal.h"
+
+namespace {
+
+constexpr int kThreads = 1024;
+constexpr int kMaxRows = 16;
+
+struct RowState {
+  int b1, k1;      // high-byte bin of the k-th key, rank left inside it
+  int tau, r;      // k-th largest key, how many keys equal to tau to take
+};
+
+__global__ void __launch_bounds__(kThreads)
+select_topk_kernel(const uint16_t* __restrict__ x, int B, int K, int k, int32_t* __restrict__ idx_out,
+                   int32_t* __restrict__ n_out) {
+  extern __shared__ uint8_t smem[];
+  uint8_t* flags = smem;                                                   // [K]
+  int* hist1 = reinterpret_cast<int*>(smem + ((K + 15) & ~15));           // [kMaxRows][256]
+  int* hist2 = hist1 + kMaxRows * 256;                                     // [kMaxRows][128]
+  __shared__ RowState st[kMaxRows];
+  __shared__ int scan_scratch[33];
+  __shared__ int bad;
+
+  const int tid = threadIdx.x;
+  int rb = 1;
+  while (rb < B) rb <<= 1;
+  const int tpr = kThreads / rb;  // threads per row
+  const int row = tid / tpr, lid = tid % tpr;
+  const bool active = row < B;
+  const uint16_t* xr = x + static_cast<size_t>(row) * K;
+
+  for (int j = tid; j < K; j += kThreads) flags[j] = 0;
+  for (int j = tid; j < kMaxRows * 256; j += kThreads) hist1[j] = 0;
+  for (int j = tid; j < kMaxRows * 128; j += kThreads) hist2[j] = 0;
+  if (tid == 0) bad = 0;
+  __syncthreads();
+
+  // pass 1: histogram of the high 8 bits of the 15-bit magnitude key
+  if (active) {
+    int* h = hist1 + row * 256;
+    for (int j = lid; j < K; j += tpr) {
+      const uint32_t v = xr[j];
+      if ((v & 0x7F80u) == 0x7F80u) bad = 1;  // Inf or NaN
+      atomicAdd(&h[(v & 0x7FFFu) >> 7], 1);
+    }
+  }
+  __syncthreads();
+  const int warp = tid >> 5, lane = tid & 31;
+  if (warp < B) {
+    // find the bin holding the k-th largest key: scan bins from the top
+    const int* h = hist1 + warp * 256;
+    int above = 0, b1 = -1, k1 = 0;
+    for (int base = 255; base >= 0 && b1 < 0; base -= 32) {
+      const int bin = base - lane;
+      const int c = h[bin];
+      int incl = c;  // inclusive prefix from the top within this chunk
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const bool hit = (above + incl >= k) && (above + incl - c < k);
+      const unsigned m = __ballot_sync(0xffffffffu, hit && k > 0);
+      if (m) {
+        const int src = __ffs(m) - 1;
+        b1 = base - src;
+        k1 = k - (above + __shfl_sync(0xffffffffu, incl - c, src));
+      }
+      above += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) { st[warp].b1 = b1; st[warp].k1 = k1; }
+  }
+  __syncthreads();
+  // pass 2: histogram of the low 7 bits inside that bin
+  if (active && st[row].b1 >= 0) {
+    int* h = hist2 + row * 128;
+    const int b1 = st[row].b1;
+    for (int j = lid; j < K; j += tpr) {
+      const uint32_t v = xr[j] & 0x7FFFu;
+      if (static_cast<int>(v >> 7) == b1) atomicAdd(&h[v & 0x7Fu], 1);
+    }
+  }
+  __syncthreads();
+  if (warp < B) {
+    const int* h = hist2 + warp * 128;
+    const int b1 = st[warp].b1, kk = st[warp].k1;
+    int above = 0, tau = -1, r = 0;
+    if (b1 >= 0) {
+      for (int base = 127; base >= 0 && tau < 0; base -= 32) {
+        const int bin = base - lane;
+        const int c = h[bin];
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const bool hit = (above + incl >= kk) && (above + incl - c < kk);
+        const unsigned m = __ballot_sync(0xffffffffu, hit);
+        if (m) {
+          const int src = __ffs(m) - 1;
+          tau = (b1 << 7) | (base - src);
+          r = kk - (above + __shfl_sync(0xffffffffu, incl - c, src));
+        }
+        above += __shfl_sync(0xffffffffu, incl, 31);
+      }
+    }
+    if (lane == 0) { st[warp].tau = tau; st[warp].r = r; }
+  }
+  __syncthreads();
+
+  // ordered pass: keys > tau always; keys == tau for the first r in index order
+  {
+    const int chunk = (K + tpr - 1) / tpr;
+    const int j0 = min(K, lid * chunk), j1 = min(K, j0 + chunk);
+    const int tau = active ? st[row].tau : -1;
+    int eq = 0;
+    if (active && tau >= 0)
+      for (int j = j0; j < j1; ++j) eq += ((xr[j] & 0x7FFF) == tau);
+    int total;
+    const int pre = sfd::block_exclusive_scan(eq, scan_scratch, &total);
+    // the row's threads are contiguous: subtract the prefix at its first thread
+    __shared__ int row_base[kMaxRows];
+    if (lid == 0 && active) row_base[row] = pre;
+    __syncthreads();
+    if (active && tau >= 0) {
+      int rank = pre - row_base[row];
+      const int r = st[row].r;
+      for (int j = j0; j < j1; ++j) {
+        const int key = xr[j] & 0x7FFF;
+        if (key > tau) {
+          flags[j] = 1;
+        } else if (key == tau) {
+          if (rank < r) flags[j] = 1;
+          ++rank;
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // ordered compaction of the union
+  {
+    const int chunk = (K + kThreads - 1) / kThreads;
+    const int j0 = min(K, tid * chunk), j1 = min(K, j0 + chunk);
+    int c = 0;
+    for (int j = j0; j < j1; ++j) c += flags[j];
+    int total;
+    int pos = sfd::block_exclusive_scan(c, scan_scratch, &total);
+    for (int j = j0; j < j1; ++j)
+      if (flags[j]) idx_out[pos++] = j;
+    if (tid == 0) *n_out = bad ? -1 : total;
+  }
+}
+
+}  // namespace
+
+extern "C" sf_status sf_select_topk(const uint16_t* x, int B, int K, int k, int32_t* idx_out, int32_t* n_out,
+                                    sf_stream_t stream) {
+  SF_REQUIRE(x && idx_out && n_out, "sf_select_topk: null pointer");
+  SF_REQUIRE(B >= 1 && B <= kMaxRows, "sf_select_topk: B must be in [1, %d]", kMaxRows);
+  SF_REQUIRE(K >= 1 && K <= 65536, "sf_select_topk: K must be in [1, 65536]");
+  SF_REQUIRE(k >= 0 && k <= K, "sf_select_topk: k must be in [0, K]");
+  const size_t smem = static_cast<size_t>((K + 15) & ~15) + sizeof(int) * kMaxRows * (256 + 128);
+  static bool attr_set = false;
+  if (!attr_set) {
+    SF_CHECK_CUDA(cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
+    attr_set = true;
+  }
+  select_topk_kernel<<<1, kThreads, smem, sf::as_cuda(stream)>>>(x, B, K, k, idx_out, n_out);
+  return sf::check_launch("select_topk_kernel");
+}

@@ -1,0 +1,78 @@
+// Internal helpers shared by the CUDA translation units of libsf.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <string>
+
+#include "sf.h"
+
+namespace sf {
+
+// Thread-local last error message (set on every non-OK return).
+void set_error(const std::string& msg);
+sf_status fail(sf_status st, const char* fmt, ...);
+sf_status cuda_fail(cudaError_t e, const char* what);
+
+inline cudaStream_t as_cuda(sf_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+#define SF_CHECK_CUDA(call)                                 \
+  do {                                                      \
+    cudaError_t e__ = (call);                               \
+    if (e__ != cudaSuccess) return ::sf::cuda_fail(e__, #call); \
+  } while (0)
+
+#define SF_REQUIRE(cond, ...)                                   \
+  do {                                                          \
+    if (!(cond)) return ::sf::fail(SF_EINVAL, __VA_ARGS__);     \
+  } while (0)
+
+// After a kernel launch: report launch-configuration errors.
+inline sf_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return SF_OK;
+}
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Device view of a refinement cache for the GEMV: where the rows live and
+// which row serves each selected position of the last prefetch.
+struct CacheView {
+  const uint32_t* rows;     // [(capacity + max_select)][unit_words]
+  const int32_t* row_of;    // [max_select]
+  int unit_words;
+};
+sf_status cache_view_for_gemv(sf_refine_cache* c, cudaStream_t stream, CacheView* v);
+sf_status cache_mark_used(sf_refine_cache* c, cudaStream_t stream);
+
+}  // namespace sf
+
+// -------- device helpers ------------------------------------------------
+namespace sfd {
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t h) {
+  return __half2float(__ushort_as_half(h));
+}
+
+// Read `bits` bits starting at stream bit `pos` of a little-endian uint32
+// bitstream (bits <= 8; may straddle a word boundary).
+__device__ __forceinline__ uint32_t read_bits(const uint32_t* s, uint32_t pos, int bits) {
+  uint32_t w = pos >> 5, sh = pos & 31;
+  uint64_t v = s[w];
+  if (sh + bits > 32) v |= static_cast<uint64_t>(s[w + 1]) << 32;
+  return static_cast<uint32_t>(v >> sh) & ((1u << bits) - 1u);
+}
+
+}  // namespace sfd

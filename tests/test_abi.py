@@ -1,0 +1,76 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point that include/sf.h declares, and rejects bad arguments on the host with
+a status code and a message (no device work is started by these calls)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[\w\s\*]*?\b(sf_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def sf():
+    import quantized_gemv_kv_b200 as sf
+    return sf
+
+
+def test_header_declares_the_hot_path():
+    names = _declared()
+    for want in ("sf_quantize_nested", "sf_select_topk", "sf_gemv_refine", "sf_attn_decode_refine",
+                 "sf_refine_cache_create", "sf_refine_cache_prefetch", "sf_refine_cache_destroy"):
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(sf):
+    lib = ctypes.CDLL(sf.LIB_PATH)
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(_declared()) <= set(sf.EXPORTED)
+
+
+def test_version_and_status_strings(sf):
+    assert "sm_100a" in sf.version()
+    assert sf._lib.sf_status_string(sf.SF_EINVAL) == b"SF_EINVAL"
+
+
+def _err(sf):
+    buf = ctypes.create_string_buffer(512)
+    sf._lib.sf_last_error(buf, len(buf))
+    return buf.value.decode()
+
+
+def test_host_validation(sf):
+    L = sf._lib
+    p = ctypes.c_void_p(16)
+    # bad bit widths, bad group size, misaligned layouts: rejected before any launch
+    assert L.sf_quantize_nested(p, 64, 64, 32, 5, 2, 0, p, p, p, p, None) == sf.SF_EINVAL
+    assert "b_r" in _err(sf)
+    assert L.sf_quantize_nested(p, 64, 64, 48, 2, 2, 0, p, p, p, p, None) == sf.SF_EINVAL
+    assert L.sf_quantize_nested(p, 48, 64, 32, 2, 2, 0, p, p, p, p, None) == sf.SF_EINVAL
+    assert L.sf_quantize_nested(None, 64, 64, 32, 2, 2, 0, p, p, p, p, None) == sf.SF_EINVAL
+    assert L.sf_select_topk(p, 17, 64, 4, p, p, None) == sf.SF_EINVAL
+    assert L.sf_select_topk(p, 1, 64, 65, p, p, None) == sf.SF_EINVAL
+    qw = sf._QWeight(16, 16, 16, None, 64, 64, 32, 2, 2)
+    assert L.sf_gemv_refine(ctypes.byref(qw), p, 17, None, None, None, p, None) == sf.SF_EINVAL
+    qw = sf._QWeight(16, 16, 16, None, 48, 64, 32, 2, 2)
+    assert L.sf_gemv_refine(ctypes.byref(qw), p, 1, None, None, None, p, None) == sf.SF_EINVAL
+    out = ctypes.c_size_t()
+    assert L.sf_attn_workspace_size(32, 8, 64, 1024, 10, ctypes.byref(out)) == sf.SF_EINVAL
+    assert L.sf_attn_workspace_size(32, 8, 128, 1024, 10, ctypes.byref(out)) == sf.SF_OK
+    assert out.value > 32 * 1024 * 4
+    h = ctypes.c_void_p()
+    assert L.sf_refine_cache_create(ctypes.byref(h), 64, 24, 8, 8, p, 0) == sf.SF_EINVAL
+    assert L.sf_refine_cache_destroy(None) == sf.SF_OK

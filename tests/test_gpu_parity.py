@@ -1,0 +1,326 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.
+
+Bit-exact: packed codes, fp16 scale/zero, selected channel indices, cache
+hit / miss / bypass sets and slot placement, selected token sets.
+Tolerance: refined GEMV |y - y_ref| <= 2e-3 * sum_j |w_eff x| per output;
+refined attention max-abs error <= 2e-3.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attn as oattn
+from oracle import cache as ocache
+from oracle import gemv as ogemv
+from oracle import quant as oquant
+from oracle import select as oselect
+from workloads import (count_fraction, gen_activations, gen_kv, gen_query, gen_weight, outlier_channels,
+                       f32_to_bf16_bits)
+
+pytestmark = pytest.mark.gpu
+
+GEMV_TOL = 2e-3
+ATTN_TOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def sf():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import quantized_gemv_kv_b200 as sf
+    return sf
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def u32(t):
+    return t.cpu().numpy().view(np.uint32)
+
+
+def f16(t):
+    return t.cpu().numpy().view(np.float16)
+
+
+def bf16_dev(bits):
+    return dev(bits.view(np.int16)).view(torch.bfloat16)
+
+
+# ---- quantization ----------------------------------------------------------
+
+@pytest.mark.parametrize("N,K,G,b_r,b_f,layout", [
+    (512, 512, 64, 2, 2, "by_column"),
+    (1024, 4096, 128, 2, 2, "by_column"),
+    (128, 384, 128, 3, 1, "by_column"),
+    (96, 256, 32, 2, 1, "by_column"),
+    (40, 256, 128, 2, 2, "by_row"),
+    (8, 128, 128, 2, 2, "by_row"),
+])
+def test_quantize_bit_exact(sf, N, K, G, b_r, b_f, layout):
+    W = gen_weight(100 + N + K, N, K)
+    qw = sf.quantize_nested(dev(W), G, b_r, b_f, layout)
+    torch.cuda.synchronize()
+    ref = oquant.pack_nested(oquant.quantize_nested(W, G, b_r, b_f), layout)
+    np.testing.assert_array_equal(u32(qw.res), ref["res"])
+    np.testing.assert_array_equal(u32(qw.ref), ref["ref"])
+    np.testing.assert_array_equal(f16(qw.scale).view(np.uint16), ref["scale"].view(np.uint16))
+    np.testing.assert_array_equal(f16(qw.zero).view(np.uint16), ref["zero"].view(np.uint16))
+
+
+def test_quantize_worked_examples(sf):
+    import json
+    import os
+    cases = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "quant_worked.json")))["cases"]
+    for c in cases:
+        if c["b_r"] + c["b_f"] != 4:
+            continue
+        row = np.tile(np.array(c["w"], np.float32), 8)     # one group of 32 with the same min/max
+        W = np.tile(row, (32, 1))
+        qw = sf.quantize_nested(dev(W), 32, c["b_r"], c["b_f"])
+        torch.cuda.synchronize()
+        codes = oquant.unpack_bits(u32(qw.res)[:1], 32, c["b_r"])[0]
+        assert codes[:4].tolist() == c["q_r"], c["name"]
+        assert float(f16(qw.scale)[0, 0]) == pytest.approx(c["scale"], abs=1e-12)
+        assert float(f16(qw.zero)[0, 0]) == c["zero"]
+        fcodes = oquant.unpack_bits(u32(qw.ref)[:4], 32, c["b_f"])[:, 0]
+        assert fcodes.tolist() == c["q_f"], c["name"]
+
+
+# ---- selection ------------------------------------------------------------
+
+@pytest.mark.parametrize("B,K,pct", [(1, 512, 5), (1, 4096, 3), (1, 14336, 3), (4, 4096, 5), (16, 12288, 5),
+                                     (3, 1000, 10), (1, 64, 100)])
+def test_select_exact(sf, B, K, pct):
+    k = count_fraction(pct, K)
+    x = gen_activations(200 + K + B, B, K, outlier_channels(7, K, max(1, K // 200)), 30.0)
+    idx, n = sf.select_topk(bf16_dev(x), k)
+    torch.cuda.synchronize()
+    want = oselect.select_topk(x, k)
+    got = idx.cpu().numpy()[: int(n.item())]
+    np.testing.assert_array_equal(got, want)
+
+
+def test_select_ties_and_edges(sf):
+    rng = np.random.default_rng(5)
+    K = 4096
+    levels = np.array([0.0, -0.0, 0.5, -0.5, 1.0, -1.0, 2.0], np.float32)
+    x = f32_to_bf16_bits(rng.choice(levels, size=(4, K)))
+    for k in (0, 1, 7, 100, 1500, K):
+        idx, n = sf.select_topk(bf16_dev(x), k)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(idx.cpu().numpy()[: int(n.item())], oselect.select_topk(x, k))
+    bad = x.copy()
+    bad[2, 17] = 0x7FC0  # NaN
+    idx, n = sf.select_topk(bf16_dev(bad), 10)
+    torch.cuda.synchronize()
+    assert int(n.item()) == -1
+
+
+# ---- refinement cache --------------------------------------------------------
+
+def _steps(seed, K, n_steps, k, hot):
+    rng = np.random.default_rng(seed)
+    hot_set = rng.choice(K, size=hot, replace=False)
+    for i in range(n_steps):
+        kk = k if i % 7 else 3 * k      # every 7th step overflows small caches (bypass)
+        rest = rng.choice(K, size=kk, replace=False)
+        yield np.array(sorted(set(hot_set.tolist()) | set(rest[:kk - hot].tolist())), np.int32)
+
+
+@pytest.mark.parametrize("K,N,b_f,C,k,hot", [(512, 256, 2, 40, 30, 5), (4096, 1024, 2, 410, 123, 20),
+                                             (1024, 128, 1, 16, 24, 4), (300, 128, 2, 300, 20, 3)])
+def test_cache_sets_and_slots(sf, K, N, b_f, C, k, hot):
+    unit_bytes = N * b_f // 8
+    rng = np.random.default_rng(K + C)
+    master = torch.from_numpy(rng.integers(0, 2 ** 31, size=(K, unit_bytes // 4), dtype=np.int64).astype(np.int32))
+    master = master.pin_memory()
+    max_sel = 3 * k + hot
+    cache = sf.RefineCache(K, unit_bytes, C, max_sel, master)
+    orc = ocache.LRUCache(K, C)
+    idx = torch.zeros(max_sel, dtype=torch.int32, device="cuda")
+    n = torch.zeros(1, dtype=torch.int32, device="cuda")
+    side = torch.cuda.Stream()
+    for S in _steps(K, K, 25, k, hot):
+        idx[: len(S)].copy_(dev(S))
+        n.fill_(len(S))
+        cache.prefetch(idx, n, torch.cuda.current_stream(), side)
+        got = cache.sets()
+        want = orc.step(S.tolist())
+        assert got["hits"] == want["hits"]
+        assert got["misses"] == want["misses"]
+        assert got["bypass"] == want["bypass"]
+        slots = cache.slots()
+        snap = orc.snapshot()
+        assert {u: s for s, u in enumerate(slots) if u >= 0} == snap
+    st = cache.stats()
+    assert st.steps == 25 and st.hits == orc.hits and st.misses == orc.misses and st.bypass == orc.bypass
+    assert st.h2d_bytes == orc.misses * unit_bytes
+    cache.reset()
+    assert cache.stats().steps == 0
+    cache.close()
+
+
+# ---- refined GEMV ----------------------------------------------------------------
+
+def _check_gemv(y_gpu, y_ref, abs_sum):
+    err = np.abs(y_gpu.astype(np.float64) - y_ref)
+    bound = GEMV_TOL * abs_sum
+    worst = (err / np.maximum(bound, 1e-300)).max()
+    assert np.all(err <= bound), f"worst err/bound = {worst:.3g}"
+
+
+def _host_master(qw):
+    return qw.ref.cpu().contiguous().pin_memory()
+
+
+def test_gemv_linear_512_preloaded_cache(sf):
+    """512x512, group 64, 2+2, 1% outliers x20, top-26, cache holds every column."""
+    N = K = 512
+    W = gen_weight(1000, N, K)
+    x = gen_activations(2000, 1, K, outlier_channels(5000, K, count_fraction(1, K)), 20.0)
+    qw = sf.quantize_nested(dev(W), 64, 2, 2)
+    k = count_fraction(5, K)
+    cache = sf.RefineCache(K, N * 2 // 8, K, k, _host_master(qw))
+    cache.preload(torch.arange(K, dtype=torch.int32, device="cuda"))
+    xd = bf16_dev(x)
+    idx, n = sf.select_topk(xd, k)
+    cache.prefetch(idx, n)
+    y = sf.gemv_refine(qw, xd, idx, n, cache=cache)
+    torch.cuda.synchronize()
+    assert cache.sets()["hits"] == oselect.select_topk(x, k).tolist()
+    qz = oquant.quantize_nested(W, 64, 2, 2)
+    y_ref, a = ogemv.gemv_refine(qz, x, oselect.select_topk(x, k))
+    _check_gemv(y.cpu().numpy(), y_ref, a)
+    # resident-only and every column refined (store read directly)
+    y0 = sf.gemv_refine(qw, xd)
+    all_idx = torch.arange(K, dtype=torch.int32, device="cuda")
+    all_n = torch.tensor([K], dtype=torch.int32, device="cuda")
+    y1 = sf.gemv_refine(qw, xd, all_idx, all_n, use_ref_store=True)
+    torch.cuda.synchronize()
+    r0, a0 = ogemv.gemv_refine(qz, x, [])
+    r1, a1 = ogemv.gemv_refine(qz, x, np.arange(K))
+    _check_gemv(y0.cpu().numpy(), r0, a0)
+    _check_gemv(y1.cpu().numpy(), r1, a1)
+    cache.close()
+
+
+@pytest.mark.parametrize("N,K,G,b_r,b_f,B,pct", [
+    (1024, 4096, 128, 3, 1, 1, 5), (1024, 4096, 128, 3, 1, 4, 5), (512, 4096, 128, 3, 1, 16, 5),
+    (256, 14336, 128, 2, 2, 1, 3), (4096, 1024, 128, 2, 2, 2, 3), (96, 2048, 64, 2, 1, 7, 5),
+])
+def test_gemv_store(sf, N, K, G, b_r, b_f, B, pct):
+    W = gen_weight(300 + N + K + B, N, K)
+    x = gen_activations(400 + B, B, K, outlier_channels(9, K, count_fraction("1/2", K)), 30.0)
+    qw = sf.quantize_nested(dev(W), G, b_r, b_f)
+    k = count_fraction(pct, K)
+    xd = bf16_dev(x)
+    idx, n = sf.select_topk(xd, k)
+    y = sf.gemv_refine(qw, xd, idx, n, use_ref_store=True)
+    torch.cuda.synchronize()
+    S = oselect.select_topk(x, k)
+    np.testing.assert_array_equal(idx.cpu().numpy()[: int(n.item())], S)
+    y_ref, a = ogemv.gemv_refine(oquant.quantize_nested(W, G, b_r, b_f), x, S)
+    _check_gemv(y.cpu().numpy(), y_ref, a)
+
+
+@pytest.mark.parametrize("N,K,cap_pct", [(14336, 4096, 10), (4096, 14336, 10)])
+def test_gemv_full_size_cache_sampled_rows(sf, N, K, cap_pct):
+    """Llama-3.1-8B gate/down shapes, 2+2, group 128, top 3%, 10% LRU cache,
+    several steps; the oracle checks 192 sampled rows each step."""
+    G, b_r, b_f = 128, 2, 2
+    W = gen_weight(1000 + N, N, K)
+    qw = sf.quantize_nested(dev(W), G, b_r, b_f)
+    k = count_fraction(3, K)
+    cap = count_fraction(cap_pct, K)
+    cache = sf.RefineCache(K, N * b_f // 8, cap, k, _host_master(qw))
+    orc = ocache.LRUCache(K, cap)
+    rows = np.sort(np.random.default_rng(N).choice(N, size=192, replace=False))
+    qz = oquant.quantize_nested(W[rows], G, b_r, b_f)
+    outl = outlier_channels(5000 + K, K, count_fraction("1/2", K))
+    side = torch.cuda.Stream()
+    for step in range(3):
+        x = gen_activations(2000 + step, 1, K, outl, 30.0)
+        xd = bf16_dev(x)
+        idx, n = sf.select_topk(xd, k)
+        cache.prefetch(idx, n, torch.cuda.current_stream(), side)
+        y = sf.gemv_refine(qw, xd, idx, n, cache=cache)
+        torch.cuda.synchronize()
+        S = oselect.select_topk(x, k)
+        want = orc.step(S.tolist())
+        got = cache.sets()
+        assert got["hits"] == want["hits"] and got["misses"] == want["misses"]
+        y_ref, a = ogemv.gemv_refine(qz, x, S)
+        _check_gemv(y.cpu().numpy()[:, rows], y_ref, a)
+    cache.close()
+
+
+# ---- refined attention -------------------------------------------------------------
+
+def _kv(sf, Hkv, T, d, seed, n_out=4):
+    Kf, Vf, _ = gen_kv(seed, Hkv, T, d, n_outlier_ch=n_out)
+    Kf2, Vf2 = Kf.reshape(Hkv * T, d), Vf.reshape(Hkv * T, d)
+    qk = sf.quantize_nested(dev(Kf2), d, 2, 2, "by_row")
+    qv = sf.quantize_nested(dev(Vf2), d, 2, 2, "by_row")
+    ok = oquant.quantize_nested(Kf2, d, 2, 2)
+    ov = oquant.quantize_nested(Vf2, d, 2, 2)
+    return sf.QKV(qk, qv), ok, ov
+
+
+@pytest.mark.parametrize("Hq,Hkv,T,pct", [(8, 2, 1000, 1), (32, 8, 4099, 1), (4, 4, 77, 10), (16, 2, 33, 100),
+                                          (8, 1, 512, 0)])
+def test_attn_small(sf, Hq, Hkv, T, pct):
+    d = 128
+    kv, ok, ov = _kv(sf, Hkv, T, d, 3000 + T)
+    qb = gen_query(4000 + T, Hq, d)
+    k = count_fraction(pct, T)
+    out, sel, sel_n = sf.attn_decode_refine(bf16_dev(qb), kv, Hkv, T, k)
+    torch.cuda.synchronize()
+    ref = oattn.attn_decode_refine(qb, ok, ov, Hkv, T, k)
+    sel_n = sel_n.cpu().numpy()
+    sel = sel.cpu().numpy()
+    for g in range(Hkv):
+        assert sel_n[g] == len(ref["union"][g])
+        np.testing.assert_array_equal(sel[g, : sel_n[g]], ref["union"][g])
+    err = np.abs(out.cpu().numpy().astype(np.float64) - ref["out"]).max()
+    assert err <= ATTN_TOL, err
+
+
+def test_attn_32k(sf):
+    """32K context, 32 query / 8 KV heads, head_dim 128, 2+2 K/V with 4
+    outlier key channels x10, top 1% tokens per query head."""
+    Hq, Hkv, T, d = 32, 8, 32768, 128
+    kv, ok, ov = _kv(sf, Hkv, T, d, 3000)
+    qb = gen_query(4000, Hq, d)
+    k = count_fraction(1, T)
+    out, sel, sel_n = sf.attn_decode_refine(bf16_dev(qb), kv, Hkv, T, k)
+    torch.cuda.synchronize()
+    ref = oattn.attn_decode_refine(qb, ok, ov, Hkv, T, k)
+    sel_n = sel_n.cpu().numpy()
+    sel = sel.cpu().numpy()
+    for g in range(Hkv):
+        np.testing.assert_array_equal(sel[g, : sel_n[g]], ref["union"][g])
+    err = np.abs(out.cpu().numpy().astype(np.float64) - ref["out"]).max()
+    assert err <= ATTN_TOL, err
+
+
+def test_attn_ties(sf):
+    """Duplicate tokens give exactly tied keys; the lower token index wins."""
+    Hq, Hkv, T, d = 8, 2, 600, 128
+    Kf, Vf, _ = gen_kv(77, Hkv, T, d)
+    for t in range(0, T, 5):
+        Kf[:, t] = Kf[:, 0]
+    Kf2, Vf2 = Kf.reshape(Hkv * T, d), Vf.reshape(Hkv * T, d)
+    kv = sf.QKV(sf.quantize_nested(dev(Kf2), d, 2, 2, "by_row"), sf.quantize_nested(dev(Vf2), d, 2, 2, "by_row"))
+    ok, ov = oquant.quantize_nested(Kf2, d, 2, 2), oquant.quantize_nested(Vf2, d, 2, 2)
+    qb = gen_query(78, Hq, d)
+    for k in (1, 13, 60, 200):
+        out, sel, sel_n = sf.attn_decode_refine(bf16_dev(qb), kv, Hkv, T, k)
+        torch.cuda.synchronize()
+        ref = oattn.attn_decode_refine(qb, ok, ov, Hkv, T, k)
+        for g in range(Hkv):
+            n = sel_n.cpu().numpy()[g]
+            np.testing.assert_array_equal(sel.cpu().numpy()[g, :n], ref["union"][g])
+        assert np.abs(out.cpu().numpy() - ref["out"]).max() <= ATTN_TOL
