@@ -272,6 +272,21 @@ def capture(torch, fn, stream):
     return g
 
 
+def reduce_max(value, dist, device):
+    """Max of a per-rank float over all ranks (identity without a group)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(bytes_per_step_per_rank, ms_per_step_max, world):
+    """Whole-job throughput: every rank's bytes over the slowest rank's time."""
+    return world * bytes_per_step_per_rank / (ms_per_step_max * 1e-3) / 1e9
+
+
 def timed(torch, dist, fn, iters, stream, sync_each=False):
     """Device time (ms) of `iters` calls of fn on `stream`, max over ranks."""
     if dist is not None:
@@ -287,11 +302,8 @@ def timed(torch, dist, fn, iters, stream, sync_each=False):
                 stream.synchronize()
         e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
+    ms = reduce_max(e0.elapsed_time(e1), dist, "cuda")
     if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     return ms
 
@@ -422,7 +434,7 @@ def run_sf(args, rank, world, local_rank, dist):
     attn_step_bytes = attn_bytes(T, union_per_layer) * args.layers
     step_bytes = gemv_step_bytes + attn_step_bytes
     ms_step = ms / args.steps
-    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    value = whole_job_gbs(step_bytes, ms_step, world)
     tok_s = world * 1e3 / ms_step
     h2d_step = (after["h2d_bytes"] - before["h2d_bytes"]) / args.steps
     hits = after["hits"] - before["hits"]
@@ -489,7 +501,7 @@ def run_sf(args, rank, world, local_rank, dist):
         ms_e2e /= args.steps
         bi = model.xin.numel() * 2 + model.qin.numel() * 2
         bo = model.y_all.numel() * 4 + model.attn_out.numel() * 4
-        e2e = {"value": world * step_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms_e2e,
+        e2e = {"value": whole_job_gbs(step_bytes, ms_e2e, world), "unit": "GB/s", "ms_per_step": ms_e2e,
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
 
     cpu = None

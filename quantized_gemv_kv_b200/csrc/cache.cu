@@ -290,6 +290,7 @@ sf_status cache_view_for_gemv(sf_refine_cache* c, cudaStream_t stream, CacheView
   v->rows = c->rows;
   v->row_of = c->row_of;
   v->unit_words = static_cast<int>(c->unit_bytes / 4);
+  v->max_select = c->max_select;
   return SF_OK;
 }
 
@@ -400,8 +401,9 @@ sf_status sf_refine_cache_prefetch(sf_refine_cache* c, const int32_t* idx, const
   SF_REQUIRE(c && idx && n, "sf_refine_cache_prefetch: null pointer");
   DeviceGuard g(c->device);
   cudaStream_t ps = sf::as_cuda(producer), ss = sf::as_cuda(side);
-  const unsigned long long cid = capture_id(ss);
-  SF_REQUIRE(capture_id(ps) == cid, "sf_refine_cache_prefetch: producer and side stream capture states differ");
+  // when the producer is being captured, waiting on its event forks the side
+  // stream into the same capture
+  const unsigned long long cid = capture_id(ps);
   SF_CHECK_CUDA(cudaEventRecord(c->ev_idx, ps));
   SF_CHECK_CUDA(cudaStreamWaitEvent(ss, c->ev_idx, 0));
   // the previous step's GEMV must have read the rows before they change

@@ -187,6 +187,7 @@ extern "C" sf_status sf_gemv_refine(const sf_qweight* W, const uint16_t* x, int 
   const uint32_t* ref_rows = nullptr;
   const int32_t* row_of = nullptr;
   int unit_words = W->N * W->b_f / 32;
+  int nmax = W->K;  // largest selection the correction may see
   if (c) {
     SF_REQUIRE(idx && n, "sf_gemv_refine: a cache needs the selection (idx, n)");
     sf::CacheView v{};
@@ -195,12 +196,15 @@ extern "C" sf_status sf_gemv_refine(const sf_qweight* W, const uint16_t* x, int 
     SF_REQUIRE(v.unit_words == unit_words, "sf_gemv_refine: cache unit size does not match N*b_f/8");
     ref_rows = v.rows;
     row_of = v.row_of;
+    nmax = v.max_select;
   } else if (W->ref) {
     SF_REQUIRE(idx && n, "sf_gemv_refine: a refinement store needs the selection (idx, n)");
     ref_rows = W->ref;
   }
-  sf_status st = W->b_r == 2 ? launch_br<2>(W, x, B, idx, n, ref_rows, row_of, unit_words, y, s)
-                             : launch_br<3>(W, x, B, idx, n, ref_rows, row_of, unit_words, y, s);
+  sf_status st = SF_OK;
+  if (!(B == 1 && sf::gemv_b1_try(W, x, idx, n, ref_rows, row_of, unit_words, nmax, y, s, &st)))
+    st = W->b_r == 2 ? launch_br<2>(W, x, B, idx, n, ref_rows, row_of, unit_words, y, s)
+                     : launch_br<3>(W, x, B, idx, n, ref_rows, row_of, unit_words, y, s);
   if (st != SF_OK) return st;
   if (c) return sf::cache_mark_used(c, s);
   return SF_OK;

@@ -49,9 +49,17 @@ struct CacheView {
   const uint32_t* rows;     // [(capacity + max_select)][unit_words]
   const int32_t* row_of;    // [max_select]
   int unit_words;
+  int max_select;
 };
 sf_status cache_view_for_gemv(sf_refine_cache* c, cudaStream_t stream, CacheView* v);
 sf_status cache_mark_used(sf_refine_cache* c, cudaStream_t stream);
+
+// Batch-1 2-bit GEMV on the integer dot-product path (gemv_b1.cu).  Returns
+// false when the shape is outside that kernel's range (the caller then runs
+// the generic kernel); otherwise launches it and reports through *st.
+bool gemv_b1_try(const sf_qweight* W, const uint16_t* x, const int32_t* idx, const int32_t* n,
+                 const uint32_t* ref_rows, const int32_t* row_of, int unit_words, int nmax, float* y,
+                 cudaStream_t s, sf_status* st);
 
 }  // namespace sf
 

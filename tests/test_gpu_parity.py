@@ -324,3 +324,41 @@ def test_attn_ties(sf):
             n = sel_n.cpu().numpy()[g]
             np.testing.assert_array_equal(sel.cpu().numpy()[g, :n], ref["union"][g])
         assert np.abs(out.cpu().numpy() - ref["out"]).max() <= ATTN_TOL
+
+
+@pytest.mark.parametrize("N,K,cap,pct", [(1024, 4096, 30, 3), (4096, 4096, 410, 3), (512, 8192, 50, 4),
+                                         (2048, 14336, 1434, 3)])
+def test_gemv_batch1_integer_path(sf, N, K, cap, pct):
+    """Batch 1, 2-bit, K a multiple of 1024: the fixed-point DP4A kernel.  The
+    activations mix zeros, values 2^-100 and outliers of 3e4 inside the same
+    32-column slabs; the cache is small enough that some steps bypass."""
+    G, b_r, b_f = 128, 2, 2
+    W = gen_weight(700 + N + K, N, K)
+    qw = sf.quantize_nested(dev(W), G, b_r, b_f)
+    qz = oquant.quantize_nested(W, G, b_r, b_f)
+    k = count_fraction(pct, K)
+    cache = sf.RefineCache(K, N * b_f // 8, cap, k, _host_master(qw))
+    orc = ocache.LRUCache(K, cap)
+    outl = outlier_channels(800 + K, K, count_fraction("1/2", K))
+    side = torch.cuda.Stream()
+    for step in range(4):
+        x = gen_activations(900 + step, 1, K, outl, 30.0)
+        rng = np.random.default_rng(step)
+        pos = rng.choice(K, size=24, replace=False)
+        x[0, pos[:8]] = 0
+        x[0, pos[8:16]] = f32_to_bf16_bits(np.full(8, 2.0 ** -100, np.float32))
+        x[0, pos[16:]] = f32_to_bf16_bits(np.array([3e4, -3e4] * 4, np.float32))
+        xd = bf16_dev(x)
+        idx, n = sf.select_topk(xd, k)
+        cache.prefetch(idx, n, torch.cuda.current_stream(), side)
+        y = sf.gemv_refine(qw, xd, idx, n, cache=cache)
+        y0 = sf.gemv_refine(qw, xd)
+        torch.cuda.synchronize()
+        S = oselect.select_topk(x, k)
+        want = orc.step(S.tolist())
+        assert cache.sets()["bypass"] == want["bypass"]
+        y_ref, a = ogemv.gemv_refine(qz, x, S)
+        _check_gemv(y.cpu().numpy(), y_ref, a)
+        r0, a0 = ogemv.gemv_refine(qz, x, [])
+        _check_gemv(y0.cpu().numpy(), r0, a0)
+    cache.close()
