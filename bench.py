@@ -136,6 +136,7 @@ class Model:
         self.sf, self.torch, self.L, self.T, self.dev = sf, torch, layers, T, device
         self.k_tok = count_fraction(TOK_PCT, T)
         self.mats = []
+        self.groups = []
         self.kv = []
         self.ksel = {s: count_fraction(TOPK_PCT, K) for s, K in SLOTS}
         ycount = sum(N for _, N, _, _ in MATS)
@@ -167,6 +168,8 @@ class Model:
                 row[name] = (qw, cache, self.y_all[l, yo:yo + N].view(1, N), slot)
                 yo += N
             self.mats.append(row)
+            self.groups.append(sf.RefineGroup([(cache, self.idx[slot][l], self.nsel[slot][l])
+                                               for qw, cache, y, slot in row.values()]))
             Kf, Vf = ds.kv(3000 + l, HKV, T, D, device=device)
             self.kv.append(sf.QKV(sf.quantize_nested(Kf, D, B_R, B_F, "by_row"),
                                   sf.quantize_nested(Vf, D, B_R, B_F, "by_row")))
@@ -207,8 +210,7 @@ class Model:
         def select_and_prefetch(l):
             for s, _ in SLOTS:
                 sf.select_topk(self.x(l, s), self.ksel[s], self.idx[s][l], self.nsel[s][l])
-            for name, (qw, cache, y, slot) in self.mats[l].items():
-                cache.prefetch(self.idx[slot][l], self.nsel[slot][l], main, self.side)
+            self.groups[l].prefetch(main, self.side)
 
         def gemv(l, name):
             qw, cache, y, slot = self.mats[l][name]
@@ -251,12 +253,14 @@ class Model:
 
     def launches_per_step(self, refine=True):
         n_mat = len(MATS) * self.L
-        attn = 5 * self.L if (refine and 0 < self.k_tok < self.T) else 4 * self.L
+        attn = 4 * self.L if (refine and 0 < self.k_tok < self.T) else 2 * self.L
         if not refine:
             return n_mat + 3 * self.L
-        return len(SLOTS) * self.L + 2 * n_mat + n_mat + attn
+        return len(SLOTS) * self.L + 2 * self.L + n_mat + attn
 
     def close(self):
+        for grp in self.groups:
+            grp.close()
         for row in self.mats:
             for qw, cache, y, slot in row.values():
                 cache.close()

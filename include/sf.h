@@ -199,6 +199,26 @@ sf_status sf_refine_cache_reset(sf_refine_cache* c);
 sf_status sf_refine_cache_destroy(sf_refine_cache* c);
 
 /*
+ * A group batches the prefetch of several caches whose selections live in
+ * fixed device buffers (typically the weight matrices of one layer): one
+ * launch resolves every cache's step (one CTA per cache) and one launch
+ * gathers all their misses, so the side stream carries two kernels per layer
+ * instead of two per matrix.  Semantics per cache are exactly those of
+ * sf_refine_cache_prefetch with (idx[i], n[i]).
+ *   caches  count distinct caches on one device (1 <= count <= 64);
+ *   idx, n  per cache, the device buffers its selection will be read from at
+ *           every sf_refine_group_prefetch (pointers captured at create).
+ * The group does not own the caches; destroy it before them.
+ */
+typedef struct sf_refine_group sf_refine_group;
+sf_status sf_refine_group_create(sf_refine_group** out, sf_refine_cache* const* caches,
+                                 const int32_t* const* idx, const int32_t* const* n, int count);
+/* One step for every cache of the group, on `side` after `producer`'s work. */
+sf_status sf_refine_group_prefetch(sf_refine_group* g, sf_stream_t producer, sf_stream_t side);
+/* Synchronizes the device, then frees the group.  NULL is accepted. */
+sf_status sf_refine_group_destroy(sf_refine_group* g);
+
+/*
  * sf_gemv_refine -- refined decode GEMV, y[b][i] = sum_j x[b][j] w_eff[i][j].
  *
  * Source: rag-lover.com explainer (解説): columns picked by activation

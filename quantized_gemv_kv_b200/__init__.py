@@ -74,6 +74,10 @@ _SIGS = {
     "sf_refine_cache_stats": ([_p, ctypes.POINTER(CacheStats)], _i),
     "sf_refine_cache_reset": ([_p], _i),
     "sf_refine_cache_destroy": ([_p], _i),
+    "sf_refine_group_create": ([ctypes.POINTER(_p), ctypes.POINTER(_p), ctypes.POINTER(_p), ctypes.POINTER(_p), _i],
+                               _i),
+    "sf_refine_group_prefetch": ([_p, _p, _p], _i),
+    "sf_refine_group_destroy": ([_p], _i),
     "sf_gemv_refine": ([ctypes.POINTER(_QWeight), _p, _i, _p, _p, _p, _p, _p], _i),
     "sf_attn_workspace_size": ([_i, _i, _i, _i, _i, ctypes.POINTER(_sz)], _i),
     "sf_attn_decode_refine": ([_p, _i, _i, _i, _i, ctypes.POINTER(_QKV), _i, _p, _p, _p, _p, _sz, _p], _i),
@@ -234,6 +238,38 @@ class RefineCache:
     def close(self) -> None:
         if getattr(self, "_h", None) is not None and self._h.value:
             _check(_lib.sf_refine_cache_destroy(self._h))
+            self._h = _p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class RefineGroup:
+    """Batched prefetch of several caches (``sf_refine_group_*``).  ``entries``
+    is a list of (RefineCache, idx tensor, n tensor); the tensors must keep
+    their storage for the group's lifetime (their device pointers are fixed at
+    creation)."""
+
+    def __init__(self, entries):
+        cnt = len(entries)
+        self._entries = list(entries)
+        caches = (_p * cnt)(*[c.handle for c, _, _ in entries])
+        idxs = (_p * cnt)(*[_ptr(i) for _, i, _ in entries])
+        ns = (_p * cnt)(*[_ptr(n) for _, _, n in entries])
+        h = _p()
+        _check(_lib.sf_refine_group_create(ctypes.byref(h), caches, idxs, ns, cnt))
+        self._h = h
+
+    def prefetch(self, producer: torch.cuda.Stream | None = None, side: torch.cuda.Stream | None = None) -> None:
+        _check(_lib.sf_refine_group_prefetch(self._h, _stream(producer),
+                                             _stream(side if side is not None else producer)))
+
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None and self._h.value:
+            _check(_lib.sf_refine_group_destroy(self._h))
             self._h = _p()
 
     def __del__(self):

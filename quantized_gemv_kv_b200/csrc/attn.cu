@@ -19,7 +19,8 @@
 //              refined (full-code) K and V for tokens in the union and the
 //              resident ones elsewhere -- refined tokens are computed directly,
 //              never by subtracting their resident contribution.
-//   M  merge   per query head: combine the splits' (max, sum, output).
+//   M  merge   per KV group, by the last CTA of pass B to finish: combine the
+//              splits' (max, sum, output).
 //
 // Every scratch array lives in the caller's workspace; nothing is allocated.
 #include <algorithm>
@@ -36,7 +37,7 @@ constexpr int kMaxGrp = 8;
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128), rounded to fp32
 
 struct Layout {
-  size_t score, cand, kap, sel, umask, part, smax, status, total;
+  size_t score, cand, kap, sel, umask, part, smax, status, count, total;
   int splits, tps, words_t;
 };
 
@@ -59,6 +60,7 @@ Layout make_layout(int Hq, int Hkv, int T, int k, int sms) {
   L.part = off; off = up256(off + sizeof(float) * Hq * static_cast<size_t>(L.splits) * (D + 2));
   L.smax = off; off = up256(off + sizeof(float) * Hkv);
   L.status = off; off = up256(off + sizeof(int32_t) * std::max(Hkv, 4));
+  L.count = off; off = up256(off + sizeof(int32_t) * Hkv);
   L.total = off;
   return L;
 }
@@ -137,6 +139,14 @@ attn_score_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k
   }
   const float m = warp_max(s);
   if ((threadIdx.x & 31) == 0) atomicMax(reinterpret_cast<unsigned int*>(smax + g), __float_as_uint(m));
+}
+
+// Histogram increment with same-bin lanes of a warp merged into one atomic;
+// bin < 0 means no increment.  Call with the whole warp.
+__device__ __forceinline__ void warp_hist_add(int* hist, int bin) {
+  const unsigned peers = __match_any_sync(0xffffffffu, bin);
+  const int leader = __ffs(peers) - 1;
+  if (bin >= 0 && (threadIdx.x & 31) == leader) atomicAdd(&hist[bin], __popc(peers));
 }
 
 // ---- pass S: exact per-head top-k ------------------------------------------
@@ -227,11 +237,16 @@ attn_select_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ 
     const int nb = 1 << widths[pass];
     for (int i = tid; i < nb; i += kSelThreads) hist[i] = 0;
     __syncthreads();
-    for (int t = tid; t < T; t += kSelThreads) {
-      const float v = sc[t];
-      if (pass == 0) amax = fmaxf(amax, fabsf(v));
-      const uint32_t key = okey32(v);
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shifts[pass]) & (nb - 1)], 1);
+    for (int t0 = tid - (tid & 31); t0 < T; t0 += kSelThreads) {
+      const int t = t0 + (tid & 31);
+      int bin = -1;
+      if (t < T) {
+        const float v = sc[t];
+        if (pass == 0) amax = fmaxf(amax, fabsf(v));
+        const uint32_t key = okey32(v);
+        if ((key & pmask) == prefix) bin = static_cast<int>((key >> shifts[pass]) & (nb - 1));
+      }
+      warp_hist_add(hist, bin);
     }
     __syncthreads();
     find_bin_from_top(hist, nb, kk, binfo);
@@ -300,9 +315,14 @@ attn_select_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ 
     const int shift = 56 - 8 * pass;
     for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
     __syncthreads();
-    for (int i = tid; i < ncand; i += kSelThreads) {
-      const unsigned long long key = okey64(kp[i]);
-      if ((key & pm64) == pre64) atomicAdd(&hist[(key >> shift) & 255], 1);
+    for (int i0 = tid - (tid & 31); i0 < ncand; i0 += kSelThreads) {
+      const int i = i0 + (tid & 31);
+      int bin = -1;
+      if (i < ncand) {
+        const unsigned long long key = okey64(kp[i]);
+        if ((key & pm64) == pre64) bin = static_cast<int>((key >> shift) & 255);
+      }
+      warp_hist_add(hist, bin);
     }
     __syncthreads();
     find_bin_from_top(hist, 256, kr, binfo);
@@ -385,7 +405,8 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
                 const uint16_t* __restrict__ k_zero, const uint32_t* __restrict__ v_res,
                 const uint32_t* __restrict__ v_ref, const uint16_t* __restrict__ v_scale,
                 const uint16_t* __restrict__ v_zero, int T, int tps, int words_t, int splits,
-                const float* __restrict__ score, const uint32_t* __restrict__ umask, float* __restrict__ part) {
+                const float* __restrict__ score, const uint32_t* __restrict__ umask, float* __restrict__ part,
+                int32_t* __restrict__ done, float* __restrict__ out) {
   __shared__ float qs[GRP][D];
   __shared__ float qsum[GRP];
   __shared__ uint32_t vr[4][32][kWordsPerRow];
@@ -518,24 +539,30 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
     }
     part[((static_cast<size_t>(g) * GRP + h) * splits + split) * (D + 2) + j] = acc;
   }
-}
-
-// ---- pass M: merge the splits ------------------------------------------------
-__global__ void __launch_bounds__(D)
-attn_merge_kernel(const float* __restrict__ part, int splits, float* __restrict__ out) {
-  const int h = blockIdx.x, d = threadIdx.x;
-  const float* p = part + static_cast<size_t>(h) * splits * (D + 2);
-  float M = -INFINITY;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, p[s * (D + 2)]);
-  float L = 0.0f, O = 0.0f;
-  for (int s = 0; s < splits; ++s) {
-    const float ms = p[s * (D + 2)];
-    if (ms == -INFINITY) continue;
-    const float f = __expf(ms - M);
-    L = fmaf(f, p[s * (D + 2) + 1], L);
-    O = fmaf(f, p[s * (D + 2) + 2 + d], O);
+  // the last CTA of this KV group to finish merges every split's partials
+  // (threadfence-then-count, so no CTA ever waits for another)
+  __shared__ int last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(done + g, 1) == splits - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  for (int e = threadIdx.x; e < GRP * D; e += blockDim.x) {
+    const int h = e / D, d = e % D;
+    const float* p = part + (static_cast<size_t>(g) * GRP + h) * splits * (D + 2);
+    float M = -INFINITY;
+    for (int sp = 0; sp < splits; ++sp) M = fmaxf(M, __ldcg(p + sp * (D + 2)));
+    float Lsum = 0.0f, O = 0.0f;
+    for (int sp = 0; sp < splits; ++sp) {
+      const float ms = __ldcg(p + sp * (D + 2));
+      if (ms == -INFINITY) continue;
+      const float f = __expf(ms - M);
+      Lsum = fmaf(f, __ldcg(p + sp * (D + 2) + 1), Lsum);
+      O = fmaf(f, __ldcg(p + sp * (D + 2) + 2 + d), O);
+    }
+    out[(static_cast<size_t>(g) * GRP + h) * D + d] = O / Lsum;
   }
-  out[static_cast<size_t>(h) * D + d] = O / L;
 }
 
 __global__ void fill_all_kernel(int T, int grp, int k, int words_t, uint32_t* umask, int32_t* sel_out,
@@ -597,12 +624,11 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
     }
   }
   dim3 gb(L.splits, Hkv);
+  int32_t* done = reinterpret_cast<int32_t*>(ws + L.count);
   attn_out_kernel<GRP><<<gb, 128, 0, s>>>(q, kv->k_res, kv->k_ref, kv->k_scale, kv->k_zero, kv->v_res, kv->v_ref,
-                                          kv->v_scale, kv->v_zero, T, L.tps, L.words_t, L.splits, score, umask, part);
-  sf_status st = sf::check_launch("attn_out_kernel");
-  if (st != SF_OK) return st;
-  attn_merge_kernel<<<Hq, D, 0, s>>>(part, L.splits, out);
-  return sf::check_launch("attn_merge_kernel");
+                                          kv->v_scale, kv->v_zero, T, L.tps, L.words_t, L.splits, score, umask, part,
+                                          done, out);
+  return sf::check_launch("attn_out_kernel");
 }
 
 }  // namespace

@@ -31,19 +31,44 @@ constexpr int kGatherThreads = 128;
 enum Meta { kOcc = 0, kStep, kHits, kMisses, kBypass, kGather, kMetaCount };
 enum Stat { kStSteps = 0, kStHits, kStMisses, kStBypass, kStBytes, kStatCount };
 
-// One cache step.  S = idx[0..n) ascending.
-__global__ void __launch_bounds__(kIndexThreads)
-cache_index_kernel(const int32_t* __restrict__ S, const int32_t* __restrict__ n_ptr, int max_select, int capacity,
-                   int64_t unit_bytes, int32_t* __restrict__ unit_slot, int32_t* __restrict__ slot_unit,
-                   int32_t* __restrict__ order, int32_t* __restrict__ order_tmp, int32_t* __restrict__ row_of,
-                   int32_t* __restrict__ hits_out, int32_t* __restrict__ misses_out, int32_t* __restrict__ bypass_out,
-                   int32_t* __restrict__ victim_unit, int32_t* __restrict__ victim_slot,
-                   int32_t* __restrict__ gather_unit, int32_t* __restrict__ gather_row, int32_t* __restrict__ meta,
-                   int64_t* __restrict__ stats) {
+// Everything one cache step touches on the device.
+struct CacheDev {
+  const int32_t* S;      // selection (ascending units)
+  const int32_t* n_ptr;  // its length
+  int max_select, capacity;
+  int64_t unit_bytes;
+  int32_t *unit_slot, *slot_unit, *order, *order_tmp, *row_of, *hits_out, *misses_out, *bypass_out, *victim_unit,
+      *victim_slot, *gather_unit, *gather_row, *meta;
+  int64_t* stats;
+  const uint4* master;  // device view of the host master
+  uint4* rows;
+  int unit_vec;         // unit_bytes / 16
+};
+
+// One cache step.  S = idx[0..n) ascending.  Runs in one CTA of
+// kIndexThreads threads with `capacity` bytes of dynamic shared memory.
+__device__ void cache_step(const CacheDev& d) {
+  const int32_t* __restrict__ S = d.S;
+  const int max_select = d.max_select, capacity = d.capacity;
+  int32_t* __restrict__ unit_slot = d.unit_slot;
+  int32_t* __restrict__ slot_unit = d.slot_unit;
+  int32_t* __restrict__ order = d.order;
+  int32_t* __restrict__ order_tmp = d.order_tmp;
+  int32_t* __restrict__ row_of = d.row_of;
+  int32_t* __restrict__ hits_out = d.hits_out;
+  int32_t* __restrict__ misses_out = d.misses_out;
+  int32_t* __restrict__ bypass_out = d.bypass_out;
+  int32_t* __restrict__ victim_unit = d.victim_unit;
+  int32_t* __restrict__ victim_slot = d.victim_slot;
+  int32_t* __restrict__ gather_unit = d.gather_unit;
+  int32_t* __restrict__ gather_row = d.gather_row;
+  int32_t* __restrict__ meta = d.meta;
+  int64_t* __restrict__ stats = d.stats;
+  const int64_t unit_bytes = d.unit_bytes;
   extern __shared__ uint8_t slot_hit[];  // [capacity]
   __shared__ int scratch[33];
   const int tid = threadIdx.x;
-  int n = *n_ptr;
+  int n = *d.n_ptr;
   n = n < 0 ? 0 : (n > max_select ? max_select : n);
   const int occ = meta[kOcc];
 
@@ -159,15 +184,65 @@ cache_index_kernel(const int32_t* __restrict__ S, const int32_t* __restrict__ n_
   }
 }
 
-// Copy every missed unit from the device-mapped host master into its row.
-__global__ void __launch_bounds__(kGatherThreads)
-cache_gather_kernel(const uint4* __restrict__ master, uint4* __restrict__ rows, const int32_t* __restrict__ gather_unit,
-                    const int32_t* __restrict__ gather_row, const int32_t* __restrict__ meta, int unit_vec) {
-  const int n = meta[kGather];
-  for (int e = blockIdx.x; e < n; e += gridDim.x) {
-    const uint4* src = master + static_cast<size_t>(gather_unit[e]) * unit_vec;
-    uint4* dst = rows + static_cast<size_t>(gather_row[e]) * unit_vec;
-    for (int w = threadIdx.x; w < unit_vec; w += kGatherThreads) dst[w] = src[w];
+__global__ void __launch_bounds__(kIndexThreads) cache_index_kernel(CacheDev d) { cache_step(d); }
+
+// One CTA per cache of a group.
+__global__ void __launch_bounds__(kIndexThreads) cache_index_many_kernel(const CacheDev* __restrict__ table) {
+  cache_step(table[blockIdx.x]);
+}
+
+// Copy the missed units of `count` caches: one warp per unit, every lane
+// keeping several 16-byte loads from the host link in flight.
+__global__ void __launch_bounds__(256)
+cache_gather_many_kernel(const CacheDev* __restrict__ table, int count) {
+  __shared__ int offs[65];
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int c = 0; c < count; ++c) { offs[c] = acc; acc += table[c].meta[kGather]; }
+    offs[count] = acc;
+  }
+  __syncthreads();
+  const int total = offs[count];
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int nwarps = gridDim.x * (blockDim.x >> 5);
+  for (int e = gw; e < total; e += nwarps) {
+    int c = 0;
+    while (offs[c + 1] <= e) ++c;
+    const CacheDev& d = table[c];
+    const int i = e - offs[c];
+    const uint4* src = d.master + static_cast<size_t>(d.gather_unit[i]) * d.unit_vec;
+    uint4* dst = d.rows + static_cast<size_t>(d.gather_row[i]) * d.unit_vec;
+    for (int w = lane; w < d.unit_vec; w += 4 * 32) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (w + 32 * u < d.unit_vec) v[u] = src[w + 32 * u];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (w + 32 * u < d.unit_vec) dst[w + 32 * u] = v[u];
+    }
+  }
+}
+
+// Copy every missed unit of one cache (descriptor by value).
+__global__ void __launch_bounds__(256) cache_gather_kernel(CacheDev d) {
+  const int n = d.meta[kGather];
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int nwarps = gridDim.x * (blockDim.x >> 5);
+  for (int i = gw; i < n; i += nwarps) {
+    const uint4* src = d.master + static_cast<size_t>(d.gather_unit[i]) * d.unit_vec;
+    uint4* dst = d.rows + static_cast<size_t>(d.gather_row[i]) * d.unit_vec;
+    for (int w = lane; w < d.unit_vec; w += 4 * 32) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (w + 32 * u < d.unit_vec) v[u] = src[w + 32 * u];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (w + 32 * u < d.unit_vec) dst[w + 32 * u] = v[u];
+    }
   }
 }
 
@@ -234,6 +309,33 @@ struct sf_refine_cache {
 };
 
 namespace {
+
+CacheDev make_dev(const sf_refine_cache* c, const int32_t* S, const int32_t* n) {
+  CacheDev d{};
+  d.S = S;
+  d.n_ptr = n;
+  d.max_select = c->max_select;
+  d.capacity = c->capacity;
+  d.unit_bytes = static_cast<int64_t>(c->unit_bytes);
+  d.unit_slot = c->unit_slot;
+  d.slot_unit = c->slot_unit;
+  d.order = c->order;
+  d.order_tmp = c->order_tmp;
+  d.row_of = c->row_of;
+  d.hits_out = c->hits;
+  d.misses_out = c->misses;
+  d.bypass_out = c->bypass;
+  d.victim_unit = c->victim_unit;
+  d.victim_slot = c->victim_slot;
+  d.gather_unit = c->gather_unit;
+  d.gather_row = c->gather_row;
+  d.meta = c->meta;
+  d.stats = c->stats;
+  d.master = static_cast<const uint4*>(c->master_dev);
+  d.rows = reinterpret_cast<uint4*>(c->rows);
+  d.unit_vec = static_cast<int>(c->unit_bytes / 16);
+  return d;
+}
 
 sf_status cache_free(sf_refine_cache* c) {
   if (!c) return SF_OK;
@@ -409,16 +511,12 @@ sf_status sf_refine_cache_prefetch(sf_refine_cache* c, const int32_t* idx, const
   // the previous step's GEMV must have read the rows before they change
   if (c->used_pending && c->used_capture == cid) SF_CHECK_CUDA(cudaStreamWaitEvent(ss, c->ev_used, 0));
   const size_t smem = std::max(c->capacity, 1);
-  cache_index_kernel<<<1, kIndexThreads, smem, ss>>>(
-      idx, n, c->max_select, c->capacity, static_cast<int64_t>(c->unit_bytes), c->unit_slot, c->slot_unit, c->order,
-      c->order_tmp, c->row_of, c->hits, c->misses, c->bypass, c->victim_unit, c->victim_slot, c->gather_unit,
-      c->gather_row, c->meta, c->stats);
+  const CacheDev d = make_dev(c, idx, n);
+  cache_index_kernel<<<1, kIndexThreads, smem, ss>>>(d);
   sf_status st = sf::check_launch("cache_index_kernel");
   if (st != SF_OK) return st;
-  const int grid = std::min(c->max_select, 2 * sf::sm_count());
-  cache_gather_kernel<<<grid, kGatherThreads, 0, ss>>>(static_cast<const uint4*>(c->master_dev),
-                                                       reinterpret_cast<uint4*>(c->rows), c->gather_unit,
-                                                       c->gather_row, c->meta, static_cast<int>(c->unit_bytes / 16));
+  const int grid = std::min((c->max_select + 7) / 8, 2 * sf::sm_count());
+  cache_gather_kernel<<<grid, 256, 0, ss>>>(d);
   st = sf::check_launch("cache_gather_kernel");
   if (st != SF_OK) return st;
   SF_CHECK_CUDA(cudaEventRecord(c->ev_ready, ss));
@@ -486,5 +584,89 @@ sf_status sf_refine_cache_reset(sf_refine_cache* c) {
 }
 
 sf_status sf_refine_cache_destroy(sf_refine_cache* c) { return cache_free(c); }
+
+// ---- groups: one index launch and one gather launch for several caches ----
+
+}  // extern "C"
+
+struct sf_refine_group {
+  int device = 0;
+  int count = 0;
+  std::vector<sf_refine_cache*> caches;
+  CacheDev* table = nullptr;  // device copy of the descriptors
+  int max_capacity = 1;
+  int total_select = 0;
+  cudaEvent_t ev_idx = nullptr;
+};
+
+extern "C" {
+
+sf_status sf_refine_group_create(sf_refine_group** out, sf_refine_cache* const* caches, const int32_t* const* idx,
+                                 const int32_t* const* n, int count) {
+  SF_REQUIRE(out && caches && idx && n, "sf_refine_group_create: null pointer");
+  *out = nullptr;
+  SF_REQUIRE(count >= 1 && count <= 64, "sf_refine_group_create: count must be in [1, 64]");
+  for (int i = 0; i < count; ++i) {
+    SF_REQUIRE(caches[i] && idx[i] && n[i], "sf_refine_group_create: null entry %d", i);
+    SF_REQUIRE(caches[i]->device == caches[0]->device, "sf_refine_group_create: caches on different devices");
+    for (int j = 0; j < i; ++j) SF_REQUIRE(caches[j] != caches[i], "sf_refine_group_create: cache listed twice");
+  }
+  DeviceGuard g(caches[0]->device);
+  auto* grp = new sf_refine_group();
+  grp->device = caches[0]->device;
+  grp->count = count;
+  std::vector<CacheDev> host(count);
+  for (int i = 0; i < count; ++i) {
+    grp->caches.push_back(caches[i]);
+    host[i] = make_dev(caches[i], idx[i], n[i]);
+    grp->max_capacity = std::max(grp->max_capacity, caches[i]->capacity);
+    grp->total_select += caches[i]->max_select;
+  }
+  cudaError_t e = cudaMalloc(&grp->table, sizeof(CacheDev) * count);
+  if (e == cudaSuccess) e = cudaMemcpy(grp->table, host.data(), sizeof(CacheDev) * count, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&grp->ev_idx, cudaEventDisableTiming);
+  if (e != cudaSuccess) {
+    if (grp->table) cudaFree(grp->table);
+    delete grp;
+    return sf::cuda_fail(e, "sf_refine_group_create");
+  }
+  *out = grp;
+  return SF_OK;
+}
+
+sf_status sf_refine_group_prefetch(sf_refine_group* grp, sf_stream_t producer, sf_stream_t side) {
+  SF_REQUIRE(grp, "sf_refine_group_prefetch: null group");
+  DeviceGuard g(grp->device);
+  cudaStream_t ps = sf::as_cuda(producer), ss = sf::as_cuda(side);
+  const unsigned long long cid = capture_id(ps);
+  SF_CHECK_CUDA(cudaEventRecord(grp->ev_idx, ps));
+  SF_CHECK_CUDA(cudaStreamWaitEvent(ss, grp->ev_idx, 0));
+  for (sf_refine_cache* c : grp->caches)
+    if (c->used_pending && c->used_capture == cid) SF_CHECK_CUDA(cudaStreamWaitEvent(ss, c->ev_used, 0));
+  cache_index_many_kernel<<<grp->count, kIndexThreads, grp->max_capacity, ss>>>(grp->table);
+  sf_status st = sf::check_launch("cache_index_many_kernel");
+  if (st != SF_OK) return st;
+  const int grid = std::min((grp->total_select + 7) / 8, 4 * sf::sm_count());
+  cache_gather_many_kernel<<<grid, 256, 0, ss>>>(grp->table, grp->count);
+  st = sf::check_launch("cache_gather_many_kernel");
+  if (st != SF_OK) return st;
+  for (sf_refine_cache* c : grp->caches) {
+    SF_CHECK_CUDA(cudaEventRecord(c->ev_ready, ss));
+    c->ready_pending = true;
+    c->ready_capture = cid;
+    c->used_pending = false;
+  }
+  return SF_OK;
+}
+
+sf_status sf_refine_group_destroy(sf_refine_group* grp) {
+  if (!grp) return SF_OK;
+  DeviceGuard g(grp->device);
+  cudaDeviceSynchronize();
+  if (grp->table) cudaFree(grp->table);
+  if (grp->ev_idx) cudaEventDestroy(grp->ev_idx);
+  delete grp;
+  return SF_OK;
+}
 
 }  // extern "C"

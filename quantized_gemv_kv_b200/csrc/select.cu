@@ -17,6 +17,15 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kMaxRows = 16;
 
+// Histogram increment with the lanes of a warp that hit the same bin merged
+// into one atomic (keys cluster in few bins, so plain atomics serialise).
+// bin < 0 means "no increment".  Call with the whole warp.
+__device__ __forceinline__ void warp_hist_add(int* hist, int bin) {
+  const unsigned peers = __match_any_sync(0xffffffffu, bin);
+  const int leader = __ffs(peers) - 1;
+  if (bin >= 0 && (threadIdx.x & 31) == leader) atomicAdd(&hist[bin], __popc(peers));
+}
+
 struct RowState {
   int b1, k1;      // high-byte bin of the k-th key, rank left inside it
   int tau, r;      // k-th largest key, how many keys equal to tau to take
@@ -50,10 +59,14 @@ select_topk_kernel(const uint16_t* __restrict__ x, int B, int K, int k, int32_t*
   // pass 1: histogram of the high 8 bits of the 15-bit magnitude key
   if (active) {
     int* h = hist1 + row * 256;
-    for (int j = lid; j < K; j += tpr) {
-      const uint32_t v = xr[j];
-      if ((v & 0x7F80u) == 0x7F80u) bad = 1;  // Inf or NaN
-      atomicAdd(&h[(v & 0x7FFFu) >> 7], 1);
+    // trip count is uniform across a warp (tpr is a multiple of 32), so the
+    // whole warp takes part in each aggregation round
+    for (int j0 = lid - (lid & 31); j0 < K; j0 += tpr) {
+      const int j = j0 + (lid & 31);
+      const bool in = j < K;
+      const uint32_t v = in ? xr[j] : 0u;
+      if (in && (v & 0x7F80u) == 0x7F80u) bad = 1;  // Inf or NaN
+      warp_hist_add(h, in ? static_cast<int>((v & 0x7FFFu) >> 7) : -1);
     }
   }
   __syncthreads();
@@ -87,9 +100,10 @@ select_topk_kernel(const uint16_t* __restrict__ x, int B, int K, int k, int32_t*
   if (active && st[row].b1 >= 0) {
     int* h = hist2 + row * 128;
     const int b1 = st[row].b1;
-    for (int j = lid; j < K; j += tpr) {
-      const uint32_t v = xr[j] & 0x7FFFu;
-      if (static_cast<int>(v >> 7) == b1) atomicAdd(&h[v & 0x7Fu], 1);
+    for (int j0 = lid - (lid & 31); j0 < K; j0 += tpr) {
+      const int j = j0 + (lid & 31);
+      const uint32_t v = j < K ? (xr[j] & 0x7FFFu) : 0xFFFFu;
+      warp_hist_add(h, (j < K && static_cast<int>(v >> 7) == b1) ? static_cast<int>(v & 0x7Fu) : -1);
     }
   }
   __syncthreads();

@@ -362,3 +362,38 @@ def test_gemv_batch1_integer_path(sf, N, K, cap, pct):
         r0, a0 = ogemv.gemv_refine(qz, x, [])
         _check_gemv(y0.cpu().numpy(), r0, a0)
     cache.close()
+
+
+def test_cache_group_matches_oracle(sf):
+    """A group prefetch of three caches (different unit sizes and capacities,
+    one of them overflowing into bypass) equals three independent LRU steps."""
+    specs = [(4096, 1024, 410, 123), (4096, 256, 40, 123), (14336, 1024, 200, 430)]
+    side = torch.cuda.Stream()
+    entries, orcs, masters, xs = [], [], [], []
+    for i, (K, unit, cap, k) in enumerate(specs):
+        rng = np.random.default_rng(50 + i)
+        m = torch.from_numpy(rng.integers(0, 2 ** 31, size=(K, unit // 4), dtype=np.int64).astype(np.int32))
+        masters.append(m.pin_memory())
+        cache = sf.RefineCache(K, unit, cap, k, masters[-1])
+        idx = torch.zeros(k, dtype=torch.int32, device="cuda")
+        n = torch.zeros(1, dtype=torch.int32, device="cuda")
+        entries.append((cache, idx, n))
+        orcs.append(ocache.LRUCache(K, cap))
+    grp = sf.RefineGroup(entries)
+    for step in range(6):
+        sels = []
+        for i, (K, unit, cap, k) in enumerate(specs):
+            x = gen_activations(60 + 10 * step + i, 1, K, outlier_channels(70 + i, K, count_fraction("1/2", K)), 30.0)
+            sf.select_topk(bf16_dev(x), k, entries[i][1], entries[i][2])
+            sels.append(oselect.select_topk(x, k))
+        grp.prefetch(torch.cuda.current_stream(), side)
+        torch.cuda.synchronize()
+        for i, (cache, idx, n) in enumerate(entries):
+            want = orcs[i].step(sels[i].tolist())
+            got = cache.sets()
+            assert got["hits"] == want["hits"] and got["misses"] == want["misses"]
+            assert got["bypass"] == want["bypass"]
+            assert {u: s for s, u in enumerate(cache.slots()) if u >= 0} == orcs[i].snapshot()
+    grp.close()
+    for cache, _, _ in entries:
+        cache.close()
