@@ -286,6 +286,29 @@ sf_status sf_attn_decode_refine(const uint16_t* q, int Hq, int Hkv, int d, int T
                                 int32_t* sel_n, float* out, void* workspace, size_t ws_bytes,
                                 sf_stream_t stream);
 
+/*
+ * sf_attn_decode_refine_noalloc -- sf_attn_decode_refine without a caller
+ * workspace and without any device allocation.  The paper has no
+ * counterpart; this exists for callers that cannot allocate device memory
+ * when attention runs (a runtime with a fixed, pre-reserved memory pool, a
+ * plugin that is handed no scratch, code where cudaMalloc is not allowed or
+ * would synchronize the device).
+ *
+ * Same arguments, semantics and accuracy as sf_attn_decode_refine minus
+ * workspace/ws_bytes.  Scratch comes from one 24 MiB array compiled into the
+ * library (every GPU that loads the library reserves it until the process
+ * exits); sizes whose scratch would exceed it (sf_attn_workspace_size > 24 MiB,
+ * e.g. Hq * T above roughly 1.4 million) are rejected with SF_EINVAL before
+ * anything is enqueued.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture.  Every call reuses the same array and
+ * clears what must start at zero, so calls whose work overlaps on the GPU
+ * (unordered streams) race; order them on one stream.
+ */
+sf_status sf_attn_decode_refine_noalloc(const uint16_t* q, int Hq, int Hkv, int d, int T,
+                                        const sf_qkv* kv, int k_tokens, int32_t* sel_out,
+                                        int32_t* sel_n, float* out, sf_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

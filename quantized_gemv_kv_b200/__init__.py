@@ -81,6 +81,7 @@ _SIGS = {
     "sf_gemv_refine": ([ctypes.POINTER(_QWeight), _p, _i, _p, _p, _p, _p, _p], _i),
     "sf_attn_workspace_size": ([_i, _i, _i, _i, _i, ctypes.POINTER(_sz)], _i),
     "sf_attn_decode_refine": ([_p, _i, _i, _i, _i, ctypes.POINTER(_QKV), _i, _p, _p, _p, _p, _sz, _p], _i),
+    "sf_attn_decode_refine_noalloc": ([_p, _i, _i, _i, _i, ctypes.POINTER(_QKV), _i, _p, _p, _p, _p], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -341,3 +342,17 @@ def attn_decode_refine(q: torch.Tensor, kv: QKV, Hkv: int, T: int, k_tokens: int
                                       _ptr(sel_n), _ptr(out), _ptr(workspace),
                                       workspace.numel() * workspace.element_size(), _stream(stream)))
     return out, sel_out, sel_n
+
+
+def attn_decode_refine_noalloc(q: torch.Tensor, kv: QKV, Hkv: int, T: int, k_tokens: int,
+                               out: torch.Tensor, sel_out: torch.Tensor, sel_n: torch.Tensor,
+                               stream: torch.cuda.Stream | None = None) -> None:
+    """Refined decode attention with the library's built-in scratch
+    (``sf_attn_decode_refine_noalloc``): for callers that must not allocate
+    device memory at this point.  The caller provides the outputs; nothing
+    is allocated by this call."""
+    _dev(q, "q")
+    Hq, d = q.shape
+    s = kv.c_struct()
+    _check(_lib.sf_attn_decode_refine_noalloc(_ptr(q), Hq, Hkv, d, T, ctypes.byref(s), k_tokens, _ptr(sel_out),
+                                              _ptr(sel_n), _ptr(out), _stream(stream)))

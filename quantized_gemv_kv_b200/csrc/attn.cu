@@ -25,6 +25,7 @@
 // Every scratch array lives in the caller's workspace; nothing is allocated.
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 
 #include "block_scan.cuh"
 #include "sf_internal.h"
@@ -668,5 +669,82 @@ extern "C" sf_status sf_attn_decode_refine(const uint16_t* q, int Hq, int Hkv, i
     case 4: return run<4>(q, Hq, Hkv, T, kv, k_tokens, sel_out, sel_n, out, ws, L, s);
     case 8: return run<8>(q, Hq, Hkv, T, kv, k_tokens, sel_out, sel_n, out, ws, L, s);
     default: return sf::fail(SF_ENOTIMPL, "sf_attn_decode_refine: Hq/Hkv must be 1, 2, 4 or 8");
+  }
+}
+
+// ---- refined attention without any device allocation ------------------------
+//
+// Some callers cannot allocate device memory at the point where they run
+// attention: a serving runtime that owns a fixed memory pool and forbids
+// allocations after start-up, a plugin inside a host framework that hands out
+// no scratch, or code running where cudaMalloc would synchronize the device
+// or is not permitted.  For them this variant takes its scratch from one
+// array compiled into the library instead of from a caller workspace.
+//
+// The array is a file-scope __device__ symbol: every GPU that loads the
+// library reserves it (kStaticScratchBytes) for the life of the process.  In
+// host code its name is only a host-side stand-in, so the device address is
+// looked up with cudaGetSymbolAddress, once per device, with that device
+// current, on the first call made on that device.  All calls share the array;
+// the per-call counters it holds are cleared at the start of every call, and
+// calls whose work overlaps on the GPU (different streams, no ordering) race
+// on it.
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t{24} << 20;  // 24 MiB
+__device__ __align__(256) unsigned char g_attn_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+sf_status static_scratch_address(void** out) {
+  int dev = 0;
+  SF_CHECK_CUDA(cudaGetDevice(&dev));
+  SF_REQUIRE(dev >= 0 && dev < kMaxDevices, "sf_attn_decode_refine_noalloc: device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_attn_scratch);
+    if (e != cudaSuccess) return sf::cuda_fail(e, "cudaGetSymbolAddress(attention scratch)");
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return SF_OK;
+}
+
+}  // namespace
+
+extern "C" sf_status sf_attn_decode_refine_noalloc(const uint16_t* q, int Hq, int Hkv, int d, int T,
+                                                   const sf_qkv* kv, int k_tokens, int32_t* sel_out, int32_t* sel_n,
+                                                   float* out, sf_stream_t stream) {
+  SF_REQUIRE(q && kv && sel_out && sel_n && out, "sf_attn_decode_refine_noalloc: null pointer");
+  SF_REQUIRE(kv->k_res && kv->k_ref && kv->v_res && kv->v_ref && kv->k_scale && kv->k_zero && kv->v_scale &&
+                 kv->v_zero,
+             "sf_attn_decode_refine_noalloc: null K/V view");
+  SF_REQUIRE(kv->b_r == 2 && kv->b_f == 2, "sf_attn_decode_refine_noalloc: only 2-bit resident + 2-bit refinement K/V");
+  SF_REQUIRE(d == D, "sf_attn_decode_refine_noalloc: head dim must be %d", D);
+  SF_REQUIRE(Hkv >= 1 && Hq >= Hkv && Hq % Hkv == 0, "sf_attn_decode_refine_noalloc: Hq must be a multiple of Hkv");
+  SF_REQUIRE(T >= 1 && T <= (1 << 24), "sf_attn_decode_refine_noalloc: T out of range");
+  SF_REQUIRE(k_tokens >= 0 && k_tokens <= T, "sf_attn_decode_refine_noalloc: k_tokens must be in [0, T]");
+  SF_REQUIRE(sf::aligned(kv->k_res, 16) && sf::aligned(kv->v_res, 16) && sf::aligned(kv->k_ref, 16) &&
+                 sf::aligned(kv->v_ref, 16),
+             "sf_attn_decode_refine_noalloc: code arrays must be 16-byte aligned");
+  const Layout L = make_layout(Hq, Hkv, T, k_tokens, sf::sm_count());
+  SF_REQUIRE(L.total <= kStaticScratchBytes,
+             "sf_attn_decode_refine_noalloc: these sizes need %zu bytes of scratch but the built-in array holds %zu; "
+             "use sf_attn_decode_refine with a caller workspace",
+             L.total, kStaticScratchBytes);
+  void* ws = nullptr;
+  const sf_status st = static_scratch_address(&ws);
+  if (st != SF_OK) return st;
+  cudaStream_t s = sf::as_cuda(stream);
+  char* w = static_cast<char*>(ws);
+  switch (Hq / Hkv) {
+    case 1: return run<1>(q, Hq, Hkv, T, kv, k_tokens, sel_out, sel_n, out, w, L, s);
+    case 2: return run<2>(q, Hq, Hkv, T, kv, k_tokens, sel_out, sel_n, out, w, L, s);
+    case 4: return run<4>(q, Hq, Hkv, T, kv, k_tokens, sel_out, sel_n, out, w, L, s);
+    case 8: return run<8>(q, Hq, Hkv, T, kv, k_tokens, sel_out, sel_n, out, w, L, s);
+    default: return sf::fail(SF_ENOTIMPL, "sf_attn_decode_refine_noalloc: Hq/Hkv must be 1, 2, 4 or 8");
   }
 }
