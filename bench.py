@@ -45,6 +45,9 @@ HQ, HKV, D = 32, 8, 128
 TOPK_PCT, CACHE_PCT, OUTLIER_PCT, OUTLIER_SCALE = 3, 10, "1/2", 30.0
 TOK_PCT = 1
 WORKLOAD = "llama31_8b_decode_hotpath_32k"
+# matrices that read the same activation row share one batch-1 GEMV launch
+GEMV_LAUNCHES = (("attn_in", ("q", "k", "v")), ("attn_out", ("o",)), ("mlp_in", ("gate", "up")),
+                 ("mlp_mid", ("down",)))
 
 
 def parse():
@@ -137,6 +140,9 @@ class Model:
         self.k_tok = count_fraction(TOK_PCT, T)
         self.mats = []
         self.groups = []
+        self.jobs = []
+        self.jobs0 = []
+        self.selects = []
         self.kv = []
         self.ksel = {s: count_fraction(TOPK_PCT, K) for s, K in SLOTS}
         ycount = sum(N for _, N, _, _ in MATS)
@@ -149,6 +155,10 @@ class Model:
         self.qin = torch.empty((layers, HQ, D), dtype=torch.bfloat16, device=device)
         self.idx = {s: torch.zeros((layers, self.ksel[s]), dtype=torch.int32, device=device) for s, _ in SLOTS}
         self.nsel = {s: torch.zeros((layers, 1), dtype=torch.int32, device=device) for s, _ in SLOTS}
+        # prepared activations: with the selection (refined step) and without (resident-only step)
+        self.act = {s: torch.zeros((layers, sf.act_bytes(K) // 4), dtype=torch.int32, device=device) for s, K in SLOTS}
+        self.act0 = {s: torch.zeros((layers, sf.act_bytes(K) // 4), dtype=torch.int32, device=device)
+                     for s, K in SLOTS}
         self.ws = torch.empty(sf.attn_workspace_size(HQ, HKV, D, T, self.k_tok), dtype=torch.uint8, device=device)
         self.xoff = {}
         off = 0
@@ -170,12 +180,19 @@ class Model:
             self.mats.append(row)
             self.groups.append(sf.RefineGroup([(cache, self.idx[slot][l], self.nsel[slot][l])
                                                for qw, cache, y, slot in row.values()]))
+            self.jobs.append({slot: sf.Batch1Jobs([(row[n][0], row[n][1], False, row[n][2].view(-1)) for n in names])
+                              for slot, names in GEMV_LAUNCHES})
+            self.jobs0.append({slot: sf.Batch1Jobs([(row[n][0], None, False, row[n][2].view(-1)) for n in names])
+                               for slot, names in GEMV_LAUNCHES})
+            self.selects.append(sf.SelectJobs([(self.x(l, s), self.ksel[s], self.idx[s][l], self.nsel[s][l],
+                                                self.act[s][l]) for s, _ in SLOTS]))
             Kf, Vf = ds.kv(3000 + l, HKV, T, D, device=device)
             self.kv.append(sf.QKV(sf.quantize_nested(Kf, D, B_R, B_F, "by_row"),
                                   sf.quantize_nested(Vf, D, B_R, B_F, "by_row")))
             del Kf, Vf
         torch.cuda.synchronize()
         self.side = torch.cuda.Stream(device=device)
+        self.sel_stream = torch.cuda.Stream(device=device)
 
     def x(self, l, slot):
         o, K = self.xoff[slot]
@@ -208,34 +225,40 @@ class Model:
         main = torch.cuda.current_stream()
 
         def select_and_prefetch(l):
-            for s, _ in SLOTS:
-                sf.select_topk(self.x(l, s), self.ksel[s], self.idx[s][l], self.nsel[s][l])
-            self.groups[l].prefetch(main, self.side)
+            # Fetch lead: layer l's selection is computed from inputs available
+            # when layer l-1 starts, on its own stream, and its misses are
+            # gathered on the side stream; main waits only where the GEMV needs
+            # the refinement rows.
+            ev = torch.cuda.Event()
+            ev.record(main)
+            self.sel_stream.wait_event(ev)
+            with torch.cuda.stream(self.sel_stream):
+                self.selects[l].run()
+            self.groups[l].prefetch(self.sel_stream, self.side)
 
-        def gemv(l, name):
-            qw, cache, y, slot = self.mats[l][name]
+        def gemv(l, slot):
             if refine:
-                sf.gemv_refine(qw, self.x(l, slot), self.idx[slot][l], self.nsel[slot][l], cache=cache, y=y)
+                self.jobs[l][slot].run(self.x(l, slot), self.act[slot][l])
             else:
-                sf.gemv_refine(qw, self.x(l, slot), y=y)
+                sf.act_prepare(self.x(l, slot), self.act0[slot][l])
+                self.jobs0[l][slot].run(self.x(l, slot), self.act0[slot][l])
 
         if refine:
             select_and_prefetch(0)
         for l in range(self.L):
             if refine and l + 1 < self.L:
                 select_and_prefetch(l + 1)
-            for name in ("q", "k", "v"):
-                gemv(l, name)
+            gemv(l, "attn_in")
             sf.attn_decode_refine(self.qin[l], self.kv[l], HKV, self.T, self.k_tok if refine else 0,
                                   workspace=self.ws, out=self.attn_out[l], sel_out=self.sel_out[l],
                                   sel_n=self.sel_n[l])
-            for name in ("o", "gate", "up", "down"):
-                gemv(l, name)
+            for slot in ("attn_out", "mlp_in", "mlp_mid"):
+                gemv(l, slot)
 
     def gemvs_only(self):
         for l in range(self.L):
-            for name, (qw, cache, y, slot) in self.mats[l].items():
-                self.sf.gemv_refine(qw, self.x(l, slot), self.idx[slot][l], self.nsel[slot][l], cache=cache, y=y)
+            for slot, _ in GEMV_LAUNCHES:
+                self.jobs[l][slot].run(self.x(l, slot), self.act[slot][l])
 
     def sync_caches(self):
         for row in self.mats:
@@ -252,11 +275,11 @@ class Model:
         return tot
 
     def launches_per_step(self, refine=True):
-        n_mat = len(MATS) * self.L
-        attn = 4 * self.L if (refine and 0 < self.k_tok < self.T) else 2 * self.L
+        gemv = len(GEMV_LAUNCHES) * self.L
+        attn = 5 * self.L if (refine and 0 < self.k_tok < self.T) else 2 * self.L
         if not refine:
-            return n_mat + 3 * self.L
-        return len(SLOTS) * self.L + 2 * self.L + n_mat + attn
+            return 2 * gemv + attn
+        return self.L + 2 * self.L + gemv + attn
 
     def close(self):
         for grp in self.groups:
@@ -463,10 +486,10 @@ def run_sf(args, rank, world, local_rank, dist):
             with torch.cuda.stream(cap_stream):
                 g2.replay()
         ms_g = timed(torch, dist, lambda i: g2.replay(), reps, cap_stream)
-        n_launch = len(MATS) * args.layers
+        n_launch = len(GEMV_LAUNCHES) * args.layers
         t_launch = ms_g / reps / n_launch * 1e-3
         achieved = gemv_step_bytes / n_launch / t_launch / 1e9
-        roofline = {"bound": "hbm", "kernel": "gemv_refine_kernel", "achieved": achieved, "peak": hbm_peak,
+        roofline = {"bound": "hbm", "kernel": "gemv_b1_act_kernel", "achieved": achieved, "peak": hbm_peak,
                     "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": None,
                     "peak_source": peak_src, "launch_us": t_launch * 1e6,
                     "bytes_per_launch": gemv_step_bytes / n_launch}

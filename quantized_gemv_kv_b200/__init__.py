@@ -55,6 +55,14 @@ class _QKV(ctypes.Structure):
                 ("b_r", _i), ("b_f", _i)]
 
 
+class _GemvJob(ctypes.Structure):
+    _fields_ = [("W", ctypes.POINTER(_QWeight)), ("cache", _p), ("use_ref_store", _i), ("y", _p)]
+
+
+class _SelectJob(ctypes.Structure):
+    _fields_ = [("x", _p), ("K", _i), ("k", _i), ("idx_out", _p), ("n_out", _p), ("act", _p)]
+
+
 class CacheStats(ctypes.Structure):
     _fields_ = [("steps", ctypes.c_int64), ("hits", ctypes.c_int64), ("misses", ctypes.c_int64),
                 ("bypass", ctypes.c_int64), ("h2d_bytes", ctypes.c_int64)]
@@ -79,6 +87,11 @@ _SIGS = {
     "sf_refine_group_prefetch": ([_p, _p, _p], _i),
     "sf_refine_group_destroy": ([_p], _i),
     "sf_gemv_refine": ([ctypes.POINTER(_QWeight), _p, _i, _p, _p, _p, _p, _p], _i),
+    "sf_act_bytes": ([_i], _sz),
+    "sf_select_topk_act": ([_p, _i, _i, _p, _p, _p, _p], _i),
+    "sf_act_prepare": ([_p, _i, _p, _p], _i),
+    "sf_select_topk_act_many": ([_p, _i, _p], _i),
+    "sf_gemv_refine_batch1": ([_p, _i, _p, _p, _p], _i),
     "sf_attn_workspace_size": ([_i, _i, _i, _i, _i, ctypes.POINTER(_sz)], _i),
     "sf_attn_decode_refine": ([_p, _i, _i, _i, _i, ctypes.POINTER(_QKV), _i, _p, _p, _p, _p, _sz, _p], _i),
     "sf_attn_decode_refine_noalloc": ([_p, _i, _i, _i, _i, ctypes.POINTER(_QKV), _i, _p, _p, _p, _p], _i),
@@ -356,3 +369,71 @@ def attn_decode_refine_noalloc(q: torch.Tensor, kv: QKV, Hkv: int, T: int, k_tok
     s = kv.c_struct()
     _check(_lib.sf_attn_decode_refine_noalloc(_ptr(q), Hq, Hkv, d, T, ctypes.byref(s), k_tokens, _ptr(sel_out),
                                               _ptr(sel_n), _ptr(out), _stream(stream)))
+
+
+# ---- batch-1 fast path ---------------------------------------------------------
+
+def act_bytes(K: int) -> int:
+    return _lib.sf_act_bytes(K)
+
+
+def select_topk_act(x: torch.Tensor, k: int, idx_out: torch.Tensor, n_out: torch.Tensor, act: torch.Tensor,
+                    stream: torch.cuda.Stream | None = None) -> None:
+    """Top-k selection of one activation row plus its prepared form
+    (``sf_select_topk_act``)."""
+    _dev(x, "x")
+    K = x.shape[-1]
+    _check(_lib.sf_select_topk_act(_ptr(x), K, k, _ptr(idx_out), _ptr(n_out), _ptr(act), _stream(stream)))
+
+
+def act_prepare(x: torch.Tensor, act: torch.Tensor, stream: torch.cuda.Stream | None = None) -> None:
+    """Prepared form of one activation row with nothing selected."""
+    _dev(x, "x")
+    _check(_lib.sf_act_prepare(_ptr(x), x.shape[-1], _ptr(act), _stream(stream)))
+
+
+class Batch1Jobs:
+    """A reusable list of (QWeight, cache or None, use_ref_store, y) for
+    ``sf_gemv_refine_batch1``; builds the C structs once."""
+
+    def __init__(self, jobs):
+        self._w = [W.c_struct(with_ref=bool(store)) for W, cache, store, y in jobs]
+        self._keep = jobs
+        arr = (_GemvJob * len(jobs))()
+        for i, (W, cache, store, y) in enumerate(jobs):
+            arr[i].W = ctypes.pointer(self._w[i])
+            arr[i].cache = cache.handle if cache is not None else None
+            arr[i].use_ref_store = 1 if store else 0
+            arr[i].y = _ptr(y)
+        self._arr = arr
+        self.count = len(jobs)
+
+    def run(self, x: torch.Tensor, act: torch.Tensor, stream: torch.cuda.Stream | None = None) -> None:
+        _check(_lib.sf_gemv_refine_batch1(ctypes.cast(self._arr, _p), self.count, _ptr(x), _ptr(act),
+                                          _stream(stream)))
+
+
+def gemv_refine_batch1(jobs, x: torch.Tensor, act: torch.Tensor, stream: torch.cuda.Stream | None = None) -> None:
+    """Refined GEMVs at batch 1 of up to 4 matrices that read the same x."""
+    Batch1Jobs(jobs).run(x, act, stream)
+
+
+class SelectJobs:
+    """A reusable list of single-row selections for
+    ``sf_select_topk_act_many``: entries (x, k, idx_out, n_out, act or None)."""
+
+    def __init__(self, jobs):
+        self._keep = jobs
+        arr = (_SelectJob * len(jobs))()
+        for i, (x, k, idx, n, act) in enumerate(jobs):
+            arr[i].x = _ptr(x)
+            arr[i].K = x.shape[-1]
+            arr[i].k = k
+            arr[i].idx_out = _ptr(idx)
+            arr[i].n_out = _ptr(n)
+            arr[i].act = _ptr(act) if act is not None else None
+        self._arr = arr
+        self.count = len(jobs)
+
+    def run(self, stream: torch.cuda.Stream | None = None) -> None:
+        _check(_lib.sf_select_topk_act_many(ctypes.cast(self._arr, _p), self.count, _stream(stream)))

@@ -35,10 +35,11 @@ namespace {
 constexpr int D = 128;                 // head dim
 constexpr int kWordsPerRow = D * 2 / 32;  // 2-bit codes of one token-head: 8 words
 constexpr int kMaxGrp = 8;
+constexpr int kMaxSplits = 256;
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128), rounded to fp32
 
 struct Layout {
-  size_t score, cand, kap, sel, umask, part, smax, status, count, total;
+  size_t score, cand, cand2, kap, sel, umask, part, smax, status, count, total;
   int splits, tps, words_t;
 };
 
@@ -46,7 +47,7 @@ size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 Layout make_layout(int Hq, int Hkv, int T, int k, int sms) {
   Layout L{};
-  const int want = std::max(1, (2 * sms + Hkv - 1) / Hkv);
+  const int want = std::max(1, std::min(kMaxSplits, sms / Hkv));  // one wave of pass-B CTAs
   int tps = (T + want - 1) / want;
   tps = std::max(128, (tps + 127) / 128 * 128);
   L.tps = tps;
@@ -55,6 +56,7 @@ Layout make_layout(int Hq, int Hkv, int T, int k, int sms) {
   size_t off = 0;
   L.score = off; off = up256(off + sizeof(float) * Hq * static_cast<size_t>(T));
   L.cand = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(T));
+  L.cand2 = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(T));
   L.kap = off; off = up256(off + sizeof(double) * Hq * static_cast<size_t>(T));
   L.sel = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(std::max(k, 1)));
   L.umask = off; off = up256(off + sizeof(uint32_t) * Hkv * static_cast<size_t>(L.words_t));
@@ -89,6 +91,19 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+
+__device__ __forceinline__ void cp_async16_attn(void* smem, const void* gmem) {
+  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async4_attn(void* smem, const void* gmem) {
+  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(sa), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit_attn() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_attn() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
 // Loads the group's query heads as fp32 into qs[GRP][D] and their sums
 // (sequential fp32 order, d ascending) into qsum[GRP].
 template <int GRP>
@@ -104,50 +119,148 @@ __device__ void load_q(const uint16_t* __restrict__ q, int g, float (*qs)[D], fl
   __syncthreads();
 }
 
-// ---- pass A: resident scores --------------------------------------------
-template <int GRP>
-__global__ void __launch_bounds__(128)
-attn_score_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
-                  const uint16_t* __restrict__ k_scale, const uint16_t* __restrict__ k_zero, int T,
-                  float* __restrict__ score, float* __restrict__ smax) {
-  __shared__ float qs[GRP][D];
-  __shared__ float qsum[GRP];
-  const int g = blockIdx.y;
-  load_q<GRP>(q, g, qs, qsum);
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  float s = 0.0f;
-  if (t < T) {
-    const size_t row = static_cast<size_t>(g) * T + t;
-    const uint4* kp = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
-    const uint4 a = kp[0], b = kp[1];
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    s = sfd::half_bits_to_float(k_scale[row]);
-    const float z = sfd::half_bits_to_float(k_zero[row]);
-    float P[GRP];
-#pragma unroll
-    for (int h = 0; h < GRP; ++h) P[h] = 0.0f;
-#pragma unroll
-    for (int d = 0; d < D; ++d) {
-      const float c = static_cast<float>((w[d >> 4] >> ((d & 15) * 2)) & 3u);
-#pragma unroll
-      for (int h = 0; h < GRP; ++h) P[h] = fmaf(qs[h][d], c, P[h]);
-    }
-#pragma unroll
-    for (int h = 0; h < GRP; ++h) {
-      const float E = fmaf(4.0f, P[h], (1.5f - z) * qsum[h]);
-      score[(static_cast<size_t>(g) * GRP + h) * T + t] = (s * E) * kInvSqrtD;
-    }
-  }
-  const float m = warp_max(s);
-  if ((threadIdx.x & 31) == 0) atomicMax(reinterpret_cast<unsigned int*>(smax + g), __float_as_uint(m));
+// ---- pass A on the tensor cores: integer MMA over code bytes ----------------
+//
+// Per KV group, the query heads become exact-as-possible fixed point: per
+// head X_d = rint(q_d 2^(23 - e)), e the binary exponent of max |q| (every
+// bf16 within 15 binades of the maximum is exact), split into three byte
+// planes.  mma.m16n8k32 (u8 codes x u8/s8 planes, s32 accumulate) gives
+// sum_d c_d X_d per plane exactly; the reduction order inside an MMA does not
+// matter, so a code word becomes a fragment register with one shift and one
+// mask ((w >> 2 tig) & 0x03030303 holds dims tig, tig+4, tig+8, tig+12), and
+// the q planes are laid out in the same permuted order.  A warp scores 16
+// tokens per MMA row tile for all heads of the group at once (n = heads).
+__device__ __forceinline__ void mma_u8u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Histogram increment with same-bin lanes of a warp merged into one atomic;
-// bin < 0 means no increment.  Call with the whole warp.
-__device__ __forceinline__ void warp_hist_add(int* hist, int bin) {
-  const unsigned peers = __match_any_sync(0xffffffffu, bin);
-  const int leader = __ffs(peers) - 1;
-  if (bin >= 0 && (threadIdx.x & 31) == leader) atomicAdd(&hist[bin], __popc(peers));
+template <int GRP>
+__global__ void __launch_bounds__(128)
+attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
+                      const uint16_t* __restrict__ k_scale, const uint16_t* __restrict__ k_zero, int T,
+                      float* __restrict__ score, float* __restrict__ smax) {
+  __shared__ int qx[GRP][D];
+  __shared__ float qsc[GRP], qsm[GRP];
+  const int g = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // fixed-point query heads (warp h builds head h, 4 dims per lane)
+  for (int h = warp; h < GRP; h += 4) {
+    float v[4];
+    float am = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[i] = sfd::bf16_bits_to_float(q[(static_cast<size_t>(g) * GRP + h) * D + 4 * lane + i]);
+      am = fmaxf(am, fabsf(v[i]));
+    }
+    am = warp_max(am);
+    int e = 0;
+    if (am > 0.0f) frexpf(am, &e);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) qx[h][4 * lane + i] = __float2int_rn(ldexpf(v[i], 23 - e));
+    if (lane == 0) qsc[h] = ldexpf(1.0f, e - 23);
+  }
+  if (tid < GRP) {
+    float sum = 0.0f;
+    for (int d = 0; d < D; ++d) sum += sfd::bf16_bits_to_float(q[(static_cast<size_t>(g) * GRP + tid) * D + d]);
+    qsm[tid] = sum;
+  }
+  __syncthreads();
+  const int g8 = lane >> 2, tig = lane & 3;
+  // B fragments: column n = g8 is query head g8 (zero beyond the group)
+  uint32_t bq[4][3][2];
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+    for (int half = 0; half < 2; ++half)
+#pragma unroll
+      for (int p = 0; p < 3; ++p) {
+        uint32_t v = 0;
+        if (g8 < GRP) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            v |= ((static_cast<uint32_t>(qx[g8][16 * (2 * ks + half) + tig + 4 * i]) >> (8 * p)) & 0xFFu) << (8 * i);
+        }
+        bq[ks][p][half] = v;
+      }
+  const int ntiles = (T + 15) / 16;
+  float smx = 0.0f;
+  // one tile = rows ta, tb of this thread: 2 x 32 bytes of codes plus the
+  // rows' scale and zero; the next tile is fetched while this one is scored
+  struct TileRegs {
+    uint32_t wa[8], wb[8];
+    uint16_t sa, za, sb, zb;
+  };
+  auto load_tile = [&](int tile, TileRegs& r) {
+    const int ta = tile * 16 + g8, tb = ta + 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { r.wa[i] = 0u; r.wb[i] = 0u; }
+    r.sa = r.za = r.sb = r.zb = 0;
+    if (ta < T) {
+      const size_t row = static_cast<size_t>(g) * T + ta;
+      const uint4* p4 = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
+      const uint4 x0 = p4[0], x1 = p4[1];
+      r.wa[0] = x0.x; r.wa[1] = x0.y; r.wa[2] = x0.z; r.wa[3] = x0.w;
+      r.wa[4] = x1.x; r.wa[5] = x1.y; r.wa[6] = x1.z; r.wa[7] = x1.w;
+      r.sa = k_scale[row];
+      r.za = k_zero[row];
+    }
+    if (tb < T) {
+      const size_t row = static_cast<size_t>(g) * T + tb;
+      const uint4* p4 = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
+      const uint4 x0 = p4[0], x1 = p4[1];
+      r.wb[0] = x0.x; r.wb[1] = x0.y; r.wb[2] = x0.z; r.wb[3] = x0.w;
+      r.wb[4] = x1.x; r.wb[5] = x1.y; r.wb[6] = x1.z; r.wb[7] = x1.w;
+      r.sb = k_scale[row];
+      r.zb = k_zero[row];
+    }
+  };
+  const int tstride = gridDim.x * 4;
+  int tile = blockIdx.x * 4 + warp;
+  TileRegs cur;
+  if (tile < ntiles) load_tile(tile, cur);
+  for (; tile < ntiles; tile += tstride) {
+    TileRegs nxt;
+    if (tile + tstride < ntiles) load_tile(tile + tstride, nxt);
+    const int ta = tile * 16 + g8, tb = ta + 8;
+    int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0}, d2[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      const uint32_t a0 = (cur.wa[2 * ks] >> (2 * tig)) & 0x03030303u;
+      const uint32_t a1 = (cur.wb[2 * ks] >> (2 * tig)) & 0x03030303u;
+      const uint32_t a2 = (cur.wa[2 * ks + 1] >> (2 * tig)) & 0x03030303u;
+      const uint32_t a3 = (cur.wb[2 * ks + 1] >> (2 * tig)) & 0x03030303u;
+      mma_u8u8(d0, a0, a1, a2, a3, bq[ks][0][0], bq[ks][0][1]);
+      mma_u8u8(d1, a0, a1, a2, a3, bq[ks][1][0], bq[ks][1][1]);
+      mma_u8s8(d2, a0, a1, a2, a3, bq[ks][2][0], bq[ks][2][1]);
+    }
+    // d[i]: i = 0,1 -> token ta, heads 2 tig, 2 tig + 1; i = 2,3 -> token tb
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int h = 2 * tig + (i & 1);
+      const int t = (i < 2) ? ta : tb;
+      if (h < GRP && t < T) {
+        const float sv = sfd::half_bits_to_float(i < 2 ? cur.sa : cur.sb);
+        const float zv = sfd::half_bits_to_float(i < 2 ? cur.za : cur.zb);
+        smx = fmaxf(smx, sv);
+        const float P = (static_cast<float>(d2[i]) * 65536.0f + static_cast<float>(d1[i]) * 256.0f +
+                         static_cast<float>(d0[i])) * qsc[h];
+        const float E = fmaf(4.0f, P, (1.5f - zv) * qsm[h]);
+        score[(static_cast<size_t>(g) * GRP + h) * T + t] = (sv * E) * kInvSqrtD;
+      }
+    }
+    cur = nxt;
+  }
+  smx = warp_max(smx);
+  if (lane == 0) atomicMax(reinterpret_cast<unsigned int*>(smax + g), __float_as_uint(smx));
 }
 
 // ---- pass S: exact per-head top-k ------------------------------------------
@@ -182,27 +295,107 @@ __device__ void find_bin_from_top(const int* hist, int nb, int kk, int* out) {
   if (lane == 0) { out[0] = 0; out[1] = kk; }
 }
 
+// Block-wide sum of two ints (all threads call; result in every thread).
+__device__ __forceinline__ void block_sum2(int& a, int& b, int* scratch /* 64 ints */) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  __syncthreads();
+  if (lane == 0) { scratch[warp] = a; scratch[32 + warp] = b; }
+  __syncthreads();
+  a = 0;
+  b = 0;
+  for (int w = 0; w < nw; ++w) { a += scratch[w]; b += scratch[32 + w]; }
+  __syncthreads();
+}
+
+// Exact per-head top-k (see the pass structure at the top of this file).
+//  1. amax over the fast scores and a strided sample of them;
+//  2. a threshold theta from the sample such that at least k scores are
+//     >= theta + 2 eps (checked by counting; lowered until true, at worst to
+//     -inf), so every token whose exact key can reach the top k has a fast
+//     score >= theta;
+//  3. G = {t : score_t >= theta} in token order, tau = k-th largest score over
+//     G by radix select (equal to the k-th largest overall);
+//  4. candidates F = {t in G : score_t >= tau - 2 eps}, re-keyed exactly in
+//     fp64, ranked by (key desc, token asc).
+// Ordered (stable) compaction of the indices i in [0, n) with pred(i), by a
+// whole block: warp w owns the contiguous segment [w seg, (w+1) seg) and walks
+// it 32 indices at a time (coalesced), with ballots giving positions inside
+// the warp; a prefix over the warps' counts gives each warp's offset.
+// Writes emit(pos, i) for the kept indices and returns their count.  Every
+// thread of the block must call it.
+template <class Pred, class Emit>
+__device__ int block_ordered_compact(int n, Pred pred, Emit emit, int* wsum /* 33 ints */) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int seg = (((n + nw - 1) / nw) + 31) & ~31;
+  const int b0 = min(n, warp * seg), b1 = min(n, b0 + seg);
+  int cnt = 0;
+  for (int base = b0; base < b1; base += 32) {
+    const int i = base + lane;
+    cnt += __popc(__ballot_sync(0xffffffffu, i < b1 && pred(i)));
+  }
+  __syncthreads();
+  if (lane == 0) wsum[warp] = cnt;
+  __syncthreads();
+  if (warp == 0) {
+    const int v = lane < nw ? wsum[lane] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane < nw) wsum[lane] = incl - v;
+    if (lane == 31) wsum[32] = incl;
+  }
+  __syncthreads();
+  int off = wsum[warp];
+  const int total = wsum[32];
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = b0; base < b1; base += 32) {
+    const int i = base + lane;
+    const bool p = i < b1 && pred(i);
+    const unsigned bal = __ballot_sync(0xffffffffu, p);
+    if (p) emit(off + __popc(bal & lt), i);
+    off += __popc(bal);
+  }
+  __syncthreads();
+  return total;
+}
+
+constexpr int kDirectRank = 1024;  // candidates ranked pairwise (one per thread)
+
 template <int GRP>
 __global__ void __launch_bounds__(kSelThreads)
 attn_select_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
                    const uint16_t* __restrict__ k_scale, const uint16_t* __restrict__ k_zero, int T, int k,
                    const float* __restrict__ score, const float* __restrict__ smax, int32_t* __restrict__ cand,
-                   double* __restrict__ kap, int32_t* __restrict__ sel_head, int32_t* __restrict__ status) {
-  __shared__ int hist[2048];
+                   int32_t* __restrict__ cand2, double* __restrict__ kap, int32_t* __restrict__ sel_head,
+                   int32_t* __restrict__ status) {
+  constexpr int kSamples = 512;
+  __shared__ __align__(16) int hist[2048];
   __shared__ double qd[D];
-  __shared__ int scan_scratch[33];
+  __shared__ float samp[kSamples];
+  __shared__ int scan_scratch[64];
   __shared__ int binfo[2];
   __shared__ float red[32];
   __shared__ double l1_sh;
+  __shared__ int qe_sh;
+  __shared__ float theta_sh;
   const int h = blockIdx.x, g = h / GRP, tid = threadIdx.x;
   const float* sc = score + static_cast<size_t>(h) * T;
-  int32_t* cd = cand + static_cast<size_t>(h) * T;
+  int32_t* G = cand + static_cast<size_t>(h) * T;
+  int32_t* F = cand2 + static_cast<size_t>(h) * T;
   double* kp = kap + static_cast<size_t>(h) * T;
 
-  for (int d = tid; d < D; d += kSelThreads) qd[d] = static_cast<double>(sfd::bf16_bits_to_float(q[static_cast<size_t>(h) * D + d]));
+  for (int d = tid; d < D; d += kSelThreads)
+    qd[d] = static_cast<double>(sfd::bf16_bits_to_float(q[static_cast<size_t>(h) * D + d]));
   __syncthreads();
   if (tid < 32) {
-    // L1 norm (exact in fp64 for 128 bf16 values) and the exponent span check
     double l1 = 0.0;
     int emin = 100000, emax = -100000;
     for (int d = tid; d < D; d += 32) {
@@ -223,40 +416,18 @@ attn_select_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ 
     }
     if (tid == 0) {
       l1_sh = l1;
+      qe_sh = emax >= emin ? emax : 0;  // binary exponent of max |q| (frexp convention)
       // 53 - 9 - b - log2(d) with b = 4, d = 128
       if (emax >= emin && emax - emin > 53 - 9 - 4 - 7) atomicOr(status + g, 1);
     }
   }
 
-  // 1. radix select of the k-th largest fast score (11 + 11 + 10 bits)
-  uint32_t prefix = 0, pmask = 0;
-  int kk = k;
+  // 1. amax and a strided sample
+  const int ns = T < kSamples ? T : kSamples;
+  const int stride = T / ns;
   float amax = 0.0f;
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
-  for (int pass = 0; pass < 3; ++pass) {
-    const int nb = 1 << widths[pass];
-    for (int i = tid; i < nb; i += kSelThreads) hist[i] = 0;
-    __syncthreads();
-    for (int t0 = tid - (tid & 31); t0 < T; t0 += kSelThreads) {
-      const int t = t0 + (tid & 31);
-      int bin = -1;
-      if (t < T) {
-        const float v = sc[t];
-        if (pass == 0) amax = fmaxf(amax, fabsf(v));
-        const uint32_t key = okey32(v);
-        if ((key & pmask) == prefix) bin = static_cast<int>((key >> shifts[pass]) & (nb - 1));
-      }
-      warp_hist_add(hist, bin);
-    }
-    __syncthreads();
-    find_bin_from_top(hist, nb, kk, binfo);
-    __syncthreads();
-    prefix |= static_cast<uint32_t>(binfo[0]) << shifts[pass];
-    pmask |= static_cast<uint32_t>(nb - 1) << shifts[pass];
-    kk = binfo[1];
-    __syncthreads();
-  }
+  for (int t = tid; t < T; t += kSelThreads) amax = fmaxf(amax, fabsf(sc[t]));
+  for (int i = tid; i < ns; i += kSelThreads) samp[i] = sc[i * stride];
   {
     const float m = warp_max(amax);
     if ((tid & 31) == 0) red[tid >> 5] = m;
@@ -268,46 +439,119 @@ attn_select_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ 
     __syncthreads();
     amax = red[0];
   }
-  const double tau = static_cast<double>(from_okey32(prefix));
 
-  // 2. error bound of the fast scores (see the pass-A arithmetic): a sum of
-  // 128 fp32 FMAs has |error| <= gamma_128 * sum |terms|.
+  // error bound of the fast scores (pass A): q rounded to 24-bit fixed point
+  // (|dq| <= 2^(e-24) per entry), exact integer products and sums, an fp32
+  // combine of the three plane sums, the fp32 sum of q (<= gamma_128 l1), and
+  // the roundings of the zero-point term, the fma, the scale and 1/sqrt(d).
   const double u = 5.9604644775390625e-8;  // 2^-24
   const double gam = 130.0 * u / (1.0 - 130.0 * u);
   const double s_max = static_cast<double>(smax[g]);
   const double l1 = l1_sh;
-  const double eps_k = s_max * l1 * (4.0 * 3.0 * gam + 16.0 * gam + 4.0 * 16.0 * u);
+  const double qround = ldexp(1.0, qe_sh - 24);
+  const double eps_k = s_max * (4.0 * 3.0 * D * qround + l1 * (136.0 * u + 16.0 * gam));
   const double eps_s = 2.0 * (static_cast<double>(kInvSqrtD) * eps_k + 4.0 * u * static_cast<double>(amax));
+
+  // 2. threshold from the sample: aim at ~2k + 64 tokens above it
+  double theta = -INFINITY;
+  for (int trial = 0; trial < 3; ++trial) {
+    int want = static_cast<int>((static_cast<long long>(2 * k + 64) * ns) / T) + 1;
+    want <<= (2 * trial);  // lower the threshold on a retry
+    if (trial == 2 || want >= ns) break;  // fall back to all tokens
+    // the want-th largest sample (rank counted from 1)
+    for (int i = tid; i < ns; i += kSelThreads) {
+      const float v = samp[i];
+      int gt = 0, ge = 0;
+      for (int j = 0; j < ns; ++j) {
+        const float w = samp[j];
+        gt += w > v;
+        ge += w >= v;
+      }
+      if (gt < want && want <= ge) theta_sh = v;
+    }
+    __syncthreads();
+    const double th = static_cast<double>(theta_sh) - 2.0 * eps_s;
+    int c1 = 0, dummy = 0;
+    for (int t = tid; t < T; t += kSelThreads) c1 += static_cast<double>(sc[t]) >= th + 2.0 * eps_s;
+    block_sum2(c1, dummy, scan_scratch);
+    if (c1 >= k) { theta = th; break; }
+  }
+
+  // 3. G in token order, then tau = k-th largest over G
+  const int nG = block_ordered_compact(
+      T, [&](int t) { return static_cast<double>(sc[t]) >= theta; }, [&](int pos, int t) { G[pos] = t; },
+      scan_scratch);
+  uint32_t prefix = 0, pmask = 0;
+  int kk = k;
+  const int shifts[3] = {21, 10, 0};
+  const int widths[3] = {11, 11, 10};
+  for (int pass = 0; pass < 3; ++pass) {
+    const int nb = 1 << widths[pass];
+    for (int i = tid; i < nb; i += kSelThreads) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < nG; i += kSelThreads) {
+      const uint32_t key = okey32(sc[G[i]]);
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shifts[pass]) & (nb - 1)], 1);
+    }
+    __syncthreads();
+    find_bin_from_top(hist, nb, kk, binfo);
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(binfo[0]) << shifts[pass];
+    pmask |= static_cast<uint32_t>(nb - 1) << shifts[pass];
+    kk = binfo[1];
+    __syncthreads();
+  }
+  const double tau = static_cast<double>(from_okey32(prefix));
   const double thr = tau - 2.0 * eps_s;
 
-  // 3. candidates (fast score >= thr), ascending token order
-  int ncand;
-  {
-    const int chunk = (T + kSelThreads - 1) / kSelThreads;
-    const int t0 = min(T, tid * chunk), t1 = min(T, t0 + chunk);
-    int c = 0;
-    for (int t = t0; t < t1; ++t) c += static_cast<double>(sc[t]) >= thr;
-    int pos = sfd::block_exclusive_scan(c, scan_scratch, &ncand);
-    for (int t = t0; t < t1; ++t)
-      if (static_cast<double>(sc[t]) >= thr) cd[pos++] = t;
+  // 4. candidates F (token order), exact keys
+  const int ncand = block_ordered_compact(
+      nG, [&](int i) { return static_cast<double>(sc[G[i]]) >= thr; }, [&](int pos, int i) { F[pos] = G[i]; },
+      scan_scratch);
+  for (int i = tid; i < ncand; i += kSelThreads) {
+    const int t = F[i];
+    const size_t row = static_cast<size_t>(g) * T + t;
+    const uint4* w4 = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
+    const uint4 x0 = w4[0], x1 = w4[1];
+    const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    const double sv = static_cast<double>(sfd::half_bits_to_float(k_scale[row]));
+    const double z = static_cast<double>(sfd::half_bits_to_float(k_zero[row]));
+    double E = 0.0;
+#pragma unroll
+    for (int wi = 0; wi < 8; ++wi) {
+      const uint32_t word = w[wi];
+#pragma unroll 4
+      for (int j = 0; j < 16; ++j) {
+        const double c = static_cast<double>((word >> (2 * j)) & 3u);
+        E = fma(qd[16 * wi + j], c * 4.0 + 1.5 - z, E);
+      }
+    }
+    kp[i] = sv * E;
   }
   __syncthreads();
 
-  // 4. exact keys of the candidates
-  for (int i = tid; i < ncand; i += kSelThreads) {
-    const int t = cd[i];
-    const size_t row = static_cast<size_t>(g) * T + t;
-    const uint32_t* w = k_res + row * kWordsPerRow;
-    const double s = static_cast<double>(sfd::half_bits_to_float(k_scale[row]));
-    const double z = static_cast<double>(sfd::half_bits_to_float(k_zero[row]));
-    double E = 0.0;
-    for (int d = 0; d < D; ++d) {
-      const double c = static_cast<double>((w[d >> 4] >> ((d & 15) * 2)) & 3u);
-      E = fma(qd[d], c * 4.0 + 1.5 - z, E);
+  // 5a. few candidates (the usual case): rank each one directly against all
+  // others by (key desc, token asc) -- no synchronised passes
+  if (ncand <= kDirectRank) {
+    double* kd = reinterpret_cast<double*>(hist);  // 2048 ints = 1024 doubles of scratch
+    for (int i = tid; i < ncand; i += kSelThreads) kd[i] = kp[i];
+    __syncthreads();
+    int take = 0;
+    const int i = tid;
+    if (i < ncand) {
+      const double ki = kd[i];
+      int rank = 0;
+      for (int j = 0; j < ncand; ++j) {
+        const double kj = kd[j];
+        rank += (kj > ki) || (kj == ki && j < i);  // F is in token order
+      }
+      take = rank < k;
     }
-    kp[i] = s * E;
+    int tot;
+    const int pos = sfd::block_exclusive_scan(take, scan_scratch, &tot);
+    if (take) sel_head[static_cast<size_t>(h) * k + pos] = F[i];
+    return;
   }
-  __syncthreads();
 
   // 5. exact top-k among the candidates by (key desc, token asc)
   unsigned long long pre64 = 0, pm64 = 0;
@@ -316,14 +560,9 @@ attn_select_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ 
     const int shift = 56 - 8 * pass;
     for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
     __syncthreads();
-    for (int i0 = tid - (tid & 31); i0 < ncand; i0 += kSelThreads) {
-      const int i = i0 + (tid & 31);
-      int bin = -1;
-      if (i < ncand) {
-        const unsigned long long key = okey64(kp[i]);
-        if ((key & pm64) == pre64) bin = static_cast<int>((key >> shift) & 255);
-      }
-      warp_hist_add(hist, bin);
+    for (int i = tid; i < ncand; i += kSelThreads) {
+      const unsigned long long key = okey64(kp[i]);
+      if ((key & pm64) == pre64) atomicAdd(&hist[(key >> shift) & 255], 1);
     }
     __syncthreads();
     find_bin_from_top(hist, 256, kr, binfo);
@@ -334,7 +573,6 @@ attn_select_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ 
     __syncthreads();
   }
   {
-    // keys above the k-th key, plus the first kr equal to it in token order
     const int chunk = (ncand + kSelThreads - 1) / kSelThreads;
     const int i0 = min(ncand, tid * chunk), i1 = min(ncand, i0 + chunk);
     int eq = 0;
@@ -356,7 +594,7 @@ attn_select_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ 
       bool ok = false;
       if (key > pre64) ok = true;
       else if (key == pre64) { ok = rank < kr; ++rank; }
-      if (ok) sel_head[static_cast<size_t>(h) * k + pos++] = cd[i];
+      if (ok) sel_head[static_cast<size_t>(h) * k + pos++] = F[i];
     }
   }
 }
@@ -398,150 +636,274 @@ attn_union_kernel(const int32_t* __restrict__ sel_head, int grp, int T, int k, i
   if (tid == 0) sel_n[g] = status[g] ? -1 - total : total;
 }
 
-// ---- pass B: softmax-weighted values over all tokens, refined where selected
+// ---- refined scores of the refined tokens ------------------------------------
+// For every token in a KV group's union, the scores of the group's query heads
+// with the full-code key k' = s (4 c_r + c_f - z) replace the resident scores
+// in the score buffer (after the selection has used them).  One warp per token,
+// lanes over 4 dims each.
 template <int GRP>
-__global__ void __launch_bounds__(128)
-attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
-                const uint32_t* __restrict__ k_ref, const uint16_t* __restrict__ k_scale,
-                const uint16_t* __restrict__ k_zero, const uint32_t* __restrict__ v_res,
-                const uint32_t* __restrict__ v_ref, const uint16_t* __restrict__ v_scale,
-                const uint16_t* __restrict__ v_zero, int T, int tps, int words_t, int splits,
-                const float* __restrict__ score, const uint32_t* __restrict__ umask, float* __restrict__ part,
-                int32_t* __restrict__ done, float* __restrict__ out) {
+__global__ void __launch_bounds__(256)
+attn_refine_scores_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
+                          const uint32_t* __restrict__ k_ref, const uint16_t* __restrict__ k_scale,
+                          const uint16_t* __restrict__ k_zero, int T, int cap, const int32_t* __restrict__ sel_out,
+                          const int32_t* __restrict__ sel_n, float* __restrict__ score) {
   __shared__ float qs[GRP][D];
   __shared__ float qsum[GRP];
-  __shared__ uint32_t vr[4][32][kWordsPerRow];
-  __shared__ uint32_t vf[4][32][kWordsPerRow];
-  __shared__ float alpha[4][32][GRP];
-  __shared__ float wm[4][GRP];
-  __shared__ float wl[4][GRP];
-  __shared__ float wo[4][GRP][D];
+  const int g = blockIdx.y;
+  load_q<GRP>(q, g, qs, qsum);
+  int n = sel_n[g];
+  n = n >= 0 ? n : -1 - n;
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int nwarps = gridDim.x * (blockDim.x >> 5);
+  for (int i = gw; i < n; i += nwarps) {
+    const int t = sel_out[static_cast<size_t>(g) * cap + i];
+    const size_t row = static_cast<size_t>(g) * T + t;
+    const uint32_t wr = k_res[row * kWordsPerRow + (lane >> 2)] >> ((lane & 3) * 8);
+    const uint32_t wf = k_ref[row * kWordsPerRow + (lane >> 2)] >> ((lane & 3) * 8);
+    float P[GRP];
+#pragma unroll
+    for (int h = 0; h < GRP; ++h) P[h] = 0.0f;
+#pragma unroll
+    for (int dd = 0; dd < 4; ++dd) {
+      const float c = static_cast<float>(((wr >> (2 * dd)) & 3u) * 4u + ((wf >> (2 * dd)) & 3u));
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) P[h] = fmaf(qs[h][4 * lane + dd], c, P[h]);
+    }
+    const float sv = sfd::half_bits_to_float(k_scale[row]);
+    const float z = sfd::half_bits_to_float(k_zero[row]);
+#pragma unroll
+    for (int h = 0; h < GRP; ++h) {
+      const float Ph = warp_sum(P[h]);
+      if (lane == 0) score[(static_cast<size_t>(g) * GRP + h) * T + t] = (sv * fmaf(-z, qsum[h], Ph)) * kInvSqrtD;
+    }
+  }
+}
+
+// ---- pass B on the tensor cores ------------------------------------------------
+//
+// o_h = sum_t p_{h,t} v_t / sum_t p_{h,t} with v_t = s_t (4 c_t + 1.5 - z_t):
+// the code part 4 sum_t alpha_{h,t} c_t is a product of the weights
+// alpha_{h,t} = p_{h,t} s_t (rows = heads) with the code matrix (tokens x dims)
+// on mma.m16n8k16 (f16 in, f32 accumulate).  alpha is split into an f16 high part and an f16 remainder
+// (rows h and GRP + h), so the products keep ~22 bits.  Codes enter as the
+// f16 values 1024 + c, exact, built for a pair of tokens and one dim with
+// one shift, one byte permute and one mask; the 1024 * sum(alpha) they add is
+// removed at the end.  The offset part sum_t alpha_{h,t} (1.5 - z_t) is a
+// scalar per head.  Refined tokens (in the union) add alpha (c_f - 1.5) s-scaled
+// codes of their refinement bits on the CUDA cores; their scores were already
+// refined in the score buffer.  Online softmax runs per 16-token tile.
+__device__ __forceinline__ void mma_f16f32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+constexpr int kOutStages = 4;
+template <int GRP>
+__host__ __device__ constexpr int out_warps() { return GRP <= 4 ? 8 : 4; }
+
+template <int GRP>
+__global__ void __launch_bounds__(256)
+attn_out_mma_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__ v_ref,
+                    const uint16_t* __restrict__ v_scale, const uint16_t* __restrict__ v_zero, int T, int tps,
+                    int words_t, int splits, const float* __restrict__ score, const uint32_t* __restrict__ umask,
+                    float* __restrict__ part, int32_t* __restrict__ done, float* __restrict__ out) {
+  constexpr int kOutWarps = out_warps<GRP>();
+  __shared__ __align__(16) uint32_t vrow[kOutWarps][kOutStages][16][kWordsPerRow];
+  __shared__ float ssc[kOutWarps][kOutStages][GRP][16];
+  __shared__ __align__(16) __half a16[kOutWarps][16][16];
+  __shared__ float wm[kOutWarps][GRP], wl[kOutWarps][GRP];
+  __shared__ float wo[kOutWarps][GRP][D];
   const int g = blockIdx.y, split = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  load_q<GRP>(q, g, qs, qsum);
-  const int t0 = split * tps, t1 = min(T, t0 + tps);
+  const int g8 = lane >> 2, tig = lane & 3;
+  const int t0s = split * tps, t1s = min(T, t0s + tps);
+  // this warp's contiguous share of the split, in 16-token tiles
+  const int ntile = (t1s - t0s + 15) / 16;
+  const int tpw = (ntile + kOutWarps - 1) / kOutWarps;
+  const int tile0 = warp * tpw, tile1 = min(ntile, tile0 + tpw);
 
-  float m[GRP], l[GRP], bs[GRP], o[GRP][4];
+  for (int e = lane; e < GRP * D; e += 32) wo[warp][e / D][e % D] = 0.0f;
+  for (int e = lane; e < 16 * 16; e += 32) a16[warp][e / 16][e % 16] = __float2half_rn(0.0f);
+
+  float m[GRP], lsum[GRP], csum[GRP], asum[GRP], uo[GRP][4];
+  float acc[16][4];
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
     m[h] = -INFINITY;
-    l[h] = 0.0f;
-    bs[h] = 0.0f;
+    lsum[h] = csum[h] = asum[h] = 0.0f;
 #pragma unroll
-    for (int dd = 0; dd < 4; ++dd) o[h][dd] = 0.0f;
+    for (int dd = 0; dd < 4; ++dd) uo[h][dd] = 0.0f;
   }
+#pragma unroll
+  for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[nt][c] = 0.0f;
 
-  for (int base = t0 + warp * 32; base < t1; base += 4 * 32) {
-    const int t = base + lane;
-    const bool valid = t < t1;
-    const size_t row = static_cast<size_t>(g) * T + (valid ? t : t0);
+  auto issue = [&](int ti) {
+    const int st = (ti - tile0) % kOutStages;
+    const int tb = t0s + ti * 16;
+    if (lane < 16) {
+      const int t = tb + lane;
+      if (t < t1s) {
+        const size_t row = static_cast<size_t>(g) * T + t;
+        const uint32_t* src = v_res + row * kWordsPerRow;
+        cp_async16_attn(&vrow[warp][st][lane][0], src);
+        cp_async16_attn(&vrow[warp][st][lane][4], src + 4);
+#pragma unroll
+        for (int h = 0; h < GRP; ++h) cp_async4_attn(&ssc[warp][st][h][lane], score + (static_cast<size_t>(g) * GRP + h) * T + t);
+      }
+    }
+  };
+  for (int i = 0; i < kOutStages - 1; ++i) {
+    if (tile0 + i < tile1) issue(tile0 + i);
+    cp_async_commit_attn();
+  }
+  for (int ti = tile0; ti < tile1; ++ti) {
+    if (ti + kOutStages - 1 < tile1) issue(ti + kOutStages - 1);
+    cp_async_commit_attn();
+    // this tile's per-token scalars (plain loads; the ring carries the bulk)
+    const int tb = t0s + ti * 16;
+    const int t = tb + (lane & 15);
+    const bool valid = lane < 16 && t < t1s;
+    float sv = 0.0f, zv = 0.0f;
     bool inU = false;
-    float sc[GRP];
     if (valid) {
+      const size_t row = static_cast<size_t>(g) * T + t;
+      sv = sfd::half_bits_to_float(v_scale[row]);
+      zv = sfd::half_bits_to_float(v_zero[row]);
       inU = (umask[static_cast<size_t>(g) * words_t + (t >> 5)] >> (t & 31)) & 1u;
-#pragma unroll
-      for (int h = 0; h < GRP; ++h) sc[h] = score[(static_cast<size_t>(g) * GRP + h) * T + t];
-      if (inU) {
-        // refined key: k' = s (4 c_r + c_f - z)
-        const uint32_t* wr = k_res + row * kWordsPerRow;
-        const uint32_t* wf = k_ref + row * kWordsPerRow;
-        const float s = sfd::half_bits_to_float(k_scale[row]);
-        const float z = sfd::half_bits_to_float(k_zero[row]);
-        float P[GRP];
-#pragma unroll
-        for (int h = 0; h < GRP; ++h) P[h] = 0.0f;
-        for (int d = 0; d < D; ++d) {
-          const uint32_t cr = (wr[d >> 4] >> ((d & 15) * 2)) & 3u;
-          const uint32_t cf = (wf[d >> 4] >> ((d & 15) * 2)) & 3u;
-          const float c = static_cast<float>(cr * 4u + cf);
-#pragma unroll
-          for (int h = 0; h < GRP; ++h) P[h] = fmaf(qs[h][d], c, P[h]);
-        }
-#pragma unroll
-        for (int h = 0; h < GRP; ++h) sc[h] = (s * fmaf(-z, qsum[h], P[h])) * kInvSqrtD;
-      }
-    } else {
-#pragma unroll
-      for (int h = 0; h < GRP; ++h) sc[h] = -INFINITY;
     }
-    // V codes of this token into the warp's staging rows
-    {
-      const uint4* pr = reinterpret_cast<const uint4*>(v_res + row * kWordsPerRow);
-      const uint4 a = pr[0], b = pr[1];
-      uint32_t* dst = vr[warp][lane];
-      dst[0] = a.x; dst[1] = a.y; dst[2] = a.z; dst[3] = a.w;
-      dst[4] = b.x; dst[5] = b.y; dst[6] = b.z; dst[7] = b.w;
-      uint32_t* dsf = vf[warp][lane];
-      if (inU) {
-        const uint4* pf = reinterpret_cast<const uint4*>(v_ref + row * kWordsPerRow);
-        const uint4 c = pf[0], e = pf[1];
-        dsf[0] = c.x; dsf[1] = c.y; dsf[2] = c.z; dsf[3] = c.w;
-        dsf[4] = e.x; dsf[5] = e.y; dsf[6] = e.z; dsf[7] = e.w;
-      } else {
-#pragma unroll
-        for (int i = 0; i < kWordsPerRow; ++i) dsf[i] = 0u;
-      }
-    }
-    const float sv = valid ? sfd::half_bits_to_float(v_scale[row]) : 0.0f;
-    const float zv = valid ? sfd::half_bits_to_float(v_zero[row]) : 0.0f;
-    const float off = inU ? -zv : 1.5f - zv;  // v = s * (code + off)
+    cp_async_wait_attn<kOutStages - 1>();
+    __syncwarp();
+    const int st = (ti - tile0) % kOutStages;
+    float alpha[GRP];
+    bool any_rescale = false;
+    float f[GRP];
 #pragma unroll
     for (int h = 0; h < GRP; ++h) {
-      const float mt = warp_max(sc[h]);
+      const float sc = valid ? ssc[warp][st][h][lane & 15] : -INFINITY;
+      const float mt = warp_max(sc);
       const float nm = fmaxf(m[h], mt);
-      const float r = (m[h] == -INFINITY) ? 0.0f : __expf(m[h] - nm);
+      f[h] = (m[h] == -INFINITY) ? 0.0f : __expf(m[h] - nm);
+      any_rescale |= (f[h] != 1.0f);
       m[h] = nm;
-      l[h] *= r;
-      bs[h] *= r;
+      const float pr = valid ? __expf(sc - nm) : 0.0f;
+      const float al = pr * sv;
+      alpha[h] = al;
+      const __half ahi = __float2half_rn(al);
+      const __half alo = __float2half_rn(al - __half2float(ahi));
+      lsum[h] = fmaf(lsum[h], f[h], pr);
+      csum[h] = fmaf(csum[h], f[h], al * (1.5f - zv));
+      asum[h] = fmaf(asum[h], f[h], __half2float(ahi) + __half2float(alo));
+      if (lane < 16) {
+        a16[warp][h][lane] = ahi;
+        a16[warp][GRP + h][lane] = alo;
+      }
 #pragma unroll
-      for (int dd = 0; dd < 4; ++dd) o[h][dd] *= r;
-      const float p = valid ? __expf(sc[h] - nm) : 0.0f;
-      l[h] += p;
-      bs[h] = fmaf(p * sv, off, bs[h]);
-      alpha[warp][lane][h] = p * sv;
+      for (int dd = 0; dd < 4; ++dd) uo[h][dd] *= f[h];
+    }
+    // rescale the accumulators of rows whose head's running max moved
+    if (__any_sync(0xffffffffu, any_rescale)) {
+      const int r0 = g8, r1 = g8 + 8;
+      float f0 = 1.0f, f1 = 1.0f;
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) {
+        if (r0 == h || r0 == GRP + h) f0 = f[h];
+        if (r1 == h || r1 == GRP + h) f1 = f[h];
+      }
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) {
+        acc[nt][0] *= f0; acc[nt][1] *= f0;
+        acc[nt][2] *= f1; acc[nt][3] *= f1;
+      }
+    }
+    // refined tokens of the tile: alpha (c_f - 1.5) on the CUDA cores
+    unsigned um = __ballot_sync(0xffffffffu, inU);
+    while (um) {
+      const int src = __ffs(um) - 1;
+      um &= um - 1u;
+      const size_t row = static_cast<size_t>(g) * T + tb + src;
+      const uint32_t wf = v_ref[row * kWordsPerRow + (lane >> 2)] >> ((lane & 3) * 8);
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) {
+        const float ah = __shfl_sync(0xffffffffu, alpha[h], src);
+#pragma unroll
+        for (int dd = 0; dd < 4; ++dd)
+          uo[h][dd] = fmaf(ah, static_cast<float>((wf >> (2 * dd)) & 3u) - 1.5f, uo[h][dd]);
+      }
     }
     __syncwarp();
-    const int wsel = lane >> 2, sh = (lane & 3) * 8;
-    for (int tt = 0; tt < 32; ++tt) {
-      const uint32_t cr = (vr[warp][tt][wsel] >> sh) & 0xFFu;
-      const uint32_t cf = (vf[warp][tt][wsel] >> sh) & 0xFFu;
+    // A: weights (rows) x tokens; B: tokens x dims, built per token pair
+    const uint32_t* arow0 = reinterpret_cast<const uint32_t*>(&a16[warp][g8][0]);
+    const uint32_t* arow1 = reinterpret_cast<const uint32_t*>(&a16[warp][g8 + 8][0]);
+    const uint32_t a0 = arow0[tig], a2 = arow0[tig + 4];
+    const uint32_t a1 = arow1[tig], a3 = arow1[tig + 4];
+    const uint4* ra = reinterpret_cast<const uint4*>(&vrow[warp][st][2 * tig][0]);
+    const uint4* rb = reinterpret_cast<const uint4*>(&vrow[warp][st][2 * tig + 1][0]);
+    const uint4* rc = reinterpret_cast<const uint4*>(&vrow[warp][st][2 * tig + 8][0]);
+    const uint4* rd = reinterpret_cast<const uint4*>(&vrow[warp][st][2 * tig + 9][0]);
 #pragma unroll
-      for (int dd = 0; dd < 4; ++dd) {
-        const float code = static_cast<float>(((cr >> (2 * dd)) & 3u) * 4u + ((cf >> (2 * dd)) & 3u));
+    for (int half = 0; half < 2; ++half) {
+      const uint4 A4 = ra[half], B4 = rb[half], C4 = rc[half], D4 = rd[half];
+      const uint32_t wa[4] = {A4.x, A4.y, A4.z, A4.w}, wb[4] = {B4.x, B4.y, B4.z, B4.w};
+      const uint32_t wc[4] = {C4.x, C4.y, C4.z, C4.w}, wd[4] = {D4.x, D4.y, D4.z, D4.w};
 #pragma unroll
-        for (int h = 0; h < GRP; ++h) o[h][dd] = fmaf(alpha[warp][tt][h], code, o[h][dd]);
+      for (int j = 0; j < 4; ++j) {
+        const int w = half * 4 + j;
+        const uint32_t xa = wa[j] >> (2 * g8), xb = wb[j] >> (2 * g8);
+        const uint32_t xc = wc[j] >> (2 * g8), xd = wd[j] >> (2 * g8);
+        const uint32_t b0lo = (__byte_perm(xa, xb, 0x5410) & 0x00030003u) | 0x64006400u;
+        const uint32_t b0hi = (__byte_perm(xa, xb, 0x7632) & 0x00030003u) | 0x64006400u;
+        const uint32_t b1lo = (__byte_perm(xc, xd, 0x5410) & 0x00030003u) | 0x64006400u;
+        const uint32_t b1hi = (__byte_perm(xc, xd, 0x7632) & 0x00030003u) | 0x64006400u;
+        mma_f16f32(acc[2 * w], a0, a1, a2, a3, b0lo, b1lo);
+        mma_f16f32(acc[2 * w + 1], a0, a1, a2, a3, b0hi, b1hi);
       }
     }
     __syncwarp();
   }
-  // per warp: l and bs are per-lane partials with the warp-uniform max m
+  cp_async_wait_attn<0>();
+  // this warp's o: rows (heads hi / lo) -> wo[warp][head][dim]
+  __syncwarp();
+#pragma unroll
+  for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int r = (c < 2) ? g8 : g8 + 8;
+      const int hh = r < GRP ? r : (r < 2 * GRP ? r - GRP : -1);
+      // resident value s (2^b_f c_r + m_f - z): the code part carries 2^b_f = 4
+      if (hh >= 0) atomicAdd(&wo[warp][hh][8 * nt + 2 * tig + (c & 1)], 4.0f * acc[nt][c]);
+    }
+  __syncwarp();
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
-    const float lt = warp_sum(l[h]);
-    const float bt = warp_sum(bs[h]);
+    const float lt = warp_sum(lsum[h]);
+    const float ct = warp_sum(csum[h]);
+    const float at = warp_sum(asum[h]);
     if (lane == 0) { wm[warp][h] = m[h]; wl[warp][h] = lt; }
 #pragma unroll
-    for (int dd = 0; dd < 4; ++dd) wo[warp][h][lane * 4 + dd] = o[h][dd] + bt;
+    for (int dd = 0; dd < 4; ++dd) wo[warp][h][4 * lane + dd] += uo[h][dd] + ct - 4.0f * 1024.0f * at;
   }
   __syncthreads();
   for (int e = threadIdx.x; e < GRP * (D + 2); e += blockDim.x) {
     const int h = e / (D + 2), j = e % (D + 2);
     float M = -INFINITY;
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w][h]);
-    float acc = 0.0f;
+    for (int w = 0; w < kOutWarps; ++w) M = fmaxf(M, wm[w][h]);
+    float accv = 0.0f;
     if (j == 0) {
-      acc = M;
+      accv = M;
     } else {
-      for (int w = 0; w < 4; ++w) {
+      for (int w = 0; w < kOutWarps; ++w) {
         if (wm[w][h] == -INFINITY) continue;
-        const float f = __expf(wm[w][h] - M);
-        acc += f * (j == 1 ? wl[w][h] : wo[w][h][j - 2]);
+        const float fct = __expf(wm[w][h] - M);
+        accv += fct * (j == 1 ? wl[w][h] : wo[w][h][j - 2]);
       }
     }
-    part[((static_cast<size_t>(g) * GRP + h) * splits + split) * (D + 2) + j] = acc;
+    part[((static_cast<size_t>(g) * GRP + h) * splits + split) * (D + 2) + j] = accv;
   }
-  // the last CTA of this KV group to finish merges every split's partials
-  // (threadfence-then-count, so no CTA ever waits for another)
   __shared__ int last;
   __threadfence();
   __syncthreads();
@@ -549,20 +911,44 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
   __syncthreads();
   if (!last) return;
   __threadfence();
+  // merge: split maxima -> per-split factors -> per (head, dim) sums whose
+  // loads are independent of one another
+  // the per-warp output tiles are dead once the partials are written: reuse
+  // them for the per-split factors (GRP * kMaxSplits <= kOutWarps * GRP * D)
+  static_assert(kMaxSplits <= 4 * D, "merge factors must fit in the output tiles");
+  float (*fct)[kMaxSplits] = reinterpret_cast<float (*)[kMaxSplits]>(&wo[0][0][0]);
+  __shared__ float Lh[GRP];
+  const float* pg = part + static_cast<size_t>(g) * GRP * splits * (D + 2);
+  for (int e = threadIdx.x; e < GRP * splits; e += blockDim.x) fct[e / splits][e % splits] = __ldcg(pg + e * (D + 2));
+  __syncthreads();
+  for (int h = warp; h < GRP; h += kOutWarps) {
+    float M = -INFINITY;
+    for (int sp = lane; sp < splits; sp += 32) M = fmaxf(M, fct[h][sp]);
+    M = warp_max(M);
+    float Ls = 0.0f;
+    for (int sp = lane; sp < splits; sp += 32) {
+      const float ms = fct[h][sp];
+      const float f = ms == -INFINITY ? 0.0f : __expf(ms - M);
+      Ls = fmaf(f, __ldcg(pg + (h * splits + sp) * (D + 2) + 1), Ls);
+      fct[h][sp] = f;
+    }
+    Ls = warp_sum(Ls);
+    if (lane == 0) Lh[h] = Ls;
+  }
+  __syncthreads();
   for (int e = threadIdx.x; e < GRP * D; e += blockDim.x) {
     const int h = e / D, d = e % D;
-    const float* p = part + (static_cast<size_t>(g) * GRP + h) * splits * (D + 2);
-    float M = -INFINITY;
-    for (int sp = 0; sp < splits; ++sp) M = fmaxf(M, __ldcg(p + sp * (D + 2)));
-    float Lsum = 0.0f, O = 0.0f;
-    for (int sp = 0; sp < splits; ++sp) {
-      const float ms = __ldcg(p + sp * (D + 2));
-      if (ms == -INFINITY) continue;
-      const float f = __expf(ms - M);
-      Lsum = fmaf(f, __ldcg(p + sp * (D + 2) + 1), Lsum);
-      O = fmaf(f, __ldcg(p + sp * (D + 2) + 2 + d), O);
+    const float* ph = pg + static_cast<size_t>(h) * splits * (D + 2) + 2 + d;
+    float O0 = 0.0f, O1 = 0.0f, O2 = 0.0f, O3 = 0.0f;
+    int sp = 0;
+    for (; sp + 3 < splits; sp += 4) {
+      O0 = fmaf(fct[h][sp], __ldcg(ph + sp * (D + 2)), O0);
+      O1 = fmaf(fct[h][sp + 1], __ldcg(ph + (sp + 1) * (D + 2)), O1);
+      O2 = fmaf(fct[h][sp + 2], __ldcg(ph + (sp + 2) * (D + 2)), O2);
+      O3 = fmaf(fct[h][sp + 3], __ldcg(ph + (sp + 3) * (D + 2)), O3);
     }
-    out[(static_cast<size_t>(g) * GRP + h) * D + d] = O / Lsum;
+    for (; sp < splits; ++sp) O0 = fmaf(fct[h][sp], __ldcg(ph + sp * (D + 2)), O0);
+    out[(static_cast<size_t>(g) * GRP + h) * D + d] = ((O0 + O1) + (O2 + O3)) / Lh[h];
   }
 }
 
@@ -584,22 +970,27 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
               float* out, char* ws, const Layout& L, cudaStream_t s) {
   float* score = reinterpret_cast<float*>(ws + L.score);
   int32_t* cand = reinterpret_cast<int32_t*>(ws + L.cand);
+  int32_t* cand2 = reinterpret_cast<int32_t*>(ws + L.cand2);
   double* kap = reinterpret_cast<double*>(ws + L.kap);
   int32_t* sel_head = reinterpret_cast<int32_t*>(ws + L.sel);
   uint32_t* umask = reinterpret_cast<uint32_t*>(ws + L.umask);
   float* part = reinterpret_cast<float*>(ws + L.part);
   float* smax = reinterpret_cast<float*>(ws + L.smax);
   int32_t* status = reinterpret_cast<int32_t*>(ws + L.status);
+  int32_t* done = reinterpret_cast<int32_t*>(ws + L.count);
   const int grp = GRP;
+  const int sms = sf::sm_count();
 
   SF_CHECK_CUDA(cudaMemsetAsync(ws + L.smax, 0, L.total - L.smax, s));
+  const int ntiles = (T + 15) / 16;
+  dim3 ga(std::max(1, std::min((ntiles + 3) / 4, (4 * sms + Hkv - 1) / Hkv)), Hkv);
+  attn_score_mma_kernel<GRP><<<ga, 128, 0, s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, score, smax);
+  sf_status st = sf::check_launch("attn_score_mma_kernel");
+  if (st != SF_OK) return st;
+  const int cap = grp * k;  // row length of sel_out
   if (k > 0 && k < T) {
-    dim3 ga((T + 127) / 128, Hkv);
-    attn_score_kernel<GRP><<<ga, 128, 0, s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, score, smax);
-    sf_status st = sf::check_launch("attn_score_kernel");
-    if (st != SF_OK) return st;
     attn_select_kernel<GRP><<<Hq, kSelThreads, 0, s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, k, score, smax,
-                                                       cand, kap, sel_head, status);
+                                                       cand, cand2, kap, sel_head, status);
     st = sf::check_launch("attn_select_kernel");
     if (st != SF_OK) return st;
     const size_t smem = sizeof(uint32_t) * L.words_t;
@@ -608,28 +999,26 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
     attn_union_kernel<<<Hkv, 1024, smem, s>>>(sel_head, grp, T, k, L.words_t, umask, sel_out, sel_n, status);
     st = sf::check_launch("attn_union_kernel");
     if (st != SF_OK) return st;
+  } else if (k == 0) {
+    SF_CHECK_CUDA(cudaMemsetAsync(umask, 0, sizeof(uint32_t) * Hkv * static_cast<size_t>(L.words_t), s));
+    SF_CHECK_CUDA(cudaMemsetAsync(sel_n, 0, sizeof(int32_t) * Hkv, s));
   } else {
-    // no selection needed: everything (k == T) or nothing (k == 0) refined,
-    // scores still come from pass A
-    dim3 ga((T + 127) / 128, Hkv);
-    attn_score_kernel<GRP><<<ga, 128, 0, s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, score, smax);
-    sf_status st = sf::check_launch("attn_score_kernel");
+    fill_all_kernel<<<dim3(32, Hkv), 256, 0, s>>>(T, grp, k, L.words_t, umask, sel_out, sel_n);
+    st = sf::check_launch("fill_all_kernel");
     if (st != SF_OK) return st;
-    if (k == 0) {
-      SF_CHECK_CUDA(cudaMemsetAsync(umask, 0, sizeof(uint32_t) * Hkv * static_cast<size_t>(L.words_t), s));
-      SF_CHECK_CUDA(cudaMemsetAsync(sel_n, 0, sizeof(int32_t) * Hkv, s));
-    } else {
-      fill_all_kernel<<<dim3(32, Hkv), 256, 0, s>>>(T, grp, k, L.words_t, umask, sel_out, sel_n);
-      st = sf::check_launch("fill_all_kernel");
-      if (st != SF_OK) return st;
-    }
+  }
+  if (k > 0) {
+    dim3 gr(std::max(1, std::min((cap + 7) / 8, 128)), Hkv);
+    attn_refine_scores_kernel<GRP><<<gr, 256, 0, s>>>(q, kv->k_res, kv->k_ref, kv->k_scale, kv->k_zero, T, cap,
+                                                      sel_out, sel_n, score);
+    st = sf::check_launch("attn_refine_scores_kernel");
+    if (st != SF_OK) return st;
   }
   dim3 gb(L.splits, Hkv);
-  int32_t* done = reinterpret_cast<int32_t*>(ws + L.count);
-  attn_out_kernel<GRP><<<gb, 128, 0, s>>>(q, kv->k_res, kv->k_ref, kv->k_scale, kv->k_zero, kv->v_res, kv->v_ref,
-                                          kv->v_scale, kv->v_zero, T, L.tps, L.words_t, L.splits, score, umask, part,
-                                          done, out);
-  return sf::check_launch("attn_out_kernel");
+  attn_out_mma_kernel<GRP><<<gb, out_warps<GRP>() * 32, 0, s>>>(kv->v_res, kv->v_ref, kv->v_scale, kv->v_zero, T,
+                                                                L.tps, L.words_t, L.splits, score, umask, part,
+                                                                done, out);
+  return sf::check_launch("attn_out_mma_kernel");
 }
 
 }  // namespace

@@ -9,6 +9,7 @@
 // to tau are taken in ascending channel order until k are chosen (an ordered
 // scan), which is the "ties to the lower index" rule.  A final ordered
 // compaction writes the union in ascending order.
+#include "act.cuh"
 #include "block_scan.cuh"
 #include "sf_internal.h"
 
@@ -33,7 +34,7 @@ struct RowState {
 
 __global__ void __launch_bounds__(kThreads)
 select_topk_kernel(const uint16_t* __restrict__ x, int B, int K, int k, int32_t* __restrict__ idx_out,
-                   int32_t* __restrict__ n_out) {
+                   int32_t* __restrict__ n_out, uint32_t* __restrict__ act) {
   extern __shared__ uint8_t smem[];
   uint8_t* flags = smem;                                                   // [K]
   int* hist1 = reinterpret_cast<int*>(smem + ((K + 15) & ~15));           // [kMaxRows][256]
@@ -177,6 +178,166 @@ select_topk_kernel(const uint16_t* __restrict__ x, int B, int K, int k, int32_t*
       if (flags[j]) idx_out[pos++] = j;
     if (tid == 0) *n_out = bad ? -1 : total;
   }
+
+  // prepared activations (batch 1): per 32-channel slab the fixed-point
+  // planes, plus which of its channels are selected and how many selected
+  // channels precede it (= the selected channel's position in idx_out)
+  if (act != nullptr) {  // K <= 32768: at most one slab per thread
+    const int nslab = K >> 5;
+    const int sl = tid;
+    const bool active = sl < nslab;
+    uint32_t m = 0;
+    if (active)
+      for (int j = 0; j < 32; ++j) m |= static_cast<uint32_t>(flags[32 * sl + j] != 0) << j;
+    int total;
+    const int pre = sfd::block_exclusive_scan(active ? __popc(m) : 0, scan_scratch, &total);
+    sfd::act_write_slab_in_block(x + 32 * (active ? sl : 0), act + static_cast<size_t>(sfd::kActWords) * sl, active,
+                                 m, pre);
+  }
+}
+
+__global__ void __launch_bounds__(256)
+act_prepare_kernel(const uint16_t* __restrict__ x, int nslab, uint32_t* __restrict__ act) {
+  const int sl = blockIdx.x * blockDim.x + threadIdx.x;
+  const bool active = sl < nslab;
+  sfd::act_write_slab_in_block(x + 32 * (active ? sl : 0), act + static_cast<size_t>(sfd::kActWords) * sl, active, 0u,
+                               0);
+}
+
+// ---- several single-row selections in one launch (one CTA each) -------------
+// The row is read once into shared memory; the histograms, the ordered
+// tie pass, the compaction and the prepared activations all work from there.
+constexpr int kMaxSelJobs = 8;
+struct SelJobDev {
+  const uint16_t* x;
+  int K, k;
+  int32_t* idx;
+  int32_t* n;
+  uint32_t* act;
+};
+struct SelManyArgs {
+  SelJobDev job[kMaxSelJobs];
+};
+
+__global__ void __launch_bounds__(kThreads)
+select_act_many_kernel(const __grid_constant__ SelManyArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const SelJobDev& J = a.job[blockIdx.x];
+  const int K = J.K, k = J.k, tid = threadIdx.x;
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [K]
+  uint8_t* flags = smem + 2 * K;                     // [K]
+  __shared__ int hist1[256], hist2[128];
+  __shared__ int scan_scratch[33];
+  __shared__ int b1_sh, k1_sh, tau_sh, r_sh, bad;
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(J.x);
+    uint4* dst = reinterpret_cast<uint4*>(xs);
+    for (int i = tid; i < K / 8; i += kThreads) dst[i] = src[i];
+  }
+  for (int j = tid; j < K; j += kThreads) flags[j] = 0;
+  for (int j = tid; j < 256; j += kThreads) hist1[j] = 0;
+  for (int j = tid; j < 128; j += kThreads) hist2[j] = 0;
+  if (tid == 0) bad = 0;
+  __syncthreads();
+  for (int j = tid; j < K; j += kThreads) {
+    const uint32_t v = xs[j];
+    if ((v & 0x7F80u) == 0x7F80u) bad = 1;
+    atomicAdd(&hist1[(v & 0x7FFFu) >> 7], 1);
+  }
+  __syncthreads();
+  const int warp = tid >> 5, lane = tid & 31;
+  if (warp == 0) {
+    int above = 0, b1 = -1, k1 = 0;
+    for (int base = 255; base >= 0 && b1 < 0; base -= 32) {
+      const int c = hist1[base - lane];
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, k > 0 && above + incl >= k && above + incl - c < k);
+      if (m) {
+        const int src = __ffs(m) - 1;
+        b1 = base - src;
+        k1 = k - (above + __shfl_sync(0xffffffffu, incl - c, src));
+      }
+      above += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) { b1_sh = b1; k1_sh = k1; }
+  }
+  __syncthreads();
+  const int b1 = b1_sh;
+  if (b1 >= 0)
+    for (int j = tid; j < K; j += kThreads) {
+      const uint32_t v = xs[j] & 0x7FFFu;
+      if (static_cast<int>(v >> 7) == b1) atomicAdd(&hist2[v & 0x7Fu], 1);
+    }
+  __syncthreads();
+  if (warp == 0) {
+    const int kk = k1_sh;
+    int above = 0, tau = -1, r = 0;
+    if (b1 >= 0) {
+      for (int base = 127; base >= 0 && tau < 0; base -= 32) {
+        const int c = hist2[base - lane];
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, above + incl >= kk && above + incl - c < kk);
+        if (m) {
+          const int src = __ffs(m) - 1;
+          tau = (b1 << 7) | (base - src);
+          r = kk - (above + __shfl_sync(0xffffffffu, incl - c, src));
+        }
+        above += __shfl_sync(0xffffffffu, incl, 31);
+      }
+    }
+    if (lane == 0) { tau_sh = tau; r_sh = r; }
+  }
+  __syncthreads();
+  const int tau = tau_sh;
+  // ordered tie pass over contiguous chunks, then the compaction
+  const int chunk = (K + kThreads - 1) / kThreads;
+  const int j0 = min(K, tid * chunk), j1 = min(K, j0 + chunk);
+  {
+    int eq = 0;
+    if (tau >= 0)
+      for (int j = j0; j < j1; ++j) eq += ((xs[j] & 0x7FFF) == tau);
+    int total;
+    int rank = sfd::block_exclusive_scan(eq, scan_scratch, &total);
+    if (tau >= 0)
+      for (int j = j0; j < j1; ++j) {
+        const int key = xs[j] & 0x7FFF;
+        if (key > tau) flags[j] = 1;
+        else if (key == tau) { if (rank < r_sh) flags[j] = 1; ++rank; }
+      }
+  }
+  __syncthreads();
+  {
+    int c = 0;
+    for (int j = j0; j < j1; ++j) c += flags[j];
+    int total;
+    int pos = sfd::block_exclusive_scan(c, scan_scratch, &total);
+    for (int j = j0; j < j1; ++j)
+      if (flags[j]) J.idx[pos++] = j;
+    if (tid == 0) *J.n = bad ? -1 : total;
+  }
+  __syncthreads();
+  if (J.act != nullptr) {  // K <= 32768: at most one slab per thread
+    const int nslab = K >> 5;
+    const int sl = tid;
+    const bool active = sl < nslab;
+    uint32_t m = 0;
+    if (active)
+      for (int j = 0; j < 32; ++j) m |= static_cast<uint32_t>(flags[32 * sl + j] != 0) << j;
+    int total;
+    const int pre = sfd::block_exclusive_scan(active ? __popc(m) : 0, scan_scratch, &total);
+    sfd::act_write_slab_in_block(xs + 32 * (active ? sl : 0), J.act + static_cast<size_t>(sfd::kActWords) * sl,
+                                 active, m, pre);
+  }
 }
 
 }  // namespace
@@ -188,11 +349,56 @@ extern "C" sf_status sf_select_topk(const uint16_t* x, int B, int K, int k, int3
   SF_REQUIRE(K >= 1 && K <= 65536, "sf_select_topk: K must be in [1, 65536]");
   SF_REQUIRE(k >= 0 && k <= K, "sf_select_topk: k must be in [0, K]");
   const size_t smem = static_cast<size_t>((K + 15) & ~15) + sizeof(int) * kMaxRows * (256 + 128);
-  static bool attr_set = false;
-  if (!attr_set) {
-    SF_CHECK_CUDA(cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
-    attr_set = true;
-  }
-  select_topk_kernel<<<1, kThreads, smem, sf::as_cuda(stream)>>>(x, B, K, k, idx_out, n_out);
+  SF_CHECK_CUDA(cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
+  select_topk_kernel<<<1, kThreads, smem, sf::as_cuda(stream)>>>(x, B, K, k, idx_out, n_out, nullptr);
   return sf::check_launch("select_topk_kernel");
+}
+
+extern "C" size_t sf_act_bytes(int K) {
+  return K > 0 ? static_cast<size_t>(K / 32) * sfd::kActWords * sizeof(uint32_t) : 0;
+}
+
+extern "C" sf_status sf_select_topk_act(const uint16_t* x, int K, int k, int32_t* idx_out, int32_t* n_out, void* act,
+                                        sf_stream_t stream) {
+  SF_REQUIRE(x && idx_out && n_out && act, "sf_select_topk_act: null pointer");
+  SF_REQUIRE(K >= 32 && K <= 32768 && K % 32 == 0, "sf_select_topk_act: K must be a multiple of 32 in [32, 32768]");
+  SF_REQUIRE(k >= 0 && k <= K, "sf_select_topk_act: k must be in [0, K]");
+  SF_REQUIRE(sf::aligned(act, 16), "sf_select_topk_act: act must be 16-byte aligned");
+  const size_t smem = static_cast<size_t>((K + 15) & ~15) + sizeof(int) * kMaxRows * (256 + 128);
+  SF_CHECK_CUDA(cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
+  select_topk_kernel<<<1, kThreads, smem, sf::as_cuda(stream)>>>(x, 1, K, k, idx_out, n_out,
+                                                                 static_cast<uint32_t*>(act));
+  return sf::check_launch("select_topk_kernel");
+}
+
+extern "C" sf_status sf_act_prepare(const uint16_t* x, int K, void* act, sf_stream_t stream) {
+  SF_REQUIRE(x && act, "sf_act_prepare: null pointer");
+  SF_REQUIRE(K >= 32 && K % 32 == 0, "sf_act_prepare: K must be a positive multiple of 32");
+  SF_REQUIRE(sf::aligned(act, 16), "sf_act_prepare: act must be 16-byte aligned");
+  const int nslab = K / 32;
+  act_prepare_kernel<<<(nslab + 255) / 256, 256, 0, sf::as_cuda(stream)>>>(x, nslab, static_cast<uint32_t*>(act));
+  return sf::check_launch("act_prepare_kernel");
+}
+
+extern "C" sf_status sf_select_topk_act_many(const sf_select_job* jobs, int count, sf_stream_t stream) {
+  SF_REQUIRE(jobs, "sf_select_topk_act_many: null pointer");
+  SF_REQUIRE(count >= 1 && count <= kMaxSelJobs, "sf_select_topk_act_many: count must be in [1, %d]", kMaxSelJobs);
+  SelManyArgs a{};
+  int kmax = 0;
+  for (int i = 0; i < count; ++i) {
+    const sf_select_job& j = jobs[i];
+    SF_REQUIRE(j.x && j.idx_out && j.n_out, "sf_select_topk_act_many: job %d has a null pointer", i);
+    SF_REQUIRE(j.K >= 32 && j.K <= 32768 && j.K % 32 == 0,
+               "sf_select_topk_act_many: K must be a multiple of 32 in [32, 32768] (job %d)", i);
+    SF_REQUIRE(j.k >= 0 && j.k <= j.K, "sf_select_topk_act_many: k out of range (job %d)", i);
+    SF_REQUIRE(sf::aligned(j.x, 16) && (j.act == nullptr || sf::aligned(j.act, 16)),
+               "sf_select_topk_act_many: x and act must be 16-byte aligned (job %d)", i);
+    a.job[i] = SelJobDev{j.x, j.K, j.k, j.idx_out, j.n_out, static_cast<uint32_t*>(j.act)};
+    kmax = j.K > kmax ? j.K : kmax;
+  }
+  const size_t smem = static_cast<size_t>(kmax) * 3;
+  SF_CHECK_CUDA(cudaFuncSetAttribute(select_act_many_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem)));
+  select_act_many_kernel<<<count, kThreads, smem, sf::as_cuda(stream)>>>(a);
+  return sf::check_launch("select_act_many_kernel");
 }

@@ -397,3 +397,129 @@ def test_cache_group_matches_oracle(sf):
     grp.close()
     for cache, _, _ in entries:
         cache.close()
+
+
+# ---- batch-1 fast path (prepared activations, several matrices per launch) -----
+
+@pytest.mark.parametrize("K,pct", [(4096, 3), (14336, 3), (1024, 10)])
+def test_select_act_matches_select(sf, K, pct):
+    k = count_fraction(pct, K)
+    x = gen_activations(31 + K, 1, K, outlier_channels(32, K, count_fraction("1/2", K)), 30.0)
+    x[0, 5] = 0
+    xd = bf16_dev(x)
+    idx = torch.zeros(k, dtype=torch.int32, device="cuda")
+    n = torch.zeros(1, dtype=torch.int32, device="cuda")
+    act = torch.zeros(sf.act_bytes(K) // 4, dtype=torch.int32, device="cuda")
+    sf.select_topk_act(xd, k, idx, n, act)
+    torch.cuda.synchronize()
+    S = oselect.select_topk(x, k)
+    np.testing.assert_array_equal(idx.cpu().numpy()[: int(n.item())], S)
+    a = act.cpu().numpy().view(np.uint32).reshape(K // 32, 32)
+    sel = [32 * s + j for s in range(K // 32) for j in range(32) if (a[s, 26] >> j) & 1]
+    assert sel == S.tolist()
+    prefix = np.concatenate([[0], np.cumsum([bin(int(m)).count("1") for m in a[:, 26]])[:-1]])
+    np.testing.assert_array_equal(a[:, 27], prefix)
+    # the planes rebuild x: X_j = signed byte 2 * 2^16 + byte 1 * 2^8 + byte 0, x = X * fscale
+    xf = (x[0].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    fscale = a[:, 25].view(np.float32).astype(np.float64)
+    for s in range(0, K // 32, max(1, K // 32 // 16)):
+        for wi in range(2):
+            for kk in range(4):
+                b0, b1, b2 = (a[s, (wi * 4 + kk) * 3 + p] for p in range(3))
+                for b in range(4):
+                    top = int((b2 >> (8 * b)) & 0xFF)
+                    top = top - 256 if top >= 128 else top
+                    X = top * 65536 + int((b1 >> (8 * b)) & 0xFF) * 256 + int((b0 >> (8 * b)) & 0xFF)
+                    j = 32 * s + 16 * wi + kk + 4 * b
+                    assert abs(X * fscale[s] - xf[j]) <= fscale[s] / 2 + 1e-300
+
+
+@pytest.mark.parametrize("K,Ns,cap_pct,pct", [(4096, (4096, 1024, 1024), 10, 3), (14336, (4096,), 10, 3),
+                                              (4096, (2048, 512), 25, 5)])
+def test_gemv_batch1_jobs_with_caches(sf, K, Ns, cap_pct, pct):
+    G, b_r, b_f = 128, 2, 2
+    k = count_fraction(pct, K)
+    cap = count_fraction(cap_pct, K)
+    mats = []
+    for i, N in enumerate(Ns):
+        W = gen_weight(1100 + 7 * i + K, N, K)
+        qw = sf.quantize_nested(dev(W), G, b_r, b_f)
+        rows = np.sort(np.random.default_rng(N + i).choice(N, size=min(N, 160), replace=False))
+        mats.append(dict(qw=qw, qz=oquant.quantize_nested(W[rows], G, b_r, b_f), rows=rows,
+                         cache=sf.RefineCache(K, N * b_f // 8, cap, k, _host_master(qw)),
+                         orc=ocache.LRUCache(K, cap), y=torch.empty(N, dtype=torch.float32, device="cuda"),
+                         y0=torch.empty(N, dtype=torch.float32, device="cuda")))
+    idx = torch.zeros(k, dtype=torch.int32, device="cuda")
+    n = torch.zeros(1, dtype=torch.int32, device="cuda")
+    act = torch.zeros(sf.act_bytes(K) // 4, dtype=torch.int32, device="cuda")
+    act0 = torch.zeros_like(act)
+    grp = sf.RefineGroup([(m["cache"], idx, n) for m in mats])
+    jobs = sf.Batch1Jobs([(m["qw"], m["cache"], False, m["y"]) for m in mats])
+    jobs0 = sf.Batch1Jobs([(m["qw"], None, False, m["y0"]) for m in mats])
+    side = torch.cuda.Stream()
+    outl = outlier_channels(1200 + K, K, count_fraction("1/2", K))
+    for step in range(3):
+        x = gen_activations(1300 + step, 1, K, outl, 30.0)
+        xd = bf16_dev(x)
+        sf.select_topk_act(xd, k, idx, n, act)
+        grp.prefetch(torch.cuda.current_stream(), side)
+        jobs.run(xd, act)
+        sf.act_prepare(xd, act0)
+        jobs0.run(xd, act0)
+        torch.cuda.synchronize()
+        S = oselect.select_topk(x, k)
+        for m in mats:
+            want = m["orc"].step(S.tolist())
+            assert m["cache"].sets()["misses"] == want["misses"]
+            y_ref, a = ogemv.gemv_refine(m["qz"], x, S)
+            _check_gemv(m["y"].cpu().numpy()[None, m["rows"]], y_ref, a)
+            r0, a0 = ogemv.gemv_refine(m["qz"], x, [])
+            _check_gemv(m["y0"].cpu().numpy()[None, m["rows"]], r0, a0)
+    grp.close()
+    for m in mats:
+        m["cache"].close()
+
+
+def test_gemv_batch1_store_mode(sf):
+    N, K, G = 1024, 8192, 128
+    W = gen_weight(1400, N, K)
+    qw = sf.quantize_nested(dev(W), G, 2, 1)
+    x = gen_activations(1401, 1, K, outlier_channels(1402, K, 40), 30.0)
+    k = count_fraction(5, K)
+    xd = bf16_dev(x)
+    idx = torch.zeros(k, dtype=torch.int32, device="cuda")
+    n = torch.zeros(1, dtype=torch.int32, device="cuda")
+    act = torch.zeros(sf.act_bytes(K) // 4, dtype=torch.int32, device="cuda")
+    y = torch.empty(N, dtype=torch.float32, device="cuda")
+    sf.select_topk_act(xd, k, idx, n, act)
+    sf.gemv_refine_batch1([(qw, None, True, y)], xd, act)
+    torch.cuda.synchronize()
+    y_ref, a = ogemv.gemv_refine(oquant.quantize_nested(W, G, 2, 1), x, oselect.select_topk(x, k))
+    _check_gemv(y.cpu().numpy()[None, :], y_ref, a)
+
+
+def test_select_act_many_matches_single(sf):
+    """One launch selecting four rows of different lengths equals four
+    single-row selections (indices and prepared bytes) and the oracle."""
+    specs = [(4096, 123), (4096, 123), (4096, 123), (14336, 430)]
+    xs, single, many = [], [], []
+    for i, (K, k) in enumerate(specs):
+        x = gen_activations(1500 + i, 1, K, outlier_channels(1510 + i, K, count_fraction("1/2", K)), 30.0)
+        xs.append(x)
+        bufs = []
+        for _ in range(2):
+            bufs.append((torch.zeros(k, dtype=torch.int32, device="cuda"), torch.zeros(1, dtype=torch.int32, device="cuda"),
+                         torch.zeros(sf.act_bytes(K) // 4, dtype=torch.int32, device="cuda")))
+        single.append(bufs[0])
+        many.append(bufs[1])
+    xds = [bf16_dev(x) for x in xs]
+    for (K, k), xd, (idx, n, act) in zip(specs, xds, single):
+        sf.select_topk_act(xd, k, idx, n, act)
+    jobs = sf.SelectJobs([(xd, k, idx, n, act) for (K, k), xd, (idx, n, act) in zip(specs, xds, many)])
+    jobs.run()
+    torch.cuda.synchronize()
+    for (K, k), x, a, b in zip(specs, xs, single, many):
+        want = oselect.select_topk(x, k)
+        np.testing.assert_array_equal(b[0].cpu().numpy()[: int(b[1].item())], want)
+        np.testing.assert_array_equal(a[0].cpu().numpy()[: int(a[1].item())], want)
+        np.testing.assert_array_equal(a[2].cpu().numpy(), b[2].cpu().numpy())
