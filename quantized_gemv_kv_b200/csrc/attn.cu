@@ -47,7 +47,7 @@ size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 Layout make_layout(int Hq, int Hkv, int T, int k, int sms) {
   Layout L{};
-  const int want = std::max(1, std::min(kMaxSplits, sms / Hkv));  // one wave of pass-B CTAs
+  const int want = std::max(1, std::min(kMaxSplits, 2 * sms / Hkv));  // one wave of pass-B CTAs at 2 per SM
   int tps = (T + want - 1) / want;
   tps = std::max(128, (tps + 127) / 128 * 128);
   L.tps = tps;
@@ -369,6 +369,167 @@ __device__ int block_ordered_compact(int n, Pred pred, Emit emit, int* wsum /* 3
 
 constexpr int kDirectRank = 1024;  // candidates ranked pairwise (one per thread)
 
+// Query-side setup of pass S (all threads call): q in fp64 into qd, its l1
+// norm and the binary exponent of max |q|; flags the KV group when the
+// nonzero q exponents span more than the exact-key precondition allows.
+__device__ void select_q_prologue(const uint16_t* __restrict__ q, int h, int g, double* qd, double* l1_out,
+                                  int* qe_out, int32_t* __restrict__ status) {
+  const int tid = threadIdx.x;
+  for (int d = tid; d < D; d += blockDim.x)
+    qd[d] = static_cast<double>(sfd::bf16_bits_to_float(q[static_cast<size_t>(h) * D + d]));
+  __syncthreads();
+  if (tid < 32) {
+    double l1 = 0.0;
+    int emin = 100000, emax = -100000;
+    for (int d = tid; d < D; d += 32) {
+      const double v = qd[d];
+      l1 += fabs(v);
+      if (v != 0.0) {
+        int e;
+        frexp(v, &e);
+        emin = min(emin, e);
+        emax = max(emax, e);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+      emin = min(emin, __shfl_xor_sync(0xffffffffu, emin, o));
+      emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+    }
+    if (tid == 0) {
+      *l1_out = l1;
+      *qe_out = emax >= emin ? emax : 0;  // binary exponent of max |q| (frexp convention)
+      // 53 - 9 - b - log2(d) with b = 4, d = 128
+      if (emax >= emin && emax - emin > 53 - 9 - 4 - 7) atomicOr(status + g, 1);
+    }
+  }
+  __syncthreads();
+}
+
+// Error bound of the fast scores (pass A): q rounded to 24-bit fixed point
+// (|dq| <= 2^(e-24) per entry), exact integer products and sums, an fp32
+// combine of the three plane sums, the fp32 sum of q (<= gamma_128 l1), and
+// the roundings of the zero-point term, the fma, the scale and 1/sqrt(d).
+// Returns the half-width eps_s of the band; two fast scores whose exact
+// values are ordered one way differ by at least -2 eps_s the other way.
+__device__ __forceinline__ double select_eps(double s_max, double l1, int qe, float amax) {
+  const double u = 5.9604644775390625e-8;  // 2^-24
+  const double gam = 130.0 * u / (1.0 - 130.0 * u);
+  const double qround = ldexp(1.0, qe - 24);
+  const double eps_k = s_max * (4.0 * 3.0 * D * qround + l1 * (136.0 * u + 16.0 * gam));
+  return 2.0 * (static_cast<double>(kInvSqrtD) * eps_k + 4.0 * u * static_cast<double>(amax));
+}
+
+// Last stage of pass S (all threads call): the candidates F[0..ncand) (token
+// order) are re-keyed exactly in fp64 and the k best by (key desc, token asc)
+// written to sel (k entries, ascending rank order is not required).
+__device__ void select_finish(const uint32_t* __restrict__ k_res, const uint16_t* __restrict__ k_scale,
+                              const uint16_t* __restrict__ k_zero, int g, int T, int k, const double* qd,
+                              const int32_t* __restrict__ F, int ncand, double* __restrict__ kp, int* hist,
+                              int* scan_scratch, int* binfo, int32_t* __restrict__ sel) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  for (int i = tid; i < ncand; i += nthr) {
+    const int t = F[i];
+    const size_t row = static_cast<size_t>(g) * T + t;
+    const uint4* w4 = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
+    const uint4 x0 = w4[0], x1 = w4[1];
+    const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    const double sv = static_cast<double>(sfd::half_bits_to_float(k_scale[row]));
+    const double z = static_cast<double>(sfd::half_bits_to_float(k_zero[row]));
+    double E = 0.0;
+#pragma unroll
+    for (int wi = 0; wi < 8; ++wi) {
+      const uint32_t word = w[wi];
+#pragma unroll 4
+      for (int j = 0; j < 16; ++j) {
+        const double c = static_cast<double>((word >> (2 * j)) & 3u);
+        E = fma(qd[16 * wi + j], c * 4.0 + 1.5 - z, E);
+      }
+    }
+    kp[i] = sv * E;
+  }
+  __syncthreads();
+
+  // few candidates (the usual case): rank each one directly against all
+  // others by (key desc, token asc) -- no synchronised passes
+  if (ncand <= kDirectRank && ncand <= nthr) {
+    double* kd = reinterpret_cast<double*>(hist);  // 2048 ints = 1024 doubles of scratch
+    for (int i = tid; i < ncand; i += nthr) kd[i] = kp[i];
+    __syncthreads();
+    int take = 0;
+    const int i = tid;
+    if (i < ncand) {
+      const double ki = kd[i];
+      int rank = 0;
+      for (int j = 0; j < ncand; ++j) {
+        const double kj = kd[j];
+        rank += (kj > ki) || (kj == ki && j < i);  // F is in token order
+      }
+      take = rank < k;
+    }
+    int tot;
+    const int pos = sfd::block_exclusive_scan(take, scan_scratch, &tot);
+    if (take) sel[pos] = F[i];
+    return;
+  }
+
+  // many candidates: exact top-k by an 8-pass radix select on the 64-bit keys
+  unsigned long long pre64 = 0, pm64 = 0;
+  int kr = k;
+  for (int pass = 0; pass < 8; ++pass) {
+    const int shift = 56 - 8 * pass;
+    for (int i = tid; i < 256; i += nthr) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < ncand; i += nthr) {
+      const unsigned long long key = okey64(kp[i]);
+      if ((key & pm64) == pre64) atomicAdd(&hist[(key >> shift) & 255], 1);
+    }
+    __syncthreads();
+    find_bin_from_top(hist, 256, kr, binfo);
+    __syncthreads();
+    pre64 |= static_cast<unsigned long long>(binfo[0]) << shift;
+    pm64 |= 255ull << shift;
+    kr = binfo[1];
+    __syncthreads();
+  }
+  {
+    const int chunk = (ncand + nthr - 1) / nthr;
+    const int i0 = min(ncand, tid * chunk), i1 = min(ncand, i0 + chunk);
+    int eq = 0;
+    for (int i = i0; i < i1; ++i) eq += okey64(kp[i]) == pre64;
+    int tot;
+    int rank = sfd::block_exclusive_scan(eq, scan_scratch, &tot);
+    int take = 0;
+    {
+      int rk = rank;
+      for (int i = i0; i < i1; ++i) {
+        const unsigned long long key = okey64(kp[i]);
+        if (key > pre64) ++take;
+        else if (key == pre64) { if (rk < kr) ++take; ++rk; }
+      }
+    }
+    int pos = sfd::block_exclusive_scan(take, scan_scratch, &tot);
+    for (int i = i0; i < i1; ++i) {
+      const unsigned long long key = okey64(kp[i]);
+      bool ok = false;
+      if (key > pre64) ok = true;
+      else if (key == pre64) { ok = rank < kr; ++rank; }
+      if (ok) sel[pos++] = F[i];
+    }
+  }
+}
+
+// Exact per-head top-k for any T, streaming the scores from global memory:
+//  1. amax over the fast scores and a strided sample of them;
+//  2. a threshold theta from the sample such that at least k scores are
+//     >= theta + 2 eps (checked by counting; lowered until true, at worst to
+//     -inf), so every token whose exact key can reach the top k has a fast
+//     score >= theta;
+//  3. G = {t : score_t >= theta} in token order, tau = k-th largest score over
+//     G by radix select (equal to the k-th largest overall);
+//  4. candidates F = {t in G : score_t >= tau - 2 eps}, re-keyed exactly in
+//     fp64, ranked by (key desc, token asc).
 template <int GRP>
 __global__ void __launch_bounds__(kSelThreads)
 attn_select_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
@@ -392,35 +553,7 @@ attn_select_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ 
   int32_t* F = cand2 + static_cast<size_t>(h) * T;
   double* kp = kap + static_cast<size_t>(h) * T;
 
-  for (int d = tid; d < D; d += kSelThreads)
-    qd[d] = static_cast<double>(sfd::bf16_bits_to_float(q[static_cast<size_t>(h) * D + d]));
-  __syncthreads();
-  if (tid < 32) {
-    double l1 = 0.0;
-    int emin = 100000, emax = -100000;
-    for (int d = tid; d < D; d += 32) {
-      const double v = qd[d];
-      l1 += fabs(v);
-      if (v != 0.0) {
-        int e;
-        frexp(v, &e);
-        emin = min(emin, e);
-        emax = max(emax, e);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-      emin = min(emin, __shfl_xor_sync(0xffffffffu, emin, o));
-      emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
-    }
-    if (tid == 0) {
-      l1_sh = l1;
-      qe_sh = emax >= emin ? emax : 0;  // binary exponent of max |q| (frexp convention)
-      // 53 - 9 - b - log2(d) with b = 4, d = 128
-      if (emax >= emin && emax - emin > 53 - 9 - 4 - 7) atomicOr(status + g, 1);
-    }
-  }
+  select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status);
 
   // 1. amax and a strided sample
   const int ns = T < kSamples ? T : kSamples;
@@ -439,18 +572,7 @@ attn_select_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ 
     __syncthreads();
     amax = red[0];
   }
-
-  // error bound of the fast scores (pass A): q rounded to 24-bit fixed point
-  // (|dq| <= 2^(e-24) per entry), exact integer products and sums, an fp32
-  // combine of the three plane sums, the fp32 sum of q (<= gamma_128 l1), and
-  // the roundings of the zero-point term, the fma, the scale and 1/sqrt(d).
-  const double u = 5.9604644775390625e-8;  // 2^-24
-  const double gam = 130.0 * u / (1.0 - 130.0 * u);
-  const double s_max = static_cast<double>(smax[g]);
-  const double l1 = l1_sh;
-  const double qround = ldexp(1.0, qe_sh - 24);
-  const double eps_k = s_max * (4.0 * 3.0 * D * qround + l1 * (136.0 * u + 16.0 * gam));
-  const double eps_s = 2.0 * (static_cast<double>(kInvSqrtD) * eps_k + 4.0 * u * static_cast<double>(amax));
+  const double eps_s = select_eps(static_cast<double>(smax[g]), l1_sh, qe_sh, amax);
 
   // 2. threshold from the sample: aim at ~2k + 64 tokens above it
   double theta = -INFINITY;
@@ -504,99 +626,154 @@ attn_select_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ 
   const double tau = static_cast<double>(from_okey32(prefix));
   const double thr = tau - 2.0 * eps_s;
 
-  // 4. candidates F (token order), exact keys
+  // 4. candidates F (token order), exact keys, ranking
   const int ncand = block_ordered_compact(
       nG, [&](int i) { return static_cast<double>(sc[G[i]]) >= thr; }, [&](int pos, int i) { F[pos] = G[i]; },
       scan_scratch);
-  for (int i = tid; i < ncand; i += kSelThreads) {
-    const int t = F[i];
-    const size_t row = static_cast<size_t>(g) * T + t;
-    const uint4* w4 = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
-    const uint4 x0 = w4[0], x1 = w4[1];
-    const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-    const double sv = static_cast<double>(sfd::half_bits_to_float(k_scale[row]));
-    const double z = static_cast<double>(sfd::half_bits_to_float(k_zero[row]));
-    double E = 0.0;
-#pragma unroll
-    for (int wi = 0; wi < 8; ++wi) {
-      const uint32_t word = w[wi];
-#pragma unroll 4
-      for (int j = 0; j < 16; ++j) {
-        const double c = static_cast<double>((word >> (2 * j)) & 3u);
-        E = fma(qd[16 * wi + j], c * 4.0 + 1.5 - z, E);
-      }
+  select_finish(k_res, k_scale, k_zero, g, T, k, qd, F, ncand, kp, hist, scan_scratch, binfo,
+                sel_head + static_cast<size_t>(h) * k);
+}
+
+// Block-parallel search of a histogram from the top (all threads call):
+// out[0] = the bin holding the kk-th largest element, out[1] = kk minus the
+// elements in higher bins.  Thread t sums its own run of bins, an exclusive
+// scan gives the count above each run, and the one thread whose run crosses
+// kk walks it.
+__device__ void find_bin_from_top_block(const int* hist, int nb, int kk, int* out, int* scratch) {
+  const int per = (nb + blockDim.x - 1) / blockDim.x;
+  const int hi = nb - static_cast<int>(threadIdx.x) * per;  // exclusive upper bin of this run
+  const int lo = max(0, hi - per);
+  int c = 0;
+  for (int b = hi - 1; b >= lo; --b) c += hist[b];
+  int tot;
+  const int above = sfd::block_exclusive_scan(c, scratch, &tot);
+  if (c > 0 && above < kk && above + c >= kk) {
+    int a = above;
+    for (int b = hi - 1; b >= lo; --b) {
+      const int n = hist[b];
+      if (a + n >= kk) { out[0] = b; out[1] = kk - a; break; }
+      a += n;
     }
-    kp[i] = sv * E;
+  }
+  if (threadIdx.x == 0 && tot < kk) { out[0] = 0; out[1] = kk; }
+  __syncthreads();
+}
+
+// Exact per-head top-k for T <= kRegKeys * kSelThreads with the scores held
+// in registers (one coalesced read of the head's scores):
+//  1. tau = the k-th largest fast score, by a 3-pass radix select (11, 11 and
+//     10 bits of the order-preserving key) over the register-held keys;
+//  2. candidates F = {t : score_t >= tau - 2 eps}, compacted in token order
+//     straight from the registers (warp w holds the contiguous token range
+//     [w seg, (w+1) seg), row i of it at w seg + 32 i + lane);
+//  3. exact fp64 keys and ranking as in the streaming kernel.
+constexpr int kRegKeys = 32;
+
+template <int GRP>
+__global__ void __launch_bounds__(kSelThreads)
+attn_select_reg_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
+                       const uint16_t* __restrict__ k_scale, const uint16_t* __restrict__ k_zero, int T, int k,
+                       const float* __restrict__ score, const float* __restrict__ smax, int32_t* __restrict__ cand2,
+                       double* __restrict__ kap, int32_t* __restrict__ sel_head, int32_t* __restrict__ status) {
+  __shared__ __align__(16) int hist[2048];
+  __shared__ double qd[D];
+  __shared__ int scan_scratch[64];
+  __shared__ int binfo[2];
+  __shared__ float red[32];
+  __shared__ double l1_sh;
+  __shared__ int qe_sh;
+  const int h = blockIdx.x, g = h / GRP, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float* sc = score + static_cast<size_t>(h) * T;
+  int32_t* F = cand2 + static_cast<size_t>(h) * T;
+  double* kp = kap + static_cast<size_t>(h) * T;
+
+  const int seg = (((T + 31) >> 5) + 31) & ~31;  // tokens per warp: a multiple of 32, <= 32 kRegKeys
+  const int t0 = warp * seg + lane;
+  const int tend = min(T, warp * seg + seg);
+  uint32_t key[kRegKeys];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kRegKeys; ++i) {
+    const int t = t0 + 32 * i;
+    const float v = t < tend ? sc[t] : 0.0f;
+    key[i] = okey32(v);
+    amax = fmaxf(amax, fabsf(v));
+  }
+  for (int i = tid; i < 2048; i += kSelThreads) hist[i] = 0;
+  select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status);  // ends with __syncthreads
+  {
+    const float m = warp_max(amax);
+    if (lane == 0) red[warp] = m;
+  }
+
+  // 1. tau by radix select over the registers
+#pragma unroll
+  for (int i = 0; i < kRegKeys; ++i)
+    if (t0 + 32 * i < tend) atomicAdd(&hist[key[i] >> 21], 1);
+  __syncthreads();
+  find_bin_from_top_block(hist, 2048, k, binfo, scan_scratch);
+  const uint32_t b1 = static_cast<uint32_t>(binfo[0]);
+  int kk = binfo[1];
+  for (int i = tid; i < 2048; i += kSelThreads) hist[i] = 0;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < kRegKeys; ++i)
+    if (t0 + 32 * i < tend && (key[i] >> 21) == b1) atomicAdd(&hist[(key[i] >> 10) & 2047u], 1);
+  __syncthreads();
+  find_bin_from_top_block(hist, 2048, kk, binfo, scan_scratch);
+  const uint32_t p2 = (b1 << 11) | static_cast<uint32_t>(binfo[0]);
+  kk = binfo[1];
+  for (int i = tid; i < 1024; i += kSelThreads) hist[i] = 0;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < kRegKeys; ++i)
+    if (t0 + 32 * i < tend && (key[i] >> 10) == p2) atomicAdd(&hist[key[i] & 1023u], 1);
+  __syncthreads();
+  find_bin_from_top_block(hist, 1024, kk, binfo, scan_scratch);
+  const float tau = from_okey32((p2 << 10) | static_cast<uint32_t>(binfo[0]));
+  if (warp == 0) {
+    const float mm = warp_max(red[lane]);
+    if (lane == 0) red[0] = mm;
+  }
+  __syncthreads();
+  const double eps_s = select_eps(static_cast<double>(smax[g]), l1_sh, qe_sh, red[0]);
+  // smallest float f with f >= tau - 2 eps: (double)x >= tau - 2 eps <=> x >= f
+  const float fthr = __double2float_ru(static_cast<double>(tau) - 2.0 * eps_s);
+
+  // 2. candidates in token order
+  int cnt = 0;
+#pragma unroll
+  for (int i = 0; i < kRegKeys; ++i)
+    cnt += __popc(__ballot_sync(0xffffffffu, t0 + 32 * i < tend && from_okey32(key[i]) >= fthr));
+  if (lane == 0) scan_scratch[warp] = cnt;
+  __syncthreads();
+  if (warp == 0) {
+    const int v = scan_scratch[lane];
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    scan_scratch[32 + lane] = incl - v;
+    if (lane == 31) binfo[0] = incl;
+  }
+  __syncthreads();
+  int off = scan_scratch[32 + warp];
+  const int ncand = binfo[0];
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int i = 0; i < kRegKeys; ++i) {
+    const bool p = t0 + 32 * i < tend && from_okey32(key[i]) >= fthr;
+    const unsigned bal = __ballot_sync(0xffffffffu, p);
+    if (p) F[off + __popc(bal & lt)] = t0 + 32 * i;
+    off += __popc(bal);
   }
   __syncthreads();
 
-  // 5a. few candidates (the usual case): rank each one directly against all
-  // others by (key desc, token asc) -- no synchronised passes
-  if (ncand <= kDirectRank) {
-    double* kd = reinterpret_cast<double*>(hist);  // 2048 ints = 1024 doubles of scratch
-    for (int i = tid; i < ncand; i += kSelThreads) kd[i] = kp[i];
-    __syncthreads();
-    int take = 0;
-    const int i = tid;
-    if (i < ncand) {
-      const double ki = kd[i];
-      int rank = 0;
-      for (int j = 0; j < ncand; ++j) {
-        const double kj = kd[j];
-        rank += (kj > ki) || (kj == ki && j < i);  // F is in token order
-      }
-      take = rank < k;
-    }
-    int tot;
-    const int pos = sfd::block_exclusive_scan(take, scan_scratch, &tot);
-    if (take) sel_head[static_cast<size_t>(h) * k + pos] = F[i];
-    return;
-  }
-
-  // 5. exact top-k among the candidates by (key desc, token asc)
-  unsigned long long pre64 = 0, pm64 = 0;
-  int kr = k;
-  for (int pass = 0; pass < 8; ++pass) {
-    const int shift = 56 - 8 * pass;
-    for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
-    __syncthreads();
-    for (int i = tid; i < ncand; i += kSelThreads) {
-      const unsigned long long key = okey64(kp[i]);
-      if ((key & pm64) == pre64) atomicAdd(&hist[(key >> shift) & 255], 1);
-    }
-    __syncthreads();
-    find_bin_from_top(hist, 256, kr, binfo);
-    __syncthreads();
-    pre64 |= static_cast<unsigned long long>(binfo[0]) << shift;
-    pm64 |= 255ull << shift;
-    kr = binfo[1];
-    __syncthreads();
-  }
-  {
-    const int chunk = (ncand + kSelThreads - 1) / kSelThreads;
-    const int i0 = min(ncand, tid * chunk), i1 = min(ncand, i0 + chunk);
-    int eq = 0;
-    for (int i = i0; i < i1; ++i) eq += okey64(kp[i]) == pre64;
-    int tot;
-    int rank = sfd::block_exclusive_scan(eq, scan_scratch, &tot);
-    int take = 0;
-    {
-      int rk = rank;
-      for (int i = i0; i < i1; ++i) {
-        const unsigned long long key = okey64(kp[i]);
-        if (key > pre64) ++take;
-        else if (key == pre64) { if (rk < kr) ++take; ++rk; }
-      }
-    }
-    int pos = sfd::block_exclusive_scan(take, scan_scratch, &tot);
-    for (int i = i0; i < i1; ++i) {
-      const unsigned long long key = okey64(kp[i]);
-      bool ok = false;
-      if (key > pre64) ok = true;
-      else if (key == pre64) { ok = rank < kr; ++rank; }
-      if (ok) sel_head[static_cast<size_t>(h) * k + pos++] = F[i];
-    }
-  }
+  // 3. exact keys and ranking
+  select_finish(k_res, k_scale, k_zero, g, T, k, qd, F, ncand, kp, hist, scan_scratch, binfo,
+                sel_head + static_cast<size_t>(h) * k);
 }
 
 // ---- pass U: union per KV head ---------------------------------------------
@@ -683,16 +860,22 @@ attn_refine_scores_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
 // ---- pass B on the tensor cores ------------------------------------------------
 //
 // o_h = sum_t p_{h,t} v_t / sum_t p_{h,t} with v_t = s_t (4 c_t + 1.5 - z_t):
-// the code part 4 sum_t alpha_{h,t} c_t is a product of the weights
-// alpha_{h,t} = p_{h,t} s_t (rows = heads) with the code matrix (tokens x dims)
-// on mma.m16n8k16 (f16 in, f32 accumulate).  alpha is split into an f16 high part and an f16 remainder
-// (rows h and GRP + h), so the products keep ~22 bits.  Codes enter as the
-// f16 values 1024 + c, exact, built for a pair of tokens and one dim with
-// one shift, one byte permute and one mask; the 1024 * sum(alpha) they add is
-// removed at the end.  The offset part sum_t alpha_{h,t} (1.5 - z_t) is a
-// scalar per head.  Refined tokens (in the union) add alpha (c_f - 1.5) s-scaled
-// codes of their refinement bits on the CUDA cores; their scores were already
-// refined in the score buffer.  Online softmax runs per 16-token tile.
+// the code part 4 sum_t alpha_{h,t} c_t, alpha_{h,t} = p_{h,t} s_t, is a
+// product of the code matrix (dims x tokens, MMA rows = dims) with the weights
+// (tokens x columns) on mma.m16n8k16 (f16 in, f32 accumulate).  Each weight
+// is split into an f16 high part and an f16 remainder (columns h and GRP + h),
+// so the products keep ~22 bits.  Codes enter as the f16 values 1024 + c,
+// exact, built for one dim and a pair of tokens with one shift, one byte
+// permute and one mask; the 1024 sum(alpha) they add is removed at the end.
+// The offset part sum_t alpha_{h,t} (1.5 - z_t) is a scalar per head.
+// Refined tokens (in the union) add alpha (c_f - 1.5), their refinement codes,
+// on the CUDA cores; their scores were already refined in the score buffer.
+//
+// A CTA owns a token range of one KV group and walks it in sub-chunks of
+// kSub tokens: the sub-chunk's score maximum per head is found first, so every
+// weight is computed once, by one thread, relative to a fixed maximum and
+// stored in shared memory (no per-tile online rescaling); the warps then run
+// the MMAs over their tiles of 16 tokens, the codes staged by cp.async.
 __device__ __forceinline__ void mma_f16f32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                            uint32_t b0, uint32_t b1) {
   asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
@@ -700,235 +883,311 @@ __device__ __forceinline__ void mma_f16f32(float (&d)[4], uint32_t a0, uint32_t 
                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-constexpr int kOutStages = 4;
-template <int GRP>
-__host__ __device__ constexpr int out_warps() { return GRP <= 4 ? 8 : 4; }
+constexpr int kSub = 2048;         // tokens per sub-chunk
+constexpr int kOutThreads = 256;
+constexpr int kOW = kOutThreads / 32;
+constexpr int kRing = 4;           // cp.async stages per warp
 
 template <int GRP>
-__global__ void __launch_bounds__(256)
-attn_out_mma_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__ v_ref,
-                    const uint16_t* __restrict__ v_scale, const uint16_t* __restrict__ v_zero, int T, int tps,
-                    int words_t, int splits, const float* __restrict__ score, const uint32_t* __restrict__ umask,
-                    float* __restrict__ part, int32_t* __restrict__ done, float* __restrict__ out) {
-  constexpr int kOutWarps = out_warps<GRP>();
-  __shared__ __align__(16) uint32_t vrow[kOutWarps][kOutStages][16][kWordsPerRow];
-  __shared__ float ssc[kOutWarps][kOutStages][GRP][16];
-  __shared__ __align__(16) __half a16[kOutWarps][16][16];
-  __shared__ float wm[kOutWarps][GRP], wl[kOutWarps][GRP];
-  __shared__ float wo[kOutWarps][GRP][D];
+struct OutCfg {
+  static constexpr int NC = 2 * GRP;           // weight columns: high parts of the heads, then remainders
+  static constexpr int NT = NC <= 8 ? 1 : 2;   // MMA n-tiles of 8 columns
+  static constexpr int kStr = kSub + 8;        // halves per weight row: conflict-free fragment loads
+  static constexpr size_t alpha_bytes = static_cast<size_t>(NT) * 8 * kStr * 2;
+  static constexpr size_t ring_bytes = static_cast<size_t>(kOW) * kRing * 16 * kWordsPerRow * 4;
+  static constexpr size_t wo_bytes = static_cast<size_t>(GRP) * D * 4;
+  static constexpr size_t ulist_bytes = static_cast<size_t>(kSub) * 4;
+  static constexpr size_t smem = alpha_bytes + ring_bytes + wo_bytes + ulist_bytes;
+  static_assert(alpha_bytes >= static_cast<size_t>(GRP) * kMaxSplits * 4, "merge factors must fit the weight tile");
+};
+
+template <int GRP>
+__global__ void __launch_bounds__(kOutThreads)
+attn_out_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__ v_ref,
+                const uint16_t* __restrict__ v_scale, const uint16_t* __restrict__ v_zero, int T, int tps, int words_t,
+                int splits, const float* __restrict__ score, const uint32_t* __restrict__ umask,
+                float* __restrict__ part, int32_t* __restrict__ done, float* __restrict__ out) {
+  using C = OutCfg<GRP>;
+  constexpr int NT = C::NT, kStr = C::kStr;
+  extern __shared__ __align__(16) unsigned char smem[];
+  __half* as = reinterpret_cast<__half*>(smem);                                      // [NT*8][kStr]
+  uint32_t* ring = reinterpret_cast<uint32_t*>(smem + C::alpha_bytes);               // [kOW][kRing][16][8]
+  float* wo = reinterpret_cast<float*>(smem + C::alpha_bytes + C::ring_bytes);       // [GRP][D]
+  int* ulist = reinterpret_cast<int*>(smem + C::alpha_bytes + C::ring_bytes + C::wo_bytes);  // [kSub]
+  __shared__ float red[kOW][GRP];
+  __shared__ float red2[kOW][3 * GRP];
+  __shared__ float Msh[GRP], Fsh[GRP];
+  __shared__ int ucount;
+
   const int g = blockIdx.y, split = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g8 = lane >> 2, tig = lane & 3;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, tig = lane & 3;
   const int t0s = split * tps, t1s = min(T, t0s + tps);
-  // this warp's contiguous share of the split, in 16-token tiles
-  const int ntile = (t1s - t0s + 15) / 16;
-  const int tpw = (ntile + kOutWarps - 1) / kOutWarps;
-  const int tile0 = warp * tpw, tile1 = min(ntile, tile0 + tpw);
+  const size_t rowg = static_cast<size_t>(g) * T;
 
-  for (int e = lane; e < GRP * D; e += 32) wo[warp][e / D][e % D] = 0.0f;
-  for (int e = lane; e < 16 * 16; e += 32) a16[warp][e / 16][e % 16] = __float2half_rn(0.0f);
+  for (int e = tid; e < (NT * 8 - C::NC) * kStr; e += kOutThreads) as[C::NC * kStr + e] = __float2half_rn(0.0f);
+  for (int e = tid; e < GRP * D; e += kOutThreads) wo[e] = 0.0f;
+  if (tid < GRP) Msh[tid] = -INFINITY;
 
-  float m[GRP], lsum[GRP], csum[GRP], asum[GRP], uo[GRP][4];
-  float acc[16][4];
+  float lsum[GRP], csum[GRP], asum[GRP], uo[GRP][4];
+  float acc[NT][8][4];
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
-    m[h] = -INFINITY;
     lsum[h] = csum[h] = asum[h] = 0.0f;
 #pragma unroll
     for (int dd = 0; dd < 4; ++dd) uo[h][dd] = 0.0f;
   }
 #pragma unroll
-  for (int nt = 0; nt < 16; ++nt)
+  for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) acc[nt][c] = 0.0f;
+    for (int w = 0; w < 8; ++w)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[nt][w][c] = 0.0f;
+  // head of each of this lane's accumulator columns (-1: padding column)
+  int colh[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int n = nt * 8 + 2 * tig + c;
+      colh[nt][c] = n < GRP ? n : (n < 2 * GRP ? n - GRP : -1);
+    }
 
-  auto issue = [&](int ti) {
-    const int st = (ti - tile0) % kOutStages;
-    const int tb = t0s + ti * 16;
-    if (lane < 16) {
-      const int t = tb + lane;
-      if (t < t1s) {
-        const size_t row = static_cast<size_t>(g) * T + t;
-        const uint32_t* src = v_res + row * kWordsPerRow;
-        cp_async16_attn(&vrow[warp][st][lane][0], src);
-        cp_async16_attn(&vrow[warp][st][lane][4], src + 4);
+  for (int c0 = t0s; c0 < t1s; c0 += kSub) {
+    const int n = min(t1s, c0 + kSub) - c0;
+    const int ntile = (n + 15) >> 4;
+    const int tpw = (ntile + kOW - 1) / kOW;
+    const int tile0 = min(ntile, warp * tpw), tile1 = min(ntile, tile0 + tpw);
+    auto issue = [&](int ti) {
+      const int st = (ti - tile0) % kRing;
+      const int tok = 16 * ti + (lane >> 1);
+      if (tok < n)
+        cp_async16_attn(ring + ((warp * kRing + st) * 16 + (lane >> 1)) * kWordsPerRow + (lane & 1) * 4,
+                        v_res + (rowg + c0 + tok) * kWordsPerRow + (lane & 1) * 4);
+    };
+    // start the code stream while the weights are being computed
+    for (int i = 0; i < kRing - 1; ++i) {
+      if (tile0 + i < tile1) issue(tile0 + i);
+      cp_async_commit_attn();
+    }
+
+    // 1. the sub-chunk's maximum score per head
+    {
+      float mx[GRP];
 #pragma unroll
-        for (int h = 0; h < GRP; ++h) cp_async4_attn(&ssc[warp][st][h][lane], score + (static_cast<size_t>(g) * GRP + h) * T + t);
+      for (int h = 0; h < GRP; ++h) mx[h] = -INFINITY;
+      for (int i = tid; i < n; i += kOutThreads)
+#pragma unroll
+        for (int h = 0; h < GRP; ++h) mx[h] = fmaxf(mx[h], score[(static_cast<size_t>(g) * GRP + h) * T + c0 + i]);
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) {
+        const float m = warp_max(mx[h]);
+        if (lane == 0) red[warp][h] = m;
       }
+      if (tid == 0) ucount = 0;
+      __syncthreads();
+      if (tid < GRP) {
+        float m = -INFINITY;
+        for (int w = 0; w < kOW; ++w) m = fmaxf(m, red[w][tid]);
+        const float mo = Msh[tid], mn = fmaxf(mo, m);
+        Fsh[tid] = mo == -INFINITY ? 0.0f : __expf(mo - mn);
+        Msh[tid] = mn;
+      }
+      __syncthreads();
     }
-  };
-  for (int i = 0; i < kOutStages - 1; ++i) {
-    if (tile0 + i < tile1) issue(tile0 + i);
-    cp_async_commit_attn();
-  }
-  for (int ti = tile0; ti < tile1; ++ti) {
-    if (ti + kOutStages - 1 < tile1) issue(ti + kOutStages - 1);
-    cp_async_commit_attn();
-    // this tile's per-token scalars (plain loads; the ring carries the bulk)
-    const int tb = t0s + ti * 16;
-    const int t = tb + (lane & 15);
-    const bool valid = lane < 16 && t < t1s;
-    float sv = 0.0f, zv = 0.0f;
-    bool inU = false;
-    if (valid) {
-      const size_t row = static_cast<size_t>(g) * T + t;
-      sv = sfd::half_bits_to_float(v_scale[row]);
-      zv = sfd::half_bits_to_float(v_zero[row]);
-      inU = (umask[static_cast<size_t>(g) * words_t + (t >> 5)] >> (t & 31)) & 1u;
-    }
-    cp_async_wait_attn<kOutStages - 1>();
-    __syncwarp();
-    const int st = (ti - tile0) % kOutStages;
-    float alpha[GRP];
-    bool any_rescale = false;
-    float f[GRP];
+    float M[GRP], F[GRP];
+    bool rescale = false;
 #pragma unroll
     for (int h = 0; h < GRP; ++h) {
-      const float sc = valid ? ssc[warp][st][h][lane & 15] : -INFINITY;
-      const float mt = warp_max(sc);
-      const float nm = fmaxf(m[h], mt);
-      f[h] = (m[h] == -INFINITY) ? 0.0f : __expf(m[h] - nm);
-      any_rescale |= (f[h] != 1.0f);
-      m[h] = nm;
-      const float pr = valid ? __expf(sc - nm) : 0.0f;
-      const float al = pr * sv;
-      alpha[h] = al;
-      const __half ahi = __float2half_rn(al);
-      const __half alo = __float2half_rn(al - __half2float(ahi));
-      lsum[h] = fmaf(lsum[h], f[h], pr);
-      csum[h] = fmaf(csum[h], f[h], al * (1.5f - zv));
-      asum[h] = fmaf(asum[h], f[h], __half2float(ahi) + __half2float(alo));
-      if (lane < 16) {
-        a16[warp][h][lane] = ahi;
-        a16[warp][GRP + h][lane] = alo;
-      }
-#pragma unroll
-      for (int dd = 0; dd < 4; ++dd) uo[h][dd] *= f[h];
+      M[h] = Msh[h];
+      F[h] = Fsh[h];
+      rescale |= F[h] != 1.0f;
     }
-    // rescale the accumulators of rows whose head's running max moved
-    if (__any_sync(0xffffffffu, any_rescale)) {
-      const int r0 = g8, r1 = g8 + 8;
-      float f0 = 1.0f, f1 = 1.0f;
+    if (rescale && c0 != t0s) {  // uniform over the block
 #pragma unroll
       for (int h = 0; h < GRP; ++h) {
-        if (r0 == h || r0 == GRP + h) f0 = f[h];
-        if (r1 == h || r1 == GRP + h) f1 = f[h];
+        lsum[h] *= F[h];
+        csum[h] *= F[h];
+        asum[h] *= F[h];
+#pragma unroll
+        for (int dd = 0; dd < 4; ++dd) uo[h][dd] *= F[h];
       }
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        acc[nt][0] *= f0; acc[nt][1] *= f0;
-        acc[nt][2] *= f1; acc[nt][3] *= f1;
+      for (int nt = 0; nt < NT; ++nt) {
+        float f0 = 1.0f, f1 = 1.0f;
+#pragma unroll
+        for (int h = 0; h < GRP; ++h) {
+          if (colh[nt][0] == h) f0 = F[h];
+          if (colh[nt][1] == h) f1 = F[h];
+        }
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          acc[nt][w][0] *= f0; acc[nt][w][1] *= f1;
+          acc[nt][w][2] *= f0; acc[nt][w][3] *= f1;
+        }
       }
     }
-    // refined tokens of the tile: alpha (c_f - 1.5) on the CUDA cores
-    unsigned um = __ballot_sync(0xffffffffu, inU);
-    while (um) {
-      const int src = __ffs(um) - 1;
-      um &= um - 1u;
-      const size_t row = static_cast<size_t>(g) * T + tb + src;
-      const uint32_t wf = v_ref[row * kWordsPerRow + (lane >> 2)] >> ((lane & 3) * 8);
+
+    // 2. weights into shared memory (zero past the end of the last tile),
+    //    sums, and the list of refined tokens
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = 0; base < 16 * ntile; base += kOutThreads) {
+      const int i = base + tid;
+      const bool valid = i < n;
+      bool inU = false;
+      if (i < 16 * ntile) {
+        if (valid) {
+          const size_t row = rowg + c0 + i;
+          const float sv = sfd::half_bits_to_float(v_scale[row]);
+          const float zv = sfd::half_bits_to_float(v_zero[row]);
+#pragma unroll
+          for (int h = 0; h < GRP; ++h) {
+            const float p = __expf(score[(static_cast<size_t>(g) * GRP + h) * T + c0 + i] - M[h]);
+            const float al = p * sv;
+            const __half ahi = __float2half_rn(al);
+            const __half alo = __float2half_rn(al - __half2float(ahi));
+            as[h * kStr + i] = ahi;
+            as[(GRP + h) * kStr + i] = alo;
+            lsum[h] += p;
+            csum[h] = fmaf(al, 1.5f - zv, csum[h]);
+            asum[h] += __half2float(ahi) + __half2float(alo);
+          }
+          const int t = c0 + i;
+          inU = (umask[static_cast<size_t>(g) * words_t + (t >> 5)] >> (t & 31)) & 1u;
+        } else {
+#pragma unroll
+          for (int h = 0; h < 2 * GRP; ++h) as[h * kStr + i] = __float2half_rn(0.0f);
+        }
+      }
+      const unsigned b = __ballot_sync(0xffffffffu, inU);
+      if (b) {
+        int pos = 0;
+        if (lane == __ffs(b) - 1) pos = atomicAdd(&ucount, __popc(b));
+        pos = __shfl_sync(0xffffffffu, pos, __ffs(b) - 1);
+        if (inU) ulist[pos + __popc(b & lt)] = i;
+      }
+    }
+    __syncthreads();
+
+    // 3. MMAs over this warp's tiles
+    for (int ti = tile0; ti < tile1; ++ti) {
+      if (ti + kRing - 1 < tile1) issue(ti + kRing - 1);
+      cp_async_commit_attn();
+      cp_async_wait_attn<kRing - 1>();
+      __syncwarp();
+      const uint32_t* vr = ring + (warp * kRing + (ti - tile0) % kRing) * 16 * kWordsPerRow;
+      uint32_t b0[NT], b1[NT];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const __half* ar = as + (nt * 8 + g8) * kStr + 16 * ti + 2 * tig;
+        b0[nt] = *reinterpret_cast<const uint32_t*>(ar);
+        b1[nt] = *reinterpret_cast<const uint32_t*>(ar + 8);
+      }
+      const uint4* ra = reinterpret_cast<const uint4*>(vr + (2 * tig) * kWordsPerRow);
+      const uint4* rb = reinterpret_cast<const uint4*>(vr + (2 * tig + 1) * kWordsPerRow);
+      const uint4* rc = reinterpret_cast<const uint4*>(vr + (2 * tig + 8) * kWordsPerRow);
+      const uint4* rd = reinterpret_cast<const uint4*>(vr + (2 * tig + 9) * kWordsPerRow);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const uint4 A4 = ra[half], B4 = rb[half], C4 = rc[half], D4 = rd[half];
+        const uint32_t wa[4] = {A4.x, A4.y, A4.z, A4.w}, wb[4] = {B4.x, B4.y, B4.z, B4.w};
+        const uint32_t wc[4] = {C4.x, C4.y, C4.z, C4.w}, wd[4] = {D4.x, D4.y, D4.z, D4.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int w = half * 4 + j;  // dims 16 w .. 16 w + 15
+          const uint32_t xa = wa[j] >> (2 * g8), xb = wb[j] >> (2 * g8);
+          const uint32_t xc = wc[j] >> (2 * g8), xd = wd[j] >> (2 * g8);
+          const uint32_t a0 = (__byte_perm(xa, xb, 0x5410) & 0x00030003u) | 0x64006400u;  // dim g8
+          const uint32_t a1 = (__byte_perm(xa, xb, 0x7632) & 0x00030003u) | 0x64006400u;  // dim g8 + 8
+          const uint32_t a2 = (__byte_perm(xc, xd, 0x5410) & 0x00030003u) | 0x64006400u;
+          const uint32_t a3 = (__byte_perm(xc, xd, 0x7632) & 0x00030003u) | 0x64006400u;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_f16f32(acc[nt][w], a0, a1, a2, a3, b0[nt], b1[nt]);
+        }
+      }
+      __syncwarp();
+    }
+    cp_async_wait_attn<0>();
+
+    // 4. refined tokens: alpha (c_f - 1.5), lane = dims 4 lane .. 4 lane + 3
+    const int nu = ucount;
+    for (int u = warp; u < nu; u += kOW) {
+      const int i = ulist[u];
+      const uint32_t wf = v_ref[(rowg + c0 + i) * kWordsPerRow + (lane >> 2)] >> ((lane & 3) * 8);
 #pragma unroll
       for (int h = 0; h < GRP; ++h) {
-        const float ah = __shfl_sync(0xffffffffu, alpha[h], src);
+        const float al = __half2float(as[h * kStr + i]) + __half2float(as[(GRP + h) * kStr + i]);
 #pragma unroll
         for (int dd = 0; dd < 4; ++dd)
-          uo[h][dd] = fmaf(ah, static_cast<float>((wf >> (2 * dd)) & 3u) - 1.5f, uo[h][dd]);
+          uo[h][dd] = fmaf(al, static_cast<float>((wf >> (2 * dd)) & 3u) - 1.5f, uo[h][dd]);
       }
     }
-    __syncwarp();
-    // A: weights (rows) x tokens; B: tokens x dims, built per token pair
-    const uint32_t* arow0 = reinterpret_cast<const uint32_t*>(&a16[warp][g8][0]);
-    const uint32_t* arow1 = reinterpret_cast<const uint32_t*>(&a16[warp][g8 + 8][0]);
-    const uint32_t a0 = arow0[tig], a2 = arow0[tig + 4];
-    const uint32_t a1 = arow1[tig], a3 = arow1[tig + 4];
-    const uint4* ra = reinterpret_cast<const uint4*>(&vrow[warp][st][2 * tig][0]);
-    const uint4* rb = reinterpret_cast<const uint4*>(&vrow[warp][st][2 * tig + 1][0]);
-    const uint4* rc = reinterpret_cast<const uint4*>(&vrow[warp][st][2 * tig + 8][0]);
-    const uint4* rd = reinterpret_cast<const uint4*>(&vrow[warp][st][2 * tig + 9][0]);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const uint4 A4 = ra[half], B4 = rb[half], C4 = rc[half], D4 = rd[half];
-      const uint32_t wa[4] = {A4.x, A4.y, A4.z, A4.w}, wb[4] = {B4.x, B4.y, B4.z, B4.w};
-      const uint32_t wc[4] = {C4.x, C4.y, C4.z, C4.w}, wd[4] = {D4.x, D4.y, D4.z, D4.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int w = half * 4 + j;
-        const uint32_t xa = wa[j] >> (2 * g8), xb = wb[j] >> (2 * g8);
-        const uint32_t xc = wc[j] >> (2 * g8), xd = wd[j] >> (2 * g8);
-        const uint32_t b0lo = (__byte_perm(xa, xb, 0x5410) & 0x00030003u) | 0x64006400u;
-        const uint32_t b0hi = (__byte_perm(xa, xb, 0x7632) & 0x00030003u) | 0x64006400u;
-        const uint32_t b1lo = (__byte_perm(xc, xd, 0x5410) & 0x00030003u) | 0x64006400u;
-        const uint32_t b1hi = (__byte_perm(xc, xd, 0x7632) & 0x00030003u) | 0x64006400u;
-        mma_f16f32(acc[2 * w], a0, a1, a2, a3, b0lo, b1lo);
-        mma_f16f32(acc[2 * w + 1], a0, a1, a2, a3, b0hi, b1hi);
-      }
-    }
-    __syncwarp();
+    __syncthreads();  // weights and the list are rewritten by the next sub-chunk
   }
-  cp_async_wait_attn<0>();
-  // this warp's o: rows (heads hi / lo) -> wo[warp][head][dim]
-  __syncwarp();
+
+  // high + remainder columns and the refined corrections into wo[head][dim]
+  // (in units of the code part: uo enters divided by 2^b_f = 4)
 #pragma unroll
-  for (int nt = 0; nt < 16; ++nt)
+  for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int r = (c < 2) ? g8 : g8 + 8;
-      const int hh = r < GRP ? r : (r < 2 * GRP ? r - GRP : -1);
-      // resident value s (2^b_f c_r + m_f - z): the code part carries 2^b_f = 4
-      if (hh >= 0) atomicAdd(&wo[warp][hh][8 * nt + 2 * tig + (c & 1)], 4.0f * acc[nt][c]);
-    }
-  __syncwarp();
+    for (int w = 0; w < 8; ++w)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int hh = colh[nt][c & 1];
+        if (hh >= 0) atomicAdd(&wo[hh * D + 16 * w + g8 + 8 * (c >> 1)], acc[nt][w][c]);
+      }
+#pragma unroll
+  for (int h = 0; h < GRP; ++h)
+#pragma unroll
+    for (int dd = 0; dd < 4; ++dd) atomicAdd(&wo[h * D + 4 * lane + dd], 0.25f * uo[h][dd]);
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
-    const float lt = warp_sum(lsum[h]);
-    const float ct = warp_sum(csum[h]);
-    const float at = warp_sum(asum[h]);
-    if (lane == 0) { wm[warp][h] = m[h]; wl[warp][h] = lt; }
-#pragma unroll
-    for (int dd = 0; dd < 4; ++dd) wo[warp][h][4 * lane + dd] += uo[h][dd] + ct - 4.0f * 1024.0f * at;
+    const float l = warp_sum(lsum[h]), cs = warp_sum(csum[h]), a = warp_sum(asum[h]);
+    if (lane == 0) {
+      red2[warp][h] = l;
+      red2[warp][GRP + h] = cs;
+      red2[warp][2 * GRP + h] = a;
+    }
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < GRP * (D + 2); e += blockDim.x) {
+  float* pg = part + static_cast<size_t>(g) * GRP * splits * (D + 2);
+  for (int e = tid; e < GRP * (D + 2); e += kOutThreads) {
     const int h = e / (D + 2), j = e % (D + 2);
-    float M = -INFINITY;
-    for (int w = 0; w < kOutWarps; ++w) M = fmaxf(M, wm[w][h]);
-    float accv = 0.0f;
+    float v;
     if (j == 0) {
-      accv = M;
+      v = Msh[h];
     } else {
-      for (int w = 0; w < kOutWarps; ++w) {
-        if (wm[w][h] == -INFINITY) continue;
-        const float fct = __expf(wm[w][h] - M);
-        accv += fct * (j == 1 ? wl[w][h] : wo[w][h][j - 2]);
+      float L = 0.0f, Cs = 0.0f, A = 0.0f;
+      for (int w = 0; w < kOW; ++w) {
+        L += red2[w][h];
+        Cs += red2[w][GRP + h];
+        A += red2[w][2 * GRP + h];
       }
+      // resident value s (2^b_f c + m_f - z): code part 4 (acc - 1024 A), offset part Cs
+      v = j == 1 ? L : fmaf(4.0f, wo[h * D + j - 2], fmaf(-4096.0f, A, Cs));
     }
-    part[((static_cast<size_t>(g) * GRP + h) * splits + split) * (D + 2) + j] = accv;
+    pg[(static_cast<size_t>(h) * splits + split) * (D + 2) + j] = v;
   }
+
+  // the last CTA of the group to finish merges the splits
   __shared__ int last;
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(done + g, 1) == splits - 1;
+  if (tid == 0) last = atomicAdd(done + g, 1) == splits - 1;
   __syncthreads();
   if (!last) return;
   __threadfence();
-  // merge: split maxima -> per-split factors -> per (head, dim) sums whose
-  // loads are independent of one another
-  // the per-warp output tiles are dead once the partials are written: reuse
-  // them for the per-split factors (GRP * kMaxSplits <= kOutWarps * GRP * D)
-  static_assert(kMaxSplits <= 4 * D, "merge factors must fit in the output tiles");
-  float (*fct)[kMaxSplits] = reinterpret_cast<float (*)[kMaxSplits]>(&wo[0][0][0]);
+  float (*fct)[kMaxSplits] = reinterpret_cast<float (*)[kMaxSplits]>(smem);  // the weight tile is dead
   __shared__ float Lh[GRP];
-  const float* pg = part + static_cast<size_t>(g) * GRP * splits * (D + 2);
-  for (int e = threadIdx.x; e < GRP * splits; e += blockDim.x) fct[e / splits][e % splits] = __ldcg(pg + e * (D + 2));
+  for (int e = tid; e < GRP * splits; e += kOutThreads) fct[e / splits][e % splits] = __ldcg(pg + e * (D + 2));
   __syncthreads();
-  for (int h = warp; h < GRP; h += kOutWarps) {
-    float M = -INFINITY;
-    for (int sp = lane; sp < splits; sp += 32) M = fmaxf(M, fct[h][sp]);
-    M = warp_max(M);
+  for (int h = warp; h < GRP; h += kOW) {
+    float Mx = -INFINITY;
+    for (int sp = lane; sp < splits; sp += 32) Mx = fmaxf(Mx, fct[h][sp]);
+    Mx = warp_max(Mx);
     float Ls = 0.0f;
     for (int sp = lane; sp < splits; sp += 32) {
       const float ms = fct[h][sp];
-      const float f = ms == -INFINITY ? 0.0f : __expf(ms - M);
+      const float f = ms == -INFINITY ? 0.0f : __expf(ms - Mx);
       Ls = fmaf(f, __ldcg(pg + (h * splits + sp) * (D + 2) + 1), Ls);
       fct[h][sp] = f;
     }
@@ -936,7 +1195,7 @@ attn_out_mma_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restri
     if (lane == 0) Lh[h] = Ls;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < GRP * D; e += blockDim.x) {
+  for (int e = tid; e < GRP * D; e += kOutThreads) {
     const int h = e / D, d = e % D;
     const float* ph = pg + static_cast<size_t>(h) * splits * (D + 2) + 2 + d;
     float O0 = 0.0f, O1 = 0.0f, O2 = 0.0f, O3 = 0.0f;
@@ -989,9 +1248,15 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
   if (st != SF_OK) return st;
   const int cap = grp * k;  // row length of sel_out
   if (k > 0 && k < T) {
-    attn_select_kernel<GRP><<<Hq, kSelThreads, 0, s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, k, score, smax,
-                                                       cand, cand2, kap, sel_head, status);
-    st = sf::check_launch("attn_select_kernel");
+    if (T <= kRegKeys * kSelThreads) {
+      attn_select_reg_kernel<GRP><<<Hq, kSelThreads, 0, s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, k, score,
+                                                             smax, cand2, kap, sel_head, status);
+      st = sf::check_launch("attn_select_reg_kernel");
+    } else {
+      attn_select_kernel<GRP><<<Hq, kSelThreads, 0, s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, k, score, smax,
+                                                         cand, cand2, kap, sel_head, status);
+      st = sf::check_launch("attn_select_kernel");
+    }
     if (st != SF_OK) return st;
     const size_t smem = sizeof(uint32_t) * L.words_t;
     SF_CHECK_CUDA(cudaFuncSetAttribute(attn_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1015,10 +1280,12 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
     if (st != SF_OK) return st;
   }
   dim3 gb(L.splits, Hkv);
-  attn_out_mma_kernel<GRP><<<gb, out_warps<GRP>() * 32, 0, s>>>(kv->v_res, kv->v_ref, kv->v_scale, kv->v_zero, T,
-                                                                L.tps, L.words_t, L.splits, score, umask, part,
-                                                                done, out);
-  return sf::check_launch("attn_out_mma_kernel");
+  SF_CHECK_CUDA(cudaFuncSetAttribute(attn_out_kernel<GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(OutCfg<GRP>::smem)));
+  attn_out_kernel<GRP><<<gb, kOutThreads, OutCfg<GRP>::smem, s>>>(kv->v_res, kv->v_ref, kv->v_scale, kv->v_zero, T,
+                                                                 L.tps, L.words_t, L.splits, score, umask, part,
+                                                                 done, out);
+  return sf::check_launch("attn_out_kernel");
 }
 
 }  // namespace

@@ -270,8 +270,11 @@ def _kv(sf, Hkv, T, d, seed, n_out=4):
 
 
 @pytest.mark.parametrize("Hq,Hkv,T,pct", [(8, 2, 1000, 1), (32, 8, 4099, 1), (4, 4, 77, 10), (16, 2, 33, 100),
-                                          (8, 1, 512, 0)])
+                                          (8, 1, 512, 0), (8, 2, 8192, 30), (8, 2, 40961, 1), (4, 1, 32768, 2)])
 def test_attn_small(sf, Hq, Hkv, T, pct):
+    """Covers both selection kernels (scores held in registers up to T = 32768,
+    streamed beyond), the pairwise ranking of few candidates and the radix
+    ranking of more than 1024 (30% of 8192)."""
     d = 128
     kv, ok, ov = _kv(sf, Hkv, T, d, 3000 + T)
     qb = gen_query(4000 + T, Hq, d)
