@@ -489,7 +489,7 @@ def run_sf(args, rank, world, local_rank, dist):
         n_launch = len(GEMV_LAUNCHES) * args.layers
         t_launch = ms_g / reps / n_launch * 1e-3
         achieved = gemv_step_bytes / n_launch / t_launch / 1e9
-        roofline = {"bound": "hbm", "kernel": "gemv_b1_act_kernel", "achieved": achieved, "peak": hbm_peak,
+        roofline = {"bound": "hbm", "kernel": "gemv_mma_kernel", "achieved": achieved, "peak": hbm_peak,
                     "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": None,
                     "peak_source": peak_src, "launch_us": t_launch * 1e6,
                     "bytes_per_launch": gemv_step_bytes / n_launch}

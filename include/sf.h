@@ -240,21 +240,21 @@ sf_status sf_gemv_refine(const sf_qweight* W, const uint16_t* x, int B, const in
 
 /* ---- batch-1 fast path: prepared activations, several matrices per launch */
 
-/* Bytes of the prepared form of one activation row of K channels
- * (K/32 slabs of 128 bytes). */
+/* Bytes of the prepared form of one activation row of K channels (K/256
+ * slices of 2112 bytes); 0 when K is not a positive multiple of 256. */
 size_t sf_act_bytes(int K);
 
 /*
  * sf_select_topk_act -- sf_select_topk for one row (B = 1) that also writes
  * the row's prepared form to act (device, sf_act_bytes(K) bytes, 16-byte
- * aligned).  Per 32-channel slab it holds the activations as exact 24-bit
- * fixed point relative to the slab's largest exponent (split into byte
- * planes for integer dot products), their sum, the scale back to real
- * values, which of the slab's channels are selected and how many selected
- * channels precede the slab.  The fixed-point scale is shared by each block
- * of 128 channels (4 slabs), and the block's activation sum is stored too.
- * Same selection rule and outputs as sf_select_topk.  K must be a multiple
- * of 32 up to 32768.
+ * aligned, owned by the caller).  Per 128-channel group the activations
+ * become fixed point relative to the group's largest exponent,
+ * X = rint(x 2^(22-e)), stored as signed 8-bit digits in the register order
+ * of the tensor-core GEMV's operand fragments, with the group's scale 2^(e-22)
+ * and sum.  Per 256-channel slice it also stores which channels are
+ * selected and how many selected channels precede the slice.  Same selection
+ * rule and outputs as sf_select_topk.  K must be a multiple of 256 up to
+ * 32768.  The layout is internal to the library.
  */
 sf_status sf_select_topk_act(const uint16_t* x, int K, int k, int32_t* idx_out, int32_t* n_out,
                              void* act, sf_stream_t stream);
@@ -262,7 +262,8 @@ sf_status sf_select_topk_act(const uint16_t* x, int K, int k, int32_t* idx_out, 
 /* Several single-row selections with prepared activations in one launch
  * (one CTA per row): each job is sf_select_topk_act(x, K, k, idx_out, n_out,
  * act); act may be NULL to skip the prepared form.  1 <= count <= 8,
- * K a multiple of 32 up to 32768, x and act 16-byte aligned. */
+ * K a multiple of 32 up to 32768 (of 256 when act is given), x and act
+ * 16-byte aligned. */
 typedef struct sf_select_job {
   const uint16_t* x;
   int K, k;
@@ -273,7 +274,7 @@ typedef struct sf_select_job {
 sf_status sf_select_topk_act_many(const sf_select_job* jobs, int count, sf_stream_t stream);
 
 /* The prepared form of x[K] with no channel selected (for resident-only
- * GEMVs).  K must be a multiple of 32. */
+ * GEMVs).  K must be a multiple of 256 up to 32768. */
 sf_status sf_act_prepare(const uint16_t* x, int K, void* act, sf_stream_t stream);
 
 /* One matrix of a batch-1 GEMV launch.  The refinement source follows
@@ -292,10 +293,13 @@ typedef struct sf_gemv_job {
  * the selected channels of x_j s (q_f - m_f), as sf_gemv_refine, in one
  * launch.  act comes from sf_select_topk_act (refined) or sf_act_prepare
  * (resident only) for this x; x is the bf16 row itself (device).
- * Constraints: b_r == 2, all jobs share K, G and b_f; N % 8 == 0; K a
- * multiple of 1024 up to 8192 or of 2048 up to 16384 (the latter split in two
- * halves whose partial sums are added onto zeroed outputs, an
- * order-independent fp32 addition).
+ * Computed on the integer tensor cores (mma.m16n8k32, 2-bit codes x 8-bit
+ * activation digits) in tiles of 16 output rows.
+ * Constraints: b_r == 2, G == 128, all jobs share K, G and b_f; N % 16 == 0;
+ * K a multiple of 256 whose K/256 slices split into at most 16 warps of one
+ * or two slices, in one or two K halves (4096 and 14336 qualify; with two
+ * halves the partial sums are added onto zeroed outputs, an order-independent
+ * fp32 addition); weight arrays 16-byte aligned.  SF_EINVAL otherwise.
  * Accuracy: as sf_gemv_refine.
  */
 sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, const uint16_t* x, const void* act,

@@ -1,168 +1,170 @@
-// Prepared activations for the batch-1 integer GEMV.
+// Prepared activations for the batch-1 GEMV on the integer tensor cores.
 //
-// Per 32-channel slab s of an activation row x[K] (bf16), 32 uint32 words:
-//   [0..24)  fixed-point byte planes: word (wi*4 + k)*3 + p holds, in byte b,
-//            byte p of X[16*wi + k + 4*b] -- the order in which a 2-bit code
-//            word w_wi yields code bytes via (w_wi >> 2k) & 0x03030303;
-//   24       sum_j x_j of the slab as fp32 (from the fixed-point values);
-//   25       fscale = 2^(e - 23) as fp32 (x_j ~= X_j * fscale);
-//   26       bit j set when channel 32*s + j is in the refined selection;
-//   27       number of selected channels in slabs before s;
-//   28       sum_j x_j over the slab's 128-channel block, fp32;
-//   29..31   zero.
-// X_j = rint(x_j * 2^(23 - e)) with e the binary exponent of the largest |x|
-// in the slab's 128-channel block (max |x| in [2^(e-1), 2^e)): the four slabs
-// of a block share one scale, so their integer dot products can be added
-// before any conversion.  |X_j| < 2^23 and every bf16 within 15 binades of
-// the block maximum is represented exactly.
+// An activation row x[K] (bf16, K a multiple of 256) is cut into 256-channel
+// slices, each made of two 128-channel groups (the weight quantization group).
+// Per group the activations become exact-as-possible fixed point
+//   X_j = rint(x_j 2^(22 - e)),  e = binary exponent of the group's max |x|
+// (max |x| in [2^(e-1), 2^e), so |X_j| <= 2^22), split into balanced base-256
+// digits X = d0 + 256 d1 + 65536 d2 with every digit in [-128, 127] (|d2| <=
+// 65), the signed 8-bit B operand of mma.m16n8k32 (u8 codes x s8 digits).
+//
+// Per slice, kAct2Words uint32 words:
+//   [0, 512)   B fragments of the slice's 8 k-steps: word (m*32 + lane)*2 + r
+//              is register b_r of lane `lane` for k-step m.  Column n (= lane
+//              / 4) of the MMA is (group slot n / 4, digit plane n % 4); a
+//              k-step m belongs to slot m / 4, so only its slot's columns are
+//              nonzero (plane 3 is always zero) and the two groups of a slice
+//              accumulate into disjoint columns of one accumulator.  Byte b
+//              of b_r in lane (n, t) holds the plane's digit of channel
+//                256 s + 128 (m/4) + 16 (2t + (m%4)/2) + 4b + 2 (m%2) + r,
+//              the channel whose 2-bit code the A fragment extracts as
+//              (w >> 2j) & 0x03030303 from weight word 8 (m/4) + 2t + (m%4)/2
+//              of the row's slice (j = 2 (m%2) + r).
+//   512, 513   group 0: fscale = 2^(e - 22), gsum = fscale * sum_j X_j (fp32)
+//   514, 515   group 1: the same
+//   516        number of selected channels in slices before this one
+//   517        number of selected channels in this slice
+//   518, 519   zero
+//   [520, 528) selection mask: bit i of word w <=> channel 256 s + 32 w + i
 #pragma once
 
 #include <cstdint>
 
+#include "block_scan.cuh"
+
 namespace sfd {
 
-constexpr int kActWords = 32;
+constexpr int kAct2Words = 528;
+constexpr int kAct2Frag = 512;
+constexpr int kAct2Info = 512;
+constexpr int kAct2Mask = 520;
 
-__device__ inline void act_planes_from_floats(const float (&xf)[32], uint32_t (&pl)[24], float* xsum,
-                                              float* fscale) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(xf[j]));
-  int e = 0;
-  if (amax > 0.0f) frexpf(amax, &e);
-  int X[32];
-  int xs = 0;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    X[j] = __float2int_rn(ldexpf(xf[j], 23 - e));
-    xs += X[j];
-  }
-  *fscale = ldexpf(1.0f, e - 23);
-  *xsum = static_cast<float>(xs) * *fscale;
-#pragma unroll
-  for (int wi = 0; wi < 2; ++wi)
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-#pragma unroll
-      for (int p = 0; p < 3; ++p) {
-        uint32_t v = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-          v |= ((static_cast<uint32_t>(X[16 * wi + k + 4 * b]) >> (8 * p)) & 0xFFu) << (8 * b);
-        pl[(wi * 4 + k) * 3 + p] = v;
-      }
+// Binary exponent (frexp convention) of |bf16| given as bits; -1000 for zero.
+__device__ __forceinline__ int bf16_exponent(uint32_t b) {
+  const uint32_t E = (b >> 7) & 0xFFu;
+  const uint32_t m = (b & 0x7Fu) | (E ? 0x80u : 0u);
+  const int Ee = E ? static_cast<int>(E) : 1;
+  return m ? (32 - __clz(m)) + Ee - 134 : -1000;
 }
 
-// Binary exponent e of the largest |x| of a slab (max |x| in [2^(e-1), 2^e));
-// -1000 for an all-zero slab.
-__device__ inline int act_slab_exponent(const uint16_t* __restrict__ x32) {
-  int e = -1000;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const uint32_t b = x32[j];
-    const uint32_t E = (b >> 7) & 0xFFu;
-    const uint32_t m = (b & 0x7Fu) | (E ? 0x80u : 0u);
-    const int Ee = E ? static_cast<int>(E) : 1;
-    if (m) e = max(e, (32 - __clz(m)) + Ee - 134);
+// X = rint(x 2^(22 - e)) from the bf16 bits with integer operations only
+// (ties to even when bits are shifted out).  Valid for e >= the value's own
+// exponent; values more than 31 binades below 2^e give 0.
+__device__ __forceinline__ int bf16_fixed(uint32_t b, int e) {
+  const uint32_t E = (b >> 7) & 0xFFu;
+  const uint32_t m = (b & 0x7Fu) | (E ? 0x80u : 0u);
+  const int Ee = E ? static_cast<int>(E) : 1;
+  const int sh = Ee - 112 - e;  // x = m 2^(Ee - 134), X = m 2^(Ee - 134 + 22 - e)
+  int v;
+  if (sh >= 0) {
+    v = static_cast<int>(m << sh);
+  } else if (sh >= -9) {
+    const int r = -sh;
+    const uint32_t q = m >> r, rem = m & ((1u << r) - 1u), half = 1u << (r - 1);
+    v = static_cast<int>(q + ((rem > half || (rem == half && (q & 1u))) ? 1u : 0u));
+  } else {
+    v = 0;
   }
-  return e;
+  return (b & 0x8000u) ? -v : v;
 }
 
-// Same planes from the bf16 bit patterns with integer operations only
-// (identical values: e is the frexp exponent of the largest |x|, and
-// X_j = rint(x_j 2^(23-e)) is formed by shifting the 8-bit significand,
-// rounding half to even when bits are shifted out).
-__device__ inline void act_planes_from_bits(const uint32_t (&xb)[32], int e_block, uint32_t (&pl)[24], float* xsum,
-                                            float* fscale) {
-  // e_block: exponent shared by the block (>= every element's own exponent)
-  int e = e_block;
-  int ef[32];
-  uint32_t mant[32];
+// Writes the prepared form of a whole row with one thread block (every thread
+// calls; contains __syncthreads).  xs: the row's bf16 bits (shared or global
+// memory); flags: one byte per channel, nonzero = selected (nullptr: none);
+// eg: K / 128 ints of shared scratch (group exponents); ginfo: 2 * (K / 128)
+// floats of shared scratch (fscale, gsum per group); scan: 33 ints of shared
+// scratch.
+__device__ inline void act2_write_block(const uint16_t* xs, const uint8_t* flags, int K, int* eg, float* ginfo,
+                                        int* scan, uint32_t* __restrict__ act) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  const int ngroups = K >> 7, nslice = K >> 8;
+  // 1. per group: exponent, fixed-point values, their sum (one warp a group)
+  for (int gi = warp; gi < ngroups; gi += nw) {
+    uint32_t b[4];
+    int e = -1000;
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const uint32_t E = (xb[j] >> 7) & 0xFFu;
-    const uint32_t m = (xb[j] & 0x7Fu) | (E ? 0x80u : 0u);
-    const int Ee = E ? static_cast<int>(E) : 1;
-    mant[j] = m;
-    ef[j] = Ee;
-  }
-  if (e == -1000) e = 0;
-  int X[32];
-  int xs = 0;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const int sh = ef[j] - 111 - e;  // X = m 2^sh
-    int v;
-    if (sh >= 0) {
-      v = static_cast<int>(mant[j] << sh);
-    } else if (sh >= -9) {
-      const int r = -sh;
-      const uint32_t q = mant[j] >> r, rem = mant[j] & ((1u << r) - 1u), half = 1u << (r - 1);
-      v = static_cast<int>(q + ((rem > half || (rem == half && (q & 1u))) ? 1u : 0u));
-    } else {
-      v = 0;
+    for (int i = 0; i < 4; ++i) {
+      b[i] = xs[128 * gi + 32 * i + lane];
+      e = max(e, bf16_exponent(b[i]));
     }
-    X[j] = (xb[j] & 0x8000u) ? -v : v;
-    xs += X[j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
+    if (e == -1000) e = 0;
+    int s = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s += bf16_fixed(b[i], e);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) {
+      eg[gi] = e;
+      const float fscale = ldexpf(1.0f, e - 22);
+      ginfo[2 * gi] = fscale;
+      ginfo[2 * gi + 1] = static_cast<float>(s) * fscale;
+    }
   }
-  *fscale = ldexpf(1.0f, e - 23);
-  *xsum = static_cast<float>(xs) * *fscale;
+  __syncthreads();
+  // 2. B fragments: one task per (slice, k-step m, column tig) converts its 8
+  //    channels once and writes their three digit-plane words for b0 and b1;
+  //    the other columns' words of the k-step are zero
+  for (int task = tid; task < nslice * 32; task += blockDim.x) {
+    const int s = task >> 5, m = (task >> 2) & 7, t = task & 3;
+    const int slot = m >> 2, mm = m & 3;
+    const int ch0 = 256 * s + 128 * slot + 16 * (2 * t + (mm >> 1)) + 2 * (mm & 1);
+    const int e = eg[ch0 >> 7];
+    uint32_t* o = act + static_cast<size_t>(s) * kAct2Words + m * 64;
 #pragma unroll
-  for (int wi = 0; wi < 2; ++wi)
+    for (int r = 0; r < 2; ++r) {
+      uint32_t w0 = 0, w1 = 0, w2 = 0;
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-#pragma unroll
-      for (int p = 0; p < 3; ++p) {
-        uint32_t v = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-          v |= ((static_cast<uint32_t>(X[16 * wi + k + 4 * b]) >> (8 * p)) & 0xFFu) << (8 * b);
-        pl[(wi * 4 + k) * 3 + p] = v;
+      for (int b = 0; b < 4; ++b) {
+        const int X = bf16_fixed(xs[ch0 + 4 * b + r], e);
+        const int d0 = ((X + 128) & 255) - 128;
+        const int X1 = (X - d0) >> 8;
+        const int d1 = ((X1 + 128) & 255) - 128;
+        const int d2 = (X1 - d1) >> 8;
+        w0 |= (static_cast<uint32_t>(d0) & 0xFFu) << (8 * b);
+        w1 |= (static_cast<uint32_t>(d1) & 0xFFu) << (8 * b);
+        w2 |= (static_cast<uint32_t>(d2) & 0xFFu) << (8 * b);
       }
-}
-
-// Block helper for a warp whose lanes hold consecutive slabs (lane l = slab
-// 32*w + l, all 32 lanes calling; inactive lanes pass e = -1000 and xsum = 0):
-// the maximum exponent and the sum over each group of 4 lanes (= one block).
-__device__ __forceinline__ int act_block_exponent(int e) {
-  e = max(e, __shfl_xor_sync(0xffffffffu, e, 1));
-  e = max(e, __shfl_xor_sync(0xffffffffu, e, 2));
-  return e;
-}
-__device__ __forceinline__ float act_block_sum(float v) {
-  v += __shfl_xor_sync(0xffffffffu, v, 1);
-  v += __shfl_xor_sync(0xffffffffu, v, 2);
-  return v;
-}
-
-// Writes the 32-word prepared form of slab x32[0..32) to out, with the
-// block exponent e_block and the block sum of x (filled in by the caller
-// once known, see act_write_block_sum).
-__device__ inline float act_write_slab(const uint16_t* __restrict__ x32, uint32_t* __restrict__ out, uint32_t selmask,
-                                       int selprefix, int e_block) {
-  uint32_t xb[32];
+      // lane (n, t) = 4 n + t; column n = 4 slot + plane
+      o[(4 * (4 * slot + 0) + t) * 2 + r] = w0;
+      o[(4 * (4 * slot + 1) + t) * 2 + r] = w1;
+      o[(4 * (4 * slot + 2) + t) * 2 + r] = w2;
+      o[(4 * (4 * slot + 3) + t) * 2 + r] = 0u;
+      o[(4 * (4 * (1 - slot) + 0) + t) * 2 + r] = 0u;
+      o[(4 * (4 * (1 - slot) + 1) + t) * 2 + r] = 0u;
+      o[(4 * (4 * (1 - slot) + 2) + t) * 2 + r] = 0u;
+      o[(4 * (4 * (1 - slot) + 3) + t) * 2 + r] = 0u;
+    }
+  }
+  // 3. group scalars, selection masks and counts (one thread a slice)
+  int carry = 0;  // selected channels in earlier rounds of slices
+  for (int base = 0; base < nslice; base += blockDim.x) {
+    const int s = base + tid;
+    const bool active = s < nslice;
+    uint32_t mw[8];
+    int c = 0;
 #pragma unroll
-  for (int j = 0; j < 32; ++j) xb[j] = x32[j];
-  uint32_t pl[24];
-  float xsum, fscale;
-  act_planes_from_bits(xb, e_block, pl, &xsum, &fscale);
-  uint4* o = reinterpret_cast<uint4*>(out);
-#pragma unroll
-  for (int q = 0; q < 6; ++q) o[q] = make_uint4(pl[4 * q], pl[4 * q + 1], pl[4 * q + 2], pl[4 * q + 3]);
-  o[6] = make_uint4(__float_as_uint(xsum), __float_as_uint(fscale), selmask, static_cast<uint32_t>(selprefix));
-  return xsum;
-}
-
-// The whole prepared form of one slab per thread (thread t = slab t of the
-// warp-aligned range; every lane of the warp calls, `active` false beyond K):
-// block exponent and block sum over groups of 4 lanes.
-__device__ inline void act_write_slab_in_block(const uint16_t* __restrict__ x32, uint32_t* __restrict__ out,
-                                               bool active, uint32_t selmask, int selprefix) {
-  const int e = active ? act_slab_exponent(x32) : -1000;
-  const int eb = act_block_exponent(e);
-  const float xs = active ? act_write_slab(x32, out, selmask, selprefix, eb) : 0.0f;
-  const float bs = act_block_sum(xs);
-  if (active) reinterpret_cast<uint4*>(out)[7] = make_uint4(__float_as_uint(bs), 0u, 0u, 0u);
+    for (int w = 0; w < 8; ++w) {
+      uint32_t v = 0;
+      if (active && flags != nullptr)
+        for (int i = 0; i < 32; ++i) v |= static_cast<uint32_t>(flags[256 * s + 32 * w + i] != 0) << i;
+      mw[w] = v;
+      c += __popc(v);
+    }
+    int total;
+    const int pre = carry + block_exclusive_scan(c, scan, &total);
+    carry += total;
+    if (active) {
+      uint32_t* o = act + static_cast<size_t>(s) * kAct2Words;
+      reinterpret_cast<uint4*>(o + kAct2Info)[0] =
+          make_uint4(__float_as_uint(ginfo[4 * s]), __float_as_uint(ginfo[4 * s + 1]),
+                     __float_as_uint(ginfo[4 * s + 2]), __float_as_uint(ginfo[4 * s + 3]));
+      reinterpret_cast<uint4*>(o + kAct2Info)[1] = make_uint4(static_cast<uint32_t>(pre), static_cast<uint32_t>(c), 0u, 0u);
+      reinterpret_cast<uint4*>(o + kAct2Mask)[0] = make_uint4(mw[0], mw[1], mw[2], mw[3]);
+      reinterpret_cast<uint4*>(o + kAct2Mask)[1] = make_uint4(mw[4], mw[5], mw[6], mw[7]);
+    }
+  }
 }
 
 }  // namespace sfd

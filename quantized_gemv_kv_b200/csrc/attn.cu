@@ -887,6 +887,8 @@ constexpr int kSub = 2048;         // tokens per sub-chunk
 constexpr int kOutThreads = 256;
 constexpr int kOW = kOutThreads / 32;
 constexpr int kRing = 4;           // cp.async stages per warp
+constexpr int kUCap = 512;         // refined rows per sub-chunk staged in shared memory
+constexpr int kPerThr = kSub / kOutThreads;  // tokens of a sub-chunk per thread in the weight pass
 
 template <int GRP>
 struct OutCfg {
@@ -897,7 +899,8 @@ struct OutCfg {
   static constexpr size_t ring_bytes = static_cast<size_t>(kOW) * kRing * 16 * kWordsPerRow * 4;
   static constexpr size_t wo_bytes = static_cast<size_t>(GRP) * D * 4;
   static constexpr size_t ulist_bytes = static_cast<size_t>(kSub) * 4;
-  static constexpr size_t smem = alpha_bytes + ring_bytes + wo_bytes + ulist_bytes;
+  static constexpr size_t vref_bytes = static_cast<size_t>(kUCap) * kWordsPerRow * 4;
+  static constexpr size_t smem = alpha_bytes + ring_bytes + wo_bytes + ulist_bytes + vref_bytes;
   static_assert(alpha_bytes >= static_cast<size_t>(GRP) * kMaxSplits * 4, "merge factors must fit the weight tile");
 };
 
@@ -914,6 +917,8 @@ attn_out_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__
   uint32_t* ring = reinterpret_cast<uint32_t*>(smem + C::alpha_bytes);               // [kOW][kRing][16][8]
   float* wo = reinterpret_cast<float*>(smem + C::alpha_bytes + C::ring_bytes);       // [GRP][D]
   int* ulist = reinterpret_cast<int*>(smem + C::alpha_bytes + C::ring_bytes + C::wo_bytes);  // [kSub]
+  uint32_t* vrs = reinterpret_cast<uint32_t*>(smem + C::alpha_bytes + C::ring_bytes + C::wo_bytes +
+                                              C::ulist_bytes);  // [kUCap][8] refinement rows of listed tokens
   __shared__ float red[kOW][GRP];
   __shared__ float red2[kOW][3 * GRP];
   __shared__ float Msh[GRP], Fsh[GRP];
@@ -970,14 +975,28 @@ attn_out_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__
       cp_async_commit_attn();
     }
 
-    // 1. the sub-chunk's maximum score per head
+    // 1. the sub-chunk's maximum score per head; this thread's tokens'
+    //    scale, zero and union bit are fetched meanwhile
+    uint32_t svz[kPerThr];
+    uint32_t ubits = 0;
     {
       float mx[GRP];
 #pragma unroll
       for (int h = 0; h < GRP; ++h) mx[h] = -INFINITY;
-      for (int i = tid; i < n; i += kOutThreads)
 #pragma unroll
-        for (int h = 0; h < GRP; ++h) mx[h] = fmaxf(mx[h], score[(static_cast<size_t>(g) * GRP + h) * T + c0 + i]);
+      for (int j = 0; j < kPerThr; ++j) {
+        const int i = tid + j * kOutThreads;
+        svz[j] = 0;
+        if (i < n) {
+          const size_t row = rowg + c0 + i;
+          svz[j] = static_cast<uint32_t>(v_scale[row]) | (static_cast<uint32_t>(v_zero[row]) << 16);
+          const int t = c0 + i;
+          ubits |= ((umask[static_cast<size_t>(g) * words_t + (t >> 5)] >> (t & 31)) & 1u) << j;
+#pragma unroll
+          for (int h = 0; h < GRP; ++h)
+            mx[h] = fmaxf(mx[h], score[(static_cast<size_t>(g) * GRP + h) * T + c0 + i]);
+        }
+      }
 #pragma unroll
       for (int h = 0; h < GRP; ++h) {
         const float m = warp_max(mx[h]);
@@ -1030,15 +1049,16 @@ attn_out_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__
     // 2. weights into shared memory (zero past the end of the last tile),
     //    sums, and the list of refined tokens
     const unsigned lt = (1u << lane) - 1u;
-    for (int base = 0; base < 16 * ntile; base += kOutThreads) {
-      const int i = base + tid;
+#pragma unroll
+    for (int j = 0; j < kPerThr; ++j) {
+      const int i = tid + j * kOutThreads;
+      if (j * kOutThreads >= 16 * ntile) break;  // uniform over the block
       const bool valid = i < n;
       bool inU = false;
       if (i < 16 * ntile) {
         if (valid) {
-          const size_t row = rowg + c0 + i;
-          const float sv = sfd::half_bits_to_float(v_scale[row]);
-          const float zv = sfd::half_bits_to_float(v_zero[row]);
+          const float sv = sfd::half_bits_to_float(svz[j] & 0xFFFFu);
+          const float zv = sfd::half_bits_to_float(svz[j] >> 16);
 #pragma unroll
           for (int h = 0; h < GRP; ++h) {
             const float p = __expf(score[(static_cast<size_t>(g) * GRP + h) * T + c0 + i] - M[h]);
@@ -1051,8 +1071,7 @@ attn_out_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__
             csum[h] = fmaf(al, 1.5f - zv, csum[h]);
             asum[h] += __half2float(ahi) + __half2float(alo);
           }
-          const int t = c0 + i;
-          inU = (umask[static_cast<size_t>(g) * words_t + (t >> 5)] >> (t & 31)) & 1u;
+          inU = (ubits >> j) & 1u;
         } else {
 #pragma unroll
           for (int h = 0; h < 2 * GRP; ++h) as[h * kStr + i] = __float2half_rn(0.0f);
@@ -1067,6 +1086,14 @@ attn_out_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__
       }
     }
     __syncthreads();
+    // refinement rows of the listed tokens, staged behind the MMA loop
+    const int nu = ucount;
+    for (int u = tid; u < min(nu, kUCap); u += kOutThreads) {
+      const uint32_t* src = v_ref + (rowg + c0 + ulist[u]) * kWordsPerRow;
+      cp_async16_attn(vrs + u * kWordsPerRow, src);
+      cp_async16_attn(vrs + u * kWordsPerRow + 4, src + 4);
+    }
+    cp_async_commit_attn();
 
     // 3. MMAs over this warp's tiles
     for (int ti = tile0; ti < tile1; ++ti) {
@@ -1107,12 +1134,14 @@ attn_out_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__
       __syncwarp();
     }
     cp_async_wait_attn<0>();
+    __syncthreads();  // the staged refinement rows come from every thread
 
     // 4. refined tokens: alpha (c_f - 1.5), lane = dims 4 lane .. 4 lane + 3
-    const int nu = ucount;
     for (int u = warp; u < nu; u += kOW) {
       const int i = ulist[u];
-      const uint32_t wf = v_ref[(rowg + c0 + i) * kWordsPerRow + (lane >> 2)] >> ((lane & 3) * 8);
+      const uint32_t wrow = u < kUCap ? vrs[u * kWordsPerRow + (lane >> 2)]
+                                      : v_ref[(rowg + c0 + i) * kWordsPerRow + (lane >> 2)];
+      const uint32_t wf = wrow >> ((lane & 3) * 8);
 #pragma unroll
       for (int h = 0; h < GRP; ++h) {
         const float al = __half2float(as[h * kStr + i]) + __half2float(as[(GRP + h) * kStr + i]);

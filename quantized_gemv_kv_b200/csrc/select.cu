@@ -17,6 +17,8 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kMaxRows = 16;
+constexpr int kActMaxK = 32768;
+constexpr int kActMaxGroups = kActMaxK / 128;
 
 // Histogram increment with the lanes of a warp that hit the same bin merged
 // into one atomic (keys cluster in few bins, so plain atomics serialise).
@@ -42,6 +44,8 @@ select_topk_kernel(const uint16_t* __restrict__ x, int B, int K, int k, int32_t*
   __shared__ RowState st[kMaxRows];
   __shared__ int scan_scratch[33];
   __shared__ int bad;
+  __shared__ int eg[kActMaxGroups];
+  __shared__ float ginfo[2 * kActMaxGroups];
 
   const int tid = threadIdx.x;
   int rb = 1;
@@ -179,29 +183,20 @@ select_topk_kernel(const uint16_t* __restrict__ x, int B, int K, int k, int32_t*
     if (tid == 0) *n_out = bad ? -1 : total;
   }
 
-  // prepared activations (batch 1): per 32-channel slab the fixed-point
-  // planes, plus which of its channels are selected and how many selected
-  // channels precede it (= the selected channel's position in idx_out)
-  if (act != nullptr) {  // K <= 32768: at most one slab per thread
-    const int nslab = K >> 5;
-    const int sl = tid;
-    const bool active = sl < nslab;
-    uint32_t m = 0;
-    if (active)
-      for (int j = 0; j < 32; ++j) m |= static_cast<uint32_t>(flags[32 * sl + j] != 0) << j;
-    int total;
-    const int pre = sfd::block_exclusive_scan(active ? __popc(m) : 0, scan_scratch, &total);
-    sfd::act_write_slab_in_block(x + 32 * (active ? sl : 0), act + static_cast<size_t>(sfd::kActWords) * sl, active,
-                                 m, pre);
+  // prepared activations (batch 1): digit planes as MMA fragments, group
+  // scalars, the selection mask and counts (act.cuh)
+  if (act != nullptr) {
+    __syncthreads();
+    sfd::act2_write_block(x, flags, K, eg, ginfo, scan_scratch, act);
   }
 }
 
-__global__ void __launch_bounds__(256)
-act_prepare_kernel(const uint16_t* __restrict__ x, int nslab, uint32_t* __restrict__ act) {
-  const int sl = blockIdx.x * blockDim.x + threadIdx.x;
-  const bool active = sl < nslab;
-  sfd::act_write_slab_in_block(x + 32 * (active ? sl : 0), act + static_cast<size_t>(sfd::kActWords) * sl, active, 0u,
-                               0);
+__global__ void __launch_bounds__(kThreads)
+act_prepare_kernel(const uint16_t* __restrict__ x, int K, uint32_t* __restrict__ act) {
+  __shared__ int eg[kActMaxGroups];
+  __shared__ float ginfo[2 * kActMaxGroups];
+  __shared__ int scan_scratch[33];
+  sfd::act2_write_block(x, nullptr, K, eg, ginfo, scan_scratch, act);
 }
 
 // ---- several single-row selections in one launch (one CTA each) -------------
@@ -229,6 +224,8 @@ select_act_many_kernel(const __grid_constant__ SelManyArgs a) {
   __shared__ int hist1[256], hist2[128];
   __shared__ int scan_scratch[33];
   __shared__ int b1_sh, k1_sh, tau_sh, r_sh, bad;
+  __shared__ int eg[kActMaxGroups];
+  __shared__ float ginfo[2 * kActMaxGroups];
   {
     const uint4* src = reinterpret_cast<const uint4*>(J.x);
     uint4* dst = reinterpret_cast<uint4*>(xs);
@@ -326,20 +323,8 @@ select_act_many_kernel(const __grid_constant__ SelManyArgs a) {
     if (tid == 0) *J.n = bad ? -1 : total;
   }
   __syncthreads();
-  if (J.act != nullptr) {  // K <= 32768: at most one slab per thread
-    const int nslab = K >> 5;
-    const int sl = tid;
-    const bool active = sl < nslab;
-    uint32_t m = 0;
-    if (active)
-      for (int j = 0; j < 32; ++j) m |= static_cast<uint32_t>(flags[32 * sl + j] != 0) << j;
-    int total;
-    const int pre = sfd::block_exclusive_scan(active ? __popc(m) : 0, scan_scratch, &total);
-    sfd::act_write_slab_in_block(xs + 32 * (active ? sl : 0), J.act + static_cast<size_t>(sfd::kActWords) * sl,
-                                 active, m, pre);
-  }
+  if (J.act != nullptr) sfd::act2_write_block(xs, flags, K, eg, ginfo, scan_scratch, J.act);
 }
-
 }  // namespace
 
 extern "C" sf_status sf_select_topk(const uint16_t* x, int B, int K, int k, int32_t* idx_out, int32_t* n_out,
@@ -355,13 +340,14 @@ extern "C" sf_status sf_select_topk(const uint16_t* x, int B, int K, int k, int3
 }
 
 extern "C" size_t sf_act_bytes(int K) {
-  return K > 0 ? static_cast<size_t>(K / 32) * sfd::kActWords * sizeof(uint32_t) : 0;
+  return (K > 0 && K % 256 == 0) ? static_cast<size_t>(K / 256) * sfd::kAct2Words * sizeof(uint32_t) : 0;
 }
 
 extern "C" sf_status sf_select_topk_act(const uint16_t* x, int K, int k, int32_t* idx_out, int32_t* n_out, void* act,
                                         sf_stream_t stream) {
   SF_REQUIRE(x && idx_out && n_out && act, "sf_select_topk_act: null pointer");
-  SF_REQUIRE(K >= 32 && K <= 32768 && K % 32 == 0, "sf_select_topk_act: K must be a multiple of 32 in [32, 32768]");
+  SF_REQUIRE(K >= 256 && K <= kActMaxK && K % 256 == 0,
+             "sf_select_topk_act: K must be a multiple of 256 in [256, %d]", kActMaxK);
   SF_REQUIRE(k >= 0 && k <= K, "sf_select_topk_act: k must be in [0, K]");
   SF_REQUIRE(sf::aligned(act, 16), "sf_select_topk_act: act must be 16-byte aligned");
   const size_t smem = static_cast<size_t>((K + 15) & ~15) + sizeof(int) * kMaxRows * (256 + 128);
@@ -373,10 +359,10 @@ extern "C" sf_status sf_select_topk_act(const uint16_t* x, int K, int k, int32_t
 
 extern "C" sf_status sf_act_prepare(const uint16_t* x, int K, void* act, sf_stream_t stream) {
   SF_REQUIRE(x && act, "sf_act_prepare: null pointer");
-  SF_REQUIRE(K >= 32 && K % 32 == 0, "sf_act_prepare: K must be a positive multiple of 32");
+  SF_REQUIRE(K >= 256 && K <= kActMaxK && K % 256 == 0,
+             "sf_act_prepare: K must be a multiple of 256 in [256, %d]", kActMaxK);
   SF_REQUIRE(sf::aligned(act, 16), "sf_act_prepare: act must be 16-byte aligned");
-  const int nslab = K / 32;
-  act_prepare_kernel<<<(nslab + 255) / 256, 256, 0, sf::as_cuda(stream)>>>(x, nslab, static_cast<uint32_t*>(act));
+  act_prepare_kernel<<<1, kThreads, 0, sf::as_cuda(stream)>>>(x, K, static_cast<uint32_t*>(act));
   return sf::check_launch("act_prepare_kernel");
 }
 
@@ -391,6 +377,8 @@ extern "C" sf_status sf_select_topk_act_many(const sf_select_job* jobs, int coun
     SF_REQUIRE(j.K >= 32 && j.K <= 32768 && j.K % 32 == 0,
                "sf_select_topk_act_many: K must be a multiple of 32 in [32, 32768] (job %d)", i);
     SF_REQUIRE(j.k >= 0 && j.k <= j.K, "sf_select_topk_act_many: k out of range (job %d)", i);
+    SF_REQUIRE(j.act == nullptr || j.K % 256 == 0,
+               "sf_select_topk_act_many: prepared activations need K a multiple of 256 (job %d)", i);
     SF_REQUIRE(sf::aligned(j.x, 16) && (j.act == nullptr || sf::aligned(j.act, 16)),
                "sf_select_topk_act_many: x and act must be 16-byte aligned (job %d)", i);
     a.job[i] = SelJobDev{j.x, j.K, j.k, j.idx_out, j.n_out, static_cast<uint32_t*>(j.act)};

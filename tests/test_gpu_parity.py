@@ -417,24 +417,57 @@ def test_select_act_matches_select(sf, K, pct):
     torch.cuda.synchronize()
     S = oselect.select_topk(x, k)
     np.testing.assert_array_equal(idx.cpu().numpy()[: int(n.item())], S)
-    a = act.cpu().numpy().view(np.uint32).reshape(K // 32, 32)
-    sel = [32 * s + j for s in range(K // 32) for j in range(32) if (a[s, 26] >> j) & 1]
-    assert sel == S.tolist()
-    prefix = np.concatenate([[0], np.cumsum([bin(int(m)).count("1") for m in a[:, 26]])[:-1]])
-    np.testing.assert_array_equal(a[:, 27], prefix)
-    # the planes rebuild x: X_j = signed byte 2 * 2^16 + byte 1 * 2^8 + byte 0, x = X * fscale
-    xf = (x[0].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    fscale = a[:, 25].view(np.float32).astype(np.float64)
-    for s in range(0, K // 32, max(1, K // 32 // 16)):
-        for wi in range(2):
-            for kk in range(4):
-                b0, b1, b2 = (a[s, (wi * 4 + kk) * 3 + p] for p in range(3))
-                for b in range(4):
-                    top = int((b2 >> (8 * b)) & 0xFF)
-                    top = top - 256 if top >= 128 else top
-                    X = top * 65536 + int((b1 >> (8 * b)) & 0xFF) * 256 + int((b0 >> (8 * b)) & 0xFF)
-                    j = 32 * s + 16 * wi + kk + 4 * b
-                    assert abs(X * fscale[s] - xf[j]) <= fscale[s] / 2 + 1e-300
+    _check_prepared(act, x[0], S, K)
+    act0 = torch.zeros_like(act)
+    sf.act_prepare(xd, act0)
+    torch.cuda.synchronize()
+    _check_prepared(act0, x[0], [], K)
+
+
+def _check_prepared(act, x_row, S, K):
+    """The prepared activations against their documented layout: per
+    256-channel slice, MMA B fragments holding balanced base-256 digits of
+    per-group fixed point, group scale and sum, selection mask and counts."""
+    a = act.cpu().numpy().view(np.uint32).reshape(K // 256, 528)
+    mask = a[:, 520:528]
+    sel = [256 * s + 32 * w + i for s in range(K // 256) for w in range(8) for i in range(32)
+           if (int(mask[s, w]) >> i) & 1]
+    assert sel == list(S)
+    counts = np.array([sum(bin(int(m)).count("1") for m in mask[s]) for s in range(K // 256)])
+    np.testing.assert_array_equal(a[:, 517], counts)
+    np.testing.assert_array_equal(a[:, 516], np.concatenate([[0], np.cumsum(counts)[:-1]]))
+    xf = (x_row.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    for s in range(0, K // 256, max(1, K // 256 // 8)):
+        digits = np.zeros((256, 3), dtype=np.int64)
+        seen = np.zeros((256, 3), dtype=np.int64)
+        for m in range(8):
+            for lane in range(32):
+                n, t = lane >> 2, lane & 3
+                slot, mm, plane = m >> 2, m & 3, n & 3
+                for r in range(2):
+                    word = int(a[s, (m * 32 + lane) * 2 + r])
+                    if (n >> 2) != slot or plane == 3:
+                        assert word == 0
+                        continue
+                    for b in range(4):
+                        ch = 128 * slot + 16 * (2 * t + (mm >> 1)) + 4 * b + 2 * (mm & 1) + r
+                        d = (word >> (8 * b)) & 0xFF
+                        digits[ch, plane] = d - 256 if d >= 128 else d
+                        seen[ch, plane] += 1
+        assert (seen == 1).all()
+        assert np.abs(digits[:, 2]).max() <= 65
+        X = digits[:, 0] + 256 * digits[:, 1] + 65536 * digits[:, 2]
+        for grp in range(2):
+            fscale = float(a[s, 512 + 2 * grp:513 + 2 * grp].view(np.float32)[0])
+            gsum = float(a[s, 513 + 2 * grp:514 + 2 * grp].view(np.float32)[0])
+            xs = xf[256 * s + 128 * grp:256 * s + 128 * grp + 128]
+            Xg = X[128 * grp:128 * grp + 128]
+            amax = np.abs(xs).max()
+            if amax > 0:
+                e = int(np.frexp(amax)[1])
+                assert fscale == 2.0 ** (e - 22)
+            assert np.all(np.abs(Xg * fscale - xs) <= fscale / 2)
+            assert gsum == float(np.float32(float(np.float32(Xg.sum())) * fscale))
 
 
 @pytest.mark.parametrize("K,Ns,cap_pct,pct", [(4096, (4096, 1024, 1024), 10, 3), (14336, (4096,), 10, 3),
