@@ -276,7 +276,7 @@ class Model:
 
     def launches_per_step(self, refine=True):
         gemv = len(GEMV_LAUNCHES) * self.L
-        attn = 5 * self.L if (refine and 0 < self.k_tok < self.T) else 2 * self.L
+        attn = 4 * self.L if (refine and 0 < self.k_tok < self.T) else 2 * self.L
         if not refine:
             return 2 * gemv + attn
         return self.L + 2 * self.L + gemv + attn

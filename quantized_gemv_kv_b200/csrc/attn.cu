@@ -5,20 +5,24 @@
 // low-bit keys (rag-lover.com explainer, 解説).  The pass structure:
 //
 //   A  score   per (KV head, token): resident scores of the Hq/Hkv query
-//              heads of the group from the 2-bit keys, fp32, into scratch.
+//              heads of the group from the 2-bit keys, fp32, into scratch, on
+//              the integer tensor cores; also a per-head histogram of the
+//              scores (top 10 bits of the order-preserving key) and max |s|.
 //   S  select  per query head: the k largest scores, exactly.  The fast fp32
 //              scores carry a proven error bound eps; every token within
 //              2*eps of the k-th largest fast score is a candidate, and the
 //              candidates are re-scored exactly in fp64 (the key s*E with
 //              E = sum_d q_d (c_d 2^b_f + m_f - z) is exact in fp64 under a
 //              precondition on q checked here) and ranked by (key desc, token
-//              asc).  So the chosen set equals the exact definition.
-//   U  union   per KV head: union of its query heads' choices, ascending,
-//              plus a token bitmask.
-//   B  output  split over tokens: online softmax over all tokens with the
-//              refined (full-code) K and V for tokens in the union and the
-//              resident ones elsewhere -- refined tokens are computed directly,
-//              never by subtracting their resident contribution.
+//              asc).  So the chosen set equals the exact definition.  Runs as
+//              a compaction over token chunks (from the histogram's bin of
+//              the k-th score) and a finish per KV group (one cluster, one CTA
+//              per query head), which also forms the group's union (ascending
+//              list and token bitmask) and the refined scores of its tokens.
+//   B  output  split over tokens: softmax over all tokens with the refined
+//              (full-code) K and V for tokens in the union and the resident
+//              ones elsewhere -- refined tokens are computed directly, never
+//              by subtracting their resident contribution.
 //   M  merge   per KV group, by the last CTA of pass B to finish: combine the
 //              splits' (max, sum, output).
 //
@@ -26,6 +30,8 @@
 #include <algorithm>
 #include <cmath>
 #include <mutex>
+
+#include <cooperative_groups.h>
 
 #include "block_scan.cuh"
 #include "sf_internal.h"
@@ -38,9 +44,13 @@ constexpr int kMaxGrp = 8;
 constexpr int kMaxSplits = 256;
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128), rounded to fp32
 
+constexpr int kHistBins = 1024;    // per-head histogram of the fast scores' top 10 key bits
+constexpr int kChunk = 4096;       // tokens per CTA of the candidate compaction
+
 struct Layout {
-  size_t score, cand, cand2, kap, sel, umask, part, smax, status, count, total;
-  int splits, tps, words_t;
+  // from smax on, everything is cleared at the start of a call
+  size_t score, cand, cand2, kap, sel, part, smax, status, count, amax, hist, umask, total;
+  int splits, tps, words_t, nchunks;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -53,17 +63,20 @@ Layout make_layout(int Hq, int Hkv, int T, int k, int sms) {
   L.tps = tps;
   L.splits = (T + tps - 1) / tps;
   L.words_t = (T + 31) / 32;
+  L.nchunks = (T + kChunk - 1) / kChunk;
   size_t off = 0;
   L.score = off; off = up256(off + sizeof(float) * Hq * static_cast<size_t>(T));
-  L.cand = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(T));
+  L.cand = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(T) + sizeof(int32_t) * Hq * L.nchunks);
   L.cand2 = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(T));
   L.kap = off; off = up256(off + sizeof(double) * Hq * static_cast<size_t>(T));
   L.sel = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(std::max(k, 1)));
-  L.umask = off; off = up256(off + sizeof(uint32_t) * Hkv * static_cast<size_t>(L.words_t));
   L.part = off; off = up256(off + sizeof(float) * Hq * static_cast<size_t>(L.splits) * (D + 2));
   L.smax = off; off = up256(off + sizeof(float) * Hkv);
   L.status = off; off = up256(off + sizeof(int32_t) * std::max(Hkv, 4));
   L.count = off; off = up256(off + sizeof(int32_t) * Hkv);
+  L.amax = off; off = up256(off + sizeof(uint32_t) * Hq);
+  L.hist = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(kHistBins));
+  L.umask = off; off = up256(off + sizeof(uint32_t) * Hkv * static_cast<size_t>(L.words_t));
   L.total = off;
   return L;
 }
@@ -95,10 +108,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 __device__ __forceinline__ void cp_async16_attn(void* smem, const void* gmem) {
   const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(gmem));
-}
-__device__ __forceinline__ void cp_async4_attn(void* smem, const void* gmem) {
-  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(sa), "l"(gmem));
 }
 __device__ __forceinline__ void cp_async_commit_attn() { asm volatile("cp.async.commit_group;\n" ::); }
 template <int N>
@@ -147,9 +156,14 @@ template <int GRP>
 __global__ void __launch_bounds__(128)
 attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
                       const uint16_t* __restrict__ k_scale, const uint16_t* __restrict__ k_zero, int T,
-                      float* __restrict__ score, float* __restrict__ smax) {
+                      float* __restrict__ score, float* __restrict__ smax, int32_t* __restrict__ hist,
+                      uint32_t* __restrict__ amaxu) {
   __shared__ int qx[GRP][D];
   __shared__ float qsc[GRP], qsm[GRP];
+  // per-head histogram of this CTA's scores over the top 10 bits of the
+  // order-preserving key (pass S starts from the cluster of all CTAs' counts)
+  __shared__ int hs[GRP][kHistBins];
+  for (int i = threadIdx.x; i < GRP * kHistBins; i += blockDim.x) (&hs[0][0])[i] = 0;
   const int g = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // fixed-point query heads (warp h builds head h, 4 dims per lane)
@@ -193,6 +207,7 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
       }
   const int ntiles = (T + 15) / 16;
   float smx = 0.0f;
+  float am0 = 0.0f, am1 = 0.0f;  // max |score| of this lane's heads 2 tig, 2 tig + 1
   // one tile = rows ta, tb of this thread: 2 x 32 bytes of codes plus the
   // rows' scale and zero; the next tile is fetched while this one is scored
   struct TileRegs {
@@ -254,17 +269,35 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
         const float P = (static_cast<float>(d2[i]) * 65536.0f + static_cast<float>(d1[i]) * 256.0f +
                          static_cast<float>(d0[i])) * qsc[h];
         const float E = fmaf(4.0f, P, (1.5f - zv) * qsm[h]);
-        score[(static_cast<size_t>(g) * GRP + h) * T + t] = (sv * E) * kInvSqrtD;
+        const float val = (sv * E) * kInvSqrtD;
+        score[(static_cast<size_t>(g) * GRP + h) * T + t] = val;
+        atomicAdd(&hs[h][okey32(val) >> 22], 1);
+        if (i & 1) am1 = fmaxf(am1, fabsf(val));
+        else am0 = fmaxf(am0, fabsf(val));
       }
     }
     cur = nxt;
   }
   smx = warp_max(smx);
   if (lane == 0) atomicMax(reinterpret_cast<unsigned int*>(smax + g), __float_as_uint(smx));
+  // max |score| per head: lanes with the same tig hold the same two heads
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    am0 = fmaxf(am0, __shfl_xor_sync(0xffffffffu, am0, o));
+    am1 = fmaxf(am1, __shfl_xor_sync(0xffffffffu, am1, o));
+  }
+  if (g8 == 0) {
+    if (2 * tig < GRP) atomicMax(amaxu + g * GRP + 2 * tig, __float_as_uint(am0));
+    if (2 * tig + 1 < GRP) atomicMax(amaxu + g * GRP + 2 * tig + 1, __float_as_uint(am1));
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < GRP * kHistBins; i += blockDim.x) {
+    const int c = (&hs[0][0])[i];
+    if (c) atomicAdd(hist + static_cast<size_t>(g) * GRP * kHistBins + i, c);
+  }
 }
 
 // ---- pass S: exact per-head top-k ------------------------------------------
-constexpr int kSelThreads = 1024;
 
 // Finds the bin holding the kk-th largest element of a histogram of nb bins
 // (scanning from the top) with warp 0.  Returns via shared out[0] = bin,
@@ -294,80 +327,6 @@ __device__ void find_bin_from_top(const int* hist, int nb, int kk, int* out) {
   }
   if (lane == 0) { out[0] = 0; out[1] = kk; }
 }
-
-// Block-wide sum of two ints (all threads call; result in every thread).
-__device__ __forceinline__ void block_sum2(int& a, int& b, int* scratch /* 64 ints */) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    a += __shfl_xor_sync(0xffffffffu, a, o);
-    b += __shfl_xor_sync(0xffffffffu, b, o);
-  }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  __syncthreads();
-  if (lane == 0) { scratch[warp] = a; scratch[32 + warp] = b; }
-  __syncthreads();
-  a = 0;
-  b = 0;
-  for (int w = 0; w < nw; ++w) { a += scratch[w]; b += scratch[32 + w]; }
-  __syncthreads();
-}
-
-// Exact per-head top-k (see the pass structure at the top of this file).
-//  1. amax over the fast scores and a strided sample of them;
-//  2. a threshold theta from the sample such that at least k scores are
-//     >= theta + 2 eps (checked by counting; lowered until true, at worst to
-//     -inf), so every token whose exact key can reach the top k has a fast
-//     score >= theta;
-//  3. G = {t : score_t >= theta} in token order, tau = k-th largest score over
-//     G by radix select (equal to the k-th largest overall);
-//  4. candidates F = {t in G : score_t >= tau - 2 eps}, re-keyed exactly in
-//     fp64, ranked by (key desc, token asc).
-// Ordered (stable) compaction of the indices i in [0, n) with pred(i), by a
-// whole block: warp w owns the contiguous segment [w seg, (w+1) seg) and walks
-// it 32 indices at a time (coalesced), with ballots giving positions inside
-// the warp; a prefix over the warps' counts gives each warp's offset.
-// Writes emit(pos, i) for the kept indices and returns their count.  Every
-// thread of the block must call it.
-template <class Pred, class Emit>
-__device__ int block_ordered_compact(int n, Pred pred, Emit emit, int* wsum /* 33 ints */) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const int seg = (((n + nw - 1) / nw) + 31) & ~31;
-  const int b0 = min(n, warp * seg), b1 = min(n, b0 + seg);
-  int cnt = 0;
-  for (int base = b0; base < b1; base += 32) {
-    const int i = base + lane;
-    cnt += __popc(__ballot_sync(0xffffffffu, i < b1 && pred(i)));
-  }
-  __syncthreads();
-  if (lane == 0) wsum[warp] = cnt;
-  __syncthreads();
-  if (warp == 0) {
-    const int v = lane < nw ? wsum[lane] : 0;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    if (lane < nw) wsum[lane] = incl - v;
-    if (lane == 31) wsum[32] = incl;
-  }
-  __syncthreads();
-  int off = wsum[warp];
-  const int total = wsum[32];
-  const unsigned lt = (1u << lane) - 1u;
-  for (int base = b0; base < b1; base += 32) {
-    const int i = base + lane;
-    const bool p = i < b1 && pred(i);
-    const unsigned bal = __ballot_sync(0xffffffffu, p);
-    if (p) emit(off + __popc(bal & lt), i);
-    off += __popc(bal);
-  }
-  __syncthreads();
-  return total;
-}
-
-constexpr int kDirectRank = 1024;  // candidates ranked pairwise (one per thread)
 
 // Query-side setup of pass S (all threads call): q in fp64 into qd, its l1
 // norm and the binary exponent of max |q|; flags the KV group when the
@@ -421,60 +380,12 @@ __device__ __forceinline__ double select_eps(double s_max, double l1, int qe, fl
   return 2.0 * (static_cast<double>(kInvSqrtD) * eps_k + 4.0 * u * static_cast<double>(amax));
 }
 
-// Last stage of pass S (all threads call): the candidates F[0..ncand) (token
-// order) are re-keyed exactly in fp64 and the k best by (key desc, token asc)
-// written to sel (k entries, ascending rank order is not required).
-__device__ void select_finish(const uint32_t* __restrict__ k_res, const uint16_t* __restrict__ k_scale,
-                              const uint16_t* __restrict__ k_zero, int g, int T, int k, const double* qd,
-                              const int32_t* __restrict__ F, int ncand, double* __restrict__ kp, int* hist,
-                              int* scan_scratch, int* binfo, int32_t* __restrict__ sel) {
+// Exact top-k of F[0..ncand) by (key desc, token asc) with an 8-pass radix
+// select on the 64-bit order-preserving keys kp (all threads call; F is in
+// token order); the k winners go to sel in no particular order.
+__device__ void select_rank_radix(const int32_t* __restrict__ F, int ncand, const double* __restrict__ kp, int k,
+                                  int* hist, int* scan_scratch, int* binfo, int32_t* __restrict__ sel) {
   const int tid = threadIdx.x, nthr = blockDim.x;
-  for (int i = tid; i < ncand; i += nthr) {
-    const int t = F[i];
-    const size_t row = static_cast<size_t>(g) * T + t;
-    const uint4* w4 = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
-    const uint4 x0 = w4[0], x1 = w4[1];
-    const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-    const double sv = static_cast<double>(sfd::half_bits_to_float(k_scale[row]));
-    const double z = static_cast<double>(sfd::half_bits_to_float(k_zero[row]));
-    double E = 0.0;
-#pragma unroll
-    for (int wi = 0; wi < 8; ++wi) {
-      const uint32_t word = w[wi];
-#pragma unroll 4
-      for (int j = 0; j < 16; ++j) {
-        const double c = static_cast<double>((word >> (2 * j)) & 3u);
-        E = fma(qd[16 * wi + j], c * 4.0 + 1.5 - z, E);
-      }
-    }
-    kp[i] = sv * E;
-  }
-  __syncthreads();
-
-  // few candidates (the usual case): rank each one directly against all
-  // others by (key desc, token asc) -- no synchronised passes
-  if (ncand <= kDirectRank && ncand <= nthr) {
-    double* kd = reinterpret_cast<double*>(hist);  // 2048 ints = 1024 doubles of scratch
-    for (int i = tid; i < ncand; i += nthr) kd[i] = kp[i];
-    __syncthreads();
-    int take = 0;
-    const int i = tid;
-    if (i < ncand) {
-      const double ki = kd[i];
-      int rank = 0;
-      for (int j = 0; j < ncand; ++j) {
-        const double kj = kd[j];
-        rank += (kj > ki) || (kj == ki && j < i);  // F is in token order
-      }
-      take = rank < k;
-    }
-    int tot;
-    const int pos = sfd::block_exclusive_scan(take, scan_scratch, &tot);
-    if (take) sel[pos] = F[i];
-    return;
-  }
-
-  // many candidates: exact top-k by an 8-pass radix select on the 64-bit keys
   unsigned long long pre64 = 0, pm64 = 0;
   int kr = k;
   for (int pass = 0; pass < 8; ++pass) {
@@ -517,122 +428,7 @@ __device__ void select_finish(const uint32_t* __restrict__ k_res, const uint16_t
       else if (key == pre64) { ok = rank < kr; ++rank; }
       if (ok) sel[pos++] = F[i];
     }
-  }
-}
-
-// Exact per-head top-k for any T, streaming the scores from global memory:
-//  1. amax over the fast scores and a strided sample of them;
-//  2. a threshold theta from the sample such that at least k scores are
-//     >= theta + 2 eps (checked by counting; lowered until true, at worst to
-//     -inf), so every token whose exact key can reach the top k has a fast
-//     score >= theta;
-//  3. G = {t : score_t >= theta} in token order, tau = k-th largest score over
-//     G by radix select (equal to the k-th largest overall);
-//  4. candidates F = {t in G : score_t >= tau - 2 eps}, re-keyed exactly in
-//     fp64, ranked by (key desc, token asc).
-template <int GRP>
-__global__ void __launch_bounds__(kSelThreads)
-attn_select_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
-                   const uint16_t* __restrict__ k_scale, const uint16_t* __restrict__ k_zero, int T, int k,
-                   const float* __restrict__ score, const float* __restrict__ smax, int32_t* __restrict__ cand,
-                   int32_t* __restrict__ cand2, double* __restrict__ kap, int32_t* __restrict__ sel_head,
-                   int32_t* __restrict__ status) {
-  constexpr int kSamples = 512;
-  __shared__ __align__(16) int hist[2048];
-  __shared__ double qd[D];
-  __shared__ float samp[kSamples];
-  __shared__ int scan_scratch[64];
-  __shared__ int binfo[2];
-  __shared__ float red[32];
-  __shared__ double l1_sh;
-  __shared__ int qe_sh;
-  __shared__ float theta_sh;
-  const int h = blockIdx.x, g = h / GRP, tid = threadIdx.x;
-  const float* sc = score + static_cast<size_t>(h) * T;
-  int32_t* G = cand + static_cast<size_t>(h) * T;
-  int32_t* F = cand2 + static_cast<size_t>(h) * T;
-  double* kp = kap + static_cast<size_t>(h) * T;
-
-  select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status);
-
-  // 1. amax and a strided sample
-  const int ns = T < kSamples ? T : kSamples;
-  const int stride = T / ns;
-  float amax = 0.0f;
-  for (int t = tid; t < T; t += kSelThreads) amax = fmaxf(amax, fabsf(sc[t]));
-  for (int i = tid; i < ns; i += kSelThreads) samp[i] = sc[i * stride];
-  {
-    const float m = warp_max(amax);
-    if ((tid & 31) == 0) red[tid >> 5] = m;
-    __syncthreads();
-    if (tid < 32) {
-      const float mm = warp_max(red[tid]);
-      if (tid == 0) red[0] = mm;
-    }
-    __syncthreads();
-    amax = red[0];
-  }
-  const double eps_s = select_eps(static_cast<double>(smax[g]), l1_sh, qe_sh, amax);
-
-  // 2. threshold from the sample: aim at ~2k + 64 tokens above it
-  double theta = -INFINITY;
-  for (int trial = 0; trial < 3; ++trial) {
-    int want = static_cast<int>((static_cast<long long>(2 * k + 64) * ns) / T) + 1;
-    want <<= (2 * trial);  // lower the threshold on a retry
-    if (trial == 2 || want >= ns) break;  // fall back to all tokens
-    // the want-th largest sample (rank counted from 1)
-    for (int i = tid; i < ns; i += kSelThreads) {
-      const float v = samp[i];
-      int gt = 0, ge = 0;
-      for (int j = 0; j < ns; ++j) {
-        const float w = samp[j];
-        gt += w > v;
-        ge += w >= v;
-      }
-      if (gt < want && want <= ge) theta_sh = v;
-    }
-    __syncthreads();
-    const double th = static_cast<double>(theta_sh) - 2.0 * eps_s;
-    int c1 = 0, dummy = 0;
-    for (int t = tid; t < T; t += kSelThreads) c1 += static_cast<double>(sc[t]) >= th + 2.0 * eps_s;
-    block_sum2(c1, dummy, scan_scratch);
-    if (c1 >= k) { theta = th; break; }
-  }
-
-  // 3. G in token order, then tau = k-th largest over G
-  const int nG = block_ordered_compact(
-      T, [&](int t) { return static_cast<double>(sc[t]) >= theta; }, [&](int pos, int t) { G[pos] = t; },
-      scan_scratch);
-  uint32_t prefix = 0, pmask = 0;
-  int kk = k;
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
-  for (int pass = 0; pass < 3; ++pass) {
-    const int nb = 1 << widths[pass];
-    for (int i = tid; i < nb; i += kSelThreads) hist[i] = 0;
-    __syncthreads();
-    for (int i = tid; i < nG; i += kSelThreads) {
-      const uint32_t key = okey32(sc[G[i]]);
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shifts[pass]) & (nb - 1)], 1);
-    }
-    __syncthreads();
-    find_bin_from_top(hist, nb, kk, binfo);
-    __syncthreads();
-    prefix |= static_cast<uint32_t>(binfo[0]) << shifts[pass];
-    pmask |= static_cast<uint32_t>(nb - 1) << shifts[pass];
-    kk = binfo[1];
-    __syncthreads();
-  }
-  const double tau = static_cast<double>(from_okey32(prefix));
-  const double thr = tau - 2.0 * eps_s;
-
-  // 4. candidates F (token order), exact keys, ranking
-  const int ncand = block_ordered_compact(
-      nG, [&](int i) { return static_cast<double>(sc[G[i]]) >= thr; }, [&](int pos, int i) { F[pos] = G[i]; },
-      scan_scratch);
-  select_finish(k_res, k_scale, k_zero, g, T, k, qd, F, ncand, kp, hist, scan_scratch, binfo,
-                sel_head + static_cast<size_t>(h) * k);
-}
+  }}
 
 // Block-parallel search of a histogram from the top (all threads call):
 // out[0] = the bin holding the kk-th largest element, out[1] = kk minus the
@@ -659,158 +455,328 @@ __device__ void find_bin_from_top_block(const int* hist, int nb, int kk, int* ou
   __syncthreads();
 }
 
-// Exact per-head top-k for T <= kRegKeys * kSelThreads with the scores held
-// in registers (one coalesced read of the head's scores):
-//  1. tau = the k-th largest fast score, by a 3-pass radix select (11, 11 and
-//     10 bits of the order-preserving key) over the register-held keys;
-//  2. candidates F = {t : score_t >= tau - 2 eps}, compacted in token order
-//     straight from the registers (warp w holds the contiguous token range
-//     [w seg, (w+1) seg), row i of it at w seg + 32 i + lane);
-//  3. exact fp64 keys and ranking as in the streaming kernel.
-constexpr int kRegKeys = 32;
+// ---- pass S, selection from the score histogram -----------------------------
+//
+// Pass A left, per query head, a histogram of its fast scores over the top 10
+// bits of the order-preserving key, and max |score|.  The bin b1 holding the
+// k-th largest score follows from the histogram alone.  Every token whose
+// exact key can reach the top k has a fast score >= tau - 2 eps >= (lower
+// edge of b1) - 2 eps, so:
+//  A  compact: per (4096-token chunk, head), the tokens with fast score >=
+//     lower(b1) - 2 eps, in token order, into the chunk's slot of a list;
+//  B  finish (one cluster per KV group, one CTA per query head): concatenate
+//     the chunks, find tau exactly by two more radix passes over the listed
+//     scores of bin b1, keep the candidates >= tau - 2 eps, re-key them
+//     exactly in fp64 and rank them (key desc, token asc); then the group's
+//     CTAs build the union of their selections (bitmask and ascending list)
+//     through distributed shared memory and each computes its head's refined
+//     scores for the union tokens.
+
+// Per-head threshold of the compaction and the histogram bin: all threads call.
+__device__ void select_band(const int32_t* __restrict__ hist_h, int k, double eps_s, int* hsh, int* scan_scratch,
+                            int* binfo, uint32_t* b1, int* kk, float* f_low) {
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hsh[i] = hist_h[i];
+  __syncthreads();
+  find_bin_from_top_block(hsh, kHistBins, k, binfo, scan_scratch);
+  *b1 = static_cast<uint32_t>(binfo[0]);
+  *kk = binfo[1];
+  const float lower = from_okey32(*b1 << 22);
+  *f_low = __double2float_rd(static_cast<double>(lower) - 2.0 * eps_s);
+}
+
+constexpr int kCompThreads = 256;
 
 template <int GRP>
-__global__ void __launch_bounds__(kSelThreads)
-attn_select_reg_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
-                       const uint16_t* __restrict__ k_scale, const uint16_t* __restrict__ k_zero, int T, int k,
-                       const float* __restrict__ score, const float* __restrict__ smax, int32_t* __restrict__ cand2,
-                       double* __restrict__ kap, int32_t* __restrict__ sel_head, int32_t* __restrict__ status) {
-  __shared__ __align__(16) int hist[2048];
-  __shared__ double qd[D];
+__global__ void __launch_bounds__(kCompThreads)
+attn_select_compact_kernel(const uint16_t* __restrict__ q, int T, int k, const float* __restrict__ score,
+                           const float* __restrict__ smax, const int32_t* __restrict__ hist,
+                           const uint32_t* __restrict__ amaxu, int32_t* __restrict__ cand, int nchunks,
+                           int32_t* __restrict__ status) {
+  const int chunk = blockIdx.x, h = blockIdx.y, g = h / GRP;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ int hsh[kHistBins];
   __shared__ int scan_scratch[64];
   __shared__ int binfo[2];
-  __shared__ float red[32];
+  __shared__ double qd[D];
   __shared__ double l1_sh;
   __shared__ int qe_sh;
-  const int h = blockIdx.x, g = h / GRP, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status);
+  const double eps_s = select_eps(static_cast<double>(smax[g]), l1_sh, qe_sh, __uint_as_float(amaxu[h]));
+  uint32_t b1;
+  int kk;
+  float f_low;
+  select_band(hist + static_cast<size_t>(h) * kHistBins, k, eps_s, hsh, scan_scratch, binfo, &b1, &kk, &f_low);
+  // warp w: tokens [chunk*4096 + 512 w, +512) as 16 rows of 32
+  constexpr int kRowsPerWarp = kChunk / (kCompThreads / 32) / 32;
+  const int t0 = chunk * kChunk + warp * 32 * kRowsPerWarp + lane;
+  const int tend = min(T, chunk * kChunk + (warp + 1) * 32 * kRowsPerWarp);
   const float* sc = score + static_cast<size_t>(h) * T;
-  int32_t* F = cand2 + static_cast<size_t>(h) * T;
-  double* kp = kap + static_cast<size_t>(h) * T;
-
-  const int seg = (((T + 31) >> 5) + 31) & ~31;  // tokens per warp: a multiple of 32, <= 32 kRegKeys
-  const int t0 = warp * seg + lane;
-  const int tend = min(T, warp * seg + seg);
-  uint32_t key[kRegKeys];
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < kRegKeys; ++i) {
-    const int t = t0 + 32 * i;
-    const float v = t < tend ? sc[t] : 0.0f;
-    key[i] = okey32(v);
-    amax = fmaxf(amax, fabsf(v));
-  }
-  for (int i = tid; i < 2048; i += kSelThreads) hist[i] = 0;
-  select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status);  // ends with __syncthreads
-  {
-    const float m = warp_max(amax);
-    if (lane == 0) red[warp] = m;
-  }
-
-  // 1. tau by radix select over the registers
-#pragma unroll
-  for (int i = 0; i < kRegKeys; ++i)
-    if (t0 + 32 * i < tend) atomicAdd(&hist[key[i] >> 21], 1);
-  __syncthreads();
-  find_bin_from_top_block(hist, 2048, k, binfo, scan_scratch);
-  const uint32_t b1 = static_cast<uint32_t>(binfo[0]);
-  int kk = binfo[1];
-  for (int i = tid; i < 2048; i += kSelThreads) hist[i] = 0;
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < kRegKeys; ++i)
-    if (t0 + 32 * i < tend && (key[i] >> 21) == b1) atomicAdd(&hist[(key[i] >> 10) & 2047u], 1);
-  __syncthreads();
-  find_bin_from_top_block(hist, 2048, kk, binfo, scan_scratch);
-  const uint32_t p2 = (b1 << 11) | static_cast<uint32_t>(binfo[0]);
-  kk = binfo[1];
-  for (int i = tid; i < 1024; i += kSelThreads) hist[i] = 0;
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < kRegKeys; ++i)
-    if (t0 + 32 * i < tend && (key[i] >> 10) == p2) atomicAdd(&hist[key[i] & 1023u], 1);
-  __syncthreads();
-  find_bin_from_top_block(hist, 1024, kk, binfo, scan_scratch);
-  const float tau = from_okey32((p2 << 10) | static_cast<uint32_t>(binfo[0]));
-  if (warp == 0) {
-    const float mm = warp_max(red[lane]);
-    if (lane == 0) red[0] = mm;
-  }
-  __syncthreads();
-  const double eps_s = select_eps(static_cast<double>(smax[g]), l1_sh, qe_sh, red[0]);
-  // smallest float f with f >= tau - 2 eps: (double)x >= tau - 2 eps <=> x >= f
-  const float fthr = __double2float_ru(static_cast<double>(tau) - 2.0 * eps_s);
-
-  // 2. candidates in token order
+  bool p[kRowsPerWarp];
   int cnt = 0;
 #pragma unroll
-  for (int i = 0; i < kRegKeys; ++i)
-    cnt += __popc(__ballot_sync(0xffffffffu, t0 + 32 * i < tend && from_okey32(key[i]) >= fthr));
+  for (int i = 0; i < kRowsPerWarp; ++i) {
+    const int t = t0 + 32 * i;
+    p[i] = t < tend && sc[t] >= f_low;
+    cnt += __popc(__ballot_sync(0xffffffffu, p[i]));
+  }
   if (lane == 0) scan_scratch[warp] = cnt;
   __syncthreads();
   if (warp == 0) {
-    const int v = scan_scratch[lane];
+    const int v = lane < kCompThreads / 32 ? scan_scratch[lane] : 0;
     int incl = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += y;
     }
-    scan_scratch[32 + lane] = incl - v;
-    if (lane == 31) binfo[0] = incl;
+    if (lane < kCompThreads / 32) scan_scratch[32 + lane] = incl - v;
+    // the chunks' counts follow the Hq x T lists
+    if (lane == 31) cand[static_cast<size_t>(gridDim.y) * T + static_cast<size_t>(h) * nchunks + chunk] = incl;
   }
   __syncthreads();
-  int off = scan_scratch[32 + warp];
-  const int ncand = binfo[0];
+  int32_t* out = cand + static_cast<size_t>(h) * T + static_cast<size_t>(chunk) * kChunk;
+  int o = scan_scratch[32 + warp];
   const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int i = 0; i < kRegKeys; ++i) {
-    const bool p = t0 + 32 * i < tend && from_okey32(key[i]) >= fthr;
-    const unsigned bal = __ballot_sync(0xffffffffu, p);
-    if (p) F[off + __popc(bal & lt)] = t0 + 32 * i;
-    off += __popc(bal);
+  for (int i = 0; i < kRowsPerWarp; ++i) {
+    const unsigned bal = __ballot_sync(0xffffffffu, p[i]);
+    if (p[i]) out[o + __popc(bal & lt)] = t0 + 32 * i;
+    o += __popc(bal);
   }
-  __syncthreads();
-
-  // 3. exact keys and ranking
-  select_finish(k_res, k_scale, k_zero, g, T, k, qd, F, ncand, kp, hist, scan_scratch, binfo,
-                sel_head + static_cast<size_t>(h) * k);
 }
 
-// ---- pass U: union per KV head ---------------------------------------------
-__global__ void __launch_bounds__(1024)
-attn_union_kernel(const int32_t* __restrict__ sel_head, int grp, int T, int k, int words_t,
-                  uint32_t* __restrict__ umask, int32_t* __restrict__ sel_out, int32_t* __restrict__ sel_n,
-                  const int32_t* __restrict__ status) {
-  extern __shared__ uint32_t bits[];  // [words_t]
-  __shared__ int scan_scratch[33];
-  const int g = blockIdx.x, tid = threadIdx.x;
-  for (int i = tid; i < words_t; i += blockDim.x) bits[i] = 0;
-  __syncthreads();
-  for (int e = tid; e < grp * k; e += blockDim.x) {
-    const int t = sel_head[static_cast<size_t>(g) * grp * k + e];
-    atomicOr(&bits[t >> 5], 1u << (t & 31));
+constexpr int kFinThreads = 512;
+constexpr int kFinKeys = 2048;     // candidates ranked pairwise from shared memory
+constexpr int kFinChunks = 4096;   // chunk prefix sums in shared memory (T <= 2^24)
+
+template <int GRP>
+__global__ void __launch_bounds__(kFinThreads)
+attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
+                          const uint32_t* __restrict__ k_ref, const uint16_t* __restrict__ k_scale,
+                          const uint16_t* __restrict__ k_zero, int T, int k, float* __restrict__ score,
+                          const float* __restrict__ smax, const int32_t* __restrict__ hist,
+                          const uint32_t* __restrict__ amaxu, int32_t* __restrict__ cand, int nchunks,
+                          int32_t* __restrict__ list, double* __restrict__ kap, int32_t* __restrict__ sel_head,
+                          uint32_t* __restrict__ umask, int words_t, int32_t* __restrict__ sel_out,
+                          int32_t* __restrict__ sel_n, int32_t* __restrict__ status) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = static_cast<int>(cl.block_rank());
+  const int h = blockIdx.x, g = h / GRP;
+  const int tid = threadIdx.x;
+  __shared__ int hr[2048];
+  __shared__ int cpre[kFinChunks];
+  __shared__ double keys[kFinKeys];
+  __shared__ double qd[D];
+  __shared__ float qs[D];
+  __shared__ float qsum_sh;
+  __shared__ int scan_scratch[64];
+  __shared__ int binfo[2];
+  __shared__ double l1_sh;
+  __shared__ int qe_sh;
+  __shared__ int cnt_sh;  // read remotely
+  const float* sc = score + static_cast<size_t>(h) * T;
+  int32_t* L = list + static_cast<size_t>(h) * T;  // concatenated list, token order
+  int32_t* F = cand + static_cast<size_t>(h) * T;  // candidates (reuses the chunk lists once L is built)
+  double* kp = kap + static_cast<size_t>(h) * T;
+  const int cap = GRP * k;
+
+  select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status);
+  for (int d = tid; d < D; d += kFinThreads) qs[d] = static_cast<float>(qd[d]);
+  if (tid == 0) {
+    float acc = 0.0f;  // sequential fp32 order, d ascending (as the refined-score pass always used)
+    for (int d = 0; d < D; ++d) acc += static_cast<float>(qd[d]);
+    qsum_sh = acc;
+  }
+  const double eps_s = select_eps(static_cast<double>(smax[g]), l1_sh, qe_sh, __uint_as_float(amaxu[h]));
+  uint32_t b1;
+  int kk;
+  float f_low;
+  select_band(hist + static_cast<size_t>(h) * kHistBins, k, eps_s, hr, scan_scratch, binfo, &b1, &kk, &f_low);
+
+  // 1. concatenate the chunk lists (token order)
+  const int32_t* counts = cand + static_cast<size_t>(gridDim.x) * T + static_cast<size_t>(h) * nchunks;
+  int m = 0;
+  for (int base = 0; base < nchunks; base += kFinThreads) {
+    const int c = base + tid;
+    const int v = c < nchunks ? counts[c] : 0;
+    int tot;
+    const int pre = sfd::block_exclusive_scan(v, scan_scratch, &tot);
+    if (c < nchunks) cpre[c] = m + pre;
+    m += tot;
   }
   __syncthreads();
-  const int chunk = (words_t + blockDim.x - 1) / blockDim.x;
-  const int w0 = min(words_t, tid * chunk), w1 = min(words_t, w0 + chunk);
-  int c = 0;
-  for (int w = w0; w < w1; ++w) {
-    c += __popc(bits[w]);
-    umask[static_cast<size_t>(g) * words_t + w] = bits[w];
+  for (int e = tid; e < m; e += kFinThreads) {
+    int lo = 0, hi = nchunks - 1;  // last chunk with cpre <= e
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cpre[mid] <= e) lo = mid;
+      else hi = mid - 1;
+    }
+    L[e] = cand[static_cast<size_t>(h) * T + static_cast<size_t>(lo) * kChunk + (e - cpre[lo])];
   }
-  int total;
-  int pos = sfd::block_exclusive_scan(c, scan_scratch, &total);
-  int32_t* out = sel_out + static_cast<size_t>(g) * grp * k;
-  for (int w = w0; w < w1; ++w) {
-    uint32_t m = bits[w];
-    while (m) {
-      const int b = __ffs(m) - 1;
-      out[pos++] = w * 32 + b;
-      m &= m - 1;
+  __syncthreads();
+
+  // 2. tau: two radix passes (11 + 11 bits) over the listed scores of bin b1
+  uint32_t pre = b1 << 22;
+  for (int pass = 0; pass < 2; ++pass) {
+    const int shift = pass == 0 ? 11 : 0;
+    for (int i = tid; i < 2048; i += kFinThreads) hr[i] = 0;
+    __syncthreads();
+    const uint32_t pmask = pass == 0 ? 0xFFC00000u : 0xFFFFF800u;
+    for (int e = tid; e < m; e += kFinThreads) {
+      const uint32_t key = okey32(sc[L[e]]);
+      if ((key & pmask) == pre) atomicAdd(&hr[(key >> shift) & 2047u], 1);
+    }
+    __syncthreads();
+    find_bin_from_top_block(hr, 2048, kk, binfo, scan_scratch);
+    pre |= static_cast<uint32_t>(binfo[0]) << shift;
+    kk = binfo[1];
+  }
+  const float tau = from_okey32(pre);
+  const float fthr = __double2float_ru(static_cast<double>(tau) - 2.0 * eps_s);
+
+  // 3. candidates >= tau - 2 eps in list (= token) order
+  int ncand = 0;
+  for (int base = 0; base < m; base += kFinThreads) {
+    const int e = base + tid;
+    const bool p = e < m && sc[L[e]] >= fthr;
+    int tot;
+    const int pos = sfd::block_exclusive_scan(p ? 1 : 0, scan_scratch, &tot);
+    if (p) F[ncand + pos] = L[e];
+    ncand += tot;
+  }
+  __syncthreads();
+
+
+  // 4. exact keys (four partial sums: exact under the precondition, so the
+  //    order does not change the key)
+  for (int i = tid; i < ncand; i += kFinThreads) {
+    const int t = F[i];
+    const size_t row = static_cast<size_t>(g) * T + t;
+    const uint4* w4 = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
+    const uint4 x0 = w4[0], x1 = w4[1];
+    const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    const double sv = static_cast<double>(sfd::half_bits_to_float(k_scale[row]));
+    const double z = static_cast<double>(sfd::half_bits_to_float(k_zero[row]));
+    double E[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+    for (int wi = 0; wi < 8; ++wi) {
+      const uint32_t word = w[wi];
+#pragma unroll 1
+      for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = 4 * jj + u;
+          const double c = static_cast<double>((word >> (2 * j)) & 3u);
+          E[u] = fma(qd[16 * wi + j], c * 4.0 + 1.5 - z, E[u]);
+        }
+    }
+    const double key = sv * ((E[0] + E[1]) + (E[2] + E[3]));
+    kp[i] = key;
+    if (ncand <= kFinKeys) keys[i] = key;
+  }
+  __syncthreads();
+
+  // 5. rank by (key desc, token asc); the k winners go to sel_head and the
+  //    group's token bitmask
+  int32_t* sel = sel_head + static_cast<size_t>(h) * k;
+  uint32_t* um = umask + static_cast<size_t>(g) * words_t;
+  if (ncand <= kFinKeys) {
+    int tpc = 1;  // threads per candidate: a power of two up to 32
+    while (tpc < 32 && 2 * tpc * max(ncand, 1) <= kFinThreads) tpc *= 2;
+    const int per = kFinThreads / tpc;
+    for (int r0 = 0; r0 < ncand; r0 += per) {  // uniform over the block
+      const int i = r0 + tid / tpc, sub = tid % tpc;
+      int rk = 0;
+      if (i < ncand) {
+        const double ki = keys[i];
+        for (int j = sub; j < ncand; j += tpc) {
+          const double kj = keys[j];
+          rk += (kj > ki) || (kj == ki && j < i);
+        }
+      }
+      for (int o = tpc / 2; o > 0; o >>= 1) rk += __shfl_xor_sync(0xffffffffu, rk, o);
+      if (i < ncand && sub == 0 && rk < k) {
+        const int t = F[i];
+        sel[rk] = t;
+        atomicOr(um + (t >> 5), 1u << (t & 31));
+      }
+    }
+  } else {
+    select_rank_radix(F, ncand, kp, k, hr, scan_scratch, binfo, sel);
+    __syncthreads();
+    for (int i = tid; i < k; i += kFinThreads) {
+      const int t = sel[i];
+      atomicOr(um + (t >> 5), 1u << (t & 31));
     }
   }
-  // a group whose query violated the exact-key precondition reports -1 - n
-  if (tid == 0) sel_n[g] = status[g] ? -1 - total : total;
+  __threadfence();
+  cl.sync();  // 1: the group's bitmask is complete
+
+  // 6. union, ascending: CTA r of the cluster compacts words [r wper, (r+1) wper)
+  const int wper = (words_t + GRP - 1) / GRP;
+  const int w0 = min(words_t, rank * wper), w1 = min(words_t, w0 + wper);
+  int mycnt = 0;
+  {
+    const int chunk = (w1 - w0 + kFinThreads - 1) / kFinThreads;
+    const int a0 = min(w1, w0 + tid * chunk), a1 = min(w1, a0 + chunk);
+    int c = 0;
+    for (int w = a0; w < a1; ++w) c += __popc(um[w]);
+    int tot;
+    int pos = sfd::block_exclusive_scan(c, scan_scratch, &tot);
+    if (tid == 0) cnt_sh = tot;
+    cl.sync();  // 2: every CTA's count is published
+    int off = 0, U = 0;
+    for (int r = 0; r < GRP; ++r) {
+      const int cr = *cl.map_shared_rank(&cnt_sh, r);
+      if (r < rank) off += cr;
+      U += cr;
+    }
+    mycnt = U;
+    int32_t* out = sel_out + static_cast<size_t>(g) * cap;
+    pos += off;
+    for (int w = a0; w < a1; ++w) {
+      uint32_t bits = um[w];
+      while (bits) {
+        const int b = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        out[pos++] = 32 * w + b;
+      }
+    }
+    if (rank == 0 && tid == 0) sel_n[g] = status[g] ? -1 - U : U;
+  }
+  __threadfence();
+  cl.sync();  // 3: the union list is complete; no shared-memory access across CTAs after this
+
+  // 7. refined scores of this head for the union tokens: full 4-bit codes
+  const int U = mycnt;
+  const int32_t* ul = sel_out + static_cast<size_t>(g) * cap;
+  const float qsum = qsum_sh;
+  for (int u = tid; u < U; u += kFinThreads) {
+    const int t = ul[u];
+    const size_t row = static_cast<size_t>(g) * T + t;
+    const uint4* r4 = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
+    const uint4* f4 = reinterpret_cast<const uint4*>(k_ref + row * kWordsPerRow);
+    const uint4 ra = r4[0], rb = r4[1], fa = f4[0], fb = f4[1];
+    const uint32_t wr[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+    const uint32_t wf[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
+    float P0 = 0.0f, P1 = 0.0f;
+#pragma unroll
+    for (int wi = 0; wi < 8; ++wi) {
+      const uint32_t xr = wr[wi], xf = wf[wi];
+#pragma unroll 2
+      for (int jj = 0; jj < 8; ++jj) {
+        const int j = 2 * jj;
+        P0 = fmaf(qs[16 * wi + j], static_cast<float>(((xr >> (2 * j)) & 3u) * 4u + ((xf >> (2 * j)) & 3u)), P0);
+        P1 = fmaf(qs[16 * wi + j + 1],
+                  static_cast<float>(((xr >> (2 * j + 2)) & 3u) * 4u + ((xf >> (2 * j + 2)) & 3u)), P1);
+      }
+    }
+    const float sv = sfd::half_bits_to_float(k_scale[row]);
+    const float z = sfd::half_bits_to_float(k_zero[row]);
+    score[static_cast<size_t>(h) * T + t] = (sv * fmaf(-z, qsum, P0 + P1)) * kInvSqrtD;
+  }
 }
 
 // ---- refined scores of the refined tokens ------------------------------------
@@ -1272,36 +1238,43 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
   SF_CHECK_CUDA(cudaMemsetAsync(ws + L.smax, 0, L.total - L.smax, s));
   const int ntiles = (T + 15) / 16;
   dim3 ga(std::max(1, std::min((ntiles + 3) / 4, (4 * sms + Hkv - 1) / Hkv)), Hkv);
-  attn_score_mma_kernel<GRP><<<ga, 128, 0, s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, score, smax);
+  int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
+  uint32_t* amaxu = reinterpret_cast<uint32_t*>(ws + L.amax);
+  attn_score_mma_kernel<GRP><<<ga, 128, 0, s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, score, smax, hist, amaxu);
   sf_status st = sf::check_launch("attn_score_mma_kernel");
   if (st != SF_OK) return st;
   const int cap = grp * k;  // row length of sel_out
   if (k > 0 && k < T) {
-    if (T <= kRegKeys * kSelThreads) {
-      attn_select_reg_kernel<GRP><<<Hq, kSelThreads, 0, s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, k, score,
-                                                             smax, cand2, kap, sel_head, status);
-      st = sf::check_launch("attn_select_reg_kernel");
-    } else {
-      attn_select_kernel<GRP><<<Hq, kSelThreads, 0, s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, k, score, smax,
-                                                         cand, cand2, kap, sel_head, status);
-      st = sf::check_launch("attn_select_kernel");
-    }
+    attn_select_compact_kernel<GRP><<<dim3(L.nchunks, Hq), kCompThreads, 0, s>>>(q, T, k, score, smax, hist, amaxu,
+                                                                                cand, L.nchunks, status);
+    st = sf::check_launch("attn_select_compact_kernel");
     if (st != SF_OK) return st;
-    const size_t smem = sizeof(uint32_t) * L.words_t;
-    SF_CHECK_CUDA(cudaFuncSetAttribute(attn_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(std::max<size_t>(smem, 1))));
-    attn_union_kernel<<<Hkv, 1024, smem, s>>>(sel_head, grp, T, k, L.words_t, umask, sel_out, sel_n, status);
-    st = sf::check_launch("attn_union_kernel");
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(Hq));
+    cfg.blockDim = dim3(kFinThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = GRP;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, attn_select_finish_kernel<GRP>, q, kv->k_res, kv->k_ref, kv->k_scale,
+                                     kv->k_zero, T, k, score, static_cast<const float*>(smax),
+                                     static_cast<const int32_t*>(hist), static_cast<const uint32_t*>(amaxu), cand,
+                                     L.nchunks, cand2, kap, sel_head, umask, L.words_t, sel_out, sel_n, status));
+    st = sf::check_launch("attn_select_finish_kernel");
     if (st != SF_OK) return st;
-  } else if (k == 0) {
-    SF_CHECK_CUDA(cudaMemsetAsync(umask, 0, sizeof(uint32_t) * Hkv * static_cast<size_t>(L.words_t), s));
+  } else if (k == 0) {  // the token bitmask was cleared with the workspace
     SF_CHECK_CUDA(cudaMemsetAsync(sel_n, 0, sizeof(int32_t) * Hkv, s));
   } else {
     fill_all_kernel<<<dim3(32, Hkv), 256, 0, s>>>(T, grp, k, L.words_t, umask, sel_out, sel_n);
     st = sf::check_launch("fill_all_kernel");
     if (st != SF_OK) return st;
   }
-  if (k > 0) {
+  if (k == T) {  // every token refined: refined scores of the whole sequence
     dim3 gr(std::max(1, std::min((cap + 7) / 8, 128)), Hkv);
     attn_refine_scores_kernel<GRP><<<gr, 256, 0, s>>>(q, kv->k_res, kv->k_ref, kv->k_scale, kv->k_zero, T, cap,
                                                       sel_out, sel_n, score);

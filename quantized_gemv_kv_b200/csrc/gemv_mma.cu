@@ -8,23 +8,30 @@
 // (act.cuh: per-group fixed point in signed 8-bit digits, laid out as MMA B
 // fragments, plus the selection mask).
 //
-// Tiles are 16 output rows.  A warp owns SPW 256-channel slices of K for the
-// whole kernel; their B fragments stay in registers.  Per tile and slice the
-// 16 rows x 256 codes go through 8 mma.m16n8k32 (u8 codes x s8 digits, s32
-// accumulate); a code word becomes four A-fragment bytes with one shift and
-// one mask.  The two 128-channel groups of a slice accumulate into disjoint
-// columns (three digit planes each), so after the 8 MMAs each pair of lanes
-// holds the plane sums of two (row, group) pairs and one swap gives each
-// lane one pair: it applies that pair's scale and zero point,
-//   s (2^b_f fscale P + (m_f - z) gsum + sum_{j in S, j in group} x_j (q_f - m_f)),
-// so the scale/zero arithmetic and the refinement correction are spread over
-// all 32 lanes.  The warps of a CTA cover consecutive slices of one tile and
-// add up in shared memory; with two K halves (ksplit = 2) the halves add
-// their partial sums onto a zeroed output (two terms onto zero: the result
-// does not depend on their order).
+// Tiles are 16 output rows; a CTA walks a contiguous block of them.  A warp
+// owns SPW 256-channel slices of K for the whole kernel; their B fragments
+// stay in registers.  Per tile and slice:
+//  * resident part: 8 mma.m16n8k32 (u8 codes x s8 digits, s32 accumulate,
+//    two independent chains); a code word becomes four A-fragment bytes with
+//    one shift and one mask.  The slice's two groups land in disjoint
+//    accumulator columns (three digit planes each), so after one lane swap
+//    each lane owns one (row, group) pair and applies its scale and zero point;
+//  * refinement correction: the 2-bit q_f of the 16 rows for the slice's
+//    selected channels (one staged word per channel) become f16 A fragments
+//    (1024 + q_f, exact) against the channels' x split into f16 high and low
+//    parts, on mma.m16n8k16; the 1024 offset and m_f are removed with
+//    per-group sums of x.
+// The warps of a CTA cover consecutive slices of one tile and add up in
+// shared memory; with two K halves (ksplit = 2) the halves add their partial
+// sums onto a zeroed output (two terms onto zero: the result does not depend
+// on their order).
 //
-// Each warp streams its own codes, scale/zero and refinement words through a
-// cp.async ring in shared memory; a warp waits only for its own copies.
+// Each warp streams its own codes (16 rows x 64 bytes per slice, 16-byte
+// chunks XOR-swizzled so the fragment loads are free of bank conflicts),
+// scale/zero and refinement words through a cp.async ring in shared memory
+// and waits only for its own copies.
+#include <cuda_fp16.h>
+
 #include <algorithm>
 
 #include "act.cuh"
@@ -33,13 +40,10 @@
 namespace {
 
 constexpr int kMaxJobs = 4;
-constexpr int kRows = 16;       // output rows per tile
-constexpr int kCodeStr = 24;    // words per staged code row (16 used): conflict-free fragment loads
-constexpr int kRefSlot = 16;    // refinement words staged per (slice, group) and tile
-constexpr int kSelCap = 128;    // list capacity per (slice, group): the whole group
-constexpr int kSzWords = 32;    // scale, zero of 2 groups x 16 rows (fp16)
-constexpr int kSliceStage = kRows * kCodeStr + kSzWords + 2 * kRefSlot;  // words per slice and stage
-constexpr int kMaxWarps = 16;
+constexpr int kRows = 16;          // output rows per tile
+constexpr int kMaxWarps = 16;      // warps per CTA
+constexpr int kCorrList = 32;      // selected channels per slice handled on the tensor cores
+constexpr int kSliceWords = 256 + 32 + 32;  // words per slice and stage: codes, scale/zero, refinement
 
 struct MJob {
   const uint32_t* res;
@@ -55,7 +59,7 @@ struct MArgs {
   MJob job[kMaxJobs];
   const uint16_t* x;
   const uint32_t* act;
-  int njobs, K, b_f, ksplit;
+  int njobs, K, ksplit;
 };
 
 __device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
@@ -76,6 +80,12 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
                : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                        uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 
 // fp16 bit pattern -> fp32 with integer/FP32 pipes only: move exponent and
 // mantissa into place and rescale by 2^112, exact for every finite fp16
@@ -83,9 +93,7 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
 __device__ __forceinline__ float h2f_bits(uint32_t h) {
   return __uint_as_float((h & 0x7FFFu) << 13) * 5.192296858534828e+33f * ((h & 0x8000u) ? -1.0f : 1.0f);
 }
-
-// int -> fp32 for |v| < 2^22 with one integer add and one FP add: 1.5 * 2^23
-// + v has v in its low mantissa bits.
+// int -> fp32 for |v| < 2^22 with one integer add and one FP add.
 __device__ __forceinline__ float i2f_small(int v) { return __int_as_float(0x4B400000 + v) - 12582912.0f; }
 
 __device__ __forceinline__ int job_of(const MArgs& a, int t) {
@@ -96,18 +104,42 @@ __device__ __forceinline__ int job_of(const MArgs& a, int t) {
   return jb;
 }
 
+// Word offset of 16-byte chunk c (0..3) of staged code row r (64 bytes a row):
+// rows 2, 3 (mod 4) swap chunk pairs, so the rows read by one half-warp's
+// 8-byte fragment loads fall on distinct banks.
+__device__ __forceinline__ int code_off(int r, int c) { return r * 16 + ((c ^ (((r >> 1) & 1) << 1)) << 2); }
+
+// f16 (1024 + q_f) pairs for rows g8 (lo_row) / g8 + 8 (hi_row) of two
+// channels whose refinement words are wa, wb (bits b_f*r + off hold row r).
+template <int BF>
+__device__ __forceinline__ void qf_frag(uint32_t wa, uint32_t wb, int g8, int off, uint32_t& lo_row,
+                                        uint32_t& hi_row) {
+  if constexpr (BF == 2) {
+    const uint32_t xa = wa >> (2 * g8 + off), xb = wb >> (2 * g8 + off);
+    lo_row = (__byte_perm(xa, xb, 0x5410) & 0x00030003u) | 0x64006400u;  // row g8: bits 0-1 of each half
+    hi_row = (__byte_perm(xa, xb, 0x7632) & 0x00030003u) | 0x64006400u;  // row g8 + 8: bits 16-17
+  } else {
+    const uint32_t xa = wa >> (g8 + off), xb = wb >> (g8 + off);
+    const uint32_t p = __byte_perm(xa, xb, 0x5410);  // row g8 at bit 0, row g8 + 8 at bit 8 of each half
+    lo_row = (p & 0x00010001u) | 0x64006400u;
+    hi_row = ((p >> 8) & 0x00010001u) | 0x64006400u;
+  }
+}
+
 template <int SPW>
 struct MCfg {
-  static constexpr int kStages = SPW == 1 ? 4 : 3;
-  static constexpr int SW = SPW * kSliceStage;  // ring words per warp and stage
+  static constexpr int kStages = SPW == 1 ? 8 : 6;
+  static constexpr int SW = SPW * kSliceWords;  // ring words per warp and stage
   static size_t smem_bytes(int W) {
-    return sizeof(uint32_t) * (static_cast<size_t>(W) * kStages * SW + 2 * static_cast<size_t>(W) * SPW * 2 * kSelCap +
-                               static_cast<size_t>(W) * SPW * 2 * kRefSlot + 2 * static_cast<size_t>(W) * kRows);
+    return sizeof(uint32_t) * (static_cast<size_t>(W) * kStages * SW           // rings
+                               + static_cast<size_t>(W) * SPW * kCorrList       // refinement rows (issue job)
+                               + static_cast<size_t>(W) * SPW * kCorrList / 2   // listed channels (u16)
+                               + 2 * static_cast<size_t>(W) * kRows);           // row partials
   }
 };
 
-template <int SPW>
-__global__ void __launch_bounds__(512, 1)
+template <int SPW, int BF>
+__global__ void __launch_bounds__(kMaxWarps * 32, 1)
 gemv_mma_kernel(const __grid_constant__ MArgs a) {
   using C = MCfg<SPW>;
   constexpr int kStages = C::kStages, SW = C::SW;
@@ -116,23 +148,27 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, tig = lane & 3;
   const int ks = blockIdx.x % a.ksplit, crow = blockIdx.x / a.ksplit, ncta = gridDim.x / a.ksplit;
   uint32_t* ring = sm + warp * kStages * SW;
-  uint32_t* after_ring = sm + W * kStages * SW;
-  float* selx = reinterpret_cast<float*>(after_ring) + warp * SPW * 2 * kSelCap;      // [SPW][2][kSelCap]
-  int* selp = reinterpret_cast<int*>(after_ring + W * SPW * 2 * kSelCap) + warp * SPW * 2 * kSelCap;
-  int* selr = reinterpret_cast<int*>(after_ring + 2 * W * SPW * 2 * kSelCap) + warp * SPW * 2 * kRefSlot;
-  float* red = reinterpret_cast<float*>(after_ring + 2 * W * SPW * 2 * kSelCap + W * SPW * 2 * kRefSlot);  // [2][W][16]
+  int* selr = reinterpret_cast<int*>(sm + W * kStages * SW) + warp * SPW * kCorrList;           // [SPW][32]
+  uint16_t* mylist = reinterpret_cast<uint16_t*>(sm + W * kStages * SW + W * SPW * kCorrList) +
+                     warp * SPW * kCorrList;                                                      // [SPW][32]
+  float* red = reinterpret_cast<float*>(sm + W * kStages * SW + W * SPW * kCorrList + W * SPW * kCorrList / 2);
 
   const int slice0 = (ks * W + warp) * SPW;
   const int myslot = tig >> 1, myrow = g8 + 8 * (tig & 1);
   const bool even = (tig & 1) == 0;
+  const float m_f = static_cast<float>((1 << BF) - 1) * 0.5f;
+  const uint32_t fmask = (1u << BF) - 1u;
 
-  // ---- per-warp setup: B fragments, group scalars, selection lists
+  // ---- per-warp setup: B fragments, group scalars, selection lists, the
+  // correction MMA's B fragments (x of the listed channels, high and low)
   uint32_t bf[SPW][8][2];
-  float fsc[SPW], gsm[SPW];
-  int ns[SPW][2];
+  uint32_t cb[SPW][2][2];
+  float fsc[SPW], gsm[SPW], cconst[SPW];
+  int nsl[SPW], psl[SPW];
 #pragma unroll
   for (int sp = 0; sp < SPW; ++sp) {
-    const uint32_t* A = a.act + static_cast<size_t>(slice0 + sp) * sfd::kAct2Words;
+    const int slice = slice0 + sp;
+    const uint32_t* A = a.act + static_cast<size_t>(slice) * sfd::kAct2Words;
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
       const uint2 v = reinterpret_cast<const uint2*>(A)[m * 32 + lane];
@@ -141,92 +177,111 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
     }
     fsc[sp] = __uint_as_float(A[sfd::kAct2Info + 2 * myslot]);
     gsm[sp] = __uint_as_float(A[sfd::kAct2Info + 2 * myslot + 1]);
-    const int prefix = static_cast<int>(A[sfd::kAct2Info + 4]);
-    // lanes 0..7 own one mask word each (32 channels); words 0..3 = group 0
-    const uint32_t mw = lane < 8 ? A[sfd::kAct2Mask + lane] : 0u;
-    const int c = __popc(mw);
-    int incl = c;
+    psl[sp] = static_cast<int>(A[sfd::kAct2Info + 4]);
+    nsl[sp] = static_cast<int>(A[sfd::kAct2Info + 5]);
+    {
+      const uint32_t mw = lane < 8 ? A[sfd::kAct2Mask + lane] : 0u;
+      const int c = __popc(mw);
+      int incl = c;
 #pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const int n0 = __shfl_sync(0xffffffffu, incl, 3);
-    const int nall = __shfl_sync(0xffffffffu, incl, 7);
-    ns[sp][0] = n0;
-    ns[sp][1] = nall - n0;
-    if (lane < 8) {
-      const int slot = lane >> 2;
-      int r = incl - c - (slot ? n0 : 0);  // rank inside the group's list
-      int p = prefix + incl - c;           // position in the selection (idx order)
+      for (int o = 1; o < 8; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int r = incl - c;
       uint32_t mm = mw;
       while (mm) {
         const int bit = __ffs(mm) - 1;
         mm &= mm - 1u;
-        const int ch = 32 * lane + bit;  // channel inside the slice
-        const int e = (sp * 2 + slot) * kSelCap + r;
-        selx[e] = sfd::bf16_bits_to_float(a.x[256 * (slice0 + sp) + ch]);
-        selp[e] = (p << 8) | ch;
+        if (r < kCorrList) mylist[sp * kCorrList + r] = static_cast<uint16_t>(32 * lane + bit);
         ++r;
-        ++p;
       }
     }
+    __syncwarp();
+    const int nl = min(nsl[sp], kCorrList);
+    uint32_t hl = 0;  // lane k: (high, low) halves of x of listed channel k
+    int grp = -1;     // and its group inside the slice
+    if (lane < nl) {
+      const int ch = mylist[sp * kCorrList + lane];
+      const float xv = sfd::bf16_bits_to_float(a.x[256 * slice + ch]);
+      const __half hi = __float2half_rn(xv);
+      const __half lo = __float2half_rn(xv - __half2float(hi));
+      hl = static_cast<uint32_t>(__half_as_ushort(hi)) | (static_cast<uint32_t>(__half_as_ushort(lo)) << 16);
+      grp = ch >> 7;
+    }
+    {
+      const float part = lane < nl ? __half2float(__ushort_as_half(static_cast<unsigned short>(hl & 0xFFFFu))) +
+                                         __half2float(__ushort_as_half(static_cast<unsigned short>(hl >> 16)))
+                                   : 0.0f;
+      float x0 = grp == 0 ? part : 0.0f, x1 = grp == 1 ? part : 0.0f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        x0 += __shfl_xor_sync(0xffffffffu, x0, o);
+        x1 += __shfl_xor_sync(0xffffffffu, x1, o);
+      }
+      cconst[sp] = -(1024.0f + m_f) * (myslot ? x1 : x0);
+    }
+    // column n of the correction MMA = (group n / 2, part n % 2)
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        uint32_t v = 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int k = 16 * kb + 2 * tig + 8 * r + h;  // < 32: a lane of the warp
+          const uint32_t hk = __shfl_sync(0xffffffffu, hl, k);
+          const int gk = __shfl_sync(0xffffffffu, grp, k);
+          if (g8 < 4 && k < nl && gk == (g8 >> 1)) v |= ((g8 & 1) ? (hk >> 16) : (hk & 0xFFFFu)) << (16 * h);
+        }
+        cb[sp][kb][r] = v;
+      }
   }
-  __syncwarp();
 
-  const float m_f = static_cast<float>((1 << a.b_f) - 1) * 0.5f;
-  const float two_bf = static_cast<float>(1 << a.b_f);
-  const uint32_t fmask = (1u << a.b_f) - 1u;
   const size_t row_words = static_cast<size_t>(a.K) / 16;
   const int last = a.njobs - 1;
   const int total_tiles = a.job[last].tile_begin + a.job[last].N / kRows;
-  const int my_tiles = crow < total_tiles ? (total_tiles - crow + ncta - 1) / ncta : 0;
+  // a contiguous block of tiles per CTA: consecutive tiles read consecutive
+  // words of each selected channel's refinement row (one sector serves 8 or 16)
+  const int per_cta = (total_tiles + ncta - 1) / ncta;
+  const int t_begin = crow * per_cta;
+  const int my_tiles = max(0, min(total_tiles, t_begin + per_cta) - t_begin);
   int issue_job = -1;
 
   auto issue = [&](int i) {
     const int st = i % kStages;
-    const int t = crow + i * ncta;
+    const int t = t_begin + i;
     const int jb = job_of(a, t);
     const MJob& J = a.job[jb];
     const int row0 = (t - J.tile_begin) * kRows;
-    if (jb != issue_job) {  // refinement rows of the staged list entries, for this matrix
+    if (jb != issue_job) {  // refinement rows of the listed channels, for this matrix
       issue_job = jb;
       if (J.ref_rows) {
 #pragma unroll
         for (int sp = 0; sp < SPW; ++sp)
-#pragma unroll
-          for (int slot = 0; slot < 2; ++slot)
-            if (lane < kRefSlot && lane < ns[sp][slot]) {
-              const int pc = selp[(sp * 2 + slot) * kSelCap + lane];
-              selr[(sp * 2 + slot) * kRefSlot + lane] =
-                  J.row_of ? J.row_of[pc >> 8] : 256 * (slice0 + sp) + (pc & 255);
-            }
+          if (lane < min(nsl[sp], kCorrList))
+            selr[sp * kCorrList + lane] =
+                J.row_of ? J.row_of[psl[sp] + lane] : 256 * (slice0 + sp) + mylist[sp * kCorrList + lane];
       }
       __syncwarp();
     }
 #pragma unroll
     for (int sp = 0; sp < SPW; ++sp) {
-      uint32_t* base = ring + st * SW + sp * kSliceStage;
+      uint32_t* base = ring + st * SW + sp * kSliceWords;
       const int slice = slice0 + sp;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int row = (lane >> 2) + 8 * h;
-        cp_async16(base + row * kCodeStr + 4 * (lane & 3),
-                   J.res + static_cast<size_t>(row0 + row) * row_words + 16 * slice + 4 * (lane & 3));
+        const int row = (lane >> 2) + 8 * h, c = lane & 3;
+        cp_async16(base + code_off(row, c), J.res + static_cast<size_t>(row0 + row) * row_words + 16 * slice + 4 * c);
       }
       if (lane < 8) {  // (group, scale|zero, half of the 16 rows)
         const int grp = lane >> 2, arr = (lane >> 1) & 1, hf = lane & 1;
         const uint16_t* src = (arr ? J.zero : J.scale) + static_cast<size_t>(2 * slice + grp) * J.N + row0 + 8 * hf;
-        cp_async16(reinterpret_cast<uint16_t*>(base + kRows * kCodeStr) + (grp * 2 + arr) * 16 + 8 * hf, src);
+        cp_async16(reinterpret_cast<uint16_t*>(base + 256) + (grp * 2 + arr) * 16 + 8 * hf, src);
       }
-      if (J.ref_rows) {
-        const int slot = lane >> 4, q = lane & (kRefSlot - 1);
-        const int n = slot ? ns[sp][1] : ns[sp][0];
-        if (q < n)
-          cp_async4(base + kRows * kCodeStr + kSzWords + lane,
-                    J.ref_rows + static_cast<size_t>(selr[(sp * 2 + slot) * kRefSlot + q]) * J.unit_words +
-                        ((row0 * a.b_f) >> 5));
-      }
+      if (J.ref_rows && lane < min(nsl[sp], kCorrList))
+        cp_async4(base + 288 + lane,
+                  J.ref_rows + static_cast<size_t>(selr[sp * kCorrList + lane]) * J.unit_words + ((row0 * BF) >> 5));
     }
   };
 
@@ -241,21 +296,19 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
     cp_async_wait<kStages - 1>();
     __syncwarp();
     const int st = i % kStages;
-    const int t = crow + i * ncta;
-    const int jb = job_of(a, t);
-    const MJob& J = a.job[jb];
+    const int t = t_begin + i;
+    const MJob& J = a.job[job_of(a, t)];
     const int row0 = (t - J.tile_begin) * kRows;
-    const int sh = ((row0 * a.b_f) & 31) + a.b_f * myrow;  // this lane's row in a refinement word
+    const int roff = (row0 * BF) & 31;
     float v = 0.0f;
 #pragma unroll
     for (int sp = 0; sp < SPW; ++sp) {
-      const uint32_t* base = ring + st * SW + sp * kSliceStage;
+      const uint32_t* base = ring + st * SW + sp * kSliceWords;
       // code words: rows g8 and g8 + 8, words 2 tig, 2 tig + 1 of each group
-      const uint2 r0a = *reinterpret_cast<const uint2*>(base + g8 * kCodeStr + 2 * tig);
-      const uint2 r0b = *reinterpret_cast<const uint2*>(base + g8 * kCodeStr + 8 + 2 * tig);
-      const uint2 r1a = *reinterpret_cast<const uint2*>(base + (g8 + 8) * kCodeStr + 2 * tig);
-      const uint2 r1b = *reinterpret_cast<const uint2*>(base + (g8 + 8) * kCodeStr + 8 + 2 * tig);
-      // two independent accumulator chains (even / odd k-steps), added at the end
+      const uint2 r0a = *reinterpret_cast<const uint2*>(base + code_off(g8, tig >> 1) + 2 * (tig & 1));
+      const uint2 r0b = *reinterpret_cast<const uint2*>(base + code_off(g8, 2 + (tig >> 1)) + 2 * (tig & 1));
+      const uint2 r1a = *reinterpret_cast<const uint2*>(base + code_off(g8 + 8, tig >> 1) + 2 * (tig & 1));
+      const uint2 r1b = *reinterpret_cast<const uint2*>(base + code_off(g8 + 8, 2 + (tig >> 1)) + 2 * (tig & 1));
       int d[4] = {0, 0, 0, 0}, e[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
@@ -278,32 +331,49 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
       const float send = even ? fmaf(f3, 256.0f, f2) : 65536.0f * f0;
       const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
       const float P = even ? fmaf(f1, 256.0f, f0) + recv : fmaf(65536.0f, f2, recv);
-      const uint16_t* szs = reinterpret_cast<const uint16_t*>(base + kRows * kCodeStr);
+      const uint16_t* szs = reinterpret_cast<const uint16_t*>(base + 256);
       const float sc = h2f_bits(szs[(myslot * 2) * 16 + myrow]);
       const float zz = h2f_bits(szs[(myslot * 2 + 1) * 16 + myrow]);
-      float tsum = fmaf(two_bf * fsc[sp], P, (m_f - zz) * gsm[sp]);
-      if (J.ref_rows) {
-        // sum_j x_j (q_f - m_f) over the group's selected channels: the staged
-        // entries two at a time (a missing second entry has x = 0 and reads a
-        // staged word that is never used), the rest from the refinement rows
-        const int n = myslot ? ns[sp][1] : ns[sp][0];
-        const int nst = min(max(ns[sp][0], ns[sp][1]), kRefSlot);
-        const float* lx = selx + (sp * 2 + myslot) * kSelCap;
-        const uint32_t* rw = base + kRows * kCodeStr + kSzWords + myslot * kRefSlot;
-        float c0 = 0.0f, c1 = 0.0f;
-        for (int q = 0; q < nst; q += 2) {
-          const float x0 = q < n ? lx[q] : 0.0f, x1 = q + 1 < n ? lx[q + 1] : 0.0f;
-          const uint32_t w0 = rw[q], w1 = rw[q + 1];
-          c0 = fmaf(x0, i2f_small(static_cast<int>((w0 >> sh) & fmask)) - m_f, c0);
-          c1 = fmaf(x1, i2f_small(static_cast<int>((w1 >> sh) & fmask)) - m_f, c1);
+      float tsum = fmaf(static_cast<float>(1 << BF) * fsc[sp], P, (m_f - zz) * gsm[sp]);
+      if (J.ref_rows && nsl[sp] > 0) {
+        const uint32_t* refw = base + 288;
+        float c4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        const int nl = min(nsl[sp], kCorrList);
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+          if (16 * kb < nl) {  // uniform over the warp
+            // entries at or beyond nl hold stale words: their B columns are zero
+            const int k0 = 16 * kb + 2 * tig;
+            uint32_t qa0, qa1, qa2, qa3;
+            qf_frag<BF>(refw[k0], refw[k0 + 1], g8, roff, qa0, qa1);
+            qf_frag<BF>(refw[k0 + 8], refw[k0 + 9], g8, roff, qa2, qa3);
+            mma_f16(c4, qa0, qa1, qa2, qa3, cb[sp][kb][0], cb[sp][kb][1]);
+          }
         }
-        tsum += c0 + c1;
-        for (int q = kRefSlot; q < n; ++q) {  // beyond the staged entries (rare)
-          const int pc = selp[(sp * 2 + myslot) * kSelCap + q];
-          const int rid = J.row_of ? J.row_of[pc >> 8] : 256 * (slice0 + sp) + (pc & 255);
-          const uint32_t word = J.ref_rows[static_cast<size_t>(rid) * J.unit_words + ((row0 * a.b_f) >> 5)];
-          tsum = fmaf(lx[q], i2f_small(static_cast<int>((word >> sh) & fmask)) - m_f, tsum);
+        // lane (g8, t), t < 2, holds group t's (high, low) columns for rows g8 and g8 + 8
+        const float u0 = __shfl_sync(0xffffffffu, c4[0] + c4[1], 4 * g8 + myslot);
+        const float u1 = __shfl_sync(0xffffffffu, c4[2] + c4[3], 4 * g8 + myslot);
+        float corr = ((tig & 1) ? u1 : u0) + cconst[sp];
+        // channels beyond the tensor-core list (more than kCorrList selected in the slice)
+        for (int k = kCorrList; k < nsl[sp]; ++k) {
+          const uint32_t* A = a.act + static_cast<size_t>(slice0 + sp) * sfd::kAct2Words;
+          int kk = k, ch = -1;
+          for (int wdx = 0; wdx < 8 && ch < 0; ++wdx) {
+            uint32_t mm = A[sfd::kAct2Mask + wdx];
+            const int c = __popc(mm);
+            if (kk < c) {
+              for (int q = 0; q < kk; ++q) mm &= mm - 1u;
+              ch = 256 * (slice0 + sp) + 32 * wdx + __ffs(mm) - 1;
+            }
+            kk -= c;
+          }
+          if (((ch >> 7) & 1) != myslot) continue;
+          const int rr = J.row_of ? J.row_of[psl[sp] + k] : ch;
+          const uint32_t word = J.ref_rows[static_cast<size_t>(rr) * J.unit_words + ((row0 * BF) >> 5)];
+          const float xv = sfd::bf16_bits_to_float(a.x[ch]);
+          corr = fmaf(xv, i2f_small(static_cast<int>((word >> (roff + BF * myrow)) & fmask)) - m_f, corr);
         }
+        tsum += corr;
       }
       v = fmaf(sc, tsum, v);
     }
@@ -359,7 +429,6 @@ extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, c
   MArgs a{};
   a.njobs = count;
   a.K = K;
-  a.b_f = b_f;
   a.ksplit = ksplit;
   a.x = x;
   a.act = static_cast<const uint32_t*>(act);
@@ -396,22 +465,21 @@ extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, c
     if (ksplit > 1) SF_CHECK_CUDA(cudaMemsetAsync(jobs[i].y, 0, sizeof(float) * W->N, s));
   }
   const int warps = K / 256 / (spw * ksplit);
-  const int threads = 32 * warps;
   const int sms = sf::sm_count();
   const int nrow_cta = std::max(1, std::min(row_tiles, std::max(1, sms / ksplit)));
-  sf_status st = SF_OK;
+  const dim3 grid(nrow_cta * ksplit), block(32 * warps);
+  auto launch = [&](auto kern, size_t smem) -> sf_status {
+    SF_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+    kern<<<grid, block, smem, s>>>(a);
+    return sf::check_launch("gemv_mma_kernel");
+  };
+  sf_status st;
   if (spw == 1) {
     const size_t smem = MCfg<1>::smem_bytes(warps);
-    SF_CHECK_CUDA(cudaFuncSetAttribute(gemv_mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem)));
-    gemv_mma_kernel<1><<<nrow_cta * ksplit, threads, smem, s>>>(a);
-    st = sf::check_launch("gemv_mma_kernel");
+    st = b_f == 2 ? launch(gemv_mma_kernel<1, 2>, smem) : launch(gemv_mma_kernel<1, 1>, smem);
   } else {
     const size_t smem = MCfg<2>::smem_bytes(warps);
-    SF_CHECK_CUDA(cudaFuncSetAttribute(gemv_mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem)));
-    gemv_mma_kernel<2><<<nrow_cta * ksplit, threads, smem, s>>>(a);
-    st = sf::check_launch("gemv_mma_kernel");
+    st = b_f == 2 ? launch(gemv_mma_kernel<2, 2>, smem) : launch(gemv_mma_kernel<2, 1>, smem);
   }
   if (st != SF_OK) return st;
   for (int i = 0; i < count; ++i)

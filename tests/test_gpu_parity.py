@@ -270,11 +270,12 @@ def _kv(sf, Hkv, T, d, seed, n_out=4):
 
 
 @pytest.mark.parametrize("Hq,Hkv,T,pct", [(8, 2, 1000, 1), (32, 8, 4099, 1), (4, 4, 77, 10), (16, 2, 33, 100),
-                                          (8, 1, 512, 0), (8, 2, 8192, 30), (8, 2, 40961, 1), (4, 1, 32768, 2)])
+                                          (8, 1, 512, 0), (8, 2, 8192, 30), (8, 2, 40961, 1), (4, 1, 32768, 2),
+                                          (4, 1, 70001, 1), (8, 8, 65536, 1)])
 def test_attn_small(sf, Hq, Hkv, T, pct):
-    """Covers both selection kernels (scores held in registers up to T = 32768,
-    streamed beyond), the pairwise ranking of few candidates and the radix
-    ranking of more than 1024 (30% of 8192)."""
+    """Covers both selection kernels (scores in registers over a cluster of up
+    to 8 CTAs per head up to T = 65536, streamed beyond), the pairwise ranking
+    of few candidates and the radix ranking of many (30% of 8192)."""
     d = 128
     kv, ok, ov = _kv(sf, Hkv, T, d, 3000 + T)
     qb = gen_query(4000 + T, Hq, d)
@@ -516,10 +517,12 @@ def test_gemv_batch1_jobs_with_caches(sf, K, Ns, cap_pct, pct):
         m["cache"].close()
 
 
-def test_gemv_batch1_store_mode(sf):
-    N, K, G = 1024, 8192, 128
-    W = gen_weight(1400, N, K)
-    qw = sf.quantize_nested(dev(W), G, 2, 1)
+@pytest.mark.parametrize("N,K,b_f", [(1024, 8192, 1), (512, 1024, 2), (2048, 4096, 1)])
+def test_gemv_batch1_store_mode(sf, N, K, b_f):
+    """Refinement read from the HBM store; b_f = 1 packs 16 rows in half a word."""
+    G = 128
+    W = gen_weight(1400 + K, N, K)
+    qw = sf.quantize_nested(dev(W), G, 2, b_f)
     x = gen_activations(1401, 1, K, outlier_channels(1402, K, 40), 30.0)
     k = count_fraction(5, K)
     xd = bf16_dev(x)
@@ -530,7 +533,7 @@ def test_gemv_batch1_store_mode(sf):
     sf.select_topk_act(xd, k, idx, n, act)
     sf.gemv_refine_batch1([(qw, None, True, y)], xd, act)
     torch.cuda.synchronize()
-    y_ref, a = ogemv.gemv_refine(oquant.quantize_nested(W, G, 2, 1), x, oselect.select_topk(x, k))
+    y_ref, a = ogemv.gemv_refine(oquant.quantize_nested(W, G, 2, b_f), x, oselect.select_topk(x, k))
     _check_gemv(y.cpu().numpy()[None, :], y_ref, a)
 
 
