@@ -332,7 +332,7 @@ __device__ void find_bin_from_top(const int* hist, int nb, int kk, int* out) {
 // norm and the binary exponent of max |q|; flags the KV group when the
 // nonzero q exponents span more than the exact-key precondition allows.
 __device__ void select_q_prologue(const uint16_t* __restrict__ q, int h, int g, double* qd, double* l1_out,
-                                  int* qe_out, int32_t* __restrict__ status) {
+                                  int* qe_out, int32_t* __restrict__ status, int* span_out = nullptr) {
   const int tid = threadIdx.x;
   for (int d = tid; d < D; d += blockDim.x)
     qd[d] = static_cast<double>(sfd::bf16_bits_to_float(q[static_cast<size_t>(h) * D + d]));
@@ -359,6 +359,7 @@ __device__ void select_q_prologue(const uint16_t* __restrict__ q, int h, int g, 
     if (tid == 0) {
       *l1_out = l1;
       *qe_out = emax >= emin ? emax : 0;  // binary exponent of max |q| (frexp convention)
+      if (span_out) *span_out = emax >= emin ? emax - emin : 0;  // binades spanned by the nonzero q
       // 53 - 9 - b - log2(d) with b = 4, d = 128
       if (emax >= emin && emax - emin > 53 - 9 - 4 - 7) atomicOr(status + g, 1);
     }
@@ -548,6 +549,8 @@ attn_select_compact_kernel(const uint16_t* __restrict__ q, int T, int k, const f
 constexpr int kFinThreads = 512;
 constexpr int kFinKeys = 2048;     // candidates ranked pairwise from shared memory
 constexpr int kFinChunks = 4096;   // chunk prefix sums in shared memory (T <= 2^24)
+constexpr int kFinList = 4096;     // listed (token, score) pairs cached in shared memory
+constexpr size_t kFinDynSmem = static_cast<size_t>(kFinList) * 8;
 
 template <int GRP>
 __global__ void __launch_bounds__(kFinThreads)
@@ -568,25 +571,44 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   __shared__ int cpre[kFinChunks];
   __shared__ double keys[kFinKeys];
   __shared__ double qd[D];
-  __shared__ float qs[D];
-  __shared__ float qsum_sh;
   __shared__ int scan_scratch[64];
   __shared__ int binfo[2];
   __shared__ double l1_sh;
-  __shared__ int qe_sh;
+  __shared__ int qe_sh, span_sh;
   __shared__ int cnt_sh;  // read remotely
+  __shared__ uint32_t qpl[3][8][4];  // byte planes of the fixed-point q, in code-extraction order
+  __shared__ long long qxsum_sh;
+  extern __shared__ int fin_dyn[];
+  int* ltok = fin_dyn;                                      // [kFinList]
+  float* lsc = reinterpret_cast<float*>(fin_dyn + kFinList);  // [kFinList]
   const float* sc = score + static_cast<size_t>(h) * T;
   int32_t* L = list + static_cast<size_t>(h) * T;  // concatenated list, token order
   int32_t* F = cand + static_cast<size_t>(h) * T;  // candidates (reuses the chunk lists once L is built)
   double* kp = kap + static_cast<size_t>(h) * T;
   const int cap = GRP * k;
 
-  select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status);
-  for (int d = tid; d < D; d += kFinThreads) qs[d] = static_cast<float>(qd[d]);
-  if (tid == 0) {
-    float acc = 0.0f;  // sequential fp32 order, d ascending (as the refined-score pass always used)
-    for (int d = 0; d < D; ++d) acc += static_cast<float>(qd[d]);
-    qsum_sh = acc;
+  select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status, &span_sh);
+  // q as 24-bit fixed point X = q 2^(23 - qe): exact for every nonzero q
+  // within 15 binades of the largest (bf16 has 8 significant bits)
+  const bool int_keys = span_sh <= 15;
+  if (int_keys) {
+    if (tid < 96) {
+      const int p = tid / 32, wi = (tid / 4) & 7, kq = tid & 3;
+      uint32_t v = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int X = static_cast<int>(ldexp(qd[16 * wi + kq + 4 * b], 23 - qe_sh));
+        v |= ((static_cast<uint32_t>(X) >> (8 * p)) & 0xFFu) << (8 * b);
+      }
+      qpl[p][wi][kq] = v;
+    }
+    if (tid < 32) {
+      long long sx = 0;
+      for (int d = tid; d < D; d += 32) sx += static_cast<long long>(ldexp(qd[d], 23 - qe_sh));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, o);
+      if (tid == 0) qxsum_sh = sx;
+    }
   }
   const double eps_s = select_eps(static_cast<double>(smax[g]), l1_sh, qe_sh, __uint_as_float(amaxu[h]));
   uint32_t b1;
@@ -594,7 +616,8 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   float f_low;
   select_band(hist + static_cast<size_t>(h) * kHistBins, k, eps_s, hr, scan_scratch, binfo, &b1, &kk, &f_low);
 
-  // 1. concatenate the chunk lists (token order)
+  // 1. concatenate the chunk lists (token order); with their fast scores in
+  //    shared memory when they fit
   const int32_t* counts = cand + static_cast<size_t>(gridDim.x) * T + static_cast<size_t>(h) * nchunks;
   int m = 0;
   for (int base = 0; base < nchunks; base += kFinThreads) {
@@ -613,9 +636,18 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
       if (cpre[mid] <= e) lo = mid;
       else hi = mid - 1;
     }
-    L[e] = cand[static_cast<size_t>(h) * T + static_cast<size_t>(lo) * kChunk + (e - cpre[lo])];
+    const int t = cand[static_cast<size_t>(h) * T + static_cast<size_t>(lo) * kChunk + (e - cpre[lo])];
+    if (m <= kFinList) {
+      ltok[e] = t;
+      lsc[e] = sc[t];
+    } else {
+      L[e] = t;
+    }
   }
   __syncthreads();
+  const bool cached = m <= kFinList;
+  auto tok_of = [&](int e) { return cached ? ltok[e] : L[e]; };
+  auto score_of = [&](int e) { return cached ? lsc[e] : sc[L[e]]; };
 
   // 2. tau: two radix passes (11 + 11 bits) over the listed scores of bin b1
   uint32_t pre = b1 << 22;
@@ -625,7 +657,7 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
     __syncthreads();
     const uint32_t pmask = pass == 0 ? 0xFFC00000u : 0xFFFFF800u;
     for (int e = tid; e < m; e += kFinThreads) {
-      const uint32_t key = okey32(sc[L[e]]);
+      const uint32_t key = okey32(score_of(e));
       if ((key & pmask) == pre) atomicAdd(&hr[(key >> shift) & 2047u], 1);
     }
     __syncthreads();
@@ -640,10 +672,10 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   int ncand = 0;
   for (int base = 0; base < m; base += kFinThreads) {
     const int e = base + tid;
-    const bool p = e < m && sc[L[e]] >= fthr;
+    const bool p = e < m && score_of(e) >= fthr;
     int tot;
     const int pos = sfd::block_exclusive_scan(p ? 1 : 0, scan_scratch, &tot);
-    if (p) F[ncand + pos] = L[e];
+    if (p) F[ncand + pos] = tok_of(e);
     ncand += tot;
   }
   __syncthreads();
@@ -659,20 +691,41 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
     const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
     const double sv = static_cast<double>(sfd::half_bits_to_float(k_scale[row]));
     const double z = static_cast<double>(sfd::half_bits_to_float(k_zero[row]));
-    double E[4] = {0.0, 0.0, 0.0, 0.0};
+    double key;
+    if (int_keys) {
+      // sum_d c_d X_d exactly with byte-plane dot products; E = 4 sum c q +
+      // (1.5 - z) sum q is exact in fp64, so one fma returns it exactly
+      unsigned d0 = 0, d1 = 0;
+      int d2 = 0;
 #pragma unroll
-    for (int wi = 0; wi < 8; ++wi) {
-      const uint32_t word = w[wi];
-#pragma unroll 1
-      for (int jj = 0; jj < 4; ++jj)
+      for (int wi = 0; wi < 8; ++wi)
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int j = 4 * jj + u;
-          const double c = static_cast<double>((word >> (2 * j)) & 3u);
-          E[u] = fma(qd[16 * wi + j], c * 4.0 + 1.5 - z, E[u]);
+        for (int kq = 0; kq < 4; ++kq) {
+          const unsigned c = (w[wi] >> (2 * kq)) & 0x03030303u;
+          d0 = __dp4a(c, qpl[0][wi][kq], d0);
+          d1 = __dp4a(c, qpl[1][wi][kq], d1);
+          d2 = __dp4a(static_cast<int>(c), static_cast<int>(qpl[2][wi][kq]), d2);
         }
+      const long long P = static_cast<long long>(d0) + 256ll * d1 + 65536ll * d2;
+      const double cq = ldexp(static_cast<double>(P), qe_sh - 23);
+      const double qsum = ldexp(static_cast<double>(qxsum_sh), qe_sh - 23);
+      key = sv * fma(1.5 - z, qsum, 4.0 * cq);
+    } else {
+      double E[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+      for (int wi = 0; wi < 8; ++wi) {
+        const uint32_t word = w[wi];
+#pragma unroll 1
+        for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int j = 4 * jj + u;
+            const double c = static_cast<double>((word >> (2 * j)) & 3u);
+            E[u] = fma(qd[16 * wi + j], c * 4.0 + 1.5 - z, E[u]);
+          }
+      }
+      key = sv * ((E[0] + E[1]) + (E[2] + E[3]));
     }
-    const double key = sv * ((E[0] + E[1]) + (E[2] + E[3]));
     kp[i] = key;
     if (ncand <= kFinKeys) keys[i] = key;
   }
@@ -717,7 +770,6 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   // 6. union, ascending: CTA r of the cluster compacts words [r wper, (r+1) wper)
   const int wper = (words_t + GRP - 1) / GRP;
   const int w0 = min(words_t, rank * wper), w1 = min(words_t, w0 + wper);
-  int mycnt = 0;
   {
     const int chunk = (w1 - w0 + kFinThreads - 1) / kFinThreads;
     const int a0 = min(w1, w0 + tid * chunk), a1 = min(w1, a0 + chunk);
@@ -733,7 +785,6 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
       if (r < rank) off += cr;
       U += cr;
     }
-    mycnt = U;
     int32_t* out = sel_out + static_cast<size_t>(g) * cap;
     pos += off;
     for (int w = a0; w < a1; ++w) {
@@ -746,81 +797,7 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
     }
     if (rank == 0 && tid == 0) sel_n[g] = status[g] ? -1 - U : U;
   }
-  __threadfence();
-  cl.sync();  // 3: the union list is complete; no shared-memory access across CTAs after this
-
-  // 7. refined scores of this head for the union tokens: full 4-bit codes
-  const int U = mycnt;
-  const int32_t* ul = sel_out + static_cast<size_t>(g) * cap;
-  const float qsum = qsum_sh;
-  for (int u = tid; u < U; u += kFinThreads) {
-    const int t = ul[u];
-    const size_t row = static_cast<size_t>(g) * T + t;
-    const uint4* r4 = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
-    const uint4* f4 = reinterpret_cast<const uint4*>(k_ref + row * kWordsPerRow);
-    const uint4 ra = r4[0], rb = r4[1], fa = f4[0], fb = f4[1];
-    const uint32_t wr[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-    const uint32_t wf[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
-    float P0 = 0.0f, P1 = 0.0f;
-#pragma unroll
-    for (int wi = 0; wi < 8; ++wi) {
-      const uint32_t xr = wr[wi], xf = wf[wi];
-#pragma unroll 2
-      for (int jj = 0; jj < 8; ++jj) {
-        const int j = 2 * jj;
-        P0 = fmaf(qs[16 * wi + j], static_cast<float>(((xr >> (2 * j)) & 3u) * 4u + ((xf >> (2 * j)) & 3u)), P0);
-        P1 = fmaf(qs[16 * wi + j + 1],
-                  static_cast<float>(((xr >> (2 * j + 2)) & 3u) * 4u + ((xf >> (2 * j + 2)) & 3u)), P1);
-      }
-    }
-    const float sv = sfd::half_bits_to_float(k_scale[row]);
-    const float z = sfd::half_bits_to_float(k_zero[row]);
-    score[static_cast<size_t>(h) * T + t] = (sv * fmaf(-z, qsum, P0 + P1)) * kInvSqrtD;
-  }
-}
-
-// ---- refined scores of the refined tokens ------------------------------------
-// For every token in a KV group's union, the scores of the group's query heads
-// with the full-code key k' = s (4 c_r + c_f - z) replace the resident scores
-// in the score buffer (after the selection has used them).  One warp per token,
-// lanes over 4 dims each.
-template <int GRP>
-__global__ void __launch_bounds__(256)
-attn_refine_scores_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
-                          const uint32_t* __restrict__ k_ref, const uint16_t* __restrict__ k_scale,
-                          const uint16_t* __restrict__ k_zero, int T, int cap, const int32_t* __restrict__ sel_out,
-                          const int32_t* __restrict__ sel_n, float* __restrict__ score) {
-  __shared__ float qs[GRP][D];
-  __shared__ float qsum[GRP];
-  const int g = blockIdx.y;
-  load_q<GRP>(q, g, qs, qsum);
-  int n = sel_n[g];
-  n = n >= 0 ? n : -1 - n;
-  const int lane = threadIdx.x & 31;
-  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int nwarps = gridDim.x * (blockDim.x >> 5);
-  for (int i = gw; i < n; i += nwarps) {
-    const int t = sel_out[static_cast<size_t>(g) * cap + i];
-    const size_t row = static_cast<size_t>(g) * T + t;
-    const uint32_t wr = k_res[row * kWordsPerRow + (lane >> 2)] >> ((lane & 3) * 8);
-    const uint32_t wf = k_ref[row * kWordsPerRow + (lane >> 2)] >> ((lane & 3) * 8);
-    float P[GRP];
-#pragma unroll
-    for (int h = 0; h < GRP; ++h) P[h] = 0.0f;
-#pragma unroll
-    for (int dd = 0; dd < 4; ++dd) {
-      const float c = static_cast<float>(((wr >> (2 * dd)) & 3u) * 4u + ((wf >> (2 * dd)) & 3u));
-#pragma unroll
-      for (int h = 0; h < GRP; ++h) P[h] = fmaf(qs[h][4 * lane + dd], c, P[h]);
-    }
-    const float sv = sfd::half_bits_to_float(k_scale[row]);
-    const float z = sfd::half_bits_to_float(k_zero[row]);
-#pragma unroll
-    for (int h = 0; h < GRP; ++h) {
-      const float Ph = warp_sum(P[h]);
-      if (lane == 0) score[(static_cast<size_t>(g) * GRP + h) * T + t] = (sv * fmaf(-z, qsum[h], Ph)) * kInvSqrtD;
-    }
-  }
+  cl.sync();  // 3: no shared-memory access across CTAs after this
 }
 
 // ---- pass B on the tensor cores ------------------------------------------------
@@ -872,10 +849,13 @@ struct OutCfg {
 
 template <int GRP>
 __global__ void __launch_bounds__(kOutThreads)
-attn_out_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__ v_ref,
-                const uint16_t* __restrict__ v_scale, const uint16_t* __restrict__ v_zero, int T, int tps, int words_t,
-                int splits, const float* __restrict__ score, const uint32_t* __restrict__ umask,
-                float* __restrict__ part, int32_t* __restrict__ done, float* __restrict__ out) {
+attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
+                const uint32_t* __restrict__ k_ref, const uint16_t* __restrict__ k_scale,
+                const uint16_t* __restrict__ k_zero, const uint32_t* __restrict__ v_res,
+                const uint32_t* __restrict__ v_ref, const uint16_t* __restrict__ v_scale,
+                const uint16_t* __restrict__ v_zero, int T, int tps, int words_t, int splits, float* __restrict__ score,
+                const uint32_t* __restrict__ umask, float* __restrict__ part, int32_t* __restrict__ done,
+                float* __restrict__ out) {
   using C = OutCfg<GRP>;
   constexpr int NT = C::NT, kStr = C::kStr;
   extern __shared__ __align__(16) unsigned char smem[];
@@ -889,6 +869,9 @@ attn_out_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__
   __shared__ float red2[kOW][3 * GRP];
   __shared__ float Msh[GRP], Fsh[GRP];
   __shared__ int ucount;
+  __shared__ float qs[GRP][D];
+  __shared__ float qsum[GRP];
+  __shared__ int uscan[33];
 
   const int g = blockIdx.y, split = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, tig = lane & 3;
@@ -898,6 +881,7 @@ attn_out_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__
   for (int e = tid; e < (NT * 8 - C::NC) * kStr; e += kOutThreads) as[C::NC * kStr + e] = __float2half_rn(0.0f);
   for (int e = tid; e < GRP * D; e += kOutThreads) wo[e] = 0.0f;
   if (tid < GRP) Msh[tid] = -INFINITY;
+  load_q<GRP>(q, g, qs, qsum);  // contains __syncthreads
 
   float lsum[GRP], csum[GRP], asum[GRP], uo[GRP][4];
   float acc[NT][8][4];
@@ -941,10 +925,62 @@ attn_out_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__
       cp_async_commit_attn();
     }
 
+    // 0. the sub-chunk's refined tokens (ascending) from the group's bitmask;
+    //    their refinement rows are staged for step 4, and their scores are
+    //    recomputed from the full 4-bit key codes into the score buffer (this
+    //    CTA owns the token range)
+    {
+      const int nw = (n + 31) >> 5;  // c0 is a multiple of 32
+      uint32_t wbits = 0;
+      if (tid < nw) {
+        wbits = umask[static_cast<size_t>(g) * words_t + (c0 >> 5) + tid];
+        const int rem = n - 32 * tid;
+        if (rem < 32) wbits &= (1u << rem) - 1u;
+      }
+      int tot;
+      int pos = sfd::block_exclusive_scan(__popc(wbits), uscan, &tot);  // nw <= kSub / 32 <= blockDim
+      while (wbits) {
+        const int b = __ffs(wbits) - 1;
+        wbits &= wbits - 1u;
+        ulist[pos++] = 32 * tid + b;
+      }
+      if (tid == 0) ucount = tot;
+      __syncthreads();
+    }
+    const int nu = ucount;
+    for (int u = tid; u < min(nu, kUCap); u += kOutThreads) {
+      const uint32_t* src = v_ref + (rowg + c0 + ulist[u]) * kWordsPerRow;
+      cp_async16_attn(vrs + u * kWordsPerRow, src);
+      cp_async16_attn(vrs + u * kWordsPerRow + 4, src + 4);
+    }
+    cp_async_commit_attn();
+    for (int u = warp; u < nu; u += kOW) {  // warp per token, lane = dims 4 lane .. 4 lane + 3
+      const int t = c0 + ulist[u];
+      const size_t row = rowg + t;
+      const uint32_t wr = k_res[row * kWordsPerRow + (lane >> 2)] >> ((lane & 3) * 8);
+      const uint32_t wf = k_ref[row * kWordsPerRow + (lane >> 2)] >> ((lane & 3) * 8);
+      float P[GRP];
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) P[h] = 0.0f;
+#pragma unroll
+      for (int dd = 0; dd < 4; ++dd) {
+        const float c = static_cast<float>(((wr >> (2 * dd)) & 3u) * 4u + ((wf >> (2 * dd)) & 3u));
+#pragma unroll
+        for (int h = 0; h < GRP; ++h) P[h] = fmaf(qs[h][4 * lane + dd], c, P[h]);
+      }
+      const float sv = sfd::half_bits_to_float(k_scale[row]);
+      const float z = sfd::half_bits_to_float(k_zero[row]);
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) {
+        const float Ph = warp_sum(P[h]);
+        if (lane == 0) score[(static_cast<size_t>(g) * GRP + h) * T + t] = (sv * fmaf(-z, qsum[h], Ph)) * kInvSqrtD;
+      }
+    }
+    __syncthreads();
+
     // 1. the sub-chunk's maximum score per head; this thread's tokens'
     //    scale, zero and union bit are fetched meanwhile
     uint32_t svz[kPerThr];
-    uint32_t ubits = 0;
     {
       float mx[GRP];
 #pragma unroll
@@ -956,8 +992,6 @@ attn_out_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__
         if (i < n) {
           const size_t row = rowg + c0 + i;
           svz[j] = static_cast<uint32_t>(v_scale[row]) | (static_cast<uint32_t>(v_zero[row]) << 16);
-          const int t = c0 + i;
-          ubits |= ((umask[static_cast<size_t>(g) * words_t + (t >> 5)] >> (t & 31)) & 1u) << j;
 #pragma unroll
           for (int h = 0; h < GRP; ++h)
             mx[h] = fmaxf(mx[h], score[(static_cast<size_t>(g) * GRP + h) * T + c0 + i]);
@@ -968,7 +1002,6 @@ attn_out_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__
         const float m = warp_max(mx[h]);
         if (lane == 0) red[warp][h] = m;
       }
-      if (tid == 0) ucount = 0;
       __syncthreads();
       if (tid < GRP) {
         float m = -INFINITY;
@@ -1012,15 +1045,12 @@ attn_out_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__
       }
     }
 
-    // 2. weights into shared memory (zero past the end of the last tile),
-    //    sums, and the list of refined tokens
-    const unsigned lt = (1u << lane) - 1u;
+    // 2. weights into shared memory (zero past the end of the last tile) and sums
 #pragma unroll
     for (int j = 0; j < kPerThr; ++j) {
       const int i = tid + j * kOutThreads;
       if (j * kOutThreads >= 16 * ntile) break;  // uniform over the block
       const bool valid = i < n;
-      bool inU = false;
       if (i < 16 * ntile) {
         if (valid) {
           const float sv = sfd::half_bits_to_float(svz[j] & 0xFFFFu);
@@ -1037,29 +1067,13 @@ attn_out_kernel(const uint32_t* __restrict__ v_res, const uint32_t* __restrict__
             csum[h] = fmaf(al, 1.5f - zv, csum[h]);
             asum[h] += __half2float(ahi) + __half2float(alo);
           }
-          inU = (ubits >> j) & 1u;
         } else {
 #pragma unroll
           for (int h = 0; h < 2 * GRP; ++h) as[h * kStr + i] = __float2half_rn(0.0f);
         }
       }
-      const unsigned b = __ballot_sync(0xffffffffu, inU);
-      if (b) {
-        int pos = 0;
-        if (lane == __ffs(b) - 1) pos = atomicAdd(&ucount, __popc(b));
-        pos = __shfl_sync(0xffffffffu, pos, __ffs(b) - 1);
-        if (inU) ulist[pos + __popc(b & lt)] = i;
-      }
     }
     __syncthreads();
-    // refinement rows of the listed tokens, staged behind the MMA loop
-    const int nu = ucount;
-    for (int u = tid; u < min(nu, kUCap); u += kOutThreads) {
-      const uint32_t* src = v_ref + (rowg + c0 + ulist[u]) * kWordsPerRow;
-      cp_async16_attn(vrs + u * kWordsPerRow, src);
-      cp_async16_attn(vrs + u * kWordsPerRow + 4, src + 4);
-    }
-    cp_async_commit_attn();
 
     // 3. MMAs over this warp's tiles
     for (int ti = tile0; ti < tile1; ++ti) {
@@ -1243,7 +1257,6 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
   attn_score_mma_kernel<GRP><<<ga, 128, 0, s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, score, smax, hist, amaxu);
   sf_status st = sf::check_launch("attn_score_mma_kernel");
   if (st != SF_OK) return st;
-  const int cap = grp * k;  // row length of sel_out
   if (k > 0 && k < T) {
     attn_select_compact_kernel<GRP><<<dim3(L.nchunks, Hq), kCompThreads, 0, s>>>(q, T, k, score, smax, hist, amaxu,
                                                                                 cand, L.nchunks, status);
@@ -1252,7 +1265,9 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(Hq));
     cfg.blockDim = dim3(kFinThreads);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = kFinDynSmem;
+    SF_CHECK_CUDA(cudaFuncSetAttribute(attn_select_finish_kernel<GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kFinDynSmem)));
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1274,17 +1289,11 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
     st = sf::check_launch("fill_all_kernel");
     if (st != SF_OK) return st;
   }
-  if (k == T) {  // every token refined: refined scores of the whole sequence
-    dim3 gr(std::max(1, std::min((cap + 7) / 8, 128)), Hkv);
-    attn_refine_scores_kernel<GRP><<<gr, 256, 0, s>>>(q, kv->k_res, kv->k_ref, kv->k_scale, kv->k_zero, T, cap,
-                                                      sel_out, sel_n, score);
-    st = sf::check_launch("attn_refine_scores_kernel");
-    if (st != SF_OK) return st;
-  }
   dim3 gb(L.splits, Hkv);
   SF_CHECK_CUDA(cudaFuncSetAttribute(attn_out_kernel<GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(OutCfg<GRP>::smem)));
-  attn_out_kernel<GRP><<<gb, kOutThreads, OutCfg<GRP>::smem, s>>>(kv->v_res, kv->v_ref, kv->v_scale, kv->v_zero, T,
+  attn_out_kernel<GRP><<<gb, kOutThreads, OutCfg<GRP>::smem, s>>>(q, kv->k_res, kv->k_ref, kv->k_scale, kv->k_zero,
+                                                                 kv->v_res, kv->v_ref, kv->v_scale, kv->v_zero, T,
                                                                  L.tps, L.words_t, L.splits, score, umask, part,
                                                                  done, out);
   return sf::check_launch("attn_out_kernel");
