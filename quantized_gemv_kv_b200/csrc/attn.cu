@@ -550,7 +550,7 @@ constexpr int kFinThreads = 512;
 constexpr int kFinKeys = 2048;     // candidates ranked pairwise from shared memory
 constexpr int kFinChunks = 4096;   // chunk prefix sums in shared memory (T <= 2^24)
 constexpr int kFinList = 4096;     // listed (token, score) pairs cached in shared memory
-constexpr size_t kFinDynSmem = static_cast<size_t>(kFinList) * 8;
+constexpr size_t kFinDynSmem = static_cast<size_t>(kFinList) * 8 + static_cast<size_t>(kFinKeys) * 4;
 
 template <int GRP>
 __global__ void __launch_bounds__(kFinThreads)
@@ -569,7 +569,7 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   const int tid = threadIdx.x;
   __shared__ int hr[2048];
   __shared__ int cpre[kFinChunks];
-  __shared__ double keys[kFinKeys];
+  __shared__ unsigned long long keys[kFinKeys];  // order-preserving exact keys, sorted with the tokens
   __shared__ double qd[D];
   __shared__ int scan_scratch[64];
   __shared__ int binfo[2];
@@ -581,6 +581,7 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   extern __shared__ int fin_dyn[];
   int* ltok = fin_dyn;                                      // [kFinList]
   float* lsc = reinterpret_cast<float*>(fin_dyn + kFinList);  // [kFinList]
+  int* ktok = fin_dyn + 2 * kFinList;                       // [kFinKeys] tokens of the sorted keys
   const float* sc = score + static_cast<size_t>(h) * T;
   int32_t* L = list + static_cast<size_t>(h) * T;  // concatenated list, token order
   int32_t* F = cand + static_cast<size_t>(h) * T;  // candidates (reuses the chunk lists once L is built)
@@ -668,17 +669,33 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   const float tau = from_okey32(pre);
   const float fthr = __double2float_ru(static_cast<double>(tau) - 2.0 * eps_s);
 
-  // 3. candidates >= tau - 2 eps in list (= token) order
-  int ncand = 0;
+  // 3. a token whose fast score exceeds tau + 2 eps outranks, by exact key,
+  //    every token with fast score <= tau, so fewer than k tokens can rank
+  //    above it: it is selected outright.  Only the band [tau - 2 eps,
+  //    tau + 2 eps] is re-keyed and ranked (its candidates in token order).
+  int32_t* sel = sel_head + static_cast<size_t>(h) * k;
+  uint32_t* um = umask + static_cast<size_t>(g) * words_t;
+  const double hi_band = static_cast<double>(tau) + 2.0 * eps_s;
+  int nA = 0, ncand = 0;
   for (int base = 0; base < m; base += kFinThreads) {
     const int e = base + tid;
-    const bool p = e < m && score_of(e) >= fthr;
-    int tot;
-    const int pos = sfd::block_exclusive_scan(p ? 1 : 0, scan_scratch, &tot);
-    if (p) F[ncand + pos] = tok_of(e);
-    ncand += tot;
+    const float sv_e = e < m ? score_of(e) : 0.0f;
+    const bool inA = e < m && static_cast<double>(sv_e) > hi_band;
+    const bool inB = e < m && !inA && sv_e >= fthr;
+    const int t = e < m ? tok_of(e) : 0;
+    int totA, totB;
+    const int posA = sfd::block_exclusive_scan(inA ? 1 : 0, scan_scratch, &totA);
+    const int posB = sfd::block_exclusive_scan(inB ? 1 : 0, scan_scratch, &totB);
+    if (inA && nA + posA < k) {  // fewer than k by the bound; guarded against corrupt scores
+      sel[nA + posA] = t;
+      atomicOr(um + (t >> 5), 1u << (t & 31));
+    }
+    if (inB) F[ncand + posB] = t;
+    nA += totA;
+    ncand += totB;
   }
   __syncthreads();
+  const int kB = max(0, k - nA);  // winners still to pick from the band (>= 1 by the bound)
 
 
   // 4. exact keys (four partial sums: exact under the precondition, so the
@@ -727,40 +744,51 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
       key = sv * ((E[0] + E[1]) + (E[2] + E[3]));
     }
     kp[i] = key;
-    if (ncand <= kFinKeys) keys[i] = key;
+    if (ncand <= kFinKeys) {
+      keys[i] = okey64(key);
+      ktok[i] = t;
+    }
   }
   __syncthreads();
 
-  // 5. rank by (key desc, token asc); the k winners go to sel_head and the
-  //    group's token bitmask
-  int32_t* sel = sel_head + static_cast<size_t>(h) * k;
-  uint32_t* um = umask + static_cast<size_t>(g) * words_t;
+  // 5. rank the band by (key desc, token asc); its kB winners go to
+  //    sel_head after the outright ones, and into the group's token bitmask
   if (ncand <= kFinKeys) {
-    int tpc = 1;  // threads per candidate: a power of two up to 32
-    while (tpc < 32 && 2 * tpc * max(ncand, 1) <= kFinThreads) tpc *= 2;
-    const int per = kFinThreads / tpc;
-    for (int r0 = 0; r0 < ncand; r0 += per) {  // uniform over the block
-      const int i = r0 + tid / tpc, sub = tid % tpc;
-      int rk = 0;
-      if (i < ncand) {
-        const double ki = keys[i];
-        for (int j = sub; j < ncand; j += tpc) {
-          const double kj = keys[j];
-          rk += (kj > ki) || (kj == ki && j < i);
+    // bitonic sort of (key desc, token asc) over a power-of-two size,
+    // padding with entries that order last; the first k are the selection
+    int n2 = 1;
+    while (n2 < ncand) n2 <<= 1;
+    for (int i = ncand + tid; i < n2; i += kFinThreads) {
+      keys[i] = 0ull;
+      ktok[i] = 0x7FFFFFFF;
+    }
+    __syncthreads();
+    for (int size = 2; size <= n2; size <<= 1)
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int i = tid; i < (n2 >> 1); i += kFinThreads) {
+          const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
+          const unsigned long long ka = keys[lo], kb = keys[hi];
+          const int ta = ktok[lo], tb = ktok[hi];
+          const bool a_first = ka > kb || (ka == kb && ta < tb);
+          if (a_first == ((lo & size) != 0)) {
+            keys[lo] = kb;
+            keys[hi] = ka;
+            ktok[lo] = tb;
+            ktok[hi] = ta;
+          }
         }
+        __syncthreads();
       }
-      for (int o = tpc / 2; o > 0; o >>= 1) rk += __shfl_xor_sync(0xffffffffu, rk, o);
-      if (i < ncand && sub == 0 && rk < k) {
-        const int t = F[i];
-        sel[rk] = t;
-        atomicOr(um + (t >> 5), 1u << (t & 31));
-      }
+    for (int r = tid; r < kB; r += kFinThreads) {
+      const int t = ktok[r];
+      sel[nA + r] = t;
+      atomicOr(um + (t >> 5), 1u << (t & 31));
     }
   } else {
-    select_rank_radix(F, ncand, kp, k, hr, scan_scratch, binfo, sel);
+    select_rank_radix(F, ncand, kp, kB, hr, scan_scratch, binfo, sel + nA);
     __syncthreads();
-    for (int i = tid; i < k; i += kFinThreads) {
-      const int t = sel[i];
+    for (int i = tid; i < kB; i += kFinThreads) {
+      const int t = sel[nA + i];
       atomicOr(um + (t >> 5), 1u << (t & 31));
     }
   }
@@ -840,11 +868,11 @@ struct OutCfg {
   static constexpr int kStr = kSub + 8;        // halves per weight row: conflict-free fragment loads
   static constexpr size_t alpha_bytes = static_cast<size_t>(NT) * 8 * kStr * 2;
   static constexpr size_t ring_bytes = static_cast<size_t>(kOW) * kRing * 16 * kWordsPerRow * 4;
-  static constexpr size_t wo_bytes = static_cast<size_t>(GRP) * D * 4;
   static constexpr size_t ulist_bytes = static_cast<size_t>(kSub) * 4;
   static constexpr size_t vref_bytes = static_cast<size_t>(kUCap) * kWordsPerRow * 4;
-  static constexpr size_t smem = alpha_bytes + ring_bytes + wo_bytes + ulist_bytes + vref_bytes;
+  static constexpr size_t smem = alpha_bytes + ring_bytes + ulist_bytes + vref_bytes;
   static_assert(alpha_bytes >= static_cast<size_t>(GRP) * kMaxSplits * 4, "merge factors must fit the weight tile");
+  static_assert(alpha_bytes >= static_cast<size_t>(kOW) * GRP * D * 4, "per-warp output tiles must fit the weight tile");
 };
 
 template <int GRP>
@@ -861,9 +889,8 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
   extern __shared__ __align__(16) unsigned char smem[];
   __half* as = reinterpret_cast<__half*>(smem);                                      // [NT*8][kStr]
   uint32_t* ring = reinterpret_cast<uint32_t*>(smem + C::alpha_bytes);               // [kOW][kRing][16][8]
-  float* wo = reinterpret_cast<float*>(smem + C::alpha_bytes + C::ring_bytes);       // [GRP][D]
-  int* ulist = reinterpret_cast<int*>(smem + C::alpha_bytes + C::ring_bytes + C::wo_bytes);  // [kSub]
-  uint32_t* vrs = reinterpret_cast<uint32_t*>(smem + C::alpha_bytes + C::ring_bytes + C::wo_bytes +
+  int* ulist = reinterpret_cast<int*>(smem + C::alpha_bytes + C::ring_bytes);  // [kSub]
+  uint32_t* vrs = reinterpret_cast<uint32_t*>(smem + C::alpha_bytes + C::ring_bytes +
                                               C::ulist_bytes);  // [kUCap][8] refinement rows of listed tokens
   __shared__ float red[kOW][GRP];
   __shared__ float red2[kOW][3 * GRP];
@@ -879,7 +906,6 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
   const size_t rowg = static_cast<size_t>(g) * T;
 
   for (int e = tid; e < (NT * 8 - C::NC) * kStr; e += kOutThreads) as[C::NC * kStr + e] = __float2half_rn(0.0f);
-  for (int e = tid; e < GRP * D; e += kOutThreads) wo[e] = 0.0f;
   if (tid < GRP) Msh[tid] = -INFINITY;
   load_q<GRP>(q, g, qs, qsum);  // contains __syncthreads
 
@@ -954,26 +980,43 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
       cp_async16_attn(vrs + u * kWordsPerRow + 4, src + 4);
     }
     cp_async_commit_attn();
-    for (int u = warp; u < nu; u += kOW) {  // warp per token, lane = dims 4 lane .. 4 lane + 3
-      const int t = c0 + ulist[u];
-      const size_t row = rowg + t;
-      const uint32_t wr = k_res[row * kWordsPerRow + (lane >> 2)] >> ((lane & 3) * 8);
-      const uint32_t wf = k_ref[row * kWordsPerRow + (lane >> 2)] >> ((lane & 3) * 8);
-      float P[GRP];
+    // warp per token, lane = dims 4 lane .. 4 lane + 3; four tokens' loads in
+    // flight at a time
+    for (int u0 = warp; u0 < nu; u0 += 4 * kOW) {
+      uint32_t wr[4], wf[4], sz[4];
 #pragma unroll
-      for (int h = 0; h < GRP; ++h) P[h] = 0.0f;
-#pragma unroll
-      for (int dd = 0; dd < 4; ++dd) {
-        const float c = static_cast<float>(((wr >> (2 * dd)) & 3u) * 4u + ((wf >> (2 * dd)) & 3u));
-#pragma unroll
-        for (int h = 0; h < GRP; ++h) P[h] = fmaf(qs[h][4 * lane + dd], c, P[h]);
+      for (int j = 0; j < 4; ++j) {
+        const int u = u0 + j * kOW;
+        wr[j] = wf[j] = sz[j] = 0;
+        if (u < nu) {
+          const size_t row = rowg + c0 + ulist[u];
+          wr[j] = k_res[row * kWordsPerRow + (lane >> 2)];
+          wf[j] = k_ref[row * kWordsPerRow + (lane >> 2)];
+          sz[j] = static_cast<uint32_t>(k_scale[row]) | (static_cast<uint32_t>(k_zero[row]) << 16);
+        }
       }
-      const float sv = sfd::half_bits_to_float(k_scale[row]);
-      const float z = sfd::half_bits_to_float(k_zero[row]);
 #pragma unroll
-      for (int h = 0; h < GRP; ++h) {
-        const float Ph = warp_sum(P[h]);
-        if (lane == 0) score[(static_cast<size_t>(g) * GRP + h) * T + t] = (sv * fmaf(-z, qsum[h], Ph)) * kInvSqrtD;
+      for (int j = 0; j < 4; ++j) {
+        const int u = u0 + j * kOW;
+        if (u >= nu) break;  // uniform over the warp
+        const uint32_t r = wr[j] >> ((lane & 3) * 8), f = wf[j] >> ((lane & 3) * 8);
+        float P[GRP];
+#pragma unroll
+        for (int h = 0; h < GRP; ++h) P[h] = 0.0f;
+#pragma unroll
+        for (int dd = 0; dd < 4; ++dd) {
+          const float c = static_cast<float>(((r >> (2 * dd)) & 3u) * 4u + ((f >> (2 * dd)) & 3u));
+#pragma unroll
+          for (int h = 0; h < GRP; ++h) P[h] = fmaf(qs[h][4 * lane + dd], c, P[h]);
+        }
+        const float sv = sfd::half_bits_to_float(sz[j] & 0xFFFFu);
+        const float z = sfd::half_bits_to_float(sz[j] >> 16);
+        const int t = c0 + ulist[u];
+#pragma unroll
+        for (int h = 0; h < GRP; ++h) {
+          const float Ph = warp_sum(P[h]);
+          if (lane == 0) score[(static_cast<size_t>(g) * GRP + h) * T + t] = (sv * fmaf(-z, qsum[h], Ph)) * kInvSqrtD;
+        }
       }
     }
     __syncthreads();
@@ -1133,21 +1176,32 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
     __syncthreads();  // weights and the list are rewritten by the next sub-chunk
   }
 
-  // high + remainder columns and the refined corrections into wo[head][dim]
-  // (in units of the code part: uo enters divided by 2^b_f = 4)
+  // this warp's output tile ww[head][dim] (in units of the code part: uo
+  // enters divided by 2^b_f = 4) in the dead weight tile, written in three
+  // phases whose stores within a warp never collide (high columns, then
+  // remainder columns, then the refined corrections); summed over warps below
+  __syncthreads();  // every warp is done with the weight tile
+  float* ww = reinterpret_cast<float*>(smem) + warp * GRP * D;
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
+  for (int ph = 0; ph < 2; ++ph) {
 #pragma unroll
-    for (int w = 0; w < 8; ++w)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int hh = colh[nt][c & 1];
-        if (hh >= 0) atomicAdd(&wo[hh * D + 16 * w + g8 + 8 * (c >> 1)], acc[nt][w][c]);
-      }
+      for (int w = 0; w < 8; ++w)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int n = nt * 8 + 2 * tig + (c & 1);
+          const int hh = colh[nt][c & 1];
+          if (hh < 0 || (n < GRP) != (ph == 0)) continue;
+          float* dst = &ww[hh * D + 16 * w + g8 + 8 * (c >> 1)];
+          *dst = ph == 0 ? acc[nt][w][c] : *dst + acc[nt][w][c];
+        }
+    __syncwarp();
+  }
 #pragma unroll
   for (int h = 0; h < GRP; ++h)
 #pragma unroll
-    for (int dd = 0; dd < 4; ++dd) atomicAdd(&wo[h * D + 4 * lane + dd], 0.25f * uo[h][dd]);
+    for (int dd = 0; dd < 4; ++dd) ww[h * D + 4 * lane + dd] += 0.25f * uo[h][dd];
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
     const float l = warp_sum(lsum[h]), cs = warp_sum(csum[h]), a = warp_sum(asum[h]);
@@ -1172,7 +1226,10 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
         A += red2[w][2 * GRP + h];
       }
       // resident value s (2^b_f c + m_f - z): code part 4 (acc - 1024 A), offset part Cs
-      v = j == 1 ? L : fmaf(4.0f, wo[h * D + j - 2], fmaf(-4096.0f, A, Cs));
+      float o = 0.0f;
+      if (j >= 2)
+        for (int w = 0; w < kOW; ++w) o += reinterpret_cast<const float*>(smem)[(w * GRP + h) * D + j - 2];
+      v = j == 1 ? L : fmaf(4.0f, o, fmaf(-4096.0f, A, Cs));
     }
     pg[(static_cast<size_t>(h) * splits + split) * (D + 2) + j] = v;
   }
@@ -1204,19 +1261,33 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
     if (lane == 0) Lh[h] = Ls;
   }
   __syncthreads();
-  for (int e = tid; e < GRP * D; e += kOutThreads) {
-    const int h = e / D, d = e % D;
-    const float* ph = pg + static_cast<size_t>(h) * splits * (D + 2) + 2 + d;
-    float O0 = 0.0f, O1 = 0.0f, O2 = 0.0f, O3 = 0.0f;
-    int sp = 0;
-    for (; sp + 3 < splits; sp += 4) {
-      O0 = fmaf(fct[h][sp], __ldcg(ph + sp * (D + 2)), O0);
-      O1 = fmaf(fct[h][sp + 1], __ldcg(ph + (sp + 1) * (D + 2)), O1);
-      O2 = fmaf(fct[h][sp + 2], __ldcg(ph + (sp + 2) * (D + 2)), O2);
-      O3 = fmaf(fct[h][sp + 3], __ldcg(ph + (sp + 3) * (D + 2)), O3);
+  // two outputs per thread, eight splits' partials of each in flight at once
+  for (int e0 = tid; e0 < GRP * D; e0 += 2 * kOutThreads) {
+    const int e1 = e0 + kOutThreads;
+    const bool has1 = e1 < GRP * D;
+    const int h0 = e0 / D, h1 = has1 ? e1 / D : h0;
+    const float* p0 = pg + static_cast<size_t>(h0) * splits * (D + 2) + 2 + e0 % D;
+    const float* p1 = pg + static_cast<size_t>(h1) * splits * (D + 2) + 2 + (has1 ? e1 % D : e0 % D);
+    float A0 = 0.0f, A1 = 0.0f;
+    for (int sp = 0; sp < splits; sp += 16) {
+      float v0[16], v1[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int q = sp + u;
+        v0[u] = q < splits ? __ldcg(p0 + static_cast<size_t>(q) * (D + 2)) : 0.0f;
+        v1[u] = (has1 && q < splits) ? __ldcg(p1 + static_cast<size_t>(q) * (D + 2)) : 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int q = sp + u;
+        if (q < splits) {
+          A0 = fmaf(fct[h0][q], v0[u], A0);
+          A1 = fmaf(fct[h1][q], v1[u], A1);
+        }
+      }
     }
-    for (; sp < splits; ++sp) O0 = fmaf(fct[h][sp], __ldcg(ph + sp * (D + 2)), O0);
-    out[(static_cast<size_t>(g) * GRP + h) * D + d] = ((O0 + O1) + (O2 + O3)) / Lh[h];
+    out[(static_cast<size_t>(g) * GRP + h0) * D + e0 % D] = A0 / Lh[h0];
+    if (has1) out[(static_cast<size_t>(g) * GRP + h1) * D + e1 % D] = A1 / Lh[h1];
   }
 }
 
