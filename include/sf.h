@@ -344,8 +344,8 @@ sf_status sf_attn_workspace_size(int Hq, int Hkv, int d, int T, int k_tokens, si
  * every key is exact in fp64).  When a head of KV group g violates it, the
  * selection still runs on the fp64 keys (then possibly not exact) and
  * sel_n[g] is written as -1 - (union length) to report it.
- * Constraints: d == 128, Hq % Hkv == 0, Hq/Hkv <= 8, 1 <= T, 0 <= k_tokens
- *   <= min(T, 4096), b_r == 2, b_f == 2.
+ * Constraints: d == 128, Hq/Hkv in {1, 2, 4, 8}, 1 <= T <= 2^24,
+ *   0 <= k_tokens <= T, b_r == 2, b_f == 2.
  * Accuracy: max |out - exact| <= 2e-3.
  */
 sf_status sf_attn_decode_refine(const uint16_t* q, int Hq, int Hkv, int d, int T,
@@ -375,6 +375,25 @@ sf_status sf_attn_decode_refine(const uint16_t* q, int Hq, int Hkv, int d, int T
 sf_status sf_attn_decode_refine_noalloc(const uint16_t* q, int Hq, int Hkv, int d, int T,
                                         const sf_qkv* kv, int k_tokens, int32_t* sel_out,
                                         int32_t* sel_n, float* out, sf_stream_t stream);
+
+/*
+ * sf_attn_set_path -- which implementation sf_attn_decode_refine and
+ * sf_attn_decode_refine_noalloc use, process-wide.  The paper has no
+ * counterpart; both implementations compute the definition above (the same
+ * selection, outputs within the same accuracy), so this is for diagnostics
+ * and benchmarking:
+ *   SF_ATTN_AUTO      the cluster kernel where it applies, else the pipeline;
+ *   SF_ATTN_CLUSTER   only the cluster kernel, one thread-block cluster of up
+ *                     to 16 CTAs per KV head doing the whole step on chip; it
+ *                     applies for T <= 32768 (Hq/Hkv <= 4) or T <= 16384
+ *                     (Hq/Hkv == 8) on a device that fits the cluster, and
+ *                     other calls return SF_ENOTIMPL;
+ *   SF_ATTN_PIPELINE  only the multi-kernel pipeline (every size).
+ * Returns SF_EINVAL for any other value.  The setting is read when a call is
+ * enqueued; a captured graph keeps the kernels it captured.
+ */
+typedef enum sf_attn_path { SF_ATTN_AUTO = 0, SF_ATTN_CLUSTER = 1, SF_ATTN_PIPELINE = 2 } sf_attn_path;
+sf_status sf_attn_set_path(int path);
 
 #ifdef __cplusplus
 }

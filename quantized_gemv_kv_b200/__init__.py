@@ -95,6 +95,7 @@ _SIGS = {
     "sf_attn_workspace_size": ([_i, _i, _i, _i, _i, ctypes.POINTER(_sz)], _i),
     "sf_attn_decode_refine": ([_p, _i, _i, _i, _i, ctypes.POINTER(_QKV), _i, _p, _p, _p, _p, _sz, _p], _i),
     "sf_attn_decode_refine_noalloc": ([_p, _i, _i, _i, _i, ctypes.POINTER(_QKV), _i, _p, _p, _p, _p], _i),
+    "sf_attn_set_path": ([_i], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -324,6 +325,16 @@ class QKV:
         return _QKV(_ptr(self.k.res), _ptr(self.k.ref), _ptr(self.v.res), _ptr(self.v.ref),
                     _ptr(self.k.scale), _ptr(self.k.zero), _ptr(self.v.scale), _ptr(self.v.zero),
                     self.k.b_r, self.k.b_f)
+
+
+ATTN_AUTO, ATTN_CLUSTER, ATTN_PIPELINE = 0, 1, 2
+
+
+def attn_set_path(path: int) -> None:
+    """Process-wide choice of the attention implementation
+    (``sf_attn_set_path``): ATTN_AUTO, ATTN_CLUSTER (one thread-block cluster
+    per KV head, T <= 32768) or ATTN_PIPELINE (the multi-kernel pipeline)."""
+    _check(_lib.sf_attn_set_path(path))
 
 
 def attn_workspace_size(Hq: int, Hkv: int, d: int, T: int, k_tokens: int) -> int:

@@ -1,0 +1,282 @@
+// Device helpers and the workspace layout shared by the two implementations
+// of refined decode attention: the multi-kernel pipeline (attn.cu) and the
+// single cluster kernel per KV group (attn_fused.cu).
+#pragma once
+
+#include <algorithm>
+#include <cmath>
+
+#include "block_scan.cuh"
+#include "sf_internal.h"
+
+namespace sf {
+
+// The single cluster kernel per KV group (attn_fused.cu): whether it applies
+// to these sizes on the current device, and the launch.  The overflow lists
+// (keys, tokens: Hq * T each; winners: Hq * k) live in the caller's workspace.
+bool attn_fused_eligible(int Hq, int Hkv, int T);
+sf_status attn_fused_run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k, int32_t* sel_out,
+                         int32_t* sel_n, float* out, double* ovf_key, int32_t* ovf_tok, int32_t* ovf_sel,
+                         cudaStream_t s);
+
+}  // namespace sf
+
+namespace {
+
+constexpr int D = 128;                 // head dim
+constexpr int kWordsPerRow = D * 2 / 32;  // 2-bit codes of one token-head: 8 words
+constexpr int kMaxGrp = 8;
+constexpr int kMaxSplits = 256;
+constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128), rounded to fp32
+
+constexpr int kHistBins = 1024;    // per-head histogram of the fast scores' top 10 key bits
+constexpr int kChunk = 4096;       // tokens per CTA of the candidate compaction
+
+struct Layout {
+  // from smax on, everything is cleared at the start of a call
+  size_t score, cand, cand2, kap, sel, part, smax, status, count, amax, hist, umask, total;
+  int splits, tps, words_t, nchunks;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+Layout make_layout(int Hq, int Hkv, int T, int k, int sms) {
+  Layout L{};
+  const int want = std::max(1, std::min(kMaxSplits, 2 * sms / Hkv));  // one wave of pass-B CTAs at 2 per SM
+  int tps = (T + want - 1) / want;
+  tps = std::max(128, (tps + 127) / 128 * 128);
+  L.tps = tps;
+  L.splits = (T + tps - 1) / tps;
+  L.words_t = (T + 31) / 32;
+  L.nchunks = (T + kChunk - 1) / kChunk;
+  size_t off = 0;
+  L.score = off; off = up256(off + sizeof(float) * Hq * static_cast<size_t>(T));
+  L.cand = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(T) + sizeof(int32_t) * Hq * L.nchunks);
+  L.cand2 = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(T));
+  L.kap = off; off = up256(off + sizeof(double) * Hq * static_cast<size_t>(T));
+  L.sel = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(std::max(k, 1)));
+  L.part = off; off = up256(off + sizeof(float) * Hq * static_cast<size_t>(L.splits) * (D + 2));
+  L.smax = off; off = up256(off + sizeof(float) * Hkv);
+  L.status = off; off = up256(off + sizeof(int32_t) * std::max(Hkv, 4));
+  L.count = off; off = up256(off + sizeof(int32_t) * Hkv);
+  L.amax = off; off = up256(off + sizeof(uint32_t) * Hq);
+  L.hist = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(kHistBins));
+  L.umask = off; off = up256(off + sizeof(uint32_t) * Hkv * static_cast<size_t>(L.words_t));
+  L.total = off;
+  return L;
+}
+
+__device__ __forceinline__ uint32_t okey32(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float from_okey32(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+__device__ __forceinline__ unsigned long long okey64(double x) {
+  const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(x));
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+
+__device__ __forceinline__ void cp_async16_attn(void* smem, const void* gmem) {
+  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit_attn() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_attn() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+// Integer tensor-core MMA over code bytes (m16n8k32, s32 accumulate).
+__device__ __forceinline__ void mma_u8u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// f16 tensor-core MMA with f32 accumulate (m16n8k16).
+__device__ __forceinline__ void mma_f16f32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---- pass S: exact per-head top-k ------------------------------------------
+
+// Finds the bin holding the kk-th largest element of a histogram of nb bins
+// (scanning from the top) with warp 0.  Returns via shared out[0] = bin,
+// out[1] = kk left inside the bin.
+__device__ void find_bin_from_top(const int* hist, int nb, int kk, int* out) {
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
+  int above = 0;
+  for (int base = nb - 1; base >= 0; base -= 32) {
+    const int bin = base - lane;
+    const int c = bin >= 0 ? hist[bin] : 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const bool hit = (above + incl >= kk) && (above + incl - c < kk);
+    const unsigned m = __ballot_sync(0xffffffffu, hit);
+    if (m) {
+      const int src = __ffs(m) - 1;
+      const int before = __shfl_sync(0xffffffffu, incl - c, src);
+      if (lane == 0) { out[0] = base - src; out[1] = kk - (above + before); }
+      return;
+    }
+    above += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) { out[0] = 0; out[1] = kk; }
+}
+
+// Query-side setup of pass S (all threads call): q in fp64 into qd, its l1
+// norm and the binary exponent of max |q|; flags the KV group when the
+// nonzero q exponents span more than the exact-key precondition allows.
+__device__ void select_q_prologue(const uint16_t* __restrict__ q, int h, int g, double* qd, double* l1_out,
+                                  int* qe_out, int32_t* __restrict__ status, int* span_out = nullptr) {
+  const int tid = threadIdx.x;
+  for (int d = tid; d < D; d += blockDim.x)
+    qd[d] = static_cast<double>(sfd::bf16_bits_to_float(q[static_cast<size_t>(h) * D + d]));
+  __syncthreads();
+  if (tid < 32) {
+    double l1 = 0.0;
+    int emin = 100000, emax = -100000;
+    for (int d = tid; d < D; d += 32) {
+      const double v = qd[d];
+      l1 += fabs(v);
+      if (v != 0.0) {
+        int e;
+        frexp(v, &e);
+        emin = min(emin, e);
+        emax = max(emax, e);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+      emin = min(emin, __shfl_xor_sync(0xffffffffu, emin, o));
+      emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+    }
+    if (tid == 0) {
+      *l1_out = l1;
+      *qe_out = emax >= emin ? emax : 0;  // binary exponent of max |q| (frexp convention)
+      if (span_out) *span_out = emax >= emin ? emax - emin : 0;  // binades spanned by the nonzero q
+      // 53 - 9 - b - log2(d) with b = 4, d = 128
+      if (emax >= emin && emax - emin > 53 - 9 - 4 - 7) atomicOr(status + g, 1);
+    }
+  }
+  __syncthreads();
+}
+
+// Error bound of the fast scores (pass A): q rounded to 24-bit fixed point
+// (|dq| <= 2^(e-24) per entry), exact integer products and sums, an fp32
+// combine of the three plane sums, the fp32 sum of q (<= gamma_128 l1), and
+// the roundings of the zero-point term, the fma, the scale and 1/sqrt(d).
+// Returns the half-width eps_s of the band; two fast scores whose exact
+// values are ordered one way differ by at least -2 eps_s the other way.
+__device__ __forceinline__ double select_eps(double s_max, double l1, int qe, float amax) {
+  const double u = 5.9604644775390625e-8;  // 2^-24
+  const double gam = 130.0 * u / (1.0 - 130.0 * u);
+  const double qround = ldexp(1.0, qe - 24);
+  const double eps_k = s_max * (4.0 * 3.0 * D * qround + l1 * (136.0 * u + 16.0 * gam));
+  return 2.0 * (static_cast<double>(kInvSqrtD) * eps_k + 4.0 * u * static_cast<double>(amax));
+}
+
+// Exact top-k of F[0..ncand) by (key desc, token asc) with an 8-pass radix
+// select on the 64-bit order-preserving keys kp (all threads call; F is in
+// token order); the k winners go to sel in no particular order.
+__device__ void select_rank_radix(const int32_t* __restrict__ F, int ncand, const double* __restrict__ kp, int k,
+                                  int* hist, int* scan_scratch, int* binfo, int32_t* __restrict__ sel) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  unsigned long long pre64 = 0, pm64 = 0;
+  int kr = k;
+  for (int pass = 0; pass < 8; ++pass) {
+    const int shift = 56 - 8 * pass;
+    for (int i = tid; i < 256; i += nthr) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < ncand; i += nthr) {
+      const unsigned long long key = okey64(kp[i]);
+      if ((key & pm64) == pre64) atomicAdd(&hist[(key >> shift) & 255], 1);
+    }
+    __syncthreads();
+    find_bin_from_top(hist, 256, kr, binfo);
+    __syncthreads();
+    pre64 |= static_cast<unsigned long long>(binfo[0]) << shift;
+    pm64 |= 255ull << shift;
+    kr = binfo[1];
+    __syncthreads();
+  }
+  {
+    const int chunk = (ncand + nthr - 1) / nthr;
+    const int i0 = min(ncand, tid * chunk), i1 = min(ncand, i0 + chunk);
+    int eq = 0;
+    for (int i = i0; i < i1; ++i) eq += okey64(kp[i]) == pre64;
+    int tot;
+    int rank = sfd::block_exclusive_scan(eq, scan_scratch, &tot);
+    int take = 0;
+    {
+      int rk = rank;
+      for (int i = i0; i < i1; ++i) {
+        const unsigned long long key = okey64(kp[i]);
+        if (key > pre64) ++take;
+        else if (key == pre64) { if (rk < kr) ++take; ++rk; }
+      }
+    }
+    int pos = sfd::block_exclusive_scan(take, scan_scratch, &tot);
+    for (int i = i0; i < i1; ++i) {
+      const unsigned long long key = okey64(kp[i]);
+      bool ok = false;
+      if (key > pre64) ok = true;
+      else if (key == pre64) { ok = rank < kr; ++rank; }
+      if (ok) sel[pos++] = F[i];
+    }
+  }}
+
+// Block-parallel search of a histogram from the top (all threads call):
+// out[0] = the bin holding the kk-th largest element, out[1] = kk minus the
+// elements in higher bins.  Thread t sums its own run of bins, an exclusive
+// scan gives the count above each run, and the one thread whose run crosses
+// kk walks it.
+__device__ void find_bin_from_top_block(const int* hist, int nb, int kk, int* out, int* scratch) {
+  const int per = (nb + blockDim.x - 1) / blockDim.x;
+  const int hi = nb - static_cast<int>(threadIdx.x) * per;  // exclusive upper bin of this run
+  const int lo = max(0, hi - per);
+  int c = 0;
+  for (int b = hi - 1; b >= lo; --b) c += hist[b];
+  int tot;
+  const int above = sfd::block_exclusive_scan(c, scratch, &tot);
+  if (c > 0 && above < kk && above + c >= kk) {
+    int a = above;
+    for (int b = hi - 1; b >= lo; --b) {
+      const int n = hist[b];
+      if (a + n >= kk) { out[0] = b; out[1] = kk - a; break; }
+      a += n;
+    }
+  }
+  if (threadIdx.x == 0 && tot < kk) { out[0] = 0; out[1] = kk; }
+  __syncthreads();
+}
+
+}  // namespace

@@ -74,3 +74,13 @@ def test_host_validation(sf):
     h = ctypes.c_void_p()
     assert L.sf_refine_cache_create(ctypes.byref(h), 64, 24, 8, 8, p, 0) == sf.SF_EINVAL
     assert L.sf_refine_cache_destroy(None) == sf.SF_OK
+
+
+def test_attn_path_switch(sf):
+    """The implementation switch accepts its three values and refuses others
+    (no GPU needed: nothing is enqueued)."""
+    L = ctypes.CDLL(sf.LIB_PATH)
+    assert L.sf_attn_set_path(7) == sf.SF_EINVAL
+    assert L.sf_attn_set_path(-1) == sf.SF_EINVAL
+    for p in (sf.ATTN_PIPELINE, sf.ATTN_CLUSTER, sf.ATTN_AUTO):
+        assert L.sf_attn_set_path(p) == sf.SF_OK

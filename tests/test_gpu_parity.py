@@ -269,13 +269,36 @@ def _kv(sf, Hkv, T, d, seed, n_out=4):
     return sf.QKV(qk, qv), ok, ov
 
 
+def _cluster_applies(Hq, Hkv, T):
+    return T <= 16 * (2048 if Hq // Hkv <= 4 else 1024)
+
+
+@pytest.fixture(params=["pipeline", "cluster"])
+def attn_path(request, sf):
+    """Runs a test once per attention implementation (the multi-kernel
+    pipeline and the single cluster kernel per KV head); restores the
+    automatic choice afterwards."""
+    sf.attn_set_path(sf.ATTN_PIPELINE if request.param == "pipeline" else sf.ATTN_CLUSTER)
+    yield request.param
+    sf.attn_set_path(sf.ATTN_AUTO)
+
+
+def _skip_unless_applies(path, Hq, Hkv, T):
+    if path == "cluster" and not _cluster_applies(Hq, Hkv, T):
+        pytest.skip("the cluster kernel does not apply to this size")
+
+
 @pytest.mark.parametrize("Hq,Hkv,T,pct", [(8, 2, 1000, 1), (32, 8, 4099, 1), (4, 4, 77, 10), (16, 2, 33, 100),
                                           (8, 1, 512, 0), (8, 2, 8192, 30), (8, 2, 40961, 1), (4, 1, 32768, 2),
-                                          (4, 1, 70001, 1), (8, 8, 65536, 1)])
-def test_attn_small(sf, Hq, Hkv, T, pct):
-    """Covers both selection kernels (scores in registers over a cluster of up
-    to 8 CTAs per head up to T = 65536, streamed beyond), the pairwise ranking
-    of few candidates and the radix ranking of many (30% of 8192)."""
+                                          (4, 1, 70001, 1), (8, 8, 65536, 1), (64, 8, 16384, 1), (16, 8, 300, 5),
+                                          (8, 2, 32768, 1), (32, 8, 1, 100)])
+def test_attn_small(sf, attn_path, Hq, Hkv, T, pct):
+    """Both implementations against the oracle: the pipeline's compaction,
+    finish and output kernels at every size, the cluster kernel up to its
+    limit (including clusters with empty CTAs at tiny T, eight query heads
+    per KV head, k = T and k = 0), the pairwise ranking of few candidates and
+    the radix ranking of many (30% of 8192)."""
+    _skip_unless_applies(attn_path, Hq, Hkv, T)
     d = 128
     kv, ok, ov = _kv(sf, Hkv, T, d, 3000 + T)
     qb = gen_query(4000 + T, Hq, d)
@@ -292,7 +315,7 @@ def test_attn_small(sf, Hq, Hkv, T, pct):
     assert err <= ATTN_TOL, err
 
 
-def test_attn_32k(sf):
+def test_attn_32k(sf, attn_path):
     """32K context, 32 query / 8 KV heads, head_dim 128, 2+2 K/V with 4
     outlier key channels x10, top 1% tokens per query head."""
     Hq, Hkv, T, d = 32, 8, 32768, 128
@@ -310,7 +333,31 @@ def test_attn_32k(sf):
     assert err <= ATTN_TOL, err
 
 
-def test_attn_ties(sf):
+def test_attn_band_overflow(sf, attn_path):
+    """Half the tokens of each KV head are copies of one token, and k puts the
+    k-th largest key of query head 0 inside that tie: thousands of exactly
+    tied candidates straddle the threshold (the cluster kernel's band then
+    overflows its owner's shared memory into the workspace)."""
+    Hq, Hkv, T, d = 8, 2, 8192, 128
+    Kf, Vf, _ = gen_kv(91, Hkv, T, d)
+    Kf[:, 0::2] = Kf[:, :1]
+    Kf2, Vf2 = Kf.reshape(Hkv * T, d), Vf.reshape(Hkv * T, d)
+    kv = sf.QKV(sf.quantize_nested(dev(Kf2), d, 2, 2, "by_row"), sf.quantize_nested(dev(Vf2), d, 2, 2, "by_row"))
+    ok, ov = oquant.quantize_nested(Kf2, d, 2, 2), oquant.quantize_nested(Vf2, d, 2, 2)
+    qb = gen_query(92, Hq, d)
+    kap = oattn.selection_keys(oattn.bf16_to_f64(qb)[0], ok, slice(0, T))
+    above = int((kap > kap[0]).sum())  # tokens ranked above the tied copies
+    k = min(T // 2, above + 100)
+    out, sel, sel_n = sf.attn_decode_refine(bf16_dev(qb), kv, Hkv, T, k)
+    torch.cuda.synchronize()
+    ref = oattn.attn_decode_refine(qb, ok, ov, Hkv, T, k)
+    for g in range(Hkv):
+        n = sel_n.cpu().numpy()[g]
+        np.testing.assert_array_equal(sel.cpu().numpy()[g, :n], ref["union"][g])
+    assert np.abs(out.cpu().numpy() - ref["out"]).max() <= ATTN_TOL
+
+
+def test_attn_ties(sf, attn_path):
     """Duplicate tokens give exactly tied keys; the lower token index wins."""
     Hq, Hkv, T, d = 8, 2, 600, 128
     Kf, Vf, _ = gen_kv(77, Hkv, T, d)
