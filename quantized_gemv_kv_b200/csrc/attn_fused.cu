@@ -58,6 +58,7 @@ constexpr int kFStop = 48;            // a chosen bin this small ends the levels
 constexpr int kFMaxLevels = 8;
 constexpr int kFBandCap = kFThreads;  // band entries per head ranked in the owner's shared memory
 constexpr int kFStgCap = 128;         // union tokens per CTA whose value refinement rows are staged
+constexpr int kFLocalBand = 256;      // band entries of one CTA listed in shared memory
 
 __host__ __device__ constexpr int fused_rmax(int grp) { return grp <= 4 ? 2048 : 1024; }
 __host__ __device__ constexpr int fused_nt(int grp) { return 2 * grp <= 8 ? 1 : 2; }
@@ -70,6 +71,7 @@ struct FusedSmem {
   int vsz;    // [R] value scale | zero << 16
   int hist;   // [2][GRP][kFBins] this CTA's level histograms (double-buffered)
   int hsum;   // [GRP][kFBins] the cluster's sum of the current level
+  int hred;   // [GRP][kFBins] (this CTA's slice of) the cluster's sum, read remotely
   int bkey;   // [kFBandCap] exact keys of the band of the head this CTA owns
   int btok;   // [kFBandCap] their tokens
   int stg;    // [kFStgCap][8 words] value refinement rows of union tokens
@@ -96,6 +98,7 @@ __host__ __device__ inline FusedSmem fused_smem(int grp, int R) {
   s.vsz = take(R * 4);
   s.hist = take(2 * grp * kFBins * 4);
   s.hsum = take(grp * kFBins * 4);
+  s.hred = take(grp * kFBins * 4);
   s.bkey = take(kFBandCap * 8);
   s.btok = take(kFBandCap * 4);
   s.stg = take(kFStgCap * kWordsPerRow * 4);
@@ -238,30 +241,46 @@ __device__ __forceinline__ double exact_key(const uint32_t* w, double sv, double
 
 // Warp search of a level's 256 summed bins from the top for the kk-th
 // largest: returns the bin (or -1 when it lies below the window), the count
-// above that bin, and the window's total.
+// above that bin, and the window's total.  Lane l holds the run of bins
+// [248 - 8 l, 256 - 8 l); one scan over the lanes finds the run that crosses
+// kk, and that lane walks it.
 __device__ __forceinline__ void window_find(const int* hs, int kk, int* bin_out, int* above_out, int* tot_out) {
   const int lane = threadIdx.x & 31;
-  int above = 0, bin = -1, abv = 0;
-  for (int base = kFBins - 1; base >= 0; base -= 32) {
-    const int b = base - lane;
-    const int c = hs[b];
-    int incl = c;
+  const int4* h4 = reinterpret_cast<const int4*>(hs + kFBins - 8 - 8 * lane);
+  const int4 lo4 = h4[0], hi4 = h4[1];
+  const int c[8] = {hi4.w, hi4.z, hi4.y, hi4.x, lo4.w, lo4.z, lo4.y, lo4.x};  // descending bins
+  int sum = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
+  for (int j = 0; j < 8; ++j) sum += c[j];
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int excl = incl - sum, tot = __shfl_sync(0xffffffffu, incl, 31);
+  const unsigned m = __ballot_sync(0xffffffffu, excl < kk && incl >= kk);
+  int bin = -1, above = tot;
+  if (m) {
+    const int src = __ffs(m) - 1;
+    int b = 0, a = 0;
+    if (lane == src) {
+      a = excl;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (a + c[j] >= kk) {
+          b = kFBins - 1 - 8 * lane - j;
+          break;
+        }
+        a += c[j];
+      }
     }
-    const unsigned m = __ballot_sync(0xffffffffu, bin < 0 && above + incl >= kk && above + incl - c < kk);
-    if (bin < 0 && m) {
-      const int src = __ffs(m) - 1;
-      bin = base - src;
-      abv = above + __shfl_sync(0xffffffffu, incl - c, src);
-    }
-    above += __shfl_sync(0xffffffffu, incl, 31);
+    bin = __shfl_sync(0xffffffffu, b, src);
+    above = __shfl_sync(0xffffffffu, a, src);
   }
   *bin_out = bin;
-  *above_out = bin >= 0 ? abv : above;
-  *tot_out = above;
+  *above_out = above;
+  *tot_out = tot;
 }
 
 // 12-pass radix selection over (exact key desc, token asc) of n entries in
@@ -375,6 +394,7 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
   uint32_t* vsz = reinterpret_cast<uint32_t*>(smem + S.vsz);
   int* hist = reinterpret_cast<int*>(smem + S.hist);
   int* hsum = reinterpret_cast<int*>(smem + S.hsum);
+  int* hred = reinterpret_cast<int*>(smem + S.hred);
   double* bkey = reinterpret_cast<double*>(smem + S.bkey);
   int* btok = reinterpret_cast<int*>(smem + S.btok);
   uint32_t* stg = reinterpret_cast<uint32_t*>(smem + S.stg);
@@ -397,6 +417,8 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
   __shared__ int s_sh[GRP], kk_sh[GRP], cnt_sh[GRP], done_sh[GRP];
   __shared__ int nal[GRP];               // published: tokens of this range selected outright, per head
   __shared__ int bcnt;                   // band entries pushed to this CTA (the owner of head r)
+  __shared__ int lbn;                    // band entries of this range
+  __shared__ int lband[kFLocalBand];     // (token << 3 | head) of this range's band entries
   __shared__ int kB_sh;
   __shared__ int ucnt, uoff;             // published: union tokens of this range
   __shared__ float part[GRP][D + 2];     // published: (max, sum, output) of this range per head
@@ -430,6 +452,7 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
   if (tid == 0) {
     l0[2 * GRP] = 0u;
     bcnt = 0;
+    lbn = 0;
     flag_sh = 0;
   }
   {
@@ -484,13 +507,18 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
       emin = min(emin, __shfl_xor_sync(0xffffffffu, emin, o));
       emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
     }
-    // the exponent of max |q| is the largest exponent
+    // the sum of q (any order: the error bound covers it), the exponent of
+    // max |q| (the largest exponent)
+    float qsum_l = (v[0] + v[1]) + (v[2] + v[3]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) qsum_l += __shfl_xor_sync(0xffffffffu, qsum_l, o);
     const int e = emax >= emin ? emax : 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) qx[h][4 * lane + i] = __float2int_rn(scale2(v[i], 23 - e));
     if (lane == 0) {
       const int span = emax >= emin ? emax - emin : 0;  // binades spanned by the nonzero q
       qsc[h] = pow2f(e - 23);
+      qsm[h] = qsum_l;
       qe_sh[h] = e;
       ikey_sh[h] = span <= 15;
       l1_sh[h] = l1;
@@ -499,12 +527,6 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
     }
   }
   __syncthreads();
-  if (tid < GRP) {
-    float s = 0.0f;
-#pragma unroll 4
-    for (int d = 0; d < D; ++d) s += qs[tid][d];
-    qsm[tid] = s;
-  }
   for (int e = tid; e < GRP * 96; e += kFThreads) {
     const int h = e / 96, x = e % 96, p = x / 32, wi = (x / 4) & 7, kq = x & 3;
     uint32_t v = 0;
@@ -697,27 +719,39 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
         if (done_sh[h]) continue;
         const uint32_t wlo = wlo_sh[h], hi = hi_sh[h];
         const int s = s_sh[h];
-#pragma unroll 2
-        for (int i = tid; i < n; i += kFThreads) {
-          const uint32_t key = okey32(sc[h * R + i]);
-          if (key >= wlo && key <= hi) atomicAdd(&hb[h * kFBins + ((key - wlo) >> s)], 1);
+        float v[kPT];  // every score of this thread is loaded before the first count
+#pragma unroll
+        for (int j = 0; j < kPT; ++j) {
+          const int i = tid + j * kFThreads;
+          v[j] = i < n ? sc[h * R + i] : 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < kPT; ++j) {
+          const uint32_t key = okey32(v[j]);
+          if (tid + j * kFThreads < n && key >= wlo && key <= hi) atomicAdd(&hb[h * kFBins + ((key - wlo) >> s)], 1);
         }
       }
       cl.sync();  // B: every CTA's histogram of this level is published
-      for (int i4 = tid; i4 < GRP * kFBins / 4; i4 += kFThreads) {
-        int4 v[kFMaxCluster];
-#pragma unroll
-        for (int c = 0; c < kFMaxCluster; ++c)
-          v[c] = c < C ? dsm_ld_v4(dsm_addr(reinterpret_cast<const int4*>(hb) + i4, c)) : make_int4(0, 0, 0, 0);
-        int4 acc = v[0];
-#pragma unroll
-        for (int c = 1; c < kFMaxCluster; ++c) {
-          acc.x += v[c].x;
-          acc.y += v[c].y;
-          acc.z += v[c].z;
-          acc.w += v[c].w;
+      // the sum over the cluster in two steps: CTA r sums its slice of the
+      // bins over every CTA, then every CTA gathers all the slices
+      {
+        constexpr int Q = GRP * kFBins / 4;  // int4s of a histogram
+        const int S4 = (Q + C - 1) / C;
+        for (int q = r * S4 + tid; q < min(Q, (r + 1) * S4); q += kFThreads) {
+          int4 acc = make_int4(0, 0, 0, 0);
+#pragma unroll 4
+          for (int c = 0; c < C; ++c) {
+            const int4 v = dsm_ld_v4(dsm_addr(reinterpret_cast<const int4*>(hb) + q, c));
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+          }
+          reinterpret_cast<int4*>(hred)[q] = acc;
         }
-        reinterpret_cast<int4*>(hsum)[i4] = acc;
+        cl.sync();  // B2: every slice is summed
+        for (int q = tid; q < Q; q += kFThreads)
+          reinterpret_cast<int4*>(hsum)[q] = dsm_ld_v4(dsm_addr(reinterpret_cast<const int4*>(hred) + q, q / S4));
       }
       __syncthreads();
       if (warp < GRP && !done_sh[warp]) {
@@ -751,25 +785,67 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
       fthr_sh[tid] = __double2float_ru(static_cast<double>(from_okey32(lo_sh[tid])) - 2.0 * eps_sh[tid]);
     }
     __syncthreads();
-    for (int i = tid; i < n; i += kFThreads) {
-      bool any = false, band = false;
-#pragma unroll 1
-      for (int h = 0; h < GRP; ++h) {
-        const float v = sc[h * R + i];
-        if (static_cast<double>(v) > hiA_sh[h]) {
-          any = true;
-          atomicAdd(&nal[h], 1);
-        } else if (v >= fthr_sh[h]) {
-          band = true;
-          band_push(a.k_res + (row0 + i) * kWordsPerRow, ksz[i], ikey_sh[h] != 0, qpl[h], qxs[h], qe_sh[h], qs[h],
-                    h, &bcnt, bkey, btok, a.ovf_key + (static_cast<size_t>(g) * GRP + h) * T,
-                    a.ovf_tok + (static_cast<size_t>(g) * GRP + h) * T, t0 + i);
+    // pass 1: the outright selections (bitmask, counts per head) and a list
+    // of this range's band entries; pass 2 re-keys the entries in parallel
+    {
+      int nA[GRP];
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) nA[h] = 0;
+#pragma unroll
+      for (int j = 0; j < kPT; ++j) {
+        const int i = tid + j * kFThreads;
+        if (i >= n) break;
+        bool any = false, band = false;
+#pragma unroll
+        for (int h = 0; h < GRP; ++h) {
+          const float v = sc[h * R + i];
+          if (static_cast<double>(v) > hiA_sh[h]) {
+            any = true;
+            ++nA[h];
+          } else if (v >= fthr_sh[h]) {
+            band = true;
+            const int pos = atomicAdd(&lbn, 1);
+            if (pos < kFLocalBand) lband[pos] = (i << 3) | h;
+          }
+        }
+        if (any) atomicOr(&umask[i >> 5], 1u << (i & 31));
+        if (any || band) {
+          l2_prefetch_line(a.k_ref + (row0 + i) * kWordsPerRow);
+          l2_prefetch_line(a.v_ref + (row0 + i) * kWordsPerRow);
         }
       }
-      if (any) atomicOr(&umask[i >> 5], 1u << (i & 31));
-      if (any || band) {
-        l2_prefetch_line(a.k_ref + (row0 + i) * kWordsPerRow);
-        l2_prefetch_line(a.v_ref + (row0 + i) * kWordsPerRow);
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) {
+        int v = nA[h];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0 && v) atomicAdd(&nal[h], v);
+      }
+    }
+    __syncthreads();
+    {
+      const int nb = lbn;
+      for (int e = tid; e < nb; e += kFThreads) {
+        int i = 0, h = 0;
+        if (nb <= kFLocalBand) {
+          i = lband[e] >> 3;
+          h = lband[e] & 7;
+        } else {  // the list overflowed: the e-th band entry in (token, head) order is found again
+          int cnt = 0;
+          bool found = false;
+          for (int ii = 0; ii < n && !found; ++ii)
+            for (int hh = 0; hh < GRP && !found; ++hh) {
+              const float v = sc[hh * R + ii];
+              if (!(static_cast<double>(v) > hiA_sh[hh]) && v >= fthr_sh[hh] && cnt++ == e) {
+                i = ii;
+                h = hh;
+                found = true;
+              }
+            }
+        }
+        band_push(a.k_res + (row0 + i) * kWordsPerRow, ksz[i], ikey_sh[h] != 0, qpl[h], qxs[h], qe_sh[h], qs[h], h,
+                  &bcnt, bkey, btok, a.ovf_key + (static_cast<size_t>(g) * GRP + h) * T,
+                  a.ovf_tok + (static_cast<size_t>(g) * GRP + h) * T, t0 + i);
       }
     }
     cl.sync();  // C: band entries and outright counts are published
@@ -824,21 +900,32 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
   // ---- 4. output over this range
   // the union tokens of the range, ascending; their value refinement rows are
   // staged for the corrections
-  int nu;
-  {
-    const int nw = (n + 31) >> 5;  // <= R / 32 <= blockDim
-    uint32_t bits = tid < nw ? umask[tid] : 0u;
-    int tot;
-    int pos = sfd::block_exclusive_scan(__popc(bits), scan_scratch, &tot);
-    while (bits) {
-      const int b = __ffs(bits) - 1;
-      bits &= bits - 1u;
-      ulist[pos++] = static_cast<uint16_t>(32 * tid + b);
+  if (warp == 0) {
+    // warp 0 scans the bitmask: lane l holds words 2 l, 2 l + 1 (R <= 2048)
+    const int nw = (n + 31) >> 5;
+    uint32_t b0 = 2 * lane < nw ? umask[2 * lane] : 0u, b1 = 2 * lane + 1 < nw ? umask[2 * lane + 1] : 0u;
+    const int cnt = __popc(b0) + __popc(b1);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
-    if (tid == 0) ucnt = tot;
-    nu = tot;
-    __syncthreads();
+    int pos = incl - cnt;
+    while (b0) {
+      const int b = __ffs(b0) - 1;
+      b0 &= b0 - 1u;
+      ulist[pos++] = static_cast<uint16_t>(64 * lane + b);
+    }
+    while (b1) {
+      const int b = __ffs(b1) - 1;
+      b1 &= b1 - 1u;
+      ulist[pos++] = static_cast<uint16_t>(64 * lane + 32 + b);
+    }
+    if (lane == 31) ucnt = incl;
   }
+  __syncthreads();
+  const int nu = ucnt;
   for (int u = tid; u < min(nu, kFStgCap); u += kFThreads) {
     const uint32_t* src = a.v_ref + (row0 + ulist[u]) * kWordsPerRow;
     cp_async16_attn(stg + u * kWordsPerRow, src);
