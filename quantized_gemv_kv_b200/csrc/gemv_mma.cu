@@ -128,13 +128,14 @@ __device__ __forceinline__ void qf_frag(uint32_t wa, uint32_t wb, int g8, int of
 
 template <int SPW>
 struct MCfg {
-  static constexpr int kStages = SPW == 1 ? 8 : 6;
+  static constexpr int kStages = SPW == 1 ? 8 : 5;  // 16 warps of two slices fit 227 KB
+  static constexpr int kRedTiles = SPW == 1 ? 16 : 4;  // tiles whose warp partials wait for one reduction
   static constexpr int SW = SPW * kSliceWords;  // ring words per warp and stage
   static size_t smem_bytes(int W) {
     return sizeof(uint32_t) * (static_cast<size_t>(W) * kStages * SW           // rings
                                + static_cast<size_t>(W) * SPW * kCorrList       // refinement rows (issue job)
                                + static_cast<size_t>(W) * SPW * kCorrList / 2   // listed channels (u16)
-                               + 2 * static_cast<size_t>(W) * kRows);           // row partials
+                               + static_cast<size_t>(kRedTiles) * W * kRows);   // row partials of the warps
   }
 };
 
@@ -142,7 +143,7 @@ template <int SPW, int BF>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1)
 gemv_mma_kernel(const __grid_constant__ MArgs a) {
   using C = MCfg<SPW>;
-  constexpr int kStages = C::kStages, SW = C::SW;
+  constexpr int kStages = C::kStages, SW = C::SW, kRedTiles = C::kRedTiles;
   extern __shared__ __align__(16) uint32_t sm[];
   const int W = blockDim.x >> 5;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, tig = lane & 3;
@@ -159,12 +160,81 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
   const float m_f = static_cast<float>((1 << BF) - 1) * 0.5f;
   const uint32_t fmask = (1u << BF) - 1u;
 
-  // ---- per-warp setup: B fragments, group scalars, selection lists, the
-  // correction MMA's B fragments (x of the listed channels, high and low)
+  const size_t row_words = static_cast<size_t>(a.K) / 16;
+  const int last = a.njobs - 1;
+  const int total_tiles = a.job[last].tile_begin + a.job[last].N / kRows;
+  // a contiguous block of tiles per CTA: consecutive tiles read consecutive
+  // words of each selected channel's refinement row (one sector serves 8 or 16)
+  const int per_cta = (total_tiles + ncta - 1) / ncta;
+  const int t_begin = crow * per_cta;
+  const int my_tiles = max(0, min(total_tiles, t_begin + per_cta) - t_begin);
+  int issue_job = -1;
+  // per-warp state filled by the setup below (after the dependency wait)
   uint32_t bf[SPW][8][2];
   uint32_t cb[SPW][2][2];
   float fsc[SPW], gsm[SPW], cconst[SPW];
   int nsl[SPW], psl[SPW];
+
+  // codes and scale/zero of tile i (they depend on nothing the previous
+  // kernel writes), then the refinement words of its listed channels
+  auto issue_codes = [&](int i) {
+    const int st = i % kStages;
+    const int t = t_begin + i;
+    const MJob& J = a.job[job_of(a, t)];
+    const int row0 = (t - J.tile_begin) * kRows;
+#pragma unroll
+    for (int sp = 0; sp < SPW; ++sp) {
+      uint32_t* base = ring + st * SW + sp * kSliceWords;
+      const int slice = slice0 + sp;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int row = (lane >> 2) + 8 * h, c = lane & 3;
+        cp_async16(base + code_off(row, c), J.res + static_cast<size_t>(row0 + row) * row_words + 16 * slice + 4 * c);
+      }
+      if (lane < 8) {  // (group, scale|zero, half of the 16 rows)
+        const int grp = lane >> 2, arr = (lane >> 1) & 1, hf = lane & 1;
+        const uint16_t* src = (arr ? J.zero : J.scale) + static_cast<size_t>(2 * slice + grp) * J.N + row0 + 8 * hf;
+        cp_async16(reinterpret_cast<uint16_t*>(base + 256) + (grp * 2 + arr) * 16 + 8 * hf, src);
+      }
+    }
+  };
+  auto issue_refs = [&](int i) {
+    const int st = i % kStages;
+    const int t = t_begin + i;
+    const int jb = job_of(a, t);
+    const MJob& J = a.job[jb];
+    const int row0 = (t - J.tile_begin) * kRows;
+    if (jb != issue_job) {  // refinement rows of the listed channels, for this matrix
+      issue_job = jb;
+      if (J.ref_rows) {
+#pragma unroll
+        for (int sp = 0; sp < SPW; ++sp)
+          if (lane < min(nsl[sp], kCorrList))
+            selr[sp * kCorrList + lane] =
+                J.row_of ? J.row_of[psl[sp] + lane] : 256 * (slice0 + sp) + mylist[sp * kCorrList + lane];
+      }
+      __syncwarp();
+    }
+    if (!J.ref_rows) return;
+#pragma unroll
+    for (int sp = 0; sp < SPW; ++sp) {
+      uint32_t* base = ring + st * SW + sp * kSliceWords;
+      if (lane < min(nsl[sp], kCorrList))
+        cp_async4(base + 288 + lane,
+                  J.ref_rows + static_cast<size_t>(selr[sp * kCorrList + lane]) * J.unit_words + ((row0 * BF) >> 5));
+    }
+  };
+
+#pragma unroll
+  for (int i = 0; i < kStages - 1; ++i) {
+    if (i < my_tiles) issue_codes(i);
+    cp_async_commit();
+  }
+  // x, the prepared activations and the refinement rows may come from the
+  // previous kernel on the stream: everything below reads them
+  sfd::pdl_wait();
+  // ---- per-warp setup: B fragments, group scalars, selection lists, the
+  // correction MMA's B fragments (x of the listed channels, high and low)
 #pragma unroll
   for (int sp = 0; sp < SPW; ++sp) {
     const int slice = slice0 + sp;
@@ -238,62 +308,25 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
       }
   }
 
-  const size_t row_words = static_cast<size_t>(a.K) / 16;
-  const int last = a.njobs - 1;
-  const int total_tiles = a.job[last].tile_begin + a.job[last].N / kRows;
-  // a contiguous block of tiles per CTA: consecutive tiles read consecutive
-  // words of each selected channel's refinement row (one sector serves 8 or 16)
-  const int per_cta = (total_tiles + ncta - 1) / ncta;
-  const int t_begin = crow * per_cta;
-  const int my_tiles = max(0, min(total_tiles, t_begin + per_cta) - t_begin);
-  int issue_job = -1;
-
-  auto issue = [&](int i) {
-    const int st = i % kStages;
-    const int t = t_begin + i;
-    const int jb = job_of(a, t);
-    const MJob& J = a.job[jb];
-    const int row0 = (t - J.tile_begin) * kRows;
-    if (jb != issue_job) {  // refinement rows of the listed channels, for this matrix
-      issue_job = jb;
-      if (J.ref_rows) {
-#pragma unroll
-        for (int sp = 0; sp < SPW; ++sp)
-          if (lane < min(nsl[sp], kCorrList))
-            selr[sp * kCorrList + lane] =
-                J.row_of ? J.row_of[psl[sp] + lane] : 256 * (slice0 + sp) + mylist[sp * kCorrList + lane];
-      }
-      __syncwarp();
-    }
-#pragma unroll
-    for (int sp = 0; sp < SPW; ++sp) {
-      uint32_t* base = ring + st * SW + sp * kSliceWords;
-      const int slice = slice0 + sp;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int row = (lane >> 2) + 8 * h, c = lane & 3;
-        cp_async16(base + code_off(row, c), J.res + static_cast<size_t>(row0 + row) * row_words + 16 * slice + 4 * c);
-      }
-      if (lane < 8) {  // (group, scale|zero, half of the 16 rows)
-        const int grp = lane >> 2, arr = (lane >> 1) & 1, hf = lane & 1;
-        const uint16_t* src = (arr ? J.zero : J.scale) + static_cast<size_t>(2 * slice + grp) * J.N + row0 + 8 * hf;
-        cp_async16(reinterpret_cast<uint16_t*>(base + 256) + (grp * 2 + arr) * 16 + 8 * hf, src);
-      }
-      if (J.ref_rows && lane < min(nsl[sp], kCorrList))
-        cp_async4(base + 288 + lane,
-                  J.ref_rows + static_cast<size_t>(selr[sp * kCorrList + lane]) * J.unit_words + ((row0 * BF) >> 5));
-    }
-  };
-
-#pragma unroll
-  for (int i = 0; i < kStages - 1; ++i) {
-    if (i < my_tiles) issue(i);
-    cp_async_commit();
-  }
+  for (int i = 0; i < kStages - 1 && i < my_tiles; ++i) issue_refs(i);
+  cp_async_commit();
   for (int i = 0; i < my_tiles; ++i) {
-    if (i + kStages - 1 < my_tiles) issue(i + kStages - 1);
+    if (i + kStages - 1 < my_tiles) {
+      issue_codes(i + kStages - 1);
+      issue_refs(i + kStages - 1);
+    }
     cp_async_commit();
-    cp_async_wait<kStages - 1>();
+    // tile i needs its code group and the prologue's refinement group, which
+    // has i + 1 newer groups while i + 1 < kStages - 1
+    switch (min(i + 1, kStages - 1)) {
+      case 1: cp_async_wait<1>(); break;
+      case 2: cp_async_wait<2>(); break;
+      case 3: cp_async_wait<3>(); break;
+      case 4: cp_async_wait<4>(); break;
+      case 5: cp_async_wait<5>(); break;
+      case 6: cp_async_wait<6>(); break;
+      default: cp_async_wait<kStages - 1>(); break;
+    }
     __syncwarp();
     const int st = i % kStages;
     const int t = t_begin + i;
@@ -377,19 +410,29 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
       }
       v = fmaf(sc, tsum, v);
     }
-    // lanes tig and tig ^ 2 hold the same row for the two groups
+    // lanes tig and tig ^ 2 hold the same row for the two groups; the warps'
+    // partials of up to kRedTiles tiles are summed together (no barrier per tile)
     v += __shfl_xor_sync(0xffffffffu, v, 2);
-    float* rb = red + (i & 1) * W * kRows;
-    if (tig < 2) rb[warp * kRows + myrow] = v;
-    __syncthreads();
-    if (tid < kRows) {
-      float acc = 0.0f;
-      for (int w = 0; w < W; ++w) acc += rb[w * kRows + tid];
-      float* dst = J.y + row0 + tid;
-      if (a.ksplit > 1) atomicAdd(dst, acc);
-      else *dst = acc;
+    if (tig < 2) red[((i % kRedTiles) * W + warp) * kRows + myrow] = v;
+    if (i % kRedTiles == kRedTiles - 1 || i == my_tiles - 1) {
+      __syncthreads();
+      const int i0 = i - i % kRedTiles, nt = i - i0 + 1;
+      for (int e = tid; e < nt * kRows; e += blockDim.x) {
+        const int ti = e / kRows, rr = e % kRows;
+        float acc = 0.0f;
+        for (int w = 0; w < W; ++w) acc += red[(ti * W + w) * kRows + rr];
+        const int tt = t_begin + i0 + ti;
+        const MJob& Jt = a.job[job_of(a, tt)];
+        float* dst = Jt.y + (tt - Jt.tile_begin) * kRows + rr;
+        if (a.ksplit > 1) atomicAdd(dst, acc);
+        else *dst = acc;
+      }
+      __syncthreads();
     }
   }
+  // the next kernel launches once every block is past its tiles (launching it
+  // earlier only makes its blocks compete for the SMs and the memory)
+  sfd::pdl_trigger();
   cp_async_wait<0>();
 }
 
@@ -468,9 +511,23 @@ extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, c
   const int sms = sf::sm_count();
   const int nrow_cta = std::max(1, std::min(row_tiles, std::max(1, sms / ksplit)));
   const dim3 grid(nrow_cta * ksplit), block(32 * warps);
+  // programmatic launch: the kernel streams its weights while the previous
+  // kernel on the stream finishes, and waits for it before reading x, the
+  // prepared activations or the refinement rows (the weights must not be
+  // written by that kernel)
   auto launch = [&](auto kern, size_t smem) -> sf_status {
     SF_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
-    kern<<<grid, block, smem, s>>>(a);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kern, a));
     return sf::check_launch("gemv_mma_kernel");
   };
   sf_status st;
