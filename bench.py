@@ -65,6 +65,13 @@ def parse():
 
 # ------------------------------------------------------------------ accounting
 
+# DRAM bytes per launch counted by ncu (dram__bytes_read.sum +
+# dram__bytes_write.sum) for the kernels as they stand; the commands are in
+# profiles/.  They are set back to None whenever the kernel changes.
+ATTN_TRAFFIC_32K = 21443328          # attn_fused_kernel<4>, Hq 32, Hkv 8, T 32768, k 1%
+GEMV_TRAFFIC_PER_LAUNCH = 15847168   # gemv_mma_kernel, mean of a layer's 4 launches (63.39 MB)
+
+
 def gemv_bytes(N, K, k_sel):
     """Algorithmic HBM bytes of one refined GEMV at batch 1."""
     return N * K * B_R // 8 + 4 * N * K // G + k_sel * N * B_F // 8 + 2 * K + 4 * N
@@ -268,6 +275,11 @@ class Model:
         for l in range(self.L):
             for slot, _ in GEMV_LAUNCHES:
                 self.jobs[l][slot].run(self.x(l, slot), self.act[slot][l])
+
+    def attn_only(self):
+        for l in range(self.L):
+            self.sf.attn_decode_refine(self.qin[l], self.kv[l], HKV, self.T, self.k_tok, workspace=self.ws,
+                                       out=self.attn_out[l], sel_out=self.sel_out[l], sel_n=self.sel_n[l])
 
     def sync_caches(self):
         for row in self.mats:
@@ -490,10 +502,29 @@ def run_sf(args, rank, world, local_rank, dist):
             pass
         hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
         peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
-        # dominant kernel: the refined GEMV; time all 224 launches of a step
+        # the dominant kernel (largest share of the step's launch list): the
+        # cluster attention; its launches of a step run in one graph, timed
+        # with events on the launch stream.  traffic: ncu DRAM bytes of one
+        # launch of the same kernel (profiles/attn_fused_kernel_32k.md)
         model.sync_caches()
-        g2 = capture(torch, model.gemvs_only, cap_stream)
         reps = 5
+        g4 = capture(torch, model.attn_only, cap_stream)
+        for _ in range(2):
+            with torch.cuda.stream(cap_stream):
+                g4.replay()
+        ms_a = timed(torch, dist, lambda i: g4.replay(), reps, cap_stream)
+        t_attn = ms_a / reps / args.layers * 1e-3
+        attn_launch_bytes = attn_step_bytes / args.layers
+        achieved_a = attn_launch_bytes / t_attn / 1e9
+        roofline = {"bound": "hbm", "kernel": "attn_fused_kernel", "achieved": achieved_a, "peak": hbm_peak,
+                    "unit": "GB/s", "frac": achieved_a / hbm_peak,
+                    "traffic": ATTN_TRAFFIC_32K if (T == 32768 and HQ == 32 and HKV == 8) else None,
+                    "peak_source": peak_src, "launch_us": t_attn * 1e6, "bytes_per_launch": attn_launch_bytes}
+        del g4
+        # the batch-1 GEMV, the next kernel by share: all its launches of a step
+        # in one graph.  traffic: ncu DRAM bytes of the four launches of a
+        # layer, per launch (profiles/gemv_mma_kernel_gateup_llama31_8b.md)
+        g2 = capture(torch, model.gemvs_only, cap_stream)
         for _ in range(2):
             with torch.cuda.stream(cap_stream):
                 g2.replay()
@@ -501,10 +532,10 @@ def run_sf(args, rank, world, local_rank, dist):
         n_launch = len(GEMV_LAUNCHES) * args.layers
         t_launch = ms_g / reps / n_launch * 1e-3
         achieved = gemv_step_bytes / n_launch / t_launch / 1e9
-        roofline = {"bound": "hbm", "kernel": "gemv_mma_kernel", "achieved": achieved, "peak": hbm_peak,
-                    "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": None,
-                    "peak_source": peak_src, "launch_us": t_launch * 1e6,
-                    "bytes_per_launch": gemv_step_bytes / n_launch}
+        extras["roofline_gemv"] = {"bound": "hbm", "kernel": "gemv_mma_kernel", "achieved": achieved,
+                                   "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                                   "traffic": GEMV_TRAFFIC_PER_LAUNCH, "peak_source": peak_src,
+                                   "launch_us": t_launch * 1e6, "bytes_per_launch": gemv_step_bytes / n_launch}
         del g2
         # resident-only (quantization-only) decode step, same kernels without refinement
         g3 = capture(torch, lambda: model.step(refine=False), cap_stream)
