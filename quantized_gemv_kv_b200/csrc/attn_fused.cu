@@ -430,10 +430,6 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
   __shared__ int binfo[2];
   __shared__ int rhist[256];
 
-  // q and the caches may come from the previous kernel on the stream, so
-  // nothing is read before it completes
-  sfd::pdl_wait();
-
   // ---- prologue: key ring, scales, q
   const int tpw = (ntile + kFW - 1) / kFW;
   const int tile0 = min(ntile, warp * tpw), tile1 = min(ntile, tile0 + tpw);
@@ -1176,7 +1172,6 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
     }
     part[h][j] = v;
   }
-  sfd::pdl_trigger();  // the next kernel launches as the cluster merges
   cl.sync();  // E: every CTA's partial and union count are published
 
   // ---- merge over the cluster: CTA r writes its share of the group's outputs
@@ -1270,10 +1265,8 @@ cudaLaunchConfig_t fused_config(dim3 grid, size_t smem, int C, cudaStream_t s, c
   attr[0].val.clusterDim.x = static_cast<unsigned>(C);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = 1;
   return cfg;
 }
 
@@ -1291,7 +1284,7 @@ bool fused_fits(const FusedPlan<GRP>& p) {
     cudaFuncSetAttribute(attn_fused_kernel<GRP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     cudaFuncSetAttribute(attn_fused_kernel<GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(fused_smem(GRP, fused_rmax(GRP)).total));
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[1];
     const cudaLaunchConfig_t cfg = fused_config(dim3(p.C, 1), p.smem, p.C, nullptr, attr);
     int nclusters = 0;
     const cudaError_t e = cudaOccupancyMaxActiveClusters(&nclusters, attn_fused_kernel<GRP>, &cfg);
@@ -1325,7 +1318,7 @@ sf_status fused_run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv,
   a.ovf_key = ovf_key;
   a.ovf_tok = ovf_tok;
   a.ovf_sel = ovf_sel;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   const cudaLaunchConfig_t cfg = fused_config(dim3(p.C, Hkv), p.smem, p.C, s, attr);
   SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, attn_fused_kernel<GRP>, a));
   return sf::check_launch("attn_fused_kernel");

@@ -168,61 +168,81 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
   const int per_cta = (total_tiles + ncta - 1) / ncta;
   const int t_begin = crow * per_cta;
   const int my_tiles = max(0, min(total_tiles, t_begin + per_cta) - t_begin);
-  int issue_job = -1;
-  // per-warp state filled by the setup below (after the dependency wait)
+  // per-warp state filled by the setup below (issued after the first code copies)
   uint32_t bf[SPW][8][2];
   uint32_t cb[SPW][2][2];
   float fsc[SPW], gsm[SPW], cconst[SPW];
   int nsl[SPW], psl[SPW];
 
-  // codes and scale/zero of tile i (they depend on nothing the previous
-  // kernel writes), then the refinement words of its listed channels
+  // Copies are issued tile by tile in order, so their addresses advance by
+  // fixed strides and are recomputed only where the next matrix begins.
+  // Code cursor: codes and scale/zero (they depend on nothing the previous
+  // kernel writes); ref cursor: the refinement words of the listed channels.
+  const int crow_l = lane >> 2, cchunk = lane & 3;
+  const int sz_grp = lane >> 2, sz_arr = (lane >> 1) & 1, sz_hf = lane & 1;  // lanes 0-7
+  int c_t = t_begin, c_jb = my_tiles > 0 ? job_of(a, t_begin) : 0, c_next = 0;
+  const uint32_t* c_code = nullptr;  // row (row0 + crow_l) of slice0, this lane's chunk
+  const uint16_t* c_sz = nullptr;    // lanes 0-7: scale or zero of (slice0, group), rows row0 + 8 hf
+  size_t c_szs = 0;                  // elements between consecutive slices' scale rows
+  auto c_seek = [&]() {              // the cursor's tile starts (or the job changes)
+    const MJob& J = a.job[c_jb];
+    const int row0 = (c_t - J.tile_begin) * kRows;
+    c_next = c_jb + 1 < a.njobs ? a.job[c_jb + 1].tile_begin : 0x7FFFFFFF;
+    c_code = J.res + static_cast<size_t>(row0 + crow_l) * row_words + 16 * slice0 + 4 * cchunk;
+    c_szs = 2 * static_cast<size_t>(J.N);
+    c_sz = (sz_arr ? J.zero : J.scale) + static_cast<size_t>(2 * slice0 + sz_grp) * J.N + row0 + 8 * sz_hf;
+  };
+  if (my_tiles > 0) c_seek();
+  const int c_jb0 = c_jb;
   auto issue_codes = [&](int i) {
-    const int st = i % kStages;
-    const int t = t_begin + i;
-    const MJob& J = a.job[job_of(a, t)];
-    const int row0 = (t - J.tile_begin) * kRows;
+    if (c_t == c_next) {
+      ++c_jb;
+      c_seek();
+    }
+    uint32_t* stage = ring + (i % kStages) * SW;
 #pragma unroll
     for (int sp = 0; sp < SPW; ++sp) {
-      uint32_t* base = ring + st * SW + sp * kSliceWords;
-      const int slice = slice0 + sp;
+      uint32_t* base = stage + sp * kSliceWords;
+      cp_async16(base + code_off(crow_l, cchunk), c_code + 16 * sp);
+      cp_async16(base + code_off(crow_l + 8, cchunk), c_code + 8 * row_words + 16 * sp);
+      if (lane < 8)
+        cp_async16(reinterpret_cast<uint16_t*>(base + 256) + (sz_grp * 2 + sz_arr) * 16 + 8 * sz_hf,
+                   c_sz + sp * c_szs);
+    }
+    c_code += kRows * row_words;
+    c_sz += kRows;
+    ++c_t;
+  };
+  int r_t = t_begin, r_jb = c_jb0, r_next = 0, r_tb = 0;
+  bool r_has = false;
+  const uint32_t* r_row[SPW];  // lanes below the list length: refinement row of listed channel lane
+  auto r_seek = [&]() {
+    const MJob& J = a.job[r_jb];
+    r_next = r_jb + 1 < a.njobs ? a.job[r_jb + 1].tile_begin : 0x7FFFFFFF;
+    r_tb = J.tile_begin;
+    r_has = J.ref_rows != nullptr;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int row = (lane >> 2) + 8 * h, c = lane & 3;
-        cp_async16(base + code_off(row, c), J.res + static_cast<size_t>(row0 + row) * row_words + 16 * slice + 4 * c);
-      }
-      if (lane < 8) {  // (group, scale|zero, half of the 16 rows)
-        const int grp = lane >> 2, arr = (lane >> 1) & 1, hf = lane & 1;
-        const uint16_t* src = (arr ? J.zero : J.scale) + static_cast<size_t>(2 * slice + grp) * J.N + row0 + 8 * hf;
-        cp_async16(reinterpret_cast<uint16_t*>(base + 256) + (grp * 2 + arr) * 16 + 8 * hf, src);
+    for (int sp = 0; sp < SPW; ++sp) {
+      r_row[sp] = J.ref_rows;
+      if (r_has && lane < min(nsl[sp], kCorrList)) {
+        const int rr = J.row_of ? J.row_of[psl[sp] + lane] : 256 * (slice0 + sp) + mylist[sp * kCorrList + lane];
+        r_row[sp] = J.ref_rows + static_cast<size_t>(rr) * J.unit_words;
       }
     }
   };
   auto issue_refs = [&](int i) {
-    const int st = i % kStages;
-    const int t = t_begin + i;
-    const int jb = job_of(a, t);
-    const MJob& J = a.job[jb];
-    const int row0 = (t - J.tile_begin) * kRows;
-    if (jb != issue_job) {  // refinement rows of the listed channels, for this matrix
-      issue_job = jb;
-      if (J.ref_rows) {
-#pragma unroll
-        for (int sp = 0; sp < SPW; ++sp)
-          if (lane < min(nsl[sp], kCorrList))
-            selr[sp * kCorrList + lane] =
-                J.row_of ? J.row_of[psl[sp] + lane] : 256 * (slice0 + sp) + mylist[sp * kCorrList + lane];
-      }
-      __syncwarp();
+    if (r_t == r_next) {
+      ++r_jb;
+      r_seek();
     }
-    if (!J.ref_rows) return;
+    if (r_has) {
+      const int woff = ((r_t - r_tb) * kRows * BF) >> 5;
+      uint32_t* stage = ring + (i % kStages) * SW;
 #pragma unroll
-    for (int sp = 0; sp < SPW; ++sp) {
-      uint32_t* base = ring + st * SW + sp * kSliceWords;
-      if (lane < min(nsl[sp], kCorrList))
-        cp_async4(base + 288 + lane,
-                  J.ref_rows + static_cast<size_t>(selr[sp * kCorrList + lane]) * J.unit_words + ((row0 * BF) >> 5));
+      for (int sp = 0; sp < SPW; ++sp)
+        if (lane < min(nsl[sp], kCorrList)) cp_async4(stage + sp * kSliceWords + 288 + lane, r_row[sp] + woff);
     }
+    ++r_t;
   };
 
 #pragma unroll
@@ -230,9 +250,6 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
     if (i < my_tiles) issue_codes(i);
     cp_async_commit();
   }
-  // x, the prepared activations and the refinement rows may come from the
-  // previous kernel on the stream: everything below reads them
-  sfd::pdl_wait();
   // ---- per-warp setup: B fragments, group scalars, selection lists, the
   // correction MMA's B fragments (x of the listed channels, high and low)
 #pragma unroll
@@ -308,8 +325,10 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
       }
   }
 
+  if (my_tiles > 0) r_seek();
   for (int i = 0; i < kStages - 1 && i < my_tiles; ++i) issue_refs(i);
   cp_async_commit();
+  int k_jb = c_jb0, k_next = c_jb0 + 1 < a.njobs ? a.job[c_jb0 + 1].tile_begin : 0x7FFFFFFF;  // compute cursor
   for (int i = 0; i < my_tiles; ++i) {
     if (i + kStages - 1 < my_tiles) {
       issue_codes(i + kStages - 1);
@@ -330,7 +349,11 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
     __syncwarp();
     const int st = i % kStages;
     const int t = t_begin + i;
-    const MJob& J = a.job[job_of(a, t)];
+    if (t == k_next) {
+      ++k_jb;
+      k_next = k_jb + 1 < a.njobs ? a.job[k_jb + 1].tile_begin : 0x7FFFFFFF;
+    }
+    const MJob& J = a.job[k_jb];
     const int row0 = (t - J.tile_begin) * kRows;
     const int roff = (row0 * BF) & 31;
     float v = 0.0f;
@@ -430,9 +453,6 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
       __syncthreads();
     }
   }
-  // the next kernel launches once every block is past its tiles (launching it
-  // earlier only makes its blocks compete for the SMs and the memory)
-  sfd::pdl_trigger();
   cp_async_wait<0>();
 }
 
@@ -511,23 +531,9 @@ extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, c
   const int sms = sf::sm_count();
   const int nrow_cta = std::max(1, std::min(row_tiles, std::max(1, sms / ksplit)));
   const dim3 grid(nrow_cta * ksplit), block(32 * warps);
-  // programmatic launch: the kernel streams its weights while the previous
-  // kernel on the stream finishes, and waits for it before reading x, the
-  // prepared activations or the refinement rows (the weights must not be
-  // written by that kernel)
   auto launch = [&](auto kern, size_t smem) -> sf_status {
     SF_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kern, a));
+    kern<<<grid, block, smem, s>>>(a);
     return sf::check_launch("gemv_mma_kernel");
   };
   sf_status st;

@@ -74,13 +74,6 @@ __device__ __forceinline__ float half_bits_to_float(uint16_t h) {
   return __half2float(__ushort_as_half(h));
 }
 
-// Programmatic dependent launch: let the next kernel on the stream launch
-// now (its blocks run once resources free up), and wait until the previous
-// kernel on the stream has completed and its writes are visible.  Both are
-// no-ops for a kernel launched without the programmatic attribute.
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
 // Read `bits` bits starting at stream bit `pos` of a little-endian uint32
 // bitstream (bits <= 8; may straddle a word boundary).
 __device__ __forceinline__ uint32_t read_bits(const uint32_t* s, uint32_t pos, int bits) {
