@@ -357,6 +357,59 @@ def test_attn_band_overflow(sf, attn_path):
     assert np.abs(out.cpu().numpy() - ref["out"]).max() <= ATTN_TOL
 
 
+def _wide_query(seed, Hq, d, scale_exp):
+    """N(0, 1) query heads with one entry of each head scaled by 2^-scale_exp,
+    so the nonzero exponents span about scale_exp binades or a few more."""
+    q = np.random.default_rng(seed).standard_normal((Hq, d)).astype(np.float32)
+    q[:, 5] = np.ldexp(np.where(q[:, 5] >= 0, 1.0, -1.0), -scale_exp).astype(np.float32) * np.abs(q[:, 0])
+    return f32_to_bf16_bits(q)
+
+
+def test_attn_wide_query_span(sf, attn_path):
+    """Query heads whose exponents span 26 binades: beyond the integer-key
+    range (15), within the exact fp64 range (33): the band is re-keyed with
+    fp64 products and the selection must still equal the exact one."""
+    Hq, Hkv, T, d = 8, 2, 6000, 128
+    kv, ok, ov = _kv(sf, Hkv, T, d, 515)
+    qb = _wide_query(516, Hq, d, 26)
+    k = count_fraction(2, T)
+    out, sel, sel_n = sf.attn_decode_refine(bf16_dev(qb), kv, Hkv, T, k)
+    torch.cuda.synchronize()
+    ref = oattn.attn_decode_refine(qb, ok, ov, Hkv, T, k)
+    for g in range(Hkv):
+        n = sel_n.cpu().numpy()[g]
+        assert n == len(ref["union"][g])
+        np.testing.assert_array_equal(sel.cpu().numpy()[g, :n], ref["union"][g])
+    assert np.abs(out.cpu().numpy() - ref["out"]).max() <= ATTN_TOL
+
+
+def test_attn_flags_inexact_query_span(sf):
+    """Query heads spanning 40 binades (beyond 33, where fp64 keys stop being
+    exact): the definition's oracle refuses them, and every KV group reports
+    -1 - (union length) in sel_n on both implementations."""
+    Hq, Hkv, T, d = 8, 2, 4000, 128
+    kv, ok, ov = _kv(sf, Hkv, T, d, 517)
+    qb = _wide_query(518, Hq, d, 40)
+    with pytest.raises(ValueError):
+        oattn.attn_decode_refine(qb, ok, ov, Hkv, T, 40)
+    for path in (sf.ATTN_PIPELINE, sf.ATTN_CLUSTER):
+        sf.attn_set_path(path)
+        try:
+            out, sel, sel_n = sf.attn_decode_refine(bf16_dev(qb), kv, Hkv, T, 40)
+            torch.cuda.synchronize()
+        finally:
+            sf.attn_set_path(sf.ATTN_AUTO)
+        sel_n = sel_n.cpu().numpy()
+        sel = sel.cpu().numpy()
+        for g in range(Hkv):
+            assert sel_n[g] < 0
+            U = -1 - sel_n[g]
+            assert 40 <= U <= (Hq // Hkv) * 40
+            u = sel[g, :U]
+            assert np.all(np.diff(u) > 0) and u[0] >= 0 and u[-1] < T
+        assert np.isfinite(out.cpu().numpy()).all()
+
+
 def test_attn_ties(sf, attn_path):
     """Duplicate tokens give exactly tied keys; the lower token index wins."""
     Hq, Hkv, T, d = 8, 2, 600, 128
