@@ -1127,7 +1127,8 @@ sf_status dispatch(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, 
   if (path != SF_ATTN_PIPELINE) {
     if (sf::attn_fused_eligible(Hq, Hkv, T))
       return sf::attn_fused_run(q, Hq, Hkv, T, kv, k, sel_out, sel_n, out, reinterpret_cast<double*>(ws + L.kap),
-                                reinterpret_cast<int32_t*>(ws + L.cand), reinterpret_cast<int32_t*>(ws + L.sel), s);
+                                reinterpret_cast<int32_t*>(ws + L.cand), reinterpret_cast<int32_t*>(ws + L.sel),
+                                reinterpret_cast<float*>(ws + L.part), reinterpret_cast<int32_t*>(ws + L.fcnt), s);
     if (path == SF_ATTN_CLUSTER)
       return sf::fail(SF_ENOTIMPL, "sf_attn_decode_refine: the cluster kernel does not apply to these sizes");
   }

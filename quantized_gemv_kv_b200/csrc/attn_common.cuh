@@ -13,11 +13,12 @@ namespace sf {
 
 // The single cluster kernel per KV group (attn_fused.cu): whether it applies
 // to these sizes on the current device, and the launch.  The overflow lists
-// (keys, tokens: Hq * T each; winners: Hq * k) live in the caller's workspace.
+// (keys, tokens: Hq * T each; winners: Hq * k), the CTAs' partials and
+// union counts live in the caller's workspace.
 bool attn_fused_eligible(int Hq, int Hkv, int T);
 sf_status attn_fused_run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k, int32_t* sel_out,
                          int32_t* sel_n, float* out, double* ovf_key, int32_t* ovf_tok, int32_t* ovf_sel,
-                         cudaStream_t s);
+                         float* gpart, int32_t* gcnt, cudaStream_t s);
 
 }  // namespace sf
 
@@ -34,7 +35,7 @@ constexpr int kChunk = 4096;       // tokens per CTA of the candidate compaction
 
 struct Layout {
   // from smax on, everything is cleared at the start of a call
-  size_t score, cand, cand2, kap, sel, part, smax, status, count, amax, hist, umask, total;
+  size_t score, cand, cand2, kap, sel, part, fcnt, smax, status, count, amax, hist, umask, total;
   int splits, tps, words_t, nchunks;
 };
 
@@ -55,7 +56,9 @@ Layout make_layout(int Hq, int Hkv, int T, int k, int sms) {
   L.cand2 = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(T));
   L.kap = off; off = up256(off + sizeof(double) * Hq * static_cast<size_t>(T));
   L.sel = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(std::max(k, 1)));
-  L.part = off; off = up256(off + sizeof(float) * Hq * static_cast<size_t>(L.splits) * (D + 2));
+  // split partials of the pipeline, or of the 16 CTAs of a cluster
+  L.part = off; off = up256(off + sizeof(float) * Hq * static_cast<size_t>(std::max(L.splits, 16)) * (D + 2));
+  L.fcnt = off; off = up256(off + sizeof(int32_t) * Hkv * 16);
   L.smax = off; off = up256(off + sizeof(float) * Hkv);
   L.status = off; off = up256(off + sizeof(int32_t) * std::max(Hkv, 4));
   L.count = off; off = up256(off + sizeof(int32_t) * Hkv);

@@ -126,20 +126,11 @@ struct FusedArgs {
   double* ovf_key;   // [Hq][T]
   int32_t* ovf_tok;  // [Hq][T]
   int32_t* ovf_sel;  // [Hq][k]
+  // caller workspace: the CTAs' (max, sum, output) partials and union counts
+  float* gpart;      // [Hkv][16][GRP][D + 2]
+  int32_t* gcnt;     // [Hkv][16]
 };
 
-// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned, size a multiple of 16).
-__device__ __forceinline__ void l2_prefetch_bulk(const void* p, size_t bytes) {
-  const char* c = static_cast<const char*>(p);
-  constexpr size_t kPiece = 16384;
-  for (size_t o = 0; o < bytes; o += kPiece) {
-    const unsigned sz = static_cast<unsigned>(bytes - o < kPiece ? bytes - o : kPiece);
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(c + o), "r"(sz) : "memory");
-  }
-}
-__device__ __forceinline__ void l2_prefetch_line(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
 
 // Distributed shared memory: the address of p in CTA `rank` of the cluster,
 // and plain (relaxed) accesses to it; the cluster barrier orders them.
@@ -155,7 +146,6 @@ __device__ __forceinline__ uint32_t dsm_ld_u32(uint32_t a) {
   asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
   return v;
 }
-__device__ __forceinline__ float dsm_ld_f32(uint32_t a) { return __uint_as_float(dsm_ld_u32(a)); }
 __device__ __forceinline__ int4 dsm_ld_v4(uint32_t a) {
   int4 v;
   asm volatile("ld.shared::cluster.v4.s32 {%0, %1, %2, %3}, [%4];"
@@ -400,6 +390,12 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
   uint32_t* stg = reinterpret_cast<uint32_t*>(smem + S.stg);
   uint32_t* umask = reinterpret_cast<uint32_t*>(smem + S.umask);
   uint16_t* ulist = reinterpret_cast<uint16_t*>(smem + S.ulist);
+  // staging of the outright selections' key rows in the histograms' space
+  // (after the radix levels): a slot per local token (0xFF: none), then the
+  // rows, 16 words each (resident codes, refinement codes)
+  uint8_t* smap = smem + S.hist;
+  uint32_t* kst = reinterpret_cast<uint32_t*>(smem + S.hist + R);
+  const int kst_cap = min(255, (S.hred - S.hist - R) / (2 * kWordsPerRow * 4));
 
   __shared__ int qx[GRP][D];         // fixed-point query heads
   __shared__ float qs[GRP][D];       // query heads in fp32 (exact: bf16)
@@ -418,10 +414,10 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
   __shared__ int nal[GRP];               // published: tokens of this range selected outright, per head
   __shared__ int bcnt;                   // band entries pushed to this CTA (the owner of head r)
   __shared__ int lbn;                    // band entries of this range
+  __shared__ int nst;                    // staged key rows
   __shared__ int lband[kFLocalBand];     // (token << 3 | head) of this range's band entries
   __shared__ int kB_sh;
-  __shared__ int ucnt, uoff;             // published: union tokens of this range
-  __shared__ float part[GRP][D + 2];     // published: (max, sum, output) of this range per head
+  __shared__ int ucnt, uoff;             // union tokens of this range, and their offset in the group's list
   __shared__ float Fc[GRP][kFMaxCluster];
   __shared__ float Lh[GRP], Msh[GRP];
   __shared__ float red[kFW][GRP];
@@ -453,6 +449,7 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
     l0[2 * GRP] = 0u;
     bcnt = 0;
     lbn = 0;
+    nst = 0;
     flag_sh = 0;
   }
   {
@@ -784,6 +781,9 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
       hiA_sh[tid] = static_cast<double>(from_okey32(hi_sh[tid])) + 2.0 * eps_sh[tid];
       fthr_sh[tid] = __double2float_ru(static_cast<double>(from_okey32(lo_sh[tid])) - 2.0 * eps_sh[tid]);
     }
+    // the histograms are dead (and no longer read remotely): their space
+    // stages the key rows of the outright selections for the refined scores
+    for (int w = tid; w < R / 4; w += kFThreads) reinterpret_cast<uint32_t*>(smap)[w] = 0xFFFFFFFFu;
     __syncthreads();
     // pass 1: the outright selections (bitmask, counts per head) and a list
     // of this range's band entries; pass 2 re-keys the entries in parallel
@@ -795,7 +795,7 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
       for (int j = 0; j < kPT; ++j) {
         const int i = tid + j * kFThreads;
         if (i >= n) break;
-        bool any = false, band = false;
+        bool any = false;
 #pragma unroll
         for (int h = 0; h < GRP; ++h) {
           const float v = sc[h * R + i];
@@ -803,15 +803,23 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
             any = true;
             ++nA[h];
           } else if (v >= fthr_sh[h]) {
-            band = true;
             const int pos = atomicAdd(&lbn, 1);
             if (pos < kFLocalBand) lband[pos] = (i << 3) | h;
           }
         }
-        if (any) atomicOr(&umask[i >> 5], 1u << (i & 31));
-        if (any || band) {
-          l2_prefetch_line(a.k_ref + (row0 + i) * kWordsPerRow);
-          l2_prefetch_line(a.v_ref + (row0 + i) * kWordsPerRow);
+        if (any) {
+          atomicOr(&umask[i >> 5], 1u << (i & 31));
+          const int s = atomicAdd(&nst, 1);
+          if (s < kst_cap) {
+            uint32_t* dst = kst + s * 2 * kWordsPerRow;
+            const uint32_t* kr = a.k_res + (row0 + i) * kWordsPerRow;
+            const uint32_t* kf = a.k_ref + (row0 + i) * kWordsPerRow;
+            cp_async16_attn(dst, kr);
+            cp_async16_attn(dst + 4, kr + 4);
+            cp_async16_attn(dst + 8, kf);
+            cp_async16_attn(dst + 12, kf + 4);
+            smap[i] = static_cast<uint8_t>(s);
+          }
         }
       }
 #pragma unroll
@@ -821,6 +829,7 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         if (lane == 0 && v) atomicAdd(&nal[h], v);
       }
+      cp_async_commit_attn();  // the staged key rows
     }
     __syncthreads();
     {
@@ -934,11 +943,20 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
   cp_async_commit_attn();
   // refined scores of the union tokens from their full 4-bit key codes:
   // thread per (head, token), a warp's threads sharing the head
+  cp_async_wait_attn<1>();  // the staged key rows (the value rows may still be in flight)
+  __syncthreads();
   for (int e = tid; e < nu * GRP; e += kFThreads) {
     const int h = e / nu, i = ulist[e - h * nu];
-    const size_t row = row0 + i;
-    const uint4* pr = reinterpret_cast<const uint4*>(a.k_res + row * kWordsPerRow);
-    const uint4* pf = reinterpret_cast<const uint4*>(a.k_ref + row * kWordsPerRow);
+    const int s = selecting ? smap[i] : 0xFF;
+    const uint4* pr;
+    const uint4* pf;
+    if (s != 0xFF) {  // staged during the selection
+      pr = reinterpret_cast<const uint4*>(kst + s * 2 * kWordsPerRow);
+      pf = pr + 2;
+    } else {
+      pr = reinterpret_cast<const uint4*>(a.k_res + (row0 + i) * kWordsPerRow);
+      pf = reinterpret_cast<const uint4*>(a.k_ref + (row0 + i) * kWordsPerRow);
+    }
     const uint4 r0 = pr[0], r1 = pr[1], f0 = pf[0], f1 = pf[1];
     const uint32_t wr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
     const uint32_t wf[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
@@ -1153,6 +1171,7 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
     }
   }
   __syncthreads();
+  float* gp = a.gpart + (static_cast<size_t>(g) * kFMaxCluster + r) * GRP * (D + 2);
   for (int e = tid; e < GRP * (D + 2); e += kFThreads) {
     const int h = e / (D + 2), j = e % (D + 2);
     float v;
@@ -1170,14 +1189,19 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
       // resident value s (2^b_f c + m_f - z): code part 4 (acc - 1024 A), offset part Cs
       v = j == 1 ? Lsum : fmaf(4.0f, o, fmaf(-4096.0f, A, Cs));
     }
-    part[h][j] = v;
+    gp[e] = v;
   }
-  cl.sync();  // E: every CTA's partial and union count are published
+  if (tid == 0) a.gcnt[g * kFMaxCluster + r] = nu;
+  // E: every CTA's partials and union count are in the workspace (the cluster
+  // barrier orders the global writes before the reads below); no shared
+  // memory is read across CTAs after it, so CTAs leave independently
+  cl.sync();
 
   // ---- merge over the cluster: CTA r writes its share of the group's outputs
+  const float* gpg = a.gpart + static_cast<size_t>(g) * kFMaxCluster * GRP * (D + 2);
   if (warp == 0) {
     // union offset of this range and the group's union length
-    const int cc = lane < C ? static_cast<int>(dsm_ld_u32(dsm_addr(&ucnt, lane))) : 0;
+    const int cc = lane < C ? __ldcg(a.gcnt + g * kFMaxCluster + lane) : 0;
     int incl = cc;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -1193,8 +1217,8 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
     for (int h0 = 0; h0 < GRP; h0 += 2) {
       const int h = h0 + (lane >> 4), c = lane & 15;
       const bool ok = h < GRP && c < C;
-      const float m = ok ? dsm_ld_f32(dsm_addr(&part[h][0], c)) : -INFINITY;
-      const float l = ok ? dsm_ld_f32(dsm_addr(&part[h][1], c)) : 0.0f;
+      const float m = ok ? __ldcg(gpg + (c * GRP + h) * (D + 2)) : -INFINITY;
+      const float l = ok ? __ldcg(gpg + (c * GRP + h) * (D + 2) + 1) : 0.0f;
       float mx = m;
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -1222,7 +1246,7 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
         h = e / D;
         d = e % D;
 #pragma unroll 4
-        for (int c = part_i; c < C; c += L) A = fmaf(Fc[h][c], dsm_ld_f32(dsm_addr(&part[h][2 + d], c)), A);
+        for (int c = part_i; c < C; c += L) A = fmaf(Fc[h][c], __ldcg(gpg + (c * GRP + h) * (D + 2) + 2 + d), A);
       }
       for (int o = L >> 1; o > 0; o >>= 1) A += __shfl_xor_sync(0xffffffffu, A, o);
       if (e < e1 && part_i == 0) a.out[(static_cast<size_t>(g) * GRP + h) * D + d] = A / Lh[h];
@@ -1235,7 +1259,6 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
     const int off = uoff, cap = GRP * k;
     for (int u = tid; u < nu && off + u < cap; u += kFThreads) so[off + u] = t0 + ulist[u];
   }
-  cl.sync();  // F: no CTA leaves while its shared memory may still be read
 }
 
 template <int GRP>
@@ -1296,7 +1319,8 @@ bool fused_fits(const FusedPlan<GRP>& p) {
 
 template <int GRP>
 sf_status fused_run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k, int32_t* sel_out,
-                    int32_t* sel_n, float* out, double* ovf_key, int32_t* ovf_tok, int32_t* ovf_sel, cudaStream_t s) {
+                    int32_t* sel_n, float* out, double* ovf_key, int32_t* ovf_tok, int32_t* ovf_sel, float* gpart,
+                    int32_t* gcnt, cudaStream_t s) {
   FusedPlan<GRP> p;
   if (!fused_plan<GRP>(T, &p) || !fused_fits<GRP>(p)) return SF_ENOTIMPL;
   FusedArgs a{};
@@ -1318,6 +1342,8 @@ sf_status fused_run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv,
   a.ovf_key = ovf_key;
   a.ovf_tok = ovf_tok;
   a.ovf_sel = ovf_sel;
+  a.gpart = gpart;
+  a.gcnt = gcnt;
   cudaLaunchAttribute attr[1];
   const cudaLaunchConfig_t cfg = fused_config(dim3(p.C, Hkv), p.smem, p.C, s, attr);
   SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, attn_fused_kernel<GRP>, a));
@@ -1341,12 +1367,12 @@ bool attn_fused_eligible(int Hq, int Hkv, int T) {
 
 sf_status attn_fused_run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k, int32_t* sel_out,
                          int32_t* sel_n, float* out, double* ovf_key, int32_t* ovf_tok, int32_t* ovf_sel,
-                         cudaStream_t s) {
+                         float* gpart, int32_t* gcnt, cudaStream_t s) {
   switch (Hq / Hkv) {
-    case 1: return fused_run<1>(q, Hq, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, s);
-    case 2: return fused_run<2>(q, Hq, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, s);
-    case 4: return fused_run<4>(q, Hq, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, s);
-    case 8: return fused_run<8>(q, Hq, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, s);
+    case 1: return fused_run<1>(q, Hq, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, gpart, gcnt, s);
+    case 2: return fused_run<2>(q, Hq, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, gpart, gcnt, s);
+    case 4: return fused_run<4>(q, Hq, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, gpart, gcnt, s);
+    case 8: return fused_run<8>(q, Hq, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, gpart, gcnt, s);
     default: return sf::fail(SF_ENOTIMPL, "attn_fused_run: Hq/Hkv must be 1, 2, 4 or 8");
   }
 }
