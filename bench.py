@@ -252,18 +252,37 @@ class Model:
                 self.selects[l].run()
             self.groups[l].prefetch(self.sel_stream, self.side)
 
+        def prepare_only(l):
+            # the resident-only step prepares its activations the same way,
+            # one layer ahead on the selection stream; main waits for them
+            ev = torch.cuda.Event()
+            ev.record(main)
+            self.sel_stream.wait_event(ev)
+            with torch.cuda.stream(self.sel_stream):
+                for s, _ in SLOTS:
+                    sf.act_prepare(self.x(l, s), self.act0[s][l])
+                done = torch.cuda.Event()
+                done.record(self.sel_stream)
+            return done
+
         def gemv(l, slot):
             if refine:
                 self.jobs[l][slot].run(self.x(l, slot), self.act[slot][l])
             else:
-                sf.act_prepare(self.x(l, slot), self.act0[slot][l])
                 self.jobs0[l][slot].run(self.x(l, slot), self.act0[slot][l])
 
+        ready = {}
         if refine:
             select_and_prefetch(0)
+        else:
+            ready[0] = prepare_only(0)
         for l in range(self.L):
             if refine and l + 1 < self.L:
                 select_and_prefetch(l + 1)
+            if not refine:
+                if l + 1 < self.L:
+                    ready[l + 1] = prepare_only(l + 1)
+                main.wait_event(ready.pop(l))
             gemv(l, "attn_in")
             sf.attn_decode_refine(self.qin[l], self.kv[l], HKV, self.T, self.k_tok if refine else 0,
                                   workspace=self.ws, out=self.attn_out[l], sel_out=self.sel_out[l],
@@ -296,11 +315,19 @@ class Model:
         return tot
 
     def launches_per_step(self, refine=True):
+        """Kernels of the library per step: per layer the four GEMV launches,
+        the attention (one cluster launch up to 32K at <= 4 query heads per KV
+        head, else the pipeline's score, selection and output kernels), and
+        either the selection, LRU index and miss gather (refined) or four
+        activation preparations (resident only)."""
         gemv = len(GEMV_LAUNCHES) * self.L
-        attn = 4 * self.L if (refine and 0 < self.k_tok < self.T) else 2 * self.L
+        if self.T <= 32768 and HQ // HKV <= 4:
+            attn = self.L
+        else:
+            attn = (4 if (refine and 0 < self.k_tok < self.T) else 2) * self.L
         if not refine:
-            return 2 * gemv + attn
-        return self.L + 2 * self.L + gemv + attn
+            return len(SLOTS) * self.L + gemv + attn
+        return 3 * self.L + gemv + attn
 
     def close(self):
         for grp in self.groups:
