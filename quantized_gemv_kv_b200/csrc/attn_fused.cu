@@ -184,6 +184,10 @@ __device__ __forceinline__ float scale2(float v, int k) {
   return k <= 127 ? v * pow2f(k) : (v * pow2f(k - 127)) * pow2f(127);
 }
 
+// Exact int -> fp32 for |v| < 2^22 on the integer and FP32 pipes (no
+// conversion instruction): v rides in the mantissa of 1.5 * 2^23.
+__device__ __forceinline__ float i2f_exact(int v) { return __int_as_float(0x4B400000 + v) - 12582912.0f; }
+
 // Smallest s >= 0 with width <= 256 << s.
 __device__ __forceinline__ int level_shift(unsigned long long width) {
   int s = 0;
@@ -617,12 +621,14 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
             const float sv = sfd::half_bits_to_float(static_cast<uint16_t>(kz & 0xFFFFu));
             const float zv = sfd::half_bits_to_float(static_cast<uint16_t>(kz >> 16));
             const int i0 = 2 * rr, i1 = 2 * rr + 1;
-            const float P0 = (static_cast<float>(d2[u][i0]) * 65536.0f + static_cast<float>(d1[u][i0]) * 256.0f +
-                              static_cast<float>(d0[u][i0])) * qsc0;
+            // plane sums are below 2^17 in magnitude: exact conversions, the
+            // same fp32 combination as the pipeline's score pass
+            const float P0 =
+                (i2f_exact(d2[u][i0]) * 65536.0f + i2f_exact(d1[u][i0]) * 256.0f + i2f_exact(d0[u][i0])) * qsc0;
             sc[h0 * R + tt] = (sv * fmaf(4.0f, P0, (1.5f - zv) * qsm0)) * kInvSqrtD;
             if (h1 < GRP) {
-              const float P1 = (static_cast<float>(d2[u][i1]) * 65536.0f + static_cast<float>(d1[u][i1]) * 256.0f +
-                                static_cast<float>(d0[u][i1])) * qsc1;
+              const float P1 =
+                  (i2f_exact(d2[u][i1]) * 65536.0f + i2f_exact(d1[u][i1]) * 256.0f + i2f_exact(d0[u][i1])) * qsc1;
               sc[h1 * R + tt] = (sv * fmaf(4.0f, P1, (1.5f - zv) * qsm1)) * kInvSqrtD;
             }
           }
@@ -966,7 +972,7 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
       const uint32_t rw = wr[w], fw = wf[w];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const float c = static_cast<float>(((rw >> (2 * j)) & 3u) * 4u + ((fw >> (2 * j)) & 3u));
+        const float c = i2f_exact(static_cast<int>(((rw >> (2 * j)) & 3u) * 4u + ((fw >> (2 * j)) & 3u)));
         P[j & 3] = fmaf(qs[h][16 * w + j], c, P[j & 3]);
       }
     }
@@ -1125,7 +1131,8 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
     for (int h = 0; h < GRP; ++h) {
       const float al = __half2float(as[h * kStr + i]) + __half2float(as[(GRP + h) * kStr + i]);
 #pragma unroll
-      for (int dd = 0; dd < 4; ++dd) uo[h][dd] = fmaf(al, static_cast<float>((wf >> (2 * dd)) & 3u) - 1.5f, uo[h][dd]);
+      for (int dd = 0; dd < 4; ++dd)
+        uo[h][dd] = fmaf(al, i2f_exact(static_cast<int>((wf >> (2 * dd)) & 3u)) - 1.5f, uo[h][dd]);
     }
   }
   __syncthreads();  // every warp is done with the weight tile
