@@ -44,7 +44,18 @@ G, B_R, B_F = 128, 2, 2
 HQ, HKV, D = 32, 8, 128
 TOPK_PCT, CACHE_PCT, OUTLIER_PCT, OUTLIER_SCALE = 3, 10, "1/2", 30.0
 TOK_PCT = 1
-WORKLOAD = "llama31_8b_decode_hotpath_32k"
+
+
+def workload(T):
+    ctx = f"{T // 1024}k" if T % 1024 == 0 else str(T)
+    return f"llama31_8b_decode_hotpath_{ctx}"
+
+
+def cluster_attention(T):
+    """True where the library runs the attention as one cluster launch per
+    layer (up to 32K tokens at <= 4 query heads per KV head), else it runs
+    the score / selection / output pipeline."""
+    return T <= 32768 and HQ // HKV <= 4
 # matrices that read the same activation row share one batch-1 GEMV launch
 GEMV_LAUNCHES = (("attn_in", ("q", "k", "v")), ("attn_out", ("o",)), ("mlp_in", ("gate", "up")),
                  ("mlp_mid", ("down",)))
@@ -68,7 +79,7 @@ def parse():
 # DRAM bytes per launch counted by ncu (dram__bytes_read.sum +
 # dram__bytes_write.sum) for the kernels as they stand; the commands are in
 # profiles/.  They are set back to None whenever the kernel changes.
-ATTN_TRAFFIC_32K = 21443328          # attn_fused_kernel<4>, Hq 32, Hkv 8, T 32768, k 1%
+ATTN_TRAFFIC_32K = 21377280          # attn_fused_kernel<4>, Hq 32, Hkv 8, T 32768, k 1%
 GEMV_TRAFFIC_PER_LAUNCH = 15847168   # gemv_mma_kernel, mean of a layer's 4 launches (63.39 MB)
 
 
@@ -317,14 +328,14 @@ class Model:
     def launches_per_step(self, refine=True):
         """Kernels of the library per step: per layer the four GEMV launches,
         the attention (one cluster launch up to 32K at <= 4 query heads per KV
-        head, else the pipeline's score, selection and output kernels), and
+        head, else the pipeline's score, selection, refinement and output kernels), and
         either the selection, LRU index and miss gather (refined) or four
         activation preparations (resident only)."""
         gemv = len(GEMV_LAUNCHES) * self.L
-        if self.T <= 32768 and HQ // HKV <= 4:
+        if cluster_attention(self.T):
             attn = self.L
         else:
-            attn = (4 if (refine and 0 < self.k_tok < self.T) else 2) * self.L
+            attn = (5 if (refine and 0 < self.k_tok < self.T) else 2) * self.L
         if not refine:
             return len(SLOTS) * self.L + gemv + attn
         return 3 * self.L + gemv + attn
@@ -455,7 +466,7 @@ def run_reference(args, rank):
         "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * t_tot / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy draws)",
-        "config": {"workload": WORKLOAD, "context": T, "layers": args.layers, "batch": 1},
+        "config": {"workload": workload(T), "context": T, "layers": args.layers, "batch": 1},
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -543,7 +554,8 @@ def run_sf(args, rank, world, local_rank, dist):
         t_attn = ms_a / reps / args.layers * 1e-3
         attn_launch_bytes = attn_step_bytes / args.layers
         achieved_a = attn_launch_bytes / t_attn / 1e9
-        roofline = {"bound": "hbm", "kernel": "attn_fused_kernel", "achieved": achieved_a, "peak": hbm_peak,
+        kname = "attn_fused_kernel" if cluster_attention(T) else "attention pipeline (score, select, out)"
+        roofline = {"bound": "hbm", "kernel": kname, "achieved": achieved_a, "peak": hbm_peak,
                     "unit": "GB/s", "frac": achieved_a / hbm_peak,
                     "traffic": ATTN_TRAFFIC_32K if (T == 32768 and HQ == 32 and HKV == 8) else None,
                     "peak_source": peak_src, "launch_us": t_attn * 1e6, "bytes_per_launch": attn_launch_bytes}
@@ -613,7 +625,7 @@ def run_sf(args, rank, world, local_rank, dist):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded on-device draws; random-init weights)",
-        "config": {"workload": WORKLOAD, "model_shape": "Llama-3.1-8B (32 layers)", "context": T,
+        "config": {"workload": workload(T), "model_shape": "Llama-3.1-8B (32 layers)", "context": T,
                    "layers": args.layers, "batch": 1, "weights": "2-bit resident + 2-bit refinement, group 128",
                    "kv": "2-bit + 2-bit, per token-head", "topk_channels": "3%", "cache": "10% LRU per matrix",
                    "topk_tokens": "1% per query head", "l2": "working set > L2, no flush",

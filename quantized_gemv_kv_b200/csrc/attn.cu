@@ -7,7 +7,8 @@
 //   A  score   per (KV head, token): resident scores of the Hq/Hkv query
 //              heads of the group from the 2-bit keys, fp32, into scratch, on
 //              the integer tensor cores; also a per-head histogram of the
-//              scores (top 10 bits of the order-preserving key) and max |s|.
+//              scores (top 11 bits of the order-preserving key), max |s| and
+//              max s.
 //   S  select  per query head: the k largest scores, exactly.  The fast fp32
 //              scores carry a proven error bound eps; every token within
 //              2*eps of the k-th largest fast score is a candidate, and the
@@ -18,7 +19,9 @@
 //              a compaction over token chunks (from the histogram's bin of
 //              the k-th score) and a finish per KV group (one cluster, one CTA
 //              per query head), which also forms the group's union (ascending
-//              list and token bitmask) and the refined scores of its tokens.
+//              list and token bitmask).
+//   R  refine  per union token: its scores from the full 4-bit key codes,
+//              in place in the score buffer, and the largest per head.
 //   B  output  split over tokens: softmax over all tokens with the refined
 //              (full-code) K and V for tokens in the union and the resident
 //              ones elsewhere -- refined tokens are computed directly, never
@@ -65,22 +68,64 @@ __device__ void load_q(const uint16_t* __restrict__ q, int g, float (*qs)[D], fl
 // the q planes are laid out in the same permuted order.  A warp scores 16
 // tokens per MMA row tile for all heads of the group at once (n = heads).
 
+// A CTA owns a contiguous token range of one group; each warp streams its run
+// of 16-token tiles through its own ring of kScRing cp.async stages (seven
+// tiles in flight while one is scored), and the range's key scales and zeros
+// are staged in shared memory at the start.
+
+constexpr int kScThreads = 256;
+constexpr int kScW = kScThreads / 32;
+constexpr int kScRing = 8;        // cp.async stages per warp, one 16-token tile each
+constexpr int kScMaxTok = 4096;   // tokens per CTA at most
+
+__host__ __device__ constexpr size_t score_smem(int grp) {
+  return static_cast<size_t>(kScW) * kScRing * 16 * kWordsPerRow * 4 + static_cast<size_t>(kScMaxTok) * 4 +
+         static_cast<size_t>(grp) * kHistBins * 4;
+}
+
 template <int GRP>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kScThreads, 2)
 attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
-                      const uint16_t* __restrict__ k_scale, const uint16_t* __restrict__ k_zero, int T,
+                      const uint16_t* __restrict__ k_scale, const uint16_t* __restrict__ k_zero, int T, int tpc,
                       float* __restrict__ score, float* __restrict__ smax, int32_t* __restrict__ hist,
-                      uint32_t* __restrict__ amaxu) {
+                      uint32_t* __restrict__ amaxu, uint32_t* __restrict__ mkey) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t* ring = reinterpret_cast<uint32_t*>(smem);               // [kScW][kScRing][16][8]
+  uint32_t* ksz = ring + kScW * kScRing * 16 * kWordsPerRow;         // [tpc] key scale | zero << 16
+  int* hs = reinterpret_cast<int*>(ksz + kScMaxTok);                 // [GRP][kHistBins]
   __shared__ int qx[GRP][D];
   __shared__ float qsc[GRP], qsm[GRP];
-  // per-head histogram of this CTA's scores over the top 10 bits of the
-  // order-preserving key (pass S starts from the cluster of all CTAs' counts)
-  __shared__ int hs[GRP][kHistBins];
-  for (int i = threadIdx.x; i < GRP * kHistBins; i += blockDim.x) (&hs[0][0])[i] = 0;
   const int g = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // fixed-point query heads (warp h builds head h, 4 dims per lane)
-  for (int h = warp; h < GRP; h += 4) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g8 = lane >> 2, tig = lane & 3;
+  const int t0 = blockIdx.x * tpc;
+  const int n = max(0, min(tpc, T - t0));
+  const int ntile = (n + 15) >> 4;
+  const int tpw = (ntile + kScW - 1) / kScW;
+  const int tile0 = min(ntile, warp * tpw), tile1 = min(ntile, tile0 + tpw);
+  const size_t row0 = static_cast<size_t>(g) * T + t0;
+  auto issue = [&](int ti) {
+    const int st = (ti - tile0) % kScRing;
+    const int row = 16 * ti + (lane >> 1);
+    if (row < n)
+      cp_async16_attn(ring + ((warp * kScRing + st) * 16 + (lane >> 1)) * kWordsPerRow + (lane & 1) * 4,
+                      k_res + (row0 + row) * kWordsPerRow + (lane & 1) * 4);
+  };
+  for (int i = 0; i < kScRing - 1; ++i) {
+    if (tile0 + i < tile1) issue(tile0 + i);
+    cp_async_commit_attn();
+  }
+  // per-head histogram of this CTA's scores over the top 11 bits of the
+  // order-preserving key (pass S starts from the sum over all CTAs)
+  for (int i = tid; i < GRP * kHistBins; i += kScThreads) hs[i] = 0;
+  float smx = 0.0f;
+  for (int i = tid; i < n; i += kScThreads) {
+    const uint32_t kz = static_cast<uint32_t>(k_scale[row0 + i]) | (static_cast<uint32_t>(k_zero[row0 + i]) << 16);
+    ksz[i] = kz;
+    smx = fmaxf(smx, sfd::half_bits_to_float(static_cast<uint16_t>(kz & 0xFFFFu)));
+  }
+  // fixed-point query heads (warp h builds head h, 4 dims per lane) and the
+  // sums of q (any order: the error bound covers it)
+  for (int h = warp; h < GRP; h += kScW) {
     float v[4];
     float am = 0.0f;
 #pragma unroll
@@ -89,19 +134,17 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
       am = fmaxf(am, fabsf(v[i]));
     }
     am = warp_max(am);
+    const float qs_l = warp_sum((v[0] + v[1]) + (v[2] + v[3]));
     int e = 0;
     if (am > 0.0f) frexpf(am, &e);
 #pragma unroll
     for (int i = 0; i < 4; ++i) qx[h][4 * lane + i] = __float2int_rn(ldexpf(v[i], 23 - e));
-    if (lane == 0) qsc[h] = ldexpf(1.0f, e - 23);
-  }
-  if (tid < GRP) {
-    float sum = 0.0f;
-    for (int d = 0; d < D; ++d) sum += sfd::bf16_bits_to_float(q[(static_cast<size_t>(g) * GRP + tid) * D + d]);
-    qsm[tid] = sum;
+    if (lane == 0) {
+      qsc[h] = ldexpf(1.0f, e - 23);
+      qsm[h] = qs_l;
+    }
   }
   __syncthreads();
-  const int g8 = lane >> 2, tig = lane & 3;
   // B fragments: column n = g8 is query head g8 (zero beyond the group)
   uint32_t bq[4][3][2];
 #pragma unroll
@@ -118,101 +161,113 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
         }
         bq[ks][p][half] = v;
       }
-  const int ntiles = (T + 15) / 16;
-  float smx = 0.0f;
-  float am0 = 0.0f, am1 = 0.0f;  // max |score| of this lane's heads 2 tig, 2 tig + 1
-  // one tile = rows ta, tb of this thread: 2 x 32 bytes of codes plus the
-  // rows' scale and zero; the next tile is fetched while this one is scored
-  struct TileRegs {
+  // this lane's heads (2 tig, 2 tig + 1; with four heads 2 (tig & 1) and the
+  // next, lanes tig >= 2 scoring the second token of the pair): max |score|
+  // and the largest score key
+  const int h0 = GRP == 4 ? 2 * (tig & 1) : 2 * tig, h1 = h0 + 1;
+  const float qsc0 = h0 < GRP ? qsc[h0] : 0.0f, qsm0 = h0 < GRP ? qsm[h0] : 0.0f;
+  const float qsc1 = h1 < GRP ? qsc[h1] : 0.0f, qsm1 = h1 < GRP ? qsm[h1] : 0.0f;
+  float am0 = 0.0f, am1 = 0.0f;
+  uint32_t km0 = 0u, km1 = 0u;
+  for (int ti = tile0; ti < tile1; ++ti) {
+    if (ti + kScRing - 1 < tile1) issue(ti + kScRing - 1);
+    cp_async_commit_attn();
+    cp_async_wait_attn<kScRing - 1>();
+    __syncwarp();
+    const uint32_t* kr = ring + (warp * kScRing + (ti - tile0) % kScRing) * 16 * kWordsPerRow;
     uint32_t wa[8], wb[8];
-    uint16_t sa, za, sb, zb;
-  };
-  auto load_tile = [&](int tile, TileRegs& r) {
-    const int ta = tile * 16 + g8, tb = ta + 8;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) { r.wa[i] = 0u; r.wb[i] = 0u; }
-    r.sa = r.za = r.sb = r.zb = 0;
-    if (ta < T) {
-      const size_t row = static_cast<size_t>(g) * T + ta;
-      const uint4* p4 = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
-      const uint4 x0 = p4[0], x1 = p4[1];
-      r.wa[0] = x0.x; r.wa[1] = x0.y; r.wa[2] = x0.z; r.wa[3] = x0.w;
-      r.wa[4] = x1.x; r.wa[5] = x1.y; r.wa[6] = x1.z; r.wa[7] = x1.w;
-      r.sa = k_scale[row];
-      r.za = k_zero[row];
+    {
+      const uint4* pa = reinterpret_cast<const uint4*>(kr + g8 * kWordsPerRow);
+      const uint4* pb = reinterpret_cast<const uint4*>(kr + (g8 + 8) * kWordsPerRow);
+      const uint4 xa0 = pa[0], xa1 = pa[1], xb0 = pb[0], xb1 = pb[1];
+      wa[0] = xa0.x; wa[1] = xa0.y; wa[2] = xa0.z; wa[3] = xa0.w;
+      wa[4] = xa1.x; wa[5] = xa1.y; wa[6] = xa1.z; wa[7] = xa1.w;
+      wb[0] = xb0.x; wb[1] = xb0.y; wb[2] = xb0.z; wb[3] = xb0.w;
+      wb[4] = xb1.x; wb[5] = xb1.y; wb[6] = xb1.z; wb[7] = xb1.w;
     }
-    if (tb < T) {
-      const size_t row = static_cast<size_t>(g) * T + tb;
-      const uint4* p4 = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
-      const uint4 x0 = p4[0], x1 = p4[1];
-      r.wb[0] = x0.x; r.wb[1] = x0.y; r.wb[2] = x0.z; r.wb[3] = x0.w;
-      r.wb[4] = x1.x; r.wb[5] = x1.y; r.wb[6] = x1.z; r.wb[7] = x1.w;
-      r.sb = k_scale[row];
-      r.zb = k_zero[row];
-    }
-  };
-  const int tstride = gridDim.x * 4;
-  int tile = blockIdx.x * 4 + warp;
-  TileRegs cur;
-  if (tile < ntiles) load_tile(tile, cur);
-  for (; tile < ntiles; tile += tstride) {
-    TileRegs nxt;
-    if (tile + tstride < ntiles) load_tile(tile + tstride, nxt);
-    const int ta = tile * 16 + g8, tb = ta + 8;
+    __syncwarp();  // the stage is refilled by a later issue
     int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0}, d2[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
-      const uint32_t a0 = (cur.wa[2 * ks] >> (2 * tig)) & 0x03030303u;
-      const uint32_t a1 = (cur.wb[2 * ks] >> (2 * tig)) & 0x03030303u;
-      const uint32_t a2 = (cur.wa[2 * ks + 1] >> (2 * tig)) & 0x03030303u;
-      const uint32_t a3 = (cur.wb[2 * ks + 1] >> (2 * tig)) & 0x03030303u;
+      const uint32_t a0 = (wa[2 * ks] >> (2 * tig)) & 0x03030303u;
+      const uint32_t a1 = (wb[2 * ks] >> (2 * tig)) & 0x03030303u;
+      const uint32_t a2 = (wa[2 * ks + 1] >> (2 * tig)) & 0x03030303u;
+      const uint32_t a3 = (wb[2 * ks + 1] >> (2 * tig)) & 0x03030303u;
       mma_u8u8(d0, a0, a1, a2, a3, bq[ks][0][0], bq[ks][0][1]);
       mma_u8u8(d1, a0, a1, a2, a3, bq[ks][1][0], bq[ks][1][1]);
       mma_u8s8(d2, a0, a1, a2, a3, bq[ks][2][0], bq[ks][2][1]);
     }
     // d[i]: i = 0,1 -> token ta, heads 2 tig, 2 tig + 1; i = 2,3 -> token tb
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int h = 2 * tig + (i & 1);
-      const int t = (i < 2) ? ta : tb;
-      if (h < GRP && t < T) {
-        const float sv = sfd::half_bits_to_float(i < 2 ? cur.sa : cur.sb);
-        const float zv = sfd::half_bits_to_float(i < 2 ? cur.za : cur.zb);
-        smx = fmaxf(smx, sv);
-        const float P = (static_cast<float>(d2[i]) * 65536.0f + static_cast<float>(d1[i]) * 256.0f +
-                         static_cast<float>(d0[i])) * qsc[h];
-        const float E = fmaf(4.0f, P, (1.5f - zv) * qsm[h]);
-        const float val = (sv * E) * kInvSqrtD;
-        score[(static_cast<size_t>(g) * GRP + h) * T + t] = val;
-        atomicAdd(&hs[h][okey32(val) >> 22], 1);
-        if (i & 1) am1 = fmaxf(am1, fabsf(val));
-        else am0 = fmaxf(am0, fabsf(val));
+    const int ta = 16 * ti + g8, tb = ta + 8;
+    if constexpr (GRP == 4) {
+      // columns 4..7 are padding: lanes tig >= 2 take token tb of lane ^ 2,
+      // so every lane scores two values
+      const bool up = tig >= 2;
+      const int x0 = __shfl_xor_sync(0xffffffffu, d0[2], 2), x1 = __shfl_xor_sync(0xffffffffu, d0[3], 2);
+      const int y0 = __shfl_xor_sync(0xffffffffu, d1[2], 2), y1 = __shfl_xor_sync(0xffffffffu, d1[3], 2);
+      const int z0 = __shfl_xor_sync(0xffffffffu, d2[2], 2), z1 = __shfl_xor_sync(0xffffffffu, d2[3], 2);
+      if (up) {
+        d0[0] = x0; d0[1] = x1;
+        d1[0] = y0; d1[1] = y1;
+        d2[0] = z0; d2[1] = z1;
       }
     }
-    cur = nxt;
+    constexpr int kVals = GRP == 4 ? 2 : 4;
+#pragma unroll
+    for (int i = 0; i < kVals; ++i) {
+      const int h = (i & 1) ? h1 : h0;
+      const int tl = GRP == 4 ? (tig >= 2 ? tb : ta) : ((i < 2) ? ta : tb);
+      if (h < GRP && tl < n) {
+        const uint32_t kz = ksz[tl];
+        const float sv = sfd::half_bits_to_float(static_cast<uint16_t>(kz & 0xFFFFu));
+        const float zv = sfd::half_bits_to_float(static_cast<uint16_t>(kz >> 16));
+        const float P = (static_cast<float>(d2[i]) * 65536.0f + static_cast<float>(d1[i]) * 256.0f +
+                         static_cast<float>(d0[i])) * ((i & 1) ? qsc1 : qsc0);
+        const float E = fmaf(4.0f, P, (1.5f - zv) * ((i & 1) ? qsm1 : qsm0));
+        const float val = (sv * E) * kInvSqrtD;
+        score[(static_cast<size_t>(g) * GRP + h) * T + t0 + tl] = val;
+        atomicAdd(&hs[h * kHistBins + (okey32(val) >> kHistShift)], 1);
+        if (i & 1) {
+          am1 = fmaxf(am1, fabsf(val));
+          km1 = max(km1, okey32(val));
+        } else {
+          am0 = fmaxf(am0, fabsf(val));
+          km0 = max(km0, okey32(val));
+        }
+      }
+    }
   }
+  cp_async_wait_attn<0>();
   smx = warp_max(smx);
   if (lane == 0) atomicMax(reinterpret_cast<unsigned int*>(smax + g), __float_as_uint(smx));
-  // max |score| per head: lanes with the same tig hold the same two heads
+  // lanes with the same tig hold the same two heads
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     am0 = fmaxf(am0, __shfl_xor_sync(0xffffffffu, am0, o));
     am1 = fmaxf(am1, __shfl_xor_sync(0xffffffffu, am1, o));
+    km0 = max(km0, __shfl_xor_sync(0xffffffffu, km0, o));
+    km1 = max(km1, __shfl_xor_sync(0xffffffffu, km1, o));
   }
   if (g8 == 0) {
-    if (2 * tig < GRP) atomicMax(amaxu + g * GRP + 2 * tig, __float_as_uint(am0));
-    if (2 * tig + 1 < GRP) atomicMax(amaxu + g * GRP + 2 * tig + 1, __float_as_uint(am1));
+    if (h0 < GRP) {
+      atomicMax(amaxu + g * GRP + h0, __float_as_uint(am0));
+      atomicMax(mkey + g * GRP + h0, km0);
+    }
+    if (h1 < GRP) {
+      atomicMax(amaxu + g * GRP + h1, __float_as_uint(am1));
+      atomicMax(mkey + g * GRP + h1, km1);
+    }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < GRP * kHistBins; i += blockDim.x) {
-    const int c = (&hs[0][0])[i];
+  for (int i = tid; i < GRP * kHistBins; i += kScThreads) {
+    const int c = hs[i];
     if (c) atomicAdd(hist + static_cast<size_t>(g) * GRP * kHistBins + i, c);
   }
 }
 
 // ---- pass S, selection from the score histogram -----------------------------
 //
-// Pass A left, per query head, a histogram of its fast scores over the top 10
+// Pass A left, per query head, a histogram of its fast scores over the top 11
 // bits of the order-preserving key, and max |score|.  The bin b1 holding the
 // k-th largest score follows from the histogram alone.  Every token whose
 // exact key can reach the top k has a fast score >= tau - 2 eps >= (lower
@@ -224,8 +279,7 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
 //     scores of bin b1, keep the candidates >= tau - 2 eps, re-key them
 //     exactly in fp64 and rank them (key desc, token asc); then the group's
 //     CTAs build the union of their selections (bitmask and ascending list)
-//     through distributed shared memory and each computes its head's refined
-//     scores for the union tokens.
+//     through distributed shared memory.
 
 // Per-head threshold of the compaction and the histogram bin: all threads call.
 __device__ void select_band(const int32_t* __restrict__ hist_h, int k, double eps_s, int* hsh, int* scan_scratch,
@@ -235,7 +289,7 @@ __device__ void select_band(const int32_t* __restrict__ hist_h, int k, double ep
   find_bin_from_top_block(hsh, kHistBins, k, binfo, scan_scratch);
   *b1 = static_cast<uint32_t>(binfo[0]);
   *kk = binfo[1];
-  const float lower = from_okey32(*b1 << 22);
+  const float lower = from_okey32(*b1 << kHistShift);
   *f_low = __double2float_rd(static_cast<double>(lower) - 2.0 * eps_s);
 }
 
@@ -315,7 +369,7 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
                           const uint32_t* __restrict__ amaxu, int32_t* __restrict__ cand, int nchunks,
                           int32_t* __restrict__ list, double* __restrict__ kap, int32_t* __restrict__ sel_head,
                           uint32_t* __restrict__ umask, int words_t, int32_t* __restrict__ sel_out,
-                          int32_t* __restrict__ sel_n, int32_t* __restrict__ status) {
+                          int32_t* __restrict__ sel_n, int32_t* __restrict__ status, uint32_t* __restrict__ mkey) {
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
   const int rank = static_cast<int>(cl.block_rank());
@@ -330,6 +384,7 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   __shared__ double l1_sh;
   __shared__ int qe_sh, span_sh;
   __shared__ int cnt_sh;  // read remotely
+  __shared__ int cntA_sh, cntB_sh;  // outright selections and band candidates listed
   __shared__ uint32_t qpl[3][8][4];  // byte planes of the fixed-point q, in code-extraction order
   __shared__ long long qxsum_sh;
   extern __shared__ int fin_dyn[];
@@ -342,6 +397,7 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   double* kp = kap + static_cast<size_t>(h) * T;
   const int cap = GRP * k;
 
+  if (tid == 0) cntA_sh = cntB_sh = 0;
   select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status, &span_sh);
   // q as 24-bit fixed point X = q 2^(23 - qe): exact for every nonzero q
   // within 15 binades of the largest (bf16 has 8 significant bits)
@@ -404,24 +460,33 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   auto tok_of = [&](int e) { return cached ? ltok[e] : L[e]; };
   auto score_of = [&](int e) { return cached ? lsc[e] : sc[L[e]]; };
 
-  // 2. tau: two radix passes (11 + 11 bits) over the listed scores of bin b1
-  uint32_t pre = b1 << 22;
+  // 2. tau: two radix passes (11 + 10 bits) over the listed scores of bin b1
+  uint32_t pre = b1 << kHistShift;
+  static_assert(kHistShift == 21, "the two passes cover the 21 key bits below the histogram's");
   for (int pass = 0; pass < 2; ++pass) {
-    const int shift = pass == 0 ? 11 : 0;
-    for (int i = tid; i < 2048; i += kFinThreads) hr[i] = 0;
+    const int shift = pass == 0 ? 10 : 0;
+    const int nb = pass == 0 ? 2048 : 1024;
+    for (int i = tid; i < nb; i += kFinThreads) hr[i] = 0;
     __syncthreads();
-    const uint32_t pmask = pass == 0 ? 0xFFC00000u : 0xFFFFF800u;
+    const uint32_t pmask = pass == 0 ? 0xFFE00000u : 0xFFFFFC00u;
     for (int e = tid; e < m; e += kFinThreads) {
       const uint32_t key = okey32(score_of(e));
-      if ((key & pmask) == pre) atomicAdd(&hr[(key >> shift) & 2047u], 1);
+      if ((key & pmask) == pre) atomicAdd(&hr[(key >> shift) & static_cast<uint32_t>(nb - 1)], 1);
     }
     __syncthreads();
-    find_bin_from_top_block(hr, 2048, kk, binfo, scan_scratch);
+    find_bin_from_top_block(hr, nb, kk, binfo, scan_scratch);
     pre |= static_cast<uint32_t>(binfo[0]) << shift;
     kk = binfo[1];
   }
   const float tau = from_okey32(pre);
   const float fthr = __double2float_ru(static_cast<double>(tau) - 2.0 * eps_s);
+  if (tid == 0) {
+    // every token left out of the union has a fast score <= tau + 2 eps: pass
+    // B's maximum needs no more (the union's resident scores, replaced by
+    // refined ones, may lie far above every score pass B uses)
+    const uint32_t b = okey32(__double2float_ru(static_cast<double>(tau) + 2.0 * eps_s));
+    mkey[h] = min(mkey[h], b);
+  }
 
   // 3. a token whose fast score exceeds tau + 2 eps outranks, by exact key,
   //    every token with fast score <= tau, so fewer than k tokens can rank
@@ -430,25 +495,35 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   int32_t* sel = sel_head + static_cast<size_t>(h) * k;
   uint32_t* um = umask + static_cast<size_t>(g) * words_t;
   const double hi_band = static_cast<double>(tau) + 2.0 * eps_s;
-  int nA = 0, ncand = 0;
-  for (int base = 0; base < m; base += kFinThreads) {
-    const int e = base + tid;
-    const float sv_e = e < m ? score_of(e) : 0.0f;
-    const bool inA = e < m && static_cast<double>(sv_e) > hi_band;
-    const bool inB = e < m && !inA && sv_e >= fthr;
-    const int t = e < m ? tok_of(e) : 0;
-    int totA, totB;
-    const int posA = sfd::block_exclusive_scan(inA ? 1 : 0, scan_scratch, &totA);
-    const int posB = sfd::block_exclusive_scan(inB ? 1 : 0, scan_scratch, &totB);
-    if (inA && nA + posA < k) {  // fewer than k by the bound; guarded against corrupt scores
-      sel[nA + posA] = t;
-      atomicOr(um + (t >> 5), 1u << (t & 31));
+  // listed in any order (the ranking orders by key and token): a warp takes
+  // its slots with one shared atomic per list
+  {
+    const int lane = tid & 31;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = 0; base < m; base += kFinThreads) {
+      const int e = base + tid;
+      const float sv_e = e < m ? score_of(e) : 0.0f;
+      const bool inA = e < m && static_cast<double>(sv_e) > hi_band;
+      const bool inB = e < m && !inA && sv_e >= fthr;
+      const int t = e < m ? tok_of(e) : 0;
+      const unsigned bA = __ballot_sync(0xffffffffu, inA), bB = __ballot_sync(0xffffffffu, inB);
+      int oA = 0, oB = 0;
+      if (lane == 0) {
+        if (bA) oA = atomicAdd(&cntA_sh, __popc(bA));
+        if (bB) oB = atomicAdd(&cntB_sh, __popc(bB));
+      }
+      oA = __shfl_sync(0xffffffffu, oA, 0);
+      oB = __shfl_sync(0xffffffffu, oB, 0);
+      const int pA = oA + __popc(bA & lt);
+      if (inA && pA < k) {  // fewer than k by the bound; guarded against corrupt scores
+        sel[pA] = t;
+        atomicOr(um + (t >> 5), 1u << (t & 31));
+      }
+      if (inB) F[oB + __popc(bB & lt)] = t;
     }
-    if (inB) F[ncand + posB] = t;
-    nA += totA;
-    ncand += totB;
   }
   __syncthreads();
+  const int nA = cntA_sh, ncand = cntB_sh;
   const int kB = max(0, k - nA);  // winners still to pick from the band (>= 1 by the bound)
 
 
@@ -582,6 +657,77 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   cl.sync();  // 3: no shared-memory access across CTAs after this
 }
 
+// ---- refined scores of the union --------------------------------------------------
+//
+// Between the selection and pass B: every token of a group's union gets its
+// scores for the group's query heads recomputed from the full 4-bit key codes,
+// in place in the score buffer, and the largest refined score per head is
+// recorded as an order-preserving key.  Pass B then weights every token
+// against one fixed maximum per head (the larger of the refined maximum and a
+// bound on the resident scores outside the union), so it needs no maximum
+// pass and no rescaling.  A thread handles one union token for all the heads
+// of the group: one load of the list, one of the token's two code rows.
+
+constexpr int kRefThreads = 256;
+
+template <int GRP>
+__global__ void __launch_bounds__(kRefThreads, 2)
+attn_refine_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
+                   const uint32_t* __restrict__ k_ref, const uint16_t* __restrict__ k_scale,
+                   const uint16_t* __restrict__ k_zero, int T, int cap, const int32_t* __restrict__ sel_out,
+                   const int32_t* __restrict__ sel_n, float* __restrict__ score, uint32_t* __restrict__ rkey) {
+  __shared__ float qs[GRP][D];
+  __shared__ float qsum[GRP];
+  const int g = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  load_q<GRP>(q, g, qs, qsum);  // contains __syncthreads
+  const int sn = sel_n[g];
+  const int U = min(cap, sn >= 0 ? sn : -1 - sn);
+  const int32_t* list = sel_out + static_cast<size_t>(g) * cap;
+  const size_t rowg = static_cast<size_t>(g) * T;
+  uint32_t mk[GRP];
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) mk[h] = 0u;
+  for (int u0 = blockIdx.x * kRefThreads; u0 < U; u0 += gridDim.x * kRefThreads) {  // uniform over the block
+    const int u = u0 + static_cast<int>(threadIdx.x);
+    if (u < U) {
+      const int t = list[u];
+      const size_t row = rowg + t;
+      const uint4* pr = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
+      const uint4* pf = reinterpret_cast<const uint4*>(k_ref + row * kWordsPerRow);
+      const uint4 r0 = pr[0], r1 = pr[1], f0 = pf[0], f1 = pf[1];
+      const float sv = sfd::half_bits_to_float(k_scale[row]);
+      const float z = sfd::half_bits_to_float(k_zero[row]);
+      const uint32_t wr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+      const uint32_t wf[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+      float P[GRP];
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) P[h] = 0.0f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float c = static_cast<float>(((wr[w] >> (2 * j)) & 3u) * 4u + ((wf[w] >> (2 * j)) & 3u));
+#pragma unroll
+          for (int h = 0; h < GRP; ++h) P[h] = fmaf(qs[h][16 * w + j], c, P[h]);
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) {
+        const float val = (sv * fmaf(-z, qsum[h], P[h])) * kInvSqrtD;
+        mk[h] = max(mk[h], okey32(val));
+        score[(static_cast<size_t>(g) * GRP + h) * T + t] = val;
+      }
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mk[h] = max(mk[h], __shfl_xor_sync(0xffffffffu, mk[h], o));
+    if (lane == 0 && mk[h]) atomicMax(rkey + g * GRP + h, mk[h]);
+  }
+}
+
 // ---- pass B on the tensor cores ------------------------------------------------
 //
 // o_h = sum_t p_{h,t} v_t / sum_t p_{h,t} with v_t = s_t (4 c_t + 1.5 - z_t):
@@ -597,55 +743,55 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
 // on the CUDA cores; their scores were already refined in the score buffer.
 //
 // A CTA owns a token range of one KV group and walks it in sub-chunks of
-// kSub tokens: the sub-chunk's score maximum per head is found first, so every
-// weight is computed once, by one thread, relative to a fixed maximum and
-// stored in shared memory (no per-tile online rescaling); the warps then run
-// the MMAs over their tiles of 16 tokens, the codes staged by cp.async.
+// kSub tokens (4096 up to four query heads per group: one sub-chunk per CTA
+// up to 128K tokens at 8 KV heads).  Every weight is computed once, by one thread, against the
+// head's maximum over all tokens (resident and refined scores, recorded by the
+// earlier passes), and stored in shared memory: no maximum pass and no
+// rescaling.  The warps then run the MMAs over their tiles of 16 tokens, the
+// codes staged by cp.async.
 
-constexpr int kSub = 2048;         // tokens per sub-chunk
 constexpr int kOutThreads = 256;
 constexpr int kOW = kOutThreads / 32;
-constexpr int kRing = 4;           // cp.async stages per warp
-constexpr int kUCap = 512;         // refined rows per sub-chunk staged in shared memory
-constexpr int kPerThr = kSub / kOutThreads;  // tokens of a sub-chunk per thread in the weight pass
+constexpr int kRing = 6;           // cp.async stages per warp
+constexpr int kUCap = 384;         // refined rows per sub-chunk staged in shared memory
 
 template <int GRP>
 struct OutCfg {
   static constexpr int NC = 2 * GRP;           // weight columns: high parts of the heads, then remainders
   static constexpr int NT = NC <= 8 ? 1 : 2;   // MMA n-tiles of 8 columns
+  static constexpr int kSub = NT == 1 ? 4096 : 2048;  // tokens per sub-chunk
+  static constexpr int kPerThr = kSub / kOutThreads;  // tokens of a sub-chunk per thread in the weight pass
+  static_assert(kPerThr % 4 == 0, "the weight pass loads four tokens per thread at a time");
   static constexpr int kStr = kSub + 8;        // halves per weight row: conflict-free fragment loads
   static constexpr size_t alpha_bytes = static_cast<size_t>(NT) * 8 * kStr * 2;
   static constexpr size_t ring_bytes = static_cast<size_t>(kOW) * kRing * 16 * kWordsPerRow * 4;
-  static constexpr size_t ulist_bytes = static_cast<size_t>(kSub) * 4;
+  static constexpr size_t ulist_bytes = static_cast<size_t>(kSub) * 2;
   static constexpr size_t vref_bytes = static_cast<size_t>(kUCap) * kWordsPerRow * 4;
   static constexpr size_t smem = alpha_bytes + ring_bytes + ulist_bytes + vref_bytes;
-  static_assert(alpha_bytes >= static_cast<size_t>(GRP) * kMaxSplits * 4, "merge factors must fit the weight tile");
   static_assert(alpha_bytes >= static_cast<size_t>(kOW) * GRP * D * 4, "per-warp output tiles must fit the weight tile");
+  static_assert(kSub / 32 <= kOutThreads, "the union scan takes a bitmask word per thread");
 };
 
 template <int GRP>
 __global__ void __launch_bounds__(kOutThreads)
-attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
-                const uint32_t* __restrict__ k_ref, const uint16_t* __restrict__ k_scale,
-                const uint16_t* __restrict__ k_zero, const uint32_t* __restrict__ v_res,
+attn_out_kernel(const uint32_t* __restrict__ v_res,
                 const uint32_t* __restrict__ v_ref, const uint16_t* __restrict__ v_scale,
-                const uint16_t* __restrict__ v_zero, int T, int tps, int words_t, int splits, float* __restrict__ score,
+                const uint16_t* __restrict__ v_zero, int T, int tps, int words_t, int splits,
+                const float* __restrict__ score, const uint32_t* __restrict__ mkey, const uint32_t* __restrict__ rkey,
                 const uint32_t* __restrict__ umask, float* __restrict__ part, int32_t* __restrict__ done,
                 float* __restrict__ out) {
   using C = OutCfg<GRP>;
-  constexpr int NT = C::NT, kStr = C::kStr;
+  constexpr int NT = C::NT, kStr = C::kStr, kSub = C::kSub, kPerThr = C::kPerThr;
   extern __shared__ __align__(16) unsigned char smem[];
   __half* as = reinterpret_cast<__half*>(smem);                                      // [NT*8][kStr]
   uint32_t* ring = reinterpret_cast<uint32_t*>(smem + C::alpha_bytes);               // [kOW][kRing][16][8]
-  int* ulist = reinterpret_cast<int*>(smem + C::alpha_bytes + C::ring_bytes);  // [kSub]
+  uint16_t* ulist = reinterpret_cast<uint16_t*>(smem + C::alpha_bytes + C::ring_bytes);  // [kSub]
   uint32_t* vrs = reinterpret_cast<uint32_t*>(smem + C::alpha_bytes + C::ring_bytes +
                                               C::ulist_bytes);  // [kUCap][8] refinement rows of listed tokens
   __shared__ float red[kOW][GRP];
   __shared__ float red2[kOW][3 * GRP];
-  __shared__ float Msh[GRP], Fsh[GRP];
+  __shared__ float Msh[GRP];
   __shared__ int ucount;
-  __shared__ float qs[GRP][D];
-  __shared__ float qsum[GRP];
   __shared__ int uscan[33];
 
   const int g = blockIdx.y, split = blockIdx.x;
@@ -654,8 +800,16 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
   const size_t rowg = static_cast<size_t>(g) * T;
 
   for (int e = tid; e < (NT * 8 - C::NC) * kStr; e += kOutThreads) as[C::NC * kStr + e] = __float2half_rn(0.0f);
-  if (tid < GRP) Msh[tid] = -INFINITY;
-  load_q<GRP>(q, g, qs, qsum);  // contains __syncthreads
+  // one maximum per head for every token: the larger of the bound on the
+  // resident scores outside the union and the refined maximum (a key of 0:
+  // no such token)
+  if (tid < GRP) {
+    const uint32_t mk = mkey[g * GRP + tid], rk = rkey[g * GRP + tid];
+    float m = mk ? from_okey32(mk) : -INFINITY;
+    if (rk) m = fmaxf(m, from_okey32(rk));
+    Msh[tid] = m;
+  }
+  __syncthreads();
 
   float lsum[GRP], csum[GRP], asum[GRP], uo[GRP][4];
   float acc[NT][8][4];
@@ -700,9 +854,8 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
     }
 
     // 0. the sub-chunk's refined tokens (ascending) from the group's bitmask;
-    //    their refinement rows are staged for step 4, and their scores are
-    //    recomputed from the full 4-bit key codes into the score buffer (this
-    //    CTA owns the token range)
+    //    their value refinement rows are staged for step 3 (their scores were
+    //    refined in the score buffer before this pass)
     {
       const int nw = (n + 31) >> 5;  // c0 is a multiple of 32
       uint32_t wbits = 0;
@@ -716,7 +869,7 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
       while (wbits) {
         const int b = __ffs(wbits) - 1;
         wbits &= wbits - 1u;
-        ulist[pos++] = 32 * tid + b;
+        ulist[pos++] = static_cast<uint16_t>(32 * tid + b);
       }
       if (tid == 0) ucount = tot;
       __syncthreads();
@@ -728,127 +881,38 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
       cp_async16_attn(vrs + u * kWordsPerRow + 4, src + 4);
     }
     cp_async_commit_attn();
-    // warp per token, lane = dims 4 lane .. 4 lane + 3; four tokens' loads in
-    // flight at a time
-    for (int u0 = warp; u0 < nu; u0 += 4 * kOW) {
-      uint32_t wr[4], wf[4], sz[4];
+    float M[GRP];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int u = u0 + j * kOW;
-        wr[j] = wf[j] = sz[j] = 0;
-        if (u < nu) {
-          const size_t row = rowg + c0 + ulist[u];
-          wr[j] = k_res[row * kWordsPerRow + (lane >> 2)];
-          wf[j] = k_ref[row * kWordsPerRow + (lane >> 2)];
-          sz[j] = static_cast<uint32_t>(k_scale[row]) | (static_cast<uint32_t>(k_zero[row]) << 16);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int u = u0 + j * kOW;
-        if (u >= nu) break;  // uniform over the warp
-        const uint32_t r = wr[j] >> ((lane & 3) * 8), f = wf[j] >> ((lane & 3) * 8);
-        float P[GRP];
-#pragma unroll
-        for (int h = 0; h < GRP; ++h) P[h] = 0.0f;
-#pragma unroll
-        for (int dd = 0; dd < 4; ++dd) {
-          const float c = static_cast<float>(((r >> (2 * dd)) & 3u) * 4u + ((f >> (2 * dd)) & 3u));
-#pragma unroll
-          for (int h = 0; h < GRP; ++h) P[h] = fmaf(qs[h][4 * lane + dd], c, P[h]);
-        }
-        const float sv = sfd::half_bits_to_float(sz[j] & 0xFFFFu);
-        const float z = sfd::half_bits_to_float(sz[j] >> 16);
-        const int t = c0 + ulist[u];
-#pragma unroll
-        for (int h = 0; h < GRP; ++h) {
-          const float Ph = warp_sum(P[h]);
-          if (lane == 0) score[(static_cast<size_t>(g) * GRP + h) * T + t] = (sv * fmaf(-z, qsum[h], Ph)) * kInvSqrtD;
-        }
-      }
-    }
-    __syncthreads();
+    for (int h = 0; h < GRP; ++h) M[h] = Msh[h];
 
-    // 1. the sub-chunk's maximum score per head; this thread's tokens'
-    //    scale, zero and union bit are fetched meanwhile
-    uint32_t svz[kPerThr];
-    {
-      float mx[GRP];
+    // 1. weights into shared memory (zero past the end of the last tile) and
+    //    sums; the scores, scales and zeros of four of this thread's tokens
+    //    are loaded before any is used
+#pragma unroll 1
+    for (int j0 = 0; j0 < kPerThr; j0 += 4) {
+      if (j0 * kOutThreads >= 16 * ntile) break;  // uniform over the block
+      float sc4[4][GRP];
+      uint16_t vs4[4], vz4[4];
 #pragma unroll
-      for (int h = 0; h < GRP; ++h) mx[h] = -INFINITY;
+      for (int jj = 0; jj < 4; ++jj) {
+        const int i = tid + (j0 + jj) * kOutThreads;
+        const bool valid = i < n;
+        vs4[jj] = valid ? v_scale[rowg + c0 + i] : 0;
+        vz4[jj] = valid ? v_zero[rowg + c0 + i] : 0;
 #pragma unroll
-      for (int j = 0; j < kPerThr; ++j) {
-        const int i = tid + j * kOutThreads;
-        svz[j] = 0;
-        if (i < n) {
-          const size_t row = rowg + c0 + i;
-          svz[j] = static_cast<uint32_t>(v_scale[row]) | (static_cast<uint32_t>(v_zero[row]) << 16);
-#pragma unroll
-          for (int h = 0; h < GRP; ++h)
-            mx[h] = fmaxf(mx[h], score[(static_cast<size_t>(g) * GRP + h) * T + c0 + i]);
-        }
+        for (int h = 0; h < GRP; ++h) sc4[jj][h] = valid ? score[(static_cast<size_t>(g) * GRP + h) * T + c0 + i] : 0.0f;
       }
 #pragma unroll
-      for (int h = 0; h < GRP; ++h) {
-        const float m = warp_max(mx[h]);
-        if (lane == 0) red[warp][h] = m;
-      }
-      __syncthreads();
-      if (tid < GRP) {
-        float m = -INFINITY;
-        for (int w = 0; w < kOW; ++w) m = fmaxf(m, red[w][tid]);
-        const float mo = Msh[tid], mn = fmaxf(mo, m);
-        Fsh[tid] = mo == -INFINITY ? 0.0f : __expf(mo - mn);
-        Msh[tid] = mn;
-      }
-      __syncthreads();
-    }
-    float M[GRP], F[GRP];
-    bool rescale = false;
-#pragma unroll
-    for (int h = 0; h < GRP; ++h) {
-      M[h] = Msh[h];
-      F[h] = Fsh[h];
-      rescale |= F[h] != 1.0f;
-    }
-    if (rescale && c0 != t0s) {  // uniform over the block
-#pragma unroll
-      for (int h = 0; h < GRP; ++h) {
-        lsum[h] *= F[h];
-        csum[h] *= F[h];
-        asum[h] *= F[h];
-#pragma unroll
-        for (int dd = 0; dd < 4; ++dd) uo[h][dd] *= F[h];
-      }
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        float f0 = 1.0f, f1 = 1.0f;
-#pragma unroll
-        for (int h = 0; h < GRP; ++h) {
-          if (colh[nt][0] == h) f0 = F[h];
-          if (colh[nt][1] == h) f1 = F[h];
-        }
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          acc[nt][w][0] *= f0; acc[nt][w][1] *= f1;
-          acc[nt][w][2] *= f0; acc[nt][w][3] *= f1;
-        }
-      }
-    }
-
-    // 2. weights into shared memory (zero past the end of the last tile) and sums
-#pragma unroll
-    for (int j = 0; j < kPerThr; ++j) {
-      const int i = tid + j * kOutThreads;
-      if (j * kOutThreads >= 16 * ntile) break;  // uniform over the block
+      for (int jj = 0; jj < 4; ++jj) {
+      const int i = tid + (j0 + jj) * kOutThreads;
       const bool valid = i < n;
       if (i < 16 * ntile) {
         if (valid) {
-          const float sv = sfd::half_bits_to_float(svz[j] & 0xFFFFu);
-          const float zv = sfd::half_bits_to_float(svz[j] >> 16);
+          const float sv = sfd::half_bits_to_float(vs4[jj]);
+          const float zv = sfd::half_bits_to_float(vz4[jj]);
 #pragma unroll
           for (int h = 0; h < GRP; ++h) {
-            const float p = __expf(score[(static_cast<size_t>(g) * GRP + h) * T + c0 + i] - M[h]);
+            const float p = __expf(sc4[jj][h] - M[h]);
             const float al = p * sv;
             const __half ahi = __float2half_rn(al);
             const __half alo = __float2half_rn(al - __half2float(ahi));
@@ -863,10 +927,11 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
           for (int h = 0; h < 2 * GRP; ++h) as[h * kStr + i] = __float2half_rn(0.0f);
         }
       }
+      }
     }
     __syncthreads();
 
-    // 3. MMAs over this warp's tiles
+    // 2. MMAs over this warp's tiles
     for (int ti = tile0; ti < tile1; ++ti) {
       if (ti + kRing - 1 < tile1) issue(ti + kRing - 1);
       cp_async_commit_attn();
@@ -907,7 +972,7 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
     cp_async_wait_attn<0>();
     __syncthreads();  // the staged refinement rows come from every thread
 
-    // 4. refined tokens: alpha (c_f - 1.5), lane = dims 4 lane .. 4 lane + 3
+    // 3. refined tokens: alpha (c_f - 1.5), lane = dims 4 lane .. 4 lane + 3
     for (int u = warp; u < nu; u += kOW) {
       const int i = ulist[u];
       const uint32_t wrow = u < kUCap ? vrs[u * kWordsPerRow + (lane >> 2)]
@@ -990,58 +1055,45 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
   __syncthreads();
   if (!last) return;
   __threadfence();
-  float (*fct)[kMaxSplits] = reinterpret_cast<float (*)[kMaxSplits]>(smem);  // the weight tile is dead
-  __shared__ float Lh[GRP];
-  for (int e = tid; e < GRP * splits; e += kOutThreads) fct[e / splits][e % splits] = __ldcg(pg + e * (D + 2));
-  __syncthreads();
-  for (int h = warp; h < GRP; h += kOW) {
-    float Mx = -INFINITY;
-    for (int sp = lane; sp < splits; sp += 32) Mx = fmaxf(Mx, fct[h][sp]);
-    Mx = warp_max(Mx);
-    float Ls = 0.0f;
-    for (int sp = lane; sp < splits; sp += 32) {
-      const float ms = fct[h][sp];
-      const float f = ms == -INFINITY ? 0.0f : __expf(ms - Mx);
-      Ls = fmaf(f, __ldcg(pg + (h * splits + sp) * (D + 2) + 1), Ls);
-      fct[h][sp] = f;
-    }
-    Ls = warp_sum(Ls);
-    if (lane == 0) Lh[h] = Ls;
-  }
-  __syncthreads();
-  // two outputs per thread, eight splits' partials of each in flight at once
+  // every split weighted its tokens against the same maximum per head: the
+  // merge sums the splits' weight sums and outputs; two outputs per thread,
+  // eight splits' partials of each in flight at once
   for (int e0 = tid; e0 < GRP * D; e0 += 2 * kOutThreads) {
     const int e1 = e0 + kOutThreads;
     const bool has1 = e1 < GRP * D;
     const int h0 = e0 / D, h1 = has1 ? e1 / D : h0;
-    const float* p0 = pg + static_cast<size_t>(h0) * splits * (D + 2) + 2 + e0 % D;
-    const float* p1 = pg + static_cast<size_t>(h1) * splits * (D + 2) + 2 + (has1 ? e1 % D : e0 % D);
-    float A0 = 0.0f, A1 = 0.0f;
-    for (int sp = 0; sp < splits; sp += 16) {
-      float v0[16], v1[16];
+    const float* p0 = pg + static_cast<size_t>(h0) * splits * (D + 2);
+    const float* p1 = pg + static_cast<size_t>(h1) * splits * (D + 2);
+    const int d0 = e0 % D, d1 = has1 ? e1 % D : d0;
+    float A0 = 0.0f, A1 = 0.0f, L0 = 0.0f, L1 = 0.0f;
+    for (int sp = 0; sp < splits; sp += 8) {
+      float v0[8], v1[8], l0[8], l1[8];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int q = sp + u;
-        v0[u] = q < splits ? __ldcg(p0 + static_cast<size_t>(q) * (D + 2)) : 0.0f;
-        v1[u] = (has1 && q < splits) ? __ldcg(p1 + static_cast<size_t>(q) * (D + 2)) : 0.0f;
+      for (int u = 0; u < 8; ++u) {
+        const size_t o = static_cast<size_t>(sp + u) * (D + 2);
+        const bool ok = sp + u < splits;
+        v0[u] = ok ? __ldcg(p0 + o + 2 + d0) : 0.0f;
+        l0[u] = ok ? __ldcg(p0 + o + 1) : 0.0f;
+        v1[u] = (ok && has1) ? __ldcg(p1 + o + 2 + d1) : 0.0f;
+        l1[u] = (ok && has1) ? __ldcg(p1 + o + 1) : 0.0f;
       }
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int q = sp + u;
-        if (q < splits) {
-          A0 = fmaf(fct[h0][q], v0[u], A0);
-          A1 = fmaf(fct[h1][q], v1[u], A1);
-        }
+      for (int u = 0; u < 8; ++u) {
+        A0 += v0[u];
+        L0 += l0[u];
+        A1 += v1[u];
+        L1 += l1[u];
       }
     }
-    out[(static_cast<size_t>(g) * GRP + h0) * D + e0 % D] = A0 / Lh[h0];
-    if (has1) out[(static_cast<size_t>(g) * GRP + h1) * D + e1 % D] = A1 / Lh[h1];
+    out[(static_cast<size_t>(g) * GRP + h0) * D + d0] = A0 / L0;
+    if (has1) out[(static_cast<size_t>(g) * GRP + h1) * D + d1] = A1 / L1;
   }
 }
 
 __global__ void fill_all_kernel(int T, int grp, int k, int words_t, uint32_t* umask, int32_t* sel_out,
-                                int32_t* sel_n) {
+                                int32_t* sel_n, uint32_t* mkey) {
   const int g = blockIdx.y;
+  if (blockIdx.x == 0 && threadIdx.x < grp) mkey[g * grp + threadIdx.x] = 0u;  // no token outside the union
   for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x)
     sel_out[static_cast<size_t>(g) * grp * k + t] = t;
   for (int w = blockIdx.x * blockDim.x + threadIdx.x; w < words_t; w += gridDim.x * blockDim.x) {
@@ -1069,11 +1121,18 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
   const int sms = sf::sm_count();
 
   SF_CHECK_CUDA(cudaMemsetAsync(ws + L.smax, 0, L.total - L.smax, s));
-  const int ntiles = (T + 15) / 16;
-  dim3 ga(std::max(1, std::min((ntiles + 3) / 4, (4 * sms + Hkv - 1) / Hkv)), Hkv);
+  // pass A: about two CTAs per SM, each a contiguous range of <= kScMaxTok tokens
+  const int want_a = std::max((2 * sms + Hkv - 1) / Hkv, (T + kScMaxTok - 1) / kScMaxTok);
+  const int tpc = ((T + want_a - 1) / want_a + 15) / 16 * 16;
+  dim3 ga((T + tpc - 1) / tpc, Hkv);
   int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
   uint32_t* amaxu = reinterpret_cast<uint32_t*>(ws + L.amax);
-  attn_score_mma_kernel<GRP><<<ga, 128, 0, s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, score, smax, hist, amaxu);
+  uint32_t* mkey = reinterpret_cast<uint32_t*>(ws + L.mkey);
+  uint32_t* rkey = reinterpret_cast<uint32_t*>(ws + L.rkey);
+  SF_CHECK_CUDA(cudaFuncSetAttribute(attn_score_mma_kernel<GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(score_smem(GRP))));
+  attn_score_mma_kernel<GRP><<<ga, kScThreads, score_smem(GRP), s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, tpc,
+                                                                     score, smax, hist, amaxu, mkey);
   sf_status st = sf::check_launch("attn_score_mma_kernel");
   if (st != SF_OK) return st;
   if (k > 0 && k < T) {
@@ -1098,23 +1157,31 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
     SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, attn_select_finish_kernel<GRP>, q, kv->k_res, kv->k_ref, kv->k_scale,
                                      kv->k_zero, T, k, score, static_cast<const float*>(smax),
                                      static_cast<const int32_t*>(hist), static_cast<const uint32_t*>(amaxu), cand,
-                                     L.nchunks, cand2, kap, sel_head, umask, L.words_t, sel_out, sel_n, status));
+                                     L.nchunks, cand2, kap, sel_head, umask, L.words_t, sel_out, sel_n, status,
+                                     mkey));
     st = sf::check_launch("attn_select_finish_kernel");
     if (st != SF_OK) return st;
   } else if (k == 0) {  // the token bitmask was cleared with the workspace
     SF_CHECK_CUDA(cudaMemsetAsync(sel_n, 0, sizeof(int32_t) * Hkv, s));
   } else {
-    fill_all_kernel<<<dim3(32, Hkv), 256, 0, s>>>(T, grp, k, L.words_t, umask, sel_out, sel_n);
+    fill_all_kernel<<<dim3(32, Hkv), 256, 0, s>>>(T, grp, k, L.words_t, umask, sel_out, sel_n, mkey);
     st = sf::check_launch("fill_all_kernel");
+    if (st != SF_OK) return st;
+  }
+  if (k > 0) {
+    const int cap = grp * k;
+    const int nblk = std::max(1, std::min((cap + kRefThreads - 1) / kRefThreads, 2 * sms / Hkv));
+    attn_refine_kernel<GRP><<<dim3(nblk, Hkv), kRefThreads, 0, s>>>(q, kv->k_res, kv->k_ref, kv->k_scale, kv->k_zero,
+                                                                   T, cap, sel_out, sel_n, score, rkey);
+    st = sf::check_launch("attn_refine_kernel");
     if (st != SF_OK) return st;
   }
   dim3 gb(L.splits, Hkv);
   SF_CHECK_CUDA(cudaFuncSetAttribute(attn_out_kernel<GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(OutCfg<GRP>::smem)));
-  attn_out_kernel<GRP><<<gb, kOutThreads, OutCfg<GRP>::smem, s>>>(q, kv->k_res, kv->k_ref, kv->k_scale, kv->k_zero,
-                                                                 kv->v_res, kv->v_ref, kv->v_scale, kv->v_zero, T,
-                                                                 L.tps, L.words_t, L.splits, score, umask, part,
-                                                                 done, out);
+  attn_out_kernel<GRP><<<gb, kOutThreads, OutCfg<GRP>::smem, s>>>(kv->v_res, kv->v_ref, kv->v_scale, kv->v_zero, T,
+                                                                 L.tps, L.words_t, L.splits, score, mkey, rkey,
+                                                                 umask, part, done, out);
   return sf::check_launch("attn_out_kernel");
 }
 

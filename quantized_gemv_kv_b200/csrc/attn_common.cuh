@@ -30,12 +30,14 @@ constexpr int kMaxGrp = 8;
 constexpr int kMaxSplits = 256;
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128), rounded to fp32
 
-constexpr int kHistBins = 1024;    // per-head histogram of the fast scores' top 10 key bits
+constexpr int kHistBits = 11;      // per-head histogram of the fast scores' top 11 key bits
+constexpr int kHistBins = 1 << kHistBits;
+constexpr int kHistShift = 32 - kHistBits;
 constexpr int kChunk = 4096;       // tokens per CTA of the candidate compaction
 
 struct Layout {
   // from smax on, everything is cleared at the start of a call
-  size_t score, cand, cand2, kap, sel, part, fcnt, smax, status, count, amax, hist, umask, total;
+  size_t score, cand, cand2, kap, sel, part, fcnt, smax, status, count, amax, mkey, rkey, hist, umask, total;
   int splits, tps, words_t, nchunks;
 };
 
@@ -63,6 +65,8 @@ Layout make_layout(int Hq, int Hkv, int T, int k, int sms) {
   L.status = off; off = up256(off + sizeof(int32_t) * std::max(Hkv, 4));
   L.count = off; off = up256(off + sizeof(int32_t) * Hkv);
   L.amax = off; off = up256(off + sizeof(uint32_t) * Hq);
+  L.mkey = off; off = up256(off + sizeof(uint32_t) * Hq);  // max resident score key per head
+  L.rkey = off; off = up256(off + sizeof(uint32_t) * Hq);  // max refined score key per head
   L.hist = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(kHistBins));
   L.umask = off; off = up256(off + sizeof(uint32_t) * Hkv * static_cast<size_t>(L.words_t));
   L.total = off;
@@ -207,55 +211,53 @@ __device__ __forceinline__ double select_eps(double s_max, double l1, int qe, fl
   return 2.0 * (static_cast<double>(kInvSqrtD) * eps_k + 4.0 * u * static_cast<double>(amax));
 }
 
-// Exact top-k of F[0..ncand) by (key desc, token asc) with an 8-pass radix
-// select on the 64-bit order-preserving keys kp (all threads call; F is in
-// token order); the k winners go to sel in no particular order.
+// Exact top-k of F[0..ncand) by (key desc, token asc): an 8-pass radix select
+// on the 64-bit order-preserving keys kp, then 4 passes on the complemented
+// token among the entries tied with the k-th key (F in any order; all threads
+// call); the k winners go to sel in no particular order.
 __device__ void select_rank_radix(const int32_t* __restrict__ F, int ncand, const double* __restrict__ kp, int k,
                                   int* hist, int* scan_scratch, int* binfo, int32_t* __restrict__ sel) {
   const int tid = threadIdx.x, nthr = blockDim.x;
   unsigned long long pre64 = 0, pm64 = 0;
+  uint32_t pt = 0, mt = 0;
   int kr = k;
-  for (int pass = 0; pass < 8; ++pass) {
-    const int shift = 56 - 8 * pass;
+  for (int pass = 0; pass < 12; ++pass) {
     for (int i = tid; i < 256; i += nthr) hist[i] = 0;
     __syncthreads();
     for (int i = tid; i < ncand; i += nthr) {
       const unsigned long long key = okey64(kp[i]);
-      if ((key & pm64) == pre64) atomicAdd(&hist[(key >> shift) & 255], 1);
+      const uint32_t nt = ~static_cast<uint32_t>(F[i]);
+      if ((key & pm64) != pre64 || (nt & mt) != pt) continue;
+      const uint32_t digit = pass < 8 ? static_cast<uint32_t>((key >> (56 - 8 * pass)) & 255u)
+                                      : (nt >> (24 - 8 * (pass - 8))) & 255u;
+      atomicAdd(&hist[digit], 1);
     }
     __syncthreads();
     find_bin_from_top(hist, 256, kr, binfo);
     __syncthreads();
-    pre64 |= static_cast<unsigned long long>(binfo[0]) << shift;
-    pm64 |= 255ull << shift;
+    if (pass < 8) {
+      pre64 |= static_cast<unsigned long long>(binfo[0]) << (56 - 8 * pass);
+      pm64 |= 255ull << (56 - 8 * pass);
+    } else {
+      pt |= static_cast<uint32_t>(binfo[0]) << (24 - 8 * (pass - 8));
+      mt |= 255u << (24 - 8 * (pass - 8));
+    }
     kr = binfo[1];
     __syncthreads();
   }
-  {
-    const int chunk = (ncand + nthr - 1) / nthr;
-    const int i0 = min(ncand, tid * chunk), i1 = min(ncand, i0 + chunk);
-    int eq = 0;
-    for (int i = i0; i < i1; ++i) eq += okey64(kp[i]) == pre64;
-    int tot;
-    int rank = sfd::block_exclusive_scan(eq, scan_scratch, &tot);
-    int take = 0;
-    {
-      int rk = rank;
-      for (int i = i0; i < i1; ++i) {
-        const unsigned long long key = okey64(kp[i]);
-        if (key > pre64) ++take;
-        else if (key == pre64) { if (rk < kr) ++take; ++rk; }
-      }
-    }
-    int pos = sfd::block_exclusive_scan(take, scan_scratch, &tot);
-    for (int i = i0; i < i1; ++i) {
-      const unsigned long long key = okey64(kp[i]);
-      bool ok = false;
-      if (key > pre64) ok = true;
-      else if (key == pre64) { ok = rank < kr; ++rank; }
-      if (ok) sel[pos++] = F[i];
-    }
-  }}
+  // (key, ~token) pairs are distinct: the winners are those >= the k-th
+  int take = 0;
+  for (int i = tid; i < ncand; i += nthr) {
+    const unsigned long long key = okey64(kp[i]);
+    take += (key > pre64 || (key == pre64 && ~static_cast<uint32_t>(F[i]) >= pt)) ? 1 : 0;
+  }
+  int tot;
+  int pos = sfd::block_exclusive_scan(take, scan_scratch, &tot);
+  for (int i = tid; i < ncand; i += nthr) {
+    const unsigned long long key = okey64(kp[i]);
+    if (key > pre64 || (key == pre64 && ~static_cast<uint32_t>(F[i]) >= pt)) sel[pos++] = F[i];
+  }
+}
 
 // Block-parallel search of a histogram from the top (all threads call):
 // out[0] = the bin holding the kk-th largest element, out[1] = kk minus the
