@@ -71,6 +71,8 @@ def parse():
     ap.add_argument("--context", type=int, default=32768)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-extras", action="store_true", help="skip e2e / resident-only / roofline legs")
+    ap.add_argument("--long-context", type=int, default=131072,
+                    help="also time the refined step at this context (0: skip); part of the extras")
     return ap.parse_args()
 
 
@@ -554,7 +556,7 @@ def run_sf(args, rank, world, local_rank, dist):
         t_attn = ms_a / reps / args.layers * 1e-3
         attn_launch_bytes = attn_step_bytes / args.layers
         achieved_a = attn_launch_bytes / t_attn / 1e9
-        kname = "attn_fused_kernel" if cluster_attention(T) else "attention pipeline (score, select, out)"
+        kname = "attn_fused_kernel" if cluster_attention(T) else "attention pipeline (score, select, refine, out)"
         roofline = {"bound": "hbm", "kernel": kname, "achieved": achieved_a, "peak": hbm_peak,
                     "unit": "GB/s", "frac": achieved_a / hbm_peak,
                     "traffic": ATTN_TRAFFIC_32K if (T == 32768 and HQ == 32 and HKV == 8) else None,
@@ -645,10 +647,62 @@ def run_sf(args, rank, world, local_rank, dist):
     if cpu is not None:
         line["cpu_baseline"] = cpu
     line.update(extras)
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    torch.cuda.synchronize()
     del g
     model.close()
+    del model
+    if not args.skip_extras and args.long_context and args.long_context != T:
+        line["long_context"] = long_context_leg(args, sf, torch, dist, dev, world, args.long_context)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def long_context_leg(args, sf, torch, dist, dev, world, T):
+    """The same refined decode step with every layer's KV at context T
+    (128K by default: the context the tokens/s figure is quoted at), timed
+    the same way over fewer steps."""
+    model = Model(sf, torch, args.layers, T, dev)
+    steps, warm = min(args.steps, 20), 3
+    n_total = min(warm + steps, 32)
+    xpool, qpool = model.make_pools(n_total)
+    cap_stream = torch.cuda.Stream(device=dev)
+    model.xin.copy_(xpool[0])
+    model.qin.copy_(qpool[0])
+    with torch.cuda.stream(cap_stream):
+        model.step()
+    torch.cuda.synchronize()
+    model.sync_caches()
+    g = capture(torch, model.step, cap_stream)
+
+    def run_step(i):
+        model.xin.copy_(xpool[i % n_total], non_blocking=True)
+        model.qin.copy_(qpool[i % n_total], non_blocking=True)
+        g.replay()
+
+    for i in range(warm):
+        with torch.cuda.stream(cap_stream):
+            run_step(i)
+    torch.cuda.synchronize()
+    ms = timed(torch, dist, lambda i: run_step(warm + i), steps, cap_stream) / steps
+    union = float(model.sel_n.cpu().clamp(min=0).sum(dim=1).float().mean())
+    nbytes = attn_bytes(T, union) * args.layers
+    for name, N, K, slot in MATS:
+        nbytes += gemv_bytes(N, K, model.ksel[slot]) * args.layers
+    # the attention alone, all layers in one graph
+    g4 = capture(torch, model.attn_only, cap_stream)
+    for _ in range(2):
+        with torch.cuda.stream(cap_stream):
+            g4.replay()
+    ms_a = timed(torch, dist, lambda i: g4.replay(), 5, cap_stream) / 5 / args.layers
+    del g, g4
+    model.close()
+    return {"context": T, "steps": steps, "warmup": warm, "ms_per_step": ms, "tokens_per_s": world * 1e3 / ms,
+            "value": whole_job_gbs(nbytes, ms, world), "unit": "GB/s", "bytes_per_step": nbytes,
+            "union_tokens_per_layer": union,
+            "attention": {"kernel": "attn_fused_kernel" if cluster_attention(T)
+                          else "attention pipeline (score, select, refine, out)",
+                          "launch_us": ms_a * 1e3, "bytes_per_launch": attn_bytes(T, union),
+                          "achieved_gbs": attn_bytes(T, union) / (ms_a * 1e-3) / 1e9}}
 
 
 def main():

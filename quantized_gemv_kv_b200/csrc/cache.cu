@@ -352,6 +352,7 @@ sf_status cache_free(sf_refine_cache* c) {
   if (c->aux) cudaStreamDestroy(c->aux);
   if (c->registered_here) cudaHostUnregister(const_cast<void*>(c->host_master));
   delete c;
+  cudaGetLastError();  // teardown is best effort: leave no error for the next launch check
   return SF_OK;
 }
 
@@ -666,6 +667,7 @@ sf_status sf_refine_group_destroy(sf_refine_group* grp) {
   if (grp->table) cudaFree(grp->table);
   if (grp->ev_idx) cudaEventDestroy(grp->ev_idx);
   delete grp;
+  cudaGetLastError();  // teardown is best effort: leave no error for the next launch check
   return SF_OK;
 }
 
