@@ -273,13 +273,14 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
 // exact key can reach the top k has a fast score >= tau - 2 eps >= (lower
 // edge of b1) - 2 eps, so:
 //  A  compact: per (4096-token chunk, head), the tokens with fast score >=
-//     lower(b1) - 2 eps, in token order, into the chunk's slot of a list;
-//  B  finish (one cluster per KV group, one CTA per query head): concatenate
-//     the chunks, find tau exactly by two more radix passes over the listed
-//     scores of bin b1, keep the candidates >= tau - 2 eps, re-key them
-//     exactly in fp64 and rank them (key desc, token asc); then the group's
-//     CTAs build the union of their selections (bitmask and ascending list)
-//     through distributed shared memory.
+//     lower(b1) - 2 eps, appended to the head's list (one atomic per chunk;
+//     the list's order does not matter);
+//  B  finish (one cluster per KV group, one CTA per query head): find tau
+//     exactly by two more radix passes over the listed scores of bin b1,
+//     keep the candidates >= tau - 2 eps, re-key them exactly in fp64 and
+//     rank them (key desc, token asc); then the group's CTAs build the union
+//     of their selections (bitmask and ascending list) through distributed
+//     shared memory.
 
 // Per-head threshold of the compaction and the histogram bin: all threads call.
 __device__ void select_band(const int32_t* __restrict__ hist_h, int k, double eps_s, int* hsh, int* scan_scratch,
@@ -299,8 +300,8 @@ template <int GRP>
 __global__ void __launch_bounds__(kCompThreads)
 attn_select_compact_kernel(const uint16_t* __restrict__ q, int T, int k, const float* __restrict__ score,
                            const float* __restrict__ smax, const int32_t* __restrict__ hist,
-                           const uint32_t* __restrict__ amaxu, int32_t* __restrict__ cand, int nchunks,
-                           int32_t* __restrict__ status) {
+                           const uint32_t* __restrict__ amaxu, int32_t* __restrict__ cand,
+                           int32_t* __restrict__ ccnt, int32_t* __restrict__ status) {
   const int chunk = blockIdx.x, h = blockIdx.y, g = h / GRP;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   __shared__ int hsh[kHistBins];
@@ -309,6 +310,7 @@ attn_select_compact_kernel(const uint16_t* __restrict__ q, int T, int k, const f
   __shared__ double qd[D];
   __shared__ double l1_sh;
   __shared__ int qe_sh;
+  __shared__ int base_sh;
   select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status);
   const double eps_s = select_eps(static_cast<double>(smax[g]), l1_sh, qe_sh, __uint_as_float(amaxu[h]));
   uint32_t b1;
@@ -339,11 +341,12 @@ attn_select_compact_kernel(const uint16_t* __restrict__ q, int T, int k, const f
       if (lane >= o) incl += y;
     }
     if (lane < kCompThreads / 32) scan_scratch[32 + lane] = incl - v;
-    // the chunks' counts follow the Hq x T lists
-    if (lane == 31) cand[static_cast<size_t>(gridDim.y) * T + static_cast<size_t>(h) * nchunks + chunk] = incl;
+    // the chunk's run of the head's list (the list's order does not matter:
+    // the finish ranks by key and token)
+    if (lane == 31) base_sh = incl ? atomicAdd(ccnt + h, incl) : 0;
   }
   __syncthreads();
-  int32_t* out = cand + static_cast<size_t>(h) * T + static_cast<size_t>(chunk) * kChunk;
+  int32_t* out = cand + static_cast<size_t>(h) * T + base_sh;
   int o = scan_scratch[32 + warp];
   const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
@@ -356,7 +359,6 @@ attn_select_compact_kernel(const uint16_t* __restrict__ q, int T, int k, const f
 
 constexpr int kFinThreads = 512;
 constexpr int kFinKeys = 2048;     // candidates ranked pairwise from shared memory
-constexpr int kFinChunks = 4096;   // chunk prefix sums in shared memory (T <= 2^24)
 constexpr int kFinList = 4096;     // listed (token, score) pairs cached in shared memory
 constexpr size_t kFinDynSmem = static_cast<size_t>(kFinList) * 8 + static_cast<size_t>(kFinKeys) * 4;
 
@@ -366,17 +368,17 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
                           const uint32_t* __restrict__ k_ref, const uint16_t* __restrict__ k_scale,
                           const uint16_t* __restrict__ k_zero, int T, int k, float* __restrict__ score,
                           const float* __restrict__ smax, const int32_t* __restrict__ hist,
-                          const uint32_t* __restrict__ amaxu, int32_t* __restrict__ cand, int nchunks,
-                          int32_t* __restrict__ list, double* __restrict__ kap, int32_t* __restrict__ sel_head,
-                          uint32_t* __restrict__ umask, int words_t, int32_t* __restrict__ sel_out,
-                          int32_t* __restrict__ sel_n, int32_t* __restrict__ status, uint32_t* __restrict__ mkey) {
+                          const uint32_t* __restrict__ amaxu, const int32_t* __restrict__ cand,
+                          const int32_t* __restrict__ ccnt, int32_t* __restrict__ list, double* __restrict__ kap,
+                          int32_t* __restrict__ sel_head, uint32_t* __restrict__ umask, int words_t,
+                          int32_t* __restrict__ sel_out, int32_t* __restrict__ sel_n, int32_t* __restrict__ status,
+                          uint32_t* __restrict__ mkey) {
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
   const int rank = static_cast<int>(cl.block_rank());
   const int h = blockIdx.x, g = h / GRP;
   const int tid = threadIdx.x;
   __shared__ int hr[2048];
-  __shared__ int cpre[kFinChunks];
   __shared__ unsigned long long keys[kFinKeys];  // order-preserving exact keys, sorted with the tokens
   __shared__ double qd[D];
   __shared__ int scan_scratch[64];
@@ -392,8 +394,8 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   float* lsc = reinterpret_cast<float*>(fin_dyn + kFinList);  // [kFinList]
   int* ktok = fin_dyn + 2 * kFinList;                       // [kFinKeys] tokens of the sorted keys
   const float* sc = score + static_cast<size_t>(h) * T;
-  int32_t* L = list + static_cast<size_t>(h) * T;  // concatenated list, token order
-  int32_t* F = cand + static_cast<size_t>(h) * T;  // candidates (reuses the chunk lists once L is built)
+  const int32_t* L = cand + static_cast<size_t>(h) * T;  // the compaction's list
+  int32_t* F = list + static_cast<size_t>(h) * T;        // band candidates
   double* kp = kap + static_cast<size_t>(h) * T;
   const int cap = GRP * k;
 
@@ -427,32 +429,13 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   float f_low;
   select_band(hist + static_cast<size_t>(h) * kHistBins, k, eps_s, hr, scan_scratch, binfo, &b1, &kk, &f_low);
 
-  // 1. concatenate the chunk lists (token order); with their fast scores in
-  //    shared memory when they fit
-  const int32_t* counts = cand + static_cast<size_t>(gridDim.x) * T + static_cast<size_t>(h) * nchunks;
-  int m = 0;
-  for (int base = 0; base < nchunks; base += kFinThreads) {
-    const int c = base + tid;
-    const int v = c < nchunks ? counts[c] : 0;
-    int tot;
-    const int pre = sfd::block_exclusive_scan(v, scan_scratch, &tot);
-    if (c < nchunks) cpre[c] = m + pre;
-    m += tot;
-  }
-  __syncthreads();
-  for (int e = tid; e < m; e += kFinThreads) {
-    int lo = 0, hi = nchunks - 1;  // last chunk with cpre <= e
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (cpre[mid] <= e) lo = mid;
-      else hi = mid - 1;
-    }
-    const int t = cand[static_cast<size_t>(h) * T + static_cast<size_t>(lo) * kChunk + (e - cpre[lo])];
-    if (m <= kFinList) {
+  // 1. the compaction's list, with its fast scores in shared memory when it fits
+  const int m = min(ccnt[h], T);
+  if (m <= kFinList) {
+    for (int e = tid; e < m; e += kFinThreads) {
+      const int t = L[e];
       ltok[e] = t;
       lsc[e] = sc[t];
-    } else {
-      L[e] = t;
     }
   }
   __syncthreads();
@@ -659,7 +642,8 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
 
 // ---- refined scores of the union --------------------------------------------------
 //
-// Between the selection and pass B: every token of a group's union gets its
+// Step R, between the selection and pass B: every token of a group's union
+// gets its
 // scores for the group's query heads recomputed from the full 4-bit key codes,
 // in place in the score buffer, and the largest refined score per head is
 // recorded as an order-preserving key.  Pass B then weights every token
@@ -1136,8 +1120,9 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
   sf_status st = sf::check_launch("attn_score_mma_kernel");
   if (st != SF_OK) return st;
   if (k > 0 && k < T) {
+    int32_t* ccnt = reinterpret_cast<int32_t*>(ws + L.ccnt);
     attn_select_compact_kernel<GRP><<<dim3(L.nchunks, Hq), kCompThreads, 0, s>>>(q, T, k, score, smax, hist, amaxu,
-                                                                                cand, L.nchunks, status);
+                                                                                cand, ccnt, status);
     st = sf::check_launch("attn_select_compact_kernel");
     if (st != SF_OK) return st;
     cudaLaunchConfig_t cfg{};
@@ -1157,8 +1142,8 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
     SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, attn_select_finish_kernel<GRP>, q, kv->k_res, kv->k_ref, kv->k_scale,
                                      kv->k_zero, T, k, score, static_cast<const float*>(smax),
                                      static_cast<const int32_t*>(hist), static_cast<const uint32_t*>(amaxu), cand,
-                                     L.nchunks, cand2, kap, sel_head, umask, L.words_t, sel_out, sel_n, status,
-                                     mkey));
+                                     static_cast<const int32_t*>(ccnt), cand2, kap, sel_head, umask, L.words_t,
+                                     sel_out, sel_n, status, mkey));
     st = sf::check_launch("attn_select_finish_kernel");
     if (st != SF_OK) return st;
   } else if (k == 0) {  // the token bitmask was cleared with the workspace

@@ -37,7 +37,7 @@ constexpr int kChunk = 4096;       // tokens per CTA of the candidate compaction
 
 struct Layout {
   // from smax on, everything is cleared at the start of a call
-  size_t score, cand, cand2, kap, sel, part, fcnt, smax, status, count, amax, mkey, rkey, hist, umask, total;
+  size_t score, cand, cand2, kap, sel, part, fcnt, smax, status, count, amax, mkey, rkey, ccnt, hist, umask, total;
   int splits, tps, words_t, nchunks;
 };
 
@@ -67,6 +67,7 @@ Layout make_layout(int Hq, int Hkv, int T, int k, int sms) {
   L.amax = off; off = up256(off + sizeof(uint32_t) * Hq);
   L.mkey = off; off = up256(off + sizeof(uint32_t) * Hq);  // max resident score key per head
   L.rkey = off; off = up256(off + sizeof(uint32_t) * Hq);  // max refined score key per head
+  L.ccnt = off; off = up256(off + sizeof(int32_t) * Hq);   // listed candidates per head
   L.hist = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(kHistBins));
   L.umask = off; off = up256(off + sizeof(uint32_t) * Hkv * static_cast<size_t>(L.words_t));
   L.total = off;
