@@ -565,8 +565,11 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
       for (int p = 0; p < 3; ++p)
 #pragma unroll
         for (int half = 0; half < 2; ++half) bq[ks][p][half] = bfr[(ks * 3 + p) * 2 + half][lane];
-    // this lane's heads 2 tig, 2 tig + 1 (the epilogue runs on lanes holding a head)
-    const int h0 = 2 * tig, h1 = 2 * tig + 1;
+    // this lane's heads 2 tig, 2 tig + 1 (the epilogue runs on lanes holding a
+    // head); with four heads, 2 (tig & 1) and the next, lanes tig >= 2 scoring
+    // the second token of each tile (columns 4..7 of the MMA are padding)
+    constexpr bool kSwap = GRP == 4;
+    const int h0 = kSwap ? 2 * (tig & 1) : 2 * tig, h1 = h0 + 1;
     const bool on = h0 < GRP;
     const float qsc0 = on ? qsc[h0] : 0.0f, qsm0 = on ? qsm[h0] : 0.0f;
     const float qsc1 = h1 < GRP ? qsc[h1] : 0.0f, qsm1 = h1 < GRP ? qsm[h1] : 0.0f;
@@ -607,15 +610,32 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
           mma_u8u8(d1[u], a0, a1, a2, a3, bq[ks][1][0], bq[ks][1][1]);
           mma_u8s8(d2[u], a0, a1, a2, a3, bq[ks][2][0], bq[ks][2][1]);
         }
-      // d[u][i]: i = 0,1 -> token ta, heads h0, h1; i = 2,3 -> token tb
+      // d[u][i]: i = 0,1 -> token ta, heads 2 tig, 2 tig + 1; i = 2,3 -> token tb
+      if constexpr (kSwap) {
+        // lanes tig >= 2 take token tb of lane ^ 2 into slots 0, 1
+        const bool up = tig >= 2;
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int i = 2; i < 4; ++i) {
+            const int x0 = __shfl_xor_sync(0xffffffffu, d0[u][i], 2);
+            const int x1 = __shfl_xor_sync(0xffffffffu, d1[u][i], 2);
+            const int x2 = __shfl_xor_sync(0xffffffffu, d2[u][i], 2);
+            if (up) {
+              d0[u][i - 2] = x0;
+              d1[u][i - 2] = x1;
+              d2[u][i - 2] = x2;
+            }
+          }
+      }
       if (on) {
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int ta = 16 * (ti + u) + g8, tb = ta + 8;
           const bool tv = ti + u < tile1;  // a missing second tile holds no keys
 #pragma unroll
-          for (int rr = 0; rr < 2; ++rr) {
-            const int tt = rr ? tb : ta;
+          for (int rr = 0; rr < (kSwap ? 1 : 2); ++rr) {
+            const int tt = kSwap ? (tig >= 2 ? tb : ta) : (rr ? tb : ta);
             if (!tv || tt >= n) continue;
             const uint32_t kz = ksz[tt];
             const float sv = sfd::half_bits_to_float(static_cast<uint16_t>(kz & 0xFFFFu));
