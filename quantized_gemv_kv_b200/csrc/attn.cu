@@ -929,27 +929,17 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
         b0[nt] = *reinterpret_cast<const uint32_t*>(ar);
         b1[nt] = *reinterpret_cast<const uint32_t*>(ar + 8);
       }
-      const uint4* ra = reinterpret_cast<const uint4*>(vr + (2 * tig) * kWordsPerRow);
-      const uint4* rb = reinterpret_cast<const uint4*>(vr + (2 * tig + 1) * kWordsPerRow);
-      const uint4* rc = reinterpret_cast<const uint4*>(vr + (2 * tig + 8) * kWordsPerRow);
-      const uint4* rd = reinterpret_cast<const uint4*>(vr + (2 * tig + 9) * kWordsPerRow);
+      // word g8 of token rows 2 tig, 2 tig + 1, 2 tig + 8, 2 tig + 9: MMA s
+      // covers dims 16 g8 + s and 16 g8 + 8 + s (vfrag)
+      uint32_t src[4][4];
+      vperm(vr[(2 * tig) * kWordsPerRow + g8], vr[(2 * tig + 1) * kWordsPerRow + g8],
+            vr[(2 * tig + 8) * kWordsPerRow + g8], vr[(2 * tig + 9) * kWordsPerRow + g8], src);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const uint4 A4 = ra[half], B4 = rb[half], C4 = rc[half], D4 = rd[half];
-        const uint32_t wa[4] = {A4.x, A4.y, A4.z, A4.w}, wb[4] = {B4.x, B4.y, B4.z, B4.w};
-        const uint32_t wc[4] = {C4.x, C4.y, C4.z, C4.w}, wd[4] = {D4.x, D4.y, D4.z, D4.w};
+      for (int s = 0; s < 8; ++s) {
+        uint32_t a0, a1, a2, a3;
+        vfrag(src, s, a0, a1, a2, a3);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int w = half * 4 + j;  // dims 16 w .. 16 w + 15
-          const uint32_t xa = wa[j] >> (2 * g8), xb = wb[j] >> (2 * g8);
-          const uint32_t xc = wc[j] >> (2 * g8), xd = wd[j] >> (2 * g8);
-          const uint32_t a0 = (__byte_perm(xa, xb, 0x5410) & 0x00030003u) | 0x64006400u;  // dim g8
-          const uint32_t a1 = (__byte_perm(xa, xb, 0x7632) & 0x00030003u) | 0x64006400u;  // dim g8 + 8
-          const uint32_t a2 = (__byte_perm(xc, xd, 0x5410) & 0x00030003u) | 0x64006400u;
-          const uint32_t a3 = (__byte_perm(xc, xd, 0x7632) & 0x00030003u) | 0x64006400u;
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_f16f32(acc[nt][w], a0, a1, a2, a3, b0[nt], b1[nt]);
-        }
+        for (int nt = 0; nt < NT; ++nt) mma_f16f32(acc[nt][s], a0, a1, a2, a3, b0[nt], b1[nt]);
       }
       __syncwarp();
     }
@@ -973,10 +963,11 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
     __syncthreads();  // weights and the list are rewritten by the next sub-chunk
   }
 
-  // this warp's output tile ww[head][dim] (in units of the code part: uo
-  // enters divided by 2^b_f = 4) in the dead weight tile, written in three
-  // phases whose stores within a warp never collide (high columns, then
-  // remainder columns, then the refined corrections); summed over warps below
+  // this warp's output tile ww[head][dim] (in units of the code part, which
+  // carries the factor 4^e of the dim's fragment position: uo enters as
+  // uo 4^e / 2^b_f) in the dead weight tile, written in three phases whose
+  // stores within a warp never collide (high columns, then remainder
+  // columns, then the refined corrections); summed over warps below
   __syncthreads();  // every warp is done with the weight tile
   float* ww = reinterpret_cast<float*>(smem) + warp * GRP * D;
 #pragma unroll
@@ -990,7 +981,7 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
           const int n = nt * 8 + 2 * tig + (c & 1);
           const int hh = colh[nt][c & 1];
           if (hh < 0 || (n < GRP) != (ph == 0)) continue;
-          float* dst = &ww[hh * D + 16 * w + g8 + 8 * (c >> 1)];
+          float* dst = &ww[hh * D + 16 * g8 + w + 8 * (c >> 1)];  // MMA w, row g8 (+ 8)
           *dst = ph == 0 ? acc[nt][w][c] : *dst + acc[nt][w][c];
         }
     __syncwarp();
@@ -998,7 +989,7 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
 #pragma unroll
   for (int h = 0; h < GRP; ++h)
 #pragma unroll
-    for (int dd = 0; dd < 4; ++dd) ww[h * D + 4 * lane + dd] += 0.25f * uo[h][dd];
+    for (int dd = 0; dd < 4; ++dd) ww[h * D + 4 * lane + dd] += (0.25f * vpos_mul(4 * lane + dd)) * uo[h][dd];
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
     const float l = warp_sum(lsum[h]), cs = warp_sum(csum[h]), a = warp_sum(asum[h]);
@@ -1022,11 +1013,13 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
         Cs += red2[w][GRP + h];
         A += red2[w][2 * GRP + h];
       }
-      // resident value s (2^b_f c + m_f - z): code part 4 (acc - 1024 A), offset part Cs
+      // resident value s (2^b_f c + m_f - z): code part 4 (acc - 1024 A) 4^-e,
+      // offset part Cs
       float o = 0.0f;
       if (j >= 2)
         for (int w = 0; w < kOW; ++w) o += reinterpret_cast<const float*>(smem)[(w * GRP + h) * D + j - 2];
-      v = j == 1 ? L : fmaf(4.0f, o, fmaf(-4096.0f, A, Cs));
+      const float f = j >= 2 ? vpos_inv(j - 2) : 1.0f;
+      v = j == 1 ? L : fmaf(4.0f * f, o, fmaf(-4096.0f * f, A, Cs));
     }
     pg[(static_cast<size_t>(h) * splits + split) * (D + 2) + j] = v;
   }

@@ -120,6 +120,47 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Value codes as f16 MMA fragments.  An MMA row (a dim of the output) need
+// not follow the dims' order: lane row g8 (g8 + 8) of MMA s takes dim
+// 16 g8 + s (16 g8 + 8 + s), so a lane reads word g8 of its four token rows
+// once per 16-token tile; two byte permutes per row pair put dims 0-7 (8-15)
+// of the two tokens in the halves of a register, four shifted copies (left
+// 6 and 2, right 2 and 6) bring the code of every s to mantissa bits 6-7 or
+// 8-9, and each fragment register is one mask and or: the exact f16 pair
+// 1024 + c 4^e, e = 3 + (s & 1).  The dim's accumulated code part carries the
+// factor 4^e, taken out when the partials are formed; against the 1024
+// offset the code part is large (64 c or 256 c), so the offset's removal
+// loses little of the fp32 accumulation's precision.
+__device__ __forceinline__ int vpos_exp(int dim) { return 3 + (dim & 1); }
+// 4^-e for the dim's exponent e (exact)
+__device__ __forceinline__ float vpos_inv(int dim) { return __int_as_float((127 - 2 * vpos_exp(dim)) << 23); }
+// 4^e
+__device__ __forceinline__ float vpos_mul(int dim) { return __int_as_float((127 + 2 * vpos_exp(dim)) << 23); }
+// The four fragment registers of MMA s (a constant after unrolling) from the
+// shifted permutes src[s / 2] (vperm).
+__device__ __forceinline__ void vfrag(const uint32_t (&src)[4][4], int s, uint32_t& a0, uint32_t& a1, uint32_t& a2,
+                                      uint32_t& a3) {
+  const uint32_t m = (s & 1) ? 0x03000300u : 0x00C000C0u;
+  a0 = (src[s >> 1][0] & m) | 0x64006400u;
+  a1 = (src[s >> 1][1] & m) | 0x64006400u;
+  a2 = (src[s >> 1][2] & m) | 0x64006400u;
+  a3 = (src[s >> 1][3] & m) | 0x64006400u;
+}
+// A lane's words for one tile: word g8 of token rows 2 tig, 2 tig + 1
+// (wa, wb: registers 0, 1 = dims 0-7, 8-15) and 2 tig + 8, 2 tig + 9 (wc, wd:
+// registers 2, 3), each in the four shifted copies.
+__device__ __forceinline__ void vperm(uint32_t wa, uint32_t wb, uint32_t wc, uint32_t wd, uint32_t (&src)[4][4]) {
+  const uint32_t p[4] = {__byte_perm(wa, wb, 0x5410), __byte_perm(wa, wb, 0x7632), __byte_perm(wc, wd, 0x5410),
+                         __byte_perm(wc, wd, 0x7632)};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    src[0][i] = p[i] << 6;  // s = 0, 1
+    src[1][i] = p[i] << 2;  // s = 2, 3
+    src[2][i] = p[i] >> 2;  // s = 4, 5
+    src[3][i] = p[i] >> 6;  // s = 6, 7
+  }
+}
+
 // f16 tensor-core MMA with f32 accumulate (m16n8k16).
 __device__ __forceinline__ void mma_f16f32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                            uint32_t b0, uint32_t b1) {

@@ -1100,37 +1100,24 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
         b0[u][nt] = (u == 0 || two) ? *reinterpret_cast<const uint32_t*>(ar) : 0u;
         b1[u][nt] = (u == 0 || two) ? *reinterpret_cast<const uint32_t*>(ar + 8) : 0u;
       }
+    // word g8 of token rows 2 tig, 2 tig + 1, 2 tig + 8, 2 tig + 9 of each
+    // tile: MMA s covers dims 16 g8 + s and 16 g8 + 8 + s (vfrag)
+    uint32_t src[2][4][4];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint32_t wa[2][4], wb[2][4], wc[2][4], wd[2][4];
+    for (int u = 0; u < 2; ++u) {
+      const uint32_t* vr = ring + (warp * kFRing + (ti + u - tile0) % kFRing) * 16 * kWordsPerRow;
+      vperm(vr[(2 * tig) * kWordsPerRow + g8], vr[(2 * tig + 1) * kWordsPerRow + g8],
+            vr[(2 * tig + 8) * kWordsPerRow + g8], vr[(2 * tig + 9) * kWordsPerRow + g8], src[u]);
+    }
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const uint32_t* vr = ring + (warp * kFRing + (ti + u - tile0) % kFRing) * 16 * kWordsPerRow;
-        const uint4 A4 = reinterpret_cast<const uint4*>(vr + (2 * tig) * kWordsPerRow)[half];
-        const uint4 B4 = reinterpret_cast<const uint4*>(vr + (2 * tig + 1) * kWordsPerRow)[half];
-        const uint4 C4 = reinterpret_cast<const uint4*>(vr + (2 * tig + 8) * kWordsPerRow)[half];
-        const uint4 D4 = reinterpret_cast<const uint4*>(vr + (2 * tig + 9) * kWordsPerRow)[half];
-        wa[u][0] = A4.x; wa[u][1] = A4.y; wa[u][2] = A4.z; wa[u][3] = A4.w;
-        wb[u][0] = B4.x; wb[u][1] = B4.y; wb[u][2] = B4.z; wb[u][3] = B4.w;
-        wc[u][0] = C4.x; wc[u][1] = C4.y; wc[u][2] = C4.z; wc[u][3] = C4.w;
-        wd[u][0] = D4.x; wd[u][1] = D4.y; wd[u][2] = D4.z; wd[u][3] = D4.w;
+        uint32_t a0, a1, a2, a3;
+        vfrag(src[u], s, a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_f16f32(acc[nt][s], a0, a1, a2, a3, b0[u][nt], b1[u][nt]);
       }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int w = half * 4 + j;  // dims 16 w .. 16 w + 15
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const uint32_t xa = wa[u][j] >> (2 * g8), xb = wb[u][j] >> (2 * g8);
-          const uint32_t xc = wc[u][j] >> (2 * g8), xd = wd[u][j] >> (2 * g8);
-          const uint32_t a0 = (__byte_perm(xa, xb, 0x5410) & 0x00030003u) | 0x64006400u;  // dim g8
-          const uint32_t a1 = (__byte_perm(xa, xb, 0x7632) & 0x00030003u) | 0x64006400u;  // dim g8 + 8
-          const uint32_t a2 = (__byte_perm(xc, xd, 0x5410) & 0x00030003u) | 0x64006400u;
-          const uint32_t a3 = (__byte_perm(xc, xd, 0x7632) & 0x00030003u) | 0x64006400u;
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_f16f32(acc[nt][w], a0, a1, a2, a3, b0[u][nt], b1[u][nt]);
-        }
-      }
-    }
     __syncwarp();
   }
   cp_async_wait_attn<0>();
@@ -1157,9 +1144,10 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
   }
   __syncthreads();  // every warp is done with the weight tile
 
-  // this warp's output tile ww[head][dim] (in units of the code part: uo
-  // enters divided by 2^b_f = 4) in the dead weight tile; the high and low
-  // weight columns of a head meet in one lane (or a lane pair)
+  // this warp's output tile ww[head][dim] (in units of the code part, which
+  // carries the factor 4^e of the dim's fragment position: uo enters as
+  // uo 4^e / 2^b_f) in the dead weight tile; the high and low weight columns
+  // of a head meet in one lane (or a lane pair)
   float* ww = reinterpret_cast<float*>(smem + S.sc) + warp * GRP * D;
 #pragma unroll
   for (int w = 0; w < 8; ++w)
@@ -1181,13 +1169,13 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
         hh = 2 * tig + (c & 1);
         st = tig < GRP / 2;
       }
-      if (st) ww[hh * D + 16 * w + g8 + 8 * (c >> 1)] = v;
+      if (st) ww[hh * D + 16 * g8 + w + 8 * (c >> 1)] = v;  // MMA w, row g8 (+ 8)
     }
   __syncwarp();
 #pragma unroll
   for (int h = 0; h < GRP; ++h)
 #pragma unroll
-    for (int dd = 0; dd < 4; ++dd) ww[h * D + 4 * lane + dd] += 0.25f * uo[h][dd];
+    for (int dd = 0; dd < 4; ++dd) ww[h * D + 4 * lane + dd] += (0.25f * vpos_mul(4 * lane + dd)) * uo[h][dd];
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
     const float l = warp_sum(lsum[h]), cs = warp_sum(csum[h]), s = warp_sum(asum[h]);
@@ -1213,8 +1201,10 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
         A += red2[w][2 * GRP + h];
         if (j >= 2) o += reinterpret_cast<const float*>(smem + S.sc)[(w * GRP + h) * D + j - 2];
       }
-      // resident value s (2^b_f c + m_f - z): code part 4 (acc - 1024 A), offset part Cs
-      v = j == 1 ? Lsum : fmaf(4.0f, o, fmaf(-4096.0f, A, Cs));
+      // resident value s (2^b_f c + m_f - z): code part 4 (acc - 1024 A) 4^-e,
+      // offset part Cs
+      const float f = j >= 2 ? vpos_inv(j - 2) : 1.0f;
+      v = j == 1 ? Lsum : fmaf(4.0f * f, o, fmaf(-4096.0f * f, A, Cs));
     }
     gp[e] = v;
   }

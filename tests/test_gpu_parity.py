@@ -333,6 +333,32 @@ def test_attn_32k(sf, attn_path):
     assert err <= ATTN_TOL, err
 
 
+def test_attn_128k_sampled_groups(sf, attn_path):
+    """The bench's long-context launch configuration: 128K context, 32 query /
+    8 KV heads, top 1% tokens per query head, all eight groups on the GPU;
+    the oracle checks the first and the last KV head (union and outputs of
+    their four query heads).  Quantization is per token-head row, so each
+    sampled group is quantized on its own for the oracle."""
+    Hq, Hkv, T, d = 32, 8, 131072, 128
+    _skip_unless_applies(attn_path, Hq, Hkv, T)
+    Kf, Vf, _ = gen_kv(3128, Hkv, T, d)
+    kv = sf.QKV(sf.quantize_nested(dev(Kf.reshape(Hkv * T, d)), d, 2, 2, "by_row"),
+                sf.quantize_nested(dev(Vf.reshape(Hkv * T, d)), d, 2, 2, "by_row"))
+    qb = gen_query(4128, Hq, d)
+    k = count_fraction(1, T)
+    out, sel, sel_n = sf.attn_decode_refine(bf16_dev(qb), kv, Hkv, T, k)
+    torch.cuda.synchronize()
+    out, sel, sel_n = out.cpu().numpy(), sel.cpu().numpy(), sel_n.cpu().numpy()
+    grp = Hq // Hkv
+    for g in (0, Hkv - 1):
+        ok, ov = oquant.quantize_nested(Kf[g], d, 2, 2), oquant.quantize_nested(Vf[g], d, 2, 2)
+        ref = oattn.attn_decode_refine(qb[g * grp:(g + 1) * grp], ok, ov, 1, T, k)
+        assert sel_n[g] == len(ref["union"][0])
+        np.testing.assert_array_equal(sel[g, : sel_n[g]], ref["union"][0])
+        err = np.abs(out[g * grp:(g + 1) * grp].astype(np.float64) - ref["out"]).max()
+        assert err <= ATTN_TOL, err
+
+
 def test_attn_band_overflow(sf, attn_path):
     """Half the tokens of each KV head are copies of one token, and k puts the
     k-th largest key of query head 0 inside that tie: thousands of exactly
