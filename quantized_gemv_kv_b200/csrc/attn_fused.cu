@@ -967,39 +967,57 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
     cp_async16_attn(stg + u * kWordsPerRow + 4, src + 4);
   }
   cp_async_commit_attn();
-  // refined scores of the union tokens from their full 4-bit key codes:
-  // thread per (head, token), a warp's threads sharing the head
+  // refined scores of the union tokens from their full 4-bit key codes: four
+  // lanes per token, lane q taking words q and q + 4 (32 dims) for every head
+  // of the group (each code extracted once), summed over the four lanes
   cp_async_wait_attn<1>();  // the staged key rows (the value rows may still be in flight)
   __syncthreads();
-  for (int e = tid; e < nu * GRP; e += kFThreads) {
-    const int h = e / nu, i = ulist[e - h * nu];
-    const int s = selecting ? smap[i] : 0xFF;
-    const uint4* pr;
-    const uint4* pf;
-    if (s != 0xFF) {  // staged during the selection
-      pr = reinterpret_cast<const uint4*>(kst + s * 2 * kWordsPerRow);
-      pf = pr + 2;
-    } else {
-      pr = reinterpret_cast<const uint4*>(a.k_res + (row0 + i) * kWordsPerRow);
-      pf = reinterpret_cast<const uint4*>(a.k_ref + (row0 + i) * kWordsPerRow);
-    }
-    const uint4 r0 = pr[0], r1 = pr[1], f0 = pf[0], f1 = pf[1];
-    const uint32_t wr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-    const uint32_t wf[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-    float P[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll 1
-    for (int w = 0; w < 8; ++w) {
-      const uint32_t rw = wr[w], fw = wf[w];
+  {
+    const int qq = lane & 3;
+    for (int base = 0; base < nu; base += kFThreads / 4) {  // uniform over the block: the shuffles
+      const int u = base + (tid >> 2);
+      const bool valid = u < nu;
+      const int i = valid ? ulist[u] : 0;
+      float P[GRP];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float c = i2f_exact(static_cast<int>(((rw >> (2 * j)) & 3u) * 4u + ((fw >> (2 * j)) & 3u)));
-        P[j & 3] = fmaf(qs[h][16 * w + j], c, P[j & 3]);
+      for (int h = 0; h < GRP; ++h) P[h] = 0.0f;
+      if (valid) {
+        const int s = selecting ? smap[i] : 0xFF;
+        const uint32_t* pr;
+        const uint32_t* pf;
+        if (s != 0xFF) {  // staged during the selection: resident words, then refinement words
+          pr = kst + s * 2 * kWordsPerRow;
+          pf = pr + kWordsPerRow;
+        } else {
+          pr = a.k_res + (row0 + i) * kWordsPerRow;
+          pf = a.k_ref + (row0 + i) * kWordsPerRow;
+        }
+        const uint32_t r0 = pr[qq], r1 = pr[qq + 4], f0 = pf[qq], f1 = pf[qq + 4];
+#pragma unroll
+        for (int ww = 0; ww < 2; ++ww) {
+          const int w = qq + 4 * ww;
+          const uint32_t rw = ww ? r1 : r0, fw = ww ? f1 : f0;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float c = i2f_exact(static_cast<int>(((rw >> (2 * j)) & 3u) * 4u + ((fw >> (2 * j)) & 3u)));
+#pragma unroll
+            for (int h = 0; h < GRP; ++h) P[h] = fmaf(qs[h][16 * w + j], c, P[h]);
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) {
+        P[h] += __shfl_xor_sync(0xffffffffu, P[h], 1);
+        P[h] += __shfl_xor_sync(0xffffffffu, P[h], 2);
+      }
+      if (valid && qq == 0) {
+        const uint32_t kz = ksz[i];
+        const float sv = sfd::half_bits_to_float(static_cast<uint16_t>(kz & 0xFFFFu));
+        const float z = sfd::half_bits_to_float(static_cast<uint16_t>(kz >> 16));
+#pragma unroll
+        for (int h = 0; h < GRP; ++h) sc[h * R + i] = (sv * fmaf(-z, qsm[h], P[h])) * kInvSqrtD;
       }
     }
-    const uint32_t kz = ksz[i];
-    const float sv = sfd::half_bits_to_float(static_cast<uint16_t>(kz & 0xFFFFu));
-    const float z = sfd::half_bits_to_float(static_cast<uint16_t>(kz >> 16));
-    sc[h * R + i] = (sv * fmaf(-z, qsm[h], (P[0] + P[1]) + (P[2] + P[3]))) * kInvSqrtD;
   }
   __syncthreads();
 
