@@ -77,6 +77,7 @@ constexpr int kScThreads = 256;
 constexpr int kScW = kScThreads / 32;
 constexpr int kScRing = 8;        // cp.async stages per warp, one 16-token tile each
 constexpr int kScMaxTok = 4096;   // tokens per CTA at most
+static_assert(kScMaxTok % kScThreads == 0, "the key scales are staged in whole rounds");
 
 __host__ __device__ constexpr size_t score_smem(int grp) {
   return static_cast<size_t>(kScW) * kScRing * 16 * kWordsPerRow * 4 + static_cast<size_t>(kScMaxTok) * 4 +
@@ -95,6 +96,7 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
   int* hs = reinterpret_cast<int*>(ksz + kScMaxTok);                 // [GRP][kHistBins]
   __shared__ int qx[GRP][D];
   __shared__ float qsc[GRP], qsm[GRP];
+  __shared__ uint32_t bfr[24][32];  // B fragments of qx, per lane
   const int g = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g8 = lane >> 2, tig = lane & 3;
   const int t0 = blockIdx.x * tpc;
@@ -117,11 +119,25 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
   // per-head histogram of this CTA's scores over the top 11 bits of the
   // order-preserving key (pass S starts from the sum over all CTAs)
   for (int i = tid; i < GRP * kHistBins; i += kScThreads) hs[i] = 0;
+  // the range's key scales and zeros: every load of this thread is issued
+  // before the first store
   float smx = 0.0f;
-  for (int i = tid; i < n; i += kScThreads) {
-    const uint32_t kz = static_cast<uint32_t>(k_scale[row0 + i]) | (static_cast<uint32_t>(k_zero[row0 + i]) << 16);
-    ksz[i] = kz;
-    smx = fmaxf(smx, sfd::half_bits_to_float(static_cast<uint16_t>(kz & 0xFFFFu)));
+  {
+    constexpr int kPer = kScMaxTok / kScThreads;
+    uint32_t kzv[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = tid + j * kScThreads;
+      kzv[j] = i < n ? static_cast<uint32_t>(k_scale[row0 + i]) | (static_cast<uint32_t>(k_zero[row0 + i]) << 16) : 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = tid + j * kScThreads;
+      if (i < n) {
+        ksz[i] = kzv[j];
+        smx = fmaxf(smx, sfd::half_bits_to_float(static_cast<uint16_t>(kzv[j] & 0xFFFFu)));
+      }
+    }
   }
   // fixed-point query heads (warp h builds head h, 4 dims per lane) and the
   // sums of q (any order: the error bound covers it)
@@ -145,22 +161,27 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
     }
   }
   __syncthreads();
-  // B fragments: column n = g8 is query head g8 (zero beyond the group)
+  // B fragments (column n = g8 is query head g8, zero beyond the group),
+  // built once per CTA: word [ks][p][half][lane]
+  for (int e = tid; e < 24 * 32; e += kScThreads) {
+    const int ln = e & 31, f = e >> 5, ks = f / 6, p = (f / 2) % 3, half = f & 1;
+    const int gg = ln >> 2, tt = ln & 3;
+    uint32_t v = 0;
+    if (gg < GRP) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        v |= ((static_cast<uint32_t>(qx[gg][16 * (2 * ks + half) + tt + 4 * i]) >> (8 * p)) & 0xFFu) << (8 * i);
+    }
+    bfr[f][ln] = v;
+  }
+  __syncthreads();
   uint32_t bq[4][3][2];
 #pragma unroll
   for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
-    for (int half = 0; half < 2; ++half)
+    for (int p = 0; p < 3; ++p)
 #pragma unroll
-      for (int p = 0; p < 3; ++p) {
-        uint32_t v = 0;
-        if (g8 < GRP) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            v |= ((static_cast<uint32_t>(qx[g8][16 * (2 * ks + half) + tig + 4 * i]) >> (8 * p)) & 0xFFu) << (8 * i);
-        }
-        bq[ks][p][half] = v;
-      }
+      for (int half = 0; half < 2; ++half) bq[ks][p][half] = bfr[(ks * 3 + p) * 2 + half][lane];
   // this lane's heads (2 tig, 2 tig + 1; with four heads 2 (tig & 1) and the
   // next, lanes tig >= 2 scoring the second token of the pair): max |score|
   // and the largest score key
