@@ -8,8 +8,7 @@
 // cluster.  Each CTA of the cluster owns a contiguous token range of the
 // group:
 //
-//   1  score    stream the range's 2-bit keys (L2-prefetched in bulk at the
-//               start, together with the values) through per-warp cp.async
+//   1  score    stream the range's 2-bit keys through per-warp cp.async
 //               rings into integer tensor-core MMAs; the fast scores of all
 //               the group's heads stay in shared memory.
 //   2  tau      the k-th largest fast score per head is bracketed by radix
