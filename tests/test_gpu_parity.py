@@ -291,13 +291,16 @@ def _skip_unless_applies(path, Hq, Hkv, T):
 @pytest.mark.parametrize("Hq,Hkv,T,pct", [(8, 2, 1000, 1), (32, 8, 4099, 1), (4, 4, 77, 10), (16, 2, 33, 100),
                                           (8, 1, 512, 0), (8, 2, 8192, 30), (8, 2, 40961, 1), (4, 1, 32768, 2),
                                           (4, 1, 70001, 1), (8, 8, 65536, 1), (64, 8, 16384, 1), (16, 8, 300, 5),
-                                          (8, 2, 32768, 1), (32, 8, 1, 100)])
+                                          (8, 2, 32768, 1), (32, 8, 1, 100), (8, 1, 20000, 2),
+                                          (16, 2, 40000, 100)])
 def test_attn_small(sf, attn_path, Hq, Hkv, T, pct):
     """Both implementations against the oracle: the pipeline's compaction,
-    finish and output kernels at every size, the cluster kernel up to its
-    limit (including clusters with empty CTAs at tiny T, eight query heads
-    per KV head, k = T and k = 0), the pairwise ranking of few candidates and
-    the radix ranking of many (30% of 8192)."""
+    finish, refine and output kernels at every size, the cluster kernel up
+    to its limit (including clusters with empty CTAs at tiny T, eight query
+    heads per KV head, k = T and k = 0), the pairwise ranking of few
+    candidates and the radix ranking of many (30% of 8192); eight query
+    heads per KV head beyond the cluster kernel's limit, and k = T at 40K
+    (every token refined by the refine kernel)."""
     _skip_unless_applies(attn_path, Hq, Hkv, T)
     d = 128
     kv, ok, ov = _kv(sf, Hkv, T, d, 3000 + T)
