@@ -310,7 +310,7 @@ sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, const uint16
 /* Quantized K and V (views).  Rows are token-heads ordered [Hkv][T], each
  * quantized as one group of d values with sf_quantize_nested(layout
  * SF_REF_BY_ROW): *_res [Hkv*T][d*b_r/32], *_ref [Hkv*T][d*b_f/32],
- * *_scale/*_zero fp16 [Hkv*T]. */
+ * *_scale, *_zero fp16 [Hkv*T]. */
 typedef struct sf_qkv {
   const uint32_t *k_res, *k_ref, *v_res, *v_ref;
   const uint16_t *k_scale, *k_zero, *v_scale, *v_zero;

@@ -793,7 +793,6 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
   uint16_t* ulist = reinterpret_cast<uint16_t*>(smem + C::alpha_bytes + C::ring_bytes);  // [kSub]
   uint32_t* vrs = reinterpret_cast<uint32_t*>(smem + C::alpha_bytes + C::ring_bytes +
                                               C::ulist_bytes);  // [kUCap][8] refinement rows of listed tokens
-  __shared__ float red[kOW][GRP];
   __shared__ float red2[kOW][3 * GRP];
   __shared__ float Msh[GRP];
   __shared__ int ucount;

@@ -1352,7 +1352,7 @@ bool fused_fits(const FusedPlan<GRP>& p) {
 }
 
 template <int GRP>
-sf_status fused_run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k, int32_t* sel_out,
+sf_status fused_run(const uint16_t* q, int Hkv, int T, const sf_qkv* kv, int k, int32_t* sel_out,
                     int32_t* sel_n, float* out, double* ovf_key, int32_t* ovf_tok, int32_t* ovf_sel, float* gpart,
                     int32_t* gcnt, cudaStream_t s) {
   FusedPlan<GRP> p;
@@ -1403,10 +1403,10 @@ sf_status attn_fused_run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv
                          int32_t* sel_n, float* out, double* ovf_key, int32_t* ovf_tok, int32_t* ovf_sel,
                          float* gpart, int32_t* gcnt, cudaStream_t s) {
   switch (Hq / Hkv) {
-    case 1: return fused_run<1>(q, Hq, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, gpart, gcnt, s);
-    case 2: return fused_run<2>(q, Hq, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, gpart, gcnt, s);
-    case 4: return fused_run<4>(q, Hq, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, gpart, gcnt, s);
-    case 8: return fused_run<8>(q, Hq, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, gpart, gcnt, s);
+    case 1: return fused_run<1>(q, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, gpart, gcnt, s);
+    case 2: return fused_run<2>(q, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, gpart, gcnt, s);
+    case 4: return fused_run<4>(q, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, gpart, gcnt, s);
+    case 8: return fused_run<8>(q, Hkv, T, kv, k, sel_out, sel_n, out, ovf_key, ovf_tok, ovf_sel, gpart, gcnt, s);
     default: return sf::fail(SF_ENOTIMPL, "attn_fused_run: Hq/Hkv must be 1, 2, 4 or 8");
   }
 }

@@ -133,7 +133,6 @@ struct MCfg {
   static constexpr int SW = SPW * kSliceWords;  // ring words per warp and stage
   static size_t smem_bytes(int W) {
     return sizeof(uint32_t) * (static_cast<size_t>(W) * kStages * SW           // rings
-                               + static_cast<size_t>(W) * SPW * kCorrList       // refinement rows (issue job)
                                + static_cast<size_t>(W) * SPW * kCorrList / 2   // listed channels (u16)
                                + static_cast<size_t>(kRedTiles) * W * kRows);   // row partials of the warps
   }
@@ -149,10 +148,8 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, tig = lane & 3;
   const int ks = blockIdx.x % a.ksplit, crow = blockIdx.x / a.ksplit, ncta = gridDim.x / a.ksplit;
   uint32_t* ring = sm + warp * kStages * SW;
-  int* selr = reinterpret_cast<int*>(sm + W * kStages * SW) + warp * SPW * kCorrList;           // [SPW][32]
-  uint16_t* mylist = reinterpret_cast<uint16_t*>(sm + W * kStages * SW + W * SPW * kCorrList) +
-                     warp * SPW * kCorrList;                                                      // [SPW][32]
-  float* red = reinterpret_cast<float*>(sm + W * kStages * SW + W * SPW * kCorrList + W * SPW * kCorrList / 2);
+  uint16_t* mylist = reinterpret_cast<uint16_t*>(sm + W * kStages * SW) + warp * SPW * kCorrList;  // [SPW][32]
+  float* red = reinterpret_cast<float*>(sm + W * kStages * SW + W * SPW * kCorrList / 2);
 
   const int slice0 = (ks * W + warp) * SPW;
   const int myslot = tig >> 1, myrow = g8 + 8 * (tig & 1);
