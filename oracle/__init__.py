@@ -37,6 +37,8 @@ select  top-k channel selection by |x|, union over the batch   (pinned)
 cache   LRU refinement cache: hits, misses, bypass, slots       (pinned)
 gemv    refined decode GEMV                                     (pinned)
 attn    refined decode attention (token selection + recompute)  (pinned)
+decode  one full decode step of a Llama-shaped model: RMSNorm, RoPE,
+        KV append, refined GEMVs and attention, SiLU MLP, LM head (pinned)
 """
 
 from . import quant, select, cache, gemv, attn  # noqa: F401
