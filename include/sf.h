@@ -395,6 +395,43 @@ sf_status sf_attn_decode_refine_noalloc(const uint16_t* q, int Hq, int Hkv, int 
 typedef enum sf_attn_path { SF_ATTN_AUTO = 0, SF_ATTN_CLUSTER = 1, SF_ATTN_PIPELINE = 2 } sf_attn_path;
 sf_status sf_attn_set_path(int path);
 
+/* ---- decode-step elementwise operations -------------------------------- */
+
+/*
+ * The elementwise steps of one decode step of a Llama-shaped layer.  Source:
+ * the benchmark configuration of the pages' end-to-end measurement names the
+ * model shape (Llama-3.1-8B: RMSNorm, RoPE, SiLU-gated MLP); the formulas are
+ * the library's reading (eps from the caller, RoPE rotate-half pairing with
+ * base theta, no frequency rescaling), identical to the oracle's.  Values are
+ * computed in fp64 and rounded once: to fp32 for fp32 outputs, to bf16 with
+ * ties to even for bf16 outputs.  All pointers are device memory owned by the
+ * caller; every call is asynchronous on `stream`.
+ *
+ * sf_add_rmsnorm -- residual add and RMSNorm, per row b of x [B][H] fp32:
+ *   when delta (fp32 [B][H]) is not NULL, x += delta first (fp32 addition,
+ *   written back); then y[b][i] = bf16(x[b][i] / sqrt(mean_i x^2 + eps) *
+ *   w[i]), w fp32 [H], y bf16 [B][H].
+ *   Constraints: B >= 1, H >= 1, eps >= 0.  SF_EINVAL otherwise.
+ */
+sf_status sf_add_rmsnorm(float* x, const float* delta, const float* w, int B, int H, float eps, uint16_t* y,
+                         sf_stream_t stream);
+
+/*
+ * sf_rope -- rotates every head of x [H][d] fp32 (in place) to position pos:
+ *   for i < d/2 the pair (x_i, x_{i+d/2}) turns by the angle
+ *   pos * theta^(-2i/d).  When y_bf16 (bf16 [H][d]) is not NULL the rotated
+ *   values are also written there as bf16.
+ *   Constraints: H >= 1, d even in [2, 2048], pos >= 0, theta > 0.
+ */
+sf_status sf_rope(float* x, int H, int d, int pos, double theta, uint16_t* y_bf16, sf_stream_t stream);
+
+/*
+ * sf_silu_mul -- the SiLU-gated product of the MLP:
+ *   y[i] = bf16(g[i] / (1 + exp(-g[i])) * u[i]) for i < n; g, u fp32 [n],
+ *   y bf16 [n].  Constraints: n >= 1.
+ */
+sf_status sf_silu_mul(const float* g, const float* u, int n, uint16_t* y, sf_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

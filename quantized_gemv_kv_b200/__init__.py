@@ -96,6 +96,9 @@ _SIGS = {
     "sf_attn_decode_refine": ([_p, _i, _i, _i, _i, ctypes.POINTER(_QKV), _i, _p, _p, _p, _p, _sz, _p], _i),
     "sf_attn_decode_refine_noalloc": ([_p, _i, _i, _i, _i, ctypes.POINTER(_QKV), _i, _p, _p, _p, _p], _i),
     "sf_attn_set_path": ([_i], _i),
+    "sf_add_rmsnorm": ([_p, _p, _p, _i, _i, ctypes.c_float, _p, _p], _i),
+    "sf_rope": ([_p, _i, _i, _i, ctypes.c_double, _p, _p], _i),
+    "sf_silu_mul": ([_p, _p, _i, _p, _p], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -448,3 +451,45 @@ class SelectJobs:
 
     def run(self, stream: torch.cuda.Stream | None = None) -> None:
         _check(_lib.sf_select_topk_act_many(ctypes.cast(self._arr, _p), self.count, _stream(stream)))
+
+
+# ---- decode-step elementwise operations ----------------------------------------
+
+def add_rmsnorm(x: torch.Tensor, w: torch.Tensor, eps: float = 1e-5, delta: torch.Tensor | None = None,
+                y: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """``sf_add_rmsnorm``: x (fp32 [B][H], updated in place by x += delta
+    when delta is given), w fp32 [H]; returns y bf16 [B][H]."""
+    _dev(x, "x")
+    if x.dtype != torch.float32 or w.dtype != torch.float32 or (delta is not None and delta.dtype != torch.float32):
+        raise ValueError("x, w and delta must be float32")
+    x2 = x if x.dim() == 2 else x.view(1, -1)
+    B, H = x2.shape
+    if y is None:
+        y = torch.empty((B, H), dtype=torch.bfloat16, device=x.device)
+    _check(_lib.sf_add_rmsnorm(_ptr(x2), _ptr(delta), _ptr(w), B, H, eps, _ptr(y), _stream(stream)))
+    return y
+
+
+def rope(x: torch.Tensor, pos: int, theta: float = 500000.0, y: torch.Tensor | None = None,
+         stream: torch.cuda.Stream | None = None) -> torch.Tensor | None:
+    """``sf_rope``: rotates the heads of x (fp32 [H][d], in place) to
+    position pos; when y (bf16 [H][d]) is given the result is also written
+    there as bf16.  Returns y."""
+    _dev(x, "x")
+    if x.dtype != torch.float32 or x.dim() != 2:
+        raise ValueError("x must be a 2-D float32 tensor")
+    H, d = x.shape
+    _check(_lib.sf_rope(_ptr(x), H, d, pos, theta, _ptr(y), _stream(stream)))
+    return y
+
+
+def silu_mul(g: torch.Tensor, u: torch.Tensor, y: torch.Tensor | None = None,
+             stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """``sf_silu_mul``: bf16(silu(g) * u) elementwise over fp32 g, u."""
+    _dev(g, "g")
+    if g.dtype != torch.float32 or u.dtype != torch.float32 or g.numel() != u.numel():
+        raise ValueError("g and u must be float32 tensors of the same size")
+    if y is None:
+        y = torch.empty(g.shape, dtype=torch.bfloat16, device=g.device)
+    _check(_lib.sf_silu_mul(_ptr(g), _ptr(u), g.numel(), _ptr(y), _stream(stream)))
+    return y
