@@ -432,6 +432,22 @@ sf_status sf_rope(float* x, int H, int d, int pos, double theta, uint16_t* y_bf1
  */
 sf_status sf_silu_mul(const float* g, const float* u, int n, uint16_t* y, sf_stream_t stream);
 
+/*
+ * sf_kv_append -- quantizes the new token's rows of K or V and writes them as
+ *   token t of every KV head of a cache allocated for row_stride tokens per
+ *   head: src fp32 [Hkv][d] (row g = KV head g) becomes cache row
+ *   g * row_stride + t, quantized exactly as sf_quantize_nested does with one
+ *   group of d values per row and SF_REF_BY_ROW (the KV quantization of the
+ *   pages' 2+2-bit KV: nested refinement, rag-lover.com explainer, 解説).
+ *   Cache arrays (caller-owned, rows = Hkv * row_stride): res uint32
+ *   [rows][d*b_r/32], ref uint32 [rows][d*b_f/32], scale and zero fp16
+ *   [rows].  Only the Hkv rows of token t are written.
+ *   Constraints: Hkv >= 1, d a multiple of 32 in [32, 512], 0 <= t <
+ *   row_stride, b_r in {2,3}, b_f in {1,2}, b_r + b_f <= 4.  src finite.
+ */
+sf_status sf_kv_append(const float* src, int Hkv, int d, int row_stride, int t, int b_r, int b_f, uint32_t* res,
+                       uint32_t* ref, uint16_t* scale, uint16_t* zero, sf_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

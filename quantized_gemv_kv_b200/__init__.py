@@ -99,6 +99,7 @@ _SIGS = {
     "sf_add_rmsnorm": ([_p, _p, _p, _i, _i, ctypes.c_float, _p, _p], _i),
     "sf_rope": ([_p, _i, _i, _i, ctypes.c_double, _p, _p], _i),
     "sf_silu_mul": ([_p, _p, _i, _p, _p], _i),
+    "sf_kv_append": ([_p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -493,3 +494,17 @@ def silu_mul(g: torch.Tensor, u: torch.Tensor, y: torch.Tensor | None = None,
         y = torch.empty(g.shape, dtype=torch.bfloat16, device=g.device)
     _check(_lib.sf_silu_mul(_ptr(g), _ptr(u), g.numel(), _ptr(y), _stream(stream)))
     return y
+
+
+def kv_append(src: torch.Tensor, res: torch.Tensor, ref: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
+              row_stride: int, t: int, b_r: int = 2, b_f: int = 2, stream: torch.cuda.Stream | None = None) -> None:
+    """``sf_kv_append``: quantizes src (fp32 [Hkv][d]) and writes it as token
+    t of every KV head of the cache (res, ref, scale, zero with rows
+    [Hkv][row_stride])."""
+    _dev(src, "src")
+    if src.dtype != torch.float32 or src.dim() != 2:
+        raise ValueError("src must be a 2-D float32 tensor")
+    Hkv, d = src.shape
+    _check(_lib.sf_kv_append(_ptr(src), Hkv, d, row_stride, t, b_r, b_f, _ptr(res), _ptr(ref), _ptr(scale),
+                             _ptr(zero), _stream(stream)))
+

@@ -1,6 +1,7 @@
-// Elementwise operations of a decode step of a Llama-shaped layer: residual
-// add with RMSNorm, RoPE of the new token's query and key heads, and the
-// SiLU-gated product of the MLP.  The benchmark configuration names the
+// Per-token operations of a decode step of a Llama-shaped layer: residual
+// add with RMSNorm, RoPE of the new token's query and key heads, the
+// SiLU-gated product of the MLP, and the quantize-and-append of the new
+// token's K or V rows into a cache allocated for a larger capacity.  The benchmark configuration names the
 // shape (Llama-3.1-8B: RMSNorm, RoPE, SiLU MLP); the readings are the
 // library's: eps given by the caller, RoPE in the rotate-half pairing with
 // base theta and no frequency rescaling.  Each value is computed in fp64 and
@@ -8,6 +9,7 @@
 // the GEMV and attention inputs), so the results sit within one rounding of
 // the exact values.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "sf_internal.h"
 
@@ -78,6 +80,75 @@ __global__ void silu_mul_kernel(const float* __restrict__ g, const float* __rest
   }
 }
 
+constexpr int kAppendMaxD = 512;
+
+// One warp per KV head: the new token's row of d values is quantized as one
+// group with the arithmetic of the nested quantizer (min/max, fp32 division,
+// fp16 scale, integer zero point, ties to even) and written as cache row
+// g * row_stride + t: resident and refinement bitstreams (row-major, little
+// endian), fp16 scale and zero.
+__global__ void kv_append_kernel(const float* __restrict__ src, int Hkv, int d, int row_stride, int t, int b_r,
+                                 int b_f, uint32_t* __restrict__ res, uint32_t* __restrict__ ref,
+                                 uint16_t* __restrict__ scale, uint16_t* __restrict__ zero) {
+  __shared__ uint8_t codes[4][kAppendMaxD];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = blockIdx.x * 4 + warp;
+  if (g >= Hkv) return;  // uniform over the warp
+  const int b = b_r + b_f;
+  const float qmax = static_cast<float>((1 << b) - 1);
+  const int per_lane = d >> 5;
+  const float* row = src + static_cast<size_t>(g) * d;
+  float v[kAppendMaxD / 32];
+  float lo = INFINITY, hi = -INFINITY;
+  for (int m = 0; m < per_lane; ++m) {
+    v[m] = row[lane + 32 * m];
+    lo = fminf(lo, v[m]);
+    hi = fmaxf(hi, v[m]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  float q32 = __fdiv_rn(__fsub_rn(hi, lo), qmax);
+  q32 = fminf(q32, 65504.0f);
+  __half s16 = __float2half_rn(q32);
+  if (__half2float(s16) == 0.0f) s16 = __float2half_rn(1.0f);
+  const float sf = __half2float(s16);
+  float zf = rintf(__fdiv_rn(-lo, sf));
+  zf = fminf(fmaxf(zf, 0.0f), qmax);
+  const int zi = static_cast<int>(zf);
+  const size_t r = static_cast<size_t>(g) * row_stride + t;
+  if (lane == 0) {
+    scale[r] = __half_as_ushort(s16);
+    zero[r] = __half_as_ushort(__int2half_rn(zi));
+  }
+  for (int m = 0; m < per_lane; ++m) {
+    float qf = rintf(__fdiv_rn(v[m], sf)) + static_cast<float>(zi);
+    qf = fminf(fmaxf(qf, 0.0f), qmax);
+    codes[warp][lane + 32 * m] = static_cast<uint8_t>(static_cast<int>(qf));
+  }
+  __syncwarp();
+  const uint32_t rmask = (1u << b_r) - 1u, fmask = (1u << b_f) - 1u;
+  const int rw = d * b_r / 32, fw = d * b_f / 32;
+  for (int ww = lane; ww < rw; ww += 32) {
+    uint32_t word = 0;
+    for (int bit = 0; bit < 32; ++bit) {
+      const int sb = ww * 32 + bit;
+      word |= (((static_cast<uint32_t>(codes[warp][sb / b_r]) >> b_f) & rmask) >> (sb % b_r) & 1u) << bit;
+    }
+    res[r * rw + ww] = word;
+  }
+  for (int ww = lane; ww < fw; ww += 32) {
+    uint32_t word = 0;
+    for (int bit = 0; bit < 32; ++bit) {
+      const int sb = ww * 32 + bit;
+      word |= ((static_cast<uint32_t>(codes[warp][sb / b_f]) & fmask) >> (sb % b_f) & 1u) << bit;
+    }
+    ref[r * fw + ww] = word;
+  }
+}
+
 }  // namespace
 
 extern "C" sf_status sf_add_rmsnorm(float* x, const float* delta, const float* w, int B, int H, float eps,
@@ -104,3 +175,19 @@ extern "C" sf_status sf_silu_mul(const float* g, const float* u, int n, uint16_t
   silu_mul_kernel<<<blocks, 256, 0, sf::as_cuda(stream)>>>(g, u, n, y);
   return sf::check_launch("silu_mul_kernel");
 }
+
+extern "C" sf_status sf_kv_append(const float* src, int Hkv, int d, int row_stride, int t, int b_r, int b_f,
+                                  uint32_t* res, uint32_t* ref, uint16_t* scale, uint16_t* zero, sf_stream_t stream) {
+  SF_REQUIRE(src && res && ref && scale && zero, "sf_kv_append: null pointer");
+  SF_REQUIRE(Hkv >= 1, "sf_kv_append: Hkv must be >= 1");
+  SF_REQUIRE(d >= 32 && d % 32 == 0 && d <= kAppendMaxD, "sf_kv_append: d must be a multiple of 32 in [32, %d]",
+             kAppendMaxD);
+  SF_REQUIRE(b_r == 2 || b_r == 3, "sf_kv_append: b_r must be 2 or 3");
+  SF_REQUIRE(b_f == 1 || b_f == 2, "sf_kv_append: b_f must be 1 or 2");
+  SF_REQUIRE(b_r + b_f <= 4, "sf_kv_append: b_r + b_f must be <= 4");
+  SF_REQUIRE(row_stride >= 1 && t >= 0 && t < row_stride, "sf_kv_append: need 0 <= t < row_stride");
+  kv_append_kernel<<<(Hkv + 3) / 4, 128, 0, sf::as_cuda(stream)>>>(src, Hkv, d, row_stride, t, b_r, b_f, res, ref,
+                                                                   scale, zero);
+  return sf::check_launch("kv_append_kernel");
+}
+

@@ -85,6 +85,37 @@ def test_silu_mul(sf, n):
     _close_bf16(_bits(y), ref)
 
 
+@pytest.mark.parametrize("Hkv,d,cap,t,b_r,b_f", [(8, 128, 64, 17, 2, 2), (8, 128, 64, 0, 2, 2),
+                                                (8, 128, 64, 63, 2, 2), (3, 96, 5, 4, 3, 1), (1, 512, 2, 1, 2, 1)])
+def test_kv_append_bit_exact(sf, Hkv, d, cap, t, b_r, b_f):
+    """Token t of every head equals the oracle's packed quantization of the
+    new rows; every other cache row keeps its sentinel."""
+    from oracle import quant as oquant
+    rng = np.random.default_rng(1000 + d + t)
+    src = (rng.standard_normal((Hkv, d)) * 2).astype(np.float32)
+    rows = Hkv * cap
+    res = torch.full((rows, d * b_r // 32), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
+    ref = torch.full((rows, d * b_f // 32), 0x3C3C3C3C, dtype=torch.int32, device="cuda")
+    scale = torch.full((rows,), 7.0, dtype=torch.float16, device="cuda")
+    zero = torch.full((rows,), 9.0, dtype=torch.float16, device="cuda")
+    sf.kv_append(torch.from_numpy(src).cuda(), res, ref, scale, zero, cap, t, b_r, b_f)
+    torch.cuda.synchronize()
+    want = oquant.pack_nested(oquant.quantize_nested(src, d, b_r, b_f), "by_row")
+    res_np = res.cpu().numpy().view(np.uint32).reshape(Hkv, cap, -1)
+    ref_np = ref.cpu().numpy().view(np.uint32).reshape(Hkv, cap, -1)
+    sc_np = scale.cpu().numpy().view(np.uint16).reshape(Hkv, cap)
+    z_np = zero.cpu().numpy().view(np.uint16).reshape(Hkv, cap)
+    np.testing.assert_array_equal(res_np[:, t], want["res"])
+    np.testing.assert_array_equal(ref_np[:, t], want["ref"])
+    np.testing.assert_array_equal(sc_np[:, t], want["scale"][0].view(np.uint16))
+    np.testing.assert_array_equal(z_np[:, t], want["zero"][0].view(np.uint16))
+    keep = np.ones(cap, bool)
+    keep[t] = False
+    assert np.all(res_np[:, keep] == 0x5A5A5A5A) and np.all(ref_np[:, keep] == 0x3C3C3C3C)
+    assert np.all(sc_np[:, keep] == np.float16(7.0).view(np.uint16)) and \
+        np.all(z_np[:, keep] == np.float16(9.0).view(np.uint16))
+
+
 def test_decode_ops_reject_bad_sizes(sf):
     x = torch.zeros((2, 7), dtype=torch.float32, device="cuda")
     with pytest.raises(sf.SfError):
