@@ -307,14 +307,18 @@ sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, const uint16
 
 /* ---- refined decode attention ----------------------------------------- */
 
-/* Quantized K and V (views).  Rows are token-heads ordered [Hkv][T], each
- * quantized as one group of d values with sf_quantize_nested(layout
- * SF_REF_BY_ROW): *_res [Hkv*T][d*b_r/32], *_ref [Hkv*T][d*b_f/32],
- * *_scale, *_zero fp16 [Hkv*T]. */
+/* Quantized K and V (views).  Rows are token-heads ordered [Hkv][S], token t
+ * of KV head g at row g*S + t, each quantized as one group of d values with
+ * sf_quantize_nested(layout SF_REF_BY_ROW) or sf_kv_append:
+ * *_res [Hkv*S][d*b_r/32], *_ref [Hkv*S][d*b_f/32], *_scale, *_zero fp16
+ * [Hkv*S].  S = row_stride when it is positive (a cache allocated for S
+ * tokens per head, of which the first T are read), else S = T; a positive
+ * row_stride below T is SF_EINVAL. */
 typedef struct sf_qkv {
   const uint32_t *k_res, *k_ref, *v_res, *v_ref;
   const uint16_t *k_scale, *k_zero, *v_scale, *v_zero;
   int b_r, b_f;
+  int row_stride;
 } sf_qkv;
 
 /* Workspace bytes sf_attn_decode_refine needs for these sizes. */

@@ -52,7 +52,7 @@ class _QWeight(ctypes.Structure):
 class _QKV(ctypes.Structure):
     _fields_ = [("k_res", _p), ("k_ref", _p), ("v_res", _p), ("v_ref", _p),
                 ("k_scale", _p), ("k_zero", _p), ("v_scale", _p), ("v_zero", _p),
-                ("b_r", _i), ("b_f", _i)]
+                ("b_r", _i), ("b_f", _i), ("row_stride", _i)]
 
 
 class _GemvJob(ctypes.Structure):
@@ -321,14 +321,17 @@ def gemv_refine(W: QWeight, x: torch.Tensor, idx: torch.Tensor | None = None, n:
 
 @dataclass
 class QKV:
-    """Quantized K and V, rows = token-heads [Hkv][T] (layout by_row, G = d)."""
+    """Quantized K and V, rows = token-heads [Hkv][S] (layout by_row, G = d):
+    S = row_stride when it is positive (a cache allocated for row_stride
+    tokens per head), else the call's T."""
     k: QWeight
     v: QWeight
+    row_stride: int = 0
 
     def c_struct(self) -> _QKV:
         return _QKV(_ptr(self.k.res), _ptr(self.k.ref), _ptr(self.v.res), _ptr(self.v.ref),
                     _ptr(self.k.scale), _ptr(self.k.zero), _ptr(self.v.scale), _ptr(self.v.zero),
-                    self.k.b_r, self.k.b_f)
+                    self.k.b_r, self.k.b_f, self.row_stride)
 
 
 ATTN_AUTO, ATTN_CLUSTER, ATTN_PIPELINE = 0, 1, 2

@@ -87,7 +87,7 @@ __host__ __device__ constexpr size_t score_smem(int grp) {
 template <int GRP>
 __global__ void __launch_bounds__(kScThreads, 2)
 attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
-                      const uint16_t* __restrict__ k_scale, const uint16_t* __restrict__ k_zero, int T, int tpc,
+                      const uint16_t* __restrict__ k_scale, const uint16_t* __restrict__ k_zero, int T, int S, int tpc,
                       float* __restrict__ score, float* __restrict__ smax, int32_t* __restrict__ hist,
                       uint32_t* __restrict__ amaxu, uint32_t* __restrict__ mkey) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -104,7 +104,7 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
   const int ntile = (n + 15) >> 4;
   const int tpw = (ntile + kScW - 1) / kScW;
   const int tile0 = min(ntile, warp * tpw), tile1 = min(ntile, tile0 + tpw);
-  const size_t row0 = static_cast<size_t>(g) * T + t0;
+  const size_t row0 = static_cast<size_t>(g) * S + t0;  // K rows: the cache's stride
   auto issue = [&](int ti) {
     const int st = (ti - tile0) % kScRing;
     const int row = 16 * ti + (lane >> 1);
@@ -387,7 +387,7 @@ template <int GRP>
 __global__ void __launch_bounds__(kFinThreads)
 attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
                           const uint32_t* __restrict__ k_ref, const uint16_t* __restrict__ k_scale,
-                          const uint16_t* __restrict__ k_zero, int T, int k, float* __restrict__ score,
+                          const uint16_t* __restrict__ k_zero, int T, int k, int S, float* __restrict__ score,
                           const float* __restrict__ smax, const int32_t* __restrict__ hist,
                           const uint32_t* __restrict__ amaxu, const int32_t* __restrict__ cand,
                           const int32_t* __restrict__ ccnt, int32_t* __restrict__ list, double* __restrict__ kap,
@@ -535,7 +535,7 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   //    order does not change the key)
   for (int i = tid; i < ncand; i += kFinThreads) {
     const int t = F[i];
-    const size_t row = static_cast<size_t>(g) * T + t;
+    const size_t row = static_cast<size_t>(g) * S + t;
     const uint4* w4 = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
     const uint4 x0 = w4[0], x1 = w4[1];
     const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
@@ -679,7 +679,7 @@ template <int GRP>
 __global__ void __launch_bounds__(kRefThreads, 2)
 attn_refine_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
                    const uint32_t* __restrict__ k_ref, const uint16_t* __restrict__ k_scale,
-                   const uint16_t* __restrict__ k_zero, int T, int cap, const int32_t* __restrict__ sel_out,
+                   const uint16_t* __restrict__ k_zero, int T, int S, int cap, const int32_t* __restrict__ sel_out,
                    const int32_t* __restrict__ sel_n, float* __restrict__ score, uint32_t* __restrict__ rkey) {
   __shared__ float qs[GRP][D];
   __shared__ float qsum[GRP];
@@ -689,7 +689,7 @@ attn_refine_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ 
   const int sn = sel_n[g];
   const int U = min(cap, sn >= 0 ? sn : -1 - sn);
   const int32_t* list = sel_out + static_cast<size_t>(g) * cap;
-  const size_t rowg = static_cast<size_t>(g) * T;
+  const size_t rowg = static_cast<size_t>(g) * S;  // K rows: the cache's stride
   uint32_t mk[GRP];
 #pragma unroll
   for (int h = 0; h < GRP; ++h) mk[h] = 0u;
@@ -781,7 +781,7 @@ template <int GRP>
 __global__ void __launch_bounds__(kOutThreads)
 attn_out_kernel(const uint32_t* __restrict__ v_res,
                 const uint32_t* __restrict__ v_ref, const uint16_t* __restrict__ v_scale,
-                const uint16_t* __restrict__ v_zero, int T, int tps, int words_t, int splits,
+                const uint16_t* __restrict__ v_zero, int T, int S, int tps, int words_t, int splits,
                 const float* __restrict__ score, const uint32_t* __restrict__ mkey, const uint32_t* __restrict__ rkey,
                 const uint32_t* __restrict__ umask, float* __restrict__ part, int32_t* __restrict__ done,
                 float* __restrict__ out) {
@@ -801,7 +801,7 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
   const int g = blockIdx.y, split = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, tig = lane & 3;
   const int t0s = split * tps, t1s = min(T, t0s + tps);
-  const size_t rowg = static_cast<size_t>(g) * T;
+  const size_t rowg = static_cast<size_t>(g) * S;  // V rows: the cache's stride
 
   for (int e = tid; e < (NT * 8 - C::NC) * kStr; e += kOutThreads) as[C::NC * kStr + e] = __float2half_rn(0.0f);
   // one maximum per head for every token: the larger of the bound on the
@@ -1104,6 +1104,7 @@ __global__ void fill_all_kernel(int T, int grp, int k, int words_t, uint32_t* um
 template <int GRP>
 sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k, int32_t* sel_out, int32_t* sel_n,
               float* out, char* ws, const Layout& L, cudaStream_t s) {
+  const int S = kv->row_stride > 0 ? kv->row_stride : T;  // rows per KV head in the K/V arrays
   float* score = reinterpret_cast<float*>(ws + L.score);
   int32_t* cand = reinterpret_cast<int32_t*>(ws + L.cand);
   int32_t* cand2 = reinterpret_cast<int32_t*>(ws + L.cand2);
@@ -1128,8 +1129,8 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
   uint32_t* rkey = reinterpret_cast<uint32_t*>(ws + L.rkey);
   SF_CHECK_CUDA(cudaFuncSetAttribute(attn_score_mma_kernel<GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(score_smem(GRP))));
-  attn_score_mma_kernel<GRP><<<ga, kScThreads, score_smem(GRP), s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, tpc,
-                                                                     score, smax, hist, amaxu, mkey);
+  attn_score_mma_kernel<GRP><<<ga, kScThreads, score_smem(GRP), s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, S,
+                                                                     tpc, score, smax, hist, amaxu, mkey);
   sf_status st = sf::check_launch("attn_score_mma_kernel");
   if (st != SF_OK) return st;
   if (k > 0 && k < T) {
@@ -1153,7 +1154,7 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, attn_select_finish_kernel<GRP>, q, kv->k_res, kv->k_ref, kv->k_scale,
-                                     kv->k_zero, T, k, score, static_cast<const float*>(smax),
+                                     kv->k_zero, T, k, S, score, static_cast<const float*>(smax),
                                      static_cast<const int32_t*>(hist), static_cast<const uint32_t*>(amaxu), cand,
                                      static_cast<const int32_t*>(ccnt), cand2, kap, sel_head, umask, L.words_t,
                                      sel_out, sel_n, status, mkey));
@@ -1170,7 +1171,7 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
     const int cap = grp * k;
     const int nblk = std::max(1, std::min((cap + kRefThreads - 1) / kRefThreads, 2 * sms / Hkv));
     attn_refine_kernel<GRP><<<dim3(nblk, Hkv), kRefThreads, 0, s>>>(q, kv->k_res, kv->k_ref, kv->k_scale, kv->k_zero,
-                                                                   T, cap, sel_out, sel_n, score, rkey);
+                                                                   T, S, cap, sel_out, sel_n, score, rkey);
     st = sf::check_launch("attn_refine_kernel");
     if (st != SF_OK) return st;
   }
@@ -1178,7 +1179,7 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
   SF_CHECK_CUDA(cudaFuncSetAttribute(attn_out_kernel<GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(OutCfg<GRP>::smem)));
   attn_out_kernel<GRP><<<gb, kOutThreads, OutCfg<GRP>::smem, s>>>(kv->v_res, kv->v_ref, kv->v_scale, kv->v_zero, T,
-                                                                 L.tps, L.words_t, L.splits, score, mkey, rkey,
+                                                                 S, L.tps, L.words_t, L.splits, score, mkey, rkey,
                                                                  umask, part, done, out);
   return sf::check_launch("attn_out_kernel");
 }
@@ -1236,6 +1237,7 @@ extern "C" sf_status sf_attn_decode_refine(const uint16_t* q, int Hq, int Hkv, i
   SF_REQUIRE(Hkv >= 1 && Hq >= Hkv && Hq % Hkv == 0, "sf_attn_decode_refine: Hq must be a multiple of Hkv");
   SF_REQUIRE(T >= 1 && T <= (1 << 24), "sf_attn_decode_refine: T out of range");
   SF_REQUIRE(k_tokens >= 0 && k_tokens <= T, "sf_attn_decode_refine: k_tokens must be in [0, T]");
+  SF_REQUIRE(kv->row_stride == 0 || kv->row_stride >= T, "sf_attn_decode_refine: row_stride must be 0 or >= T");
   SF_REQUIRE(sf::aligned(kv->k_res, 16) && sf::aligned(kv->v_res, 16) && sf::aligned(kv->k_ref, 16) &&
                  sf::aligned(kv->v_ref, 16),
              "sf_attn_decode_refine: code arrays must be 16-byte aligned");
@@ -1303,6 +1305,7 @@ extern "C" sf_status sf_attn_decode_refine_noalloc(const uint16_t* q, int Hq, in
   SF_REQUIRE(Hkv >= 1 && Hq >= Hkv && Hq % Hkv == 0, "sf_attn_decode_refine_noalloc: Hq must be a multiple of Hkv");
   SF_REQUIRE(T >= 1 && T <= (1 << 24), "sf_attn_decode_refine_noalloc: T out of range");
   SF_REQUIRE(k_tokens >= 0 && k_tokens <= T, "sf_attn_decode_refine_noalloc: k_tokens must be in [0, T]");
+  SF_REQUIRE(kv->row_stride == 0 || kv->row_stride >= T, "sf_attn_decode_refine_noalloc: row_stride must be 0 or >= T");
   SF_REQUIRE(sf::aligned(kv->k_res, 16) && sf::aligned(kv->v_res, 16) && sf::aligned(kv->k_ref, 16) &&
                  sf::aligned(kv->v_ref, 16),
              "sf_attn_decode_refine_noalloc: code arrays must be 16-byte aligned");

@@ -118,6 +118,7 @@ struct FusedArgs {
   const uint16_t* v_scale;
   const uint16_t* v_zero;
   int T, k, R;
+  int S;              // rows per KV head in the K/V arrays (the cache's stride)
   int32_t* sel_out;
   int32_t* sel_n;
   float* out;
@@ -376,7 +377,7 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
   const int t0 = r * R;
   const int n = max(0, min(R, T - t0));  // tokens of this CTA: [t0, t0 + n)
   const int ntile = (n + 15) >> 4;
-  const size_t row0 = static_cast<size_t>(g) * T + t0;
+  const size_t row0 = static_cast<size_t>(g) * a.S + t0;
   const int kStr = R + 8;  // halves per weight row: conflict-free fragment loads
   const FusedSmem S = fused_smem(GRP, R);
   extern __shared__ __align__(16) unsigned char smem[];
@@ -1370,6 +1371,7 @@ sf_status fused_run(const uint16_t* q, int Hkv, int T, const sf_qkv* kv, int k, 
   a.T = T;
   a.k = k;
   a.R = p.R;
+  a.S = kv->row_stride > 0 ? kv->row_stride : T;
   a.sel_out = sel_out;
   a.sel_n = sel_n;
   a.out = out;
