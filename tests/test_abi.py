@@ -84,3 +84,27 @@ def test_attn_path_switch(sf):
     assert L.sf_attn_set_path(-1) == sf.SF_EINVAL
     for p in (sf.ATTN_PIPELINE, sf.ATTN_CLUSTER, sf.ATTN_AUTO):
         assert L.sf_attn_set_path(p) == sf.SF_OK
+
+
+def test_host_validation_decode_step_ops(sf):
+    """The decode-step entry points and the K/V row stride reject bad sizes
+    on the host, before any device work."""
+    L = sf._lib
+    p = ctypes.c_void_p(256)
+    assert L.sf_add_rmsnorm(p, None, p, 0, 4096, ctypes.c_float(1e-5), p, None) == sf.SF_EINVAL
+    assert L.sf_add_rmsnorm(p, None, p, 1, 4096, ctypes.c_float(-1.0), p, None) == sf.SF_EINVAL
+    assert L.sf_add_rmsnorm(None, None, p, 1, 4096, ctypes.c_float(1e-5), p, None) == sf.SF_EINVAL
+    assert L.sf_rope(p, 8, 127, 0, ctypes.c_double(500000.0), None, None) == sf.SF_EINVAL
+    assert "even d" in _err(sf)
+    assert L.sf_rope(p, 8, 128, -1, ctypes.c_double(500000.0), None, None) == sf.SF_EINVAL
+    assert L.sf_rope(p, 8, 128, 0, ctypes.c_double(0.0), None, None) == sf.SF_EINVAL
+    assert L.sf_silu_mul(p, p, 0, p, None) == sf.SF_EINVAL
+    # append: t must lie inside the stride, d a multiple of 32, widths as the quantizer's
+    assert L.sf_kv_append(p, 8, 128, 64, 64, 2, 2, p, p, p, p, None) == sf.SF_EINVAL
+    assert L.sf_kv_append(p, 8, 100, 64, 3, 2, 2, p, p, p, p, None) == sf.SF_EINVAL
+    assert L.sf_kv_append(p, 8, 128, 64, 3, 3, 2, p, p, p, p, None) == sf.SF_EINVAL
+    # attention over a strided cache: a stride below T is refused
+    kv = sf._QKV(256, 256, 256, 256, 256, 256, 256, 256, 2, 2, 299)
+    assert L.sf_attn_decode_refine(p, 8, 2, 128, 300, ctypes.byref(kv), 3, p, p, p, p,
+                                   ctypes.c_size_t(1 << 30), None) == sf.SF_EINVAL
+    assert "row_stride" in _err(sf)
