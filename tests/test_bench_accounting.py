@@ -38,3 +38,15 @@ def test_workload_names_follow_the_context():
 def test_whole_job_value():
     # every rank's bytes over the slowest rank's time
     assert bench.whole_job_gbs(2e9, 1.0, 4) == 8000.0
+
+
+def test_bench_defaults(monkeypatch):
+    """No flags: one GPU, a minutes-scale run, W >= 3 warm-up steps, the
+    128K leg on; --impl reference selects the oracle arm."""
+    monkeypatch.setattr("sys.argv", ["bench.py"])
+    a = bench.parse()
+    assert (a.gpus, a.impl, a.context, a.long_context) == (1, "sf", 32768, 131072)
+    assert a.warmup >= 3 and 1 <= a.steps <= 1000
+    monkeypatch.setattr("sys.argv", ["bench.py", "--impl", "reference", "--steps", "2", "--warmup", "3"])
+    a = bench.parse()
+    assert (a.impl, a.steps, a.warmup) == ("reference", 2, 3)
