@@ -368,11 +368,37 @@ def attn_decode_refine(q: torch.Tensor, kv: QKV, Hkv: int, T: int, k_tokens: int
         sel_out = torch.empty((Hkv, max(grp * k_tokens, 1)), dtype=torch.int32, device=dev)
     if sel_n is None:
         sel_n = torch.empty(Hkv, dtype=torch.int32, device=dev)
+    _check_attn_outputs(q, Hkv, k_tokens, out, sel_out, sel_n)
     s = kv.c_struct()
     _check(_lib.sf_attn_decode_refine(_ptr(q), Hq, Hkv, d, T, ctypes.byref(s), k_tokens, _ptr(sel_out),
                                       _ptr(sel_n), _ptr(out), _ptr(workspace),
                                       workspace.numel() * workspace.element_size(), _stream(stream)))
     return out, sel_out, sel_n
+
+
+def _check_attn_outputs(q: torch.Tensor, Hkv: int, k_tokens: int, out: torch.Tensor, sel_out: torch.Tensor,
+                        sel_n: torch.Tensor) -> None:
+    """Shapes, dtypes and devices of the attention's caller-provided buffers,
+    checked before anything reaches the library (an undersized output would
+    be written out of bounds by the kernels)."""
+    if q.dtype != torch.bfloat16 or q.dim() != 2:
+        raise ValueError("q must be a 2-D bfloat16 tensor [Hq][d]")
+    Hq, d = q.shape
+    if Hkv < 1 or Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    if out.dtype != torch.float32 or out.numel() < Hq * d:
+        raise ValueError(f"out must be float32 with at least Hq*d = {Hq * d} elements")
+    need = Hkv * (Hq // Hkv) * k_tokens
+    if sel_out.dtype != torch.int32 or sel_out.numel() < need:
+        raise ValueError(f"sel_out must be int32 with at least Hkv*(Hq/Hkv)*k_tokens = {need} elements")
+    if sel_n.dtype != torch.int32 or sel_n.numel() < Hkv:
+        raise ValueError(f"sel_n must be int32 with at least Hkv = {Hkv} elements")
+    for name, t in (("q", q), ("out", out), ("sel_out", sel_out), ("sel_n", sel_n)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        _dev(t, name)
+        if t.device != q.device:
+            raise ValueError(f"{name} is on {t.device}, q on {q.device}")
 
 
 def attn_decode_refine_noalloc(q: torch.Tensor, kv: QKV, Hkv: int, T: int, k_tokens: int,
@@ -382,7 +408,7 @@ def attn_decode_refine_noalloc(q: torch.Tensor, kv: QKV, Hkv: int, T: int, k_tok
     (``sf_attn_decode_refine_noalloc``): for callers that must not allocate
     device memory at this point.  The caller provides the outputs; nothing
     is allocated by this call."""
-    _dev(q, "q")
+    _check_attn_outputs(q, Hkv, k_tokens, out, sel_out, sel_n)
     Hq, d = q.shape
     s = kv.c_struct()
     _check(_lib.sf_attn_decode_refine_noalloc(_ptr(q), Hq, Hkv, d, T, ctypes.byref(s), k_tokens, _ptr(sel_out),

@@ -108,3 +108,29 @@ def test_host_validation_decode_step_ops(sf):
     assert L.sf_attn_decode_refine(p, 8, 2, 128, 300, ctypes.byref(kv), 3, p, p, p, p,
                                    ctypes.c_size_t(1 << 30), None) == sf.SF_EINVAL
     assert "row_stride" in _err(sf)
+
+
+def test_attention_binding_refuses_bad_output_buffers_before_any_call(sf):
+    """An undersized or mistyped output would be written out of bounds by the
+    kernels: the binding refuses it before the library is reached (so this
+    runs without a GPU)."""
+    import torch
+    Hq, Hkv, d, k = 32, 8, 128, 10
+    q = torch.zeros((Hq, d), dtype=torch.bfloat16)
+    out = torch.empty((Hq, d), dtype=torch.float32)
+    sel = torch.empty((Hkv, Hq // Hkv * k), dtype=torch.int32)
+    sel_n = torch.empty((Hkv,), dtype=torch.int32)
+    kv = None  # never reached
+    with pytest.raises(ValueError, match="sel_out"):
+        sf.attn_decode_refine_noalloc(q, kv, Hkv, 64, k, out, sel[:, :-1].contiguous(), sel_n)
+    with pytest.raises(ValueError, match="sel_out"):
+        sf.attn_decode_refine_noalloc(q, kv, Hkv, 64, k, out, sel.to(torch.int64), sel_n)
+    with pytest.raises(ValueError, match="out must be"):
+        sf.attn_decode_refine_noalloc(q, kv, Hkv, 64, k, out[:-1], sel, sel_n)
+    with pytest.raises(ValueError, match="sel_n"):
+        sf.attn_decode_refine_noalloc(q, kv, Hkv, 64, k, out, sel, sel_n[:-1])
+    with pytest.raises(ValueError, match="q must be"):
+        sf.attn_decode_refine_noalloc(q.float(), kv, Hkv, 64, k, out, sel, sel_n)
+    # well-formed buffers still stop at the device check on a CPU tensor
+    with pytest.raises(ValueError, match="CUDA"):
+        sf.attn_decode_refine_noalloc(q, kv, Hkv, 64, k, out, sel, sel_n)

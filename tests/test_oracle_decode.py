@@ -175,3 +175,88 @@ def test_decode_step_runs_two_layers():
                                  Fraction(1, 100))
     assert logits.shape == (96,) and np.all(np.isfinite(logits))
     assert all(kv["k"]["q"].shape == (Hkv * (T + 1), 16) for kv in kvs)
+
+
+# ---- the whole step (layers chained, final norm, LM head) against a plain model ----
+
+def _plain_step(x, layers, kvs, Hq, Hkv, T, final_w, Whead, refined, d=16, eps=1e-5):
+    """Textbook chain written without the oracle's decode code: each layer
+    appends its own rotated k and its v (quantized per token-head, then taken
+    at full code or resident value), runs the plain layer, and the final
+    RMSNorm feeds a dense LM head.  Returns (logits, appended K rows, appended
+    V rows) -- the rows as quantized codes [layer][Hkv][d]."""
+    deq = dequant_full if refined else dequant_resident
+    k_rows, v_rows = [], []
+    for layer, kv in zip(layers, kvs):
+        W = {n: deq(layer[n]) for n in ("q", "k", "v", "o", "gate", "up", "down")}
+        W["norm1"], W["norm2"] = layer["norm1"], layer["norm2"]
+        n1 = _bf16(W["norm1"] * x / np.sqrt(np.dot(x, x) / x.size + eps))
+        k_new = quantize_nested(_rope_complex((W["k"] @ n1).reshape(Hkv, d), T).astype(np.float32), d, 2, 2)
+        v_new = quantize_nested((W["v"] @ n1).reshape(Hkv, d).astype(np.float32), d, 2, 2)
+        k_rows.append(k_new["q"])
+        v_rows.append(v_new["q"])
+        K = np.concatenate([deq(kv["k"]).reshape(Hkv, T, d), deq(k_new).reshape(Hkv, 1, d)], axis=1)
+        V = np.concatenate([deq(kv["v"]).reshape(Hkv, T, d), deq(v_new).reshape(Hkv, 1, d)], axis=1)
+        x = _plain_layer(x, W, K, V, Hq, Hkv, T)
+    nf = _bf16(final_w * x / np.sqrt(np.dot(x, x) / x.size + eps))
+    return deq(Whead) @ nf, k_rows, v_rows
+
+
+def _two_layer_model():
+    l0, kv0, x = _tiny_model(23)
+    l1, kv1, _ = _tiny_model(29)
+    rng = np.random.default_rng(31)
+    head = quantize_nested((rng.standard_normal((96, 64)) * 0.1).astype(np.float32), 16, 3, 1)
+    final_w = 1.0 + 0.2 * rng.standard_normal(64)
+    return [l0, l1], [kv0, kv1], x, head, final_w
+
+
+@pytest.mark.parametrize("refined", [True, False])
+def test_decode_step_equals_plain_two_layer_model(refined):
+    """p = 1 refines every channel and token (full-code weights and K/V
+    everywhere); p = 0 refines none (resident values everywhere).  Either way
+    the oracle's step must equal the plain chain: both layers in order, each
+    with its own cache, then the final RMSNorm and the LM head on its output."""
+    Hq, Hkv, T = 4, 2, 12
+    layers, kvs, x, head, final_w = _two_layer_model()
+    p = Fraction(1) if refined else Fraction(0)
+    logits, kvs2 = od.decode_step(x, layers, kvs, T, Hq, Hkv, final_w, head, p, p)
+    ref, k_rows, v_rows = _plain_step(x, layers, kvs, Hq, Hkv, T, final_w, head, refined)
+    np.testing.assert_allclose(logits, ref, rtol=1e-9, atol=1e-9)
+    for li, kv2 in enumerate(kvs2):
+        np.testing.assert_array_equal(kv2["k"]["q"].reshape(Hkv, T + 1, 16)[:, T], k_rows[li])
+        np.testing.assert_array_equal(kv2["v"]["q"].reshape(Hkv, T + 1, 16)[:, T], v_rows[li])
+        # the old tokens are untouched
+        np.testing.assert_array_equal(kv2["k"]["q"].reshape(Hkv, T + 1, 16)[:, :T],
+                                      kvs[li]["k"]["q"].reshape(Hkv, T, 16))
+
+
+def _step_with_mistake(x, layers, kvs, T, Hq, Hkv, final_w, head, p, mistake):
+    """The oracle's step assembled from its own pieces with one planted
+    mistake: the pin above must tell each of them apart from the plain model."""
+    if mistake == "caches_swapped":
+        kvs = kvs[::-1]
+    if mistake == "layers_reversed":
+        layers = layers[::-1]
+    for layer, kv in zip(layers, kvs):
+        x, _ = od.decode_layer(x, layer, kv, T, Hq, Hkv, p, p)
+    if mistake == "no_final_norm":
+        n = x
+    elif mistake == "final_norm_unit_weight":
+        n = od.rms_norm(x, np.ones_like(final_w))
+    else:
+        n = od.rms_norm(x, final_w)
+    return od.refined_linear(head, n, p)
+
+
+@pytest.mark.parametrize("mistake", ["caches_swapped", "layers_reversed", "no_final_norm",
+                                     "final_norm_unit_weight"])
+def test_decode_step_pin_catches_planted_mistakes(mistake):
+    Hq, Hkv, T = 4, 2, 12
+    layers, kvs, x, head, final_w = _two_layer_model()
+    p = Fraction(1)
+    ref, _, _ = _plain_step(x, layers, kvs, Hq, Hkv, T, final_w, head, True)
+    good = _step_with_mistake(x, layers, kvs, T, Hq, Hkv, final_w, head, p, None)
+    np.testing.assert_allclose(good, ref, rtol=1e-9, atol=1e-9)
+    bad = _step_with_mistake(x, layers, kvs, T, Hq, Hkv, final_w, head, p, mistake)
+    assert np.max(np.abs(bad - ref)) > 1e-3 * np.max(np.abs(ref))
