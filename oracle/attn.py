@@ -20,6 +20,12 @@ A5  k'_t, v'_t are full-code values (Q5) for t in U_g and resident values
     otherwise; s'[h][t] = q_h . k'_t / sqrt(d); o_h = sum_t softmax(s'_h)_t v'_t
     in fp64, reported as fp32.
 A6  the GPU output is accepted within 2e-3 max-abs.
+A7  refinement bits held in a cache (the deadline reading of a KV
+    refinement cache): only the union tokens whose bits are on the device
+    when the step starts are refined, E_g = U_g ∩ available_g; the others
+    keep resident K and V this step (a miss keeps resident precision:
+    rag-lover.com explainer, 限界と未検証の範囲) and are fetched for later
+    steps.  The selection and the reported union do not change.
 """
 
 from __future__ import annotations
@@ -79,12 +85,14 @@ def topk_tokens(kappa: np.ndarray, k: int) -> np.ndarray:
 
 
 def attn_decode_refine(q_bits: np.ndarray, qzk: dict, qzv: dict, Hkv: int, T: int, k_tokens: int,
-                       refine: bool = True) -> dict:
-    """A1-A5.  q_bits [Hq][d] bf16 patterns; qzk / qzv quantized K and V with
-    rows = token-heads ordered [Hkv][T] and groups of the full head dim.
+                       refine: bool = True, available: np.ndarray | None = None) -> dict:
+    """A1-A5 (A7 when ``available``, bool [Hkv][T], is given).  q_bits
+    [Hq][d] bf16 patterns; qzk / qzv quantized K and V with rows =
+    token-heads ordered [Hkv][T] and groups of the full head dim.
 
     Returns dict(out fp64 [Hq][d], sel list of per-head ascending token
-    arrays, union list of per-KV-head ascending token arrays)."""
+    arrays, union list of per-KV-head ascending token arrays, refined list
+    of per-KV-head ascending arrays of the tokens actually refined)."""
     q = bf16_to_f64(q_bits)
     Hq, d = q.shape
     if Hq % Hkv:
@@ -96,7 +104,7 @@ def attn_decode_refine(q_bits: np.ndarray, qzk: dict, qzv: dict, Hkv: int, T: in
     k_full = dequant_full(qzk) if refine else None
     v_full = dequant_full(qzv) if refine else None
     out = np.zeros((Hq, d))
-    sel, union = [], []
+    sel, union, refined = [], [], []
     for g in range(Hkv):
         rows = slice(g * T, (g + 1) * T)
         heads = range(g * grp, (g + 1) * grp)
@@ -110,11 +118,13 @@ def attn_decode_refine(q_bits: np.ndarray, qzk: dict, qzv: dict, Hkv: int, T: in
             picked.update(int(t) for t in st)
         U = np.array(sorted(picked), dtype=np.int64)
         union.append(U.astype(np.int32))
+        E = U if available is None else U[np.asarray(available[g], dtype=bool)[U]]   # A7
+        refined.append(E.astype(np.int32))
         kk = k_res[rows].copy()
         vv = v_res[rows].copy()
-        if U.size:
-            kk[U] = k_full[rows][U]
-            vv[U] = v_full[rows][U]
+        if E.size:
+            kk[E] = k_full[rows][E]
+            vv[E] = v_full[rows][E]
         for h in heads:
             out[h] = attend(q[h], kk, vv)
-    return dict(out=out, sel=sel, union=union)
+    return dict(out=out, sel=sel, union=union, refined=refined)

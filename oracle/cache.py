@@ -18,6 +18,12 @@ C5  every inserted unit gets last_use = t; then t advances by one.
 C6  for weights the correction always uses all of S (every fetch completes
     before use), so the GEMV result does not depend on cache state; what is
     compared is the hit / miss / bypass sets and the slot each unit lands in.
+C7  a fetch budget F (the deadline reading, for caches whose consumer does
+    not wait for the fetch): only the first F misses in ascending unit order
+    are fetched and go through C4; the misses after them are *late* --
+    neither fetched nor cached nor touched, so their precision stays the
+    resident one (a miss keeps resident precision: rag-lover.com explainer,
+    限界と未検証の範囲).  No budget (F = None) is C1-C5 unchanged.
 
 ``preload`` fills an empty cache with the given units in slots 0, 1, ...
 with last_use = -1 (older than any step), and counts nothing.
@@ -36,7 +42,7 @@ class LRUCache:
         self.last_use: dict[int, int] = {}
         self.free: list[int] = list(range(capacity))
         self.t = 0
-        self.hits = self.misses = self.bypass = 0
+        self.hits = self.misses = self.bypass = self.late = 0
 
     def preload(self, units) -> None:
         units = list(units)
@@ -49,7 +55,7 @@ class LRUCache:
             self.slot_of[u] = slot
             self.last_use[u] = -1
 
-    def step(self, S) -> dict:
+    def step(self, S, budget: int | None = None) -> dict:
         S = [int(u) for u in S]
         if S != sorted(set(S)):
             raise ValueError("S must be strictly ascending")
@@ -57,6 +63,10 @@ class LRUCache:
         in_S = set(S)
         H = [u for u in S if u in self.slot_of]                       # C1
         M = [u for u in S if u not in self.slot_of]
+        if budget is not None and budget < 0:
+            raise ValueError("negative budget")
+        nf = len(M) if budget is None else min(len(M), budget)        # C7
+        fetched, late = M[:nf], M[nf:]
         for u in H:                                                    # C2
             self.last_use[u] = t
         victims = sorted((u for u in self.slot_of if u not in in_S),  # C3
@@ -64,7 +74,7 @@ class LRUCache:
         free_sorted = sorted(self.free)
         avail = [("free", s, None) for s in free_sorted] + [("victim", self.slot_of[v], v) for v in victims]
         inserted, bypass = [], []
-        for i, u in enumerate(M):                                      # C4
+        for i, u in enumerate(fetched):                                # C4
             if i >= len(avail):
                 bypass.append(u)
                 continue
@@ -81,7 +91,8 @@ class LRUCache:
         self.hits += len(H)
         self.misses += len(M)
         self.bypass += len(bypass)
-        return dict(hits=H, misses=M, bypass=bypass, inserted=inserted)
+        self.late += len(late)
+        return dict(hits=H, misses=M, bypass=bypass, late=late, inserted=inserted)
 
     def snapshot(self) -> dict[int, int]:
         """unit -> slot for every cached unit."""

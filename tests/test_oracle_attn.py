@@ -120,3 +120,41 @@ def test_refinement_reduces_error():
     e_ref = np.abs(attn.attn_decode_refine(qb, qk, qv, Hkv, T, count_fraction(1, T))["out"] - exact).mean()
     e_res = np.abs(attn.attn_decode_refine(qb, qk, qv, Hkv, T, 0)["out"] - exact).mean()
     assert e_ref < e_res
+
+
+def test_available_mask_refines_only_cached_union_tokens():
+    """A7: with a per-token availability mask the union is unchanged and
+    only its available tokens take full-code K and V; all available equals
+    A5, none available gives the resident attention.  The mixed case is
+    checked against library softmax on K/V assembled here token by token."""
+    from scipy.special import softmax
+    from oracle.quant import dequant_full, dequant_resident, quantize_nested
+    from workloads import gen_kv, gen_query
+    Hq, Hkv, T, d, k = 8, 2, 300, 32, 20
+    Kf, Vf, _ = gen_kv(71, Hkv, T, d)
+    qk, qv = quantize_nested(Kf.reshape(-1, d), d, 2, 2), quantize_nested(Vf.reshape(-1, d), d, 2, 2)
+    qb = gen_query(72, Hq, d)
+    attn_decode_refine = attn.attn_decode_refine
+    full = attn_decode_refine(qb, qk, qv, Hkv, T, k)
+    r_all = attn_decode_refine(qb, qk, qv, Hkv, T, k, available=np.ones((Hkv, T), bool))
+    np.testing.assert_array_equal(r_all["out"], full["out"])
+    r_none = attn_decode_refine(qb, qk, qv, Hkv, T, k, available=np.zeros((Hkv, T), bool))
+    res = attn_decode_refine(qb, qk, qv, Hkv, T, k, refine=False)
+    np.testing.assert_allclose(r_none["out"], res["out"], rtol=0, atol=1e-12)
+    for g in range(Hkv):
+        np.testing.assert_array_equal(r_none["union"][g], full["union"][g])
+        assert r_none["refined"][g].size == 0
+    avail = np.random.default_rng(73).random((Hkv, T)) < 0.5
+    r = attn_decode_refine(qb, qk, qv, Hkv, T, k, available=avail)
+    kf, kr, vf, vr = dequant_full(qk), dequant_resident(qk), dequant_full(qv), dequant_resident(qv)
+    q = (qb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    grp = Hq // Hkv
+    for g in range(Hkv):
+        U = set(full["union"][g].tolist())
+        assert r["refined"][g].tolist() == sorted(t for t in U if avail[g, t])
+        use_full = np.array([t in U and avail[g, t] for t in range(T)])
+        Kg = np.where(use_full[:, None], kf[g * T:(g + 1) * T], kr[g * T:(g + 1) * T])
+        Vg = np.where(use_full[:, None], vf[g * T:(g + 1) * T], vr[g * T:(g + 1) * T])
+        for h in range(g * grp, (g + 1) * grp):
+            want = softmax(Kg @ q[h] / np.sqrt(d)) @ Vg
+            np.testing.assert_allclose(r["out"][h], want, rtol=1e-10, atol=1e-12)

@@ -21,9 +21,11 @@ class OrderedLRU:
         self.od = OrderedDict()       # unit -> slot, least recent first
         self.free = list(range(capacity))
 
-    def step(self, S):
+    def step(self, S, budget=None):
         hits = [u for u in S if u in self.od]
         misses = [u for u in S if u not in self.od]
+        late = [] if budget is None else misses[budget:]
+        misses = misses if budget is None else misses[:budget]
         in_S = set(S)
         victims = [u for u in self.od if u not in in_S]     # recency order
         avail = [(s, None) for s in sorted(self.free)] + [(self.od[v], v) for v in victims]
@@ -41,7 +43,7 @@ class OrderedLRU:
                 bypass.append(u)
         for u in sorted(hits + [u for u, _ in placed]):
             self.od.move_to_end(u)
-        return hits, misses, bypass, placed
+        return hits, misses + late, bypass, placed
 
 
 def _random_steps(seed, K, C, n_steps, k, hot):
@@ -94,3 +96,34 @@ def test_rejects_unsorted():
     c = LRUCache(10, 3)
     with pytest.raises(ValueError):
         c.step([3, 1])
+
+
+@pytest.mark.parametrize("K,C,k,hot,budget", [(512, 40, 30, 5, 7), (256, 100, 24, 4, 0), (128, 16, 20, 3, 3),
+                                              (300, 60, 25, 10, 1000)])
+def test_fetch_budget_against_ordered_dict(K, C, k, hot, budget):
+    """C7: with a per-step fetch budget only the first F misses (ascending)
+    are fetched; the late ones are neither cached nor touched."""
+    a, b = LRUCache(K, C), OrderedLRU(C)
+    late_total = 0
+    for S in _random_steps(K + C + 1, K, C, 60, k, hot):
+        r = a.step(S, budget=budget)
+        h, m, by, placed = b.step(S, budget=budget)
+        assert r["hits"] == h and r["misses"] == m and r["bypass"] == by and r["inserted"] == placed
+        assert r["late"] == r["misses"][min(len(r["misses"]), budget):]
+        assert not set(r["late"]) & set(a.snapshot())
+        late_total += len(r["late"])
+        assert a.snapshot() == dict(b.od)
+    assert a.late == late_total
+
+
+def test_fetch_budget_by_hand():
+    c = LRUCache(10, 3)
+    r = c.step([1, 4, 7], budget=2)   # two fetched, 7 is late
+    assert r["inserted"] == [(1, 0), (4, 1)] and r["late"] == [7]
+    r = c.step([4, 7, 8], budget=1)   # 4 hits; 7 fetched into the free slot; 8 late
+    assert r["hits"] == [4] and r["inserted"] == [(7, 2)] and r["late"] == [8]
+    r = c.step([2, 3], budget=0)      # nothing fetched, nothing evicted
+    assert r["inserted"] == [] and r["late"] == [2, 3]
+    assert c.snapshot() == {1: 0, 4: 1, 7: 2}
+    r = c.step([2, 3])                # no budget: C1-C5 (victims by (last use, unit): 1, then 4)
+    assert r["inserted"] == [(2, 0), (3, 1)] and r["late"] == []
