@@ -126,6 +126,7 @@ typedef struct sf_cache_stats {
   int64_t misses;    /* selected units not found (bypass included) */
   int64_t bypass;    /* misses fetched for one step only (no slot left) */
   int64_t h2d_bytes; /* bytes moved from host memory for misses */
+  int64_t late;      /* misses beyond the fetch budget: neither fetched nor cached */
 } sf_cache_stats;
 
 /*
@@ -197,6 +198,21 @@ sf_status sf_refine_cache_reset(sf_refine_cache* c);
 
 /* Free everything the cache owns.  Synchronizes.  NULL is accepted. */
 sf_status sf_refine_cache_destroy(sf_refine_cache* c);
+
+/*
+ * sf_refine_cache_set_budget -- a per-step fetch budget, for a cache whose
+ * consumer does not wait for this step's fetches (the KV refinement cache of
+ * sf_attn_decode_refine).  At each later prefetch only the first `budget`
+ * misses in ascending unit order are fetched (and placed as above); the
+ * misses after them are late: neither fetched nor cached, counted in
+ * sf_cache_stats.late, and their precision stays the resident one (a miss
+ * keeps resident precision: rag-lover.com explainer, 限界と未検証の範囲).
+ * budget -1 removes the limit (the default).  A cache with a budget below
+ * max_select cannot serve a GEMV (SF_EINVAL there: a GEMV refines every
+ * selected column).  Takes effect at the next sf_refine_cache_prefetch; a
+ * group (below) keeps the budget its caches had when it was created.
+ */
+sf_status sf_refine_cache_set_budget(sf_refine_cache* c, int budget);
 
 /*
  * A group batches the prefetch of several caches whose selections live in
@@ -277,14 +293,31 @@ sf_status sf_select_topk_act_many(const sf_select_job* jobs, int count, sf_strea
  * GEMVs).  K must be a multiple of 256 up to 32768. */
 sf_status sf_act_prepare(const uint16_t* x, int K, void* act, sf_stream_t stream);
 
+/*
+ * sf_gemv_pack_batch1 -- the resident codes of a matrix in the layout the
+ * batch-1 tensor-core GEMV reads (an internal re-arrangement of the same
+ * bits, written once when the weights are loaded).  res: canonical resident
+ * codes [N][K*b_r/32] (device); out: device, N*K*b_r/32 words, 16-byte
+ * aligned, owned by the caller.  For b_r == 2 the layout is the canonical one
+ * (a plain copy; out may equal res).  For b_r == 3 each 256-channel slice of
+ * a row (24 words) holds the codes' low 2 bits in the 2-bit arrangement and
+ * their high bits in a separate 8-word plane, so that a code becomes an MMA
+ * operand byte with shifts and masks only; out must not alias res.
+ * Constraints: b_r in {2, 3}, N >= 1, K a positive multiple of 256.
+ */
+sf_status sf_gemv_pack_batch1(const uint32_t* res, int N, int K, int b_r, uint32_t* out, sf_stream_t stream);
+
 /* One matrix of a batch-1 GEMV launch.  The refinement source follows
  * sf_gemv_refine: cache (its last prefetch must have used the selection that
- * produced act), else W->ref when use_ref_store, else resident only. */
+ * produced act), else W->ref when use_ref_store, else resident only.
+ * res_b1: the resident codes in the batch-1 layout (sf_gemv_pack_batch1);
+ * NULL means W->res, allowed for b_r == 2 only. */
 typedef struct sf_gemv_job {
   const sf_qweight* W;
   sf_refine_cache* cache;
   int use_ref_store;
   float* y; /* device fp32 [W->N] */
+  const uint32_t* res_b1;
 } sf_gemv_job;
 
 /*
@@ -293,14 +326,21 @@ typedef struct sf_gemv_job {
  * the selected channels of x_j s (q_f - m_f), as sf_gemv_refine, in one
  * launch.  act comes from sf_select_topk_act (refined) or sf_act_prepare
  * (resident only) for this x; x is the bf16 row itself (device).
- * Computed on the integer tensor cores (mma.m16n8k32, 2-bit codes x 8-bit
- * activation digits) in tiles of 16 output rows.
- * Constraints: b_r == 2, G == 128, all jobs share K, G and b_f; N % 16 == 0;
- * K a multiple of 256 whose K/256 slices split into at most 16 warps of one
- * or two slices, in one or two K halves (4096 and 14336 qualify; with two
- * halves the partial sums are added onto zeroed outputs, an order-independent
- * fp32 addition); weight arrays 16-byte aligned.  SF_EINVAL otherwise.
- * Accuracy: as sf_gemv_refine.
+ * Computed on the integer tensor cores (mma.m16n8k32, 2- or 3-bit codes x
+ * 8-bit activation digits) in tiles of 16 output rows; the refinement
+ * correction on the f16 tensor cores (fp32 for a slice whose selected |x|
+ * reaches 2^15).
+ * Constraints: b_r in {2, 3}, b_f in {1, 2}, b_r + b_f <= 4, G == 128, all
+ * jobs share K, G and bit widths; N % 16 == 0; K a multiple of 256 whose
+ * K/256 slices split into at most 16 warps of one or two slices, in one or
+ * two K halves (4096 and 14336 qualify; with two halves the partial sums are
+ * added onto zeroed outputs, an order-independent fp32 addition); weight
+ * arrays 16-byte aligned; 3-bit codes given as res_b1.  SF_EINVAL otherwise.
+ * Accuracy: as sf_gemv_refine, given that within every 128-channel group
+ * the channels that matter are within 2^14 of the group's largest |x|: x is
+ * taken in fixed point relative to that maximum, with an absolute error of
+ * at most 2^(e-23) per channel (e its binary exponent), so channels far
+ * below it keep few bits.
  */
 sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, const uint16_t* x, const void* act,
                                 sf_stream_t stream);
@@ -319,6 +359,17 @@ typedef struct sf_qkv {
   const uint16_t *k_scale, *k_zero, *v_scale, *v_zero;
   int b_r, b_f;
   int row_stride;
+  /* NULL: k_ref / v_ref hold every token-head's refinement bits.  Non-NULL:
+   * the refinement bits live in this cache instead (k_ref and v_ref are
+   * ignored and may be NULL): one unit per token-head, unit g*S + t for token
+   * t of KV head g, unit_bytes 64 = the token-head's K refinement words
+   * followed by its V refinement words (both d*b_f/32 = 8 words).  A union
+   * token whose unit is not cached when the call runs keeps its resident K
+   * and V this step (the deadline reading of a KV refinement cache: a miss
+   * keeps resident precision, rag-lover.com explainer, 限界と未検証の範囲);
+   * the union and sel_out are unchanged.  The call orders its stream after
+   * the cache's last prefetch, and the next prefetch after the call. */
+  sf_refine_cache* ref_cache;
 } sf_qkv;
 
 /* Workspace bytes sf_attn_decode_refine needs for these sizes. */
@@ -381,6 +432,19 @@ sf_status sf_attn_decode_refine_noalloc(const uint16_t* q, int Hq, int Hkv, int 
                                         int32_t* sel_n, float* out, sf_stream_t stream);
 
 /*
+ * sf_attn_union_units -- the units of a KV refinement cache (see
+ * sf_qkv.ref_cache) that one attention call selected: for each KV head g in
+ * order, g*S + t for every token t of its ascending union, so the list is
+ * ascending.  sel_out [Hkv][cap] and sel_n [Hkv] as written by the attention
+ * (a negative sel_n[g] = -1 - length counts as its length); units device
+ * int32 [Hkv*cap]; n_units device int32 scalar.  Feed (units, n_units) to
+ * sf_refine_cache_prefetch to fetch the missed refinements for later steps.
+ * Constraints: Hkv in [1, 64], cap >= 1, S >= 1.
+ */
+sf_status sf_attn_union_units(const int32_t* sel_out, const int32_t* sel_n, int Hkv, int cap, int S,
+                              int32_t* units, int32_t* n_units, sf_stream_t stream);
+
+/*
  * sf_attn_set_path -- which implementation sf_attn_decode_refine and
  * sf_attn_decode_refine_noalloc use, process-wide.  The paper has no
  * counterpart; both implementations compute the definition above (the same
@@ -392,7 +456,8 @@ sf_status sf_attn_decode_refine_noalloc(const uint16_t* q, int Hq, int Hkv, int 
  *                     applies for T <= 32768 (Hq/Hkv <= 4) or T <= 16384
  *                     (Hq/Hkv == 8) on a device that fits the cluster, and
  *                     other calls return SF_ENOTIMPL;
- *   SF_ATTN_PIPELINE  only the multi-kernel pipeline (every size).
+ *   SF_ATTN_PIPELINE  only the multi-kernel pipeline (every size; the only
+ *                     one that reads refinements from a ref_cache).
  * Returns SF_EINVAL for any other value.  The setting is read when a call is
  * enqueued; a captured graph keeps the kernels it captured.
  */
@@ -437,6 +502,13 @@ sf_status sf_rope(float* x, int H, int d, int pos, double theta, uint16_t* y_bf1
 sf_status sf_silu_mul(const float* g, const float* u, int n, uint16_t* y, sf_stream_t stream);
 
 /*
+ * sf_round_bf16 -- y[i] = bf16(x[i]) (to nearest, ties to even) for i < n:
+ *   the attention's fp32 output as the bf16 input of the o projection.
+ *   x fp32 [n], y bf16 [n].  Constraints: n >= 1.
+ */
+sf_status sf_round_bf16(const float* x, int n, uint16_t* y, sf_stream_t stream);
+
+/*
  * sf_kv_append -- quantizes the new token's rows of K or V and writes them as
  *   token t of every KV head of a cache allocated for row_stride tokens per
  *   head: src fp32 [Hkv][d] (row g = KV head g) becomes cache row
@@ -451,6 +523,22 @@ sf_status sf_silu_mul(const float* g, const float* u, int n, uint16_t* y, sf_str
  */
 sf_status sf_kv_append(const float* src, int Hkv, int d, int row_stride, int t, int b_r, int b_f, uint32_t* res,
                        uint32_t* ref, uint16_t* scale, uint16_t* zero, sf_stream_t stream);
+
+/*
+ * sf_kv_append_cached -- sf_kv_append for K/V whose refinement bits live in a
+ *   KV refinement cache (sf_qkv.ref_cache): the resident codes, scale and zero
+ *   of token t go to res / scale / zero as in sf_kv_append; the refinement
+ *   words go to the cache's host master, unit g * row_stride + t, in its K
+ *   half (part 0) or V half (part 1), and also to the unit's cache row if it
+ *   is cached (so no cached copy goes stale).  The host master is written
+ *   through its device mapping, and must stay as the cache was created with.
+ *   Ordered after the cache's last prefetch; the next prefetch waits for it.
+ *   Constraints: as sf_kv_append; the cache's units are 2*d*b_f/8 bytes and
+ *   number at least Hkv * row_stride; part in {0, 1}.
+ */
+sf_status sf_kv_append_cached(const float* src, int Hkv, int d, int row_stride, int t, int b_r, int b_f,
+                              uint32_t* res, uint16_t* scale, uint16_t* zero, sf_refine_cache* ref_cache, int part,
+                              sf_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -52,11 +52,11 @@ class _QWeight(ctypes.Structure):
 class _QKV(ctypes.Structure):
     _fields_ = [("k_res", _p), ("k_ref", _p), ("v_res", _p), ("v_ref", _p),
                 ("k_scale", _p), ("k_zero", _p), ("v_scale", _p), ("v_zero", _p),
-                ("b_r", _i), ("b_f", _i), ("row_stride", _i)]
+                ("b_r", _i), ("b_f", _i), ("row_stride", _i), ("ref_cache", _p)]
 
 
 class _GemvJob(ctypes.Structure):
-    _fields_ = [("W", ctypes.POINTER(_QWeight)), ("cache", _p), ("use_ref_store", _i), ("y", _p)]
+    _fields_ = [("W", ctypes.POINTER(_QWeight)), ("cache", _p), ("use_ref_store", _i), ("y", _p), ("res_b1", _p)]
 
 
 class _SelectJob(ctypes.Structure):
@@ -65,7 +65,7 @@ class _SelectJob(ctypes.Structure):
 
 class CacheStats(ctypes.Structure):
     _fields_ = [("steps", ctypes.c_int64), ("hits", ctypes.c_int64), ("misses", ctypes.c_int64),
-                ("bypass", ctypes.c_int64), ("h2d_bytes", ctypes.c_int64)]
+                ("bypass", ctypes.c_int64), ("h2d_bytes", ctypes.c_int64), ("late", ctypes.c_int64)]
 
 
 _SIGS = {
@@ -82,6 +82,7 @@ _SIGS = {
     "sf_refine_cache_stats": ([_p, ctypes.POINTER(CacheStats)], _i),
     "sf_refine_cache_reset": ([_p], _i),
     "sf_refine_cache_destroy": ([_p], _i),
+    "sf_refine_cache_set_budget": ([_p, _i], _i),
     "sf_refine_group_create": ([ctypes.POINTER(_p), ctypes.POINTER(_p), ctypes.POINTER(_p), ctypes.POINTER(_p), _i],
                                _i),
     "sf_refine_group_prefetch": ([_p, _p, _p], _i),
@@ -92,14 +93,18 @@ _SIGS = {
     "sf_act_prepare": ([_p, _i, _p, _p], _i),
     "sf_select_topk_act_many": ([_p, _i, _p], _i),
     "sf_gemv_refine_batch1": ([_p, _i, _p, _p, _p], _i),
+    "sf_gemv_pack_batch1": ([_p, _i, _i, _i, _p, _p], _i),
     "sf_attn_workspace_size": ([_i, _i, _i, _i, _i, ctypes.POINTER(_sz)], _i),
     "sf_attn_decode_refine": ([_p, _i, _i, _i, _i, ctypes.POINTER(_QKV), _i, _p, _p, _p, _p, _sz, _p], _i),
     "sf_attn_decode_refine_noalloc": ([_p, _i, _i, _i, _i, ctypes.POINTER(_QKV), _i, _p, _p, _p, _p], _i),
     "sf_attn_set_path": ([_i], _i),
+    "sf_attn_union_units": ([_p, _p, _i, _i, _i, _p, _p, _p], _i),
     "sf_add_rmsnorm": ([_p, _p, _p, _i, _i, ctypes.c_float, _p, _p], _i),
     "sf_rope": ([_p, _i, _i, _i, ctypes.c_double, _p, _p], _i),
     "sf_silu_mul": ([_p, _p, _i, _p, _p], _i),
+    "sf_round_bf16": ([_p, _i, _p, _p], _i),
     "sf_kv_append": ([_p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p], _i),
+    "sf_kv_append_cached": ([_p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _i, _p], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -153,6 +158,7 @@ class QWeight:
     b_r: int
     b_f: int
     layout: str = "by_column"
+    res_b1: torch.Tensor | None = None  # resident codes in the batch-1 layout (pack_batch1)
 
     def c_struct(self, with_ref: bool = False) -> _QWeight:
         return _QWeight(_ptr(self.res), _ptr(self.scale), _ptr(self.zero),
@@ -254,6 +260,10 @@ class RefineCache:
     def reset(self) -> None:
         _check(_lib.sf_refine_cache_reset(self._h))
 
+    def set_budget(self, budget: int | None) -> None:
+        """Per-step fetch budget (``sf_refine_cache_set_budget``); None = no limit."""
+        _check(_lib.sf_refine_cache_set_budget(self._h, -1 if budget is None else int(budget)))
+
     def close(self) -> None:
         if getattr(self, "_h", None) is not None and self._h.value:
             _check(_lib.sf_refine_cache_destroy(self._h))
@@ -323,15 +333,19 @@ def gemv_refine(W: QWeight, x: torch.Tensor, idx: torch.Tensor | None = None, n:
 class QKV:
     """Quantized K and V, rows = token-heads [Hkv][S] (layout by_row, G = d):
     S = row_stride when it is positive (a cache allocated for row_stride
-    tokens per head), else the call's T."""
+    tokens per head), else the call's T.  ``ref_cache``: the refinement bits
+    live in this RefineCache (units g*S + t of 64 bytes: K words then V
+    words) instead of k.ref / v.ref, which may then be None."""
     k: QWeight
     v: QWeight
     row_stride: int = 0
+    ref_cache: "RefineCache | None" = None
 
     def c_struct(self) -> _QKV:
         return _QKV(_ptr(self.k.res), _ptr(self.k.ref), _ptr(self.v.res), _ptr(self.v.ref),
                     _ptr(self.k.scale), _ptr(self.k.zero), _ptr(self.v.scale), _ptr(self.v.zero),
-                    self.k.b_r, self.k.b_f, self.row_stride)
+                    self.k.b_r, self.k.b_f, self.row_stride,
+                    self.ref_cache.handle if self.ref_cache is not None else None)
 
 
 ATTN_AUTO, ATTN_CLUSTER, ATTN_PIPELINE = 0, 1, 2
@@ -401,6 +415,18 @@ def _check_attn_outputs(q: torch.Tensor, Hkv: int, k_tokens: int, out: torch.Ten
             raise ValueError(f"{name} is on {t.device}, q on {q.device}")
 
 
+def attn_union_units(sel_out: torch.Tensor, sel_n: torch.Tensor, Hkv: int, cap: int, S: int, units: torch.Tensor,
+                     n_units: torch.Tensor, stream: torch.cuda.Stream | None = None) -> None:
+    """``sf_attn_union_units``: the KV-refinement-cache units (g*S + t) of
+    the union an attention call selected, ascending, into units / n_units.
+    cap = (Hq/Hkv) * k_tokens of that call (the row stride of sel_out)."""
+    if sel_out.numel() < Hkv * cap or units.dtype != torch.int32 or units.numel() < Hkv * cap or \
+            n_units.dtype != torch.int32:
+        raise ValueError("units must be int32 with room for Hkv * cap entries, n_units int32")
+    _check(_lib.sf_attn_union_units(_ptr(sel_out), _ptr(sel_n), Hkv, cap, S, _ptr(units), _ptr(n_units),
+                                    _stream(stream)))
+
+
 def attn_decode_refine_noalloc(q: torch.Tensor, kv: QKV, Hkv: int, T: int, k_tokens: int,
                                out: torch.Tensor, sel_out: torch.Tensor, sel_n: torch.Tensor,
                                stream: torch.cuda.Stream | None = None) -> None:
@@ -416,6 +442,23 @@ def attn_decode_refine_noalloc(q: torch.Tensor, kv: QKV, Hkv: int, T: int, k_tok
 
 
 # ---- batch-1 fast path ---------------------------------------------------------
+
+def pack_batch1(W: QWeight, drop_canonical: bool = False, stream: torch.cuda.Stream | None = None) -> QWeight:
+    """Writes W.res_b1, the resident codes in the layout of the batch-1
+    tensor-core GEMV (``sf_gemv_pack_batch1``); for 2-bit codes that is the
+    canonical layout itself.  ``drop_canonical`` releases W.res afterwards
+    (the batch-1 GEMV then reads only W.res_b1)."""
+    _dev(W.res, "W.res")
+    if W.b_r == 2:
+        W.res_b1 = W.res
+    else:
+        out = torch.empty_like(W.res)
+        _check(_lib.sf_gemv_pack_batch1(_ptr(W.res), W.N, W.K, W.b_r, _ptr(out), _stream(stream)))
+        W.res_b1 = out
+        if drop_canonical:
+            W.res = None
+    return W
+
 
 def act_bytes(K: int) -> int:
     return _lib.sf_act_bytes(K)
@@ -449,6 +492,7 @@ class Batch1Jobs:
             arr[i].cache = cache.handle if cache is not None else None
             arr[i].use_ref_store = 1 if store else 0
             arr[i].y = _ptr(y)
+            arr[i].res_b1 = _ptr(W.res_b1) if W.res_b1 is not None else None
         self._arr = arr
         self.count = len(jobs)
 
@@ -525,6 +569,20 @@ def silu_mul(g: torch.Tensor, u: torch.Tensor, y: torch.Tensor | None = None,
     return y
 
 
+def round_bf16(x: torch.Tensor, y: torch.Tensor | None = None,
+               stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """``sf_round_bf16``: bf16 (ties to even) of fp32 x, elementwise."""
+    _dev(x, "x")
+    if x.dtype != torch.float32:
+        raise ValueError("x must be float32")
+    if y is None:
+        y = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+    if y.dtype != torch.bfloat16 or y.numel() < x.numel():
+        raise ValueError("y must be bfloat16 with at least x.numel() elements")
+    _check(_lib.sf_round_bf16(_ptr(x), x.numel(), _ptr(y), _stream(stream)))
+    return y
+
+
 def kv_append(src: torch.Tensor, res: torch.Tensor, ref: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
               row_stride: int, t: int, b_r: int = 2, b_f: int = 2, stream: torch.cuda.Stream | None = None) -> None:
     """``sf_kv_append``: quantizes src (fp32 [Hkv][d]) and writes it as token
@@ -537,3 +595,16 @@ def kv_append(src: torch.Tensor, res: torch.Tensor, ref: torch.Tensor, scale: to
     _check(_lib.sf_kv_append(_ptr(src), Hkv, d, row_stride, t, b_r, b_f, _ptr(res), _ptr(ref), _ptr(scale),
                              _ptr(zero), _stream(stream)))
 
+
+
+def kv_append_cached(src: torch.Tensor, res: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
+                     cache: RefineCache, part: int, row_stride: int, t: int, b_r: int = 2, b_f: int = 2,
+                     stream: torch.cuda.Stream | None = None) -> None:
+    """``sf_kv_append_cached``: as kv_append, with the refinement bits written
+    to the KV refinement cache's host master (part 0: K half, 1: V half)."""
+    _dev(src, "src")
+    if src.dtype != torch.float32 or src.dim() != 2:
+        raise ValueError("src must be a 2-D float32 tensor")
+    Hkv, d = src.shape
+    _check(_lib.sf_kv_append_cached(_ptr(src), Hkv, d, row_stride, t, b_r, b_f, _ptr(res), _ptr(scale), _ptr(zero),
+                                    cache.handle, part, _stream(stream)))

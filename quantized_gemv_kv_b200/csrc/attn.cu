@@ -674,13 +674,24 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
 // of the group: one load of the list, one of the token's two code rows.
 
 constexpr int kRefThreads = 256;
+// A unit of a KV refinement cache: the token-head's 8 K refinement words,
+// then its 8 V refinement words.
+constexpr int kCacheUnitWords = 2 * kWordsPerRow;
+
+// The V refinement words of K/V row `row`: from the store (uslot == nullptr)
+// or from the cache slot that holds the row's unit.
+__device__ __forceinline__ const uint32_t* vref_row(const uint32_t* v_ref, const int32_t* uslot, size_t row) {
+  return uslot != nullptr ? v_ref + static_cast<size_t>(uslot[row]) * kCacheUnitWords + kWordsPerRow
+                          : v_ref + row * kWordsPerRow;
+}
 
 template <int GRP>
 __global__ void __launch_bounds__(kRefThreads, 2)
 attn_refine_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
-                   const uint32_t* __restrict__ k_ref, const uint16_t* __restrict__ k_scale,
-                   const uint16_t* __restrict__ k_zero, int T, int S, int cap, const int32_t* __restrict__ sel_out,
-                   const int32_t* __restrict__ sel_n, float* __restrict__ score, uint32_t* __restrict__ rkey) {
+                   const uint32_t* __restrict__ k_ref, const int32_t* __restrict__ uslot,
+                   const uint16_t* __restrict__ k_scale, const uint16_t* __restrict__ k_zero, int T, int S, int cap,
+                   const int32_t* __restrict__ sel_out, const int32_t* __restrict__ sel_n, float* __restrict__ score,
+                   uint32_t* __restrict__ rkey, uint32_t* __restrict__ umask, int words_t) {
   __shared__ float qs[GRP][D];
   __shared__ float qsum[GRP];
   const int g = blockIdx.y;
@@ -695,11 +706,21 @@ attn_refine_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ 
   for (int h = 0; h < GRP; ++h) mk[h] = 0u;
   for (int u0 = blockIdx.x * kRefThreads; u0 < U; u0 += gridDim.x * kRefThreads) {  // uniform over the block
     const int u = u0 + static_cast<int>(threadIdx.x);
-    if (u < U) {
-      const int t = list[u];
-      const size_t row = rowg + t;
+    const int t = u < U ? list[u] : 0;
+    const size_t row = rowg + t;
+    const int slot = (u < U && uslot != nullptr) ? uslot[row] : 0;
+    if (u < U && slot < 0) {
+      // refinement bits not on the device (a cache miss): the token keeps its
+      // resident key and value this step; it leaves the refined set, and its
+      // resident scores still bound the weights' maximum
+      atomicAnd(umask + static_cast<size_t>(g) * words_t + (t >> 5), ~(1u << (t & 31)));
+#pragma unroll
+      for (int h = 0; h < GRP; ++h)
+        mk[h] = max(mk[h], okey32(score[(static_cast<size_t>(g) * GRP + h) * T + t]));
+    } else if (u < U) {
       const uint4* pr = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
-      const uint4* pf = reinterpret_cast<const uint4*>(k_ref + row * kWordsPerRow);
+      const uint4* pf = reinterpret_cast<const uint4*>(
+          uslot != nullptr ? k_ref + static_cast<size_t>(slot) * kCacheUnitWords : k_ref + row * kWordsPerRow);
       const uint4 r0 = pr[0], r1 = pr[1], f0 = pf[0], f1 = pf[1];
       const float sv = sfd::half_bits_to_float(k_scale[row]);
       const float z = sfd::half_bits_to_float(k_zero[row]);
@@ -780,7 +801,8 @@ struct OutCfg {
 template <int GRP>
 __global__ void __launch_bounds__(kOutThreads)
 attn_out_kernel(const uint32_t* __restrict__ v_res,
-                const uint32_t* __restrict__ v_ref, const uint16_t* __restrict__ v_scale,
+                const uint32_t* __restrict__ v_ref, const int32_t* __restrict__ uslot,
+                const uint16_t* __restrict__ v_scale,
                 const uint16_t* __restrict__ v_zero, int T, int S, int tps, int words_t, int splits,
                 const float* __restrict__ score, const uint32_t* __restrict__ mkey, const uint32_t* __restrict__ rkey,
                 const uint32_t* __restrict__ umask, float* __restrict__ part, int32_t* __restrict__ done,
@@ -880,7 +902,7 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
     }
     const int nu = ucount;
     for (int u = tid; u < min(nu, kUCap); u += kOutThreads) {
-      const uint32_t* src = v_ref + (rowg + c0 + ulist[u]) * kWordsPerRow;
+      const uint32_t* src = vref_row(v_ref, uslot, rowg + c0 + ulist[u]);
       cp_async16_attn(vrs + u * kWordsPerRow, src);
       cp_async16_attn(vrs + u * kWordsPerRow + 4, src + 4);
     }
@@ -970,7 +992,7 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
     for (int u = warp; u < nu; u += kOW) {
       const int i = ulist[u];
       const uint32_t wrow = u < kUCap ? vrs[u * kWordsPerRow + (lane >> 2)]
-                                      : v_ref[(rowg + c0 + i) * kWordsPerRow + (lane >> 2)];
+                                      : vref_row(v_ref, uslot, rowg + c0 + i)[lane >> 2];
       const uint32_t wf = wrow >> ((lane & 3) * 8);
 #pragma unroll
       for (int h = 0; h < GRP; ++h) {
@@ -1105,6 +1127,21 @@ template <int GRP>
 sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k, int32_t* sel_out, int32_t* sel_n,
               float* out, char* ws, const Layout& L, cudaStream_t s) {
   const int S = kv->row_stride > 0 ? kv->row_stride : T;  // rows per KV head in the K/V arrays
+  // refinement source: the stores k_ref / v_ref, or a KV refinement cache
+  const uint32_t* k_ref = kv->k_ref;
+  const uint32_t* v_ref = kv->v_ref;
+  const int32_t* uslot = nullptr;
+  if (kv->ref_cache) {
+    sf::CacheView v{};
+    const sf_status cs = sf::cache_view_for_reader(kv->ref_cache, s, &v);
+    if (cs != SF_OK) return cs;
+    SF_REQUIRE(v.unit_words == kCacheUnitWords, "sf_attn_decode_refine: ref_cache units must be %d bytes",
+               4 * kCacheUnitWords);
+    SF_REQUIRE(static_cast<long long>(v.num_units) >= static_cast<long long>(Hkv) * S,
+               "sf_attn_decode_refine: ref_cache has fewer units than Hkv * row_stride");
+    k_ref = v_ref = v.rows;
+    uslot = v.unit_slot;
+  }
   float* score = reinterpret_cast<float*>(ws + L.score);
   int32_t* cand = reinterpret_cast<int32_t*>(ws + L.cand);
   int32_t* cand2 = reinterpret_cast<int32_t*>(ws + L.cand2);
@@ -1170,18 +1207,22 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
   if (k > 0) {
     const int cap = grp * k;
     const int nblk = std::max(1, std::min((cap + kRefThreads - 1) / kRefThreads, 2 * sms / Hkv));
-    attn_refine_kernel<GRP><<<dim3(nblk, Hkv), kRefThreads, 0, s>>>(q, kv->k_res, kv->k_ref, kv->k_scale, kv->k_zero,
-                                                                   T, S, cap, sel_out, sel_n, score, rkey);
+    attn_refine_kernel<GRP><<<dim3(nblk, Hkv), kRefThreads, 0, s>>>(q, kv->k_res, k_ref, uslot, kv->k_scale,
+                                                                   kv->k_zero, T, S, cap, sel_out, sel_n, score,
+                                                                   rkey, umask, L.words_t);
     st = sf::check_launch("attn_refine_kernel");
     if (st != SF_OK) return st;
   }
   dim3 gb(L.splits, Hkv);
   SF_CHECK_CUDA(cudaFuncSetAttribute(attn_out_kernel<GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(OutCfg<GRP>::smem)));
-  attn_out_kernel<GRP><<<gb, kOutThreads, OutCfg<GRP>::smem, s>>>(kv->v_res, kv->v_ref, kv->v_scale, kv->v_zero, T,
-                                                                 S, L.tps, L.words_t, L.splits, score, mkey, rkey,
+  attn_out_kernel<GRP><<<gb, kOutThreads, OutCfg<GRP>::smem, s>>>(kv->v_res, v_ref, uslot, kv->v_scale, kv->v_zero,
+                                                                 T, S, L.tps, L.words_t, L.splits, score, mkey, rkey,
                                                                  umask, part, done, out);
-  return sf::check_launch("attn_out_kernel");
+  st = sf::check_launch("attn_out_kernel");
+  if (st != SF_OK) return st;
+  if (kv->ref_cache) return sf::cache_mark_used(kv->ref_cache, s);
+  return SF_OK;
 }
 
 std::atomic<int> g_attn_path{SF_ATTN_AUTO};
@@ -1190,7 +1231,9 @@ std::atomic<int> g_attn_path{SF_ATTN_AUTO};
 sf_status dispatch(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k, int32_t* sel_out,
                    int32_t* sel_n, float* out, char* ws, const Layout& L, cudaStream_t s) {
   const int path = g_attn_path.load(std::memory_order_relaxed);
-  if (path != SF_ATTN_PIPELINE) {
+  if (path == SF_ATTN_CLUSTER && kv->ref_cache)
+    return sf::fail(SF_ENOTIMPL, "sf_attn_decode_refine: the cluster kernel does not read a ref_cache");
+  if (path != SF_ATTN_PIPELINE && !kv->ref_cache) {
     if (sf::attn_fused_eligible(Hq, Hkv, T))
       return sf::attn_fused_run(q, Hq, Hkv, T, kv, k, sel_out, sel_n, out, reinterpret_cast<double*>(ws + L.kap),
                                 reinterpret_cast<int32_t*>(ws + L.cand), reinterpret_cast<int32_t*>(ws + L.sel),
@@ -1229,8 +1272,8 @@ extern "C" sf_status sf_attn_decode_refine(const uint16_t* q, int Hq, int Hkv, i
                                            int k_tokens, int32_t* sel_out, int32_t* sel_n, float* out,
                                            void* workspace, size_t ws_bytes, sf_stream_t stream) {
   SF_REQUIRE(q && kv && sel_out && sel_n && out && workspace, "sf_attn_decode_refine: null pointer");
-  SF_REQUIRE(kv->k_res && kv->k_ref && kv->v_res && kv->v_ref && kv->k_scale && kv->k_zero && kv->v_scale &&
-                 kv->v_zero,
+  SF_REQUIRE(kv->k_res && kv->v_res && kv->k_scale && kv->k_zero && kv->v_scale && kv->v_zero &&
+                 (kv->ref_cache || (kv->k_ref && kv->v_ref)),
              "sf_attn_decode_refine: null K/V view");
   SF_REQUIRE(kv->b_r == 2 && kv->b_f == 2, "sf_attn_decode_refine: only 2-bit resident + 2-bit refinement K/V");
   SF_REQUIRE(d == D, "sf_attn_decode_refine: head dim must be %d", D);
@@ -1248,6 +1291,42 @@ extern "C" sf_status sf_attn_decode_refine(const uint16_t* q, int Hq, int Hkv, i
              "sf_attn_decode_refine: Hq/Hkv must be 1, 2, 4 or 8");
   return dispatch(q, Hq, Hkv, T, kv, k_tokens, sel_out, sel_n, out, static_cast<char*>(workspace), L,
                   sf::as_cuda(stream));
+}
+
+// ---- units of a KV refinement cache selected by one call -----------------------
+
+namespace {
+
+__global__ void union_units_kernel(const int32_t* __restrict__ sel_out, const int32_t* __restrict__ sel_n, int Hkv,
+                                   int cap, int S, int32_t* __restrict__ units, int32_t* __restrict__ n_units) {
+  __shared__ int off[65];
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int g = 0; g < Hkv; ++g) {
+      off[g] = acc;
+      const int n = sel_n[g];
+      acc += min(cap, n >= 0 ? n : -1 - n);
+    }
+    off[Hkv] = acc;
+    *n_units = acc;
+  }
+  __syncthreads();
+  for (int g = 0; g < Hkv; ++g) {
+    const int n = off[g + 1] - off[g];
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+      units[off[g] + i] = g * S + sel_out[static_cast<size_t>(g) * cap + i];
+  }
+}
+
+}  // namespace
+
+extern "C" sf_status sf_attn_union_units(const int32_t* sel_out, const int32_t* sel_n, int Hkv, int cap, int S,
+                                         int32_t* units, int32_t* n_units, sf_stream_t stream) {
+  SF_REQUIRE(sel_out && sel_n && units && n_units, "sf_attn_union_units: null pointer");
+  SF_REQUIRE(Hkv >= 1 && Hkv <= 64 && cap >= 1 && S >= 1, "sf_attn_union_units: need Hkv in [1, 64], cap, S >= 1");
+  SF_REQUIRE(static_cast<long long>(Hkv) * S <= 0x7FFFFFFFLL, "sf_attn_union_units: Hkv * S overflows int32");
+  union_units_kernel<<<1, 1024, 0, sf::as_cuda(stream)>>>(sel_out, sel_n, Hkv, cap, S, units, n_units);
+  return sf::check_launch("union_units_kernel");
 }
 
 // ---- refined attention without any device allocation ------------------------
@@ -1297,8 +1376,8 @@ extern "C" sf_status sf_attn_decode_refine_noalloc(const uint16_t* q, int Hq, in
                                                    const sf_qkv* kv, int k_tokens, int32_t* sel_out, int32_t* sel_n,
                                                    float* out, sf_stream_t stream) {
   SF_REQUIRE(q && kv && sel_out && sel_n && out, "sf_attn_decode_refine_noalloc: null pointer");
-  SF_REQUIRE(kv->k_res && kv->k_ref && kv->v_res && kv->v_ref && kv->k_scale && kv->k_zero && kv->v_scale &&
-                 kv->v_zero,
+  SF_REQUIRE(kv->k_res && kv->v_res && kv->k_scale && kv->k_zero && kv->v_scale && kv->v_zero &&
+                 (kv->ref_cache || (kv->k_ref && kv->v_ref)),
              "sf_attn_decode_refine_noalloc: null K/V view");
   SF_REQUIRE(kv->b_r == 2 && kv->b_f == 2, "sf_attn_decode_refine_noalloc: only 2-bit resident + 2-bit refinement K/V");
   SF_REQUIRE(d == D, "sf_attn_decode_refine_noalloc: head dim must be %d", D);

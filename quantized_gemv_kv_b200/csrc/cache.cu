@@ -29,13 +29,17 @@ constexpr int kIndexThreads = 1024;
 constexpr int kGatherThreads = 128;
 
 enum Meta { kOcc = 0, kStep, kHits, kMisses, kBypass, kGather, kMetaCount };
-enum Stat { kStSteps = 0, kStHits, kStMisses, kStBypass, kStBytes, kStatCount };
+enum Stat { kStSteps = 0, kStHits, kStMisses, kStBypass, kStBytes, kStLate, kStatCount };
+
+// Largest capacity: the index step keeps one byte per slot in shared memory.
+constexpr int kMaxCapacity = 196608;
 
 // Everything one cache step touches on the device.
 struct CacheDev {
   const int32_t* S;      // selection (ascending units)
   const int32_t* n_ptr;  // its length
   int max_select, capacity;
+  int budget;            // misses fetched per step at most (the rest are late)
   int64_t unit_bytes;
   int32_t *unit_slot, *slot_unit, *order, *order_tmp, *row_of, *hits_out, *misses_out, *bypass_out, *victim_unit,
       *victim_slot, *gather_unit, *gather_row, *meta;
@@ -93,8 +97,9 @@ __device__ void cache_step(const CacheDev& d) {
     }
   }
   const int mi = n - H;
+  const int fetch = min(mi, d.budget);  // the misses after these are late: not fetched, not cached
   const int avail = capacity - H;
-  const int ins = min(mi, avail);
+  const int ins = min(fetch, avail);
   const int use_free = min(ins, capacity - occ);
   const int v = ins - use_free;
 
@@ -115,8 +120,8 @@ __device__ void cache_step(const CacheDev& d) {
   }
   __syncthreads();
 
-  // 3. place the misses: free slots first, then victims, then bypass rows
-  for (int r = tid; r < mi; r += kIndexThreads) {
+  // 3. place the fetched misses: free slots first, then victims, then bypass rows
+  for (int r = tid; r < fetch; r += kIndexThreads) {
     const int u = misses_out[r];
     int row;
     if (r < use_free) {
@@ -144,7 +149,7 @@ __device__ void cache_step(const CacheDev& d) {
       // in ascending order, so compare with the miss list entry at rank mm
       const bool is_miss = (mm < mi) && (misses_out[mm] == u);
       if (is_miss) {
-        row_of[p] = gather_row[mm];
+        row_of[p] = mm < fetch ? gather_row[mm] : -1;
         if (mm < ins) ++touched;
         ++mm;
       } else {
@@ -174,13 +179,14 @@ __device__ void cache_step(const CacheDev& d) {
     meta[kStep] += 1;
     meta[kHits] = H;
     meta[kMisses] = mi;
-    meta[kBypass] = mi - ins;
-    meta[kGather] = mi;
+    meta[kBypass] = fetch - ins;
+    meta[kGather] = fetch;
     stats[kStSteps] += 1;
     stats[kStHits] += H;
     stats[kStMisses] += mi;
-    stats[kStBypass] += mi - ins;
-    stats[kStBytes] += static_cast<int64_t>(mi) * unit_bytes;
+    stats[kStBypass] += fetch - ins;
+    stats[kStBytes] += static_cast<int64_t>(fetch) * unit_bytes;
+    stats[kStLate] += mi - fetch;
   }
 }
 
@@ -293,6 +299,7 @@ struct sf_refine_cache {
   size_t unit_bytes = 0;
   int capacity = 0;
   int max_select = 0;
+  int budget = 0;  // per-step fetch limit; max_select = no limit
   const void* host_master = nullptr;
   const void* master_dev = nullptr;
   bool registered_here = false;
@@ -316,6 +323,7 @@ CacheDev make_dev(const sf_refine_cache* c, const int32_t* S, const int32_t* n) 
   d.n_ptr = n;
   d.max_select = c->max_select;
   d.capacity = c->capacity;
+  d.budget = c->budget;
   d.unit_bytes = static_cast<int64_t>(c->unit_bytes);
   d.unit_slot = c->unit_slot;
   d.slot_unit = c->slot_unit;
@@ -383,6 +391,12 @@ sf_status wait_ready(sf_refine_cache* c) {
 namespace sf {
 
 sf_status cache_view_for_gemv(sf_refine_cache* c, cudaStream_t stream, CacheView* v) {
+  SF_REQUIRE(c->budget >= c->max_select,
+             "sf_gemv_refine: a GEMV needs every selected column fetched; this cache has a fetch budget");
+  return cache_view_for_reader(c, stream, v);
+}
+
+sf_status cache_view_for_reader(sf_refine_cache* c, cudaStream_t stream, CacheView* v) {
   if (c->ready_pending) {
     const unsigned long long cid = capture_id(stream);
     SF_REQUIRE(cid == c->ready_capture,
@@ -392,8 +406,22 @@ sf_status cache_view_for_gemv(sf_refine_cache* c, cudaStream_t stream, CacheView
   }
   v->rows = c->rows;
   v->row_of = c->row_of;
+  v->unit_slot = c->unit_slot;
+  v->num_units = c->num_units;
   v->unit_words = static_cast<int>(c->unit_bytes / 4);
   v->max_select = c->max_select;
+  return SF_OK;
+}
+
+sf_status cache_view_for_writer(sf_refine_cache* c, cudaStream_t stream, CacheWriteView* w) {
+  CacheView v{};
+  const sf_status st = cache_view_for_reader(c, stream, &v);
+  if (st != SF_OK) return st;
+  w->master = static_cast<uint32_t*>(const_cast<void*>(c->master_dev));
+  w->rows = c->rows;
+  w->unit_slot = c->unit_slot;
+  w->num_units = c->num_units;
+  w->unit_words = static_cast<int>(c->unit_bytes / 4);
   return SF_OK;
 }
 
@@ -414,8 +442,8 @@ sf_status sf_refine_cache_create(sf_refine_cache** out, int num_units, size_t un
   *out = nullptr;
   SF_REQUIRE(num_units >= 1, "sf_refine_cache_create: num_units must be >= 1");
   SF_REQUIRE(unit_bytes >= 16 && unit_bytes % 16 == 0, "sf_refine_cache_create: unit_bytes must be a positive multiple of 16");
-  SF_REQUIRE(capacity >= 0 && capacity <= num_units && capacity <= 65536,
-             "sf_refine_cache_create: capacity must be in [0, min(num_units, 65536)]");
+  SF_REQUIRE(capacity >= 0 && capacity <= num_units && capacity <= kMaxCapacity,
+             "sf_refine_cache_create: capacity must be in [0, min(num_units, %d)]", kMaxCapacity);
   SF_REQUIRE(max_select >= 1 && max_select <= 1 << 20, "sf_refine_cache_create: max_select out of range");
   SF_REQUIRE(sf::aligned(host_master, 16), "sf_refine_cache_create: host_master must be 16-byte aligned");
   DeviceGuard g(device);
@@ -425,6 +453,7 @@ sf_status sf_refine_cache_create(sf_refine_cache** out, int num_units, size_t un
   c->unit_bytes = unit_bytes;
   c->capacity = capacity;
   c->max_select = max_select;
+  c->budget = max_select;
   c->host_master = host_master;
   const size_t master_bytes = static_cast<size_t>(num_units) * unit_bytes;
 
@@ -513,6 +542,8 @@ sf_status sf_refine_cache_prefetch(sf_refine_cache* c, const int32_t* idx, const
   if (c->used_pending && c->used_capture == cid) SF_CHECK_CUDA(cudaStreamWaitEvent(ss, c->ev_used, 0));
   const size_t smem = std::max(c->capacity, 1);
   const CacheDev d = make_dev(c, idx, n);
+  SF_CHECK_CUDA(cudaFuncSetAttribute(cache_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem)));
   cache_index_kernel<<<1, kIndexThreads, smem, ss>>>(d);
   sf_status st = sf::check_launch("cache_index_kernel");
   if (st != SF_OK) return st;
@@ -568,6 +599,7 @@ sf_status sf_refine_cache_stats(sf_refine_cache* c, sf_cache_stats* out) {
   out->misses = s[kStMisses];
   out->bypass = s[kStBypass];
   out->h2d_bytes = s[kStBytes];
+  out->late = s[kStLate];
   return SF_OK;
 }
 
@@ -585,6 +617,13 @@ sf_status sf_refine_cache_reset(sf_refine_cache* c) {
 }
 
 sf_status sf_refine_cache_destroy(sf_refine_cache* c) { return cache_free(c); }
+
+sf_status sf_refine_cache_set_budget(sf_refine_cache* c, int budget) {
+  SF_REQUIRE(c, "sf_refine_cache_set_budget: null cache");
+  SF_REQUIRE(budget >= -1, "sf_refine_cache_set_budget: budget must be >= 0, or -1 for none");
+  c->budget = budget < 0 || budget > c->max_select ? c->max_select : budget;
+  return SF_OK;
+}
 
 // ---- groups: one index launch and one gather launch for several caches ----
 
@@ -644,6 +683,8 @@ sf_status sf_refine_group_prefetch(sf_refine_group* grp, sf_stream_t producer, s
   SF_CHECK_CUDA(cudaStreamWaitEvent(ss, grp->ev_idx, 0));
   for (sf_refine_cache* c : grp->caches)
     if (c->used_pending && c->used_capture == cid) SF_CHECK_CUDA(cudaStreamWaitEvent(ss, c->ev_used, 0));
+  SF_CHECK_CUDA(cudaFuncSetAttribute(cache_index_many_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     grp->max_capacity));
   cache_index_many_kernel<<<grp->count, kIndexThreads, grp->max_capacity, ss>>>(grp->table);
   sf_status st = sf::check_launch("cache_index_many_kernel");
   if (st != SF_OK) return st;

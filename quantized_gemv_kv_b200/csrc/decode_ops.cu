@@ -72,6 +72,11 @@ __global__ void rope_kernel(float* __restrict__ x, int d, int pos, double theta,
   }
 }
 
+__global__ void round_bf16_kernel(const float* __restrict__ x, int n, uint16_t* __restrict__ y) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    y[i] = __bfloat16_as_ushort(__float2bfloat16_rn(x[i]));
+}
+
 __global__ void silu_mul_kernel(const float* __restrict__ g, const float* __restrict__ u, int n,
                                 uint16_t* __restrict__ y) {
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
@@ -87,8 +92,13 @@ constexpr int kAppendMaxD = 512;
 // fp16 scale, integer zero point, ties to even) and written as cache row
 // g * row_stride + t: resident and refinement bitstreams (row-major, little
 // endian), fp16 scale and zero.
+// The refinement words go to ref + r * ref_pitch + ref_off (the store:
+// pitch d*b_f/32, offset 0; a KV refinement cache's host master: the unit's
+// pitch and the K or V half).  When unit_slot is given and unit r is cached,
+// the same words also go to its cache row, so a cached copy never goes stale.
 __global__ void kv_append_kernel(const float* __restrict__ src, int Hkv, int d, int row_stride, int t, int b_r,
-                                 int b_f, uint32_t* __restrict__ res, uint32_t* __restrict__ ref,
+                                 int b_f, uint32_t* __restrict__ res, uint32_t* __restrict__ ref, int ref_pitch,
+                                 int ref_off, const int32_t* __restrict__ unit_slot, uint32_t* __restrict__ crows,
                                  uint16_t* __restrict__ scale, uint16_t* __restrict__ zero) {
   __shared__ uint8_t codes[4][kAppendMaxD];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -145,7 +155,11 @@ __global__ void kv_append_kernel(const float* __restrict__ src, int Hkv, int d, 
       const int sb = ww * 32 + bit;
       word |= ((static_cast<uint32_t>(codes[warp][sb / b_f]) & fmask) >> (sb % b_f) & 1u) << bit;
     }
-    ref[r * fw + ww] = word;
+    ref[r * ref_pitch + ref_off + ww] = word;
+    if (unit_slot != nullptr) {
+      const int slot = unit_slot[r];
+      if (slot >= 0) crows[static_cast<size_t>(slot) * ref_pitch + ref_off + ww] = word;
+    }
   }
 }
 
@@ -176,6 +190,14 @@ extern "C" sf_status sf_silu_mul(const float* g, const float* u, int n, uint16_t
   return sf::check_launch("silu_mul_kernel");
 }
 
+extern "C" sf_status sf_round_bf16(const float* x, int n, uint16_t* y, sf_stream_t stream) {
+  SF_REQUIRE(x && y, "sf_round_bf16: null pointer");
+  SF_REQUIRE(n >= 1, "sf_round_bf16: n must be >= 1");
+  const int blocks = std::min((n + 255) / 256, sf::sm_count() * 8);
+  round_bf16_kernel<<<blocks, 256, 0, sf::as_cuda(stream)>>>(x, n, y);
+  return sf::check_launch("round_bf16_kernel");
+}
+
 extern "C" sf_status sf_kv_append(const float* src, int Hkv, int d, int row_stride, int t, int b_r, int b_f,
                                   uint32_t* res, uint32_t* ref, uint16_t* scale, uint16_t* zero, sf_stream_t stream) {
   SF_REQUIRE(src && res && ref && scale && zero, "sf_kv_append: null pointer");
@@ -187,7 +209,35 @@ extern "C" sf_status sf_kv_append(const float* src, int Hkv, int d, int row_stri
   SF_REQUIRE(b_r + b_f <= 4, "sf_kv_append: b_r + b_f must be <= 4");
   SF_REQUIRE(row_stride >= 1 && t >= 0 && t < row_stride, "sf_kv_append: need 0 <= t < row_stride");
   kv_append_kernel<<<(Hkv + 3) / 4, 128, 0, sf::as_cuda(stream)>>>(src, Hkv, d, row_stride, t, b_r, b_f, res, ref,
-                                                                   scale, zero);
+                                                                   d * b_f / 32, 0, nullptr, nullptr, scale, zero);
   return sf::check_launch("kv_append_kernel");
+}
+
+extern "C" sf_status sf_kv_append_cached(const float* src, int Hkv, int d, int row_stride, int t, int b_r, int b_f,
+                                         uint32_t* res, uint16_t* scale, uint16_t* zero, sf_refine_cache* ref_cache,
+                                         int part, sf_stream_t stream) {
+  SF_REQUIRE(src && res && scale && zero && ref_cache, "sf_kv_append_cached: null pointer");
+  SF_REQUIRE(Hkv >= 1, "sf_kv_append_cached: Hkv must be >= 1");
+  SF_REQUIRE(d >= 32 && d % 32 == 0 && d <= kAppendMaxD,
+             "sf_kv_append_cached: d must be a multiple of 32 in [32, %d]", kAppendMaxD);
+  SF_REQUIRE(b_r == 2 || b_r == 3, "sf_kv_append_cached: b_r must be 2 or 3");
+  SF_REQUIRE(b_f == 1 || b_f == 2, "sf_kv_append_cached: b_f must be 1 or 2");
+  SF_REQUIRE(b_r + b_f <= 4, "sf_kv_append_cached: b_r + b_f must be <= 4");
+  SF_REQUIRE(row_stride >= 1 && t >= 0 && t < row_stride, "sf_kv_append_cached: need 0 <= t < row_stride");
+  SF_REQUIRE(part == 0 || part == 1, "sf_kv_append_cached: part must be 0 (K) or 1 (V)");
+  cudaStream_t s = sf::as_cuda(stream);
+  sf::CacheWriteView w{};
+  sf_status st = sf::cache_view_for_writer(ref_cache, s, &w);
+  if (st != SF_OK) return st;
+  const int fw = d * b_f / 32;
+  SF_REQUIRE(w.unit_words == 2 * fw, "sf_kv_append_cached: the cache's units must be %d bytes (K then V words)",
+             8 * fw);
+  SF_REQUIRE(static_cast<long long>(w.num_units) >= static_cast<long long>(Hkv) * row_stride,
+             "sf_kv_append_cached: the cache has fewer units than Hkv * row_stride");
+  kv_append_kernel<<<(Hkv + 3) / 4, 128, 0, s>>>(src, Hkv, d, row_stride, t, b_r, b_f, res, w.master, 2 * fw,
+                                                 part * fw, w.unit_slot, w.rows, scale, zero);
+  st = sf::check_launch("kv_append_kernel");
+  if (st != SF_OK) return st;
+  return sf::cache_mark_used(ref_cache, s);
 }
 

@@ -26,10 +26,23 @@
 // sums onto a zeroed output (two terms onto zero: the result does not depend
 // on their order).
 //
-// Each warp streams its own codes (16 rows x 64 bytes per slice, 16-byte
-// chunks XOR-swizzled so the fragment loads are free of bank conflicts),
+// Each warp streams its own codes (16 rows x 64 or 96 bytes per slice; the
+// 2-bit rows' 16-byte chunks XOR-swizzled, the 3-bit rows' 24-word stride
+// already conflict-free, so the fragment loads never collide on a bank),
 // scale/zero and refinement words through a cp.async ring in shared memory
 // and waits only for its own copies.
+//
+// 3-bit resident codes are read from a split layout written once by
+// sf_gemv_pack_batch1 (a 3-bit code straddles bytes in the canonical
+// bitstream, so it cannot become an A-fragment byte with one shift and one
+// mask).  Per row and 256-channel slice, 24 words:
+//   words 0-15  the low 2 bits of the codes, arranged as 2-bit codes are
+//               (word w, byte b, bits 2j..2j+1: channel 16 w + 4 b + j);
+//   words 16-23 the high bits: word 16 + 2 t + slot covers the low words
+//               8 slot + 2 t + h (h = 0, 1), bit 4 h + j of its byte b holding
+//               the high bit of channel 16 (8 slot + 2 t + h) + 4 b + j.
+// A fragment byte is then ((w >> 2j) & 0x03030303) | (high bit moved to bit
+// 2 of each byte): two shifts and two logic operations per register.
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -43,10 +56,12 @@ constexpr int kMaxJobs = 4;
 constexpr int kRows = 16;          // output rows per tile
 constexpr int kMaxWarps = 16;      // warps per CTA
 constexpr int kCorrList = 32;      // selected channels per slice handled on the tensor cores
-constexpr int kSliceWords = 256 + 32 + 32;  // words per slice and stage: codes, scale/zero, refinement
+// selected x at or above this magnitude would overflow the f16 (high, low)
+// split of the correction MMA: such a slice takes the fp32 correction loop
+constexpr float kCorrXMax = 32768.0f;
 
 struct MJob {
-  const uint32_t* res;
+  const uint32_t* res;       // resident codes in the batch-1 layout
   const uint16_t* scale;
   const uint16_t* zero;
   const uint32_t* ref_rows;  // nullptr: resident only
@@ -104,10 +119,22 @@ __device__ __forceinline__ int job_of(const MArgs& a, int t) {
   return jb;
 }
 
-// Word offset of 16-byte chunk c (0..3) of staged code row r (64 bytes a row):
-// rows 2, 3 (mod 4) swap chunk pairs, so the rows read by one half-warp's
-// 8-byte fragment loads fall on distinct banks.
-__device__ __forceinline__ int code_off(int r, int c) { return r * 16 + ((c ^ (((r >> 1) & 1) << 1)) << 2); }
+// Word offset of 16-byte chunk c of staged code row r.  2-bit rows (64 bytes,
+// chunks 0..3): rows 2, 3 (mod 4) swap chunk pairs, so the rows read by one
+// half-warp's 8-byte fragment loads fall on distinct banks.  3-bit rows (96
+// bytes, chunks 0..5): a 24-word row stride already spreads them.
+template <int BR>
+__device__ __forceinline__ int code_off(int r, int c) {
+  if constexpr (BR == 2) return r * 16 + ((c ^ (((r >> 1) & 1) << 1)) << 2);
+  else return r * 24 + 4 * c;
+}
+
+// Bit s of every byte of h moved to bit 2 (the high bit of a 3-bit code).
+template <int S>
+__device__ __forceinline__ uint32_t hi_bit(uint32_t h) {
+  if constexpr (S >= 2) return (h >> (S - 2)) & 0x04040404u;
+  else return (h << (2 - S)) & 0x04040404u;
+}
 
 // f16 (1024 + q_f) pairs for rows g8 (lo_row) / g8 + 8 (hi_row) of two
 // channels whose refinement words are wa, wb (bits b_f*r + off hold row r).
@@ -126,9 +153,14 @@ __device__ __forceinline__ void qf_frag(uint32_t wa, uint32_t wb, int g8, int of
   }
 }
 
-template <int SPW>
+template <int SPW, int BR>
 struct MCfg {
-  static constexpr int kStages = SPW == 1 ? 8 : 5;  // 16 warps of two slices fit 227 KB
+  static constexpr int kCodeWords = 128 * BR;              // 16 rows x 8 BR words
+  static constexpr int kSZ = kCodeWords;                   // scale/zero: 32 words
+  static constexpr int kRF = kCodeWords + 32;              // refinement: 32 words
+  static constexpr int kSliceWords = kCodeWords + 64;      // words per slice and stage
+  // 16 warps (14 of two slices) fit 227 KB
+  static constexpr int kStages = SPW == 1 ? (BR == 2 ? 8 : 7) : (BR == 2 ? 5 : 4);
   static constexpr int kRedTiles = SPW == 1 ? 16 : 4;  // tiles whose warp partials wait for one reduction
   static constexpr int SW = SPW * kSliceWords;  // ring words per warp and stage
   static size_t smem_bytes(int W) {
@@ -138,11 +170,12 @@ struct MCfg {
   }
 };
 
-template <int SPW, int BF>
+template <int SPW, int BF, int BR>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1)
 gemv_mma_kernel(const __grid_constant__ MArgs a) {
-  using C = MCfg<SPW>;
+  using C = MCfg<SPW, BR>;
   constexpr int kStages = C::kStages, SW = C::SW, kRedTiles = C::kRedTiles;
+  constexpr int kSliceWords = C::kSliceWords, kSZ = C::kSZ, kRF = C::kRF;
   extern __shared__ __align__(16) uint32_t sm[];
   const int W = blockDim.x >> 5;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, tig = lane & 3;
@@ -157,7 +190,7 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
   const float m_f = static_cast<float>((1 << BF) - 1) * 0.5f;
   const uint32_t fmask = (1u << BF) - 1u;
 
-  const size_t row_words = static_cast<size_t>(a.K) / 16;
+  const size_t row_words = static_cast<size_t>(a.K) * BR / 32;
   const int last = a.njobs - 1;
   const int total_tiles = a.job[last].tile_begin + a.job[last].N / kRows;
   // a contiguous block of tiles per CTA: consecutive tiles read consecutive
@@ -170,22 +203,32 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
   uint32_t cb[SPW][2][2];
   float fsc[SPW], gsm[SPW], cconst[SPW];
   int nsl[SPW], psl[SPW];
+  int ntc[SPW];  // selected channels of the slice corrected on the tensor cores (the rest in fp32)
 
   // Copies are issued tile by tile in order, so their addresses advance by
   // fixed strides and are recomputed only where the next matrix begins.
   // Code cursor: codes and scale/zero (they depend on nothing the previous
   // kernel writes); ref cursor: the refinement words of the listed channels.
-  const int crow_l = lane >> 2, cchunk = lane & 3;
+  // this lane's BR code chunks of a tile's slice: chunk lane + 32 i of the
+  // slice's 16 rows x 2 BR chunks
+  int c_soff[BR];      // word offset in the stage
+  size_t c_goff[BR];   // word offset from the tile's first row in the matrix
+#pragma unroll
+  for (int i = 0; i < BR; ++i) {
+    const int c = lane + 32 * i, r = c / (2 * BR), ch = c % (2 * BR);
+    c_soff[i] = code_off<BR>(r, ch);
+    c_goff[i] = static_cast<size_t>(r) * row_words + 4 * ch;
+  }
   const int sz_grp = lane >> 2, sz_arr = (lane >> 1) & 1, sz_hf = lane & 1;  // lanes 0-7
   int c_t = t_begin, c_jb = my_tiles > 0 ? job_of(a, t_begin) : 0, c_next = 0;
-  const uint32_t* c_code = nullptr;  // row (row0 + crow_l) of slice0, this lane's chunk
+  const uint32_t* c_code = nullptr;  // the tile's first row, slice0
   const uint16_t* c_sz = nullptr;    // lanes 0-7: scale or zero of (slice0, group), rows row0 + 8 hf
   size_t c_szs = 0;                  // elements between consecutive slices' scale rows
   auto c_seek = [&]() {              // the cursor's tile starts (or the job changes)
     const MJob& J = a.job[c_jb];
     const int row0 = (c_t - J.tile_begin) * kRows;
     c_next = c_jb + 1 < a.njobs ? a.job[c_jb + 1].tile_begin : 0x7FFFFFFF;
-    c_code = J.res + static_cast<size_t>(row0 + crow_l) * row_words + 16 * slice0 + 4 * cchunk;
+    c_code = J.res + static_cast<size_t>(row0) * row_words + 8 * BR * slice0;
     c_szs = 2 * static_cast<size_t>(J.N);
     c_sz = (sz_arr ? J.zero : J.scale) + static_cast<size_t>(2 * slice0 + sz_grp) * J.N + row0 + 8 * sz_hf;
   };
@@ -200,10 +243,10 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
 #pragma unroll
     for (int sp = 0; sp < SPW; ++sp) {
       uint32_t* base = stage + sp * kSliceWords;
-      cp_async16(base + code_off(crow_l, cchunk), c_code + 16 * sp);
-      cp_async16(base + code_off(crow_l + 8, cchunk), c_code + 8 * row_words + 16 * sp);
+#pragma unroll
+      for (int q = 0; q < BR; ++q) cp_async16(base + c_soff[q], c_code + c_goff[q] + 8 * BR * sp);
       if (lane < 8)
-        cp_async16(reinterpret_cast<uint16_t*>(base + 256) + (sz_grp * 2 + sz_arr) * 16 + 8 * sz_hf,
+        cp_async16(reinterpret_cast<uint16_t*>(base + kSZ) + (sz_grp * 2 + sz_arr) * 16 + 8 * sz_hf,
                    c_sz + sp * c_szs);
     }
     c_code += kRows * row_words;
@@ -221,7 +264,7 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
 #pragma unroll
     for (int sp = 0; sp < SPW; ++sp) {
       r_row[sp] = J.ref_rows;
-      if (r_has && lane < min(nsl[sp], kCorrList)) {
+      if (r_has && lane < ntc[sp]) {
         const int rr = J.row_of ? J.row_of[psl[sp] + lane] : 256 * (slice0 + sp) + mylist[sp * kCorrList + lane];
         r_row[sp] = J.ref_rows + static_cast<size_t>(rr) * J.unit_words;
       }
@@ -237,7 +280,7 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
       uint32_t* stage = ring + (i % kStages) * SW;
 #pragma unroll
       for (int sp = 0; sp < SPW; ++sp)
-        if (lane < min(nsl[sp], kCorrList)) cp_async4(stage + sp * kSliceWords + 288 + lane, r_row[sp] + woff);
+        if (lane < ntc[sp]) cp_async4(stage + sp * kSliceWords + kRF + lane, r_row[sp] + woff);
     }
     ++r_t;
   };
@@ -282,12 +325,17 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
       }
     }
     __syncwarp();
-    const int nl = min(nsl[sp], kCorrList);
+    int nl = min(nsl[sp], kCorrList);
+    float xv = 0.0f;
+    if (lane < nl) xv = sfd::bf16_bits_to_float(a.x[256 * slice + mylist[sp * kCorrList + lane]]);
+    // a listed |x| at or above 2^15 would overflow the f16 split: the whole
+    // slice is then corrected by the fp32 loop
+    if (__any_sync(0xffffffffu, !(fabsf(xv) < kCorrXMax))) nl = 0;
+    ntc[sp] = nl;
     uint32_t hl = 0;  // lane k: (high, low) halves of x of listed channel k
     int grp = -1;     // and its group inside the slice
     if (lane < nl) {
       const int ch = mylist[sp * kCorrList + lane];
-      const float xv = sfd::bf16_bits_to_float(a.x[256 * slice + ch]);
       const __half hi = __float2half_rn(xv);
       const __half lo = __float2half_rn(xv - __half2float(hi));
       hl = static_cast<uint32_t>(__half_as_ushort(hi)) | (static_cast<uint32_t>(__half_as_ushort(lo)) << 16);
@@ -357,21 +405,37 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
 #pragma unroll
     for (int sp = 0; sp < SPW; ++sp) {
       const uint32_t* base = ring + st * SW + sp * kSliceWords;
-      // code words: rows g8 and g8 + 8, words 2 tig, 2 tig + 1 of each group
-      const uint2 r0a = *reinterpret_cast<const uint2*>(base + code_off(g8, tig >> 1) + 2 * (tig & 1));
-      const uint2 r0b = *reinterpret_cast<const uint2*>(base + code_off(g8, 2 + (tig >> 1)) + 2 * (tig & 1));
-      const uint2 r1a = *reinterpret_cast<const uint2*>(base + code_off(g8 + 8, tig >> 1) + 2 * (tig & 1));
-      const uint2 r1b = *reinterpret_cast<const uint2*>(base + code_off(g8 + 8, 2 + (tig >> 1)) + 2 * (tig & 1));
+      // (low) code words: rows g8 and g8 + 8, words 2 tig, 2 tig + 1 of each group
+      const uint2 r0a = *reinterpret_cast<const uint2*>(base + code_off<BR>(g8, tig >> 1) + 2 * (tig & 1));
+      const uint2 r0b = *reinterpret_cast<const uint2*>(base + code_off<BR>(g8, 2 + (tig >> 1)) + 2 * (tig & 1));
+      const uint2 r1a = *reinterpret_cast<const uint2*>(base + code_off<BR>(g8 + 8, tig >> 1) + 2 * (tig & 1));
+      const uint2 r1b = *reinterpret_cast<const uint2*>(base + code_off<BR>(g8 + 8, 2 + (tig >> 1)) + 2 * (tig & 1));
+      // 3-bit: the high-bit words of both groups (.x group 0, .y group 1)
+      uint2 h0 = make_uint2(0u, 0u), h1 = make_uint2(0u, 0u);
+      if constexpr (BR == 3) {
+        h0 = *reinterpret_cast<const uint2*>(base + g8 * 24 + 16 + 2 * tig);
+        h1 = *reinterpret_cast<const uint2*>(base + (g8 + 8) * 24 + 16 + 2 * tig);
+      }
       int d[4] = {0, 0, 0, 0}, e[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
         const int slot = m >> 2, hi = (m >> 1) & 1, j = 2 * (m & 1);
         const uint32_t w0 = slot ? (hi ? r0b.y : r0b.x) : (hi ? r0a.y : r0a.x);
         const uint32_t w1 = slot ? (hi ? r1b.y : r1b.x) : (hi ? r1a.y : r1a.x);
-        const uint32_t a0 = (w0 >> (2 * j)) & 0x03030303u;
-        const uint32_t a1 = (w1 >> (2 * j)) & 0x03030303u;
-        const uint32_t a2 = (w0 >> (2 * j + 2)) & 0x03030303u;
-        const uint32_t a3 = (w1 >> (2 * j + 2)) & 0x03030303u;
+        uint32_t a0 = (w0 >> (2 * j)) & 0x03030303u;
+        uint32_t a1 = (w1 >> (2 * j)) & 0x03030303u;
+        uint32_t a2 = (w0 >> (2 * j + 2)) & 0x03030303u;
+        uint32_t a3 = (w1 >> (2 * j + 2)) & 0x03030303u;
+        if constexpr (BR == 3) {
+          const uint32_t x0 = slot ? h0.y : h0.x, x1 = slot ? h1.y : h1.x;
+          // channel offset j (j + 1) of low word `hi`: bit 4 hi + j (+ 1)
+          switch (4 * hi + j) {
+            case 0: a0 |= hi_bit<0>(x0); a1 |= hi_bit<0>(x1); a2 |= hi_bit<1>(x0); a3 |= hi_bit<1>(x1); break;
+            case 2: a0 |= hi_bit<2>(x0); a1 |= hi_bit<2>(x1); a2 |= hi_bit<3>(x0); a3 |= hi_bit<3>(x1); break;
+            case 4: a0 |= hi_bit<4>(x0); a1 |= hi_bit<4>(x1); a2 |= hi_bit<5>(x0); a3 |= hi_bit<5>(x1); break;
+            default: a0 |= hi_bit<6>(x0); a1 |= hi_bit<6>(x1); a2 |= hi_bit<7>(x0); a3 |= hi_bit<7>(x1); break;
+          }
+        }
         if (m & 1) mma_u8s8(e, a0, a1, a2, a3, bf[sp][m][0], bf[sp][m][1]);
         else mma_u8s8(d, a0, a1, a2, a3, bf[sp][m][0], bf[sp][m][1]);
       }
@@ -379,19 +443,20 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
       for (int c = 0; c < 4; ++c) d[c] += e[c];
       // even lanes: d0, d1 = planes 0, 1 of row g8 and d2, d3 = planes 0, 1 of
       // row g8 + 8; odd lanes: d0, d2 = plane 2 of rows g8, g8 + 8.  Plane sums
-      // are below 2^17 in magnitude: exact small-integer conversions.
+      // are below 7 * 128 * 128 < 2^17 in magnitude: exact small-integer
+      // conversions.
       const float f0 = i2f_small(d[0]), f1 = i2f_small(d[1]), f2 = i2f_small(d[2]), f3 = i2f_small(d[3]);
       const float send = even ? fmaf(f3, 256.0f, f2) : 65536.0f * f0;
       const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
       const float P = even ? fmaf(f1, 256.0f, f0) + recv : fmaf(65536.0f, f2, recv);
-      const uint16_t* szs = reinterpret_cast<const uint16_t*>(base + 256);
+      const uint16_t* szs = reinterpret_cast<const uint16_t*>(base + kSZ);
       const float sc = h2f_bits(szs[(myslot * 2) * 16 + myrow]);
       const float zz = h2f_bits(szs[(myslot * 2 + 1) * 16 + myrow]);
       float tsum = fmaf(static_cast<float>(1 << BF) * fsc[sp], P, (m_f - zz) * gsm[sp]);
       if (J.ref_rows && nsl[sp] > 0) {
-        const uint32_t* refw = base + 288;
+        const uint32_t* refw = base + kRF;
         float c4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        const int nl = min(nsl[sp], kCorrList);
+        const int nl = ntc[sp];
 #pragma unroll
         for (int kb = 0; kb < 2; ++kb) {
           if (16 * kb < nl) {  // uniform over the warp
@@ -406,9 +471,10 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
         // lane (g8, t), t < 2, holds group t's (high, low) columns for rows g8 and g8 + 8
         const float u0 = __shfl_sync(0xffffffffu, c4[0] + c4[1], 4 * g8 + myslot);
         const float u1 = __shfl_sync(0xffffffffu, c4[2] + c4[3], 4 * g8 + myslot);
-        float corr = ((tig & 1) ? u1 : u0) + cconst[sp];
-        // channels beyond the tensor-core list (more than kCorrList selected in the slice)
-        for (int k = kCorrList; k < nsl[sp]; ++k) {
+        float corr = nl > 0 ? ((tig & 1) ? u1 : u0) + cconst[sp] : 0.0f;
+        // channels beyond the tensor-core list (more than kCorrList selected in
+        // the slice, or every selected channel of a slice with a huge |x|)
+        for (int k = nl; k < nsl[sp]; ++k) {
           const uint32_t* A = a.act + static_cast<size_t>(slice0 + sp) * sfd::kAct2Words;
           int kk = k, ch = -1;
           for (int wdx = 0; wdx < 8 && ch < 0; ++wdx) {
@@ -468,7 +534,55 @@ bool pick_split(int nslice, int* spw, int* ksplit) {
   return false;
 }
 
+
+// Canonical 3-bit rows -> the split batch-1 layout: one thread per (row,
+// 256-channel slice); the slice's 256 codes are 24 whole words in both.
+__global__ void pack_res3_kernel(const uint32_t* __restrict__ res, int nrows, int nslice,
+                                 uint32_t* __restrict__ out) {
+  const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= static_cast<long long>(nrows) * nslice) return;
+  const uint32_t* src = res + e * 24;
+  uint32_t lo[16], hb[8];
+#pragma unroll
+  for (int w = 0; w < 16; ++w) lo[w] = 0u;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) hb[w] = 0u;
+  for (int c = 0; c < 256; ++c) {
+    const int bit = 3 * c, wd = bit >> 5, sh = bit & 31;
+    uint32_t v = src[wd] >> sh;
+    if (sh > 29) v |= src[wd + 1] << (32 - sh);
+    v &= 7u;
+    const int w = c >> 4, b = (c >> 2) & 3, j = c & 3;
+    lo[w] |= (v & 3u) << (8 * b + 2 * j);
+    const int slot = w >> 3, t = (w & 7) >> 1, h = w & 1;
+    hb[2 * t + slot] |= (v >> 2) << (8 * b + 4 * h + j);
+  }
+  uint32_t* dst = out + e * 24;
+#pragma unroll
+  for (int w = 0; w < 16; ++w) dst[w] = lo[w];
+#pragma unroll
+  for (int w = 0; w < 8; ++w) dst[16 + w] = hb[w];
+}
+
 }  // namespace
+
+extern "C" sf_status sf_gemv_pack_batch1(const uint32_t* res, int N, int K, int b_r, uint32_t* out,
+                                         sf_stream_t stream) {
+  SF_REQUIRE(res && out, "sf_gemv_pack_batch1: null pointer");
+  SF_REQUIRE(b_r == 2 || b_r == 3, "sf_gemv_pack_batch1: b_r must be 2 or 3");
+  SF_REQUIRE(N >= 1 && K >= 256 && K % 256 == 0, "sf_gemv_pack_batch1: need N >= 1 and K a positive multiple of 256");
+  cudaStream_t s = sf::as_cuda(stream);
+  const size_t words = static_cast<size_t>(N) * K / 32 * b_r;
+  if (b_r == 2) {
+    if (out != res) SF_CHECK_CUDA(cudaMemcpyAsync(out, res, words * 4, cudaMemcpyDeviceToDevice, s));
+    return SF_OK;
+  }
+  SF_REQUIRE(out != res, "sf_gemv_pack_batch1: the 3-bit layout cannot be written in place");
+  const long long n = static_cast<long long>(N) * (K / 256);
+  const int threads = 128;
+  pack_res3_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0, s>>>(res, N, K / 256, out);
+  return sf::check_launch("pack_res3_kernel");
+}
 
 extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, const uint16_t* x, const void* act,
                                            sf_stream_t stream) {
@@ -477,9 +591,10 @@ extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, c
   SF_REQUIRE(sf::aligned(act, 16) && sf::aligned(x, 4), "sf_gemv_refine_batch1: act must be 16-byte aligned");
   const sf_qweight* W0 = jobs[0].W;
   SF_REQUIRE(W0, "sf_gemv_refine_batch1: null weight");
-  const int K = W0->K, G = W0->G, b_f = W0->b_f;
-  SF_REQUIRE(W0->b_r == 2, "sf_gemv_refine_batch1: 2-bit resident codes only");
+  const int K = W0->K, G = W0->G, b_f = W0->b_f, b_r = W0->b_r;
+  SF_REQUIRE(b_r == 2 || b_r == 3, "sf_gemv_refine_batch1: b_r must be 2 or 3");
   SF_REQUIRE(b_f == 1 || b_f == 2, "sf_gemv_refine_batch1: b_f must be 1 or 2");
+  SF_REQUIRE(b_r + b_f <= 4, "sf_gemv_refine_batch1: b_r + b_f must be at most 4");
   SF_REQUIRE(G == 128, "sf_gemv_refine_batch1: group size must be 128 (the prepared activations' group)");
   SF_REQUIRE(K >= 256 && K % 256 == 0, "sf_gemv_refine_batch1: K must be a positive multiple of 256");
   int spw = 0, ksplit = 0;
@@ -495,14 +610,18 @@ extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, c
   int row_tiles = 0;
   for (int i = 0; i < count; ++i) {
     const sf_qweight* W = jobs[i].W;
-    SF_REQUIRE(W && W->res && W->scale && W->zero && jobs[i].y, "sf_gemv_refine_batch1: job %d incomplete", i);
-    SF_REQUIRE(W->K == K && W->G == G && W->b_f == b_f && W->b_r == 2,
+    SF_REQUIRE(W && W->scale && W->zero && jobs[i].y, "sf_gemv_refine_batch1: job %d incomplete", i);
+    SF_REQUIRE(W->K == K && W->G == G && W->b_f == b_f && W->b_r == b_r,
                "sf_gemv_refine_batch1: jobs must share K, G and bit widths");
+    const uint32_t* res = jobs[i].res_b1 ? jobs[i].res_b1 : W->res;
+    SF_REQUIRE(res, "sf_gemv_refine_batch1: job %d has no resident codes", i);
+    SF_REQUIRE(b_r == 2 || jobs[i].res_b1,
+               "sf_gemv_refine_batch1: 3-bit codes must be given in the batch-1 layout (res_b1, sf_gemv_pack_batch1)");
     SF_REQUIRE(W->N >= kRows && W->N % kRows == 0, "sf_gemv_refine_batch1: N must be a multiple of %d", kRows);
-    SF_REQUIRE(sf::aligned(W->res, 16) && sf::aligned(W->scale, 16) && sf::aligned(W->zero, 16),
+    SF_REQUIRE(sf::aligned(res, 16) && sf::aligned(W->scale, 16) && sf::aligned(W->zero, 16),
                "sf_gemv_refine_batch1: weight arrays must be 16-byte aligned");
     MJob& J = a.job[i];
-    J.res = W->res;
+    J.res = res;
     J.scale = W->scale;
     J.zero = W->zero;
     J.N = W->N;
@@ -534,12 +653,17 @@ extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, c
     return sf::check_launch("gemv_mma_kernel");
   };
   sf_status st;
-  if (spw == 1) {
-    const size_t smem = MCfg<1>::smem_bytes(warps);
-    st = b_f == 2 ? launch(gemv_mma_kernel<1, 2>, smem) : launch(gemv_mma_kernel<1, 1>, smem);
-  } else {
-    const size_t smem = MCfg<2>::smem_bytes(warps);
-    st = b_f == 2 ? launch(gemv_mma_kernel<2, 2>, smem) : launch(gemv_mma_kernel<2, 1>, smem);
+  if (b_r == 2) {
+    if (spw == 1) {
+      const size_t smem = MCfg<1, 2>::smem_bytes(warps);
+      st = b_f == 2 ? launch(gemv_mma_kernel<1, 2, 2>, smem) : launch(gemv_mma_kernel<1, 1, 2>, smem);
+    } else {
+      const size_t smem = MCfg<2, 2>::smem_bytes(warps);
+      st = b_f == 2 ? launch(gemv_mma_kernel<2, 2, 2>, smem) : launch(gemv_mma_kernel<2, 1, 2>, smem);
+    }
+  } else {  // b_r == 3, b_f == 1
+    st = spw == 1 ? launch(gemv_mma_kernel<1, 1, 3>, MCfg<1, 3>::smem_bytes(warps))
+                  : launch(gemv_mma_kernel<2, 1, 3>, MCfg<2, 3>::smem_bytes(warps));
   }
   if (st != SF_OK) return st;
   for (int i = 0; i < count; ++i)

@@ -48,11 +48,30 @@ int sm_count();
 struct CacheView {
   const uint32_t* rows;     // [(capacity + max_select)][unit_words]
   const int32_t* row_of;    // [max_select]
+  const int32_t* unit_slot; // [num_units]: slot of a cached unit, -1 if not cached
+  int num_units;
   int unit_words;
   int max_select;
 };
+// For a GEMV: refuses a cache with a fetch budget (every selected column must
+// be fetched); makes `stream` wait for the last prefetch.
 sf_status cache_view_for_gemv(sf_refine_cache* c, cudaStream_t stream, CacheView* v);
+// For a reader that looks units up by unit_slot (the cached set as the last
+// prefetch left it); makes `stream` wait for that prefetch.
+sf_status cache_view_for_reader(sf_refine_cache* c, cudaStream_t stream, CacheView* v);
 sf_status cache_mark_used(sf_refine_cache* c, cudaStream_t stream);
+
+// For a writer of units (the KV append): the host master's device-mapped
+// address and the device rows, so a new unit's bytes go to both; makes
+// `stream` wait for the last prefetch.
+struct CacheWriteView {
+  uint32_t* master;          // device address of the host master [num_units][unit_words]
+  uint32_t* rows;            // cache rows
+  const int32_t* unit_slot;  // [num_units]
+  int num_units;
+  int unit_words;
+};
+sf_status cache_view_for_writer(sf_refine_cache* c, cudaStream_t stream, CacheWriteView* v);
 
 // Batch-1 2-bit GEMV on the integer dot-product path (gemv_b1.cu).  Returns
 // false when the shape is outside that kernel's range (the caller then runs

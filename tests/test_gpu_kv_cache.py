@@ -1,0 +1,130 @@
+"""GPU parity of refined attention that reads its refinement bits from a KV
+refinement cache (sf_qkv.ref_cache): one cache unit per token-head, the
+deadline reading (only the union tokens cached when the step starts are
+refined; the misses are fetched for later steps, at most a budget per step,
+the rest late), against the oracle's attention with an availability mask and
+its LRU with a fetch budget.
+
+Bit-exact: union sets, cache hit / miss / bypass sets, late counts.
+Tolerance: attention max-abs error <= 2e-3.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attn as oattn
+from oracle import cache as ocache
+from oracle import quant as oquant
+from workloads import count_fraction, gen_kv, gen_query
+
+pytestmark = pytest.mark.gpu
+
+ATTN_TOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def sf():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import quantized_gemv_kv_b200 as sf
+    return sf
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _setup(sf, Hq, Hkv, T, S, d, seed, cap_pct):
+    Kf, Vf, _ = gen_kv(seed, Hkv, S, d)           # S tokens allocated per head, the first T used
+    k = sf.quantize_nested(dev(Kf.reshape(-1, d)), d, 2, 2, "by_row")
+    v = sf.quantize_nested(dev(Vf.reshape(-1, d)), d, 2, 2, "by_row")
+    master = torch.cat([k.ref.view(-1, 8), v.ref.view(-1, 8)], dim=1).cpu().contiguous().pin_memory()
+    k_tokens = count_fraction(1, T)
+    grp = Hq // Hkv
+    cap = count_fraction(cap_pct, Hkv * T)
+    cache = sf.RefineCache(Hkv * S, 64, cap, Hkv * grp * k_tokens, master)
+    k.ref = v.ref = None                            # the stores are not read
+    kvc = sf.QKV(k, v, row_stride=S, ref_cache=cache)
+    ok = oquant.quantize_nested(Kf[:, :T].reshape(-1, d), d, 2, 2)
+    ov = oquant.quantize_nested(Vf[:, :T].reshape(-1, d), d, 2, 2)
+    return kvc, cache, ok, ov, k_tokens, cap
+
+
+@pytest.mark.parametrize("path", ["auto", "pipeline"])
+def test_attention_with_kv_refinement_cache(sf, path):
+    Hq, Hkv, d, T, S = 32, 8, 128, 6000, 6040
+    kvc, cache, ok, ov, k_tokens, cap = _setup(sf, Hq, Hkv, T, S, d, 811, 10)
+    budget = 700
+    cache.set_budget(budget)
+    orc = ocache.LRUCache(Hkv * S, cap)
+    grp = Hq // Hkv
+    units = torch.zeros(Hkv * grp * k_tokens, dtype=torch.int32, device="cuda")
+    n_units = torch.zeros(1, dtype=torch.int32, device="cuda")
+    side = torch.cuda.Stream()
+    sf.attn_set_path(sf.ATTN_PIPELINE if path == "pipeline" else sf.ATTN_AUTO)
+    late = 0
+    try:
+        for step, qseed in enumerate([901, 901, 902, 901, 901]):
+            qb = gen_query(qseed, Hq, d)
+            snap = orc.snapshot()
+            avail = np.zeros((Hkv, T), dtype=bool)
+            for u in snap:
+                g, t = divmod(u, S)
+                if t < T:
+                    avail[g, t] = True
+            out, sel, sel_n = sf.attn_decode_refine(dev(qb.view(np.int16)).view(torch.bfloat16), kvc, Hkv, T,
+                                                    k_tokens)
+            sf.attn_union_units(sel, sel_n, Hkv, grp * k_tokens, S, units, n_units)
+            cache.prefetch(units, n_units, torch.cuda.current_stream(), side)
+            torch.cuda.synchronize()
+            ref = oattn.attn_decode_refine(qb, ok, ov, Hkv, T, k_tokens, available=avail)
+            sel_c, n_c = sel.cpu().numpy(), sel_n.cpu().numpy()
+            want_units = []
+            for g in range(Hkv):
+                np.testing.assert_array_equal(sel_c[g, : n_c[g]], ref["union"][g])
+                want_units += [g * S + int(t) for t in ref["union"][g]]
+            assert int(n_units.item()) == len(want_units)
+            np.testing.assert_array_equal(units.cpu().numpy()[: len(want_units)], want_units)
+            err = np.abs(out.cpu().numpy().astype(np.float64) - ref["out"]).max()
+            assert err <= ATTN_TOL, f"step {step}: max-abs error {err}"
+            want = orc.step(want_units, budget=budget)
+            got = cache.sets()
+            assert got["hits"] == want["hits"] and got["misses"] == want["misses"]
+            assert got["bypass"] == want["bypass"]
+            late += len(want["late"])
+            assert cache.stats().late == late
+            if step == 0:
+                assert not any(len(e) for e in ref["refined"])        # a cold cache refines nothing
+            if step == 1:
+                assert sum(len(e) for e in ref["refined"]) == min(budget, len(want_units))
+        assert late > 0 and orc.hits > 0
+        assert {u: s for s, u in enumerate(cache.slots()) if u >= 0} == orc.snapshot()
+    finally:
+        sf.attn_set_path(sf.ATTN_AUTO)
+        cache.close()
+
+
+def test_kv_cache_refusals(sf):
+    Hq, Hkv, d, T, S = 8, 2, 128, 512, 512
+    kvc, cache, ok, ov, k_tokens, cap = _setup(sf, Hq, Hkv, T, S, d, 812, 10)
+    q = torch.zeros((Hq, d), dtype=torch.bfloat16, device="cuda")
+    sf.attn_set_path(sf.ATTN_CLUSTER)
+    try:
+        with pytest.raises(sf.SfError, match="ref_cache"):
+            sf.attn_decode_refine(q, kvc, Hkv, T, k_tokens)
+    finally:
+        sf.attn_set_path(sf.ATTN_AUTO)
+    # a cache with a fetch budget cannot serve a GEMV
+    W = torch.randn(256, 256, device="cuda") * 0.02
+    qw = sf.quantize_nested(W, 128, 2, 2)
+    wc = sf.RefineCache(256, 256 * 2 // 8, 32, 8, qw.ref.cpu().contiguous().pin_memory())
+    wc.set_budget(4)
+    x = torch.randn(1, 256, device="cuda").to(torch.bfloat16)
+    idx, n = sf.select_topk(x, 8)
+    wc.prefetch(idx, n)
+    with pytest.raises(sf.SfError, match="fetch budget"):
+        sf.gemv_refine(qw, x, idx, n, cache=wc)
+    torch.cuda.synchronize()
+    wc.close()
+    cache.close()
