@@ -1,25 +1,26 @@
 #!/usr/bin/env python
-"""Benchmark of the StrataFlux refined low-bit decode hot path on B200.
+"""Benchmark of StrataFlux refined low-bit decoding on B200.
 
-One step = the whole hot path of one decode token of a 32-layer
-Llama-3.1-8B-shaped model at 32K context, batch 1:
+Headline: one full decode step of a random-init 32-layer Llama-3.1-8B-shaped
+model at 131072-token context, batch 1 (the configuration the pages' 128K
+measurement names: 3-bit resident + 1-bit refinement weights, 2-bit + 2-bit
+KV, RMSNorm, RoPE, SiLU MLP, LM head of 128256).  Per layer: top-3% channel
+selection of every GEMV input, one LRU step per weight matrix (10% of its
+columns cached in HBM, misses gathered from page-locked host memory on a side
+stream before the GEMV that needs them), the refined GEMVs on the tensor
+cores, RoPE, the new token quantized and appended, refined attention over
+all 131072 tokens (top 1% tokens per query head; refinement bits from a KV
+refinement cache of 10% of the token-heads, misses fetched for later steps
+within a per-step budget), the MLP; then RMSNorm and the refined LM head.
+The whole step is one CUDA graph; the working set (~5.7 GB) is far larger
+than L2, so no flush is needed.
 
-  per layer: top-3% channel selection of the four linear-layer inputs
-  (qkv, o, gate/up, down), one LRU refinement-cache step per weight matrix
-  (10% of columns cached, misses gathered from pinned host memory on a side
-  stream, issued one layer ahead = fetch lead), the seven refined GEMVs
-  (2-bit resident + 2-bit refinement, group 128), and refined decode
-  attention over 32768 tokens (2-bit + 2-bit K/V, top-1% tokens per query
-  head refined).
-
-The step is captured once in a CUDA graph and replayed.  Weights (1.96 GB),
-KV (0.6 GB) and the refinement stores stay resident; per step only the
-synthetic activations/queries change (staged device-to-device inside the
-timed region).  The working set (> 2.5 GB) is far larger than L2 (126 MB),
-so no L2 flush is needed.
-
-Metric: effective HBM GB/s = algorithmic bytes of the step / step time, with
-tokens/s (= steps/s) alongside.  Prints one JSON line (rank 0).
+Metric: effective HBM GB/s (algorithmic bytes of the step / step time) and
+tokens/s.  Extras: the quantization-only step (refinement overhead), the
+attention's and the GEMVs' rooflines, host-link GB/s, GPU memory, the
+end-to-end step through the public API with host buffers, and the 32K hot
+path of round one (2+2-bit weights, independent per-layer inputs).  Prints
+one JSON line (rank 0).
 """
 
 from __future__ import annotations
@@ -51,6 +52,16 @@ def workload(T):
     return f"llama31_8b_decode_hotpath_{ctx}"
 
 
+def workload_step(T):
+    ctx = f"{T // 1024}k" if T % 1024 == 0 else str(T)
+    return f"llama31_8b_decode_step_{ctx}"
+
+
+# the full decode step: 3-bit resident + 1-bit refinement weights, LM head 128256
+STEP_W_BITS = (3, 1)
+VOCAB = 128256
+
+
 def cluster_attention(T):
     """True where the library runs the attention as one cluster launch per
     layer (up to 32K tokens at <= 4 query heads per KV head), else it runs
@@ -68,11 +79,15 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("sf", "reference"), default="sf")
     ap.add_argument("--layers", type=int, default=32)
-    ap.add_argument("--context", type=int, default=32768)
+    ap.add_argument("--context", type=int, default=131072, help="tokens attended by the timed step")
+    ap.add_argument("--kv-cache-pct", type=float, default=10.0,
+                    help="KV refinement cache, percent of the token-heads (negative: the whole store in HBM)")
+    ap.add_argument("--kv-budget", type=int, default=4096,
+                    help="KV refinement misses fetched per layer and step at most (negative: no limit)")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-extras", action="store_true", help="skip e2e / resident-only / roofline legs")
-    ap.add_argument("--long-context", type=int, default=131072,
-                    help="also time the refined step at this context (0: skip); part of the extras")
+    ap.add_argument("--hotpath-context", type=int, default=32768,
+                    help="also time the 2+2-bit hot path at this context (0: skip); part of the extras")
     return ap.parse_args()
 
 
@@ -85,9 +100,11 @@ ATTN_TRAFFIC_32K = 21377792          # attn_fused_kernel<4>, Hq 32, Hkv 8, T 327
 GEMV_TRAFFIC_PER_LAUNCH = 15849088   # gemv_mma_kernel, mean of a layer's 4 launches (63.40 MB)
 
 
-def gemv_bytes(N, K, k_sel):
-    """Algorithmic HBM bytes of one refined GEMV at batch 1."""
-    return N * K * B_R // 8 + 4 * N * K // G + k_sel * N * B_F // 8 + 2 * K + 4 * N
+def gemv_bytes(N, K, k_sel, b_r=B_R, b_f=B_F):
+    """Algorithmic HBM bytes of one refined GEMV at batch 1: resident codes,
+    fp16 scale and zero per group, the selected columns' refinement bits, x
+    in (bf16), y out (fp32)."""
+    return N * K * b_r // 8 + 4 * N * K // G + k_sel * N * b_f // 8 + 2 * K + 4 * N
 
 
 def attn_bytes(T, union_tokens):
@@ -447,40 +464,94 @@ def blas_threads():
 
 # ------------------------------------------------------------------ arms
 
+def oracle_sample_step5(T, which, full=False):
+    """The CPU oracle on a bounded sample of the full decode step at context T
+    (3-bit resident + 1-bit refinement weights, 2+2-bit KV).  Item `which`
+    cycles over the seven layer matrices (selection of the top 3% channels,
+    one LRU step of a 10% cache, the refined GEMV) and the refined attention
+    of one KV head (four query heads) over min(T, 16384) tokens; full=True
+    takes all seven matrices and the attention over all T tokens.  Returns
+    (seconds, algorithmic bytes, description)."""
+    from oracle import attn as oattn, cache as ocache, gemv as ogemv, quant as oquant, select as oselect
+    from workloads import synth, count_fraction
+    b_r, b_f = STEP_W_BITS
+    items = list(range(8)) if full else [which % 8]
+    t_tot, nbytes, desc = 0.0, 0, []
+    for it in items:
+        if it < 7:
+            name, N, K, slot = MATS[it]
+            W = synth.gen_weight(1000 + it, N, K)
+            qz = oquant.quantize_nested(W, G, b_r, b_f)
+            outl = synth.outlier_channels(5000 + it, K, count_fraction(OUTLIER_PCT, K))
+            x = synth.gen_activations(2000 + it, 1, K, outl, OUTLIER_SCALE)
+            k = count_fraction(TOPK_PCT, K)
+            t0 = time.perf_counter()
+            S = oselect.select_topk(x, k)
+            ocache.LRUCache(K, count_fraction(CACHE_PCT, K)).step(S.tolist())
+            ogemv.gemv_refine(qz, x, S)
+            t_tot += time.perf_counter() - t0
+            nbytes += gemv_bytes(N, K, len(S), b_r, b_f)
+            desc.append(name)
+        else:
+            Ts = T if full else min(T, 16384)
+            Kf, Vf, _ = synth.gen_kv(3000 + which, 1, Ts, D)
+            qk = oquant.quantize_nested(Kf.reshape(-1, D), D, B_R, B_F)
+            qv = oquant.quantize_nested(Vf.reshape(-1, D), D, B_R, B_F)
+            qb = synth.gen_query(4000 + which, HQ // HKV, D)
+            t0 = time.perf_counter()
+            r = oattn.attn_decode_refine(qb, qk, qv, 1, Ts, count_fraction(TOK_PCT, Ts))
+            t_tot += time.perf_counter() - t0
+            U = len(r["union"][0])
+            nbytes += Ts * 2 * (D * B_R // 8 + 4) + U * 2 * D * B_F // 8 + (HQ // HKV) * D * 6
+            desc.append(f"attention of one KV head over {Ts} tokens")
+    return t_tot, nbytes, ", ".join(desc)
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def run_reference(args, rank):
-    """The CPU oracle as the reference arm (rank 0 only)."""
+    """The CPU oracle as the reference arm (rank 0 only), on the headline's
+    workload: each step one bounded item of the full decode step."""
     if rank != 0:
         return
     T = args.context
     for i in range(args.warmup):
-        oracle_sample_step(T, which=i)
+        oracle_sample_step5(T, i)
     t_tot, b_tot = 0.0, 0
     for i in range(args.steps):
-        dt, nb = oracle_sample_step(T, which=args.warmup + i)
+        dt, nb, _ = oracle_sample_step5(T, args.warmup + i)
         t_tot += dt
         b_tot += nb
     gbs = b_tot / t_tot / 1e9
     cores = blas_threads()
-    sample = (f"per step one of the 7 Llama-3.1-8B-shaped linear layers (cycled) with selection, one LRU step and "
-              f"the refined GEMV, plus refined attention of one KV head (4 query heads) at T={T}")
+    sample = (f"per step one item of the full decode step at T={T}, cycled: one of the 7 Llama-3.1-8B-shaped "
+              f"linear layers (3+1 bits: selection, LRU step, refined GEMV) or the refined attention of one KV "
+              f"head over 16384 tokens; CPU {cpu_model()}")
     line = {
-        "impl": "reference", "metric": "effective HBM GB/s (refined low-bit decode hot path)", "value": gbs,
+        "impl": "reference", "metric": "effective HBM GB/s (refined low-bit decode step)", "value": gbs,
         "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * t_tot / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy draws)",
-        "config": {"workload": workload(T), "context": T, "layers": args.layers, "batch": 1},
+        "config": {"workload": workload_step(T), "context": T, "layers": args.layers, "batch": 1},
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def run_sf(args, rank, world, local_rank, dist):
-    import torch
-    import quantized_gemv_kv_b200 as sf
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    T = args.context
+def hotpath_leg(args, sf, torch, dist, dev, world, T, phys):
+    """The 2+2-bit hot path of one decode token at context T (round one's
+    headline): per layer the four selections, seven cache steps and misses,
+    seven refined GEMVs and the refined attention, every layer's inputs drawn
+    independently.  Returns its numbers as a dict (an extra of the line)."""
     model = Model(sf, torch, args.layers, T, dev)
     # distinct per-step inputs, cycled: 32 steps apart, a channel's reuse
     # distance exceeds every refinement cache's capacity, so the cycle adds no
@@ -508,8 +579,6 @@ def run_sf(args, rank, world, local_rank, dist):
             run_step(i)
     torch.cuda.synchronize()
     before = model.cache_totals()
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-    phys = vis.split(",")[local_rank].strip() if vis else str(local_rank)
     with ClockSampler(phys) as clk:
         ms = timed(torch, dist, lambda i: run_step(args.warmup + i), args.steps, cap_stream)
     clocks = clk.summary()
@@ -615,29 +684,325 @@ def run_sf(args, rank, world, local_rank, dist):
         e2e = {"value": whole_job_gbs(step_bytes, ms_e2e, world), "unit": "GB/s", "ms_per_step": ms_e2e,
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
 
+    out = {"workload": workload(T), "value": value, "unit": "GB/s", "ms_per_step": ms_step, "tokens_per_s": tok_s,
+           "weights": "2-bit resident + 2-bit refinement, group 128", "bytes_per_step": step_bytes,
+           "h2d_miss_bytes_per_step": h2d_step, "cache_hit_rate": hits / max(1, hits + miss),
+           "union_tokens_per_layer": union_per_layer, "steps": args.steps, "clocks": clocks}
+    if roofline is not None:
+        out["roofline"] = roofline
+    if e2e is not None:
+        out["e2e"] = e2e
+    out.update(extras)
+    torch.cuda.synchronize()
+    del g
+    model.close()
+    del model
+    torch.cuda.empty_cache()
+    return out
+
+
+def graph_kernels(g):
+    """Kernel nodes of a captured graph, by kernel name (the library's
+    launches counted from the graph itself; memsets and copies excluded)."""
+    try:
+        from cuda.bindings import runtime as cr
+        graph = g.raw_cuda_graph()
+        err, _, n = cr.cudaGraphGetNodes(graph, numNodes=0)
+        err, nodes, n = cr.cudaGraphGetNodes(graph, numNodes=n)
+        names = {}
+        for nd in nodes[:n]:
+            err, t = cr.cudaGraphNodeGetType(nd)
+            if t != cr.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                continue
+            err, prm = cr.cudaGraphKernelNodeGetParams(nd)
+            err, name = cr.cudaFuncGetName(prm.func)
+            key = name.decode() if isinstance(name, bytes) else str(name)
+            names[key] = names.get(key, 0) + 1
+        return names
+    except Exception:
+        return None
+
+
+def host_link(torch, dev, nbytes=256 << 20, reps=5):
+    """Page-locked host <-> HBM copy bandwidth (GB/s) measured in this run:
+    the roofline of the refinement misses."""
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    s = torch.cuda.Stream(device=dev)
+    out = {}
+    for name, fn in (("h2d_gbs", lambda: d.copy_(h, non_blocking=True)),
+                     ("d2h_gbs", lambda: h.copy_(d, non_blocking=True))):
+        with torch.cuda.stream(s):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            e0.record(s)
+            for _ in range(reps):
+                fn()
+            e1.record(s)
+        torch.cuda.synchronize()
+        out[name] = reps * nbytes / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    del h, d
+    return out
+
+
+def phys_gpu(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    return vis.split(",")[local_rank].strip() if vis else str(local_rank)
+
+
+def step_model(args, sf, torch, dev, layers):
+    """The full decode step's model: random-init Llama-3.1-8B shape (RMSNorm
+    weights 1), 3+1-bit weights with 10% LRU caches per matrix, the initial
+    context of every layer N(0, 1) K/V with 4 outlier key channels per KV head
+    x10, 2+2-bit KV behind a KV refinement cache."""
+    from fractions import Fraction
+    from workloads import device_synth as ds
+    from quantized_gemv_kv_b200.decode import DecodeModel, Shape
+    T = args.context - 1
+    shape = Shape(layers=layers)
+    names = ("q", "k", "v", "o", "gate", "up", "down")
+
+    def weight(l, name, N, K):
+        seed = 1000 + l * 16 + names.index(name) if l >= 0 else 999
+        return ds.weight(seed, N, K, device=dev)
+
+    def norm(l, which):
+        return torch.ones(shape.hidden, dtype=torch.float32)
+
+    def kv(l):
+        Kf, Vf = ds.kv(3000 + l, shape.n_kv, T, shape.head_dim, device=dev)
+        return Kf.view(shape.n_kv, T, shape.head_dim), Vf.view(shape.n_kv, T, shape.head_dim)
+
+    kv_pct = None if args.kv_cache_pct < 0 else args.kv_cache_pct
+    budget = None if args.kv_budget < 0 else args.kv_budget
+    m = DecodeModel(shape, weight, norm, kv, capacity=args.context, p=Fraction(TOPK_PCT, 100),
+                    p_tok=Fraction(TOK_PCT, 100), weight_cache_pct=CACHE_PCT, kv_cache_pct=kv_pct,
+                    kv_budget=budget, device=dev)
+    return m, T
+
+
+def step_bytes(model, T, refined_tokens_per_layer):
+    """Algorithmic HBM bytes of one decode step: every GEMV (resident codes,
+    scale/zero, the selected columns' refinement bits from the HBM cache, x,
+    y) and the attention of every layer (resident K/V codes and scale/zero of
+    the T + 1 tokens, the refined token-heads' K and V refinement bits, q,
+    out); the per-token norms, RoPE and append are a few KB and left out."""
+    s = model.s
+    b_r, b_f = s.w_bits
+    gemv = 0
+    slot_of = {"q": "attn_in", "k": "attn_in", "v": "attn_in", "o": "attn_out", "gate": "mlp_in",
+               "up": "mlp_in", "down": "mlp_mid"}
+    for name, slot in slot_of.items():
+        N, K = s.mat_shape(name)
+        gemv += gemv_bytes(N, K, model.k_in[slot], b_r, b_f)
+    gemv *= s.layers
+    Nh, Kh = s.mat_shape("head")
+    gemv += gemv_bytes(Nh, Kh, model.k_in["head"], b_r, b_f)
+    attn = s.layers * attn_bytes(T + 1, refined_tokens_per_layer)
+    return gemv, attn
+
+
+def run_sf(args, rank, world, local_rank, dist):
+    import torch
+    import quantized_gemv_kv_b200 as sf
+    from workloads import device_synth as ds
+    from workloads import count_fraction
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    phys = phys_gpu(local_rank)
+    torch.cuda.synchronize()
+    free0, total = torch.cuda.mem_get_info()
+    model, T = step_model(args, sf, torch, dev, args.layers)
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    free1, _ = torch.cuda.mem_get_info()
+    H = model.s.hidden
+    n_total = min(args.warmup + args.steps, 32)
+    outl = ds.outlier_channels(5000, H, count_fraction(OUTLIER_PCT, H), dev)
+    pool = torch.stack([ds.activations(2000 + i, 1, H, outl, OUTLIER_SCALE, dev)[0].float()
+                        for i in range(n_total)])
+    cap_stream = torch.cuda.Stream(device=dev)
+    # one eager step (cold caches fill), then the step as one graph
+    model.x_in.copy_(pool[0])
+    with torch.cuda.stream(cap_stream):
+        model.step(T)
+    torch.cuda.synchronize()
+    model.sync()
+    g = capture(torch, lambda: model.step(T), cap_stream)
+    kernels = graph_kernels(g)
+
+    def run_step(i):
+        model.x_in.copy_(pool[i % n_total], non_blocking=True)
+        g.replay()
+
+    for i in range(args.warmup):
+        with torch.cuda.stream(cap_stream):
+            run_step(i)
+    torch.cuda.synchronize()
+    model.sync()
+    w0, k0 = model.cache_totals("weights"), model.cache_totals("kv")
+    with ClockSampler(phys) as clk:
+        ms = timed(torch, dist, lambda i: run_step(args.warmup + i), args.steps, cap_stream)
+    clocks = clk.summary()
+    model.sync()
+    w1, k1 = model.cache_totals("weights"), model.cache_totals("kv")
+    ms_step = ms / args.steps
+    L = args.layers
+    union = sum(float(sum(len(u) for u in model.union(l))) for l in range(L)) / L
+    if model.kv_cache_pct is not None:
+        refined = (k1["hits"] - k0["hits"]) / args.steps / L
+    else:
+        refined = union
+    gemv_b, attn_b = step_bytes(model, T, refined)
+    nbytes = gemv_b + attn_b
+    value = whole_job_gbs(nbytes, ms_step, world)
+    free2, _ = torch.cuda.mem_get_info()
+    wmiss = w1["h2d_bytes"] - w0["h2d_bytes"]
+    kmiss = k1["h2d_bytes"] - k0["h2d_bytes"]
+
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except OSError:
+        pass
+    hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
+    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
+    extras, roofline, e2e = {}, None, None
+    if not args.skip_extras:
+        model.sync()
+        k_tok = model.k_tok
+        # the attention of every layer, in one graph (the step's dominant kernels)
+        def attn_only():
+            for l, Ly in enumerate(model.layers):
+                sf.attn_decode_refine(model.q_bf[l], Ly["kv"], model.s.n_kv, T + 1, k_tok, workspace=model.ws,
+                                      out=model.att[l], sel_out=model.sel[l], sel_n=model.sel_n[l])
+        ga = capture(torch, attn_only, cap_stream)
+        for _ in range(2):
+            with torch.cuda.stream(cap_stream):
+                ga.replay()
+        reps = 5
+        t_attn = timed(torch, dist, lambda i: ga.replay(), reps, cap_stream) / reps / L * 1e-3
+        achieved = attn_b / L / t_attn / 1e9
+        roofline = {"bound": "hbm", "kernel": "attention pipeline (attn_score_mma, select_compact, select_finish, "
+                                              "refine, attn_out)",
+                    "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                    "traffic": None, "peak_source": peak_src, "launch_us": t_attn * 1e6,
+                    "bytes_per_launch": attn_b / L}
+        del ga
+        # the GEMVs of the step (four launches per layer and the LM head), in one graph
+        def gemvs_only():
+            for l in range(L):
+                for slot in ("attn_in", "attn_out", "mlp_in", "mlp_mid"):
+                    b = model.buf[slot]
+                    model.jobs0[l][slot].run(b["x"][l:l + 1], b["act"][l])
+            model.head_job0.run(model.buf["head"]["x"], model.buf["head"]["act"][0])
+        gg = capture(torch, gemvs_only, cap_stream)
+        for _ in range(2):
+            with torch.cuda.stream(cap_stream):
+                gg.replay()
+        n_launch = 4 * L + 1
+        t_g = timed(torch, dist, lambda i: gg.replay(), reps, cap_stream) / reps / n_launch * 1e-3
+        res_b = sum(gemv_bytes(*model.s.mat_shape(n), 0, *model.s.w_bits) for n in
+                    ("q", "k", "v", "o", "gate", "up", "down")) * L + gemv_bytes(*model.s.mat_shape("head"), 0,
+                                                                                  *model.s.w_bits)
+        ach_g = res_b / n_launch / t_g / 1e9
+        extras["roofline_gemv"] = {"bound": "hbm", "kernel": "gemv_mma_kernel (3-bit resident, resident-only "
+                                                             "launches as in the quantization-only step)",
+                                   "achieved": ach_g, "peak": hbm_peak, "unit": "GB/s", "frac": ach_g / hbm_peak,
+                                   "traffic": None, "peak_source": peak_src, "launch_us": t_g * 1e6,
+                                   "bytes_per_launch": res_b / n_launch}
+        del gg
+        # the quantization-only step: same kernels, nothing selected, fetched or refined
+        g0 = capture(torch, lambda: model.step(T, refine=False), cap_stream)
+
+        def run_res(i):
+            model.x_in.copy_(pool[i % n_total], non_blocking=True)
+            g0.replay()
+        for i in range(3):
+            with torch.cuda.stream(cap_stream):
+                run_res(i)
+        ms_res = timed(torch, dist, run_res, args.steps, cap_stream) / args.steps
+        extras["resident_only_ms_per_step"] = ms_res
+        extras["refinement_overhead_pct"] = 100.0 * (ms_step / ms_res - 1.0)
+        del g0
+        # end to end through the public API: the token's embedding from
+        # page-locked host memory in, the logits back to host memory, every step
+        hx = pool.cpu().pin_memory()
+        hl = torch.empty(model.logits.shape, dtype=torch.float32).pin_memory()
+
+        def run_e2e(i):
+            model.x_in.copy_(hx[i % n_total], non_blocking=True)
+            g.replay()
+            hl.copy_(model.logits, non_blocking=True)
+        for i in range(2):
+            with torch.cuda.stream(cap_stream):
+                run_e2e(i)
+        ms_e2e = timed(torch, dist, lambda i: run_e2e(args.warmup + i), args.steps, cap_stream,
+                       sync_each=True) / args.steps
+        e2e = {"value": whole_job_gbs(nbytes, ms_e2e, world), "unit": "GB/s", "ms_per_step": ms_e2e,
+               "tokens_per_s": world * 1e3 / ms_e2e, "h2d_bytes_per_step": H * 4,
+               "d2h_bytes_per_step": model.logits.numel() * 4}
+        link = host_link(torch, dev)
+        extras["host_link"] = dict(link, miss_bytes_per_step=(wmiss + kmiss) / args.steps,
+                                   weight_miss_bytes_per_step=wmiss / args.steps,
+                                   kv_miss_bytes_per_step=kmiss / args.steps,
+                                   miss_gbs_over_step=(wmiss + kmiss) / args.steps / (ms_step * 1e-3) / 1e9)
+    torch.cuda.synchronize()
+    del g
+    hot = None
+    if not args.skip_extras and args.hotpath_context:
+        model.close()
+        del model
+        torch.cuda.empty_cache()
+        hot = hotpath_leg(args, sf, torch, dist, dev, world, args.hotpath_context, phys)
+        model = None
+
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
-        dt, nb = oracle_sample_step(T)
+        try:
+            from threadpoolctl import threadpool_limits
+        except ImportError:
+            threadpool_limits = None
+        dt, nb, desc = oracle_sample_step5(T + 1, 0, full=True)
         cpu = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"one full layer: 7 refined linears (selection, LRU step, GEMV) + refined attention "
-                         f"of all 8 KV heads at T={T}; {dt:.1f} s"}
+               "cpu_model": cpu_model(), "logical_cpus": os.cpu_count(),
+               "sample": f"one layer of the step: {desc} ({dt:.1f} s)"}
+        if threadpool_limits is not None:
+            with threadpool_limits(limits=1):
+                dt1, nb1, _ = oracle_sample_step5(T + 1, 0, full=False)
+            cpu["one_core"] = {"value": nb1 / dt1 / 1e9, "unit": "GB/s", "cores": 1,
+                               "sample": "the q projection's selection, LRU step and refined GEMV"}
 
+    hits, miss = w1["hits"] - w0["hits"], w1["misses"] - w0["misses"]
+    khits, kmisses = k1["hits"] - k0["hits"], k1["misses"] - k0["misses"]
     line = {
-        "metric": "effective HBM GB/s (refined low-bit decode hot path)", "value": value, "unit": "GB/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "metric": "effective HBM GB/s (refined low-bit decode step) and tokens/s at 128K", "value": value,
+        "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic (seeded on-device draws; random-init weights)",
-        "config": {"workload": workload(T), "model_shape": "Llama-3.1-8B (32 layers)", "context": T,
-                   "layers": args.layers, "batch": 1, "weights": "2-bit resident + 2-bit refinement, group 128",
-                   "kv": "2-bit + 2-bit, per token-head", "topk_channels": "3%", "cache": "10% LRU per matrix",
-                   "topk_tokens": "1% per query head", "l2": "working set > L2, no flush",
-                   "parallelism": f"replicas x{world}", "graph": "CUDA graph per step"},
-        "tokens_per_s": tok_s,
-        "bytes_per_step": step_bytes,
-        "h2d_miss_bytes_per_step": h2d_step,
-        "cache_hit_rate": hits / max(1, hits + miss),
-        "union_tokens_per_layer": union_per_layer,
-        "gpu_launches": model.launches_per_step() * args.steps,
+        "data": "synthetic (seeded on-device draws; random-init weights and initial context)",
+        "config": {"workload": workload_step(args.context), "model_shape": "Llama-3.1-8B (32 layers, LM head 128256)",
+                   "context": args.context, "layers": args.layers, "batch": 1,
+                   "weights": "3-bit resident + 1-bit refinement, group 128", "kv": "2-bit + 2-bit, per token-head",
+                   "topk_channels": "3% of each GEMV input", "weight_cache": "10% LRU per matrix",
+                   "topk_tokens": "1% per query head", "kv_cache": (f"{args.kv_cache_pct}% of token-heads, "
+                                                                    f"budget {args.kv_budget} per layer-step"
+                                                                    if args.kv_cache_pct >= 0 else "store in HBM"),
+                   "position": "the step decodes position T = context - 1 every time (rewriting that row)",
+                   "l2": "working set > L2, no flush", "parallelism": f"replicas x{world}",
+                   "graph": "CUDA graph per step"},
+        "tokens_per_s": world * 1e3 / ms_step,
+        "bytes_per_step": nbytes,
+        "gpu_memory_gb": (free0 - free1) / 1e9,
+        "gpu_memory_gb_after_run": (free0 - free2) / 1e9,
+        "weight_cache_hit_rate": hits / max(1, hits + miss),
+        "kv_cache_hit_rate": khits / max(1, khits + kmisses),
+        "kv_late_per_layer_step": (k1["late"] - k0["late"]) / args.steps / L,
+        "union_tokens_per_layer": union,
+        "refined_tokens_per_layer": refined,
+        "gpu_launches": (sum(kernels.values()) * args.steps) if kernels else None,
+        "kernels_per_step": kernels,
         "clocks": clocks,
     }
     if roofline is not None:
@@ -647,62 +1012,12 @@ def run_sf(args, rank, world, local_rank, dist):
     if cpu is not None:
         line["cpu_baseline"] = cpu
     line.update(extras)
-    torch.cuda.synchronize()
-    del g
-    model.close()
-    del model
-    if not args.skip_extras and args.long_context and args.long_context != T:
-        line["long_context"] = long_context_leg(args, sf, torch, dist, dev, world, args.long_context)
+    if hot is not None:
+        line["hotpath_32k"] = hot
+    if model is not None:
+        model.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
-
-
-def long_context_leg(args, sf, torch, dist, dev, world, T):
-    """The same refined decode step with every layer's KV at context T
-    (128K by default: the context the tokens/s figure is quoted at), timed
-    the same way over fewer steps."""
-    model = Model(sf, torch, args.layers, T, dev)
-    steps, warm = min(args.steps, 20), 3
-    n_total = min(warm + steps, 32)
-    xpool, qpool = model.make_pools(n_total)
-    cap_stream = torch.cuda.Stream(device=dev)
-    model.xin.copy_(xpool[0])
-    model.qin.copy_(qpool[0])
-    with torch.cuda.stream(cap_stream):
-        model.step()
-    torch.cuda.synchronize()
-    model.sync_caches()
-    g = capture(torch, model.step, cap_stream)
-
-    def run_step(i):
-        model.xin.copy_(xpool[i % n_total], non_blocking=True)
-        model.qin.copy_(qpool[i % n_total], non_blocking=True)
-        g.replay()
-
-    for i in range(warm):
-        with torch.cuda.stream(cap_stream):
-            run_step(i)
-    torch.cuda.synchronize()
-    ms = timed(torch, dist, lambda i: run_step(warm + i), steps, cap_stream) / steps
-    union = float(model.sel_n.cpu().clamp(min=0).sum(dim=1).float().mean())
-    nbytes = attn_bytes(T, union) * args.layers
-    for name, N, K, slot in MATS:
-        nbytes += gemv_bytes(N, K, model.ksel[slot]) * args.layers
-    # the attention alone, all layers in one graph
-    g4 = capture(torch, model.attn_only, cap_stream)
-    for _ in range(2):
-        with torch.cuda.stream(cap_stream):
-            g4.replay()
-    ms_a = timed(torch, dist, lambda i: g4.replay(), 5, cap_stream) / 5 / args.layers
-    del g, g4
-    model.close()
-    return {"context": T, "steps": steps, "warmup": warm, "ms_per_step": ms, "tokens_per_s": world * 1e3 / ms,
-            "value": whole_job_gbs(nbytes, ms, world), "unit": "GB/s", "bytes_per_step": nbytes,
-            "union_tokens_per_layer": union,
-            "attention": {"kernel": "attn_fused_kernel" if cluster_attention(T)
-                          else "attention pipeline (score, select, refine, out)",
-                          "launch_us": ms_a * 1e3, "bytes_per_launch": attn_bytes(T, union),
-                          "achieved_gbs": attn_bytes(T, union) / (ms_a * 1e-3) / 1e9}}
 
 
 def main():

@@ -40,12 +40,36 @@ def test_whole_job_value():
     assert bench.whole_job_gbs(2e9, 1.0, 4) == 8000.0
 
 
+def test_step_bytes_of_the_128k_decode_step():
+    """The full decode step at 128K: 3-bit codes + scale/zero of 32 layers
+    (~2.84 GB) and the LM head (~213 MB), 2-bit K/V of 131072 tokens x 8 KV
+    heads x 32 layers (~2.42 GB); about 5.47 GB per token in all."""
+    from fractions import Fraction
+    from types import SimpleNamespace
+    from quantized_gemv_kv_b200.decode import Shape, count_half_up
+    s = Shape()
+    p = Fraction(3, 100)
+    k_in = {"attn_in": count_half_up(p, 4096), "attn_out": count_half_up(p, 4096), "mlp_in": count_half_up(p, 4096),
+            "mlp_mid": count_half_up(p, 14336), "head": count_half_up(p, 4096)}
+    assert k_in == {"attn_in": 123, "attn_out": 123, "mlp_in": 123, "mlp_mid": 430, "head": 123}
+    gemv, attn = bench.step_bytes(SimpleNamespace(s=s, k_in=k_in), 131071, 0)
+    layer_res = sum(N * K * 3 // 8 + N * K // 32 for N, K in (s.mat_shape(n) for n in
+                    ("q", "k", "v", "o", "gate", "up", "down")))
+    head_res = 128256 * 4096 * 3 // 8 + 128256 * 4096 // 32
+    assert 2.83e9 < 32 * layer_res < 2.85e9 and 2.1e8 < head_res < 2.15e8
+    assert 0 < gemv - 32 * layer_res - head_res < 4.0e7      # refinement columns (~29 MB) and activations
+    assert attn == 32 * (8 * 131072 * 72 + 32 * 128 * 6)
+    assert 5.4e9 < gemv + attn < 5.55e9
+
+
 def test_bench_defaults(monkeypatch):
     """No flags: one GPU, a minutes-scale run, W >= 3 warm-up steps, the
-    128K leg on; --impl reference selects the oracle arm."""
+    headline at 128K with the 32K hot path as an extra; --impl reference
+    selects the oracle arm."""
     monkeypatch.setattr("sys.argv", ["bench.py"])
     a = bench.parse()
-    assert (a.gpus, a.impl, a.context, a.long_context) == (1, "sf", 32768, 131072)
+    assert (a.gpus, a.impl, a.context, a.hotpath_context) == (1, "sf", 131072, 32768)
+    assert a.kv_cache_pct == 10.0 and a.kv_budget > 0
     assert a.warmup >= 3 and 1 <= a.steps <= 1000
     monkeypatch.setattr("sys.argv", ["bench.py", "--impl", "reference", "--steps", "2", "--warmup", "3"])
     a = bench.parse()
