@@ -82,8 +82,8 @@ def parse():
     ap.add_argument("--context", type=int, default=131072, help="tokens attended by the timed step")
     ap.add_argument("--kv-cache-pct", type=float, default=10.0,
                     help="KV refinement cache, percent of the token-heads (negative: the whole store in HBM)")
-    ap.add_argument("--kv-budget", type=int, default=4096,
-                    help="KV refinement misses fetched per layer and step at most (negative: no limit)")
+    ap.add_argument("--kv-budget", type=int, default=512,
+                    help="KV refinement misses fetched per KV head and step at most (negative: no limit)")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-extras", action="store_true", help="skip e2e / resident-only / roofline legs")
     ap.add_argument("--hotpath-context", type=int, default=32768,
@@ -367,12 +367,14 @@ class Model:
                 cache.close()
 
 
-def capture(torch, fn, stream):
-    g = torch.cuda.CUDAGraph()
+def capture(torch, fn, stream, keep=False):
+    g = torch.cuda.CUDAGraph(keep_graph=True) if keep else torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         g.capture_begin(capture_error_mode="relaxed")
         fn()
         g.capture_end()
+    if keep:
+        g.instantiate()
     torch.cuda.synchronize()
     return g
 
@@ -702,25 +704,30 @@ def hotpath_leg(args, sf, torch, dist, dev, world, T, phys):
 
 
 def graph_kernels(g):
-    """Kernel nodes of a captured graph, by kernel name (the library's
-    launches counted from the graph itself; memsets and copies excluded)."""
+    """Kernel nodes of a captured graph (made with keep_graph=True), counted
+    by kernel name: the library's launches read from the graph itself (memset
+    and copy nodes are not counted)."""
+    import re
     try:
-        from cuda.bindings import runtime as cr
-        graph = g.raw_cuda_graph()
-        err, _, n = cr.cudaGraphGetNodes(graph, numNodes=0)
-        err, nodes, n = cr.cudaGraphGetNodes(graph, numNodes=n)
+        from cuda.bindings import driver as cd
+        graph = cd.CUgraph(g.raw_cuda_graph())
+        err, _, n = cd.cuGraphGetNodes(graph, 0)
+        err, nodes, n = cd.cuGraphGetNodes(graph, n)
         names = {}
         for nd in nodes[:n]:
-            err, t = cr.cudaGraphNodeGetType(nd)
-            if t != cr.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+            err, t = cd.cuGraphNodeGetType(nd)
+            if t != cd.CUgraphNodeType.CU_GRAPH_NODE_TYPE_KERNEL:
                 continue
-            err, prm = cr.cudaGraphKernelNodeGetParams(nd)
-            err, name = cr.cudaFuncGetName(prm.func)
-            key = name.decode() if isinstance(name, bytes) else str(name)
+            err, prm = cd.cuGraphKernelNodeGetParams(nd)
+            err, raw = cd.cuFuncGetName(prm.func)
+            raw = raw.decode() if isinstance(raw, bytes) else str(raw)
+            m = re.findall(r"[A-Za-z_]\w*kernel\w*", raw)
+            key = max(m, key=len) if m else raw
+            key = re.sub(r"^\d+", "", key)
             names[key] = names.get(key, 0) + 1
         return names
-    except Exception:
-        return None
+    except Exception as e:  # reported in the line instead of a count
+        return {"error": repr(e)[:200]}
 
 
 def host_link(torch, dev, nbytes=256 << 20, reps=5):
@@ -830,7 +837,7 @@ def run_sf(args, rank, world, local_rank, dist):
         model.step(T)
     torch.cuda.synchronize()
     model.sync()
-    g = capture(torch, lambda: model.step(T), cap_stream)
+    g = capture(torch, lambda: model.step(T), cap_stream, keep=True)
     kernels = graph_kernels(g)
 
     def run_step(i):
@@ -987,7 +994,7 @@ def run_sf(args, rank, world, local_rank, dist):
                    "weights": "3-bit resident + 1-bit refinement, group 128", "kv": "2-bit + 2-bit, per token-head",
                    "topk_channels": "3% of each GEMV input", "weight_cache": "10% LRU per matrix",
                    "topk_tokens": "1% per query head", "kv_cache": (f"{args.kv_cache_pct}% of token-heads, "
-                                                                    f"budget {args.kv_budget} per layer-step"
+                                                                    f"one LRU per KV head, budget {args.kv_budget} per head and step"
                                                                     if args.kv_cache_pct >= 0 else "store in HBM"),
                    "position": "the step decodes position T = context - 1 every time (rewriting that row)",
                    "l2": "working set > L2, no flush", "parallelism": f"replicas x{world}",
@@ -1001,7 +1008,7 @@ def run_sf(args, rank, world, local_rank, dist):
         "kv_late_per_layer_step": (k1["late"] - k0["late"]) / args.steps / L,
         "union_tokens_per_layer": union,
         "refined_tokens_per_layer": refined,
-        "gpu_launches": (sum(kernels.values()) * args.steps) if kernels else None,
+        "gpu_launches": (sum(kernels.values()) * args.steps) if kernels and "error" not in kernels else None,
         "kernels_per_step": kernels,
         "clocks": clocks,
     }

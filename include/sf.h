@@ -141,7 +141,7 @@ typedef struct sf_cache_stats {
  * used this step gets last use = this step.
  *   num_units   units addressable (K for a weight matrix);
  *   unit_bytes  bytes per unit (N*b_f/8 for a weight column), a multiple of 16;
- *   capacity    cache slots, 0 <= capacity <= num_units;
+ *   capacity    cache slots, 0 <= capacity <= min(num_units, 196608);
  *   max_select  largest selection a prefetch will see (B*k), >= 1;
  *   host_master host copy of all units, [num_units][unit_bytes], 16-byte
  *               aligned.  It must stay valid and unchanged until destroy.  If it
@@ -155,6 +155,24 @@ typedef struct sf_cache_stats {
 sf_status sf_refine_cache_create(sf_refine_cache** out, int num_units, size_t unit_bytes,
                                  int capacity, int max_select, const void* host_master,
                                  int device);
+
+/*
+ * sf_refine_cache_create_parts -- `parts` independent LRU caches under one
+ * handle: part p owns units [p*num_units/parts, (p+1)*num_units/parts) with
+ * `capacity` slots of its own and sees at most `max_select` of them per step,
+ * and each part follows the policy above on the run of the (ascending)
+ * selection that falls in its range; its fetch budget is per part.  A KV
+ * refinement cache uses one part per KV head (units g*S + t), so every
+ * head's LRU step runs in parallel.  Slot numbers are global (part p's slots
+ * are p*capacity ...), sf_refine_cache_slots writes parts*capacity entries,
+ * and sf_refine_cache_sets concatenates the parts' lists (each host array
+ * needs parts*max_select entries).  A partitioned cache cannot be preloaded
+ * or join a group.  parts = 1 is sf_refine_cache_create.
+ * Constraints: 1 <= parts <= 64, parts divides num_units, capacity at most
+ * num_units/parts; otherwise as sf_refine_cache_create.
+ */
+sf_status sf_refine_cache_create_parts(sf_refine_cache** out, int num_units, size_t unit_bytes, int parts,
+                                       int capacity, int max_select, const void* host_master, int device);
 
 /* Fill an empty cache with n distinct units (device int32, ascending,
  * n <= capacity) in slots 0..n-1 with last use older than any step.  Counts

@@ -75,6 +75,7 @@ _SIGS = {
     "sf_quantize_nested": ([_p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p], _i),
     "sf_select_topk": ([_p, _i, _i, _i, _p, _p, _p], _i),
     "sf_refine_cache_create": ([ctypes.POINTER(_p), _i, _sz, _i, _i, _p, _i], _i),
+    "sf_refine_cache_create_parts": ([ctypes.POINTER(_p), _i, _sz, _i, _i, _i, _p, _i], _i),
     "sf_refine_cache_preload": ([_p, _p, _i, _p], _i),
     "sf_refine_cache_prefetch": ([_p, _p, _p, _p, _p], _i),
     "sf_refine_cache_sets": ([_p, _p, _p, _p, _p], _i),
@@ -208,20 +209,24 @@ def select_topk(x: torch.Tensor, k: int, idx_out: torch.Tensor | None = None, n_
 class RefineCache:
     """LRU refinement cache in device memory fed from a host master copy
     (``sf_refine_cache_*``).  ``host_master`` is a CPU uint8/int32 tensor of
-    num_units * unit_bytes bytes; it is kept alive by this object."""
+    num_units * unit_bytes bytes; it is kept alive by this object.  With
+    parts > 1 the units are split into that many consecutive ranges, each an
+    LRU of ``capacity`` slots seeing at most ``max_select`` units per step
+    (``sf_refine_cache_create_parts``)."""
 
     def __init__(self, num_units: int, unit_bytes: int, capacity: int, max_select: int,
-                 host_master: torch.Tensor, device: int | None = None):
+                 host_master: torch.Tensor, device: int | None = None, parts: int = 1):
         if host_master.is_cuda or not host_master.is_contiguous():
             raise ValueError("host_master must be a contiguous CPU tensor")
         if host_master.numel() * host_master.element_size() < num_units * unit_bytes:
             raise ValueError("host_master is smaller than num_units * unit_bytes")
         self._master = host_master
         self.num_units, self.unit_bytes, self.capacity, self.max_select = num_units, unit_bytes, capacity, max_select
+        self.parts = parts
         self.device = torch.cuda.current_device() if device is None else device
         h = _p()
-        _check(_lib.sf_refine_cache_create(ctypes.byref(h), num_units, unit_bytes, capacity, max_select,
-                                           host_master.data_ptr(), self.device))
+        _check(_lib.sf_refine_cache_create_parts(ctypes.byref(h), num_units, unit_bytes, parts, capacity, max_select,
+                                                 host_master.data_ptr(), self.device))
         self._h = h
 
     @property
@@ -239,18 +244,18 @@ class RefineCache:
 
     def sets(self) -> dict:
         import numpy as np
-        h = np.zeros(self.max_select, np.int32)
-        m = np.zeros(self.max_select, np.int32)
-        b = np.zeros(self.max_select, np.int32)
+        h = np.zeros(self.max_select * self.parts, np.int32)
+        m = np.zeros(self.max_select * self.parts, np.int32)
+        b = np.zeros(self.max_select * self.parts, np.int32)
         c = np.zeros(3, np.int32)
         _check(_lib.sf_refine_cache_sets(self._h, h.ctypes.data, m.ctypes.data, b.ctypes.data, c.ctypes.data))
         return dict(hits=h[:c[0]].tolist(), misses=m[:c[1]].tolist(), bypass=b[:c[2]].tolist())
 
     def slots(self) -> list[int]:
         import numpy as np
-        s = np.zeros(max(self.capacity, 1), np.int32)
+        s = np.zeros(max(self.capacity * self.parts, 1), np.int32)
         _check(_lib.sf_refine_cache_slots(self._h, s.ctypes.data))
-        return s[:self.capacity].tolist()
+        return s[:self.capacity * self.parts].tolist()
 
     def stats(self) -> CacheStats:
         st = CacheStats()

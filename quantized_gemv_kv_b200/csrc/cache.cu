@@ -40,6 +40,9 @@ struct CacheDev {
   const int32_t* n_ptr;  // its length
   int max_select, capacity;
   int budget;            // misses fetched per step at most (the rest are late)
+  int slot_base;         // global slot number of this LRU's slot 0 (parts: p * capacity)
+  int bypass_base;       // global row of this LRU's first bypass row
+  int unit_lo, unit_hi;  // a part's unit range: its selection is the sub-range of S in it (unit_lo < 0: all of S)
   int64_t unit_bytes;
   int32_t *unit_slot, *slot_unit, *order, *order_tmp, *row_of, *hits_out, *misses_out, *bypass_out, *victim_unit,
       *victim_slot, *gather_unit, *gather_row, *meta;
@@ -52,7 +55,7 @@ struct CacheDev {
 // One cache step.  S = idx[0..n) ascending.  Runs in one CTA of
 // kIndexThreads threads with `capacity` bytes of dynamic shared memory.
 __device__ void cache_step(const CacheDev& d) {
-  const int32_t* __restrict__ S = d.S;
+  const int32_t* __restrict__ S = d.S;  // shifted to a part's sub-range below
   const int max_select = d.max_select, capacity = d.capacity;
   int32_t* __restrict__ unit_slot = d.unit_slot;
   int32_t* __restrict__ slot_unit = d.slot_unit;
@@ -73,6 +76,26 @@ __device__ void cache_step(const CacheDev& d) {
   __shared__ int scratch[33];
   const int tid = threadIdx.x;
   int n = *d.n_ptr;
+  const int slot_base = d.slot_base;
+  if (d.unit_lo >= 0) {
+    // a part of a partitioned cache: its units form one contiguous run of
+    // the ascending selection, found by binary search
+    __shared__ int range[2];
+    n = n < 0 ? 0 : n;
+    if (tid < 2) {
+      const int key = tid == 0 ? d.unit_lo : d.unit_hi;
+      int a = 0, b = n;  // first position with S[pos] >= key
+      while (a < b) {
+        const int m = (a + b) >> 1;
+        if (S[m] < key) a = m + 1; else b = m;
+      }
+      range[tid] = a;
+    }
+    __syncthreads();
+    S += range[0];
+    row_of += range[0];
+    n = range[1] - range[0];
+  }
   n = n < 0 ? 0 : (n > max_select ? max_select : n);
   const int occ = meta[kOcc];
 
@@ -85,7 +108,7 @@ __device__ void cache_step(const CacheDev& d) {
   int h = 0;
   for (int p = p0; p < p1; ++p) {
     const int sl = unit_slot[S[p]];
-    if (sl >= 0) { ++h; slot_hit[sl] = 1; }
+    if (sl >= 0) { ++h; slot_hit[sl - slot_base] = 1; }
   }
   int H;
   const int h_before = sfd::block_exclusive_scan(h, scratch, &H);
@@ -107,12 +130,12 @@ __device__ void cache_step(const CacheDev& d) {
   const int ochunk = (occ + kIndexThreads - 1) / kIndexThreads;
   const int o0 = min(occ, tid * ochunk), o1 = min(occ, o0 + ochunk);
   int keep = 0;
-  for (int i = o0; i < o1; ++i) keep += !slot_hit[unit_slot[order[i]]];
+  for (int i = o0; i < o1; ++i) keep += !slot_hit[unit_slot[order[i]] - slot_base];
   int F;
   int fpos = sfd::block_exclusive_scan(keep, scratch, &F);
   for (int i = o0; i < o1; ++i) {
     const int u = order[i];
-    const int sl = unit_slot[u];
+    const int sl = unit_slot[u] - slot_base;  // local slot
     if (slot_hit[sl]) continue;
     if (fpos < v) { victim_unit[fpos] = u; victim_slot[fpos] = sl; }
     else order_tmp[fpos - v] = u;
@@ -125,15 +148,15 @@ __device__ void cache_step(const CacheDev& d) {
     const int u = misses_out[r];
     int row;
     if (r < use_free) {
-      row = occ + r;
+      row = slot_base + occ + r;
     } else if (r < ins) {
-      row = victim_slot[r - use_free];
+      row = slot_base + victim_slot[r - use_free];
       unit_slot[victim_unit[r - use_free]] = -1;
     } else {
-      row = capacity + (r - ins);
+      row = d.bypass_base + (r - ins);
       bypass_out[r - ins] = u;
     }
-    if (r < ins) { unit_slot[u] = row; slot_unit[row] = u; }
+    if (r < ins) { unit_slot[u] = row; slot_unit[row - slot_base] = u; }
     gather_unit[r] = u;
     gather_row[r] = row;
   }
@@ -195,6 +218,15 @@ __global__ void __launch_bounds__(kIndexThreads) cache_index_kernel(CacheDev d) 
 // One CTA per cache of a group.
 __global__ void __launch_bounds__(kIndexThreads) cache_index_many_kernel(const CacheDev* __restrict__ table) {
   cache_step(table[blockIdx.x]);
+}
+
+// The parts of a partitioned cache, one CTA each, on the selection (S, n).
+__global__ void __launch_bounds__(kIndexThreads)
+cache_index_parts_kernel(const CacheDev* __restrict__ table, const int32_t* S, const int32_t* n) {
+  CacheDev d = table[blockIdx.x];
+  d.S = S;
+  d.n_ptr = n;
+  cache_step(d);
 }
 
 // Copy the missed units of `count` caches: one warp per unit, every lane
@@ -297,8 +329,10 @@ struct sf_refine_cache {
   int device = 0;
   int num_units = 0;
   size_t unit_bytes = 0;
-  int capacity = 0;
-  int max_select = 0;
+  int parts = 1;       // independent LRUs over consecutive unit ranges of part_units units
+  int part_units = 0;
+  int capacity = 0;    // slots per part
+  int max_select = 0;  // selected units per part and step at most
   int budget = 0;  // per-step fetch limit; max_select = no limit
   const void* host_master = nullptr;
   const void* master_dev = nullptr;
@@ -309,6 +343,7 @@ struct sf_refine_cache {
           *hits = nullptr, *misses = nullptr, *bypass = nullptr, *victim_unit = nullptr, *victim_slot = nullptr,
           *gather_unit = nullptr, *gather_row = nullptr, *meta = nullptr;
   int64_t* stats = nullptr;
+  CacheDev* table = nullptr;  // parts > 1: the parts' descriptors on the device
   cudaEvent_t ev_idx = nullptr, ev_ready = nullptr, ev_used = nullptr;
   cudaStream_t aux = nullptr;
   bool ready_pending = false, used_pending = false;
@@ -317,28 +352,35 @@ struct sf_refine_cache {
 
 namespace {
 
-CacheDev make_dev(const sf_refine_cache* c, const int32_t* S, const int32_t* n) {
+// Descriptor of part `p` (parts == 1: the whole cache).  Per-part arrays are
+// laid out part after part; slot numbers and rows are global.
+CacheDev make_dev(const sf_refine_cache* c, const int32_t* S, const int32_t* n, int p = 0) {
   CacheDev d{};
+  const size_t cap1 = std::max(c->capacity, 1), ms = c->max_select;
   d.S = S;
   d.n_ptr = n;
   d.max_select = c->max_select;
   d.capacity = c->capacity;
   d.budget = c->budget;
+  d.slot_base = p * c->capacity;
+  d.bypass_base = c->parts * c->capacity + p * c->max_select;
+  d.unit_lo = c->parts > 1 ? p * c->part_units : -1;
+  d.unit_hi = c->parts > 1 ? (p + 1) * c->part_units : -1;
   d.unit_bytes = static_cast<int64_t>(c->unit_bytes);
   d.unit_slot = c->unit_slot;
-  d.slot_unit = c->slot_unit;
-  d.order = c->order;
-  d.order_tmp = c->order_tmp;
+  d.slot_unit = c->slot_unit + p * cap1;
+  d.order = c->order + p * cap1;
+  d.order_tmp = c->order_tmp + p * cap1;
   d.row_of = c->row_of;
-  d.hits_out = c->hits;
-  d.misses_out = c->misses;
-  d.bypass_out = c->bypass;
-  d.victim_unit = c->victim_unit;
-  d.victim_slot = c->victim_slot;
-  d.gather_unit = c->gather_unit;
-  d.gather_row = c->gather_row;
-  d.meta = c->meta;
-  d.stats = c->stats;
+  d.hits_out = c->hits + p * ms;
+  d.misses_out = c->misses + p * ms;
+  d.bypass_out = c->bypass + p * ms;
+  d.victim_unit = c->victim_unit + p * ms;
+  d.victim_slot = c->victim_slot + p * ms;
+  d.gather_unit = c->gather_unit + p * ms;
+  d.gather_row = c->gather_row + p * ms;
+  d.meta = c->meta + p * kMetaCount;
+  d.stats = c->stats + p * kStatCount;
   d.master = static_cast<const uint4*>(c->master_dev);
   d.rows = reinterpret_cast<uint4*>(c->rows);
   d.unit_vec = static_cast<int>(c->unit_bytes / 16);
@@ -353,6 +395,7 @@ sf_status cache_free(sf_refine_cache* c) {
   if (c->ev_used) cudaEventSynchronize(c->ev_used);
   if (c->rows) cudaFree(c->rows);
   if (c->ints) cudaFree(c->ints);
+  if (c->table) cudaFree(c->table);
   if (c->stats) cudaFree(c->stats);
   if (c->ev_idx) cudaEventDestroy(c->ev_idx);
   if (c->ev_ready) cudaEventDestroy(c->ev_ready);
@@ -366,9 +409,9 @@ sf_status cache_free(sf_refine_cache* c) {
 
 sf_status cache_clear(sf_refine_cache* c, cudaStream_t s) {
   SF_CHECK_CUDA(cudaMemsetAsync(c->unit_slot, 0xFF, sizeof(int32_t) * c->num_units, s));
-  SF_CHECK_CUDA(cudaMemsetAsync(c->slot_unit, 0xFF, sizeof(int32_t) * std::max(c->capacity, 1), s));
-  SF_CHECK_CUDA(cudaMemsetAsync(c->meta, 0, sizeof(int32_t) * kMetaCount, s));
-  SF_CHECK_CUDA(cudaMemsetAsync(c->stats, 0, sizeof(int64_t) * kStatCount, s));
+  SF_CHECK_CUDA(cudaMemsetAsync(c->slot_unit, 0xFF, sizeof(int32_t) * std::max(c->capacity, 1) * c->parts, s));
+  SF_CHECK_CUDA(cudaMemsetAsync(c->meta, 0, sizeof(int32_t) * kMetaCount * c->parts, s));
+  SF_CHECK_CUDA(cudaMemsetAsync(c->stats, 0, sizeof(int64_t) * kStatCount * c->parts, s));
   return SF_OK;
 }
 
@@ -383,6 +426,16 @@ sf_status wait_ready(sf_refine_cache* c) {
     c->ready_pending = false;
   }
   SF_CHECK_CUDA(cudaStreamSynchronize(c->aux));
+  return SF_OK;
+}
+
+// parts > 1: the parts' descriptors (selection pointers filled per prefetch
+// by the kernel's arguments) on the device.
+sf_status upload_table(sf_refine_cache* c) {
+  std::vector<CacheDev> host(c->parts);
+  for (int q = 0; q < c->parts; ++q) host[q] = make_dev(c, nullptr, nullptr, q);
+  if (!c->table) SF_CHECK_CUDA(cudaMalloc(&c->table, sizeof(CacheDev) * c->parts));
+  SF_CHECK_CUDA(cudaMemcpy(c->table, host.data(), sizeof(CacheDev) * c->parts, cudaMemcpyHostToDevice));
   return SF_OK;
 }
 
@@ -409,7 +462,7 @@ sf_status cache_view_for_reader(sf_refine_cache* c, cudaStream_t stream, CacheVi
   v->unit_slot = c->unit_slot;
   v->num_units = c->num_units;
   v->unit_words = static_cast<int>(c->unit_bytes / 4);
-  v->max_select = c->max_select;
+  v->max_select = c->max_select * c->parts;
   return SF_OK;
 }
 
@@ -436,21 +489,28 @@ sf_status cache_mark_used(sf_refine_cache* c, cudaStream_t stream) {
 
 extern "C" {
 
-sf_status sf_refine_cache_create(sf_refine_cache** out, int num_units, size_t unit_bytes, int capacity,
-                                 int max_select, const void* host_master, int device) {
+sf_status sf_refine_cache_create_parts(sf_refine_cache** out, int num_units, size_t unit_bytes, int parts,
+                                       int capacity, int max_select, const void* host_master, int device) {
   SF_REQUIRE(out && host_master, "sf_refine_cache_create: null pointer");
   *out = nullptr;
   SF_REQUIRE(num_units >= 1, "sf_refine_cache_create: num_units must be >= 1");
+  SF_REQUIRE(parts >= 1 && parts <= 64 && num_units % parts == 0,
+             "sf_refine_cache_create: parts must be in [1, 64] and divide num_units");
+  const int part_units = num_units / parts;
   SF_REQUIRE(unit_bytes >= 16 && unit_bytes % 16 == 0, "sf_refine_cache_create: unit_bytes must be a positive multiple of 16");
-  SF_REQUIRE(capacity >= 0 && capacity <= num_units && capacity <= kMaxCapacity,
-             "sf_refine_cache_create: capacity must be in [0, min(num_units, %d)]", kMaxCapacity);
+  SF_REQUIRE(capacity >= 0 && capacity <= part_units && capacity <= kMaxCapacity,
+             "sf_refine_cache_create: capacity must be in [0, min(units per part, %d)]", kMaxCapacity);
   SF_REQUIRE(max_select >= 1 && max_select <= 1 << 20, "sf_refine_cache_create: max_select out of range");
+  SF_REQUIRE(static_cast<long long>(parts) * (capacity + max_select) < (1LL << 31),
+             "sf_refine_cache_create: too many rows");
   SF_REQUIRE(sf::aligned(host_master, 16), "sf_refine_cache_create: host_master must be 16-byte aligned");
   DeviceGuard g(device);
   auto* c = new sf_refine_cache();
   c->device = device;
   c->num_units = num_units;
   c->unit_bytes = unit_bytes;
+  c->parts = parts;
+  c->part_units = part_units;
   c->capacity = capacity;
   c->max_select = max_select;
   c->budget = max_select;
@@ -473,28 +533,29 @@ sf_status sf_refine_cache_create(sf_refine_cache** out, int num_units, size_t un
   if (e != cudaSuccess) { cache_free(c); return sf::cuda_fail(e, "cudaHostGetDevicePointer(host_master)"); }
   c->master_dev = dptr;
 
-  const size_t rows_bytes = (static_cast<size_t>(capacity) + max_select) * unit_bytes;
+  const size_t P = parts;
+  const size_t rows_bytes = P * (static_cast<size_t>(capacity) + max_select) * unit_bytes;
   e = cudaMalloc(&c->rows, rows_bytes);
   if (e != cudaSuccess) { cache_free(c); return sf::fail(SF_ENOMEM, "sf_refine_cache_create: cudaMalloc rows: %s", cudaGetErrorString(e)); }
-  const size_t cap1 = std::max(capacity, 1);
-  const size_t n_ints = static_cast<size_t>(num_units) + 3 * cap1 + 8 * static_cast<size_t>(max_select) + kMetaCount;
+  const size_t cap1 = std::max(capacity, 1), ms = max_select;
+  const size_t n_ints = static_cast<size_t>(num_units) + P * (3 * cap1 + 8 * ms + kMetaCount);
   e = cudaMalloc(&c->ints, n_ints * sizeof(int32_t));
   if (e != cudaSuccess) { cache_free(c); return sf::fail(SF_ENOMEM, "sf_refine_cache_create: cudaMalloc index: %s", cudaGetErrorString(e)); }
-  e = cudaMalloc(&c->stats, kStatCount * sizeof(int64_t));
+  e = cudaMalloc(&c->stats, P * kStatCount * sizeof(int64_t));
   if (e != cudaSuccess) { cache_free(c); return sf::fail(SF_ENOMEM, "sf_refine_cache_create: cudaMalloc stats: %s", cudaGetErrorString(e)); }
   int32_t* p = c->ints;
   c->unit_slot = p; p += num_units;
-  c->slot_unit = p; p += cap1;
-  c->order = p; p += cap1;
-  c->order_tmp = p; p += cap1;
-  c->row_of = p; p += max_select;
-  c->hits = p; p += max_select;
-  c->misses = p; p += max_select;
-  c->bypass = p; p += max_select;
-  c->victim_unit = p; p += max_select;
-  c->victim_slot = p; p += max_select;
-  c->gather_unit = p; p += max_select;
-  c->gather_row = p; p += max_select;
+  c->slot_unit = p; p += P * cap1;
+  c->order = p; p += P * cap1;
+  c->order_tmp = p; p += P * cap1;
+  c->row_of = p; p += P * ms;
+  c->hits = p; p += P * ms;
+  c->misses = p; p += P * ms;
+  c->bypass = p; p += P * ms;
+  c->victim_unit = p; p += P * ms;
+  c->victim_slot = p; p += P * ms;
+  c->gather_unit = p; p += P * ms;
+  c->gather_row = p; p += P * ms;
   c->meta = p;
   if ((e = cudaEventCreateWithFlags(&c->ev_idx, cudaEventDisableTiming)) != cudaSuccess ||
       (e = cudaEventCreateWithFlags(&c->ev_ready, cudaEventDisableTiming)) != cudaSuccess ||
@@ -504,6 +565,7 @@ sf_status sf_refine_cache_create(sf_refine_cache** out, int num_units, size_t un
     return sf::cuda_fail(e, "sf_refine_cache_create: events/stream");
   }
   sf_status st = cache_clear(c, c->aux);
+  if (st == SF_OK && parts > 1) st = upload_table(c);
   if (st == SF_OK) {
     e = cudaStreamSynchronize(c->aux);
     if (e != cudaSuccess) st = sf::cuda_fail(e, "sf_refine_cache_create: init");
@@ -513,8 +575,14 @@ sf_status sf_refine_cache_create(sf_refine_cache** out, int num_units, size_t un
   return SF_OK;
 }
 
+sf_status sf_refine_cache_create(sf_refine_cache** out, int num_units, size_t unit_bytes, int capacity,
+                                 int max_select, const void* host_master, int device) {
+  return sf_refine_cache_create_parts(out, num_units, unit_bytes, 1, capacity, max_select, host_master, device);
+}
+
 sf_status sf_refine_cache_preload(sf_refine_cache* c, const int32_t* units, int n, sf_stream_t stream) {
   SF_REQUIRE(c, "sf_refine_cache_preload: null cache");
+  SF_REQUIRE(c->parts == 1, "sf_refine_cache_preload: not available for a partitioned cache");
   SF_REQUIRE(n >= 0 && n <= c->capacity, "sf_refine_cache_preload: n must be in [0, capacity]");
   SF_REQUIRE(n == 0 || units, "sf_refine_cache_preload: null units");
   DeviceGuard g(c->device);
@@ -541,15 +609,27 @@ sf_status sf_refine_cache_prefetch(sf_refine_cache* c, const int32_t* idx, const
   // the previous step's GEMV must have read the rows before they change
   if (c->used_pending && c->used_capture == cid) SF_CHECK_CUDA(cudaStreamWaitEvent(ss, c->ev_used, 0));
   const size_t smem = std::max(c->capacity, 1);
-  const CacheDev d = make_dev(c, idx, n);
-  SF_CHECK_CUDA(cudaFuncSetAttribute(cache_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(smem)));
-  cache_index_kernel<<<1, kIndexThreads, smem, ss>>>(d);
-  sf_status st = sf::check_launch("cache_index_kernel");
-  if (st != SF_OK) return st;
-  const int grid = std::min((c->max_select + 7) / 8, 2 * sf::sm_count());
-  cache_gather_kernel<<<grid, 256, 0, ss>>>(d);
-  st = sf::check_launch("cache_gather_kernel");
+  sf_status st;
+  if (c->parts == 1) {
+    const CacheDev d = make_dev(c, idx, n);
+    SF_CHECK_CUDA(cudaFuncSetAttribute(cache_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem)));
+    cache_index_kernel<<<1, kIndexThreads, smem, ss>>>(d);
+    st = sf::check_launch("cache_index_kernel");
+    if (st != SF_OK) return st;
+    const int grid = std::min((c->max_select + 7) / 8, 2 * sf::sm_count());
+    cache_gather_kernel<<<grid, 256, 0, ss>>>(d);
+    st = sf::check_launch("cache_gather_kernel");
+  } else {  // one CTA per part, then one gather over every part's misses
+    SF_CHECK_CUDA(cudaFuncSetAttribute(cache_index_parts_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem)));
+    cache_index_parts_kernel<<<c->parts, kIndexThreads, smem, ss>>>(c->table, idx, n);
+    st = sf::check_launch("cache_index_parts_kernel");
+    if (st != SF_OK) return st;
+    const int grid = std::min((c->parts * c->max_select + 7) / 8, 4 * sf::sm_count());
+    cache_gather_many_kernel<<<grid, 256, 0, ss>>>(c->table, c->parts);
+    st = sf::check_launch("cache_gather_many_kernel");
+  }
   if (st != SF_OK) return st;
   SF_CHECK_CUDA(cudaEventRecord(c->ev_ready, ss));
   c->ready_pending = true;
@@ -564,16 +644,25 @@ sf_status sf_refine_cache_sets(sf_refine_cache* c, int32_t* hits, int32_t* misse
   DeviceGuard g(c->device);
   sf_status st = wait_ready(c);
   if (st != SF_OK) return st;
-  int32_t meta[kMetaCount];
-  SF_CHECK_CUDA(cudaMemcpy(meta, c->meta, sizeof(meta), cudaMemcpyDeviceToHost));
-  counts[0] = meta[kHits];
-  counts[1] = meta[kMisses];
-  counts[2] = meta[kBypass];
-  if (hits && meta[kHits]) SF_CHECK_CUDA(cudaMemcpy(hits, c->hits, sizeof(int32_t) * meta[kHits], cudaMemcpyDeviceToHost));
-  if (misses && meta[kMisses])
-    SF_CHECK_CUDA(cudaMemcpy(misses, c->misses, sizeof(int32_t) * meta[kMisses], cudaMemcpyDeviceToHost));
-  if (bypass && meta[kBypass])
-    SF_CHECK_CUDA(cudaMemcpy(bypass, c->bypass, sizeof(int32_t) * meta[kBypass], cudaMemcpyDeviceToHost));
+  // the parts' lists, concatenated in part order (so each stays ascending)
+  std::vector<int32_t> meta(static_cast<size_t>(kMetaCount) * c->parts);
+  SF_CHECK_CUDA(cudaMemcpy(meta.data(), c->meta, sizeof(int32_t) * meta.size(), cudaMemcpyDeviceToHost));
+  counts[0] = counts[1] = counts[2] = 0;
+  const size_t ms = c->max_select;
+  for (int q = 0; q < c->parts; ++q) {
+    const int32_t* m = meta.data() + q * kMetaCount;
+    if (hits && m[kHits])
+      SF_CHECK_CUDA(cudaMemcpy(hits + counts[0], c->hits + q * ms, sizeof(int32_t) * m[kHits], cudaMemcpyDeviceToHost));
+    if (misses && m[kMisses])
+      SF_CHECK_CUDA(cudaMemcpy(misses + counts[1], c->misses + q * ms, sizeof(int32_t) * m[kMisses],
+                               cudaMemcpyDeviceToHost));
+    if (bypass && m[kBypass])
+      SF_CHECK_CUDA(cudaMemcpy(bypass + counts[2], c->bypass + q * ms, sizeof(int32_t) * m[kBypass],
+                               cudaMemcpyDeviceToHost));
+    counts[0] += m[kHits];
+    counts[1] += m[kMisses];
+    counts[2] += m[kBypass];
+  }
   return SF_OK;
 }
 
@@ -582,8 +671,10 @@ sf_status sf_refine_cache_slots(sf_refine_cache* c, int32_t* slot_units) {
   DeviceGuard g(c->device);
   sf_status st = wait_ready(c);
   if (st != SF_OK) return st;
-  if (c->capacity)
-    SF_CHECK_CUDA(cudaMemcpy(slot_units, c->slot_unit, sizeof(int32_t) * c->capacity, cudaMemcpyDeviceToHost));
+  for (int q = 0; q < c->parts && c->capacity; ++q)
+    SF_CHECK_CUDA(cudaMemcpy(slot_units + static_cast<size_t>(q) * c->capacity,
+                             c->slot_unit + static_cast<size_t>(q) * std::max(c->capacity, 1),
+                             sizeof(int32_t) * c->capacity, cudaMemcpyDeviceToHost));
   return SF_OK;
 }
 
@@ -592,8 +683,12 @@ sf_status sf_refine_cache_stats(sf_refine_cache* c, sf_cache_stats* out) {
   DeviceGuard g(c->device);
   sf_status st = wait_ready(c);
   if (st != SF_OK) return st;
-  int64_t s[kStatCount];
-  SF_CHECK_CUDA(cudaMemcpy(s, c->stats, sizeof(s), cudaMemcpyDeviceToHost));
+  std::vector<int64_t> all(static_cast<size_t>(kStatCount) * c->parts);
+  SF_CHECK_CUDA(cudaMemcpy(all.data(), c->stats, sizeof(int64_t) * all.size(), cudaMemcpyDeviceToHost));
+  int64_t s[kStatCount] = {};
+  for (int q = 0; q < c->parts; ++q)
+    for (int k = 0; k < kStatCount; ++k) s[k] += all[q * kStatCount + k];
+  s[kStSteps] /= c->parts;  // every part counts each step
   out->steps = s[kStSteps];
   out->hits = s[kStHits];
   out->misses = s[kStMisses];
@@ -622,6 +717,7 @@ sf_status sf_refine_cache_set_budget(sf_refine_cache* c, int budget) {
   SF_REQUIRE(c, "sf_refine_cache_set_budget: null cache");
   SF_REQUIRE(budget >= -1, "sf_refine_cache_set_budget: budget must be >= 0, or -1 for none");
   c->budget = budget < 0 || budget > c->max_select ? c->max_select : budget;
+  if (c->parts > 1) return upload_table(c);
   return SF_OK;
 }
 
@@ -648,6 +744,7 @@ sf_status sf_refine_group_create(sf_refine_group** out, sf_refine_cache* const* 
   SF_REQUIRE(count >= 1 && count <= 64, "sf_refine_group_create: count must be in [1, 64]");
   for (int i = 0; i < count; ++i) {
     SF_REQUIRE(caches[i] && idx[i] && n[i], "sf_refine_group_create: null entry %d", i);
+    SF_REQUIRE(caches[i]->parts == 1, "sf_refine_group_create: a partitioned cache cannot join a group");
     SF_REQUIRE(caches[i]->device == caches[0]->device, "sf_refine_group_create: caches on different devices");
     for (int j = 0; j < i; ++j) SF_REQUIRE(caches[j] != caches[i], "sf_refine_group_create: cache listed twice");
   }

@@ -28,10 +28,11 @@ refinement store in device memory; a percentage gives each matrix an LRU
 cache of that share of its columns fed from page-locked host memory on a side
 stream (every fetch completes before its GEMV).  ``kv_cache_pct`` None keeps
 the K/V refinement bits in device memory; a percentage keeps them in host
-memory behind one LRU cache per layer (units = token-heads, 64 bytes) that
+memory behind a KV refinement cache per layer (units = token-heads, 64
+bytes; one LRU per KV head holding that share of the head's capacity) that
 the attention reads with the deadline reading: only the union tokens cached
 when the step starts are refined, the misses are fetched for later steps
-(at most ``kv_budget`` per layer and step; the rest are late).
+(at most ``kv_budget`` per KV head and step; the rest are late).
 
 Every call is enqueued on the current stream (plus the side stream), so a
 step can be captured in a CUDA graph; before capturing after eager steps
@@ -174,8 +175,9 @@ class DecodeModel:
             qk.ref = qv.ref = None
             grp = s.n_q // Hkv
             k_max = count_half_up(self.p_tok, S)
-            cap = count_half_up(Fraction(cache_pct) / 100, Hkv * S)
-            cache = RefineCache(rows, host.shape[1] * 4, cap, max(1, Hkv * grp * k_max), host)
+            # one LRU per KV head: its share of the head's token-heads, its own budget
+            cap = count_half_up(Fraction(cache_pct) / 100, S)
+            cache = RefineCache(rows, host.shape[1] * 4, cap, max(1, grp * k_max), host, parts=Hkv)
             if budget is not None:
                 cache.set_budget(budget)
             kvq.ref_cache = cache

@@ -250,24 +250,27 @@ def test_decode_step_cache_mode_against_oracle(sf):
     refining only the union tokens cached when the step starts, and the cache
     sets of one weight matrix per input and of each layer's KV cache."""
     host = _host_model()
-    budget = 40
+    budget = 12                                   # per KV head and step
     m = _build(sf, host, weight_cache_pct=25, kv_cache_pct=20, kv_budget=budget)
     olayers, ohead, ofinal, okv = _oracle_model(host)
     # oracle LRUs: q (attn_in), o, gate (mlp_in), down, head; the KV caches
     worcs = {slot: [ocache.LRUCache(K, od.count_half_up(Fraction(25, 100), K)) for _ in range(NL)]
              for slot, K in (("attn_in", H), ("attn_out", HQ * D), ("mlp_in", H), ("mlp_mid", F))}
     horc = ocache.LRUCache(H, od.count_half_up(Fraction(25, 100), H))
-    korcs = [ocache.LRUCache(HKV * CAP, od.count_half_up(Fraction(20, 100), HKV * CAP)) for _ in range(NL)]
+    # one LRU per layer and KV head, over the head's units [g CAP, (g + 1) CAP)
+    kcap = od.count_half_up(Fraction(20, 100), CAP)
+    korcs = [[ocache.LRUCache(HKV * CAP, kcap) for _ in range(HKV)] for _ in range(NL)]
     first_of = {"attn_in": "q", "attn_out": "o", "mlp_in": "gate", "mlp_mid": "down"}
     for step in range(3):
         T = T0 + step
         avail = []
         for l in range(NL):
             a = np.zeros((HKV, T + 1), dtype=bool)
-            for u in korcs[l].snapshot():
-                gh, t = divmod(u, CAP)
-                if t <= T:
-                    a[gh, t] = True
+            for o in korcs[l]:
+                for u in o.snapshot():
+                    gh, t = divmod(u, CAP)
+                    if t <= T:
+                        a[gh, t] = True
             avail.append(a)
         m.x_in.copy_(torch.from_numpy(_embedding(7200 + step)))
         m.step(T)
@@ -286,11 +289,13 @@ def test_decode_step_cache_mode_against_oracle(sf):
         want = horc.step(hb["idx"][0].cpu().numpy()[: int(hb["n"][0].item())].tolist())
         assert m.head.cache.sets()["misses"] == want["misses"]
         for l in range(NL):
-            units = [g * CAP + int(t) for g, u in enumerate(m.union(l)) for t in u]
-            want = korcs[l].step(units, budget=budget)
+            wants = [korcs[l][g].step([g * CAP + int(t) for t in u], budget=budget)
+                     for g, u in enumerate(m.union(l))]
             got = m.layers[l]["kv_cache"].sets()
-            assert got["hits"] == want["hits"] and got["misses"] == want["misses"]
-            assert got["bypass"] == want["bypass"]
-    assert sum(o.late for o in korcs) > 0 and sum(o.hits for o in korcs) > 0
-    assert m.cache_totals("kv")["late"] == sum(o.late for o in korcs)
+            assert got["hits"] == sum((w["hits"] for w in wants), [])
+            assert got["misses"] == sum((w["misses"] for w in wants), [])
+            assert got["bypass"] == sum((w["bypass"] for w in wants), [])
+    ko = [o for lo in korcs for o in lo]
+    assert sum(o.late for o in ko) > 0 and sum(o.hits for o in ko) > 0
+    assert m.cache_totals("kv")["late"] == sum(o.late for o in ko)
     m.close()

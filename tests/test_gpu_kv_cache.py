@@ -42,8 +42,8 @@ def _setup(sf, Hq, Hkv, T, S, d, seed, cap_pct):
     master = torch.cat([k.ref.view(-1, 8), v.ref.view(-1, 8)], dim=1).cpu().contiguous().pin_memory()
     k_tokens = count_fraction(1, T)
     grp = Hq // Hkv
-    cap = count_fraction(cap_pct, Hkv * T)
-    cache = sf.RefineCache(Hkv * S, 64, cap, Hkv * grp * k_tokens, master)
+    cap = count_fraction(cap_pct, T)                # per KV head: one LRU each
+    cache = sf.RefineCache(Hkv * S, 64, cap, grp * k_tokens, master, parts=Hkv)
     k.ref = v.ref = None                            # the stores are not read
     kvc = sf.QKV(k, v, row_stride=S, ref_cache=cache)
     ok = oquant.quantize_nested(Kf[:, :T].reshape(-1, d), d, 2, 2)
@@ -55,9 +55,9 @@ def _setup(sf, Hq, Hkv, T, S, d, seed, cap_pct):
 def test_attention_with_kv_refinement_cache(sf, path):
     Hq, Hkv, d, T, S = 32, 8, 128, 6000, 6040
     kvc, cache, ok, ov, k_tokens, cap = _setup(sf, Hq, Hkv, T, S, d, 811, 10)
-    budget = 700
+    budget = 90                                     # per KV head and step
     cache.set_budget(budget)
-    orc = ocache.LRUCache(Hkv * S, cap)
+    orcs = [ocache.LRUCache(Hkv * S, cap) for _ in range(Hkv)]   # the parts: units [g S, (g + 1) S)
     grp = Hq // Hkv
     units = torch.zeros(Hkv * grp * k_tokens, dtype=torch.int32, device="cuda")
     n_units = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -67,12 +67,12 @@ def test_attention_with_kv_refinement_cache(sf, path):
     try:
         for step, qseed in enumerate([901, 901, 902, 901, 901]):
             qb = gen_query(qseed, Hq, d)
-            snap = orc.snapshot()
             avail = np.zeros((Hkv, T), dtype=bool)
-            for u in snap:
-                g, t = divmod(u, S)
-                if t < T:
-                    avail[g, t] = True
+            for orc in orcs:
+                for u in orc.snapshot():
+                    g, t = divmod(u, S)
+                    if t < T:
+                        avail[g, t] = True
             out, sel, sel_n = sf.attn_decode_refine(dev(qb.view(np.int16)).view(torch.bfloat16), kvc, Hkv, T,
                                                     k_tokens)
             sf.attn_union_units(sel, sel_n, Hkv, grp * k_tokens, S, units, n_units)
@@ -88,18 +88,22 @@ def test_attention_with_kv_refinement_cache(sf, path):
             np.testing.assert_array_equal(units.cpu().numpy()[: len(want_units)], want_units)
             err = np.abs(out.cpu().numpy().astype(np.float64) - ref["out"]).max()
             assert err <= ATTN_TOL, f"step {step}: max-abs error {err}"
-            want = orc.step(want_units, budget=budget)
+            wants = [orcs[g].step([u for u in want_units if u // S == g], budget=budget) for g in range(Hkv)]
             got = cache.sets()
-            assert got["hits"] == want["hits"] and got["misses"] == want["misses"]
-            assert got["bypass"] == want["bypass"]
-            late += len(want["late"])
+            assert got["hits"] == sum((w["hits"] for w in wants), [])
+            assert got["misses"] == sum((w["misses"] for w in wants), [])
+            assert got["bypass"] == sum((w["bypass"] for w in wants), [])
+            late += sum(len(w["late"]) for w in wants)
             assert cache.stats().late == late
             if step == 0:
                 assert not any(len(e) for e in ref["refined"])        # a cold cache refines nothing
             if step == 1:
-                assert sum(len(e) for e in ref["refined"]) == min(budget, len(want_units))
-        assert late > 0 and orc.hits > 0
-        assert {u: s for s, u in enumerate(cache.slots()) if u >= 0} == orc.snapshot()
+                for g in range(Hkv):
+                    assert len(ref["refined"][g]) == min(budget, len(ref["union"][g]))
+        assert late > 0 and sum(o.hits for o in orcs) > 0
+        got_slots = {u: s for s, u in enumerate(cache.slots()) if u >= 0}
+        want_slots = {u: g * cap + sl for g, o in enumerate(orcs) for u, sl in o.snapshot().items()}
+        assert got_slots == want_slots
     finally:
         sf.attn_set_path(sf.ATTN_AUTO)
         cache.close()
