@@ -84,6 +84,9 @@ def parse():
                     help="KV refinement cache, percent of the token-heads (negative: the whole store in HBM)")
     ap.add_argument("--kv-budget", type=int, default=512,
                     help="KV refinement misses fetched per KV head and step at most (negative: no limit)")
+    ap.add_argument("--weight-deadline", type=int, default=1,
+                    help="1: GEMVs refine the selected columns already cached and misses are fetched for later "
+                         "steps; 0: every GEMV waits for the fetch of its own selection")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-extras", action="store_true", help="skip e2e / resident-only / roofline legs")
     ap.add_argument("--hotpath-context", type=int, default=32768,
@@ -786,7 +789,7 @@ def step_model(args, sf, torch, dev, layers):
     budget = None if args.kv_budget < 0 else args.kv_budget
     m = DecodeModel(shape, weight, norm, kv, capacity=args.context, p=Fraction(TOPK_PCT, 100),
                     p_tok=Fraction(TOK_PCT, 100), weight_cache_pct=CACHE_PCT, kv_cache_pct=kv_pct,
-                    kv_budget=budget, device=dev)
+                    kv_budget=budget, weight_deadline=bool(args.weight_deadline), device=dev)
     return m, T
 
 
@@ -992,7 +995,10 @@ def run_sf(args, rank, world, local_rank, dist):
         "config": {"workload": workload_step(args.context), "model_shape": "Llama-3.1-8B (32 layers, LM head 128256)",
                    "context": args.context, "layers": args.layers, "batch": 1,
                    "weights": "3-bit resident + 1-bit refinement, group 128", "kv": "2-bit + 2-bit, per token-head",
-                   "topk_channels": "3% of each GEMV input", "weight_cache": "10% LRU per matrix",
+                   "topk_channels": "3% of each GEMV input",
+                   "weight_cache": "10% LRU per matrix, " + ("deadline reading (misses fetched for later steps)"
+                                                              if args.weight_deadline else
+                                                              "every GEMV waits for its misses"),
                    "topk_tokens": "1% per query head", "kv_cache": (f"{args.kv_cache_pct}% of token-heads, "
                                                                     f"one LRU per KV head, budget {args.kv_budget} per head and step"
                                                                     if args.kv_cache_pct >= 0 else "store in HBM"),

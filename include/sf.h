@@ -233,6 +233,21 @@ sf_status sf_refine_cache_destroy(sf_refine_cache* c);
 sf_status sf_refine_cache_set_budget(sf_refine_cache* c, int budget);
 
 /*
+ * sf_refine_cache_set_deadline -- the deadline reading for the cache of one
+ * weight matrix (on != 0; off by default).  A batch-1 GEMV given this cache
+ * (sf_gemv_refine_batch1) then does not wait for the fetches of its own
+ * selection: it refines the selected columns that are cached when it runs
+ * (E = S ∩ cached, read from the cache's index as its last prefetch left
+ * it) and leaves the others at resident precision (a miss keeps resident
+ * precision: rag-lover.com explainer, 限界と未検証の範囲).  The caller issues
+ * the prefetch of S after the GEMV, so the misses arrive for later steps and
+ * no host-link transfer sits between the selection and the GEMV.  The
+ * generic sf_gemv_refine refuses such a cache (SF_EINVAL).
+ * Constraints: a cache of parts = 1.
+ */
+sf_status sf_refine_cache_set_deadline(sf_refine_cache* c, int on);
+
+/*
  * A group batches the prefetch of several caches whose selections live in
  * fixed device buffers (typically the weight matrices of one layer): one
  * launch resolves every cache's step (one CTA per cache) and one launch

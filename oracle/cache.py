@@ -24,6 +24,11 @@ C7  a fetch budget F (the deadline reading, for caches whose consumer does
     neither fetched nor cached nor touched, so their precision stays the
     resident one (a miss keeps resident precision: rag-lover.com explainer,
     限界と未検証の範囲).  No budget (F = None) is C1-C5 unchanged.
+C8  the deadline reading of a weight matrix's cache (its GEMV does not wait
+    for the fetch of its own selection): the GEMV refines E = S ∩ (units
+    cached when the step starts), :func:`effective_set`; then the step runs
+    as above on S, so the misses are fetched for later steps.  C6 then holds
+    with E in place of S.
 
 ``preload`` fills an empty cache with the given units in slots 0, 1, ...
 with last_use = -1 (older than any step), and counts nothing.
@@ -97,3 +102,9 @@ class LRUCache:
     def snapshot(self) -> dict[int, int]:
         """unit -> slot for every cached unit."""
         return dict(self.slot_of)
+
+
+def effective_set(S, cached) -> list[int]:
+    """C8: the selected units that were cached when the step started
+    (``cached``: a set or dict of units), ascending."""
+    return [int(u) for u in S if int(u) in cached]

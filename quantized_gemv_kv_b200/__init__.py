@@ -84,6 +84,7 @@ _SIGS = {
     "sf_refine_cache_reset": ([_p], _i),
     "sf_refine_cache_destroy": ([_p], _i),
     "sf_refine_cache_set_budget": ([_p, _i], _i),
+    "sf_refine_cache_set_deadline": ([_p, _i], _i),
     "sf_refine_group_create": ([ctypes.POINTER(_p), ctypes.POINTER(_p), ctypes.POINTER(_p), ctypes.POINTER(_p), _i],
                                _i),
     "sf_refine_group_prefetch": ([_p, _p, _p], _i),
@@ -264,6 +265,12 @@ class RefineCache:
 
     def reset(self) -> None:
         _check(_lib.sf_refine_cache_reset(self._h))
+
+    def set_deadline(self, on: bool = True) -> None:
+        """Deadline reading for a weight matrix's cache
+        (``sf_refine_cache_set_deadline``): the batch-1 GEMV refines only the
+        selected columns already cached and does not wait for fetches."""
+        _check(_lib.sf_refine_cache_set_deadline(self._h, 1 if on else 0))
 
     def set_budget(self, budget: int | None) -> None:
         """Per-step fetch budget (``sf_refine_cache_set_budget``); None = no limit."""

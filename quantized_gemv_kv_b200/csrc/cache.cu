@@ -334,6 +334,7 @@ struct sf_refine_cache {
   int capacity = 0;    // slots per part
   int max_select = 0;  // selected units per part and step at most
   int budget = 0;  // per-step fetch limit; max_select = no limit
+  bool deadline = false;  // GEMVs refine only the selected units cached when they run
   const void* host_master = nullptr;
   const void* master_dev = nullptr;
   bool registered_here = false;
@@ -445,7 +446,9 @@ namespace sf {
 
 sf_status cache_view_for_gemv(sf_refine_cache* c, cudaStream_t stream, CacheView* v) {
   SF_REQUIRE(c->budget >= c->max_select,
-             "sf_gemv_refine: a GEMV needs every selected column fetched; this cache has a fetch budget");
+             "sf_gemv_refine: a GEMV needs every selected column fetched; this cache has a fetch budget "
+             "(use the deadline reading, sf_refine_cache_set_deadline)");
+  SF_REQUIRE(!c->deadline, "sf_gemv_refine: only the batch-1 GEMV reads a cache in the deadline reading");
   return cache_view_for_reader(c, stream, v);
 }
 
@@ -477,6 +480,8 @@ sf_status cache_view_for_writer(sf_refine_cache* c, cudaStream_t stream, CacheWr
   w->unit_words = static_cast<int>(c->unit_bytes / 4);
   return SF_OK;
 }
+
+bool cache_deadline(const sf_refine_cache* c) { return c->deadline; }
 
 sf_status cache_mark_used(sf_refine_cache* c, cudaStream_t stream) {
   SF_CHECK_CUDA(cudaEventRecord(c->ev_used, stream));
@@ -712,6 +717,13 @@ sf_status sf_refine_cache_reset(sf_refine_cache* c) {
 }
 
 sf_status sf_refine_cache_destroy(sf_refine_cache* c) { return cache_free(c); }
+
+sf_status sf_refine_cache_set_deadline(sf_refine_cache* c, int on) {
+  SF_REQUIRE(c, "sf_refine_cache_set_deadline: null cache");
+  SF_REQUIRE(c->parts == 1, "sf_refine_cache_set_deadline: for the cache of one weight matrix (parts = 1)");
+  c->deadline = on != 0;
+  return SF_OK;
+}
 
 sf_status sf_refine_cache_set_budget(sf_refine_cache* c, int budget) {
   SF_REQUIRE(c, "sf_refine_cache_set_budget: null cache");

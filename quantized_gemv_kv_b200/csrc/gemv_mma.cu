@@ -66,6 +66,7 @@ struct MJob {
   const uint16_t* zero;
   const uint32_t* ref_rows;  // nullptr: resident only
   const int32_t* row_of;     // nullptr: refinement row = channel index
+  const int32_t* unit_slot;  // deadline reading: refinement row of channel j = unit_slot[j] (-1: not refined)
   float* y;
   int N, unit_words, tile_begin;
 };
@@ -204,6 +205,8 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
   float fsc[SPW], gsm[SPW], cconst[SPW];
   int nsl[SPW], psl[SPW];
   int ntc[SPW];  // selected channels of the slice corrected on the tensor cores (the rest in fp32)
+  uint32_t hl_l[SPW];  // lane k < ntc: (high, low) halves of x of listed channel k
+  int grp_l[SPW];      // and its group inside the slice (-1: none)
 
   // Copies are issued tile by tile in order, so their addresses advance by
   // fixed strides and are recomputed only where the next matrix begins.
@@ -265,7 +268,9 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
     for (int sp = 0; sp < SPW; ++sp) {
       r_row[sp] = J.ref_rows;
       if (r_has && lane < ntc[sp]) {
-        const int rr = J.row_of ? J.row_of[psl[sp] + lane] : 256 * (slice0 + sp) + mylist[sp * kCorrList + lane];
+        const int ch = 256 * (slice0 + sp) + mylist[sp * kCorrList + lane];
+        int rr = J.unit_slot ? J.unit_slot[ch] : (J.row_of ? J.row_of[psl[sp] + lane] : ch);
+        rr = rr < 0 ? 0 : rr;  // not cached (deadline reading): any row; its B column is zero
         r_row[sp] = J.ref_rows + static_cast<size_t>(rr) * J.unit_words;
       }
     }
@@ -332,8 +337,8 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
     // slice is then corrected by the fp32 loop
     if (__any_sync(0xffffffffu, !(fabsf(xv) < kCorrXMax))) nl = 0;
     ntc[sp] = nl;
-    uint32_t hl = 0;  // lane k: (high, low) halves of x of listed channel k
-    int grp = -1;     // and its group inside the slice
+    uint32_t hl = 0;
+    int grp = -1;
     if (lane < nl) {
       const int ch = mylist[sp * kCorrList + lane];
       const __half hi = __float2half_rn(xv);
@@ -341,7 +346,20 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
       hl = static_cast<uint32_t>(__half_as_ushort(hi)) | (static_cast<uint32_t>(__half_as_ushort(lo)) << 16);
       grp = ch >> 7;
     }
-    {
+    hl_l[sp] = hl;
+    grp_l[sp] = grp;
+  }
+  // the correction MMA's B fragments and offset constant for the job the
+  // compute cursor is in: a job reading a cache in the deadline reading drops
+  // the listed channels not cached (their x becomes 0)
+  auto build_corr = [&](const MJob& J) {
+#pragma unroll
+    for (int sp = 0; sp < SPW; ++sp) {
+      const int nl = ntc[sp];
+      uint32_t hl = hl_l[sp];
+      const int grp = grp_l[sp];
+      if (J.unit_slot != nullptr && lane < nl && J.unit_slot[256 * (slice0 + sp) + mylist[sp * kCorrList + lane]] < 0)
+        hl = 0u;
       const float part = lane < nl ? __half2float(__ushort_as_half(static_cast<unsigned short>(hl & 0xFFFFu))) +
                                          __half2float(__ushort_as_half(static_cast<unsigned short>(hl >> 16)))
                                    : 0.0f;
@@ -352,23 +370,24 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
         x1 += __shfl_xor_sync(0xffffffffu, x1, o);
       }
       cconst[sp] = -(1024.0f + m_f) * (myslot ? x1 : x0);
-    }
-    // column n of the correction MMA = (group n / 2, part n % 2)
+      // column n of the correction MMA = (group n / 2, part n % 2)
 #pragma unroll
-    for (int kb = 0; kb < 2; ++kb)
+      for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        uint32_t v = 0;
+        for (int r = 0; r < 2; ++r) {
+          uint32_t v = 0;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int k = 16 * kb + 2 * tig + 8 * r + h;  // < 32: a lane of the warp
-          const uint32_t hk = __shfl_sync(0xffffffffu, hl, k);
-          const int gk = __shfl_sync(0xffffffffu, grp, k);
-          if (g8 < 4 && k < nl && gk == (g8 >> 1)) v |= ((g8 & 1) ? (hk >> 16) : (hk & 0xFFFFu)) << (16 * h);
+          for (int h = 0; h < 2; ++h) {
+            const int k = 16 * kb + 2 * tig + 8 * r + h;  // < 32: a lane of the warp
+            const uint32_t hk = __shfl_sync(0xffffffffu, hl, k);
+            const int gk = __shfl_sync(0xffffffffu, grp, k);
+            if (g8 < 4 && k < nl && gk == (g8 >> 1)) v |= ((g8 & 1) ? (hk >> 16) : (hk & 0xFFFFu)) << (16 * h);
+          }
+          cb[sp][kb][r] = v;
         }
-        cb[sp][kb][r] = v;
-      }
-  }
+    }
+  };
+  if (my_tiles > 0) build_corr(a.job[c_jb0]);
 
   if (my_tiles > 0) r_seek();
   for (int i = 0; i < kStages - 1 && i < my_tiles; ++i) issue_refs(i);
@@ -397,6 +416,7 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
     if (t == k_next) {
       ++k_jb;
       k_next = k_jb + 1 < a.njobs ? a.job[k_jb + 1].tile_begin : 0x7FFFFFFF;
+      build_corr(a.job[k_jb]);
     }
     const MJob& J = a.job[k_jb];
     const int row0 = (t - J.tile_begin) * kRows;
@@ -487,7 +507,8 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
             kk -= c;
           }
           if (((ch >> 7) & 1) != myslot) continue;
-          const int rr = J.row_of ? J.row_of[psl[sp] + k] : ch;
+          const int rr = J.unit_slot ? J.unit_slot[ch] : (J.row_of ? J.row_of[psl[sp] + k] : ch);
+          if (rr < 0) continue;  // not cached at the step's start (deadline reading): resident precision
           const uint32_t word = J.ref_rows[static_cast<size_t>(rr) * J.unit_words + ((row0 * BF) >> 5)];
           const float xv = sfd::bf16_bits_to_float(a.x[ch]);
           corr = fmaf(xv, i2f_small(static_cast<int>((word >> (roff + BF * myrow)) & fmask)) - m_f, corr);
@@ -631,11 +652,15 @@ extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, c
     row_tiles += W->N / kRows;
     if (jobs[i].cache) {
       sf::CacheView v{};
-      const sf_status st = sf::cache_view_for_gemv(jobs[i].cache, s, &v);
+      const bool deadline = sf::cache_deadline(jobs[i].cache);
+      const sf_status st = deadline ? sf::cache_view_for_reader(jobs[i].cache, s, &v)
+                                    : sf::cache_view_for_gemv(jobs[i].cache, s, &v);
       if (st != SF_OK) return st;
       SF_REQUIRE(v.unit_words == J.unit_words, "sf_gemv_refine_batch1: cache unit size does not match N*b_f/8");
+      SF_REQUIRE(!deadline || v.num_units == K, "sf_gemv_refine_batch1: a deadline cache must have K units");
       J.ref_rows = v.rows;
-      J.row_of = v.row_of;
+      J.row_of = deadline ? nullptr : v.row_of;
+      J.unit_slot = deadline ? v.unit_slot : nullptr;
     } else if (jobs[i].use_ref_store) {
       SF_REQUIRE(W->ref, "sf_gemv_refine_batch1: use_ref_store without W->ref");
       J.ref_rows = W->ref;

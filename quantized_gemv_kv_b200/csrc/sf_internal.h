@@ -60,6 +60,8 @@ sf_status cache_view_for_gemv(sf_refine_cache* c, cudaStream_t stream, CacheView
 // prefetch left it); makes `stream` wait for that prefetch.
 sf_status cache_view_for_reader(sf_refine_cache* c, cudaStream_t stream, CacheView* v);
 sf_status cache_mark_used(sf_refine_cache* c, cudaStream_t stream);
+// Whether the cache is read in the deadline reading (sf_refine_cache_set_deadline).
+bool cache_deadline(const sf_refine_cache* c);
 
 // For a writer of units (the KV append): the host master's device-mapped
 // address and the device rows, so a new unit's bytes go to both; makes

@@ -26,7 +26,9 @@ refines the top round_half_up(p_tok (T + 1)) tokens per query head.
 Refinement sources.  ``weight_cache_pct`` None keeps every weight matrix's
 refinement store in device memory; a percentage gives each matrix an LRU
 cache of that share of its columns fed from page-locked host memory on a side
-stream (every fetch completes before its GEMV).  ``kv_cache_pct`` None keeps
+stream: every fetch completes before its GEMV, or, with
+``weight_deadline``, the GEMV refines only the selected columns already
+cached and the misses are fetched after it for later steps.  ``kv_cache_pct`` None keeps
 the K/V refinement bits in device memory; a percentage keeps them in host
 memory behind a KV refinement cache per layer (units = token-heads, 64
 bytes; one LRU per KV head holding that share of the head's capacity) that
@@ -83,7 +85,7 @@ def count_half_up(p: Fraction, n: int) -> int:
 class _Matrix:
     """A quantized weight matrix with its refinement source."""
 
-    def __init__(self, W: torch.Tensor, shape: Shape, k_sel: int, cache_pct, device):
+    def __init__(self, W: torch.Tensor, shape: Shape, k_sel: int, cache_pct, device, deadline: bool = False):
         b_r, b_f = shape.w_bits
         N, K = W.shape
         self.qw = pack_batch1(quantize_nested(W, shape.group, b_r, b_f), drop_canonical=True)
@@ -94,6 +96,8 @@ class _Matrix:
             self.qw.ref = None
             cap = count_half_up(Fraction(cache_pct) / 100, K)
             self.cache = RefineCache(K, N * b_f // 8, cap, max(k_sel, 1), self.host)
+            if deadline:
+                self.cache.set_deadline(True)
         self.y = torch.empty(N, dtype=torch.float32, device=device)
 
     def close(self):
@@ -113,12 +117,13 @@ class DecodeModel:
 
     def __init__(self, shape: Shape, weight, norm, kv, capacity: int, p: Fraction = Fraction(3, 100),
                  p_tok: Fraction = Fraction(1, 100), weight_cache_pct=None, kv_cache_pct=None,
-                 kv_budget: int | None = None, record: bool = False, device=None):
+                 kv_budget: int | None = None, weight_deadline: bool = False, record: bool = False, device=None):
         self.s = shape
         self.dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
         self.p, self.p_tok = Fraction(p), Fraction(p_tok)
         self.S = capacity
         self.record = record
+        self.deadline = weight_deadline and weight_cache_pct is not None
         H, F, d = shape.hidden, shape.mlp, shape.head_dim
         Hq, Hkv = shape.n_q, shape.n_kv
         dev = self.dev
@@ -137,7 +142,7 @@ class DecodeModel:
             for name in MATS:
                 N, K = shape.mat_shape(name)
                 W = weight(l, name, N, K)
-                L[name] = _Matrix(W, shape, self.k_in[slot_of[name]], weight_cache_pct, dev)
+                L[name] = _Matrix(W, shape, self.k_in[slot_of[name]], weight_cache_pct, dev, self.deadline)
                 del W
             L["norm1"] = norm(l, "norm1").to(dev, torch.float32).contiguous()
             L["norm2"] = norm(l, "norm2").to(dev, torch.float32).contiguous()
@@ -151,7 +156,8 @@ class DecodeModel:
             L["T0"] = T0
             self.layers.append(L)
         Nh, Kh = shape.mat_shape("head")
-        self.head = _Matrix(weight(-1, "head", Nh, Kh), shape, self.k_in["head"], weight_cache_pct, dev)
+        self.head = _Matrix(weight(-1, "head", Nh, Kh), shape, self.k_in["head"], weight_cache_pct, dev,
+                            self.deadline)
         self.final_norm = norm(-1, "final").to(dev, torch.float32).contiguous()
         self._alloc_buffers()
         self._build_jobs(weight_cache_pct is not None)
@@ -254,9 +260,11 @@ class DecodeModel:
         if refine:
             (self.sel_jobs[slot][l] if l >= 0 else self.sel_head).run()
             grp = self.wgroups[l].get(slot) if l >= 0 else self.head_group
-            if grp is not None:
-                grp.prefetch(main, self.side)
+            if grp is not None and not self.deadline:
+                grp.prefetch(main, self.side)   # the GEMV waits for these fetches
             (self.jobs[l][slot] if l >= 0 else self.head_job).run(x, b["act"][li])
+            if grp is not None and self.deadline:
+                grp.prefetch(main, self.side)   # for later steps; nothing waits within this one
         else:
             act_prepare(x, b["act"][li])
             (self.jobs0[l][slot] if l >= 0 else self.head_job0).run(x, b["act"][li])

@@ -179,3 +179,50 @@ def test_gemv_batch1_huge_selected_outliers(sf, b_r, b_f):
     assert np.all(np.isfinite(y))
     y_ref, a = ogemv.gemv_refine(m["qz"], x, S)
     _check_gemv(y[None, :], y_ref, a)
+
+
+@pytest.mark.parametrize("b_r,b_f", [(3, 1), (2, 2)])
+def test_gemv_batch1_deadline_caches(sf, b_r, b_f):
+    """The deadline reading: each GEMV refines only the selected columns its
+    cache held when the step started (oracle: C8), then the step's prefetch
+    fetches the misses for later steps; four steps over q/k/v-shaped jobs."""
+    K, Ns = 4096, (4096, 1024, 1024)
+    k = count_fraction(3, K)
+    cap = count_fraction(10, K)
+    mats = _mats(sf, K, Ns, 2700 + b_r, b_r=b_r, b_f=b_f)
+    for m in mats:
+        N = m["qw"].N
+        m["cache"] = sf.RefineCache(K, N * b_f // 8, cap, k, m["qw"].ref.cpu().contiguous().pin_memory())
+        m["cache"].set_deadline(True)
+        m["orc"] = ocache.LRUCache(K, cap)
+    idx = torch.zeros(k, dtype=torch.int32, device="cuda")
+    n = torch.zeros(1, dtype=torch.int32, device="cuda")
+    act = torch.zeros(sf.act_bytes(K) // 4, dtype=torch.int32, device="cuda")
+    grp = sf.RefineGroup([(m["cache"], idx, n) for m in mats])
+    jobs = sf.Batch1Jobs([(m["qw"], m["cache"], False, m["y"]) for m in mats])
+    side = torch.cuda.Stream()
+    outl = outlier_channels(2800 + K, K, count_fraction("1/2", K))
+    refined = 0
+    for step in range(4):
+        x = gen_activations(2900 + step, 1, K, outl, 30.0)
+        xd = bf16_dev(x)
+        sf.select_topk_act(xd, k, idx, n, act)
+        jobs.run(xd, act)                                  # refines S ∩ cached
+        grp.prefetch(torch.cuda.current_stream(), side)    # then fetches the misses
+        torch.cuda.synchronize()
+        S = oselect.select_topk(x, k)
+        for m in mats:
+            E = ocache.effective_set(S, m["orc"].snapshot())
+            y_ref, a = ogemv.gemv_refine(m["qz"], x, E)
+            _check_gemv(m["y"].cpu().numpy()[None, m["rows"]], y_ref, a)
+            want = m["orc"].step(S.tolist())
+            got = m["cache"].sets()
+            assert got["hits"] == want["hits"] and got["misses"] == want["misses"]
+        refined += len(E)
+    assert refined > 0                                     # later steps do refine cached columns
+    # the generic GEMV refuses a cache in the deadline reading
+    with pytest.raises(sf.SfError, match="deadline"):
+        sf.gemv_refine(mats[0]["qw"], xd, idx, n, cache=mats[0]["cache"])
+    grp.close()
+    for m in mats:
+        m["cache"].close()

@@ -110,10 +110,13 @@ def _check_gemv(y_gpu, y_ref, abs_sum):
     assert np.all(err <= bound), f"worst err/bound = {(err / np.maximum(bound, 1e-300)).max():.3g}"
 
 
-def _linear_check(qz, x_bits, idx, n, y_gpu, k):
+def _linear_check(qz, x_bits, idx, n, y_gpu, k, cached=None):
+    """Selection bit-exact; the GEMV refines S, or in the deadline reading
+    (``cached``: the units its cache held when the step started) S ∩ cached."""
     S = oselect.select_topk(x_bits[None, :], k)
     np.testing.assert_array_equal(idx[:n], S)
-    y_ref, a = ogemv.gemv_refine(qz, x_bits[None, :], S)
+    E = S if cached is None else ocache.effective_set(S, cached)
+    y_ref, a = ogemv.gemv_refine(qz, x_bits[None, :], E)
     _check_gemv(np.asarray(y_gpu)[None, :], y_ref, a)
     return S
 
@@ -123,9 +126,11 @@ def _append_rows(kv, new_rows, T):
     return od.kv_append(kv, new_rows, HKV, T, 2, 2)
 
 
-def _check_step(m, olayers, ohead, ofinal, okv, T, available=None):
+def _check_step(m, olayers, ohead, ofinal, okv, T, available=None, wcached=None):
     """Teacher-forced checks of one recorded step at position T; returns the
-    oracle caches with the GPU's new token appended."""
+    oracle caches with the GPU's new token appended.  ``wcached[(l, slot)]``:
+    the deadline reading's cached units of the matrices reading that input."""
+    wc = (lambda l, slot: None) if wcached is None else (lambda l, slot: wcached[(l, slot)])
     k_tok = od.count_half_up(P_TOK, T + 1)
     nxt = []
     x_hist = m.x_hist.cpu().numpy().astype(np.float64)
@@ -139,9 +144,9 @@ def _check_step(m, olayers, ohead, ofinal, okv, T, available=None):
         raw = m.qkv_raw[l].cpu().numpy()
         idx, n = b["attn_in"]["idx"][l].cpu().numpy(), int(b["attn_in"]["n"][l].item())
         k_in = m.k_in["attn_in"]
-        _linear_check(OL["q"], n1, idx, n, raw[:HQ * D], k_in)
-        _linear_check(OL["k"], n1, idx, n, raw[HQ * D:(HQ + HKV) * D], k_in)
-        _linear_check(OL["v"], n1, idx, n, raw[(HQ + HKV) * D:], k_in)
+        _linear_check(OL["q"], n1, idx, n, raw[:HQ * D], k_in, wc(l, "attn_in"))
+        _linear_check(OL["k"], n1, idx, n, raw[HQ * D:(HQ + HKV) * D], k_in, wc(l, "attn_in"))
+        _linear_check(OL["v"], n1, idx, n, raw[(HQ + HKV) * D:], k_in, wc(l, "attn_in"))
         q_raw = raw[:HQ * D].astype(np.float64).reshape(HQ, D)
         k_raw = raw[HQ * D:(HQ + HKV) * D].astype(np.float64).reshape(HKV, D)
         v_raw = raw[(HQ + HKV) * D:].astype(np.float32).reshape(HKV, D)
@@ -176,7 +181,7 @@ def _check_step(m, olayers, ohead, ofinal, okv, T, available=None):
         ab = _bits(b["attn_out"]["x"][l])
         np.testing.assert_array_equal(ab, f32_to_bf16_bits(att.reshape(-1)))
         idx, n = b["attn_out"]["idx"][l].cpu().numpy(), int(b["attn_out"]["n"][l].item())
-        _linear_check(OL["o"], ab, idx, n, L["o"].y.cpu().numpy(), m.k_in["attn_out"])
+        _linear_check(OL["o"], ab, idx, n, L["o"].y.cpu().numpy(), m.k_in["attn_out"], wc(l, "attn_out"))
         np.testing.assert_array_equal(h_hist[l], (x_hist[l].astype(np.float32) + L["o"].y.cpu().numpy()))
         # MLP
         n2 = _bits(b["mlp_in"]["x"][l])
@@ -184,20 +189,20 @@ def _check_step(m, olayers, ohead, ofinal, okv, T, available=None):
         idx, n = b["mlp_in"]["idx"][l].cpu().numpy(), int(b["mlp_in"]["n"][l].item())
         g = L["gate"].y.cpu().numpy()
         u = L["up"].y.cpu().numpy()
-        _linear_check(OL["gate"], n2, idx, n, g, m.k_in["mlp_in"])
-        _linear_check(OL["up"], n2, idx, n, u, m.k_in["mlp_in"])
+        _linear_check(OL["gate"], n2, idx, n, g, m.k_in["mlp_in"], wc(l, "mlp_in"))
+        _linear_check(OL["up"], n2, idx, n, u, m.k_in["mlp_in"], wc(l, "mlp_in"))
         mid = _bits(b["mlp_mid"]["x"][l])
         _check_bf16(mid, od.silu(g.astype(np.float64)) * u.astype(np.float64))
         idx, n = b["mlp_mid"]["idx"][l].cpu().numpy(), int(b["mlp_mid"]["n"][l].item())
         dn = L["down"].y.cpu().numpy()
-        _linear_check(OL["down"], mid, idx, n, dn, m.k_in["mlp_mid"])
+        _linear_check(OL["down"], mid, idx, n, dn, m.k_in["mlp_mid"], wc(l, "mlp_mid"))
         np.testing.assert_array_equal(x_hist[l + 1], h_hist[l].astype(np.float32) + dn)
         nxt.append(okv2)
     # final norm and LM head
     nf = _bits(m.buf["head"]["x"][0])
     _check_bf16(nf, od.rms_norm(x_hist[NL], ofinal))
     idx, n = m.buf["head"]["idx"][0].cpu().numpy(), int(m.buf["head"]["n"][0].item())
-    _linear_check(ohead, nf, idx, n, m.logits.cpu().numpy(), m.k_in["head"])
+    _linear_check(ohead, nf, idx, n, m.logits.cpu().numpy(), m.k_in["head"], wc(-1, "head"))
     return nxt
 
 
@@ -243,15 +248,18 @@ def test_decode_step_store_mode_against_oracle(sf):
     m.close()
 
 
-def test_decode_step_cache_mode_against_oracle(sf):
+@pytest.mark.parametrize("deadline", [False, True])
+def test_decode_step_cache_mode_against_oracle(sf, deadline):
     """Weight refinements behind 25% LRU caches and K/V refinements behind a
     20% KV refinement cache per layer with a fetch budget, over three decode
     steps at positions T0, T0+1, T0+2: every op of every step, the attention
     refining only the union tokens cached when the step starts, and the cache
-    sets of one weight matrix per input and of each layer's KV cache."""
+    sets of one weight matrix per input and of each layer's KV cache.  With
+    the deadline reading the GEMVs refine only the selected columns cached
+    when the step starts (and never wait for a fetch)."""
     host = _host_model()
     budget = 12                                   # per KV head and step
-    m = _build(sf, host, weight_cache_pct=25, kv_cache_pct=20, kv_budget=budget)
+    m = _build(sf, host, weight_cache_pct=25, kv_cache_pct=20, kv_budget=budget, weight_deadline=deadline)
     olayers, ohead, ofinal, okv = _oracle_model(host)
     # oracle LRUs: q (attn_in), o, gate (mlp_in), down, head; the KV caches
     worcs = {slot: [ocache.LRUCache(K, od.count_half_up(Fraction(25, 100), K)) for _ in range(NL)]
@@ -272,11 +280,15 @@ def test_decode_step_cache_mode_against_oracle(sf):
                     if t <= T:
                         a[gh, t] = True
             avail.append(a)
+        wcached = None
+        if deadline:
+            wcached = {(l, slot): set(orcs[l].snapshot()) for slot, orcs in worcs.items() for l in range(NL)}
+            wcached[(-1, "head")] = set(horc.snapshot())
         m.x_in.copy_(torch.from_numpy(_embedding(7200 + step)))
         m.step(T)
         torch.cuda.synchronize()
         m.sync()
-        okv = _check_step(m, olayers, ohead, ofinal, okv, T, available=avail)
+        okv = _check_step(m, olayers, ohead, ofinal, okv, T, available=avail, wcached=wcached)
         for slot, orcs in worcs.items():
             for l in range(NL):
                 b = m.buf[slot]

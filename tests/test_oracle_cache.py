@@ -12,7 +12,7 @@ from collections import OrderedDict
 import numpy as np
 import pytest
 
-from oracle.cache import LRUCache
+from oracle.cache import LRUCache, effective_set
 
 
 class OrderedLRU:
@@ -127,3 +127,15 @@ def test_fetch_budget_by_hand():
     assert c.snapshot() == {1: 0, 4: 1, 7: 2}
     r = c.step([2, 3])                # no budget: C1-C5 (victims by (last use, unit): 1, then 4)
     assert r["inserted"] == [(2, 0), (3, 1)] and r["late"] == []
+
+
+def test_effective_set_of_the_deadline_reading():
+    """C8: the GEMV refines the selected units cached when the step starts;
+    the step itself then runs on the whole selection."""
+    c = LRUCache(20, 4)
+    c.step([1, 2, 3])
+    cached = c.snapshot()
+    assert effective_set([2, 3, 5, 9], cached) == [2, 3]
+    assert effective_set([], cached) == [] and effective_set([7], {}) == []
+    r = c.step([2, 3, 5, 9])
+    assert r["hits"] == [2, 3] and r["misses"] == [5, 9]
