@@ -535,6 +535,35 @@ sf_status sf_rope(float* x, int H, int d, int pos, double theta, uint16_t* y_bf1
 sf_status sf_silu_mul(const float* g, const float* u, int n, uint16_t* y, sf_stream_t stream);
 
 /*
+ * Producer + selection in one launch (one thread block of 1024 threads, batch
+ * 1): each writes the bf16 row y [K] that a GEMV reads, exactly as the
+ * stand-alone op does, then selects its top k channels and writes the
+ * prepared activations, exactly as sf_select_topk_act does (idx_out
+ * ascending, *n_out its length or -1 for a NaN/Inf row; act as there, or NULL
+ * to skip; k = 0 selects nothing, so act is then sf_act_prepare's form).
+ *   sf_norm_select     -- sf_add_rmsnorm of one row (x += delta first when
+ *                         delta is not NULL), y = bf16(RMSNorm(x) w);
+ *   sf_round_select    -- y = bf16(a), a fp32 [K];
+ *   sf_silu_mul_select -- y = bf16(silu(g) u), g, u fp32 [K].
+ * Constraints: K (H) a multiple of 256 up to 32768, 0 <= k <= K, act 16-byte
+ * aligned; idx_out has room for k entries.
+ */
+sf_status sf_norm_select(float* x, const float* delta, const float* w, int H, float eps, uint16_t* y, int k,
+                         int32_t* idx_out, int32_t* n_out, void* act, sf_stream_t stream);
+sf_status sf_round_select(const float* a, int K, uint16_t* y, int k, int32_t* idx_out, int32_t* n_out, void* act,
+                          sf_stream_t stream);
+sf_status sf_silu_mul_select(const float* g, const float* u, int K, uint16_t* y, int k, int32_t* idx_out,
+                             int32_t* n_out, void* act, sf_stream_t stream);
+
+/*
+ * sf_rope_qk -- sf_rope of the query heads q [Hq][d] (also written as bf16 to
+ *   q_bf16 [Hq][d] when it is not NULL) and of the key heads k [Hkv][d], in
+ *   one launch.  Same constraints as sf_rope (Hkv may be 0).
+ */
+sf_status sf_rope_qk(float* q, int Hq, float* k, int Hkv, int d, int pos, double theta, uint16_t* q_bf16,
+                     sf_stream_t stream);
+
+/*
  * sf_round_bf16 -- y[i] = bf16(x[i]) (to nearest, ties to even) for i < n:
  *   the attention's fp32 output as the bf16 input of the o projection.
  *   x fp32 [n], y bf16 [n].  Constraints: n >= 1.

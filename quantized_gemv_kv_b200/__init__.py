@@ -105,6 +105,10 @@ _SIGS = {
     "sf_rope": ([_p, _i, _i, _i, ctypes.c_double, _p, _p], _i),
     "sf_silu_mul": ([_p, _p, _i, _p, _p], _i),
     "sf_round_bf16": ([_p, _i, _p, _p], _i),
+    "sf_norm_select": ([_p, _p, _p, _i, ctypes.c_float, _p, _i, _p, _p, _p, _p], _i),
+    "sf_round_select": ([_p, _i, _p, _i, _p, _p, _p, _p], _i),
+    "sf_silu_mul_select": ([_p, _p, _i, _p, _i, _p, _p, _p, _p], _i),
+    "sf_rope_qk": ([_p, _i, _p, _i, _i, _i, ctypes.c_double, _p, _p], _i),
     "sf_kv_append": ([_p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p], _i),
     "sf_kv_append_cached": ([_p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _i, _p], _i),
 }
@@ -620,3 +624,38 @@ def kv_append_cached(src: torch.Tensor, res: torch.Tensor, scale: torch.Tensor, 
     Hkv, d = src.shape
     _check(_lib.sf_kv_append_cached(_ptr(src), Hkv, d, row_stride, t, b_r, b_f, _ptr(res), _ptr(scale), _ptr(zero),
                                     cache.handle, part, _stream(stream)))
+
+
+def norm_select(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor, k: int, idx: torch.Tensor, n: torch.Tensor,
+                act: torch.Tensor | None, eps: float = 1e-5, delta: torch.Tensor | None = None,
+                stream: torch.cuda.Stream | None = None) -> None:
+    """``sf_norm_select``: x += delta, y = bf16(RMSNorm(x) w), then the top-k
+    selection of y and its prepared activations, in one launch (batch 1)."""
+    _dev(x, "x")
+    _check(_lib.sf_norm_select(_ptr(x), _ptr(delta), _ptr(w), x.numel(), eps, _ptr(y), k, _ptr(idx), _ptr(n),
+                               _ptr(act), _stream(stream)))
+
+
+def round_select(a: torch.Tensor, y: torch.Tensor, k: int, idx: torch.Tensor, n: torch.Tensor,
+                 act: torch.Tensor | None, stream: torch.cuda.Stream | None = None) -> None:
+    """``sf_round_select``: y = bf16(a), then its top-k selection and prepared activations."""
+    _dev(a, "a")
+    _check(_lib.sf_round_select(_ptr(a), a.numel(), _ptr(y), k, _ptr(idx), _ptr(n), _ptr(act), _stream(stream)))
+
+
+def silu_mul_select(g: torch.Tensor, u: torch.Tensor, y: torch.Tensor, k: int, idx: torch.Tensor, n: torch.Tensor,
+                    act: torch.Tensor | None, stream: torch.cuda.Stream | None = None) -> None:
+    """``sf_silu_mul_select``: y = bf16(silu(g) u), then its top-k selection and prepared activations."""
+    _dev(g, "g")
+    if g.numel() != u.numel():
+        raise ValueError("g and u must have the same size")
+    _check(_lib.sf_silu_mul_select(_ptr(g), _ptr(u), g.numel(), _ptr(y), k, _ptr(idx), _ptr(n), _ptr(act),
+                                   _stream(stream)))
+
+
+def rope_qk(q: torch.Tensor, k: torch.Tensor, pos: int, theta: float = 500000.0, q_bf16: torch.Tensor | None = None,
+            stream: torch.cuda.Stream | None = None) -> None:
+    """``sf_rope_qk``: RoPE of q [Hq][d] (and its bf16 copy) and k [Hkv][d] in one launch."""
+    _dev(q, "q")
+    Hq, d = q.shape
+    _check(_lib.sf_rope_qk(_ptr(q), Hq, _ptr(k), k.shape[0], d, pos, theta, _ptr(q_bf16), _stream(stream)))

@@ -11,6 +11,7 @@
 // compaction writes the union in ascending order.
 #include "act.cuh"
 #include "block_scan.cuh"
+#include "select_row.cuh"
 #include "sf_internal.h"
 
 namespace {
@@ -218,112 +219,16 @@ __global__ void __launch_bounds__(kThreads)
 select_act_many_kernel(const __grid_constant__ SelManyArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
   const SelJobDev& J = a.job[blockIdx.x];
-  const int K = J.K, k = J.k, tid = threadIdx.x;
+  const int K = J.K, tid = threadIdx.x;
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [K]
   uint8_t* flags = smem + 2 * K;                     // [K]
-  __shared__ int hist1[256], hist2[128];
-  __shared__ int scan_scratch[33];
-  __shared__ int b1_sh, k1_sh, tau_sh, r_sh, bad;
-  __shared__ int eg[kActMaxGroups];
-  __shared__ float ginfo[2 * kActMaxGroups];
   {
     const uint4* src = reinterpret_cast<const uint4*>(J.x);
     uint4* dst = reinterpret_cast<uint4*>(xs);
     for (int i = tid; i < K / 8; i += kThreads) dst[i] = src[i];
   }
-  for (int j = tid; j < K; j += kThreads) flags[j] = 0;
-  for (int j = tid; j < 256; j += kThreads) hist1[j] = 0;
-  for (int j = tid; j < 128; j += kThreads) hist2[j] = 0;
-  if (tid == 0) bad = 0;
   __syncthreads();
-  for (int j = tid; j < K; j += kThreads) {
-    const uint32_t v = xs[j];
-    if ((v & 0x7F80u) == 0x7F80u) bad = 1;
-    atomicAdd(&hist1[(v & 0x7FFFu) >> 7], 1);
-  }
-  __syncthreads();
-  const int warp = tid >> 5, lane = tid & 31;
-  if (warp == 0) {
-    int above = 0, b1 = -1, k1 = 0;
-    for (int base = 255; base >= 0 && b1 < 0; base -= 32) {
-      const int c = hist1[base - lane];
-      int incl = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const unsigned m = __ballot_sync(0xffffffffu, k > 0 && above + incl >= k && above + incl - c < k);
-      if (m) {
-        const int src = __ffs(m) - 1;
-        b1 = base - src;
-        k1 = k - (above + __shfl_sync(0xffffffffu, incl - c, src));
-      }
-      above += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) { b1_sh = b1; k1_sh = k1; }
-  }
-  __syncthreads();
-  const int b1 = b1_sh;
-  if (b1 >= 0)
-    for (int j = tid; j < K; j += kThreads) {
-      const uint32_t v = xs[j] & 0x7FFFu;
-      if (static_cast<int>(v >> 7) == b1) atomicAdd(&hist2[v & 0x7Fu], 1);
-    }
-  __syncthreads();
-  if (warp == 0) {
-    const int kk = k1_sh;
-    int above = 0, tau = -1, r = 0;
-    if (b1 >= 0) {
-      for (int base = 127; base >= 0 && tau < 0; base -= 32) {
-        const int c = hist2[base - lane];
-        int incl = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        const unsigned m = __ballot_sync(0xffffffffu, above + incl >= kk && above + incl - c < kk);
-        if (m) {
-          const int src = __ffs(m) - 1;
-          tau = (b1 << 7) | (base - src);
-          r = kk - (above + __shfl_sync(0xffffffffu, incl - c, src));
-        }
-        above += __shfl_sync(0xffffffffu, incl, 31);
-      }
-    }
-    if (lane == 0) { tau_sh = tau; r_sh = r; }
-  }
-  __syncthreads();
-  const int tau = tau_sh;
-  // ordered tie pass over contiguous chunks, then the compaction
-  const int chunk = (K + kThreads - 1) / kThreads;
-  const int j0 = min(K, tid * chunk), j1 = min(K, j0 + chunk);
-  {
-    int eq = 0;
-    if (tau >= 0)
-      for (int j = j0; j < j1; ++j) eq += ((xs[j] & 0x7FFF) == tau);
-    int total;
-    int rank = sfd::block_exclusive_scan(eq, scan_scratch, &total);
-    if (tau >= 0)
-      for (int j = j0; j < j1; ++j) {
-        const int key = xs[j] & 0x7FFF;
-        if (key > tau) flags[j] = 1;
-        else if (key == tau) { if (rank < r_sh) flags[j] = 1; ++rank; }
-      }
-  }
-  __syncthreads();
-  {
-    int c = 0;
-    for (int j = j0; j < j1; ++j) c += flags[j];
-    int total;
-    int pos = sfd::block_exclusive_scan(c, scan_scratch, &total);
-    for (int j = j0; j < j1; ++j)
-      if (flags[j]) J.idx[pos++] = j;
-    if (tid == 0) *J.n = bad ? -1 : total;
-  }
-  __syncthreads();
-  if (J.act != nullptr) sfd::act2_write_block(xs, flags, K, eg, ginfo, scan_scratch, J.act);
+  sfd::select_row_block(xs, flags, K, J.k, J.idx, J.n, J.act);
 }
 }  // namespace
 

@@ -6,17 +6,18 @@ The pages measure StrataFlux end to end on a decode step of a Llama-3.1-8B
 sized model at 128K context (arXiv 2611.08363 abstract: tokens/s and GPU
 memory with 3-bit weights and 2-bit KV).  Per layer, batch 1:
 
-  n1 = RMSNorm(x)                         sf_add_rmsnorm (adds the previous
-                                          layer's MLP output to x first)
-  q, k, v = refined GEMVs of n1           sf_select_topk_act, the weight
-                                          caches' prefetch, sf_gemv_refine_batch1
-  q, k rotated to position T              sf_rope (q also as bf16)
+  n1 = RMSNorm(x)                         sf_norm_select (adds the previous
+                                          layer's MLP output to x first, and
+                                          selects n1's top channels)
+  q, k, v = refined GEMVs of n1           the weight caches' prefetch,
+                                          sf_gemv_refine_batch1
+  q, k rotated to position T              sf_rope_qk (q also as bf16)
   k, v quantized, appended as token T     sf_kv_append
   a = refined attention over T + 1        sf_attn_decode_refine (+ the KV
                                           refinement cache's prefetch)
-  h = x + o(bf16(a))                      sf_round_bf16, GEMV, sf_add_rmsnorm
+  h = x + o(bf16(a))                      sf_round_select, GEMV, sf_norm_select
   n2 = RMSNorm(h)
-  x' = h + down(bf16(silu(gate(n2)) up(n2)))   sf_silu_mul, GEMVs
+  x' = h + down(bf16(silu(gate(n2)) up(n2)))   sf_silu_mul_select, GEMVs
 
 then RMSNorm and the refined LM head give the logits.  Each GEMV refines the
 top round_half_up(p K) channels of its own input (the explainer's 解説:
@@ -48,9 +49,9 @@ from fractions import Fraction
 
 import torch
 
-from . import (QKV, Batch1Jobs, RefineCache, RefineGroup, SelectJobs, act_bytes, act_prepare, add_rmsnorm,
-               attn_decode_refine, attn_union_units, attn_workspace_size, kv_append, kv_append_cached, pack_batch1,
-               quantize_nested, rope, round_bf16, silu_mul)
+from . import (QKV, Batch1Jobs, RefineCache, RefineGroup, act_bytes, attn_decode_refine, attn_union_units,
+               attn_workspace_size, kv_append, kv_append_cached, norm_select, pack_batch1, quantize_nested, rope_qk,
+               round_select, silu_mul_select)
 
 MATS = ("q", "k", "v", "o", "gate", "up", "down")
 
@@ -242,23 +243,24 @@ class DecodeModel:
         self.head_job = Batch1Jobs([(self.head.qw, self.head.cache, not cached, self.logits)])
         self.head_job0 = Batch1Jobs([(self.head.qw, None, False, self.logits)])
         self.head_group = RefineGroup([(self.head.cache, hb["idx"][0], hb["n"][0])]) if cached else None
-        self.sel_jobs = {}
-        for slot in ("attn_in", "attn_out", "mlp_in", "mlp_mid"):
-            b = self.buf[slot]
-            self.sel_jobs[slot] = [SelectJobs([(b["x"][l:l + 1], self.k_in[slot], b["idx"][l], b["n"][l],
-                                                b["act"][l])]) for l in range(self.s.layers)]
-        self.sel_head = SelectJobs([(hb["x"], self.k_in["head"], hb["idx"][0], hb["n"][0], hb["act"][0])])
 
     # ---- the step -----------------------------------------------------------------------
 
+    def _sel(self, l, slot, refine):
+        """The (idx, n, act, k) arguments of the fused producer + selection
+        that makes the input row of `slot` (k = 0: nothing selected)."""
+        b = self.buf[slot]
+        li = max(l, 0)
+        return dict(k=self.k_in[slot] if refine else 0, idx=b["idx"][li], n=b["n"][li], act=b["act"][li])
+
     def _linear(self, l, slot, refine, main):
-        """Selection (or plain preparation), the caches' step on the side
-        stream, and the batch-1 GEMV launch of the matrices reading `slot`."""
+        """The caches' step on the side stream and the batch-1 GEMV launch of
+        the matrices reading `slot` (its row, selection and prepared
+        activations made by the producer just before)."""
         b = self.buf[slot]
         x = b["x"][l:l + 1] if l >= 0 else b["x"]
         li = max(l, 0)
         if refine:
-            (self.sel_jobs[slot][l] if l >= 0 else self.sel_head).run()
             grp = self.wgroups[l].get(slot) if l >= 0 else self.head_group
             if grp is not None and not self.deadline:
                 grp.prefetch(main, self.side)   # the GEMV waits for these fetches
@@ -266,7 +268,6 @@ class DecodeModel:
             if grp is not None and self.deadline:
                 grp.prefetch(main, self.side)   # for later steps; nothing waits within this one
         else:
-            act_prepare(x, b["act"][li])
             (self.jobs0[l][slot] if l >= 0 else self.head_job0).run(x, b["act"][li])
 
     def step(self, T: int, refine: bool = True) -> None:
@@ -286,8 +287,8 @@ class DecodeModel:
         self.x.copy_(self.x_in)
         prev = None
         for l, L in enumerate(self.layers):
-            bi = self.buf["attn_in"]["x"][l]
-            add_rmsnorm(self.x, L["norm1"], s.eps, delta=prev, y=bi.view(1, H))
+            norm_select(self.x, L["norm1"], self.buf["attn_in"]["x"][l], eps=s.eps, delta=prev,
+                        **self._sel(l, "attn_in", refine))
             if self.record:
                 self.x_hist[l].copy_(self.x)
             self._linear(l, "attn_in", refine, main)
@@ -296,8 +297,7 @@ class DecodeModel:
                 self.qkv_raw[l, :Hq * d].copy_(L["q"].y)
                 self.qkv_raw[l, Hq * d:(Hq + Hkv) * d].copy_(L["k"].y)
                 self.qkv_raw[l, (Hq + Hkv) * d:].copy_(L["v"].y)
-            rope(q, T, s.theta, y=self.q_bf[l])
-            rope(k, T, s.theta)
+            rope_qk(q, k, T, s.theta, q_bf16=self.q_bf[l])
             if self.record:
                 self.k_rot[l].copy_(k)
             kq, vq = L["kv"].k, L["kv"].v
@@ -314,16 +314,18 @@ class DecodeModel:
                                  self.n_units[l])
                 L["kv_cache"].prefetch(self.units[l], self.n_units[l], main, self.side)
                 side_used = True
-            round_bf16(self.att[l].view(-1), y=self.buf["attn_out"]["x"][l])
+            round_select(self.att[l].view(-1), self.buf["attn_out"]["x"][l], **self._sel(l, "attn_out", refine))
             self._linear(l, "attn_out", refine, main)
-            add_rmsnorm(self.x, L["norm2"], s.eps, delta=L["o"].y, y=self.buf["mlp_in"]["x"][l].view(1, H))
+            norm_select(self.x, L["norm2"], self.buf["mlp_in"]["x"][l], eps=s.eps, delta=L["o"].y,
+                        **self._sel(l, "mlp_in", refine))
             if self.record:
                 self.h_hist[l].copy_(self.x)
             self._linear(l, "mlp_in", refine, main)
-            silu_mul(L["gate"].y, L["up"].y, y=self.buf["mlp_mid"]["x"][l])
+            silu_mul_select(L["gate"].y, L["up"].y, self.buf["mlp_mid"]["x"][l], **self._sel(l, "mlp_mid", refine))
             self._linear(l, "mlp_mid", refine, main)
             prev = L["down"].y
-        add_rmsnorm(self.x, self.final_norm, s.eps, delta=prev, y=self.buf["head"]["x"])
+        norm_select(self.x, self.final_norm, self.buf["head"]["x"][0], eps=s.eps, delta=prev,
+                    **self._sel(-1, "head", refine))
         if self.record:
             self.x_hist[s.layers].copy_(self.x)
         self._linear(-1, "head", refine, main)

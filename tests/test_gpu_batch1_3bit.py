@@ -63,7 +63,7 @@ def _expected_pack3(codes):
 
 
 def test_pack_batch1_layout(sf):
-    N, K = 48, 1024
+    N, K = 96, 1024
     W = gen_weight(77, N, K)
     qw = sf.quantize_nested(dev(W), 128, 3, 1)
     sf.pack_batch1(qw)

@@ -122,3 +122,94 @@ def test_decode_ops_reject_bad_sizes(sf):
         sf.rope(x, 0)                   # odd head dim
     with pytest.raises(sf.SfError):
         sf.rope(torch.zeros((2, 8), dtype=torch.float32, device="cuda"), -1)
+
+
+# ---- producer + selection in one launch ---------------------------------------
+
+def _selection_and_act(sf, y_bits_dev, K, k):
+    """The stand-alone selection of a bf16 row (sf_select_topk_act)."""
+    idx = torch.zeros(max(k, 1), dtype=torch.int32, device="cuda")
+    n = torch.zeros(1, dtype=torch.int32, device="cuda")
+    act = torch.zeros(sf.act_bytes(K) // 4, dtype=torch.int32, device="cuda")
+    if k > 0:
+        sf.select_topk_act(y_bits_dev.view(1, K), k, idx, n, act)
+    else:
+        sf.act_prepare(y_bits_dev.view(1, K), act)
+    return idx, n, act
+
+
+def _fused_buffers(sf, K, k):
+    return (torch.zeros(K, dtype=torch.bfloat16, device="cuda"), torch.full((max(k, 1),), -1, dtype=torch.int32,
+            device="cuda"), torch.full((1,), -7, dtype=torch.int32, device="cuda"),
+            torch.zeros(sf.act_bytes(K) // 4, dtype=torch.int32, device="cuda"))
+
+
+@pytest.mark.parametrize("H,k,with_delta", [(4096, 123, True), (14336, 430, False), (4096, 0, True)])
+def test_norm_select_equals_norm_then_select(sf, H, k, with_delta):
+    from oracle import select as oselect
+    rng = np.random.default_rng(300 + H + k)
+    x = (rng.standard_normal(H) * 3).astype(np.float32)
+    x[rng.choice(H, 20, replace=False)] *= 30
+    d = (rng.standard_normal(H)).astype(np.float32) if with_delta else None
+    w = (1 + 0.1 * rng.standard_normal(H)).astype(np.float32)
+    x1, x2 = torch.from_numpy(x).cuda(), torch.from_numpy(x).cuda()
+    dd = torch.from_numpy(d).cuda() if with_delta else None
+    wd = torch.from_numpy(w).cuda()
+    y_ref = sf.add_rmsnorm(x1.view(1, H), wd, 1e-5, delta=dd.view(1, H) if with_delta else None)
+    y, idx, n, act = _fused_buffers(sf, H, k)
+    sf.norm_select(x2, wd, y, k, idx, n, act, eps=1e-5, delta=dd)
+    torch.cuda.synchronize()
+    assert torch.equal(x1, x2)                       # the residual update is the same fp32 addition
+    _close_bf16(_bits(y), _bits(y_ref.view(-1)))
+    yb = _bits(y)
+    S = oselect.select_topk(yb[None, :], k)
+    assert int(n.item()) == len(S)
+    np.testing.assert_array_equal(idx.cpu().numpy()[: len(S)], S)
+    i2, n2, act2 = _selection_and_act(sf, y, H, k)   # same row, same prepared bytes
+    torch.cuda.synchronize()
+    assert torch.equal(act, act2)
+
+
+@pytest.mark.parametrize("K,k", [(4096, 123), (4096, 0)])
+def test_round_select_equals_round_then_select(sf, K, k):
+    rng = np.random.default_rng(400 + K + k)
+    a = torch.from_numpy((rng.standard_normal(K) * 2).astype(np.float32)).cuda()
+    y_ref = sf.round_bf16(a)
+    y, idx, n, act = _fused_buffers(sf, K, k)
+    sf.round_select(a, y, k, idx, n, act)
+    i2, n2, act2 = _selection_and_act(sf, y_ref, K, k)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
+    if k:
+        assert int(n.item()) == int(n2.item()) == k
+        assert torch.equal(idx[:k], i2[:k])
+    assert torch.equal(act, act2)
+
+
+def test_silu_mul_select_equals_silu_mul_then_select(sf):
+    K, k = 14336, 430
+    rng = np.random.default_rng(500)
+    g = torch.from_numpy((rng.standard_normal(K) * 2).astype(np.float32)).cuda()
+    u = torch.from_numpy((rng.standard_normal(K) * 2).astype(np.float32)).cuda()
+    y_ref = sf.silu_mul(g, u)
+    y, idx, n, act = _fused_buffers(sf, K, k)
+    sf.silu_mul_select(g, u, y, k, idx, n, act)
+    i2, n2, act2 = _selection_and_act(sf, y_ref, K, k)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
+    assert torch.equal(idx[:k], i2[:k]) and int(n.item()) == k
+    assert torch.equal(act, act2)
+
+
+def test_rope_qk_equals_two_ropes(sf):
+    rng = np.random.default_rng(600)
+    q = torch.from_numpy(rng.standard_normal((32, 128)).astype(np.float32)).cuda()
+    k = torch.from_numpy(rng.standard_normal((8, 128)).astype(np.float32)).cuda()
+    q2, k2 = q.clone(), k.clone()
+    qb = torch.zeros((32, 128), dtype=torch.bfloat16, device="cuda")
+    qb2 = torch.zeros_like(qb)
+    sf.rope(q, 131071, y=qb)
+    sf.rope(k, 131071)
+    sf.rope_qk(q2, k2, 131071, q_bf16=qb2)
+    torch.cuda.synchronize()
+    assert torch.equal(q, q2) and torch.equal(k, k2) and torch.equal(qb.view(torch.int16), qb2.view(torch.int16))
