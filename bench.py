@@ -204,10 +204,6 @@ class Model:
         self.qin = torch.empty((layers, HQ, D), dtype=torch.bfloat16, device=device)
         self.idx = {s: torch.zeros((layers, self.ksel[s]), dtype=torch.int32, device=device) for s, _ in SLOTS}
         self.nsel = {s: torch.zeros((layers, 1), dtype=torch.int32, device=device) for s, _ in SLOTS}
-        # prepared activations: with the selection (refined step) and without (resident-only step)
-        self.act = {s: torch.zeros((layers, sf.act_bytes(K) // 4), dtype=torch.int32, device=device) for s, K in SLOTS}
-        self.act0 = {s: torch.zeros((layers, sf.act_bytes(K) // 4), dtype=torch.int32, device=device)
-                     for s, K in SLOTS}
         self.ws = torch.empty(sf.attn_workspace_size(HQ, HKV, D, T, self.k_tok), dtype=torch.uint8, device=device)
         self.xoff = {}
         off = 0
@@ -233,8 +229,8 @@ class Model:
                               for slot, names in GEMV_LAUNCHES})
             self.jobs0.append({slot: sf.Batch1Jobs([(row[n][0], None, False, row[n][2].view(-1)) for n in names])
                                for slot, names in GEMV_LAUNCHES})
-            self.selects.append(sf.SelectJobs([(self.x(l, s), self.ksel[s], self.idx[s][l], self.nsel[s][l],
-                                                self.act[s][l]) for s, _ in SLOTS]))
+            self.selects.append(sf.SelectJobs([(self.x(l, s), self.ksel[s], self.idx[s][l], self.nsel[s][l], None)
+                                               for s, _ in SLOTS]))
             Kf, Vf = ds.kv(3000 + l, HKV, T, D, device=device)
             self.kv.append(sf.QKV(sf.quantize_nested(Kf, D, B_R, B_F, "by_row"),
                                   sf.quantize_nested(Vf, D, B_R, B_F, "by_row")))
@@ -285,37 +281,18 @@ class Model:
                 self.selects[l].run()
             self.groups[l].prefetch(self.sel_stream, self.side)
 
-        def prepare_only(l):
-            # the resident-only step prepares its activations the same way,
-            # one layer ahead on the selection stream; main waits for them
-            ev = torch.cuda.Event()
-            ev.record(main)
-            self.sel_stream.wait_event(ev)
-            with torch.cuda.stream(self.sel_stream):
-                for s, _ in SLOTS:
-                    sf.act_prepare(self.x(l, s), self.act0[s][l])
-                done = torch.cuda.Event()
-                done.record(self.sel_stream)
-            return done
 
         def gemv(l, slot):
             if refine:
-                self.jobs[l][slot].run(self.x(l, slot), self.act[slot][l])
+                self.jobs[l][slot].run(self.x(l, slot), self.idx[slot][l], self.nsel[slot][l])
             else:
-                self.jobs0[l][slot].run(self.x(l, slot), self.act0[slot][l])
+                self.jobs0[l][slot].run(self.x(l, slot))
 
-        ready = {}
         if refine:
             select_and_prefetch(0)
-        else:
-            ready[0] = prepare_only(0)
         for l in range(self.L):
             if refine and l + 1 < self.L:
                 select_and_prefetch(l + 1)
-            if not refine:
-                if l + 1 < self.L:
-                    ready[l + 1] = prepare_only(l + 1)
-                main.wait_event(ready.pop(l))
             gemv(l, "attn_in")
             sf.attn_decode_refine(self.qin[l], self.kv[l], HKV, self.T, self.k_tok if refine else 0,
                                   workspace=self.ws, out=self.attn_out[l], sel_out=self.sel_out[l],
@@ -326,7 +303,7 @@ class Model:
     def gemvs_only(self):
         for l in range(self.L):
             for slot, _ in GEMV_LAUNCHES:
-                self.jobs[l][slot].run(self.x(l, slot), self.act[slot][l])
+                self.jobs[l][slot].run(self.x(l, slot), self.idx[slot][l], self.nsel[slot][l])
 
     def attn_only(self):
         for l in range(self.L):
@@ -906,8 +883,8 @@ def run_sf(args, rank, world, local_rank, dist):
             for l in range(L):
                 for slot in ("attn_in", "attn_out", "mlp_in", "mlp_mid"):
                     b = model.buf[slot]
-                    model.jobs0[l][slot].run(b["x"][l:l + 1], b["act"][l])
-            model.head_job0.run(model.buf["head"]["x"], model.buf["head"]["act"][0])
+                    model.jobs0[l][slot].run(b["x"][l:l + 1])
+            model.head_job0.run(model.buf["head"]["x"])
         gg = capture(torch, gemvs_only, cap_stream)
         for _ in range(2):
             with torch.cuda.stream(cap_stream):

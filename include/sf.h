@@ -357,12 +357,16 @@ typedef struct sf_gemv_job {
  * sf_gemv_refine_batch1 -- refined GEMV at batch 1 for up to 4 matrices that
  * read the same activation row (q/k/v, gate/up): y_i = W_i,res x + sum over
  * the selected channels of x_j s (q_f - m_f), as sf_gemv_refine, in one
- * launch.  act comes from sf_select_topk_act (refined) or sf_act_prepare
- * (resident only) for this x; x is the bf16 row itself (device).
- * Computed on the integer tensor cores (mma.m16n8k32, 2- or 3-bit codes x
- * 8-bit activation digits) in tiles of 16 output rows; the refinement
- * correction on the f16 tensor cores (fp32 for a slice whose selected |x|
- * reaches 2^15).
+ * launch.  x: the bf16 row (device, 16-byte aligned); (idx, n): its selection
+ * as sf_select_topk writes it (device; both NULL: nothing selected, the
+ * resident-only GEMV).  Each warp turns its slice of x into the fixed-point
+ * operand fragments itself (per 128-channel group X = rint(x 2^(22-e)), e the
+ * exponent of the group's largest |x|, in signed 8-bit digits: the layout
+ * sf_select_topk_act documents) and finds the slice's selected channels in
+ * idx.  Computed on the integer tensor cores (mma.m16n8k32, 2- or 3-bit
+ * codes x 8-bit activation digits) in tiles of 16 output rows; the
+ * refinement correction on the f16 tensor cores (fp32 for a slice whose
+ * selected |x| reaches 2^15).
  * Constraints: b_r in {2, 3}, b_f in {1, 2}, b_r + b_f <= 4, G == 128, all
  * jobs share K, G and bit widths; N % 16 == 0; K a multiple of 256 whose
  * K/256 slices split into at most 16 warps of one or two slices, in one or
@@ -375,8 +379,8 @@ typedef struct sf_gemv_job {
  * at most 2^(e-23) per channel (e its binary exponent), so channels far
  * below it keep few bits.
  */
-sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, const uint16_t* x, const void* act,
-                                sf_stream_t stream);
+sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, const uint16_t* x, const int32_t* idx,
+                                const int32_t* n, sf_stream_t stream);
 
 /* ---- refined decode attention ----------------------------------------- */
 

@@ -94,7 +94,7 @@ _SIGS = {
     "sf_select_topk_act": ([_p, _i, _i, _p, _p, _p, _p], _i),
     "sf_act_prepare": ([_p, _i, _p, _p], _i),
     "sf_select_topk_act_many": ([_p, _i, _p], _i),
-    "sf_gemv_refine_batch1": ([_p, _i, _p, _p, _p], _i),
+    "sf_gemv_refine_batch1": ([_p, _i, _p, _p, _p, _p], _i),
     "sf_gemv_pack_batch1": ([_p, _i, _i, _i, _p, _p], _i),
     "sf_attn_workspace_size": ([_i, _i, _i, _i, _i, ctypes.POINTER(_sz)], _i),
     "sf_attn_decode_refine": ([_p, _i, _i, _i, _i, ctypes.POINTER(_QKV), _i, _p, _p, _p, _p, _sz, _p], _i),
@@ -512,14 +512,17 @@ class Batch1Jobs:
         self._arr = arr
         self.count = len(jobs)
 
-    def run(self, x: torch.Tensor, act: torch.Tensor, stream: torch.cuda.Stream | None = None) -> None:
-        _check(_lib.sf_gemv_refine_batch1(ctypes.cast(self._arr, _p), self.count, _ptr(x), _ptr(act),
+    def run(self, x: torch.Tensor, idx: torch.Tensor | None = None, n: torch.Tensor | None = None,
+            stream: torch.cuda.Stream | None = None) -> None:
+        """x: the bf16 row; (idx, n): its selection (None: nothing selected)."""
+        _check(_lib.sf_gemv_refine_batch1(ctypes.cast(self._arr, _p), self.count, _ptr(x), _ptr(idx), _ptr(n),
                                           _stream(stream)))
 
 
-def gemv_refine_batch1(jobs, x: torch.Tensor, act: torch.Tensor, stream: torch.cuda.Stream | None = None) -> None:
+def gemv_refine_batch1(jobs, x: torch.Tensor, idx: torch.Tensor | None = None, n: torch.Tensor | None = None,
+                       stream: torch.cuda.Stream | None = None) -> None:
     """Refined GEMVs at batch 1 of up to 4 matrices that read the same x."""
-    Batch1Jobs(jobs).run(x, act, stream)
+    Batch1Jobs(jobs).run(x, idx, n, stream)
 
 
 class SelectJobs:

@@ -47,7 +47,7 @@
 
 #include <algorithm>
 
-#include "act.cuh"
+#include "act.cuh"  // bf16_exponent, bf16_fixed
 #include "sf_internal.h"
 
 namespace {
@@ -74,7 +74,8 @@ struct MJob {
 struct MArgs {
   MJob job[kMaxJobs];
   const uint16_t* x;
-  const uint32_t* act;
+  const int32_t* idx;    // the selection: ascending channels (nullptr: none)
+  const int32_t* n_sel;  // its length (negative counts as 0)
   int njobs, K, ksplit;
 };
 
@@ -295,39 +296,89 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
     if (i < my_tiles) issue_codes(i);
     cp_async_commit();
   }
-  // ---- per-warp setup: B fragments, group scalars, selection lists, the
-  // correction MMA's B fragments (x of the listed channels, high and low)
+  // ---- per-warp setup, from x and the selection list: the B fragments of
+  // the slice's fixed-point activations, the group scalars, the slice's
+  // selected channels, the correction MMA's B fragments (x of the listed
+  // channels, high and low)
+  int n_all = a.idx != nullptr ? *a.n_sel : 0;
+  n_all = n_all < 0 ? 0 : n_all;
 #pragma unroll
   for (int sp = 0; sp < SPW; ++sp) {
     const int slice = slice0 + sp;
-    const uint32_t* A = a.act + static_cast<size_t>(slice) * sfd::kAct2Words;
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      const uint2 v = reinterpret_cast<const uint2*>(A)[m * 32 + lane];
-      bf[sp][m][0] = v.x;
-      bf[sp][m][1] = v.y;
-    }
-    fsc[sp] = __uint_as_float(A[sfd::kAct2Info + 2 * myslot]);
-    gsm[sp] = __uint_as_float(A[sfd::kAct2Info + 2 * myslot + 1]);
-    psl[sp] = static_cast<int>(A[sfd::kAct2Info + 4]);
-    nsl[sp] = static_cast<int>(A[sfd::kAct2Info + 5]);
     {
-      const uint32_t mw = lane < 8 ? A[sfd::kAct2Mask + lane] : 0u;
-      const int c = __popc(mw);
-      int incl = c;
+      // lane (col n, t): group slot_b = n / 4, digit plane n % 4 (3: zero),
+      // channels 128 slot_b + 32 t + [0, 32) of the slice
+      const int bn = lane >> 2, slot_b = bn >> 2, plane = bn & 3;
+      const uint4* xp = reinterpret_cast<const uint4*>(a.x + 256 * static_cast<size_t>(slice) + 128 * slot_b +
+                                                       32 * tig);
+      uint32_t xw[16];
 #pragma unroll
-      for (int o = 1; o < 8; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+      for (int q = 0; q < 4; ++q) {
+        const uint4 v = xp[q];
+        xw[4 * q] = v.x; xw[4 * q + 1] = v.y; xw[4 * q + 2] = v.z; xw[4 * q + 3] = v.w;
       }
-      int r = incl - c;
-      uint32_t mm = mw;
-      while (mm) {
-        const int bit = __ffs(mm) - 1;
-        mm &= mm - 1u;
-        if (r < kCorrList) mylist[sp * kCorrList + r] = static_cast<uint16_t>(32 * lane + bit);
-        ++r;
+      // the group's largest |x| (15-bit magnitude keys order as |x| does)
+      uint32_t kmax = 0u;
+#pragma unroll
+      for (int w = 0; w < 16; ++w) kmax = max(kmax, max(xw[w] & 0x7FFFu, (xw[w] >> 16) & 0x7FFFu));
+      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, 1));
+      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, 2));  // lanes t = 0..3 hold the 128 channels
+      int e = sfd::bf16_exponent(kmax);
+      if (e == -1000) e = 0;
+      // X = rint(x 2^(22 - e)): the scaling is exact (|x| < 2^e, the result
+      // below 2^22 in magnitude), the conversion rounds to nearest even
+      // (two exact power-of-two factors, so a group of bf16 subnormals with
+      // 22 - e above 127 does not overflow the factor)
+      const int s1 = min(22 - e, 126);
+      const float sc1 = ldexpf(1.0f, s1), sc2 = ldexpf(1.0f, 22 - e - s1);
+      int gs = 0;
+      uint32_t dg[8][2];
+#pragma unroll
+      for (int mm = 0; mm < 4; ++mm)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) dg[mm][r] = 0u;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const int X = __float2int_rn(__uint_as_float(((xw[c >> 1] >> (16 * (c & 1))) & 0xFFFFu) << 16) * sc1 * sc2);
+        gs += X;
+        const int d0 = ((X + 128) & 255) - 128;
+        const int X1 = (X - d0) >> 8;
+        const int d1 = ((X1 + 128) & 255) - 128;
+        const int d2 = (X1 - d1) >> 8;
+        const int dv = plane == 0 ? d0 : (plane == 1 ? d1 : (plane == 2 ? d2 : 0));
+        // channel c = 16 (mm / 2) + 4 b + 2 (mm % 2) + r of k-step 4 slot_b + mm
+        const int mm = 2 * (c >> 4) + ((c >> 1) & 1), b = (c >> 2) & 3, r = c & 1;
+        dg[mm][r] |= (static_cast<uint32_t>(dv) & 0xFFu) << (8 * b);
       }
+      gs += __shfl_xor_sync(0xffffffffu, gs, 1);
+      gs += __shfl_xor_sync(0xffffffffu, gs, 2);
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) bf[sp][m][r] = (m >> 2) == slot_b ? dg[m & 3][r] : 0u;
+      // the epilogue's lane (row, group myslot) takes its group's scalars
+      const float fs = ldexpf(1.0f, e - 22);
+      const float gsum = static_cast<float>(gs) * fs;
+      fsc[sp] = __shfl_sync(0xffffffffu, fs, 16 * myslot);
+      gsm[sp] = __shfl_sync(0xffffffffu, gsum, 16 * myslot);
+    }
+    {
+      // the slice's run of the ascending selection
+      const int lo = 256 * slice, hi = lo + 256;
+      int c_lo = 0, c_hi = 0;
+      for (int i = lane; i < n_all; i += 32) {
+        const int v = a.idx[i];
+        c_lo += v < lo;
+        c_hi += v < hi;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        c_lo += __shfl_xor_sync(0xffffffffu, c_lo, o);
+        c_hi += __shfl_xor_sync(0xffffffffu, c_hi, o);
+      }
+      psl[sp] = c_lo;
+      nsl[sp] = c_hi - c_lo;
+      if (lane < min(nsl[sp], kCorrList)) mylist[sp * kCorrList + lane] = static_cast<uint16_t>(a.idx[c_lo + lane] - lo);
     }
     __syncwarp();
     int nl = min(nsl[sp], kCorrList);
@@ -495,17 +546,7 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
         // channels beyond the tensor-core list (more than kCorrList selected in
         // the slice, or every selected channel of a slice with a huge |x|)
         for (int k = nl; k < nsl[sp]; ++k) {
-          const uint32_t* A = a.act + static_cast<size_t>(slice0 + sp) * sfd::kAct2Words;
-          int kk = k, ch = -1;
-          for (int wdx = 0; wdx < 8 && ch < 0; ++wdx) {
-            uint32_t mm = A[sfd::kAct2Mask + wdx];
-            const int c = __popc(mm);
-            if (kk < c) {
-              for (int q = 0; q < kk; ++q) mm &= mm - 1u;
-              ch = 256 * (slice0 + sp) + 32 * wdx + __ffs(mm) - 1;
-            }
-            kk -= c;
-          }
+          const int ch = a.idx[psl[sp] + k];  // the slice's k-th selected channel (global)
           if (((ch >> 7) & 1) != myslot) continue;
           const int rr = J.unit_slot ? J.unit_slot[ch] : (J.row_of ? J.row_of[psl[sp] + k] : ch);
           if (rr < 0) continue;  // not cached at the step's start (deadline reading): resident precision
@@ -605,11 +646,12 @@ extern "C" sf_status sf_gemv_pack_batch1(const uint32_t* res, int N, int K, int 
   return sf::check_launch("pack_res3_kernel");
 }
 
-extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, const uint16_t* x, const void* act,
-                                           sf_stream_t stream) {
-  SF_REQUIRE(jobs && x && act, "sf_gemv_refine_batch1: null pointer");
+extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, const uint16_t* x, const int32_t* idx,
+                                           const int32_t* n, sf_stream_t stream) {
+  SF_REQUIRE(jobs && x, "sf_gemv_refine_batch1: null pointer");
+  SF_REQUIRE((idx == nullptr) == (n == nullptr), "sf_gemv_refine_batch1: idx and n go together");
   SF_REQUIRE(count >= 1 && count <= kMaxJobs, "sf_gemv_refine_batch1: count must be in [1, %d]", kMaxJobs);
-  SF_REQUIRE(sf::aligned(act, 16) && sf::aligned(x, 4), "sf_gemv_refine_batch1: act must be 16-byte aligned");
+  SF_REQUIRE(sf::aligned(x, 16), "sf_gemv_refine_batch1: x must be 16-byte aligned");
   const sf_qweight* W0 = jobs[0].W;
   SF_REQUIRE(W0, "sf_gemv_refine_batch1: null weight");
   const int K = W0->K, G = W0->G, b_f = W0->b_f, b_r = W0->b_r;
@@ -627,7 +669,8 @@ extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, c
   a.K = K;
   a.ksplit = ksplit;
   a.x = x;
-  a.act = static_cast<const uint32_t*>(act);
+  a.idx = idx;
+  a.n_sel = n;
   int row_tiles = 0;
   for (int i = 0; i < count; ++i) {
     const sf_qweight* W = jobs[i].W;

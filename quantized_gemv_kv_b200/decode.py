@@ -251,7 +251,7 @@ class DecodeModel:
         that makes the input row of `slot` (k = 0: nothing selected)."""
         b = self.buf[slot]
         li = max(l, 0)
-        return dict(k=self.k_in[slot] if refine else 0, idx=b["idx"][li], n=b["n"][li], act=b["act"][li])
+        return dict(k=self.k_in[slot] if refine else 0, idx=b["idx"][li], n=b["n"][li], act=None)
 
     def _linear(self, l, slot, refine, main):
         """The caches' step on the side stream and the batch-1 GEMV launch of
@@ -264,11 +264,11 @@ class DecodeModel:
             grp = self.wgroups[l].get(slot) if l >= 0 else self.head_group
             if grp is not None and not self.deadline:
                 grp.prefetch(main, self.side)   # the GEMV waits for these fetches
-            (self.jobs[l][slot] if l >= 0 else self.head_job).run(x, b["act"][li])
+            (self.jobs[l][slot] if l >= 0 else self.head_job).run(x, b["idx"][li], b["n"][li])
             if grp is not None and self.deadline:
                 grp.prefetch(main, self.side)   # for later steps; nothing waits within this one
         else:
-            (self.jobs0[l][slot] if l >= 0 else self.head_job0).run(x, b["act"][li])
+            (self.jobs0[l][slot] if l >= 0 else self.head_job0).run(x)
 
     def step(self, T: int, refine: bool = True) -> None:
         """One decode step of the token at position T (T tokens already in
@@ -310,9 +310,12 @@ class DecodeModel:
             attn_decode_refine(self.q_bf[l], L["kv"], Hkv, T + 1, k_tok, workspace=self.ws, out=self.att[l],
                                sel_out=self.sel[l], sel_n=self.sel_n[l])
             if L["kv_cache"] is not None and refine and k_tok > 0:
+                # the union's units, the KV cache's step and its fetches all run
+                # on the side stream: nothing later in this step waits for them
+                self.side.wait_stream(main)
                 attn_union_units(self.sel[l], self.sel_n[l], Hkv, (Hq // Hkv) * k_tok, self.S, self.units[l],
-                                 self.n_units[l])
-                L["kv_cache"].prefetch(self.units[l], self.n_units[l], main, self.side)
+                                 self.n_units[l], stream=self.side)
+                L["kv_cache"].prefetch(self.units[l], self.n_units[l], self.side, self.side)
                 side_used = True
             round_select(self.att[l].view(-1), self.buf["attn_out"]["x"][l], **self._sel(l, "attn_out", refine))
             self._linear(l, "attn_out", refine, main)

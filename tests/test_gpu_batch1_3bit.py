@@ -116,9 +116,8 @@ def test_gemv_batch1_3bit_jobs_with_caches(sf, K, Ns, cap_pct, pct):
         xd = bf16_dev(x)
         sf.select_topk_act(xd, k, idx, n, act)
         grp.prefetch(torch.cuda.current_stream(), side)
-        jobs.run(xd, act)
-        sf.act_prepare(xd, act0)
-        jobs0.run(xd, act0)
+        jobs.run(xd, idx, n)
+        jobs0.run(xd)
         torch.cuda.synchronize()
         S = oselect.select_topk(x, k)
         for m in mats:
@@ -148,7 +147,7 @@ def test_gemv_batch1_3bit_lm_head_size(sf):
     n = torch.zeros(1, dtype=torch.int32, device="cuda")
     act = torch.zeros(sf.act_bytes(K) // 4, dtype=torch.int32, device="cuda")
     sf.select_topk_act(xd, k, idx, n, act)
-    sf.gemv_refine_batch1([(m["qw"], None, True, m["y"])], xd, act)
+    sf.gemv_refine_batch1([(m["qw"], None, True, m["y"])], xd, idx, n)
     torch.cuda.synchronize()
     y_ref, a = ogemv.gemv_refine(m["qz"], x, oselect.select_topk(x, k))
     _check_gemv(m["y"].cpu().numpy()[None, m["rows"]], y_ref, a)
@@ -171,7 +170,7 @@ def test_gemv_batch1_huge_selected_outliers(sf, b_r, b_f):
     n = torch.zeros(1, dtype=torch.int32, device="cuda")
     act = torch.zeros(sf.act_bytes(K) // 4, dtype=torch.int32, device="cuda")
     sf.select_topk_act(xd, k, idx, n, act)
-    sf.gemv_refine_batch1([(m["qw"], None, True, m["y"])], xd, act)
+    sf.gemv_refine_batch1([(m["qw"], None, True, m["y"])], xd, idx, n)
     torch.cuda.synchronize()
     S = oselect.select_topk(x, k)
     assert {5, 300, 1800, 4000} <= set(S.tolist())
@@ -207,7 +206,7 @@ def test_gemv_batch1_deadline_caches(sf, b_r, b_f):
         x = gen_activations(2900 + step, 1, K, outl, 30.0)
         xd = bf16_dev(x)
         sf.select_topk_act(xd, k, idx, n, act)
-        jobs.run(xd, act)                                  # refines S ∩ cached
+        jobs.run(xd, idx, n)                               # refines S ∩ cached
         grp.prefetch(torch.cuda.current_stream(), side)    # then fetches the misses
         torch.cuda.synchronize()
         S = oselect.select_topk(x, k)

@@ -629,9 +629,8 @@ def test_gemv_batch1_jobs_with_caches(sf, K, Ns, cap_pct, pct):
         xd = bf16_dev(x)
         sf.select_topk_act(xd, k, idx, n, act)
         grp.prefetch(torch.cuda.current_stream(), side)
-        jobs.run(xd, act)
-        sf.act_prepare(xd, act0)
-        jobs0.run(xd, act0)
+        jobs.run(xd, idx, n)
+        jobs0.run(xd)
         torch.cuda.synchronize()
         S = oselect.select_topk(x, k)
         for m in mats:
@@ -660,7 +659,7 @@ def test_gemv_batch1_store_mode(sf, N, K, b_f):
     act = torch.zeros(sf.act_bytes(K) // 4, dtype=torch.int32, device="cuda")
     y = torch.empty(N, dtype=torch.float32, device="cuda")
     sf.select_topk_act(xd, k, idx, n, act)
-    sf.gemv_refine_batch1([(qw, None, True, y)], xd, act)
+    sf.gemv_refine_batch1([(qw, None, True, y)], xd, idx, n)
     torch.cuda.synchronize()
     y_ref, a = ogemv.gemv_refine(oquant.quantize_nested(W, G, 2, b_f), x, oselect.select_topk(x, k))
     _check_gemv(y.cpu().numpy()[None, :], y_ref, a)
