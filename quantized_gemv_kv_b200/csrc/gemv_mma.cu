@@ -306,52 +306,73 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
   for (int sp = 0; sp < SPW; ++sp) {
     const int slice = slice0 + sp;
     {
-      // lane (col n, t): group slot_b = n / 4, digit plane n % 4 (3: zero),
-      // channels 128 slot_b + 32 t + [0, 32) of the slice
+      // lane (col n, t): group slot_b = n / 4, digit plane n % 4 (3: zero);
+      // its B registers hold that plane's digits of channels
+      // 128 slot_b + 32 t + [0, 32) of the slice.  The four lanes of one
+      // (slot_b, t) share those channels: lane plane q converts channels
+      // 8q .. 8q + 7 and the lanes swap digit bytes by shuffles.
       const int bn = lane >> 2, slot_b = bn >> 2, plane = bn & 3;
-      const uint4* xp = reinterpret_cast<const uint4*>(a.x + 256 * static_cast<size_t>(slice) + 128 * slot_b +
-                                                       32 * tig);
-      uint32_t xw[16];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 v = xp[q];
-        xw[4 * q] = v.x; xw[4 * q + 1] = v.y; xw[4 * q + 2] = v.z; xw[4 * q + 3] = v.w;
-      }
-      // the group's largest |x| (15-bit magnitude keys order as |x| does)
+      const uint4 v = *reinterpret_cast<const uint4*>(a.x + 256 * static_cast<size_t>(slice) + 128 * slot_b +
+                                                     32 * tig + 8 * plane);
+      const uint32_t xw[4] = {v.x, v.y, v.z, v.w};
+      // the group's largest |x| (15-bit magnitude keys order as |x| does):
+      // lanes of one slot_b hold its 128 channels
       uint32_t kmax = 0u;
 #pragma unroll
-      for (int w = 0; w < 16; ++w) kmax = max(kmax, max(xw[w] & 0x7FFFu, (xw[w] >> 16) & 0x7FFFu));
-      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, 1));
-      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, 2));  // lanes t = 0..3 hold the 128 channels
+      for (int w = 0; w < 4; ++w) kmax = max(kmax, max(xw[w] & 0x7FFFu, (xw[w] >> 16) & 0x7FFFu));
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
       int e = sfd::bf16_exponent(kmax);
       if (e == -1000) e = 0;
-      // X = rint(x 2^(22 - e)): the scaling is exact (|x| < 2^e, the result
-      // below 2^22 in magnitude), the conversion rounds to nearest even
-      // (two exact power-of-two factors, so a group of bf16 subnormals with
-      // 22 - e above 127 does not overflow the factor)
+      // X = rint(x 2^(22 - e)): exact power-of-two factors (two, so a group
+      // of bf16 subnormals does not overflow one), rounding to nearest even
       const int s1 = min(22 - e, 126);
       const float sc1 = ldexpf(1.0f, s1), sc2 = ldexpf(1.0f, 22 - e - s1);
       int gs = 0;
-      uint32_t dg[8][2];
+      // pk[p][h]: plane-p digits of my channels 8 plane + 4 h + [0, 4): bytes
+      // in channel order
+      uint32_t pk[3][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}};
 #pragma unroll
-      for (int mm = 0; mm < 4; ++mm)
-#pragma unroll
-        for (int r = 0; r < 2; ++r) dg[mm][r] = 0u;
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
+      for (int c = 0; c < 8; ++c) {
         const int X = __float2int_rn(__uint_as_float(((xw[c >> 1] >> (16 * (c & 1))) & 0xFFFFu) << 16) * sc1 * sc2);
         gs += X;
         const int d0 = ((X + 128) & 255) - 128;
         const int X1 = (X - d0) >> 8;
         const int d1 = ((X1 + 128) & 255) - 128;
         const int d2 = (X1 - d1) >> 8;
-        const int dv = plane == 0 ? d0 : (plane == 1 ? d1 : (plane == 2 ? d2 : 0));
-        // channel c = 16 (mm / 2) + 4 b + 2 (mm % 2) + r of k-step 4 slot_b + mm
-        const int mm = 2 * (c >> 4) + ((c >> 1) & 1), b = (c >> 2) & 3, r = c & 1;
-        dg[mm][r] |= (static_cast<uint32_t>(dv) & 0xFFu) << (8 * b);
+        pk[0][c >> 2] |= (static_cast<uint32_t>(d0) & 0xFFu) << (8 * (c & 3));
+        pk[1][c >> 2] |= (static_cast<uint32_t>(d1) & 0xFFu) << (8 * (c & 3));
+        pk[2][c >> 2] |= (static_cast<uint32_t>(d2) & 0xFFu) << (8 * (c & 3));
       }
-      gs += __shfl_xor_sync(0xffffffffu, gs, 1);
-      gs += __shfl_xor_sync(0xffffffffu, gs, 2);
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) gs += __shfl_xor_sync(0xffffffffu, gs, o);  // the group's 128
+      // channel c of my run -> k-step 4 slot_b + mm, register r, byte b:
+      // mm = 2 (c >> 4) + ((c >> 1) & 1), b = (c >> 2) & 3, r = c & 1.  The
+      // channels 8q + [0, 8) of lane plane q fill bytes 2 (q & 1) + {0, 1} of
+      // the words (mm, r) with mm >> 1 = q >> 1.
+      uint32_t dg[4][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}, {0u, 0u}};
+#pragma unroll
+      for (int d = 0; d < 4; ++d) {
+        const int q = plane ^ d;  // the lane I receive from (and send to)
+        // send the digits of the receiver's plane (plane ^ d == q's plane)
+        const int rp = q;         // receiver of my data has plane q
+        const uint32_t s0 = rp == 0 ? pk[0][0] : (rp == 1 ? pk[1][0] : (rp == 2 ? pk[2][0] : 0u));
+        const uint32_t s1w = rp == 0 ? pk[0][1] : (rp == 1 ? pk[1][1] : (rp == 2 ? pk[2][1] : 0u));
+        const uint32_t r0 = __shfl_xor_sync(0xffffffffu, s0, 4 * d);
+        const uint32_t r1 = __shfl_xor_sync(0xffffffffu, s1w, 4 * d);
+        // r0 bytes: channels 8q + {0..3} = (mm = 2 (q >> 1) + 0/1 by bit 1 of c, r by bit 0, b = 2 (q & 1))
+        //   c = 8q + i, i = 0..3: (c >> 1) & 1 = i >> 1, r = i & 1, b = 2 (q & 1)
+        // r1 bytes: channels 8q + 4 + i: b = 2 (q & 1) + 1
+        const bool upper = (q >> 1) != 0;  // k-steps mm = 2, 3 (else 0, 1): selects keep dg in registers
+        const int bb = 2 * (q & 1);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = i & 1;
+          const uint32_t bits = (((r0 >> (8 * i)) & 0xFFu) << (8 * bb)) | (((r1 >> (8 * i)) & 0xFFu) << (8 * (bb + 1)));
+          dg[(i >> 1)][r] |= upper ? 0u : bits;
+          dg[2 + (i >> 1)][r] |= upper ? bits : 0u;
+        }
+      }
 #pragma unroll
       for (int m = 0; m < 8; ++m)
 #pragma unroll
@@ -363,18 +384,36 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
       gsm[sp] = __shfl_sync(0xffffffffu, gsum, 16 * myslot);
     }
     {
-      // the slice's run of the ascending selection
+      // the slice's run of the ascending selection: two rounds of a 32-way
+      // search (the first on every ceil(n / 32)-th entry, the second inside
+      // the segment it finds), for both ends of the slice
       const int lo = 256 * slice, hi = lo + 256;
+      const int step = (n_all + 31) >> 5;
       int c_lo = 0, c_hi = 0;
-      for (int i = lane; i < n_all; i += 32) {
-        const int v = a.idx[i];
-        c_lo += v < lo;
-        c_hi += v < hi;
-      }
+      if (step > 32) {  // more than 1024 selected: count by a plain sweep
+        for (int i = lane; i < n_all; i += 32) {
+          const int w = a.idx[i];
+          c_lo += w < lo;
+          c_hi += w < hi;
+        }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        c_lo += __shfl_xor_sync(0xffffffffu, c_lo, o);
-        c_hi += __shfl_xor_sync(0xffffffffu, c_hi, o);
+        for (int o = 16; o > 0; o >>= 1) {
+          c_lo += __shfl_xor_sync(0xffffffffu, c_lo, o);
+          c_hi += __shfl_xor_sync(0xffffffffu, c_hi, o);
+        }
+      } else if (n_all > 0) {
+        const int p1 = min(n_all - 1, lane * step);
+        const int v1 = a.idx[p1];
+        const bool in1 = lane * step < n_all;
+        const int seg_lo = __popc(__ballot_sync(0xffffffffu, in1 && v1 < lo));  // segments entirely below lo
+        const int seg_hi = __popc(__ballot_sync(0xffffffffu, in1 && v1 < hi));
+        // entries before segment seg - 1 are all below the bound; search it
+        const int b_lo = max(seg_lo - 1, 0) * step, b_hi = max(seg_hi - 1, 0) * step;
+        const bool ok_lo = lane < step && b_lo + lane < n_all, ok_hi = lane < step && b_hi + lane < n_all;
+        const int w_lo = ok_lo ? a.idx[b_lo + lane] : 0x7FFFFFFF;
+        const int w_hi = ok_hi ? a.idx[b_hi + lane] : 0x7FFFFFFF;
+        c_lo = b_lo + __popc(__ballot_sync(0xffffffffu, ok_lo && w_lo < lo));
+        c_hi = b_hi + __popc(__ballot_sync(0xffffffffu, ok_hi && w_hi < hi));
       }
       psl[sp] = c_lo;
       nsl[sp] = c_hi - c_lo;
