@@ -97,10 +97,10 @@ def parse():
 # ------------------------------------------------------------------ accounting
 
 # DRAM bytes per launch counted by ncu (dram__bytes_read.sum +
-# dram__bytes_write.sum) for the kernels as they stand; the commands are in
-# profiles/.  They are set back to None whenever the kernel changes.
+# dram__bytes_write.sum) in a capture of the kernel as it stands, or None when
+# the kernel has changed since its last capture.
 ATTN_TRAFFIC_32K = 21377792          # attn_fused_kernel<4>, Hq 32, Hkv 8, T 32768, k 1%
-GEMV_TRAFFIC_PER_LAUNCH = 15849088   # gemv_mma_kernel, mean of a layer's 4 launches (63.40 MB)
+GEMV_TRAFFIC_PER_LAUNCH = None       # gemv_mma_kernel (changed since its capture)
 
 
 def gemv_bytes(N, K, k_sel, b_r=B_R, b_f=B_F):
@@ -596,7 +596,7 @@ def hotpath_leg(args, sf, torch, dist, dev, world, T, phys):
         # the dominant kernel (largest share of the step's launch list): the
         # cluster attention; its launches of a step run in one graph, timed
         # with events on the launch stream.  traffic: ncu DRAM bytes of one
-        # launch of the same kernel (profiles/attn_fused_kernel_32k.md)
+        # launch of the same kernel (ATTN_TRAFFIC_32K)
         model.sync_caches()
         reps = 5
         g4 = capture(torch, model.attn_only, cap_stream)
@@ -615,7 +615,7 @@ def hotpath_leg(args, sf, torch, dist, dev, world, T, phys):
         del g4
         # the batch-1 GEMV, the next kernel by share: all its launches of a step
         # in one graph.  traffic: ncu DRAM bytes of the four launches of a
-        # layer, per launch (profiles/gemv_mma_kernel_gateup_llama31_8b.md)
+        # layer, per launch (GEMV_TRAFFIC_PER_LAUNCH)
         g2 = capture(torch, model.gemvs_only, cap_stream)
         for _ in range(2):
             with torch.cuda.stream(cap_stream):
