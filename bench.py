@@ -87,6 +87,9 @@ def parse():
     ap.add_argument("--weight-deadline", type=int, default=1,
                     help="1: GEMVs refine the selected columns already cached and misses are fetched for later "
                          "steps; 0: every GEMV waits for the fetch of its own selection")
+    ap.add_argument("--fetch-lead", type=int, default=1,
+                    help="1: prefetch the next residual-fed inputs' predicted channels a block ahead (with the "
+                         "deadline reading)")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-extras", action="store_true", help="skip e2e / resident-only / roofline legs")
     ap.add_argument("--hotpath-context", type=int, default=32768,
@@ -766,7 +769,8 @@ def step_model(args, sf, torch, dev, layers):
     budget = None if args.kv_budget < 0 else args.kv_budget
     m = DecodeModel(shape, weight, norm, kv, capacity=args.context, p=Fraction(TOPK_PCT, 100),
                     p_tok=Fraction(TOK_PCT, 100), weight_cache_pct=CACHE_PCT, kv_cache_pct=kv_pct,
-                    kv_budget=budget, weight_deadline=bool(args.weight_deadline), device=dev)
+                    kv_budget=budget, weight_deadline=bool(args.weight_deadline),
+                    fetch_lead=bool(args.fetch_lead), device=dev)
     return m, T
 
 
@@ -975,7 +979,9 @@ def run_sf(args, rank, world, local_rank, dist):
                    "topk_channels": "3% of each GEMV input",
                    "weight_cache": "10% LRU per matrix, " + ("deadline reading (misses fetched for later steps)"
                                                               if args.weight_deadline else
-                                                              "every GEMV waits for its misses"),
+                                                              "every GEMV waits for its misses")
+                   + ("; fetch lead: q/k/v, gate/up and LM-head channels predicted from the residual stream "
+                      "a block ahead and prefetched" if args.fetch_lead and args.weight_deadline else ""),
                    "topk_tokens": "1% per query head", "kv_cache": (f"{args.kv_cache_pct}% of token-heads, "
                                                                     f"one LRU per KV head, budget {args.kv_budget} per head and step"
                                                                     if args.kv_cache_pct >= 0 else "store in HBM"),

@@ -58,15 +58,18 @@ __device__ void load_q(const uint16_t* __restrict__ q, int g, float (*qs)[D], fl
 
 // ---- pass A on the tensor cores: integer MMA over code bytes ----------------
 //
-// Per KV group, the query heads become exact-as-possible fixed point: per
-// head X_d = rint(q_d 2^(23 - e)), e the binary exponent of max |q| (every
-// bf16 within 15 binades of the maximum is exact), split into three byte
-// planes.  mma.m16n8k32 (u8 codes x u8/s8 planes, s32 accumulate) gives
-// sum_d c_d X_d per plane exactly; the reduction order inside an MMA does not
-// matter, so a code word becomes a fragment register with one shift and one
-// mask ((w >> 2 tig) & 0x03030303 holds dims tig, tig+4, tig+8, tig+12), and
-// the q planes are laid out in the same permuted order.  A warp scores 16
-// tokens per MMA row tile for all heads of the group at once (n = heads).
+// Per KV group, the query heads become fixed point: per head
+// X_d = rint(q_d 2^(14 - e)), e the binary exponent of max |q| (|X| <= 2^14;
+// the rounding, |dq| <= 2^(e - 15), is inside the band's error bound eps),
+// split into two signed byte planes X = d0 + 256 d1.  mma.m16n8k32 (u8 codes
+// x s8 planes, s32 accumulate) gives sum_d c_d X_d per plane exactly; the
+// reduction order inside an MMA does not matter, so a code word becomes a
+// fragment register with one shift and one mask ((w >> 2 tig) & 0x03030303
+// holds dims tig, tig+4, tig+8, tig+12), and the q planes are laid out in the
+// same permuted order.  MMA column 2 h + p is (head h, plane p), so one MMA
+// per 32 dims covers four heads and lane tig ends with both planes of head
+// tig for its two tokens: a warp scores 16 tokens of four heads per four
+// MMAs (two n-tiles for eight heads per group).
 
 // A CTA owns a contiguous token range of one group; each warp streams its run
 // of 16-token tiles through its own ring of kScRing cp.async stages (seven
@@ -74,6 +77,7 @@ __device__ void load_q(const uint16_t* __restrict__ q, int g, float (*qs)[D], fl
 // are staged in shared memory at the start.
 
 constexpr int kScThreads = 256;
+constexpr int kScQFrac = 14;      // fraction bits of the fixed-point q (relative to 2^e)
 constexpr int kScW = kScThreads / 32;
 constexpr int kScRing = 8;        // cp.async stages per warp, one 16-token tile each
 constexpr int kScMaxTok = 4096;   // tokens per CTA at most
@@ -96,7 +100,7 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
   int* hs = reinterpret_cast<int*>(ksz + kScMaxTok);                 // [GRP][kHistBins]
   __shared__ int qx[GRP][D];
   __shared__ float qsc[GRP], qsm[GRP];
-  __shared__ uint32_t bfr[24][32];  // B fragments of qx, per lane
+  __shared__ uint32_t bfr[4 * ((2 * GRP + 7) / 8) * 2][32];  // B fragments of qx, per lane
   const int g = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g8 = lane >> 2, tig = lane & 3;
   const int t0 = blockIdx.x * tpc;
@@ -154,42 +158,52 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
     int e = 0;
     if (am > 0.0f) frexpf(am, &e);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) qx[h][4 * lane + i] = __float2int_rn(ldexpf(v[i], 23 - e));
+    for (int i = 0; i < 4; ++i) qx[h][4 * lane + i] = __float2int_rn(ldexpf(v[i], kScQFrac - e));
     if (lane == 0) {
-      qsc[h] = ldexpf(1.0f, e - 23);
+      qsc[h] = ldexpf(1.0f, e - kScQFrac);
       qsm[h] = qs_l;
     }
   }
   __syncthreads();
-  // B fragments (column n = g8 is query head g8, zero beyond the group),
-  // built once per CTA: word [ks][p][half][lane]
-  for (int e = tid; e < 24 * 32; e += kScThreads) {
-    const int ln = e & 31, f = e >> 5, ks = f / 6, p = (f / 2) % 3, half = f & 1;
-    const int gg = ln >> 2, tt = ln & 3;
+  // B fragments, built once per CTA: word [ks][nt][half][lane]; column
+  // n = lane / 4 of n-tile nt is (head (8 nt + n) / 2, plane n % 2), zero
+  // beyond the group
+  constexpr int NT = (2 * GRP + 7) / 8;
+  for (int e = tid; e < 4 * NT * 2 * 32; e += kScThreads) {
+    const int ln = e & 31, f = e >> 5, half = f & 1, nt = (f >> 1) % NT, ks = (f >> 1) / NT;
+    const int col = 8 * nt + (ln >> 2), hh = col >> 1, pl = col & 1, tt = ln & 3;
     uint32_t v = 0;
-    if (gg < GRP) {
+    if (hh < GRP) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        v |= ((static_cast<uint32_t>(qx[gg][16 * (2 * ks + half) + tt + 4 * i]) >> (8 * p)) & 0xFFu) << (8 * i);
+      for (int i = 0; i < 4; ++i) {
+        const int X = qx[hh][16 * (2 * ks + half) + tt + 4 * i];
+        const int d0 = ((X + 128) & 255) - 128;
+        const int dv = pl == 0 ? d0 : (X - d0) >> 8;
+        v |= (static_cast<uint32_t>(dv) & 0xFFu) << (8 * i);
+      }
     }
     bfr[f][ln] = v;
   }
   __syncthreads();
-  uint32_t bq[4][3][2];
+  uint32_t bq[4][NT][2];
 #pragma unroll
   for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
-    for (int p = 0; p < 3; ++p)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int half = 0; half < 2; ++half) bq[ks][p][half] = bfr[(ks * 3 + p) * 2 + half][lane];
-  // this lane's heads (2 tig, 2 tig + 1; with four heads 2 (tig & 1) and the
-  // next, lanes tig >= 2 scoring the second token of the pair): max |score|
-  // and the largest score key
-  const int h0 = GRP == 4 ? 2 * (tig & 1) : 2 * tig, h1 = h0 + 1;
-  const float qsc0 = h0 < GRP ? qsc[h0] : 0.0f, qsm0 = h0 < GRP ? qsm[h0] : 0.0f;
-  const float qsc1 = h1 < GRP ? qsc[h1] : 0.0f, qsm1 = h1 < GRP ? qsm[h1] : 0.0f;
-  float am0 = 0.0f, am1 = 0.0f;
-  uint32_t km0 = 0u, km1 = 0u;
+      for (int half = 0; half < 2; ++half) bq[ks][nt][half] = bfr[(ks * NT + nt) * 2 + half][lane];
+  // this lane's head of each n-tile (4 nt + tig): max |score| and the largest
+  // score key
+  float qscv[NT], qsmv[NT], am[NT];
+  uint32_t km[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int h = 4 * nt + tig;
+    qscv[nt] = h < GRP ? qsc[h] : 0.0f;
+    qsmv[nt] = h < GRP ? qsm[h] : 0.0f;
+    am[nt] = 0.0f;
+    km[nt] = 0u;
+  }
   for (int ti = tile0; ti < tile1; ++ti) {
     if (ti + kScRing - 1 < tile1) issue(ti + kScRing - 1);
     cp_async_commit_attn();
@@ -207,53 +221,38 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
       wb[4] = xb1.x; wb[5] = xb1.y; wb[6] = xb1.z; wb[7] = xb1.w;
     }
     __syncwarp();  // the stage is refilled by a later issue
-    int d0[4] = {0, 0, 0, 0}, d1[4] = {0, 0, 0, 0}, d2[4] = {0, 0, 0, 0};
+    int d[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) d[nt][0] = d[nt][1] = d[nt][2] = d[nt][3] = 0;
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
       const uint32_t a0 = (wa[2 * ks] >> (2 * tig)) & 0x03030303u;
       const uint32_t a1 = (wb[2 * ks] >> (2 * tig)) & 0x03030303u;
       const uint32_t a2 = (wa[2 * ks + 1] >> (2 * tig)) & 0x03030303u;
       const uint32_t a3 = (wb[2 * ks + 1] >> (2 * tig)) & 0x03030303u;
-      mma_u8u8(d0, a0, a1, a2, a3, bq[ks][0][0], bq[ks][0][1]);
-      mma_u8u8(d1, a0, a1, a2, a3, bq[ks][1][0], bq[ks][1][1]);
-      mma_u8s8(d2, a0, a1, a2, a3, bq[ks][2][0], bq[ks][2][1]);
-    }
-    // d[i]: i = 0,1 -> token ta, heads 2 tig, 2 tig + 1; i = 2,3 -> token tb
-    const int ta = 16 * ti + g8, tb = ta + 8;
-    if constexpr (GRP == 4) {
-      // columns 4..7 are padding: lanes tig >= 2 take token tb of lane ^ 2,
-      // so every lane scores two values
-      const bool up = tig >= 2;
-      const int x0 = __shfl_xor_sync(0xffffffffu, d0[2], 2), x1 = __shfl_xor_sync(0xffffffffu, d0[3], 2);
-      const int y0 = __shfl_xor_sync(0xffffffffu, d1[2], 2), y1 = __shfl_xor_sync(0xffffffffu, d1[3], 2);
-      const int z0 = __shfl_xor_sync(0xffffffffu, d2[2], 2), z1 = __shfl_xor_sync(0xffffffffu, d2[3], 2);
-      if (up) {
-        d0[0] = x0; d0[1] = x1;
-        d1[0] = y0; d1[1] = y1;
-        d2[0] = z0; d2[1] = z1;
-      }
-    }
-    constexpr int kVals = GRP == 4 ? 2 : 4;
 #pragma unroll
-    for (int i = 0; i < kVals; ++i) {
-      const int h = (i & 1) ? h1 : h0;
-      const int tl = GRP == 4 ? (tig >= 2 ? tb : ta) : ((i < 2) ? ta : tb);
-      if (h < GRP && tl < n) {
-        const uint32_t kz = ksz[tl];
-        const float sv = sfd::half_bits_to_float(static_cast<uint16_t>(kz & 0xFFFFu));
-        const float zv = sfd::half_bits_to_float(static_cast<uint16_t>(kz >> 16));
-        const float P = (static_cast<float>(d2[i]) * 65536.0f + static_cast<float>(d1[i]) * 256.0f +
-                         static_cast<float>(d0[i])) * ((i & 1) ? qsc1 : qsc0);
-        const float E = fmaf(4.0f, P, (1.5f - zv) * ((i & 1) ? qsm1 : qsm0));
-        const float val = (sv * E) * kInvSqrtD;
-        score[(static_cast<size_t>(g) * GRP + h) * T + t0 + tl] = val;
-        atomicAdd(&hs[h * kHistBins + (okey32(val) >> kHistShift)], 1);
-        if (i & 1) {
-          am1 = fmaxf(am1, fabsf(val));
-          km1 = max(km1, okey32(val));
-        } else {
-          am0 = fmaxf(am0, fabsf(val));
-          km0 = max(km0, okey32(val));
+      for (int nt = 0; nt < NT; ++nt) mma_u8s8(d[nt], a0, a1, a2, a3, bq[ks][nt][0], bq[ks][nt][1]);
+    }
+    // d[nt][0], [1]: token ta, planes 0 and 1 of head 4 nt + tig; [2], [3]: token tb
+    const int ta = 16 * ti + g8, tb = ta + 8;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int h = 4 * nt + tig;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int tl = i ? tb : ta;
+        if (h < GRP && tl < n) {
+          const uint32_t kz = ksz[tl];
+          const float sv = sfd::half_bits_to_float(static_cast<uint16_t>(kz & 0xFFFFu));
+          const float zv = sfd::half_bits_to_float(static_cast<uint16_t>(kz >> 16));
+          // sum_d c_d X_d is below 3 * 128 * 2^14 < 2^23: exact in fp32
+          const float P = static_cast<float>(d[nt][2 * i] + 256 * d[nt][2 * i + 1]) * qscv[nt];
+          const float E = fmaf(4.0f, P, (1.5f - zv) * qsmv[nt]);
+          const float val = (sv * E) * kInvSqrtD;
+          score[(static_cast<size_t>(g) * GRP + h) * T + t0 + tl] = val;
+          atomicAdd(&hs[h * kHistBins + (okey32(val) >> kHistShift)], 1);
+          am[nt] = fmaxf(am[nt], fabsf(val));
+          km[nt] = max(km[nt], okey32(val));
         }
       }
     }
@@ -261,22 +260,18 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
   cp_async_wait_attn<0>();
   smx = warp_max(smx);
   if (lane == 0) atomicMax(reinterpret_cast<unsigned int*>(smax + g), __float_as_uint(smx));
-  // lanes with the same tig hold the same two heads
+  // lanes with the same tig hold the same heads
 #pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    am0 = fmaxf(am0, __shfl_xor_sync(0xffffffffu, am0, o));
-    am1 = fmaxf(am1, __shfl_xor_sync(0xffffffffu, am1, o));
-    km0 = max(km0, __shfl_xor_sync(0xffffffffu, km0, o));
-    km1 = max(km1, __shfl_xor_sync(0xffffffffu, km1, o));
-  }
-  if (g8 == 0) {
-    if (h0 < GRP) {
-      atomicMax(amaxu + g * GRP + h0, __float_as_uint(am0));
-      atomicMax(mkey + g * GRP + h0, km0);
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      am[nt] = fmaxf(am[nt], __shfl_xor_sync(0xffffffffu, am[nt], o));
+      km[nt] = max(km[nt], __shfl_xor_sync(0xffffffffu, km[nt], o));
     }
-    if (h1 < GRP) {
-      atomicMax(amaxu + g * GRP + h1, __float_as_uint(am1));
-      atomicMax(mkey + g * GRP + h1, km1);
+    const int h = 4 * nt + tig;
+    if (g8 == 0 && h < GRP) {
+      atomicMax(amaxu + g * GRP + h, __float_as_uint(am[nt]));
+      atomicMax(mkey + g * GRP + h, km[nt]);
     }
   }
   __syncthreads();
@@ -333,7 +328,7 @@ attn_select_compact_kernel(const uint16_t* __restrict__ q, int T, int k, const f
   __shared__ int qe_sh;
   __shared__ int base_sh;
   select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status);
-  const double eps_s = select_eps(static_cast<double>(smax[g]), l1_sh, qe_sh, __uint_as_float(amaxu[h]));
+  const double eps_s = select_eps(static_cast<double>(smax[g]), l1_sh, qe_sh, __uint_as_float(amaxu[h]), kScQFrac);
   uint32_t b1;
   int kk;
   float f_low;
@@ -444,7 +439,7 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
       if (tid == 0) qxsum_sh = sx;
     }
   }
-  const double eps_s = select_eps(static_cast<double>(smax[g]), l1_sh, qe_sh, __uint_as_float(amaxu[h]));
+  const double eps_s = select_eps(static_cast<double>(smax[g]), l1_sh, qe_sh, __uint_as_float(amaxu[h]), kScQFrac);
   uint32_t b1;
   int kk;
   float f_low;

@@ -239,16 +239,18 @@ __device__ void select_q_prologue(const uint16_t* __restrict__ q, int h, int g, 
   __syncthreads();
 }
 
-// Error bound of the fast scores (pass A): q rounded to 24-bit fixed point
-// (|dq| <= 2^(e-24) per entry), exact integer products and sums, an fp32
-// combine of the three plane sums, the fp32 sum of q (<= gamma_128 l1), and
-// the roundings of the zero-point term, the fma, the scale and 1/sqrt(d).
+// Error bound of the fast scores (pass A): q rounded to fixed point with
+// qfrac fraction bits relative to 2^e, X = rint(q 2^(qfrac - e)), so
+// |dq| <= 2^(e - qfrac - 1) per entry (the cluster kernel: 23 bits; the
+// pipeline's score pass: 14), exact integer products and sums, an fp32
+// combine of the plane sums, the fp32 sum of q (<= gamma_128 l1), and the
+// roundings of the zero-point term, the fma, the scale and 1/sqrt(d).
 // Returns the half-width eps_s of the band; two fast scores whose exact
 // values are ordered one way differ by at least -2 eps_s the other way.
-__device__ __forceinline__ double select_eps(double s_max, double l1, int qe, float amax) {
+__device__ __forceinline__ double select_eps(double s_max, double l1, int qe, float amax, int qfrac) {
   const double u = 5.9604644775390625e-8;  // 2^-24
   const double gam = 130.0 * u / (1.0 - 130.0 * u);
-  const double qround = ldexp(1.0, qe - 24);
+  const double qround = ldexp(1.0, qe - qfrac - 1);
   const double eps_k = s_max * (4.0 * 3.0 * D * qround + l1 * (136.0 * u + 16.0 * gam));
   return 2.0 * (static_cast<double>(kInvSqrtD) * eps_k + 4.0 * u * static_cast<double>(amax));
 }

@@ -710,7 +710,7 @@ __global__ void __launch_bounds__(kFThreads, 2) attn_fused_kernel(const FusedArg
     __syncthreads();
     if (tid < GRP) {
       const float amax = fmaxf(fabsf(from_okey32(gl0[tid])), fabsf(from_okey32(gl0[GRP + tid])));
-      eps_sh[tid] = select_eps(static_cast<double>(__uint_as_float(gl0[2 * GRP])), l1_sh[tid], qe_sh[tid], amax);
+      eps_sh[tid] = select_eps(static_cast<double>(__uint_as_float(gl0[2 * GRP])), l1_sh[tid], qe_sh[tid], amax, 23);
       lo_sh[tid] = gl0[GRP + tid];
       hi_sh[tid] = gl0[tid];
       kk_sh[tid] = k;

@@ -118,13 +118,15 @@ class DecodeModel:
 
     def __init__(self, shape: Shape, weight, norm, kv, capacity: int, p: Fraction = Fraction(3, 100),
                  p_tok: Fraction = Fraction(1, 100), weight_cache_pct=None, kv_cache_pct=None,
-                 kv_budget: int | None = None, weight_deadline: bool = False, record: bool = False, device=None):
+                 kv_budget: int | None = None, weight_deadline: bool = False, fetch_lead: bool = False,
+                 record: bool = False, device=None):
         self.s = shape
         self.dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
         self.p, self.p_tok = Fraction(p), Fraction(p_tok)
         self.S = capacity
         self.record = record
         self.deadline = weight_deadline and weight_cache_pct is not None
+        self.lead = fetch_lead and self.deadline
         H, F, d = shape.hidden, shape.mlp, shape.head_dim
         Hq, Hkv = shape.n_q, shape.n_kv
         dev = self.dev
@@ -134,7 +136,8 @@ class DecodeModel:
         self.K_in = {"attn_in": H, "attn_out": Hq * d, "mlp_in": H, "mlp_mid": F, "head": H}
         slot_of = {"q": "attn_in", "k": "attn_in", "v": "attn_in", "o": "attn_out", "gate": "mlp_in",
                    "up": "mlp_in", "down": "mlp_mid"}
-        self.side = torch.cuda.Stream(device=dev)
+        self.side = torch.cuda.Stream(device=dev)      # weight caches' steps and gathers
+        self.side_kv = torch.cuda.Stream(device=dev)   # the KV caches' bookkeeping and gathers
         self.layers = []
         kv_b_r, kv_b_f = shape.kv_bits
         self.kv_cache_pct = kv_cache_pct
@@ -243,6 +246,21 @@ class DecodeModel:
         self.head_job = Batch1Jobs([(self.head.qw, self.head.cache, not cached, self.logits)])
         self.head_job0 = Batch1Jobs([(self.head.qw, None, False, self.logits)])
         self.head_group = RefineGroup([(self.head.cache, hb["idx"][0], hb["n"][0])]) if cached else None
+        # fetch lead: the predicted selections of the inputs fed by the
+        # residual stream (q/k/v, gate/up, LM head) and their groups
+        self.pred, self.pgroups, self.head_pgroup = {}, [], None
+        if self.lead:
+            dev, nl = self.dev, self.s.layers
+            for slot in ("attn_in", "mlp_in", "head"):
+                K, rows = self.K_in[slot], (1 if slot == "head" else nl)
+                self.pred[slot] = dict(x=torch.zeros((rows, K), dtype=torch.bfloat16, device=dev),
+                                       idx=torch.zeros((rows, max(1, self.k_in[slot])), dtype=torch.int32, device=dev),
+                                       n=torch.zeros((rows, 1), dtype=torch.int32, device=dev))
+            for l, L in enumerate(self.layers):
+                self.pgroups.append({slot: RefineGroup([(L[n].cache, self.pred[slot]["idx"][l], self.pred[slot]["n"][l])
+                                                        for n in groups[slot]]) for slot in ("attn_in", "mlp_in")})
+            ph = self.pred["head"]
+            self.head_pgroup = RefineGroup([(self.head.cache, ph["idx"][0], ph["n"][0])])
 
     # ---- the step -----------------------------------------------------------------------
 
@@ -270,6 +288,25 @@ class DecodeModel:
         else:
             (self.jobs0[l][slot] if l >= 0 else self.head_job0).run(x)
 
+    def _predict(self, l, slot, norm_w, main):
+        """Fetch lead: select the channels the input of `slot` (layer l; the LM
+        head for l < 0) will have, from the residual stream as it is now
+        (RMSNorm of the current residual with that input's norm weights), and
+        step those matrices' caches with the prediction, on the side stream,
+        while the main stream goes on.  The main stream waits for the
+        prediction's read of the residual before it changes the residual."""
+        pr = self.pred[slot]
+        li = max(l, 0)
+        self.side.wait_stream(main)
+        with torch.cuda.stream(self.side):
+            norm_select(self.x, norm_w, pr["x"][li], k=self.k_in[slot], idx=pr["idx"][li], n=pr["n"][li], act=None,
+                        eps=self.s.eps, delta=None)
+            ev = torch.cuda.Event()
+            ev.record(self.side)
+        grp = self.pgroups[l][slot] if l >= 0 else self.head_pgroup
+        grp.prefetch(self.side, self.side)
+        return ev
+
     def step(self, T: int, refine: bool = True) -> None:
         """One decode step of the token at position T (T tokens already in
         every layer's cache); x_in holds the token's embedding.  refine=False
@@ -284,11 +321,18 @@ class DecodeModel:
         k_tok = count_half_up(self.p_tok, T + 1) if refine else 0
         self.k_tok = k_tok
         side_used = refine and any(self.wgroups) or (refine and self.head_group is not None)
+        kv_used = False
+        lead = refine and self.lead
         self.x.copy_(self.x_in)
         prev = None
+        read_done = None  # the last prediction's read of the residual
         for l, L in enumerate(self.layers):
+            if read_done is not None:
+                main.wait_event(read_done)
             norm_select(self.x, L["norm1"], self.buf["attn_in"]["x"][l], eps=s.eps, delta=prev,
                         **self._sel(l, "attn_in", refine))
+            if lead:  # gate/up of this layer, from the residual before the attention
+                read_done = self._predict(l, "mlp_in", L["norm2"], main)
             if self.record:
                 self.x_hist[l].copy_(self.x)
             self._linear(l, "attn_in", refine, main)
@@ -311,22 +355,31 @@ class DecodeModel:
                                sel_out=self.sel[l], sel_n=self.sel_n[l])
             if L["kv_cache"] is not None and refine and k_tok > 0:
                 # the union's units, the KV cache's step and its fetches all run
-                # on the side stream: nothing later in this step waits for them
-                self.side.wait_stream(main)
+                # on their own side stream: nothing later in this step waits
+                self.side_kv.wait_stream(main)
                 attn_union_units(self.sel[l], self.sel_n[l], Hkv, (Hq // Hkv) * k_tok, self.S, self.units[l],
-                                 self.n_units[l], stream=self.side)
-                L["kv_cache"].prefetch(self.units[l], self.n_units[l], self.side, self.side)
-                side_used = True
+                                 self.n_units[l], stream=self.side_kv)
+                L["kv_cache"].prefetch(self.units[l], self.n_units[l], self.side_kv, self.side_kv)
+                kv_used = True
             round_select(self.att[l].view(-1), self.buf["attn_out"]["x"][l], **self._sel(l, "attn_out", refine))
             self._linear(l, "attn_out", refine, main)
+            if read_done is not None:
+                main.wait_event(read_done)
             norm_select(self.x, L["norm2"], self.buf["mlp_in"]["x"][l], eps=s.eps, delta=L["o"].y,
                         **self._sel(l, "mlp_in", refine))
+            read_done = None
+            if lead:  # the next layer's q/k/v (or the LM head), from the residual after the attention
+                nxt = self.layers[l + 1]["norm1"] if l + 1 < s.layers else self.final_norm
+                read_done = self._predict(l + 1 if l + 1 < s.layers else -1, "attn_in" if l + 1 < s.layers else "head",
+                                          nxt, main)
             if self.record:
                 self.h_hist[l].copy_(self.x)
             self._linear(l, "mlp_in", refine, main)
             silu_mul_select(L["gate"].y, L["up"].y, self.buf["mlp_mid"]["x"][l], **self._sel(l, "mlp_mid", refine))
             self._linear(l, "mlp_mid", refine, main)
             prev = L["down"].y
+        if read_done is not None:
+            main.wait_event(read_done)
         norm_select(self.x, self.final_norm, self.buf["head"]["x"][0], eps=s.eps, delta=prev,
                     **self._sel(-1, "head", refine))
         if self.record:
@@ -336,6 +389,8 @@ class DecodeModel:
         # included) completes within the step
         if side_used:
             main.wait_stream(self.side)
+        if kv_used:
+            main.wait_stream(self.side_kv)
 
     def union(self, l: int) -> list:
         """Layer l's union token lists of the last step (host lists)."""
@@ -380,9 +435,11 @@ class DecodeModel:
         return tot
 
     def close(self) -> None:
-        for G in self.wgroups:
+        for G in self.wgroups + self.pgroups:
             for g in G.values():
                 g.close()
+        if self.head_pgroup is not None:
+            self.head_pgroup.close()
         if self.head_group is not None:
             self.head_group.close()
         for L in self.layers:

@@ -248,18 +248,21 @@ def test_decode_step_store_mode_against_oracle(sf):
     m.close()
 
 
-@pytest.mark.parametrize("deadline", [False, True])
-def test_decode_step_cache_mode_against_oracle(sf, deadline):
+@pytest.mark.parametrize("deadline,lead", [(False, False), (True, False), (True, True)])
+def test_decode_step_cache_mode_against_oracle(sf, deadline, lead):
     """Weight refinements behind 25% LRU caches and K/V refinements behind a
     20% KV refinement cache per layer with a fetch budget, over three decode
     steps at positions T0, T0+1, T0+2: every op of every step, the attention
     refining only the union tokens cached when the step starts, and the cache
     sets of one weight matrix per input and of each layer's KV cache.  With
     the deadline reading the GEMVs refine only the selected columns cached
-    when the step starts (and never wait for a fetch)."""
+    when the step starts (and never wait for a fetch); with fetch lead the
+    q/k/v, gate/up and LM-head caches are first stepped with the channels
+    predicted from the residual stream a block ahead."""
     host = _host_model()
     budget = 12                                   # per KV head and step
-    m = _build(sf, host, weight_cache_pct=25, kv_cache_pct=20, kv_budget=budget, weight_deadline=deadline)
+    m = _build(sf, host, weight_cache_pct=25, kv_cache_pct=20, kv_budget=budget, weight_deadline=deadline,
+               fetch_lead=lead)
     olayers, ohead, ofinal, okv = _oracle_model(host)
     # oracle LRUs: q (attn_in), o, gate (mlp_in), down, head; the KV caches
     worcs = {slot: [ocache.LRUCache(K, od.count_half_up(Fraction(25, 100), K)) for _ in range(NL)]
@@ -280,14 +283,29 @@ def test_decode_step_cache_mode_against_oracle(sf, deadline):
                     if t <= T:
                         a[gh, t] = True
             avail.append(a)
-        wcached = None
-        if deadline:
-            wcached = {(l, slot): set(orcs[l].snapshot()) for slot, orcs in worcs.items() for l in range(NL)}
-            wcached[(-1, "head")] = set(horc.snapshot())
         m.x_in.copy_(torch.from_numpy(_embedding(7200 + step)))
         m.step(T)
         torch.cuda.synchronize()
         m.sync()
+        if lead:
+            # the predictions: each from the residual as it stood (teacher
+            # forced), selected exactly, and stepped into the caches first
+            xh, hh = m.x_hist.cpu().numpy().astype(np.float64), m.h_hist.cpu().numpy().astype(np.float64)
+            preds = [("mlp_in", l, xh[l], olayers[l]["norm2"]) for l in range(NL)]
+            preds += [("attn_in", l + 1, hh[l], olayers[l + 1]["norm1"]) for l in range(NL - 1)]
+            preds += [("head", -1, hh[NL - 1], ofinal)]
+            for slot, l, resid, wn in preds:
+                pr = m.pred[slot]
+                li = max(l, 0)
+                pb = _bits(pr["x"][li])
+                _check_bf16(pb, od.rms_norm(resid, wn))
+                S = oselect.select_topk(pb[None, :], m.k_in[slot])
+                np.testing.assert_array_equal(pr["idx"][li].cpu().numpy()[: int(pr["n"][li].item())], S)
+                (horc if slot == "head" else worcs[slot][l]).step(S.tolist())
+        wcached = None
+        if deadline:
+            wcached = {(l, slot): set(orcs[l].snapshot()) for slot, orcs in worcs.items() for l in range(NL)}
+            wcached[(-1, "head")] = set(horc.snapshot())
         okv = _check_step(m, olayers, ohead, ofinal, okv, T, available=avail, wcached=wcached)
         for slot, orcs in worcs.items():
             for l in range(NL):
