@@ -287,6 +287,43 @@ sf_status sf_refine_group_destroy(sf_refine_group* g);
 sf_status sf_gemv_refine(const sf_qweight* W, const uint16_t* x, int B, const int32_t* idx,
                          const int32_t* n, sf_refine_cache* c, float* y, sf_stream_t stream);
 
+/* ---- comparator modes (rag-lover.com explainer, 既存手法との違い) -------- */
+
+/*
+ * sf_select_random -- random selection of k of K channels (the ablation the
+ * explainer sets against selection by activation magnitude): the k largest
+ * keys key_j = (splitmix64(seed + K*step + j) >> 49) mod 32640 (Steele, Lea
+ * and Flood's splitmix64 finalizer: z += 0x9E3779B97F4A7C15; z = (z ^ z>>30)
+ * * 0xBF58476D1CE4E5B9; z = (z ^ z>>27) * 0x94D049BB133111EB; z ^ z>>31), ties
+ * to the lower channel; idx_out ascending (device, capacity k), *n_out = k.
+ * Counter-based: any (seed, step) is reproducible on its own.
+ * Constraints: 1 <= K <= 32768, 0 <= k <= K.
+ */
+sf_status sf_select_random(int K, int k, uint64_t seed, uint64_t step, int32_t* idx_out, int32_t* n_out,
+                           sf_stream_t stream);
+
+/*
+ * sf_quantize_residual -- the FP16-fetch comparator's store (DecDEC-like
+ * residual columns): out[j][i] = fp16_RNE(W[i][j] - w_res[i][j]), W the fp32
+ * weights [N][K] that Wq quantizes, w_res their resident values; the
+ * difference is exact in fp64 and rounded once.  out: device fp16 [K][N]
+ * (column-major: one column = one transfer unit of N*2 bytes).
+ */
+sf_status sf_quantize_residual(const float* W, const sf_qweight* Wq, uint16_t* out, sf_stream_t stream);
+
+/*
+ * sf_gemv_fp16_fetch -- the FP16-fetch comparator of sf_gemv_refine: the
+ * selected columns use w_res + r (r from sf_quantize_residual) instead of
+ * their refinement bits, the others w_res:
+ *   y[b][i] = sum_j x[b][j] w_res[i][j] + sum_{j in S} x[b][j] r[j][i].
+ * resid: the residual store [K][N] fp16 in device memory, or c: a cache of
+ * its columns (units of N*2 bytes; its last prefetch used (idx, n)); exactly
+ * one of the two.  Computed on the CUDA cores (the generic GEMV with an fp16
+ * correction).  Constraints and accuracy as sf_gemv_refine.
+ */
+sf_status sf_gemv_fp16_fetch(const sf_qweight* W, const uint16_t* x, int B, const int32_t* idx, const int32_t* n,
+                             const uint16_t* resid, sf_refine_cache* c, float* y, sf_stream_t stream);
+
 /* ---- batch-1 fast path: prepared activations, several matrices per launch */
 
 /* Bytes of the prepared form of one activation row of K channels (K/256

@@ -91,6 +91,9 @@ _SIGS = {
     "sf_refine_group_destroy": ([_p], _i),
     "sf_gemv_refine": ([ctypes.POINTER(_QWeight), _p, _i, _p, _p, _p, _p, _p], _i),
     "sf_act_bytes": ([_i], _sz),
+    "sf_select_random": ([_i, _i, ctypes.c_uint64, ctypes.c_uint64, _p, _p, _p], _i),
+    "sf_quantize_residual": ([_p, ctypes.POINTER(_QWeight), _p, _p], _i),
+    "sf_gemv_fp16_fetch": ([ctypes.POINTER(_QWeight), _p, _i, _p, _p, _p, _p, _p, _p], _i),
     "sf_select_topk_act": ([_p, _i, _i, _p, _p, _p, _p], _i),
     "sf_act_prepare": ([_p, _i, _p, _p], _i),
     "sf_select_topk_act_many": ([_p, _i, _p], _i),
@@ -662,3 +665,39 @@ def rope_qk(q: torch.Tensor, k: torch.Tensor, pos: int, theta: float = 500000.0,
     _dev(q, "q")
     Hq, d = q.shape
     _check(_lib.sf_rope_qk(_ptr(q), Hq, _ptr(k), k.shape[0], d, pos, theta, _ptr(q_bf16), _stream(stream)))
+
+
+# ---- comparator modes ------------------------------------------------------------
+
+def select_random(K: int, k: int, seed: int, step: int, idx: torch.Tensor, n: torch.Tensor,
+                  stream: torch.cuda.Stream | None = None) -> None:
+    """``sf_select_random``: k of K channels from a counter-based draw."""
+    _dev(idx, "idx")
+    if idx.dtype != torch.int32 or idx.numel() < max(k, 1):
+        raise ValueError("idx must be int32 with room for k entries")
+    _check(_lib.sf_select_random(K, k, seed, step, _ptr(idx), _ptr(n), _stream(stream)))
+
+
+def quantize_residual(W: torch.Tensor, qw: QWeight, stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """``sf_quantize_residual``: fp16 [K][N] residuals of W against its resident values."""
+    _dev(W, "W")
+    out = torch.empty((qw.K, qw.N), dtype=torch.float16, device=W.device)
+    s = qw.c_struct()
+    _check(_lib.sf_quantize_residual(_ptr(W), ctypes.byref(s), _ptr(out), _stream(stream)))
+    return out
+
+
+def gemv_fp16_fetch(W: QWeight, x: torch.Tensor, idx: torch.Tensor, n: torch.Tensor, resid: torch.Tensor | None = None,
+                    cache: RefineCache | None = None, y: torch.Tensor | None = None,
+                    stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """``sf_gemv_fp16_fetch``: the FP16-fetch comparator GEMV (residual store or a cache of its columns)."""
+    _dev(x, "x")
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    B = x.shape[0]
+    if y is None:
+        y = torch.empty((B, W.N), dtype=torch.float32, device=x.device)
+    s = W.c_struct()
+    _check(_lib.sf_gemv_fp16_fetch(ctypes.byref(s), _ptr(x), B, _ptr(idx), _ptr(n), _ptr(resid),
+                                   cache.handle if cache is not None else None, _ptr(y), _stream(stream)))
+    return y

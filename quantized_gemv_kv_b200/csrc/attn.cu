@@ -125,7 +125,7 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
   for (int i = tid; i < GRP * kHistBins; i += kScThreads) hs[i] = 0;
   // the range's key scales and zeros: every load of this thread is issued
   // before the first store
-  float smx = 0.0f;
+  float smx = 0.0f, szx = 0.0f;
   {
     constexpr int kPer = kScMaxTok / kScThreads;
     uint32_t kzv[kPer];
@@ -139,12 +139,16 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
       const int i = tid + j * kScThreads;
       if (i < n) {
         ksz[i] = kzv[j];
-        smx = fmaxf(smx, sfd::half_bits_to_float(static_cast<uint16_t>(kzv[j] & 0xFFFFu)));
+        const float sv = sfd::half_bits_to_float(static_cast<uint16_t>(kzv[j] & 0xFFFFu));
+        const float zv = sfd::half_bits_to_float(static_cast<uint16_t>(kzv[j] >> 16));
+        smx = fmaxf(smx, sv);
+        szx = fmaxf(szx, __double2float_ru(static_cast<double>(sv) * fabs(1.5 - static_cast<double>(zv))));
       }
     }
   }
   // fixed-point query heads (warp h builds head h, 4 dims per lane) and the
-  // sums of q (any order: the error bound covers it)
+  // sums of q: exact in fp64 (the bf16 exponents span at most 33 binades
+  // where the result is used), then one rounding to fp32
   for (int h = warp; h < GRP; h += kScW) {
     float v[4];
     float am = 0.0f;
@@ -154,7 +158,10 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
       am = fmaxf(am, fabsf(v[i]));
     }
     am = warp_max(am);
-    const float qs_l = warp_sum((v[0] + v[1]) + (v[2] + v[3]));
+    double qs_d = (static_cast<double>(v[0]) + v[1]) + (static_cast<double>(v[2]) + v[3]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) qs_d += __shfl_xor_sync(0xffffffffu, qs_d, o);
+    const float qs_l = static_cast<float>(qs_d);
     int e = 0;
     if (am > 0.0f) frexpf(am, &e);
 #pragma unroll
@@ -259,7 +266,11 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
   }
   cp_async_wait_attn<0>();
   smx = warp_max(smx);
-  if (lane == 0) atomicMax(reinterpret_cast<unsigned int*>(smax + g), __float_as_uint(smx));
+  szx = warp_max(szx);
+  if (lane == 0) {
+    atomicMax(reinterpret_cast<unsigned int*>(smax + g), __float_as_uint(smx));
+    atomicMax(reinterpret_cast<unsigned int*>(smax + gridDim.y + g), __float_as_uint(szx));
+  }
   // lanes with the same tig hold the same heads
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -324,11 +335,12 @@ attn_select_compact_kernel(const uint16_t* __restrict__ q, int T, int k, const f
   __shared__ int scan_scratch[64];
   __shared__ int binfo[2];
   __shared__ double qd[D];
-  __shared__ double l1_sh;
+  __shared__ double l1_sh, dq_sh;
   __shared__ int qe_sh;
   __shared__ int base_sh;
-  select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status);
-  const double eps_s = select_eps(static_cast<double>(smax[g]), l1_sh, qe_sh, __uint_as_float(amaxu[h]), kScQFrac);
+  select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status, nullptr, kScQFrac, &dq_sh);
+  const double eps_s = select_eps_pipe(static_cast<double>(smax[g]), static_cast<double>(smax[gridDim.y / GRP + g]),
+                                       l1_sh, dq_sh, __uint_as_float(amaxu[h]));
   uint32_t b1;
   int kk;
   float f_low;
@@ -399,7 +411,7 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   __shared__ double qd[D];
   __shared__ int scan_scratch[64];
   __shared__ int binfo[2];
-  __shared__ double l1_sh;
+  __shared__ double l1_sh, dq_sh;
   __shared__ int qe_sh, span_sh;
   __shared__ int cnt_sh;  // read remotely
   __shared__ int cntA_sh, cntB_sh;  // outright selections and band candidates listed
@@ -416,7 +428,7 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
   const int cap = GRP * k;
 
   if (tid == 0) cntA_sh = cntB_sh = 0;
-  select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status, &span_sh);
+  select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status, &span_sh, kScQFrac, &dq_sh);
   // q as 24-bit fixed point X = q 2^(23 - qe): exact for every nonzero q
   // within 15 binades of the largest (bf16 has 8 significant bits)
   const bool int_keys = span_sh <= 15;
@@ -439,7 +451,8 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
       if (tid == 0) qxsum_sh = sx;
     }
   }
-  const double eps_s = select_eps(static_cast<double>(smax[g]), l1_sh, qe_sh, __uint_as_float(amaxu[h]), kScQFrac);
+  const double eps_s = select_eps_pipe(static_cast<double>(smax[g]), static_cast<double>(smax[gridDim.x / GRP + g]),
+                                       l1_sh, dq_sh, __uint_as_float(amaxu[h]));
   uint32_t b1;
   int kk;
   float f_low;

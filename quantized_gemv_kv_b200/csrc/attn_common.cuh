@@ -61,7 +61,7 @@ Layout make_layout(int Hq, int Hkv, int T, int k, int sms) {
   // split partials of the pipeline, or of the 16 CTAs of a cluster
   L.part = off; off = up256(off + sizeof(float) * Hq * static_cast<size_t>(std::max(L.splits, 16)) * (D + 2));
   L.fcnt = off; off = up256(off + sizeof(int32_t) * Hkv * 16);
-  L.smax = off; off = up256(off + sizeof(float) * Hkv);
+  L.smax = off; off = up256(off + sizeof(float) * 2 * Hkv);  // max key scale, then max s |1.5 - z|, per group
   L.status = off; off = up256(off + sizeof(int32_t) * std::max(Hkv, 4));
   L.count = off; off = up256(off + sizeof(int32_t) * Hkv);
   L.amax = off; off = up256(off + sizeof(uint32_t) * Hq);
@@ -203,8 +203,12 @@ __device__ void find_bin_from_top(const int* hist, int nb, int kk, int* out) {
 // Query-side setup of pass S (all threads call): q in fp64 into qd, its l1
 // norm and the binary exponent of max |q|; flags the KV group when the
 // nonzero q exponents span more than the exact-key precondition allows.
+// With dq_out, also the l1 norm of the fixed-point rounding of q with qfrac
+// fraction bits (sum_d |q_d - rint(q_d 2^(qfrac - e)) 2^(e - qfrac)|, each
+// term exact in fp64; the sum is rounded up by a relative 2^-44).
 __device__ void select_q_prologue(const uint16_t* __restrict__ q, int h, int g, double* qd, double* l1_out,
-                                  int* qe_out, int32_t* __restrict__ status, int* span_out = nullptr) {
+                                  int* qe_out, int32_t* __restrict__ status, int* span_out = nullptr,
+                                  int qfrac = 0, double* dq_out = nullptr) {
   const int tid = threadIdx.x;
   for (int d = tid; d < D; d += blockDim.x)
     qd[d] = static_cast<double>(sfd::bf16_bits_to_float(q[static_cast<size_t>(h) * D + d]));
@@ -227,6 +231,17 @@ __device__ void select_q_prologue(const uint16_t* __restrict__ q, int h, int g, 
       l1 += __shfl_xor_sync(0xffffffffu, l1, o);
       emin = min(emin, __shfl_xor_sync(0xffffffffu, emin, o));
       emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+    }
+    if (dq_out) {
+      const int e = emax >= emin ? emax : 0;
+      double dq = 0.0;
+      for (int d = tid; d < D; d += 32) {
+        const double v = qd[d];
+        dq += fabs(v - ldexp(rint(ldexp(v, qfrac - e)), e - qfrac));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dq += __shfl_xor_sync(0xffffffffu, dq, o);
+      if (tid == 0) *dq_out = dq * (1.0 + 0x1p-44);
     }
     if (tid == 0) {
       *l1_out = l1;
@@ -253,6 +268,25 @@ __device__ __forceinline__ double select_eps(double s_max, double l1, int qe, fl
   const double qround = ldexp(1.0, qe - qfrac - 1);
   const double eps_k = s_max * (4.0 * 3.0 * D * qround + l1 * (136.0 * u + 16.0 * gam));
   return 2.0 * (static_cast<double>(kInvSqrtD) * eps_k + 4.0 * u * static_cast<double>(amax));
+}
+
+// The same bound for the pipeline's score pass, from the actual rounding of
+// q rather than its worst case.  There q~ = X 2^(e - qfrac) (dq = q - q~,
+// dq1 = sum |dq|), P = sum_d c_d q~_d exactly, Q = fp32 of the exact sum of
+// q (one rounding), a = fl(1.5 - z), b = fl(a Q), E' = fl(4 P + b), score =
+// fl(fl(s E') c) with c the fp32 1/sqrt(d); the exact key is s E with E =
+// sum_d q_d (4 c_d + 1.5 - z).  Then
+//   |4 P - 4 sum c q| <= 12 dq1 (codes <= 3),
+//   |b - (1.5 - z) sum q| <= gamma_3 |1.5 - z| l1,
+//   the rounding of E' <= u (12 (l1 + dq1) + (1 + gamma_3) |1.5 - z| l1),
+//   the two last roundings <= gamma_2 / (1 - u)^2 |score| <= 2.0001 u amax,
+// so |score - c s E| <= c (s_max (12 (1 + u) dq1 + 12 u l1) + 4.0002 u
+// sz_max l1) + 2.0001 u amax, with s_max = max s and sz_max = max s |1.5 -
+// z| over the group's tokens; the result is rounded up by a relative 2^-40.
+__device__ __forceinline__ double select_eps_pipe(double s_max, double sz_max, double l1, double dq1, float amax) {
+  const double u = 5.9604644775390625e-8;  // 2^-24
+  const double inner = s_max * (12.0 * (1.0 + u) * dq1 + 12.0 * u * l1) + 4.0002 * u * sz_max * l1;
+  return (static_cast<double>(kInvSqrtD) * inner + 2.0001 * u * static_cast<double>(amax)) * (1.0 + 0x1p-40);
 }
 
 // Exact top-k of F[0..ncand) by (key desc, token asc): an 8-pass radix select

@@ -230,7 +230,42 @@ select_act_many_kernel(const __grid_constant__ SelManyArgs a) {
   __syncthreads();
   sfd::select_row_block(xs, flags, K, J.k, J.idx, J.n, J.act);
 }
+// ---- random selection (the comparator of the explainer's 既存手法との違い) -----
+// key_j = (splitmix64(seed + K step + j) >> 49) mod 32640 (Steele, Lea and
+// Flood's finalizer: a counter-based generator, so every channel's key is
+// drawn on its own), read as a finite positive bf16 magnitude; the k largest
+// keys (ties to the lower channel) are the selection.
+__device__ __forceinline__ uint64_t splitmix64(uint64_t z) {
+  z += 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+__global__ void __launch_bounds__(kThreads)
+select_random_kernel(int K, int k, uint64_t seed, uint64_t step, int32_t* __restrict__ idx, int32_t* __restrict__ n) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [K]
+  uint8_t* flags = smem + 2 * K;                     // [K]
+  const uint64_t base = seed + static_cast<uint64_t>(K) * step;
+  for (int j = threadIdx.x; j < K; j += kThreads)
+    xs[j] = static_cast<uint16_t>((splitmix64(base + static_cast<uint64_t>(j)) >> 49) % 0x7F80u);
+  __syncthreads();
+  sfd::select_row_block(xs, flags, K, k, idx, n, nullptr);
+}
+
 }  // namespace
+
+extern "C" sf_status sf_select_random(int K, int k, uint64_t seed, uint64_t step, int32_t* idx_out, int32_t* n_out,
+                                      sf_stream_t stream) {
+  SF_REQUIRE(idx_out && n_out, "sf_select_random: null pointer");
+  SF_REQUIRE(K >= 1 && K <= 32768 && k >= 0 && k <= K, "sf_select_random: need 1 <= K <= 32768, 0 <= k <= K");
+  const size_t smem = 3 * static_cast<size_t>(K);
+  SF_CHECK_CUDA(cudaFuncSetAttribute(select_random_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem)));
+  select_random_kernel<<<1, kThreads, smem, sf::as_cuda(stream)>>>(K, k, seed, step, idx_out, n_out);
+  return sf::check_launch("select_random_kernel");
+}
 
 extern "C" sf_status sf_select_topk(const uint16_t* x, int B, int K, int k, int32_t* idx_out, int32_t* n_out,
                                     sf_stream_t stream) {
