@@ -15,11 +15,10 @@
 //              candidates are re-scored exactly in fp64 (the key s*E with
 //              E = sum_d q_d (c_d 2^b_f + m_f - z) is exact in fp64 under a
 //              precondition on q checked here) and ranked by (key desc, token
-//              asc).  So the chosen set equals the exact definition.  Runs as
-//              a compaction over token chunks (from the histogram's bin of
-//              the k-th score) and a finish per KV group (one cluster, one CTA
-//              per query head), which also forms the group's union (ascending
-//              list and token bitmask).
+//              asc).  So the chosen set equals the exact definition.  One
+//              cluster per KV group, one CTA per query head, which also forms
+//              the group's union (ascending list and token bitmask) and runs
+//              step R on it.
 //   R  refine  per union token: its scores from the full 4-bit key codes,
 //              in place in the score buffer, and the largest per head.
 //   B  output  split over tokens: softmax over all tokens with the refined
@@ -101,6 +100,7 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
   __shared__ int qx[GRP][D];
   __shared__ float qsc[GRP], qsm[GRP];
   __shared__ uint32_t bfr[4 * ((2 * GRP + 7) / 8) * 2][32];  // B fragments of qx, per lane
+  pdl_launch_dependents();  // the listing pass may launch; it waits for this grid
   const int g = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g8 = lane >> 2, tig = lane & 3;
   const int t0 = blockIdx.x * tpc;
@@ -292,44 +292,26 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
   }
 }
 
-// ---- pass S, selection from the score histogram -----------------------------
+// ---- pass S, listing: the tokens of each head with fast score >= f_low ----------
 //
-// Pass A left, per query head, a histogram of its fast scores over the top 11
-// bits of the order-preserving key, and max |score|.  The bin b1 holding the
-// k-th largest score follows from the histogram alone.  Every token whose
-// exact key can reach the top k has a fast score >= tau - 2 eps >= (lower
-// edge of b1) - 2 eps, so:
-//  A  compact: per (4096-token chunk, head), the tokens with fast score >=
-//     lower(b1) - 2 eps, appended to the head's list (one atomic per chunk;
-//     the list's order does not matter);
-//  B  finish (one cluster per KV group, one CTA per query head): find tau
-//     exactly by two more radix passes over the listed scores of bin b1,
-//     keep the candidates >= tau - 2 eps, re-key them exactly in fp64 and
-//     rank them (key desc, token asc); then the group's CTAs build the union
-//     of their selections (bitmask and ascending list) through distributed
-//     shared memory.
-
-// Per-head threshold of the compaction and the histogram bin: all threads call.
-__device__ void select_band(const int32_t* __restrict__ hist_h, int k, double eps_s, int* hsh, int* scan_scratch,
-                            int* binfo, uint32_t* b1, int* kk, float* f_low) {
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hsh[i] = hist_h[i];
-  __syncthreads();
-  find_bin_from_top_block(hsh, kHistBins, k, binfo, scan_scratch);
-  *b1 = static_cast<uint32_t>(binfo[0]);
-  *kk = binfo[1];
-  const float lower = from_okey32(*b1 << kHistShift);
-  *f_low = __double2float_rd(static_cast<double>(lower) - 2.0 * eps_s);
-}
+// Per (8192-token chunk, query head), after the head's band from the score
+// pass's histogram and maxima (the bin b1 of the k-th largest fast score and
+// f_low = lower(b1) - 2 eps; the CTA of chunk 0 records it for the ranking):
+// a warp ballots 32 consecutive tokens a row; one atomic per CTA takes the
+// chunk's run of the head's list (the list's order does not matter: the
+// ranking orders by key and token).  The q terms of eps come first: they need
+// no earlier pass.
 
 constexpr int kCompThreads = 256;
+constexpr int kChunk = 8192;
+constexpr int kCompRows = kChunk / kCompThreads;  // rows of 32 tokens per warp
 
-template <int GRP>
 __global__ void __launch_bounds__(kCompThreads)
-attn_select_compact_kernel(const uint16_t* __restrict__ q, int T, int k, const float* __restrict__ score,
-                           const float* __restrict__ smax, const int32_t* __restrict__ hist,
-                           const uint32_t* __restrict__ amaxu, int32_t* __restrict__ cand,
-                           int32_t* __restrict__ ccnt, int32_t* __restrict__ status) {
-  const int chunk = blockIdx.x, h = blockIdx.y, g = h / GRP;
+attn_compact_kernel(const uint16_t* __restrict__ q, int T, int k, const float* __restrict__ score,
+                    const float* __restrict__ smax, const int32_t* __restrict__ hist,
+                    const uint32_t* __restrict__ amaxu, SelBand* __restrict__ band, int32_t* __restrict__ cand,
+                    int32_t* __restrict__ ccnt, int32_t* __restrict__ status, int grp) {
+  const int chunk = blockIdx.x, h = blockIdx.y, g = h / grp;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   __shared__ int hsh[kHistBins];
   __shared__ int scan_scratch[64];
@@ -337,98 +319,242 @@ attn_select_compact_kernel(const uint16_t* __restrict__ q, int T, int k, const f
   __shared__ double qd[D];
   __shared__ double l1_sh, dq_sh;
   __shared__ int qe_sh;
+  __shared__ int wcnt[kCompThreads / 32], woff[kCompThreads / 32];
   __shared__ int base_sh;
+  pdl_launch_dependents();
   select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status, nullptr, kScQFrac, &dq_sh);
-  const double eps_s = select_eps_pipe(static_cast<double>(smax[g]), static_cast<double>(smax[gridDim.y / GRP + g]),
-                                       l1_sh, dq_sh, __uint_as_float(amaxu[h]));
-  uint32_t b1;
-  int kk;
-  float f_low;
-  select_band(hist + static_cast<size_t>(h) * kHistBins, k, eps_s, hsh, scan_scratch, binfo, &b1, &kk, &f_low);
-  // warp w: tokens [chunk*4096 + 512 w, +512) as 16 rows of 32
-  constexpr int kRowsPerWarp = kChunk / (kCompThreads / 32) / 32;
-  const int t0 = chunk * kChunk + warp * 32 * kRowsPerWarp + lane;
-  const int tend = min(T, chunk * kChunk + (warp + 1) * 32 * kRowsPerWarp);
+  pdl_wait();  // the score pass's scores, histogram and maxima
+  // the head's histogram, every load in flight
+  {
+    constexpr int kPer = kHistBins / kCompThreads;
+    const int32_t* hg = hist + static_cast<size_t>(h) * kHistBins;
+    int hv[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) hv[j] = hg[tid + j * kCompThreads];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) hsh[tid + j * kCompThreads] = hv[j];
+  }
+  // the chunk's scores are loaded while the band is found
+  const int t0 = chunk * kChunk + warp * 32 * kCompRows + lane;
   const float* sc = score + static_cast<size_t>(h) * T;
-  bool p[kRowsPerWarp];
+  float v[kCompRows];
+#pragma unroll
+  for (int i = 0; i < kCompRows; ++i) {
+    const int t = t0 + 32 * i;
+    v[i] = t < T ? sc[t] : 0.0f;
+  }
+  const int Hkv = gridDim.y / grp;
+  const double eps_s = select_eps_pipe(static_cast<double>(smax[g]), static_cast<double>(smax[Hkv + g]), l1_sh,
+                                       dq_sh, __uint_as_float(amaxu[h]));
+  __syncthreads();
+  find_bin_from_top_block(hsh, kHistBins, k, binfo, scan_scratch);
+  const uint32_t b1 = static_cast<uint32_t>(binfo[0]);
+  const float f_low = __double2float_rd(static_cast<double>(from_okey32(b1 << kHistShift)) - 2.0 * eps_s);
+  if (chunk == 0 && tid == 0) band[h] = SelBand{eps_s, f_low, b1, binfo[1], 0};
+  bool p[kCompRows];
   int cnt = 0;
 #pragma unroll
-  for (int i = 0; i < kRowsPerWarp; ++i) {
-    const int t = t0 + 32 * i;
-    p[i] = t < tend && sc[t] >= f_low;
+  for (int i = 0; i < kCompRows; ++i) {
+    p[i] = t0 + 32 * i < T && v[i] >= f_low;
     cnt += __popc(__ballot_sync(0xffffffffu, p[i]));
   }
-  if (lane == 0) scan_scratch[warp] = cnt;
+  if (lane == 0) wcnt[warp] = cnt;
   __syncthreads();
-  if (warp == 0) {
-    const int v = lane < kCompThreads / 32 ? scan_scratch[lane] : 0;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
+  if (tid == 0) {
+    int a = 0;
+    for (int w = 0; w < kCompThreads / 32; ++w) {
+      woff[w] = a;
+      a += wcnt[w];
     }
-    if (lane < kCompThreads / 32) scan_scratch[32 + lane] = incl - v;
-    // the chunk's run of the head's list (the list's order does not matter:
-    // the finish ranks by key and token)
-    if (lane == 31) base_sh = incl ? atomicAdd(ccnt + h, incl) : 0;
+    base_sh = a ? atomicAdd(ccnt + h, a) : 0;
   }
   __syncthreads();
   int32_t* out = cand + static_cast<size_t>(h) * T + base_sh;
-  int o = scan_scratch[32 + warp];
+  int o = woff[warp];
   const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int i = 0; i < kRowsPerWarp; ++i) {
+  for (int i = 0; i < kCompRows; ++i) {
     const unsigned bal = __ballot_sync(0xffffffffu, p[i]);
     if (p[i]) out[o + __popc(bal & lt)] = t0 + 32 * i;
     o += __popc(bal);
   }
 }
 
-constexpr int kFinThreads = 512;
-constexpr int kFinKeys = 2048;     // candidates ranked pairwise from shared memory
-constexpr int kFinList = 4096;     // listed (token, score) pairs cached in shared memory
-constexpr size_t kFinDynSmem = static_cast<size_t>(kFinList) * 8 + static_cast<size_t>(kFinKeys) * 4;
+// ---- refined scores of the union --------------------------------------------------
+//
+// Step R, at the start of pass B: every union token of a CTA's range gets its
+// scores for the group's query heads recomputed from the full 4-bit key
+// codes, in place in the score buffer.  The CTA then weights its tokens
+// against one maximum per head (the larger of its refined maximum and a
+// bound on the resident scores outside the union), so it needs no maximum
+// pass; the merge rescales the ranges' partials.  A thread handles one union
+// token for all the heads of the group: one load of each of the token's two
+// code rows.
+
+// A unit of a KV refinement cache: the token-head's 8 K refinement words,
+// then its 8 V refinement words.
+constexpr int kCacheUnitWords = 2 * kWordsPerRow;
+
+// The V refinement words of K/V row `row`: from the store (uslot == nullptr)
+// or from the cache slot that holds the row's unit.
+__device__ __forceinline__ const uint32_t* vref_row(const uint32_t* v_ref, const int32_t* uslot, size_t row) {
+  return uslot != nullptr ? v_ref + static_cast<size_t>(uslot[row]) * kCacheUnitWords + kWordsPerRow
+                          : v_ref + row * kWordsPerRow;
+}
+
+// Refines union token t of group g (row = g S + t).  Returns false when its
+// refinement bits are not on the device (a cache slot < 0): the token keeps
+// its resident key and value this step and leaves the refined set, and its
+// resident scores still bound the weights' maximum.  mk[h] takes the max of
+// the token's (refined or resident) score keys.
+template <int GRP>
+__device__ __forceinline__ bool refine_token(const uint32_t* __restrict__ k_res, const uint32_t* __restrict__ k_ref,
+                                             const int32_t* __restrict__ uslot, const uint16_t* __restrict__ k_scale,
+                                             const uint16_t* __restrict__ k_zero, int T, size_t rowg, int g, int t,
+                                             const float (&qs)[GRP][D], const float (&qsum)[GRP],
+                                             float* __restrict__ score, uint32_t (&mk)[GRP]) {
+  const size_t row = rowg + t;
+  const int slot = uslot != nullptr ? uslot[row] : 0;
+  float* srow = score + static_cast<size_t>(g) * GRP * T + t;  // head h at srow[h T]
+  if (slot < 0) {
+#pragma unroll
+    for (int h = 0; h < GRP; ++h) mk[h] = max(mk[h], okey32(srow[static_cast<size_t>(h) * T]));
+    return false;
+  }
+  const uint4* pr = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
+  const uint4* pf = reinterpret_cast<const uint4*>(
+      uslot != nullptr ? k_ref + static_cast<size_t>(slot) * kCacheUnitWords : k_ref + row * kWordsPerRow);
+  const uint4 r0 = pr[0], r1 = pr[1], f0 = pf[0], f1 = pf[1];  // both rows in flight at once
+  const float sv = sfd::half_bits_to_float(k_scale[row]);
+  const float z = sfd::half_bits_to_float(k_zero[row]);
+  uint32_t wr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+  uint32_t wf[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+  float P[GRP];
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) P[h] = 0.0f;
+  // one word per iteration, the words shifted down (static register indices)
+#pragma unroll 1
+  for (int w = 0; w < 8; ++w) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float c = static_cast<float>(((wr[0] >> (2 * j)) & 3u) * 4u + ((wf[0] >> (2 * j)) & 3u));
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) P[h] = fmaf(qs[h][16 * w + j], c, P[h]);
+    }
+#pragma unroll
+    for (int i = 0; i < 7; ++i) {
+      wr[i] = wr[i + 1];
+      wf[i] = wf[i + 1];
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    const float val = (sv * fmaf(-z, qsum[h], P[h])) * kInvSqrtD;
+    mk[h] = max(mk[h], okey32(val));
+    srow[static_cast<size_t>(h) * T] = val;
+  }
+  return true;
+}
+
+// ---- pass S, ranking: one cluster per KV group, one CTA per query head ----------
+//
+// The score pass left, per query head, its selection band (the histogram bin
+// b1 of the k-th largest fast score and a lower bound f_low of every fast
+// score that can reach the top k) and the listing pass the head's tokens with
+// fast score >= f_low.  Every token whose exact key can reach the top k has a
+// fast score >= tau - 2 eps >= f_low.  Per head:
+//  1  the list and its scores into shared memory (beyond kSelList: read in
+//     place);
+//  2  tau exactly by two more radix passes over the listed scores of b1;
+//  3  the tokens above tau + 2 eps selected outright; the band [tau - 2 eps,
+//     tau + 2 eps] re-keyed exactly in fp64 and ranked (key desc, token asc);
+//  4  the selection marked in the group's token bitmask, whose words are
+//     spread over the cluster's shared memory, then the union listed in
+//     ascending order (CTA r the words of its range) and the bitmask written
+//     for pass B.
+
+constexpr int kSelThreads = 512;
+constexpr int kSelKeys = 2048;      // band entries ranked pairwise in shared memory
+constexpr int kSelList = 4096;      // listed (token, score) pairs in shared memory
+constexpr int kSelMaxWords = 8192;  // bitmask words per CTA held in shared memory (beyond: global atomics)
+
+__host__ __device__ constexpr size_t sel_dyn_smem(int words_sm) {
+  return static_cast<size_t>(kSelList) * 8 + static_cast<size_t>(kSelKeys) * 4 + static_cast<size_t>(words_sm) * 4;
+}
 
 template <int GRP>
-__global__ void __launch_bounds__(kFinThreads)
-attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
-                          const uint32_t* __restrict__ k_ref, const uint16_t* __restrict__ k_scale,
-                          const uint16_t* __restrict__ k_zero, int T, int k, int S, float* __restrict__ score,
-                          const float* __restrict__ smax, const int32_t* __restrict__ hist,
-                          const uint32_t* __restrict__ amaxu, const int32_t* __restrict__ cand,
-                          const int32_t* __restrict__ ccnt, int32_t* __restrict__ list, double* __restrict__ kap,
-                          int32_t* __restrict__ sel_head, uint32_t* __restrict__ umask, int words_t,
-                          int32_t* __restrict__ sel_out, int32_t* __restrict__ sel_n, int32_t* __restrict__ status,
-                          uint32_t* __restrict__ mkey) {
+__global__ void __launch_bounds__(kSelThreads)
+attn_select_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
+                   const uint16_t* __restrict__ k_scale, const uint16_t* __restrict__ k_zero, int T, int k, int S,
+                   const float* __restrict__ score, const SelBand* __restrict__ band, const int32_t* __restrict__ cand,
+                   const int32_t* __restrict__ ccnt, int32_t* __restrict__ list, double* __restrict__ kap,
+                   int32_t* __restrict__ sel_head, uint32_t* __restrict__ umask, int words_t, int wper, int dsm,
+                   int32_t* __restrict__ sel_out, int32_t* __restrict__ sel_n, int32_t* __restrict__ status,
+                   uint32_t* __restrict__ mkey) {
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
   const int rank = static_cast<int>(cl.block_rank());
   const int h = blockIdx.x, g = h / GRP;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
   __shared__ int hr[2048];
-  __shared__ unsigned long long keys[kFinKeys];  // order-preserving exact keys, sorted with the tokens
+  __shared__ unsigned long long keys[kSelKeys];  // order-preserving exact keys, sorted with the tokens
   __shared__ double qd[D];
   __shared__ int scan_scratch[64];
   __shared__ int binfo[2];
-  __shared__ double l1_sh, dq_sh;
+  __shared__ double l1_sh;
   __shared__ int qe_sh, span_sh;
   __shared__ int cnt_sh;  // read remotely
-  __shared__ int cntA_sh, cntB_sh;  // outright selections and band candidates listed
+  __shared__ int cntA_sh, cntB_sh;  // outright selections and band candidates
   __shared__ uint32_t qpl[3][8][4];  // byte planes of the fixed-point q, in code-extraction order
   __shared__ long long qxsum_sh;
-  extern __shared__ int fin_dyn[];
-  int* ltok = fin_dyn;                                      // [kFinList]
-  float* lsc = reinterpret_cast<float*>(fin_dyn + kFinList);  // [kFinList]
-  int* ktok = fin_dyn + 2 * kFinList;                       // [kFinKeys] tokens of the sorted keys
+  extern __shared__ __align__(16) int sel_dyn[];
+  int* ltok = sel_dyn;                                       // [kSelList]
+  float* lsc = reinterpret_cast<float*>(sel_dyn + kSelList);  // [kSelList]
+  int* ktok = sel_dyn + 2 * kSelList;                        // [kSelKeys] tokens of the sorted keys
+  uint32_t* wsm = reinterpret_cast<uint32_t*>(ktok + kSelKeys);  // [wper] bitmask words of this CTA's range
   const float* sc = score + static_cast<size_t>(h) * T;
-  const int32_t* L = cand + static_cast<size_t>(h) * T;  // the compaction's list
-  int32_t* F = list + static_cast<size_t>(h) * T;        // band candidates
+  const int32_t* Lg = cand + static_cast<size_t>(h) * T;  // the listing pass's tokens
+  int32_t* F = list + static_cast<size_t>(h) * T;         // band candidates beyond kSelKeys
   double* kp = kap + static_cast<size_t>(h) * T;
+  uint32_t* um_g = umask + static_cast<size_t>(g) * words_t;
   const int cap = GRP * k;
+  const int w0 = min(words_t, rank * wper), w1 = min(words_t, w0 + wper);
 
   if (tid == 0) cntA_sh = cntB_sh = 0;
-  select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status, &span_sh, kScQFrac, &dq_sh);
+  if (dsm)
+    for (int w = tid; w < wper; w += kSelThreads) wsm[w] = 0u;
+  select_q_prologue(q, h, g, qd, &l1_sh, &qe_sh, status, &span_sh);  // contains __syncthreads
+  pdl_wait();  // the listing pass, and through it the score pass
+  const SelBand bd = band[h];
+  const double eps_s = bd.eps;
+  int kk = bd.kk;
+  const int m = min(ccnt[h], T);
+  // 1. the list with its fast scores: each thread's tokens, then their
+  //    scores, every load of a round in flight
+  {
+    constexpr int kPer = kSelList / kSelThreads;
+    const int mm = min(m, kSelList);
+    int tv[kPer];
+    float sv[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int e = tid + j * kSelThreads;
+      tv[j] = e < mm ? Lg[e] : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int e = tid + j * kSelThreads;
+      sv[j] = e < mm ? sc[tv[j]] : 0.0f;
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int e = tid + j * kSelThreads;
+      if (e < mm) {
+        ltok[e] = tv[j];
+        lsc[e] = sv[j];
+      }
+    }
+  }
   // q as 24-bit fixed point X = q 2^(23 - qe): exact for every nonzero q
   // within 15 binades of the largest (bf16 has 8 significant bits)
   const bool int_keys = span_sh <= 15;
@@ -443,45 +569,29 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
       }
       qpl[p][wi][kq] = v;
     }
-    if (tid < 32) {
+    if (tid >= 96 && tid < 128) {
       long long sx = 0;
-      for (int d = tid; d < D; d += 32) sx += static_cast<long long>(ldexp(qd[d], 23 - qe_sh));
+      for (int d = tid - 96; d < D; d += 32) sx += static_cast<long long>(ldexp(qd[d], 23 - qe_sh));
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, o);
-      if (tid == 0) qxsum_sh = sx;
+      if (tid == 96) qxsum_sh = sx;
     }
   }
-  const double eps_s = select_eps_pipe(static_cast<double>(smax[g]), static_cast<double>(smax[gridDim.x / GRP + g]),
-                                       l1_sh, dq_sh, __uint_as_float(amaxu[h]));
-  uint32_t b1;
-  int kk;
-  float f_low;
-  select_band(hist + static_cast<size_t>(h) * kHistBins, k, eps_s, hr, scan_scratch, binfo, &b1, &kk, &f_low);
-
-  // 1. the compaction's list, with its fast scores in shared memory when it fits
-  const int m = min(ccnt[h], T);
-  if (m <= kFinList) {
-    for (int e = tid; e < m; e += kFinThreads) {
-      const int t = L[e];
-      ltok[e] = t;
-      lsc[e] = sc[t];
-    }
-  }
-  __syncthreads();
-  const bool cached = m <= kFinList;
-  auto tok_of = [&](int e) { return cached ? ltok[e] : L[e]; };
-  auto score_of = [&](int e) { return cached ? lsc[e] : sc[L[e]]; };
+  cl.sync();  // 0: every CTA's bitmask words are cleared before any remote update
+  auto tok_of = [&](int e) { return e < kSelList ? ltok[e] : Lg[e]; };
+  auto score_of = [&](int e) { return e < kSelList ? lsc[e] : sc[Lg[e]]; };
+  const unsigned lt = (1u << lane) - 1u;
 
   // 2. tau: two radix passes (11 + 10 bits) over the listed scores of bin b1
-  uint32_t pre = b1 << kHistShift;
+  uint32_t pre = bd.b1 << kHistShift;
   static_assert(kHistShift == 21, "the two passes cover the 21 key bits below the histogram's");
   for (int pass = 0; pass < 2; ++pass) {
     const int shift = pass == 0 ? 10 : 0;
     const int nb = pass == 0 ? 2048 : 1024;
-    for (int i = tid; i < nb; i += kFinThreads) hr[i] = 0;
+    for (int i = tid; i < nb; i += kSelThreads) hr[i] = 0;
     __syncthreads();
     const uint32_t pmask = pass == 0 ? 0xFFE00000u : 0xFFFFFC00u;
-    for (int e = tid; e < m; e += kFinThreads) {
+    for (int e = tid; e < m; e += kSelThreads) {
       const uint32_t key = okey32(score_of(e));
       if ((key & pmask) == pre) atomicAdd(&hr[(key >> shift) & static_cast<uint32_t>(nb - 1)], 1);
     }
@@ -500,49 +610,58 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
     mkey[h] = min(mkey[h], b);
   }
 
+  // the group's token bitmask: words [r wper, (r + 1) wper) in CTA r's shared
+  // memory, or the global words
+  auto mark = [&](int t) {
+    const int w = t >> 5;
+    const uint32_t bit = 1u << (t & 31);
+    if (dsm) {
+      const int r = w / wper;
+      atomicOr(cl.map_shared_rank(wsm, r) + (w - r * wper), bit);
+    } else {
+      atomicOr(um_g + w, bit);
+    }
+  };
+
   // 3. a token whose fast score exceeds tau + 2 eps outranks, by exact key,
   //    every token with fast score <= tau, so fewer than k tokens can rank
   //    above it: it is selected outright.  Only the band [tau - 2 eps,
-  //    tau + 2 eps] is re-keyed and ranked (its candidates in token order).
+  //    tau + 2 eps] is re-keyed and ranked.
   int32_t* sel = sel_head + static_cast<size_t>(h) * k;
-  uint32_t* um = umask + static_cast<size_t>(g) * words_t;
   const double hi_band = static_cast<double>(tau) + 2.0 * eps_s;
-  // listed in any order (the ranking orders by key and token): a warp takes
-  // its slots with one shared atomic per list
-  {
-    const int lane = tid & 31;
-    const unsigned lt = (1u << lane) - 1u;
-    for (int base = 0; base < m; base += kFinThreads) {
-      const int e = base + tid;
-      const float sv_e = e < m ? score_of(e) : 0.0f;
-      const bool inA = e < m && static_cast<double>(sv_e) > hi_band;
-      const bool inB = e < m && !inA && sv_e >= fthr;
-      const int t = e < m ? tok_of(e) : 0;
-      const unsigned bA = __ballot_sync(0xffffffffu, inA), bB = __ballot_sync(0xffffffffu, inB);
-      int oA = 0, oB = 0;
-      if (lane == 0) {
-        if (bA) oA = atomicAdd(&cntA_sh, __popc(bA));
-        if (bB) oB = atomicAdd(&cntB_sh, __popc(bB));
-      }
-      oA = __shfl_sync(0xffffffffu, oA, 0);
-      oB = __shfl_sync(0xffffffffu, oB, 0);
-      const int pA = oA + __popc(bA & lt);
-      if (inA && pA < k) {  // fewer than k by the bound; guarded against corrupt scores
-        sel[pA] = t;
-        atomicOr(um + (t >> 5), 1u << (t & 31));
-      }
-      if (inB) F[oB + __popc(bB & lt)] = t;
+  for (int base = 0; base < m; base += kSelThreads) {  // uniform over the block
+    const int e = base + tid;
+    const float sv_e = e < m ? score_of(e) : 0.0f;
+    const bool inA = e < m && static_cast<double>(sv_e) > hi_band;
+    const bool inB = e < m && !inA && sv_e >= fthr;
+    const int t = e < m ? tok_of(e) : 0;
+    const unsigned bA = __ballot_sync(0xffffffffu, inA), bB = __ballot_sync(0xffffffffu, inB);
+    int oA = 0, oB = 0;
+    if (lane == 0) {
+      if (bA) oA = atomicAdd(&cntA_sh, __popc(bA));
+      if (bB) oB = atomicAdd(&cntB_sh, __popc(bB));
+    }
+    oA = __shfl_sync(0xffffffffu, oA, 0);
+    oB = __shfl_sync(0xffffffffu, oB, 0);
+    const int pA = oA + __popc(bA & lt);
+    if (inA && pA < k) {  // fewer than k by the bound; guarded against corrupt scores
+      sel[pA] = t;
+      mark(t);
+    }
+    if (inB) {
+      const int pB = oB + __popc(bB & lt);
+      if (pB < kSelKeys) ktok[pB] = t;
+      F[pB] = t;
     }
   }
   __syncthreads();
   const int nA = cntA_sh, ncand = cntB_sh;
   const int kB = max(0, k - nA);  // winners still to pick from the band (>= 1 by the bound)
 
-
-  // 4. exact keys (four partial sums: exact under the precondition, so the
-  //    order does not change the key)
-  for (int i = tid; i < ncand; i += kFinThreads) {
-    const int t = F[i];
+  // 4. exact keys (exact under the precondition, so the summation order does
+  //    not change the key)
+  for (int i = tid; i < ncand; i += kSelThreads) {
+    const int t = i < kSelKeys ? ktok[i] : F[i];
     const size_t row = static_cast<size_t>(g) * S + t;
     const uint4* w4 = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
     const uint4 x0 = w4[0], x1 = w4[1];
@@ -566,8 +685,8 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
         }
       const long long P = static_cast<long long>(d0) + 256ll * d1 + 65536ll * d2;
       const double cq = ldexp(static_cast<double>(P), qe_sh - 23);
-      const double qsum = ldexp(static_cast<double>(qxsum_sh), qe_sh - 23);
-      key = sv * fma(1.5 - z, qsum, 4.0 * cq);
+      const double qsm = ldexp(static_cast<double>(qxsum_sh), qe_sh - 23);
+      key = sv * fma(1.5 - z, qsm, 4.0 * cq);
     } else {
       double E[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
@@ -585,28 +704,25 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
       key = sv * ((E[0] + E[1]) + (E[2] + E[3]));
     }
     kp[i] = key;
-    if (ncand <= kFinKeys) {
-      keys[i] = okey64(key);
-      ktok[i] = t;
-    }
+    if (i < kSelKeys) keys[i] = okey64(key);
   }
   __syncthreads();
 
-  // 5. rank the band by (key desc, token asc); its kB winners go to
-  //    sel_head after the outright ones, and into the group's token bitmask
-  if (ncand <= kFinKeys) {
+  // rank the band by (key desc, token asc); its kB winners go to sel_head
+  // after the outright ones, and into the bitmask
+  if (ncand <= kSelKeys) {
     // bitonic sort of (key desc, token asc) over a power-of-two size,
-    // padding with entries that order last; the first k are the selection
+    // padding with entries that order last; the first kB are the winners
     int n2 = 1;
     while (n2 < ncand) n2 <<= 1;
-    for (int i = ncand + tid; i < n2; i += kFinThreads) {
+    for (int i = ncand + tid; i < n2; i += kSelThreads) {
       keys[i] = 0ull;
       ktok[i] = 0x7FFFFFFF;
     }
     __syncthreads();
     for (int size = 2; size <= n2; size <<= 1)
       for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int i = tid; i < (n2 >> 1); i += kFinThreads) {
+        for (int i = tid; i < (n2 >> 1); i += kSelThreads) {
           const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
           const unsigned long long ka = keys[lo], kb = keys[hi];
           const int ta = ktok[lo], tb = ktok[hi];
@@ -620,146 +736,56 @@ attn_select_finish_kernel(const uint16_t* __restrict__ q, const uint32_t* __rest
         }
         __syncthreads();
       }
-    for (int r = tid; r < kB; r += kFinThreads) {
+    for (int r = tid; r < kB; r += kSelThreads) {
       const int t = ktok[r];
       sel[nA + r] = t;
-      atomicOr(um + (t >> 5), 1u << (t & 31));
+      mark(t);
     }
   } else {
     select_rank_radix(F, ncand, kp, kB, hr, scan_scratch, binfo, sel + nA);
     __syncthreads();
-    for (int i = tid; i < kB; i += kFinThreads) {
-      const int t = sel[nA + i];
-      atomicOr(um + (t >> 5), 1u << (t & 31));
-    }
+    for (int i = tid; i < kB; i += kSelThreads) mark(sel[nA + i]);
   }
-  __threadfence();
+  if (!dsm) __threadfence();
+  pdl_launch_dependents();  // pass B's CTAs may start their prologue during the union
   cl.sync();  // 1: the group's bitmask is complete
 
-  // 6. union, ascending: CTA r of the cluster compacts words [r wper, (r+1) wper)
-  const int wper = (words_t + GRP - 1) / GRP;
-  const int w0 = min(words_t, rank * wper), w1 = min(words_t, w0 + wper);
+  // 5. union, ascending: CTA r lists the tokens of words [w0, w1)
+  auto word = [&](int w) -> uint32_t { return dsm ? wsm[w - w0] : __ldcg(um_g + w); };
+  int32_t* uout = sel_out + static_cast<size_t>(g) * cap;
   {
-    const int chunk = (w1 - w0 + kFinThreads - 1) / kFinThreads;
+    int off = 0, uloc = 0;
+    const int chunk = (w1 - w0 + kSelThreads - 1) / kSelThreads;
     const int a0 = min(w1, w0 + tid * chunk), a1 = min(w1, a0 + chunk);
     int c = 0;
-    for (int w = a0; w < a1; ++w) c += __popc(um[w]);
-    int tot;
-    int pos = sfd::block_exclusive_scan(c, scan_scratch, &tot);
-    if (tid == 0) cnt_sh = tot;
+    for (int w = a0; w < a1; ++w) c += __popc(word(w));
+    int pos = sfd::block_exclusive_scan(c, scan_scratch, &uloc);
+    if (tid == 0) cnt_sh = uloc;
     cl.sync();  // 2: every CTA's count is published
-    int off = 0, U = 0;
+    int U = 0;
     for (int r = 0; r < GRP; ++r) {
       const int cr = *cl.map_shared_rank(&cnt_sh, r);
       if (r < rank) off += cr;
       U += cr;
     }
-    int32_t* out = sel_out + static_cast<size_t>(g) * cap;
-    pos += off;
+    cl.barrier_arrive();  // 3 (arrive): no remote shared-memory access by this CTA after this
     for (int w = a0; w < a1; ++w) {
-      uint32_t bits = um[w];
+      uint32_t bits = word(w);
       while (bits) {
         const int b = __ffs(bits) - 1;
         bits &= bits - 1u;
-        out[pos++] = 32 * w + b;
+        const int t = 32 * w + b;
+        uout[off + pos] = t;
+        ++pos;
       }
     }
     if (rank == 0 && tid == 0) sel_n[g] = status[g] ? -1 - U : U;
   }
-  cl.sync();  // 3: no shared-memory access across CTAs after this
-}
-
-// ---- refined scores of the union --------------------------------------------------
-//
-// Step R, between the selection and pass B: every token of a group's union
-// gets its
-// scores for the group's query heads recomputed from the full 4-bit key codes,
-// in place in the score buffer, and the largest refined score per head is
-// recorded as an order-preserving key.  Pass B then weights every token
-// against one fixed maximum per head (the larger of the refined maximum and a
-// bound on the resident scores outside the union), so it needs no maximum
-// pass and no rescaling.  A thread handles one union token for all the heads
-// of the group: one load of the list, one of the token's two code rows.
-
-constexpr int kRefThreads = 256;
-// A unit of a KV refinement cache: the token-head's 8 K refinement words,
-// then its 8 V refinement words.
-constexpr int kCacheUnitWords = 2 * kWordsPerRow;
-
-// The V refinement words of K/V row `row`: from the store (uslot == nullptr)
-// or from the cache slot that holds the row's unit.
-__device__ __forceinline__ const uint32_t* vref_row(const uint32_t* v_ref, const int32_t* uslot, size_t row) {
-  return uslot != nullptr ? v_ref + static_cast<size_t>(uslot[row]) * kCacheUnitWords + kWordsPerRow
-                          : v_ref + row * kWordsPerRow;
-}
-
-template <int GRP>
-__global__ void __launch_bounds__(kRefThreads, 2)
-attn_refine_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
-                   const uint32_t* __restrict__ k_ref, const int32_t* __restrict__ uslot,
-                   const uint16_t* __restrict__ k_scale, const uint16_t* __restrict__ k_zero, int T, int S, int cap,
-                   const int32_t* __restrict__ sel_out, const int32_t* __restrict__ sel_n, float* __restrict__ score,
-                   uint32_t* __restrict__ rkey, uint32_t* __restrict__ umask, int words_t) {
-  __shared__ float qs[GRP][D];
-  __shared__ float qsum[GRP];
-  const int g = blockIdx.y;
-  const int lane = threadIdx.x & 31;
-  load_q<GRP>(q, g, qs, qsum);  // contains __syncthreads
-  const int sn = sel_n[g];
-  const int U = min(cap, sn >= 0 ? sn : -1 - sn);
-  const int32_t* list = sel_out + static_cast<size_t>(g) * cap;
-  const size_t rowg = static_cast<size_t>(g) * S;  // K rows: the cache's stride
-  uint32_t mk[GRP];
-#pragma unroll
-  for (int h = 0; h < GRP; ++h) mk[h] = 0u;
-  for (int u0 = blockIdx.x * kRefThreads; u0 < U; u0 += gridDim.x * kRefThreads) {  // uniform over the block
-    const int u = u0 + static_cast<int>(threadIdx.x);
-    const int t = u < U ? list[u] : 0;
-    const size_t row = rowg + t;
-    const int slot = (u < U && uslot != nullptr) ? uslot[row] : 0;
-    if (u < U && slot < 0) {
-      // refinement bits not on the device (a cache miss): the token keeps its
-      // resident key and value this step; it leaves the refined set, and its
-      // resident scores still bound the weights' maximum
-      atomicAnd(umask + static_cast<size_t>(g) * words_t + (t >> 5), ~(1u << (t & 31)));
-#pragma unroll
-      for (int h = 0; h < GRP; ++h)
-        mk[h] = max(mk[h], okey32(score[(static_cast<size_t>(g) * GRP + h) * T + t]));
-    } else if (u < U) {
-      const uint4* pr = reinterpret_cast<const uint4*>(k_res + row * kWordsPerRow);
-      const uint4* pf = reinterpret_cast<const uint4*>(
-          uslot != nullptr ? k_ref + static_cast<size_t>(slot) * kCacheUnitWords : k_ref + row * kWordsPerRow);
-      const uint4 r0 = pr[0], r1 = pr[1], f0 = pf[0], f1 = pf[1];
-      const float sv = sfd::half_bits_to_float(k_scale[row]);
-      const float z = sfd::half_bits_to_float(k_zero[row]);
-      const uint32_t wr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-      const uint32_t wf[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-      float P[GRP];
-#pragma unroll
-      for (int h = 0; h < GRP; ++h) P[h] = 0.0f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float c = static_cast<float>(((wr[w] >> (2 * j)) & 3u) * 4u + ((wf[w] >> (2 * j)) & 3u));
-#pragma unroll
-          for (int h = 0; h < GRP; ++h) P[h] = fmaf(qs[h][16 * w + j], c, P[h]);
-        }
-      }
-#pragma unroll
-      for (int h = 0; h < GRP; ++h) {
-        const float val = (sv * fmaf(-z, qsum[h], P[h])) * kInvSqrtD;
-        mk[h] = max(mk[h], okey32(val));
-        score[(static_cast<size_t>(g) * GRP + h) * T + t] = val;
-      }
-    }
+  if (dsm) {
+    __syncthreads();
+    for (int w = w0 + tid; w < w1; w += kSelThreads) um_g[w] = wsm[w - w0];
   }
-#pragma unroll
-  for (int h = 0; h < GRP; ++h) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mk[h] = max(mk[h], __shfl_xor_sync(0xffffffffu, mk[h], o));
-    if (lane == 0 && mk[h]) atomicMax(rkey + g * GRP + h, mk[h]);
-  }
+  cl.barrier_wait();  // 3 (wait): no CTA leaves while another may read its count
 }
 
 // ---- pass B on the tensor cores ------------------------------------------------
@@ -788,6 +814,8 @@ constexpr int kOutThreads = 256;
 constexpr int kOW = kOutThreads / 32;
 constexpr int kRing = 6;           // cp.async stages per warp
 constexpr int kUCap = 384;         // refined rows per sub-chunk staged in shared memory
+constexpr int kUMiss = 0x8000;     // union-list flag: refinement bits not on the device
+constexpr int kUOff = 0x7FFF;      // union-list offset bits
 
 template <int GRP>
 struct OutCfg {
@@ -807,12 +835,14 @@ struct OutCfg {
 };
 
 template <int GRP>
-__global__ void __launch_bounds__(kOutThreads)
-attn_out_kernel(const uint32_t* __restrict__ v_res,
+__global__ void __launch_bounds__(kOutThreads, GRP >= 8 ? 1 : 2)
+attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_res,
+                const uint32_t* __restrict__ k_ref, const uint16_t* __restrict__ k_scale,
+                const uint16_t* __restrict__ k_zero, const uint32_t* __restrict__ v_res,
                 const uint32_t* __restrict__ v_ref, const int32_t* __restrict__ uslot,
                 const uint16_t* __restrict__ v_scale,
                 const uint16_t* __restrict__ v_zero, int T, int S, int tps, int words_t, int splits,
-                const float* __restrict__ score, const uint32_t* __restrict__ mkey, const uint32_t* __restrict__ rkey,
+                float* __restrict__ score, const uint32_t* __restrict__ mkey,
                 const uint32_t* __restrict__ umask, float* __restrict__ part, int32_t* __restrict__ done,
                 float* __restrict__ out) {
   using C = OutCfg<GRP>;
@@ -825,8 +855,12 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
                                               C::ulist_bytes);  // [kUCap][8] refinement rows of listed tokens
   __shared__ float red2[kOW][3 * GRP];
   __shared__ float Msh[GRP];
+  __shared__ uint32_t mkr_sh[GRP];
   __shared__ int ucount;
   __shared__ int uscan[33];
+  __shared__ float qsum[GRP];
+  // the group's query heads for step R, in the weight tile (written later)
+  float (&qs)[GRP][D] = *reinterpret_cast<float (*)[GRP][D]>(smem);
 
   const int g = blockIdx.y, split = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, tig = lane & 3;
@@ -834,11 +868,81 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
   const size_t rowg = static_cast<size_t>(g) * S;  // V rows: the cache's stride
 
   for (int e = tid; e < (NT * 8 - C::NC) * kStr; e += kOutThreads) as[C::NC * kStr + e] = __float2half_rn(0.0f);
-  // one maximum per head for every token: the larger of the bound on the
-  // resident scores outside the union and the refined maximum (a key of 0:
-  // no such token)
+  // a warp's value-code stream of a sub-chunk: 16-token tiles through its
+  // ring of kRing cp.async stages (the stage of tile ti is (ti - tile0) mod kRing)
+  auto issue_st = [&](int c0, int n, int ti, int st) {
+    const int tok = 16 * ti + (lane >> 1);
+    if (tok < n)
+      cp_async16_attn(ring + ((warp * kRing + st) * 16 + (lane >> 1)) * kWordsPerRow + (lane & 1) * 4,
+                      v_res + (rowg + c0 + tok) * kWordsPerRow + (lane & 1) * 4);
+  };
+  auto issue_at = [&](int c0, int n, int tile0, int ti) { issue_st(c0, n, ti, (ti - tile0) % kRing); };
+  auto start_stream = [&](int c0) {
+    const int n = min(t1s, c0 + kSub) - c0;
+    const int ntile = (n + 15) >> 4;
+    const int tpw = (ntile + kOW - 1) / kOW;
+    const int tile0 = min(ntile, warp * tpw), tile1 = min(ntile, tile0 + tpw);
+    for (int i = 0; i < kRing - 1; ++i) {
+      if (tile0 + i < tile1) issue_at(c0, n, tile0, tile0 + i);
+      cp_async_commit_attn();
+    }
+  };
+  start_stream(t0s);  // the value codes are inputs: no earlier pass writes them
+  if (tid < GRP) mkr_sh[tid] = 0u;
+  load_q<GRP>(q, g, qs, qsum);  // contains __syncthreads
+  pdl_wait();  // the selection (and every pass before it)
+
+  // the sub-chunk's union tokens (ascending offsets) from the group's bitmask;
+  // a token whose refinement bits are not on the device (a cache slot < 0)
+  // is flagged kUMiss: it keeps its resident key and value this step
+  auto list_union = [&](int c0, int n) {
+    const int nw = (n + 31) >> 5;  // c0 is a multiple of 32
+    uint32_t wbits = 0;
+    if (tid < nw) {
+      wbits = umask[static_cast<size_t>(g) * words_t + (c0 >> 5) + tid];
+      const int rem = n - 32 * tid;
+      if (rem < 32) wbits &= (1u << rem) - 1u;
+    }
+    int tot;
+    int pos = sfd::block_exclusive_scan(__popc(wbits), uscan, &tot);  // nw <= kSub / 32 <= blockDim
+    while (wbits) {
+      const int b = __ffs(wbits) - 1;
+      wbits &= wbits - 1u;
+      const int i = 32 * tid + b;
+      const bool miss = uslot != nullptr && uslot[rowg + c0 + i] < 0;
+      ulist[pos++] = static_cast<uint16_t>(i | (miss ? kUMiss : 0));
+    }
+    if (tid == 0) ucount = tot;
+    __syncthreads();
+  };
+
+
+  // R. the range's union tokens get their refined scores before any weight
+  //    is formed: the CTA's maximum per head covers them
+  {
+    uint32_t mk[GRP];
+#pragma unroll
+    for (int h = 0; h < GRP; ++h) mk[h] = 0u;
+    for (int c0 = t0s; c0 < t1s; c0 += kSub) {
+      list_union(c0, min(t1s, c0 + kSub) - c0);
+      for (int u = tid; u < ucount; u += kOutThreads)
+        refine_token<GRP>(k_res, k_ref, uslot, k_scale, k_zero, T, rowg, g, c0 + (ulist[u] & kUOff), qs, qsum, score,
+                          mk);
+      __syncthreads();  // the list is rebuilt for the next sub-chunk
+    }
+#pragma unroll
+    for (int h = 0; h < GRP; ++h) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mk[h] = max(mk[h], __shfl_xor_sync(0xffffffffu, mk[h], o));
+      if (lane == 0 && mk[h]) atomicMax(&mkr_sh[h], mk[h]);
+    }
+    __syncthreads();
+  }
+  // this CTA's maximum per head for every token of its range: the larger of
+  // the bound on the resident scores outside the union and the union's
+  // (refined or resident) maximum in the range (a key of 0: no such token)
   if (tid < GRP) {
-    const uint32_t mk = mkey[g * GRP + tid], rk = rkey[g * GRP + tid];
+    const uint32_t mk = mkey[g * GRP + tid], rk = mkr_sh[tid];
     float m = mk ? from_okey32(mk) : -INFINITY;
     if (rk) m = fmaxf(m, from_okey32(rk));
     Msh[tid] = m;
@@ -874,43 +978,19 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
     const int ntile = (n + 15) >> 4;
     const int tpw = (ntile + kOW - 1) / kOW;
     const int tile0 = min(ntile, warp * tpw), tile1 = min(ntile, tile0 + tpw);
-    auto issue = [&](int ti) {
-      const int st = (ti - tile0) % kRing;
-      const int tok = 16 * ti + (lane >> 1);
-      if (tok < n)
-        cp_async16_attn(ring + ((warp * kRing + st) * 16 + (lane >> 1)) * kWordsPerRow + (lane & 1) * 4,
-                        v_res + (rowg + c0 + tok) * kWordsPerRow + (lane & 1) * 4);
-    };
-    // start the code stream while the weights are being computed
-    for (int i = 0; i < kRing - 1; ++i) {
-      if (tile0 + i < tile1) issue(tile0 + i);
-      cp_async_commit_attn();
-    }
+    // start the code stream while the weights are being computed (the first
+    // sub-chunk's started before step R)
+    if (c0 != t0s) start_stream(c0);
 
-    // 0. the sub-chunk's refined tokens (ascending) from the group's bitmask;
-    //    their value refinement rows are staged for step 3 (their scores were
-    //    refined in the score buffer before this pass)
-    {
-      const int nw = (n + 31) >> 5;  // c0 is a multiple of 32
-      uint32_t wbits = 0;
-      if (tid < nw) {
-        wbits = umask[static_cast<size_t>(g) * words_t + (c0 >> 5) + tid];
-        const int rem = n - 32 * tid;
-        if (rem < 32) wbits &= (1u << rem) - 1u;
-      }
-      int tot;
-      int pos = sfd::block_exclusive_scan(__popc(wbits), uscan, &tot);  // nw <= kSub / 32 <= blockDim
-      while (wbits) {
-        const int b = __ffs(wbits) - 1;
-        wbits &= wbits - 1u;
-        ulist[pos++] = static_cast<uint16_t>(32 * tid + b);
-      }
-      if (tid == 0) ucount = tot;
-      __syncthreads();
-    }
+    // 0. the sub-chunk's union tokens (the list of step R when the range is
+    //    one sub-chunk); the value refinement rows of the refined ones are
+    //    staged for step 3
+    if (t1s - t0s > kSub) list_union(c0, n);
     const int nu = ucount;
     for (int u = tid; u < min(nu, kUCap); u += kOutThreads) {
-      const uint32_t* src = vref_row(v_ref, uslot, rowg + c0 + ulist[u]);
+      const int e = ulist[u];
+      if (e & kUMiss) continue;
+      const uint32_t* src = vref_row(v_ref, uslot, rowg + c0 + e);
       cp_async16_attn(vrs + u * kWordsPerRow, src);
       cp_async16_attn(vrs + u * kWordsPerRow + 4, src + 4);
     }
@@ -920,33 +1000,34 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
     for (int h = 0; h < GRP; ++h) M[h] = Msh[h];
 
     // 1. weights into shared memory (zero past the end of the last tile) and
-    //    sums; the scores, scales and zeros of four of this thread's tokens
+    //    sums; the scores, scales and zeros of kWB of this thread's tokens
     //    are loaded before any is used
+    constexpr int kWB = GRP >= 4 ? 4 : 8;
+    static_assert(kPerThr % kWB == 0, "whole batches of tokens in the weight pass");
 #pragma unroll 1
-    for (int j0 = 0; j0 < kPerThr; j0 += 4) {
+    for (int j0 = 0; j0 < kPerThr; j0 += kWB) {
       if (j0 * kOutThreads >= 16 * ntile) break;  // uniform over the block
-      float sc4[4][GRP];
-      uint16_t vs4[4], vz4[4];
+      float scb[kWB][GRP];
+      uint16_t vsb[kWB], vzb[kWB];
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
+      for (int jj = 0; jj < kWB; ++jj) {
         const int i = tid + (j0 + jj) * kOutThreads;
         const bool valid = i < n;
-        vs4[jj] = valid ? v_scale[rowg + c0 + i] : 0;
-        vz4[jj] = valid ? v_zero[rowg + c0 + i] : 0;
+        vsb[jj] = valid ? v_scale[rowg + c0 + i] : 0;
+        vzb[jj] = valid ? v_zero[rowg + c0 + i] : 0;
 #pragma unroll
-        for (int h = 0; h < GRP; ++h) sc4[jj][h] = valid ? score[(static_cast<size_t>(g) * GRP + h) * T + c0 + i] : 0.0f;
+        for (int h = 0; h < GRP; ++h) scb[jj][h] = valid ? score[(static_cast<size_t>(g) * GRP + h) * T + c0 + i] : 0.0f;
       }
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-      const int i = tid + (j0 + jj) * kOutThreads;
-      const bool valid = i < n;
-      if (i < 16 * ntile) {
-        if (valid) {
-          const float sv = sfd::half_bits_to_float(vs4[jj]);
-          const float zv = sfd::half_bits_to_float(vz4[jj]);
+      for (int jj = 0; jj < kWB; ++jj) {
+        const int i = tid + (j0 + jj) * kOutThreads;
+        if (i >= 16 * ntile) continue;
+        if (i < n) {
+          const float sv = sfd::half_bits_to_float(vsb[jj]);
+          const float zv = sfd::half_bits_to_float(vzb[jj]);
 #pragma unroll
           for (int h = 0; h < GRP; ++h) {
-            const float p = __expf(sc4[jj][h] - M[h]);
+            const float p = __expf(scb[jj][h] - M[h]);
             const float al = p * sv;
             const __half ahi = __float2half_rn(al);
             const __half alo = __float2half_rn(al - __half2float(ahi));
@@ -961,17 +1042,20 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
           for (int h = 0; h < 2 * GRP; ++h) as[h * kStr + i] = __float2half_rn(0.0f);
         }
       }
-      }
     }
     __syncthreads();
 
-    // 2. MMAs over this warp's tiles
+    // 2. MMAs over this warp's tiles (stage counters instead of the modulus)
+    const uint32_t* ringw = ring + warp * kRing * 16 * kWordsPerRow;
+    int st_use = 0, st_iss = kRing - 1;
     for (int ti = tile0; ti < tile1; ++ti) {
-      if (ti + kRing - 1 < tile1) issue(ti + kRing - 1);
+      if (ti + kRing - 1 < tile1) issue_st(c0, n, ti + kRing - 1, st_iss);
+      st_iss = st_iss == kRing - 1 ? 0 : st_iss + 1;
       cp_async_commit_attn();
       cp_async_wait_attn<kRing - 1>();
       __syncwarp();
-      const uint32_t* vr = ring + (warp * kRing + (ti - tile0) % kRing) * 16 * kWordsPerRow;
+      const uint32_t* vr = ringw + st_use * 16 * kWordsPerRow;
+      st_use = st_use == kRing - 1 ? 0 : st_use + 1;
       uint32_t b0[NT], b1[NT];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -998,7 +1082,9 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
 
     // 3. refined tokens: alpha (c_f - 1.5), lane = dims 4 lane .. 4 lane + 3
     for (int u = warp; u < nu; u += kOW) {
-      const int i = ulist[u];
+      const int e = ulist[u];
+      if (e & kUMiss) continue;  // uniform over the warp
+      const int i = e;
       const uint32_t wrow = u < kUCap ? vrs[u * kWordsPerRow + (lane >> 2)]
                                       : vref_row(v_ref, uslot, rowg + c0 + i)[lane >> 2];
       const uint32_t wf = wrow >> ((lane & 3) * 8);
@@ -1082,9 +1168,23 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
   __syncthreads();
   if (!last) return;
   __threadfence();
-  // every split weighted its tokens against the same maximum per head: the
-  // merge sums the splits' weight sums and outputs; two outputs per thread,
-  // eight splits' partials of each in flight at once
+  // every split weighted its tokens against its own maximum per head M_c:
+  // factors e^(M_c - M) per head and split (M the largest of the head's),
+  // in the dead weight tile
+  float* fac = reinterpret_cast<float*>(smem);  // [GRP][splits]
+  for (int h = warp; h < GRP; h += kOW) {
+    const float* ph = pg + static_cast<size_t>(h) * splits * (D + 2);
+    float mx = -INFINITY;
+    for (int c = lane; c < splits; c += 32) mx = fmaxf(mx, __ldcg(ph + static_cast<size_t>(c) * (D + 2)));
+    mx = warp_max(mx);
+    for (int c = lane; c < splits; c += 32) {
+      const float mc = __ldcg(ph + static_cast<size_t>(c) * (D + 2));
+      fac[h * splits + c] = mc == -INFINITY ? 0.0f : __expf(mc - mx);
+    }
+  }
+  __syncthreads();
+  // the merge sums the splits' scaled weight sums and outputs; two outputs
+  // per thread, sixteen splits' partials of each in flight at once
   for (int e0 = tid; e0 < GRP * D; e0 += 2 * kOutThreads) {
     const int e1 = e0 + kOutThreads;
     const bool has1 = e1 < GRP * D;
@@ -1093,10 +1193,10 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
     const float* p1 = pg + static_cast<size_t>(h1) * splits * (D + 2);
     const int d0 = e0 % D, d1 = has1 ? e1 % D : d0;
     float A0 = 0.0f, A1 = 0.0f, L0 = 0.0f, L1 = 0.0f;
-    for (int sp = 0; sp < splits; sp += 8) {
-      float v0[8], v1[8], l0[8], l1[8];
+    for (int sp = 0; sp < splits; sp += 16) {
+      float v0[16], v1[16], l0[16], l1[16];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 16; ++u) {
         const size_t o = static_cast<size_t>(sp + u) * (D + 2);
         const bool ok = sp + u < splits;
         v0[u] = ok ? __ldcg(p0 + o + 2 + d0) : 0.0f;
@@ -1105,11 +1205,13 @@ attn_out_kernel(const uint32_t* __restrict__ v_res,
         l1[u] = (ok && has1) ? __ldcg(p1 + o + 1) : 0.0f;
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        A0 += v0[u];
-        L0 += l0[u];
-        A1 += v1[u];
-        L1 += l1[u];
+      for (int u = 0; u < 16; ++u) {
+        const bool ok = sp + u < splits;
+        const float f0 = ok ? fac[h0 * splits + sp + u] : 0.0f, f1 = ok ? fac[h1 * splits + sp + u] : 0.0f;
+        A0 = fmaf(f0, v0[u], A0);
+        L0 = fmaf(f0, l0[u], L0);
+        A1 = fmaf(f1, v1[u], A1);
+        L1 = fmaf(f1, l1[u], L1);
       }
     }
     out[(static_cast<size_t>(g) * GRP + h0) * D + d0] = A0 / L0;
@@ -1171,62 +1273,84 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
   int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
   uint32_t* amaxu = reinterpret_cast<uint32_t*>(ws + L.amax);
   uint32_t* mkey = reinterpret_cast<uint32_t*>(ws + L.mkey);
-  uint32_t* rkey = reinterpret_cast<uint32_t*>(ws + L.rkey);
+  const bool selecting = k > 0 && k < T;
+  SelBand* band = reinterpret_cast<SelBand*>(ws + L.band);
+  int32_t* ccnt = reinterpret_cast<int32_t*>(ws + L.ccnt);
   SF_CHECK_CUDA(cudaFuncSetAttribute(attn_score_mma_kernel<GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(score_smem(GRP))));
   attn_score_mma_kernel<GRP><<<ga, kScThreads, score_smem(GRP), s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, S,
                                                                      tpc, score, smax, hist, amaxu, mkey);
   sf_status st = sf::check_launch("attn_score_mma_kernel");
   if (st != SF_OK) return st;
-  if (k > 0 && k < T) {
-    int32_t* ccnt = reinterpret_cast<int32_t*>(ws + L.ccnt);
-    attn_select_compact_kernel<GRP><<<dim3(L.nchunks, Hq), kCompThreads, 0, s>>>(q, T, k, score, smax, hist, amaxu,
-                                                                                cand, ccnt, status);
-    st = sf::check_launch("attn_select_compact_kernel");
-    if (st != SF_OK) return st;
+  if (selecting) {
+    {
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = dim3(static_cast<unsigned>((T + kChunk - 1) / kChunk), static_cast<unsigned>(Hq));
+      cfg.blockDim = dim3(kCompThreads);
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, attn_compact_kernel, q, T, k, static_cast<const float*>(score),
+                                       static_cast<const float*>(smax), static_cast<const int32_t*>(hist),
+                                       static_cast<const uint32_t*>(amaxu), band, cand, ccnt, status, grp));
+      st = sf::check_launch("attn_compact_kernel");
+      if (st != SF_OK) return st;
+    }
+    // the group's bitmask words in the cluster's shared memory when they fit
+    const int wper = (L.words_t + GRP - 1) / GRP;
+    const int dsm = wper <= kSelMaxWords ? 1 : 0;
+    const size_t dyn = sel_dyn_smem(dsm ? wper : 0);
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(Hq));
-    cfg.blockDim = dim3(kFinThreads);
-    cfg.dynamicSmemBytes = kFinDynSmem;
-    SF_CHECK_CUDA(cudaFuncSetAttribute(attn_select_finish_kernel<GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kFinDynSmem)));
+    cfg.blockDim = dim3(kSelThreads);
+    cfg.dynamicSmemBytes = dyn;
+    SF_CHECK_CUDA(cudaFuncSetAttribute(attn_select_kernel<GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(dyn)));
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = GRP;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, attn_select_finish_kernel<GRP>, q, kv->k_res, kv->k_ref, kv->k_scale,
-                                     kv->k_zero, T, k, S, score, static_cast<const float*>(smax),
-                                     static_cast<const int32_t*>(hist), static_cast<const uint32_t*>(amaxu), cand,
-                                     static_cast<const int32_t*>(ccnt), cand2, kap, sel_head, umask, L.words_t,
-                                     sel_out, sel_n, status, mkey));
-    st = sf::check_launch("attn_select_finish_kernel");
+    cfg.numAttrs = 2;
+    SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, attn_select_kernel<GRP>, q, kv->k_res, kv->k_scale, kv->k_zero, T, k, S,
+                                     static_cast<const float*>(score), static_cast<const SelBand*>(band),
+                                     static_cast<const int32_t*>(cand), static_cast<const int32_t*>(ccnt), cand2, kap,
+                                     sel_head, umask, L.words_t, wper, dsm, sel_out, sel_n, status, mkey));
+    st = sf::check_launch("attn_select_kernel");
     if (st != SF_OK) return st;
   } else if (k == 0) {  // the token bitmask was cleared with the workspace
     SF_CHECK_CUDA(cudaMemsetAsync(sel_n, 0, sizeof(int32_t) * Hkv, s));
-  } else {
+  } else {  // every token is in the union
     fill_all_kernel<<<dim3(32, Hkv), 256, 0, s>>>(T, grp, k, L.words_t, umask, sel_out, sel_n, mkey);
     st = sf::check_launch("fill_all_kernel");
-    if (st != SF_OK) return st;
-  }
-  if (k > 0) {
-    const int cap = grp * k;
-    const int nblk = std::max(1, std::min((cap + kRefThreads - 1) / kRefThreads, 2 * sms / Hkv));
-    attn_refine_kernel<GRP><<<dim3(nblk, Hkv), kRefThreads, 0, s>>>(q, kv->k_res, k_ref, uslot, kv->k_scale,
-                                                                   kv->k_zero, T, S, cap, sel_out, sel_n, score,
-                                                                   rkey, umask, L.words_t);
-    st = sf::check_launch("attn_refine_kernel");
     if (st != SF_OK) return st;
   }
   dim3 gb(L.splits, Hkv);
   SF_CHECK_CUDA(cudaFuncSetAttribute(attn_out_kernel<GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(OutCfg<GRP>::smem)));
-  attn_out_kernel<GRP><<<gb, kOutThreads, OutCfg<GRP>::smem, s>>>(kv->v_res, v_ref, uslot, kv->v_scale, kv->v_zero,
-                                                                 T, S, L.tps, L.words_t, L.splits, score, mkey, rkey,
-                                                                 umask, part, done, out);
+  {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = gb;
+    cfg.blockDim = dim3(kOutThreads);
+    cfg.dynamicSmemBytes = OutCfg<GRP>::smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, attn_out_kernel<GRP>, q, kv->k_res, k_ref, kv->k_scale, kv->k_zero,
+                                     static_cast<const uint32_t*>(kv->v_res), v_ref, uslot, kv->v_scale, kv->v_zero,
+                                     T, S, L.tps, L.words_t, L.splits, score, static_cast<const uint32_t*>(mkey),
+                                     static_cast<const uint32_t*>(umask), part, done, out));
+  }
   st = sf::check_launch("attn_out_kernel");
   if (st != SF_OK) return st;
   if (kv->ref_cache) return sf::cache_mark_used(kv->ref_cache, s);

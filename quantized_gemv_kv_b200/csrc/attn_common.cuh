@@ -33,12 +33,24 @@ constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128), rounded to fp
 constexpr int kHistBits = 11;      // per-head histogram of the fast scores' top 11 key bits
 constexpr int kHistBins = 1 << kHistBits;
 constexpr int kHistShift = 32 - kHistBits;
-constexpr int kChunk = 4096;       // tokens per CTA of the candidate compaction
+
+// A head's selection band, derived once from the score pass's histogram:
+// every token whose exact key can reach the top k has a fast score >= f_low;
+// the k-th largest fast score lies in histogram bin b1, kk-th from its top;
+// eps bounds |fast score - exact key / sqrt(d)|.
+struct SelBand {
+  double eps;
+  float f_low;
+  uint32_t b1;
+  int kk;
+  int pad;
+};
 
 struct Layout {
   // from smax on, everything is cleared at the start of a call
-  size_t score, cand, cand2, kap, sel, part, fcnt, smax, status, count, amax, mkey, rkey, ccnt, hist, umask, total;
-  int splits, tps, words_t, nchunks;
+  size_t score, cand, cand2, kap, sel, part, fcnt, smax, status, count, amax, mkey, band, ccnt, hist,
+      umask, total;
+  int splits, tps, words_t;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -51,10 +63,9 @@ Layout make_layout(int Hq, int Hkv, int T, int k, int sms) {
   L.tps = tps;
   L.splits = (T + tps - 1) / tps;
   L.words_t = (T + 31) / 32;
-  L.nchunks = (T + kChunk - 1) / kChunk;
   size_t off = 0;
   L.score = off; off = up256(off + sizeof(float) * Hq * static_cast<size_t>(T));
-  L.cand = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(T) + sizeof(int32_t) * Hq * L.nchunks);
+  L.cand = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(T));
   L.cand2 = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(T));
   L.kap = off; off = up256(off + sizeof(double) * Hq * static_cast<size_t>(T));
   L.sel = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(std::max(k, 1)));
@@ -66,8 +77,8 @@ Layout make_layout(int Hq, int Hkv, int T, int k, int sms) {
   L.count = off; off = up256(off + sizeof(int32_t) * Hkv);
   L.amax = off; off = up256(off + sizeof(uint32_t) * Hq);
   L.mkey = off; off = up256(off + sizeof(uint32_t) * Hq);  // max resident score key per head
-  L.rkey = off; off = up256(off + sizeof(uint32_t) * Hq);  // max refined score key per head
-  L.ccnt = off; off = up256(off + sizeof(int32_t) * Hq);   // listed candidates per head
+  L.band = off; off = up256(off + sizeof(SelBand) * Hq);     // selection band per head
+  L.ccnt = off; off = up256(off + sizeof(int32_t) * Hq);     // listed candidates per head
   L.hist = off; off = up256(off + sizeof(int32_t) * Hq * static_cast<size_t>(kHistBins));
   L.umask = off; off = up256(off + sizeof(uint32_t) * Hkv * static_cast<size_t>(L.words_t));
   L.total = off;
@@ -85,6 +96,14 @@ __device__ __forceinline__ unsigned long long okey64(double x) {
   const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(x));
   return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
 }
+
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while its predecessor runs; pdl_wait() returns once
+// the predecessor grid has completed and its memory is visible, and must come
+// before the first read of anything the predecessor writes.
+// pdl_launch_dependents() lets the next such kernel start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::); }
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -360,6 +379,18 @@ __device__ void find_bin_from_top_block(const int* hist, int nb, int kk, int* ou
   }
   if (threadIdx.x == 0 && tot < kk) { out[0] = 0; out[1] = kk; }
   __syncthreads();
+}
+
+// Per-head lower bound of the listed scores and the histogram bin: all threads call.
+__device__ void select_band(const int32_t* __restrict__ hist_h, int k, double eps_s, int* hsh, int* scan_scratch,
+                            int* binfo, uint32_t* b1, int* kk, float* f_low) {
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hsh[i] = hist_h[i];
+  __syncthreads();
+  find_bin_from_top_block(hsh, kHistBins, k, binfo, scan_scratch);
+  *b1 = static_cast<uint32_t>(binfo[0]);
+  *kk = binfo[1];
+  const float lower = from_okey32(*b1 << kHistShift);
+  *f_low = __double2float_rd(static_cast<double>(lower) - 2.0 * eps_s);
 }
 
 }  // namespace
