@@ -92,6 +92,8 @@ def parse():
                          "deadline reading)")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-extras", action="store_true", help="skip e2e / resident-only / roofline legs")
+    ap.add_argument("--qwen3-batches", type=int, default=1,
+                    help="also time Qwen3-8B decode linear layers at batch 1, 4 and 16 (0: skip); part of the extras")
     ap.add_argument("--hotpath-context", type=int, default=32768,
                     help="also time the 2+2-bit hot path at this context (0: skip); part of the extras")
     return ap.parse_args()
@@ -686,6 +688,83 @@ def hotpath_leg(args, sf, torch, dist, dev, world, T, phys):
     return out
 
 
+def qwen3_batch_leg(sf, torch, dist, dev, iters=20):
+    """Qwen3-8B-shaped decode linear layers at 3+1 bits, group 128, batch 1,
+    4 and 16: top 5% of channels per row, their union refined, a 25% LRU
+    refinement cache per matrix; one layer's seven GEMVs (batch 1: the
+    tensor-core batch-1 path; 4: CUDA cores; 16: the tensor-core batch path)
+    with the selection and the caches' step, graph-timed over a pool of 8
+    seeded inputs per batch size."""
+    from fractions import Fraction
+    from workloads import device_synth as ds
+    from quantized_gemv_kv_b200.decode import count_half_up
+    shapes = (("q", 4096, 4096), ("k", 1024, 4096), ("v", 1024, 4096), ("o", 4096, 4096),
+              ("gate", 12288, 4096), ("up", 12288, 4096), ("down", 4096, 12288))
+    b_r, b_f, G = 3, 1, 128
+    mats = {}
+    for i, (name, N, K) in enumerate(shapes):
+        W = ds.weight(5000 + i, N, K, device=dev)
+        qw = sf.quantize_nested(W, G, b_r, b_f)
+        del W
+        mats[name] = (qw, sf.pack_batch1(qw))
+    torch.cuda.synchronize()
+    out = {}
+    stream = torch.cuda.Stream()
+    for B in (1, 4, 16):
+        caches, ys, bufs = {}, {}, {}
+        for name, N, K in shapes:
+            qw = mats[name][0]
+            k = count_half_up(Fraction(5, 100), K)
+            master = qw.ref.cpu().contiguous().pin_memory()
+            caches[name] = sf.RefineCache(K, N * b_f // 8, count_half_up(Fraction(25, 100), K), min(K, B * k), master)
+            ys[name] = torch.empty((B, N), dtype=torch.float32, device=dev)
+        for K in (4096, 12288):
+            k = count_half_up(Fraction(5, 100), K)
+            pool = []
+            for j in range(8):
+                outl = torch.randperm(K, generator=torch.Generator(device="cpu").manual_seed(60 + j))[:K // 200]
+                xf = torch.randn((B, K), generator=torch.Generator(device="cpu").manual_seed(70 + j))
+                xf[:, outl] *= 30.0
+                pool.append(xf.to(torch.bfloat16).to(dev))
+            bufs[K] = (pool, k, torch.empty(B * k, dtype=torch.int32, device=dev),
+                       torch.empty(1, dtype=torch.int32, device=dev))
+        jobs1 = {name: sf.Batch1Jobs([(mats[name][1], caches[name], False, ys[name][0])]) for name, _, _ in shapes}
+
+        def layer(i):
+            for name, N, K in shapes:
+                pool, k, idx, n = bufs[K]
+                x = pool[i % 8]
+                sf.select_topk(x, k, idx, n)
+                caches[name].prefetch(idx, n)
+                if B == 1:
+                    jobs1[name].run(x, idx, n)
+                else:
+                    sf.gemv_refine(mats[name][0], x, idx, n, cache=caches[name], y=ys[name])
+
+        with torch.cuda.stream(stream):
+            for i in range(8):
+                layer(i)
+        torch.cuda.synchronize()
+        graphs = [capture(torch, lambda i=i: layer(i), stream) for i in range(8)]
+        for i in range(3):
+            graphs[i % 8].replay()
+        ms = timed(torch, dist, lambda i: graphs[i % 8].replay(), iters, stream)
+        nbytes = 0
+        for name, N, K in shapes:
+            nbytes += gemv_bytes(N, K, bufs[K][1] * B, b_r, b_f) + 2 * K * (B - 1) + 4 * N * (B - 1)
+        us = ms * 1e3 / iters
+        out[f"batch_{B}"] = {"us_per_layer": us, "tokens_per_s_per_layer": B * 1e6 / us,
+                             "effective_gbs": nbytes / (us * 1e-6) / 1e9,
+                             "path": {1: "integer tensor cores (batch 1)", 4: "CUDA cores",
+                                      16: "f16 tensor cores (batch 8-16)"}[B]}
+        del graphs
+        for c in caches.values():
+            c.close()
+    return {"workload": "Qwen3-8B decode linear layers (q/k/v/o 4096, gate/up/down 12288), 3+1 bits, group 128, "
+                        "top 5% per row, union refined, 25% LRU cache per matrix; one layer's seven GEMVs",
+            **out}
+
+
 def graph_kernels(g):
     """Kernel nodes of a captured graph (made with keep_graph=True), counted
     by kernel name: the library's launches read from the graph itself (memset
@@ -949,6 +1028,13 @@ def run_sf(args, rank, world, local_rank, dist):
         torch.cuda.empty_cache()
         hot = hotpath_leg(args, sf, torch, dist, dev, world, args.hotpath_context, phys)
         model = None
+    if not args.skip_extras and args.qwen3_batches:
+        if model is not None:
+            model.close()
+            del model
+            model = None
+        torch.cuda.empty_cache()
+        extras["qwen3_batches"] = qwen3_batch_leg(sf, torch, dist, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:

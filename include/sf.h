@@ -643,6 +643,24 @@ sf_status sf_kv_append_cached(const float* src, int Hkv, int d, int row_stride, 
                               uint32_t* res, uint16_t* scale, uint16_t* zero, sf_refine_cache* ref_cache, int part,
                               sf_stream_t stream);
 
+/*
+ * sf_kv_append_pair_cached -- sf_kv_append_cached for the key rows (k_src,
+ *   part 0) and value rows (v_src, part 1) of token t in one launch, with the
+ *   host master's copy taken off `stream`: on `stream` the refinement words
+ *   go to a device staging area of the cache (and to the cached copy of a
+ *   cached unit); one 2-D copy then moves them to the host master on `side`,
+ *   after what `stream` has enqueued so far.  Work enqueued on `side` after
+ *   this call (the cache's prefetch) reads the new words; the next append
+ *   waits for that copy (under stream capture: when it belongs to the same
+ *   capture).  side may equal stream.  The first call per cache allocates the
+ *   staging area and must not be under stream capture.
+ *   Constraints: as sf_kv_append_cached, for both rows.
+ */
+sf_status sf_kv_append_pair_cached(const float* k_src, const float* v_src, int Hkv, int d, int row_stride, int t,
+                                   int b_r, int b_f, uint32_t* k_res, uint16_t* k_scale, uint16_t* k_zero,
+                                   uint32_t* v_res, uint16_t* v_scale, uint16_t* v_zero, sf_refine_cache* ref_cache,
+                                   sf_stream_t stream, sf_stream_t side);
+
 #ifdef __cplusplus
 }
 #endif

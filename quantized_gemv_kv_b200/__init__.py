@@ -114,6 +114,7 @@ _SIGS = {
     "sf_rope_qk": ([_p, _i, _p, _i, _i, _i, ctypes.c_double, _p, _p], _i),
     "sf_kv_append": ([_p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p], _i),
     "sf_kv_append_cached": ([_p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _i, _p], _i),
+    "sf_kv_append_pair_cached": ([_p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -630,6 +631,22 @@ def kv_append_cached(src: torch.Tensor, res: torch.Tensor, scale: torch.Tensor, 
     Hkv, d = src.shape
     _check(_lib.sf_kv_append_cached(_ptr(src), Hkv, d, row_stride, t, b_r, b_f, _ptr(res), _ptr(scale), _ptr(zero),
                                     cache.handle, part, _stream(stream)))
+
+
+def kv_append_pair_cached(k_src: torch.Tensor, v_src: torch.Tensor, kq: "QWeight", vq: "QWeight", cache: RefineCache,
+                          row_stride: int, t: int, b_r: int = 2, b_f: int = 2, stream: torch.cuda.Stream | None = None,
+                          side: torch.cuda.Stream | None = None) -> None:
+    """``sf_kv_append_pair_cached``: the key and value rows of token t in one
+    launch; the host master's copy runs on ``side`` (default: ``stream``)."""
+    _dev(k_src, "k_src")
+    _dev(v_src, "v_src")
+    if k_src.dtype != torch.float32 or k_src.dim() != 2 or v_src.shape != k_src.shape or v_src.dtype != torch.float32:
+        raise ValueError("k_src and v_src must be 2-D float32 tensors of one shape")
+    Hkv, d = k_src.shape
+    st = _stream(stream)
+    _check(_lib.sf_kv_append_pair_cached(_ptr(k_src), _ptr(v_src), Hkv, d, row_stride, t, b_r, b_f, _ptr(kq.res),
+                                         _ptr(kq.scale), _ptr(kq.zero), _ptr(vq.res), _ptr(vq.scale), _ptr(vq.zero),
+                                         cache.handle, st, _stream(side) if side is not None else st))
 
 
 def norm_select(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor, k: int, idx: torch.Tensor, n: torch.Tensor,

@@ -349,6 +349,12 @@ struct sf_refine_cache {
   cudaStream_t aux = nullptr;
   bool ready_pending = false, used_pending = false;
   unsigned long long ready_capture = 0, used_capture = 0;
+  // a writer's staging area for the host master (sf_kv_append_pair_cached)
+  uint32_t* stage = nullptr;
+  size_t stage_words = 0;
+  cudaEvent_t ev_staged = nullptr, ev_flushed = nullptr;
+  bool flush_pending = false;
+  unsigned long long flush_capture = 0;
 };
 
 namespace {
@@ -401,6 +407,9 @@ sf_status cache_free(sf_refine_cache* c) {
   if (c->ev_idx) cudaEventDestroy(c->ev_idx);
   if (c->ev_ready) cudaEventDestroy(c->ev_ready);
   if (c->ev_used) cudaEventDestroy(c->ev_used);
+  if (c->stage) cudaFree(c->stage);
+  if (c->ev_staged) cudaEventDestroy(c->ev_staged);
+  if (c->ev_flushed) cudaEventDestroy(c->ev_flushed);
   if (c->aux) cudaStreamDestroy(c->aux);
   if (c->registered_here) cudaHostUnregister(const_cast<void*>(c->host_master));
   delete c;
@@ -482,6 +491,44 @@ sf_status cache_view_for_writer(sf_refine_cache* c, cudaStream_t stream, CacheWr
 }
 
 bool cache_deadline(const sf_refine_cache* c) { return c->deadline; }
+
+sf_status cache_append_stage(sf_refine_cache* c, cudaStream_t stream, size_t words, uint32_t** stage) {
+  if (c->stage_words < words) {
+    SF_REQUIRE(capture_id(stream) == 0,
+               "sf_kv_append_pair_cached: the first call per cache must not be under stream capture");
+    DeviceGuard guard(c->device);
+    if (c->stage) {
+      SF_CHECK_CUDA(cudaStreamSynchronize(stream));
+      cudaFree(c->stage);
+      c->stage = nullptr;
+      c->stage_words = 0;
+    }
+    SF_CHECK_CUDA(cudaMalloc(&c->stage, words * 4));
+    c->stage_words = words;
+    if (!c->ev_staged) SF_CHECK_CUDA(cudaEventCreateWithFlags(&c->ev_staged, cudaEventDisableTiming));
+    if (!c->ev_flushed) SF_CHECK_CUDA(cudaEventCreateWithFlags(&c->ev_flushed, cudaEventDisableTiming));
+  }
+  // the last flush read the staging area: the next write waits for it
+  if (c->flush_pending && c->flush_capture == capture_id(stream))
+    SF_CHECK_CUDA(cudaStreamWaitEvent(stream, c->ev_flushed, 0));
+  *stage = c->stage;
+  return SF_OK;
+}
+
+sf_status cache_append_flush(sf_refine_cache* c, cudaStream_t stream, cudaStream_t side, size_t dst_off,
+                             size_t dpitch, size_t width, int height) {
+  if (side != stream) {
+    SF_CHECK_CUDA(cudaEventRecord(c->ev_staged, stream));
+    SF_CHECK_CUDA(cudaStreamWaitEvent(side, c->ev_staged, 0));
+  }
+  char* dst = static_cast<char*>(const_cast<void*>(c->host_master)) + dst_off;
+  SF_CHECK_CUDA(cudaMemcpy2DAsync(dst, dpitch, c->stage, width, width, static_cast<size_t>(height),
+                                  cudaMemcpyDeviceToHost, side));
+  SF_CHECK_CUDA(cudaEventRecord(c->ev_flushed, side));
+  c->flush_pending = true;
+  c->flush_capture = capture_id(side);
+  return SF_OK;
+}
 
 sf_status cache_mark_used(sf_refine_cache* c, cudaStream_t stream) {
   SF_CHECK_CUDA(cudaEventRecord(c->ev_used, stream));

@@ -19,6 +19,25 @@ constexpr int kThreads = 1024;
 
 __device__ __forceinline__ uint16_t to_bf16(double v) { return __bfloat16_as_ushort(__double2bfloat16(v)); }
 
+// bf16(silu(g) u) rounded once from the exact value.  The fp32 evaluation
+// r = fl(fl(g / fl(1 + expf(-g))) u) is within 7 * 2^-24 |r| of the exact
+// value (expf within 2 ulp, CUDA math API accuracy table; four correctly
+// rounded operations), i.e. within 16 steps of r's fp32 bit pattern even
+// across a binade.  RNE to bf16 changes only at the midpoints (low 16 bits
+// 0x8000), so when r's low half lies farther than 16 from 0x8000 the exact
+// value rounds as r does; otherwise (and for non-normal or huge r) the value
+// is recomputed in fp64 and rounded once.
+__device__ __forceinline__ uint16_t silu_mul_bf16(float g, float u) {
+  const float e = expf(-g);
+  const float r = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, e)), u);
+  const uint32_t b = __float_as_uint(r) & 0x7FFFFFFFu;
+  const int low = static_cast<int>(b & 0xFFFFu);
+  if (isfinite(e) && b >= 0x00800000u && b < 0x7E800000u && (low < 0x8000 - 16 || low > 0x8000 + 16))
+    return __bfloat16_as_ushort(__float2bfloat16_rn(r));
+  const double gv = g;
+  return to_bf16(gv / (1.0 + exp(-gv)) * static_cast<double>(u));
+}
+
 // Writes the producer's row to xs (shared) and y (global), then selects.
 enum Producer { kNorm = 0, kRound = 1, kSilu = 2 };
 
@@ -44,14 +63,37 @@ __global__ void __launch_bounds__(kThreads) produce_select_kernel(const __grid_c
   if (A.op == kNorm) {
     __shared__ double part[kThreads / 32];
     __shared__ double inv_sh;
+    // up to kPer entries of x, delta and w per thread in registers, every
+    // load in flight; longer rows take a second sweep over x and w
+    constexpr int kPer = 8;
+    const bool in_regs = K <= kPer * kThreads;
+    float xv[kPer], wv[kPer];
     double ss = 0.0;
-    for (int i = tid; i < K; i += kThreads) {
-      float v = A.x[i];
-      if (A.delta) {
-        v = __fadd_rn(v, A.delta[i]);
-        A.x[i] = v;
+    if (in_regs) {
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = tid + j * kThreads;
+        xv[j] = i < K ? A.x[i] : 0.0f;
+        wv[j] = i < K ? A.w[i] : 0.0f;
+        if (A.delta && i < K) xv[j] = __fadd_rn(xv[j], A.delta[i]);
       }
-      ss = fma(static_cast<double>(v), static_cast<double>(v), ss);
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = tid + j * kThreads;
+        if (i < K) {
+          if (A.delta) A.x[i] = xv[j];
+          ss = fma(static_cast<double>(xv[j]), static_cast<double>(xv[j]), ss);
+        }
+      }
+    } else {
+      for (int i = tid; i < K; i += kThreads) {
+        float v = A.x[i];
+        if (A.delta) {
+          v = __fadd_rn(v, A.delta[i]);
+          A.x[i] = v;
+        }
+        ss = fma(static_cast<double>(v), static_cast<double>(v), ss);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -64,23 +106,62 @@ __global__ void __launch_bounds__(kThreads) produce_select_kernel(const __grid_c
     }
     __syncthreads();
     const double inv = inv_sh;
-    for (int i = tid; i < K; i += kThreads) {
-      const uint16_t v = to_bf16(static_cast<double>(A.x[i]) * inv * static_cast<double>(A.w[i]));
-      xs[i] = v;
-      A.y[i] = v;
+    if (in_regs) {
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = tid + j * kThreads;
+        if (i < K) {
+          const uint16_t v = to_bf16(static_cast<double>(xv[j]) * inv * static_cast<double>(wv[j]));
+          xs[i] = v;
+          A.y[i] = v;
+        }
+      }
+    } else {
+      for (int i = tid; i < K; i += kThreads) {
+        const uint16_t v = to_bf16(static_cast<double>(A.x[i]) * inv * static_cast<double>(A.w[i]));
+        xs[i] = v;
+        A.y[i] = v;
+      }
     }
   } else if (A.op == kRound) {
-    for (int i = tid; i < K; i += kThreads) {
-      const uint16_t v = __bfloat16_as_ushort(__float2bfloat16_rn(A.a[i]));
-      xs[i] = v;
-      A.y[i] = v;
+    constexpr int kPer = 16;
+    for (int i0 = 0; i0 < K; i0 += kPer * kThreads) {
+      float av[kPer];
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = i0 + tid + j * kThreads;
+        av[j] = i < K ? A.a[i] : 0.0f;
+      }
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = i0 + tid + j * kThreads;
+        if (i < K) {
+          const uint16_t v = __bfloat16_as_ushort(__float2bfloat16_rn(av[j]));
+          xs[i] = v;
+          A.y[i] = v;
+        }
+      }
     }
   } else {
-    for (int i = tid; i < K; i += kThreads) {
-      const double gv = A.a[i];
-      const uint16_t v = to_bf16(gv / (1.0 + exp(-gv)) * static_cast<double>(A.b[i]));
-      xs[i] = v;
-      A.y[i] = v;
+    // eight entries of g and u per thread in flight at a time
+    constexpr int kPer = 8;
+    for (int i0 = 0; i0 < K; i0 += kPer * kThreads) {
+      float gv[kPer], uv[kPer];
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = i0 + tid + j * kThreads;
+        gv[j] = i < K ? A.a[i] : 0.0f;
+        uv[j] = i < K ? A.b[i] : 0.0f;
+      }
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int i = i0 + tid + j * kThreads;
+        if (i < K) {
+          const uint16_t v = silu_mul_bf16(gv[j], uv[j]);
+          xs[i] = v;
+          A.y[i] = v;
+        }
+      }
     }
   }
   __syncthreads();

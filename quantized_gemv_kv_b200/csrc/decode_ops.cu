@@ -91,23 +91,16 @@ constexpr int kAppendMaxD = 512;
 // group with the arithmetic of the nested quantizer (min/max, fp32 division,
 // fp16 scale, integer zero point, ties to even) and written as cache row
 // g * row_stride + t: resident and refinement bitstreams (row-major, little
-// endian), fp16 scale and zero.
-// The refinement words go to ref + r * ref_pitch + ref_off (the store:
-// pitch d*b_f/32, offset 0; a KV refinement cache's host master: the unit's
-// pitch and the K or V half).  When unit_slot is given and unit r is cached,
-// the same words also go to its cache row, so a cached copy never goes stale.
-__global__ void kv_append_kernel(const float* __restrict__ src, int Hkv, int d, int row_stride, int t, int b_r,
-                                 int b_f, uint32_t* __restrict__ res, uint32_t* __restrict__ ref, int ref_pitch,
-                                 int ref_off, const int32_t* __restrict__ unit_slot, uint32_t* __restrict__ crows,
-                                 uint16_t* __restrict__ scale, uint16_t* __restrict__ zero) {
-  __shared__ uint8_t codes[4][kAppendMaxD];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = blockIdx.x * 4 + warp;
-  if (g >= Hkv) return;  // uniform over the warp
+// endian), fp16 scale and zero.  The refinement words go to ref_row and, when
+// crow is not null (the unit is cached), to crow as well, so a cached copy
+// never goes stale.
+__device__ void append_row(const float* __restrict__ row, int d, int b_r, int b_f, size_t r, uint32_t* __restrict__ res,
+                           uint16_t* __restrict__ scale, uint16_t* __restrict__ zero, uint32_t* __restrict__ ref_row,
+                           uint32_t* __restrict__ crow, uint8_t* codes) {
+  const int lane = threadIdx.x & 31;
   const int b = b_r + b_f;
   const float qmax = static_cast<float>((1 << b) - 1);
   const int per_lane = d >> 5;
-  const float* row = src + static_cast<size_t>(g) * d;
   float v[kAppendMaxD / 32];
   float lo = INFINITY, hi = -INFINITY;
   for (int m = 0; m < per_lane; ++m) {
@@ -128,7 +121,6 @@ __global__ void kv_append_kernel(const float* __restrict__ src, int Hkv, int d, 
   float zf = rintf(__fdiv_rn(-lo, sf));
   zf = fminf(fmaxf(zf, 0.0f), qmax);
   const int zi = static_cast<int>(zf);
-  const size_t r = static_cast<size_t>(g) * row_stride + t;
   if (lane == 0) {
     scale[r] = __half_as_ushort(s16);
     zero[r] = __half_as_ushort(__int2half_rn(zi));
@@ -136,7 +128,7 @@ __global__ void kv_append_kernel(const float* __restrict__ src, int Hkv, int d, 
   for (int m = 0; m < per_lane; ++m) {
     float qf = rintf(__fdiv_rn(v[m], sf)) + static_cast<float>(zi);
     qf = fminf(fmaxf(qf, 0.0f), qmax);
-    codes[warp][lane + 32 * m] = static_cast<uint8_t>(static_cast<int>(qf));
+    codes[lane + 32 * m] = static_cast<uint8_t>(static_cast<int>(qf));
   }
   __syncwarp();
   const uint32_t rmask = (1u << b_r) - 1u, fmask = (1u << b_f) - 1u;
@@ -145,7 +137,7 @@ __global__ void kv_append_kernel(const float* __restrict__ src, int Hkv, int d, 
     uint32_t word = 0;
     for (int bit = 0; bit < 32; ++bit) {
       const int sb = ww * 32 + bit;
-      word |= (((static_cast<uint32_t>(codes[warp][sb / b_r]) >> b_f) & rmask) >> (sb % b_r) & 1u) << bit;
+      word |= (((static_cast<uint32_t>(codes[sb / b_r]) >> b_f) & rmask) >> (sb % b_r) & 1u) << bit;
     }
     res[r * rw + ww] = word;
   }
@@ -153,14 +145,60 @@ __global__ void kv_append_kernel(const float* __restrict__ src, int Hkv, int d, 
     uint32_t word = 0;
     for (int bit = 0; bit < 32; ++bit) {
       const int sb = ww * 32 + bit;
-      word |= ((static_cast<uint32_t>(codes[warp][sb / b_f]) & fmask) >> (sb % b_f) & 1u) << bit;
+      word |= ((static_cast<uint32_t>(codes[sb / b_f]) & fmask) >> (sb % b_f) & 1u) << bit;
     }
-    ref[r * ref_pitch + ref_off + ww] = word;
-    if (unit_slot != nullptr) {
-      const int slot = unit_slot[r];
-      if (slot >= 0) crows[static_cast<size_t>(slot) * ref_pitch + ref_off + ww] = word;
-    }
+    ref_row[ww] = word;
+    if (crow != nullptr) crow[ww] = word;
   }
+}
+
+// The refinement words go to ref + r * ref_pitch + ref_off (the store: pitch
+// d*b_f/32, offset 0; a KV refinement cache's host master: the unit's pitch
+// and the K or V half); unit_slot / crows: the cache's slots and rows.
+__global__ void kv_append_kernel(const float* __restrict__ src, int Hkv, int d, int row_stride, int t, int b_r,
+                                 int b_f, uint32_t* __restrict__ res, uint32_t* __restrict__ ref, int ref_pitch,
+                                 int ref_off, const int32_t* __restrict__ unit_slot, uint32_t* __restrict__ crows,
+                                 uint16_t* __restrict__ scale, uint16_t* __restrict__ zero) {
+  __shared__ uint8_t codes[4][kAppendMaxD];
+  const int warp = threadIdx.x >> 5;
+  const int g = blockIdx.x * 4 + warp;
+  if (g >= Hkv) return;  // uniform over the warp
+  const size_t r = static_cast<size_t>(g) * row_stride + t;
+  uint32_t* crow = nullptr;
+  if (unit_slot != nullptr) {
+    const int slot = unit_slot[r];
+    if (slot >= 0) crow = crows + static_cast<size_t>(slot) * ref_pitch + ref_off;
+  }
+  append_row(src + static_cast<size_t>(g) * d, d, b_r, b_f, r, res, scale, zero, ref + r * ref_pitch + ref_off, crow,
+             codes[warp]);
+}
+
+// The key and value rows of token t in one launch (blockIdx.y: 0 keys, 1
+// values); the refinement words go to the device staging rows stage[g] (K
+// words, then V words: the unit's layout) and to the cached copy of a cached
+// unit.
+struct AppendPair {
+  const float* src[2];
+  uint32_t* res[2];
+  uint16_t* scale[2];
+  uint16_t* zero[2];
+  uint32_t* stage;
+  const int32_t* unit_slot;
+  uint32_t* crows;
+  int Hkv, d, row_stride, t, b_r, b_f;
+};
+
+__global__ void kv_append_pair_kernel(const __grid_constant__ AppendPair A) {
+  __shared__ uint8_t codes[4][kAppendMaxD];
+  const int warp = threadIdx.x >> 5, part = blockIdx.y;
+  const int g = blockIdx.x * 4 + warp;
+  if (g >= A.Hkv) return;  // uniform over the warp
+  const int fw = A.d * A.b_f / 32;
+  const size_t r = static_cast<size_t>(g) * A.row_stride + A.t;
+  const int slot = A.unit_slot[r];
+  uint32_t* crow = slot >= 0 ? A.crows + static_cast<size_t>(slot) * 2 * fw + part * fw : nullptr;
+  append_row(A.src[part] + static_cast<size_t>(g) * A.d, A.d, A.b_r, A.b_f, r, A.res[part], A.scale[part],
+             A.zero[part], A.stage + static_cast<size_t>(g) * 2 * fw + part * fw, crow, codes[warp]);
 }
 
 }  // namespace
@@ -211,6 +249,59 @@ extern "C" sf_status sf_kv_append(const float* src, int Hkv, int d, int row_stri
   kv_append_kernel<<<(Hkv + 3) / 4, 128, 0, sf::as_cuda(stream)>>>(src, Hkv, d, row_stride, t, b_r, b_f, res, ref,
                                                                    d * b_f / 32, 0, nullptr, nullptr, scale, zero);
   return sf::check_launch("kv_append_kernel");
+}
+
+extern "C" sf_status sf_kv_append_pair_cached(const float* k_src, const float* v_src, int Hkv, int d, int row_stride,
+                                              int t, int b_r, int b_f, uint32_t* k_res, uint16_t* k_scale,
+                                              uint16_t* k_zero, uint32_t* v_res, uint16_t* v_scale, uint16_t* v_zero,
+                                              sf_refine_cache* ref_cache, sf_stream_t stream, sf_stream_t side) {
+  SF_REQUIRE(k_src && v_src && k_res && k_scale && k_zero && v_res && v_scale && v_zero && ref_cache,
+             "sf_kv_append_pair_cached: null pointer");
+  SF_REQUIRE(Hkv >= 1, "sf_kv_append_pair_cached: Hkv must be >= 1");
+  SF_REQUIRE(d >= 32 && d % 32 == 0 && d <= kAppendMaxD,
+             "sf_kv_append_pair_cached: d must be a multiple of 32 in [32, %d]", kAppendMaxD);
+  SF_REQUIRE(b_r == 2 || b_r == 3, "sf_kv_append_pair_cached: b_r must be 2 or 3");
+  SF_REQUIRE(b_f == 1 || b_f == 2, "sf_kv_append_pair_cached: b_f must be 1 or 2");
+  SF_REQUIRE(b_r + b_f <= 4, "sf_kv_append_pair_cached: b_r + b_f must be <= 4");
+  SF_REQUIRE(row_stride >= 1 && t >= 0 && t < row_stride, "sf_kv_append_pair_cached: need 0 <= t < row_stride");
+  cudaStream_t s = sf::as_cuda(stream);
+  sf::CacheWriteView w{};
+  sf_status st = sf::cache_view_for_writer(ref_cache, s, &w);
+  if (st != SF_OK) return st;
+  const int fw = d * b_f / 32;
+  SF_REQUIRE(w.unit_words == 2 * fw, "sf_kv_append_pair_cached: the cache's units must be %d bytes (K then V words)",
+             8 * fw);
+  SF_REQUIRE(static_cast<long long>(w.num_units) >= static_cast<long long>(Hkv) * row_stride,
+             "sf_kv_append_pair_cached: the cache has fewer units than Hkv * row_stride");
+  uint32_t* stage = nullptr;
+  st = sf::cache_append_stage(ref_cache, s, static_cast<size_t>(Hkv) * 2 * fw, &stage);
+  if (st != SF_OK) return st;
+  AppendPair A{};
+  A.src[0] = k_src;
+  A.src[1] = v_src;
+  A.res[0] = k_res;
+  A.res[1] = v_res;
+  A.scale[0] = k_scale;
+  A.scale[1] = v_scale;
+  A.zero[0] = k_zero;
+  A.zero[1] = v_zero;
+  A.stage = stage;
+  A.unit_slot = w.unit_slot;
+  A.crows = w.rows;
+  A.Hkv = Hkv;
+  A.d = d;
+  A.row_stride = row_stride;
+  A.t = t;
+  A.b_r = b_r;
+  A.b_f = b_f;
+  kv_append_pair_kernel<<<dim3((Hkv + 3) / 4, 2), 128, 0, s>>>(A);
+  st = sf::check_launch("kv_append_pair_kernel");
+  if (st != SF_OK) return st;
+  st = sf::cache_mark_used(ref_cache, s);
+  if (st != SF_OK) return st;
+  // rows g * row_stride + t of the master, one per KV head
+  return sf::cache_append_flush(ref_cache, s, sf::as_cuda(side), static_cast<size_t>(t) * 2 * fw * 4,
+                                static_cast<size_t>(row_stride) * 2 * fw * 4, static_cast<size_t>(2 * fw) * 4, Hkv);
 }
 
 extern "C" sf_status sf_kv_append_cached(const float* src, int Hkv, int d, int row_stride, int t, int b_r, int b_f,

@@ -74,6 +74,23 @@ struct CacheWriteView {
   int unit_words;
 };
 sf_status cache_view_for_writer(sf_refine_cache* c, cudaStream_t stream, CacheWriteView* v);
+// A writer's device staging area of at least `words` words (allocated on the
+// first call, which must not be under stream capture); makes `stream` wait
+// for the last flush of the staging area when that flush is visible to it.
+sf_status cache_append_stage(sf_refine_cache* c, cudaStream_t stream, size_t words, uint32_t** stage);
+// Copies `height` rows of `width` bytes from the staging area (packed) to the
+// host master at byte offset dst_off with pitch dpitch, on `side` after the
+// work enqueued so far on `stream` (side == stream: in order).
+sf_status cache_append_flush(sf_refine_cache* c, cudaStream_t stream, cudaStream_t side, size_t dst_off,
+                             size_t dpitch, size_t width, int height);
+
+// Batch 8-16 GEMV with the resident part on the tensor cores (gemv_tc.cu).
+// Returns false when the shape is outside that kernel's range (the caller
+// then runs the CUDA-core kernel); otherwise launches it and reports through
+// *st.
+bool gemv_tc_try(const sf_qweight* W, const uint16_t* x, int B, const int32_t* idx, const int32_t* n,
+                 const uint32_t* ref_rows, const int32_t* row_of, int unit_words, float* y, cudaStream_t s,
+                 sf_status* st);
 
 // Batch-1 2-bit GEMV on the integer dot-product path (gemv_b1.cu).  Returns
 // false when the shape is outside that kernel's range (the caller then runs

@@ -12,7 +12,8 @@ memory with 3-bit weights and 2-bit KV).  Per layer, batch 1:
   q, k, v = refined GEMVs of n1           the weight caches' prefetch,
                                           sf_gemv_refine_batch1
   q, k rotated to position T              sf_rope_qk (q also as bf16)
-  k, v quantized, appended as token T     sf_kv_append
+  k, v quantized, appended as token T     sf_kv_append (with a KV refinement
+                                          cache: sf_kv_append_pair_cached)
   a = refined attention over T + 1        sf_attn_decode_refine (+ the KV
                                           refinement cache's prefetch)
   h = x + o(bf16(a))                      sf_round_select, GEMV, sf_norm_select
@@ -50,7 +51,7 @@ from fractions import Fraction
 import torch
 
 from . import (QKV, Batch1Jobs, RefineCache, RefineGroup, act_bytes, attn_decode_refine, attn_union_units,
-               attn_workspace_size, kv_append, kv_append_cached, norm_select, pack_batch1, quantize_nested, rope_qk,
+               attn_workspace_size, kv_append, kv_append_pair_cached, norm_select, pack_batch1, quantize_nested, rope_qk,
                round_select, silu_mul_select)
 
 MATS = ("q", "k", "v", "o", "gate", "up", "down")
@@ -348,9 +349,10 @@ class DecodeModel:
             if L["kv_cache"] is None:
                 kv_append(k, kq.res, kq.ref, kq.scale, kq.zero, self.S, T, b_r, b_f)
                 kv_append(v, vq.res, vq.ref, vq.scale, vq.zero, self.S, T, b_r, b_f)
-            else:  # the new token's refinement bits go to the host master (and a cached copy)
-                kv_append_cached(k, kq.res, kq.scale, kq.zero, L["kv_cache"], 0, self.S, T, b_r, b_f)
-                kv_append_cached(v, vq.res, vq.scale, vq.zero, L["kv_cache"], 1, self.S, T, b_r, b_f)
+            else:  # the new token's refinement bits go to the host master (and a cached copy); the
+                # master's copy runs on the KV side stream, ahead of that stream's prefetch
+                kv_append_pair_cached(k, v, kq, vq, L["kv_cache"], self.S, T, b_r, b_f, stream=main, side=self.side_kv)
+                kv_used = True
             attn_decode_refine(self.q_bf[l], L["kv"], Hkv, T + 1, k_tok, workspace=self.ws, out=self.att[l],
                                sel_out=self.sel[l], sel_n=self.sel_n[l])
             if L["kv_cache"] is not None and refine and k_tok > 0:

@@ -201,6 +201,23 @@ def test_silu_mul_select_equals_silu_mul_then_select(sf):
     assert torch.equal(act, act2)
 
 
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_silu_mul_select_wide_range(sf, seed):
+    """The fused SiLU product takes an fp32 path with a rounding test and
+    falls back to fp64 near bf16 midpoints: over gates in [-100, 100] and up
+    projections spanning 60 binades (overflow and subnormal products
+    included) it must match the stand-alone fp64 evaluation bit for bit."""
+    K, k = 32768, 983
+    rng = np.random.default_rng(700 + seed)
+    g = torch.from_numpy(rng.uniform(-100.0, 100.0, K).astype(np.float32)).cuda()
+    u = torch.from_numpy((np.sign(rng.standard_normal(K)) * 10.0 ** rng.uniform(-30, 30, K)).astype(np.float32)).cuda()
+    y_ref = sf.silu_mul(g, u)
+    y, idx, n, act = _fused_buffers(sf, K, k)
+    sf.silu_mul_select(g, u, y, k, idx, n, act)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
+
+
 def test_rope_qk_equals_two_ropes(sf):
     rng = np.random.default_rng(600)
     q = torch.from_numpy(rng.standard_normal((32, 128)).astype(np.float32)).cuda()

@@ -132,3 +132,52 @@ def test_kv_cache_refusals(sf):
     torch.cuda.synchronize()
     wc.close()
     cache.close()
+
+
+@pytest.mark.parametrize("t,b_f", [(17, 2), (0, 2), (63, 1)])
+def test_kv_append_pair_cached(sf, t, b_f):
+    """Key and value rows of token t in one launch: resident codes, scale and
+    zero bit-exact against the oracle's quantizer; the refinement words reach
+    the host master (K half, then V half of unit g S + t) through the side
+    stream's copy; every other unit of the master keeps its sentinel."""
+    Hkv, d, S, b_r = 8, 128, 64, 2
+    rng = np.random.default_rng(900 + t + b_f)
+    ksrc = (rng.standard_normal((Hkv, d)) * 2).astype(np.float32)
+    vsrc = (rng.standard_normal((Hkv, d)) * 2).astype(np.float32)
+    fw = d * b_f // 32
+    unit = 2 * fw * 4
+    master = torch.full((Hkv * S * unit,), 0xA5, dtype=torch.uint8).pin_memory()
+    cache = sf.RefineCache(Hkv * S, unit, 8, 8, master)
+    cache.preload(torch.tensor([2 * S + t, 5 * S + 3], dtype=torch.int32, device="cuda"))
+
+    rows = Hkv * S
+    kres = torch.full((rows, d * b_r // 32), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
+    vres = torch.full((rows, d * b_r // 32), 0x1E1E1E1E, dtype=torch.int32, device="cuda")
+    ksc = torch.full((rows,), 7.0, dtype=torch.float16, device="cuda")
+    kz = torch.full((rows,), 9.0, dtype=torch.float16, device="cuda")
+    vsc = torch.full((rows,), 3.0, dtype=torch.float16, device="cuda")
+    vz = torch.full((rows,), 5.0, dtype=torch.float16, device="cuda")
+
+    class _Q:  # the views the binding reads
+        def __init__(self, res, scale, zero):
+            self.res, self.scale, self.zero = res, scale, zero
+
+    side = torch.cuda.Stream()
+    sf.kv_append_pair_cached(dev(ksrc), dev(vsrc), _Q(kres, ksc, kz), _Q(vres, vsc, vz), cache, S, t, b_r, b_f,
+                             side=side)
+    side.synchronize()
+    torch.cuda.synchronize()
+    for src, res, sc, z, half in ((ksrc, kres, ksc, kz, 0), (vsrc, vres, vsc, vz, 1)):
+        want = oquant.pack_nested(oquant.quantize_nested(src, d, b_r, b_f), "by_row")
+        res_np = res.cpu().numpy().view(np.uint32).reshape(Hkv, S, -1)
+        np.testing.assert_array_equal(res_np[:, t], want["res"])
+        np.testing.assert_array_equal(sc.cpu().numpy().view(np.uint16).reshape(Hkv, S)[:, t],
+                                      want["scale"][0].view(np.uint16))
+        np.testing.assert_array_equal(z.cpu().numpy().view(np.uint16).reshape(Hkv, S)[:, t],
+                                      want["zero"][0].view(np.uint16))
+        m = master.numpy().view(np.uint32).reshape(Hkv, S, 2 * fw)
+        np.testing.assert_array_equal(m[:, t, half * fw:(half + 1) * fw], want["ref"])
+    keep = np.ones(S, bool)
+    keep[t] = False
+    assert np.all(master.numpy().reshape(Hkv, S, unit)[:, keep] == 0xA5)
+    cache.close()

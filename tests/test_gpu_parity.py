@@ -226,6 +226,63 @@ def test_gemv_store(sf, N, K, G, b_r, b_f, B, pct):
     _check_gemv(y.cpu().numpy(), y_ref, a)
 
 
+@pytest.mark.parametrize("N,K,G,b_r,b_f,B,pct", [
+    (1024, 4096, 128, 3, 1, 16, 5), (1024, 4096, 128, 3, 1, 8, 5), (96, 2048, 128, 2, 2, 9, 3),
+    (512, 6144, 128, 2, 1, 12, 5), (256, 12288, 256, 3, 1, 16, 5), (160, 1024, 128, 3, 1, 16, 0),
+])
+def test_gemv_batch_tensor_cores(sf, N, K, G, b_r, b_f, B, pct):
+    """Batches of 8-16 rows run the resident part on the tensor cores (f16
+    MMAs over exact code values, one selection for the batch): several K
+    chunks, a half-filled last row tile (N = 96, 160), group 256, and no
+    selection at all (pct 0)."""
+    W = gen_weight(700 + N + K + B, N, K)
+    x = gen_activations(710 + B, B, K, outlier_channels(19, K, count_fraction("1/2", K)), 30.0)
+    qw = sf.quantize_nested(dev(W), G, b_r, b_f)
+    xd = bf16_dev(x)
+    qz = oquant.quantize_nested(W, G, b_r, b_f)
+    if pct:
+        k = count_fraction(pct, K)
+        idx, n = sf.select_topk(xd, k)
+        y = sf.gemv_refine(qw, xd, idx, n, use_ref_store=True)
+        S = oselect.select_topk(x, k)
+    else:
+        y = sf.gemv_refine(qw, xd)
+        S = np.zeros(0, np.int64)
+    torch.cuda.synchronize()
+    y_ref, a = ogemv.gemv_refine(qz, x, S)
+    _check_gemv(y.cpu().numpy(), y_ref, a)
+
+
+def test_gemv_batch_tensor_cores_cache(sf):
+    """Qwen3-8B's gate shape at 3+1 bits, batch 16, top 5% of channels as the
+    union over the batch, 25% LRU cache, three steps; the oracle checks 128
+    sampled rows each step."""
+    N, K, G, b_r, b_f, B = 12288, 4096, 128, 3, 1, 16
+    W = gen_weight(4321, N, K)
+    qw = sf.quantize_nested(dev(W), G, b_r, b_f)
+    k = count_fraction(5, K)
+    cap = count_fraction(25, K)
+    cache = sf.RefineCache(K, N * b_f // 8, cap, min(K, B * k), _host_master(qw))  # the union: up to B k channels
+    orc = ocache.LRUCache(K, cap)
+    rows = np.sort(np.random.default_rng(7).choice(N, size=128, replace=False))
+    qz = oquant.quantize_nested(W[rows], G, b_r, b_f)
+    outl = outlier_channels(77, K, count_fraction("1/2", K))
+    for step in range(3):
+        x = gen_activations(3100 + step, B, K, outl, 30.0)
+        xd = bf16_dev(x)
+        idx, n = sf.select_topk(xd, k)
+        cache.prefetch(idx, n)
+        y = sf.gemv_refine(qw, xd, idx, n, cache=cache)
+        torch.cuda.synchronize()
+        S = oselect.select_topk(x, k)
+        want = orc.step(S.tolist())
+        got = cache.sets()
+        assert got["hits"] == want["hits"] and got["misses"] == want["misses"]
+        y_ref, a = ogemv.gemv_refine(qz, x, S)
+        _check_gemv(y.cpu().numpy()[:, rows], y_ref, a)
+    cache.close()
+
+
 @pytest.mark.parametrize("N,K,cap_pct", [(14336, 4096, 10), (4096, 14336, 10)])
 def test_gemv_full_size_cache_sampled_rows(sf, N, K, cap_pct):
     """Llama-3.1-8B gate/down shapes, 2+2, group 128, top 3%, 10% LRU cache,
