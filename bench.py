@@ -690,11 +690,14 @@ def hotpath_leg(args, sf, torch, dist, dev, world, T, phys):
 
 def qwen3_batch_leg(sf, torch, dist, dev, iters=20):
     """Qwen3-8B-shaped decode linear layers at 3+1 bits, group 128, batch 1,
-    4 and 16: top 5% of channels per row, their union refined, a 25% LRU
-    refinement cache per matrix; one layer's seven GEMVs (batch 1: the
-    tensor-core batch-1 path; 4: CUDA cores; 16: the tensor-core batch path)
-    with the selection and the caches' step, graph-timed over a pool of 8
-    seeded inputs per batch size."""
+    4 and 16: top 5% of channels per row, their union refined; one layer's
+    seven GEMVs (batch 1: the tensor-core batch-1 path; 4: CUDA cores; 16:
+    the tensor-core batch path) with the selection, graph-timed over a pool
+    of 8 seeded inputs per batch size.  "store": refinement bits read from
+    HBM; "cache": a 25% LRU refinement cache per matrix stepped with the
+    selection, its misses fetched from pinned host memory in the step (the
+    union of 16 rows' selections misses most of such a cache, so that leg
+    measures the host link)."""
     from fractions import Fraction
     from workloads import device_synth as ds
     from quantized_gemv_kv_b200.decode import count_half_up
@@ -729,39 +732,44 @@ def qwen3_batch_leg(sf, torch, dist, dev, iters=20):
             bufs[K] = (pool, k, torch.empty(B * k, dtype=torch.int32, device=dev),
                        torch.empty(1, dtype=torch.int32, device=dev))
         jobs1 = {name: sf.Batch1Jobs([(mats[name][1], caches[name], False, ys[name][0])]) for name, _, _ in shapes}
+        jobs1s = {name: sf.Batch1Jobs([(mats[name][1], None, True, ys[name][0])]) for name, _, _ in shapes}
 
-        def layer(i):
+        def layer(i, cached):
             for name, N, K in shapes:
                 pool, k, idx, n = bufs[K]
                 x = pool[i % 8]
                 sf.select_topk(x, k, idx, n)
-                caches[name].prefetch(idx, n)
+                if cached:
+                    caches[name].prefetch(idx, n)
                 if B == 1:
-                    jobs1[name].run(x, idx, n)
-                else:
+                    (jobs1 if cached else jobs1s)[name].run(x, idx, n)
+                elif cached:
                     sf.gemv_refine(mats[name][0], x, idx, n, cache=caches[name], y=ys[name])
+                else:
+                    sf.gemv_refine(mats[name][0], x, idx, n, use_ref_store=True, y=ys[name])
 
-        with torch.cuda.stream(stream):
-            for i in range(8):
-                layer(i)
-        torch.cuda.synchronize()
-        graphs = [capture(torch, lambda i=i: layer(i), stream) for i in range(8)]
-        for i in range(3):
-            graphs[i % 8].replay()
-        ms = timed(torch, dist, lambda i: graphs[i % 8].replay(), iters, stream)
-        nbytes = 0
-        for name, N, K in shapes:
-            nbytes += gemv_bytes(N, K, bufs[K][1] * B, b_r, b_f) + 2 * K * (B - 1) + 4 * N * (B - 1)
-        us = ms * 1e3 / iters
-        out[f"batch_{B}"] = {"us_per_layer": us, "tokens_per_s_per_layer": B * 1e6 / us,
-                             "effective_gbs": nbytes / (us * 1e-6) / 1e9,
-                             "path": {1: "integer tensor cores (batch 1)", 4: "CUDA cores",
-                                      16: "f16 tensor cores (batch 8-16)"}[B]}
-        del graphs
+        row = {"path": {1: "integer tensor cores (batch 1)", 4: "CUDA cores", 16: "f16 tensor cores (batch 8-16)"}[B]}
+        for cached in (False, True):
+            with torch.cuda.stream(stream):
+                for i in range(8):
+                    layer(i, cached)
+            torch.cuda.synchronize()
+            graphs = [capture(torch, lambda i=i: layer(i, cached), stream) for i in range(8)]
+            for i in range(3):
+                graphs[i % 8].replay()
+            ms = timed(torch, dist, lambda i: graphs[i % 8].replay(), iters, stream)
+            nbytes = 0
+            for name, N, K in shapes:
+                nbytes += gemv_bytes(N, K, bufs[K][1] * B, b_r, b_f) + 2 * K * (B - 1) + 4 * N * (B - 1)
+            us = ms * 1e3 / iters
+            row["cache" if cached else "store"] = {"us_per_layer": us, "tokens_per_s_per_layer": B * 1e6 / us,
+                                                   "effective_gbs": nbytes / (us * 1e-6) / 1e9}
+            del graphs
+        out[f"batch_{B}"] = row
         for c in caches.values():
             c.close()
     return {"workload": "Qwen3-8B decode linear layers (q/k/v/o 4096, gate/up/down 12288), 3+1 bits, group 128, "
-                        "top 5% per row, union refined, 25% LRU cache per matrix; one layer's seven GEMVs",
+                        "top 5% per row, union refined; one layer's seven GEMVs with the selection",
             **out}
 
 
@@ -955,8 +963,8 @@ def run_sf(args, rank, world, local_rank, dist):
         reps = 5
         t_attn = timed(torch, dist, lambda i: ga.replay(), reps, cap_stream) / reps / L * 1e-3
         achieved = attn_b / L / t_attn / 1e9
-        roofline = {"bound": "hbm", "kernel": "attention pipeline (attn_score_mma, select_compact, select_finish, "
-                                              "refine, attn_out)",
+        roofline = {"bound": "hbm", "kernel": "attention pipeline (attn_score_mma, attn_compact, attn_select, "
+                                              "attn_out)",
                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
                     "traffic": None, "peak_source": peak_src, "launch_us": t_attn * 1e6,
                     "bytes_per_launch": attn_b / L}

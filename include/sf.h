@@ -419,6 +419,20 @@ typedef struct sf_gemv_job {
 sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, const uint16_t* x, const int32_t* idx,
                                 const int32_t* n, sf_stream_t stream);
 
+/*
+ * sf_gemv_set_launch_overlap -- on != 0: sf_gemv_refine_batch1 launches with
+ *   programmatic stream serialization, so its CTAs may start while the
+ *   previous kernel on the stream still runs (typically the one-CTA producer
+ *   of x and its selection: sf_norm_select, sf_round_select,
+ *   sf_silu_mul_select) and read the weights' resident codes, scales and
+ *   zero points before it has finished; x, the selection and the refinement
+ *   rows are read only after it has completed.  The caller guarantees that
+ *   no kernel that may still be running when the GEMV starts writes those
+ *   weight arrays.  Launches that first zero y (two K halves) are never
+ *   overlapped.  Process-wide; default off.
+ */
+sf_status sf_gemv_set_launch_overlap(int on);
+
 /* ---- refined decode attention ----------------------------------------- */
 
 /* Quantized K and V (views).  Rows are token-heads ordered [Hkv][S], token t

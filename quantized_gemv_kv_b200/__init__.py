@@ -114,6 +114,7 @@ _SIGS = {
     "sf_rope_qk": ([_p, _i, _p, _i, _i, _i, ctypes.c_double, _p, _p], _i),
     "sf_kv_append": ([_p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p], _i),
     "sf_kv_append_cached": ([_p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _i, _p], _i),
+    "sf_gemv_set_launch_overlap": ([_i], _i),
     "sf_kv_append_pair_cached": ([_p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -521,6 +522,20 @@ class Batch1Jobs:
         """x: the bf16 row; (idx, n): its selection (None: nothing selected)."""
         _check(_lib.sf_gemv_refine_batch1(ctypes.cast(self._arr, _p), self.count, _ptr(x), _ptr(idx), _ptr(n),
                                           _stream(stream)))
+
+
+_gemv_overlap = False
+
+
+def gemv_set_launch_overlap(on: bool) -> bool:
+    """``sf_gemv_set_launch_overlap``: batch-1 GEMV launches may overlap the
+    previous kernel (which must not write the weights).  Returns the
+    previous setting."""
+    global _gemv_overlap
+    prev = _gemv_overlap
+    _check(_lib.sf_gemv_set_launch_overlap(1 if on else 0))
+    _gemv_overlap = bool(on)
+    return prev
 
 
 def gemv_refine_batch1(jobs, x: torch.Tensor, idx: torch.Tensor | None = None, n: torch.Tensor | None = None,

@@ -56,6 +56,10 @@ struct FusedArgs {
 };
 
 __global__ void __launch_bounds__(kThreads) produce_select_kernel(const __grid_constant__ FusedArgs A) {
+  // a GEMV launched after this kernel with programmatic stream serialization
+  // may start streaming its weight codes now; it waits for this grid before
+  // it reads the row or the selection
+  asm volatile("griddepcontrol.launch_dependents;\n" ::);
   extern __shared__ __align__(16) uint8_t smem[];
   const int K = A.K, tid = threadIdx.x;
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [K]

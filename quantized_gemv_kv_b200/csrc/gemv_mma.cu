@@ -46,6 +46,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "act.cuh"  // bf16_exponent, bf16_fixed
 #include "sf_internal.h"
@@ -88,6 +89,9 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+// Programmatic dependent launch: returns once the preceding kernel (the
+// producer of x and the selection) has completed and its writes are visible.
+__device__ __forceinline__ void pdl_wait_gemv() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
@@ -299,7 +303,10 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
   // ---- per-warp setup, from x and the selection list: the B fragments of
   // the slice's fixed-point activations, the group scalars, the slice's
   // selected channels, the correction MMA's B fragments (x of the listed
-  // channels, high and low)
+  // channels, high and low).  Launched with programmatic stream
+  // serialization, the kernel may have started before the producer of x and
+  // the selection finished: the code copies above need nothing it writes.
+  pdl_wait_gemv();
   int n_all = a.idx != nullptr ? *a.n_sel : 0;
   n_all = n_all < 0 ? 0 : n_all;
 #pragma unroll
@@ -620,6 +627,8 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
   cp_async_wait<0>();
 }
 
+std::atomic<int> g_gemv_overlap{0};
+
 // (slices per warp, K halves) for K / 256 slices: at most 16 warps per CTA.
 bool pick_split(int nslice, int* spw, int* ksplit) {
   const int cand[4][2] = {{1, 1}, {1, 2}, {2, 1}, {2, 2}};
@@ -756,7 +765,20 @@ extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, c
   const dim3 grid(nrow_cta * ksplit), block(32 * warps);
   auto launch = [&](auto kern, size_t smem) -> sf_status {
     SF_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
-    kern<<<grid, block, smem, s>>>(a);
+    // programmatic stream serialization: the CTAs may start streaming codes
+    // while the previous kernel (typically the one-CTA producer of x) runs;
+    // not when memsets of y were just enqueued (ksplit > 1)
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = (ksplit > 1 || !g_gemv_overlap.load(std::memory_order_relaxed)) ? 0 : 1;
+    SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kern, a));
     return sf::check_launch("gemv_mma_kernel");
   };
   sf_status st;
@@ -778,5 +800,10 @@ extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, c
       const sf_status m = sf::cache_mark_used(jobs[i].cache, s);
       if (m != SF_OK) return m;
     }
+  return SF_OK;
+}
+
+extern "C" sf_status sf_gemv_set_launch_overlap(int on) {
+  g_gemv_overlap.store(on != 0 ? 1 : 0, std::memory_order_relaxed);
   return SF_OK;
 }

@@ -9,6 +9,8 @@
 // to tau are taken in ascending channel order until k are chosen (an ordered
 // scan), which is the "ties to the lower index" rule.  A final ordered
 // compaction writes the union in ascending order.
+#include <cooperative_groups.h>
+
 #include "act.cuh"
 #include "block_scan.cuh"
 #include "select_row.cuh"
@@ -254,6 +256,66 @@ select_random_kernel(int K, int k, uint64_t seed, uint64_t step, int32_t* __rest
   sfd::select_row_block(xs, flags, K, k, idx, n, nullptr);
 }
 
+// ---- the union over a batch, one CTA per row in one thread-block cluster ---
+//
+// CTA b selects row b's top k (select_row_block, its list in idx_out's row b
+// as scratch) and marks them in the union bitmask held in rank 0's shared
+// memory (distributed-shared-memory atomics); rank 0 then lists the union in
+// ascending order into idx_out (the rows' scratch lists are read before).
+constexpr int kUnionMaxWords = kActMaxK / 32;
+
+__global__ void __launch_bounds__(kThreads)
+select_union_cluster_kernel(const uint16_t* __restrict__ x, int K, int k, int32_t* __restrict__ idx_out,
+                            int32_t* __restrict__ n_out) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [K]
+  uint8_t* flags = smem + 2 * K;                     // [K]
+  __shared__ uint32_t mask[kUnionMaxWords];          // rank 0's: the union
+  __shared__ int nrow, bad_any, scan_scratch[33];
+  const int b = static_cast<int>(cl.block_rank()), tid = threadIdx.x;
+  const int nw = (K + 31) >> 5;
+  if (b == 0) {
+    for (int w = tid; w < nw; w += kThreads) mask[w] = 0u;
+    if (tid == 0) bad_any = 0;
+  }
+  const uint16_t* xr = x + static_cast<size_t>(b) * K;
+  for (int j = tid; j < K; j += kThreads) xs[j] = xr[j];
+  __syncthreads();
+  int32_t* mine = idx_out + static_cast<size_t>(b) * k;
+  sfd::select_row_block(xs, flags, K, k, mine, &nrow, nullptr);
+  __syncthreads();  // this row's list (global) and count are complete
+  cl.sync();        // rank 0's bitmask is cleared
+  uint32_t* m0 = cl.map_shared_rank(mask, 0);
+  const int nr = nrow;
+  if (nr < 0) {
+    if (tid == 0) atomicOr(cl.map_shared_rank(&bad_any, 0), 1);
+  } else {
+    for (int e = tid; e < nr; e += kThreads) {
+      const int j = mine[e];
+      atomicOr(m0 + (j >> 5), 1u << (j & 31));
+    }
+  }
+  cl.sync();  // the union is complete; every row's scratch list has been read
+  if (b != 0) return;
+  const int per = (nw + kThreads - 1) / kThreads;
+  const int w0 = min(nw, tid * per), w1 = min(nw, w0 + per);
+  int c = 0;
+  for (int w = w0; w < w1; ++w) c += __popc(mask[w]);
+  int total;
+  int pos = sfd::block_exclusive_scan(c, scan_scratch, &total);
+  for (int w = w0; w < w1; ++w) {
+    uint32_t bits = mask[w];
+    while (bits) {
+      const int bi = __ffs(bits) - 1;
+      bits &= bits - 1u;
+      idx_out[pos++] = 32 * w + bi;
+    }
+  }
+  if (tid == 0) *n_out = bad_any ? -1 : total;
+}
+
 }  // namespace
 
 extern "C" sf_status sf_select_random(int K, int k, uint64_t seed, uint64_t step, int32_t* idx_out, int32_t* n_out,
@@ -273,6 +335,27 @@ extern "C" sf_status sf_select_topk(const uint16_t* x, int B, int K, int k, int3
   SF_REQUIRE(B >= 1 && B <= kMaxRows, "sf_select_topk: B must be in [1, %d]", kMaxRows);
   SF_REQUIRE(K >= 1 && K <= 65536, "sf_select_topk: K must be in [1, 65536]");
   SF_REQUIRE(k >= 0 && k <= K, "sf_select_topk: k must be in [0, K]");
+  if (B >= 2 && K <= kActMaxK && k >= 1) {
+    // one CTA per row, the union through a thread-block cluster
+    const size_t smem = 3 * static_cast<size_t>(K);
+    SF_CHECK_CUDA(cudaFuncSetAttribute(select_union_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem)));
+    SF_CHECK_CUDA(cudaFuncSetAttribute(select_union_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(B));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = sf::as_cuda(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(B);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, select_union_cluster_kernel, x, K, k, idx_out, n_out));
+    return sf::check_launch("select_union_cluster_kernel");
+  }
   const size_t smem = static_cast<size_t>((K + 15) & ~15) + sizeof(int) * kMaxRows * (256 + 128);
   SF_CHECK_CUDA(cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
   select_topk_kernel<<<1, kThreads, smem, sf::as_cuda(stream)>>>(x, B, K, k, idx_out, n_out, nullptr);

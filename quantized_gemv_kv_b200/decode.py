@@ -51,7 +51,7 @@ from fractions import Fraction
 import torch
 
 from . import (QKV, Batch1Jobs, RefineCache, RefineGroup, act_bytes, attn_decode_refine, attn_union_units,
-               attn_workspace_size, kv_append, kv_append_pair_cached, norm_select, pack_batch1, quantize_nested, rope_qk,
+               attn_workspace_size, gemv_set_launch_overlap, kv_append, kv_append_pair_cached, norm_select, pack_batch1, quantize_nested, rope_qk,
                round_select, silu_mul_select)
 
 MATS = ("q", "k", "v", "o", "gate", "up", "down")
@@ -313,6 +313,13 @@ class DecodeModel:
         every layer's cache); x_in holds the token's embedding.  refine=False
         is the quantization-only baseline: same kernels, nothing selected,
         fetched or refined."""
+        prev = gemv_set_launch_overlap(True)  # no kernel of the step writes weights
+        try:
+            self._step(T, refine)
+        finally:
+            gemv_set_launch_overlap(prev)
+
+    def _step(self, T: int, refine: bool) -> None:
         s = self.s
         if T + 1 > self.S:
             raise ValueError("the KV cache is full")

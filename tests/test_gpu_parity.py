@@ -92,7 +92,7 @@ def test_quantize_worked_examples(sf):
 # ---- selection ------------------------------------------------------------
 
 @pytest.mark.parametrize("B,K,pct", [(1, 512, 5), (1, 4096, 3), (1, 14336, 3), (4, 4096, 5), (16, 12288, 5),
-                                     (3, 1000, 10), (1, 64, 100)])
+                                     (3, 1000, 10), (1, 64, 100), (2, 32768, 3), (16, 32768, 1), (16, 40000, 2)])
 def test_select_exact(sf, B, K, pct):
     k = count_fraction(pct, K)
     x = gen_activations(200 + K + B, B, K, outlier_channels(7, K, max(1, K // 200)), 30.0)
