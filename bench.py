@@ -691,8 +691,8 @@ def hotpath_leg(args, sf, torch, dist, dev, world, T, phys):
 def qwen3_batch_leg(sf, torch, dist, dev, iters=20):
     """Qwen3-8B-shaped decode linear layers at 3+1 bits, group 128, batch 1,
     4 and 16: top 5% of channels per row, their union refined; one layer's
-    seven GEMVs (batch 1: the tensor-core batch-1 path; 4: CUDA cores; 16:
-    the tensor-core batch path) with the selection, graph-timed over a pool
+    seven GEMVs (batch 1: the integer tensor-core batch-1 path; 4 and 16:
+    the f16 tensor-core batch path) with the selection, graph-timed over a pool
     of 8 seeded inputs per batch size.  "store": refinement bits read from
     HBM; "cache": a 25% LRU refinement cache per matrix stepped with the
     selection, its misses fetched from pinned host memory in the step (the
@@ -748,7 +748,8 @@ def qwen3_batch_leg(sf, torch, dist, dev, iters=20):
                 else:
                     sf.gemv_refine(mats[name][0], x, idx, n, use_ref_store=True, y=ys[name])
 
-        row = {"path": {1: "integer tensor cores (batch 1)", 4: "CUDA cores", 16: "f16 tensor cores (batch 8-16)"}[B]}
+        row = {"path": {1: "integer tensor cores (batch 1)", 4: "f16 tensor cores (batch 2-16)",
+                        16: "f16 tensor cores (batch 2-16)"}[B]}
         for cached in (False, True):
             with torch.cuda.stream(stream):
                 for i in range(8):

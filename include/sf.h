@@ -282,6 +282,11 @@ sf_status sf_refine_group_destroy(sf_refine_group* g);
  *          NULL and W->ref NULL: resident-only GEMV (idx, n ignored).
  * Constraints: 1 <= B <= 16, b_r in {2,3}, b_f in {1,2}, G % 32 == 0,
  *   K % G == 0, K <= 32768, N % 32 == 0.
+ * Paths: B = 1 the integer dot-product kernel (2-bit) or the CUDA cores;
+ *   2 <= B <= 16 with G % 128 == 0 and 16-byte aligned res and x the f16
+ *   tensor cores (x scaled per 2048-channel chunk and row by a power of two
+ *   and converted to f16: exact for entries within 28 binades of the row's
+ *   maximum in the chunk), else the CUDA cores.
  * Accuracy: |y - exact| <= 2e-3 * sum_j |w_eff[i][j] x[b][j]| per output.
  */
 sf_status sf_gemv_refine(const sf_qweight* W, const uint16_t* x, int B, const int32_t* idx,

@@ -265,6 +265,7 @@ attn_score_mma_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict
     }
   }
   cp_async_wait_attn<0>();
+  pdl_wait();  // the cleared counters (everything read above was final before the clear began)
   smx = warp_max(smx);
   szx = warp_max(szx);
   if (lane == 0) {
@@ -1219,6 +1220,17 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
   }
 }
 
+// Clears the workspace's per-call counters and accumulators (a plain launch:
+// it starts after the previous kernel of the stream); the score pass, launched
+// with programmatic stream serialization, may start meanwhile and waits for
+// it only before its first update of the cleared words.
+__global__ void ws_clear_kernel(uint4* __restrict__ p, size_t n16) {
+  pdl_launch_dependents();
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    p[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 __global__ void fill_all_kernel(int T, int grp, int k, int words_t, uint32_t* umask, int32_t* sel_out,
                                 int32_t* sel_n, uint32_t* mkey) {
   const int g = blockIdx.y;
@@ -1265,7 +1277,13 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
   const int grp = GRP;
   const int sms = sf::sm_count();
 
-  SF_CHECK_CUDA(cudaMemsetAsync(ws + L.smax, 0, L.total - L.smax, s));
+  {
+    const size_t n16 = (L.total - L.smax) / 16;  // offsets are multiples of 256 bytes
+    const int blocks = static_cast<int>(std::min<size_t>((n16 + 255) / 256, static_cast<size_t>(2 * sms)));
+    ws_clear_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<uint4*>(ws + L.smax), n16);
+    const sf_status cs = sf::check_launch("ws_clear_kernel");
+    if (cs != SF_OK) return cs;
+  }
   // pass A: about two CTAs per SM, each a contiguous range of <= kScMaxTok tokens
   const int want_a = std::max((2 * sms + Hkv - 1) / Hkv, (T + kScMaxTok - 1) / kScMaxTok);
   const int tpc = ((T + want_a - 1) / want_a + 15) / 16 * 16;
@@ -1278,8 +1296,20 @@ sf_status run(const uint16_t* q, int Hq, int Hkv, int T, const sf_qkv* kv, int k
   int32_t* ccnt = reinterpret_cast<int32_t*>(ws + L.ccnt);
   SF_CHECK_CUDA(cudaFuncSetAttribute(attn_score_mma_kernel<GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(score_smem(GRP))));
-  attn_score_mma_kernel<GRP><<<ga, kScThreads, score_smem(GRP), s>>>(q, kv->k_res, kv->k_scale, kv->k_zero, T, S,
-                                                                     tpc, score, smax, hist, amaxu, mkey);
+  {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = ga;
+    cfg.blockDim = dim3(kScThreads);
+    cfg.dynamicSmemBytes = score_smem(GRP);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, attn_score_mma_kernel<GRP>, q, kv->k_res, kv->k_scale, kv->k_zero, T, S,
+                                     tpc, score, smax, hist, amaxu, mkey));
+  }
   sf_status st = sf::check_launch("attn_score_mma_kernel");
   if (st != SF_OK) return st;
   if (selecting) {

@@ -228,7 +228,7 @@ extern "C" sf_status sf_gemv_refine(const sf_qweight* W, const uint16_t* x, int 
   }
   sf_status st = SF_OK;
   if (!(B == 1 && sf::gemv_b1_try(W, x, idx, n, ref_rows, row_of, unit_words, nmax, y, s, &st)) &&
-      !(B >= 8 && sf::gemv_tc_try(W, x, B, idx, n, ref_rows, row_of, unit_words, y, s, &st)))
+      !(B >= 2 && sf::gemv_tc_try(W, x, B, idx, n, ref_rows, row_of, unit_words, y, s, &st)))
     st = W->b_r == 2 ? launch_br<2, 0>(W, x, B, idx, n, ref_rows, row_of, unit_words, y, s)
                      : launch_br<3, 0>(W, x, B, idx, n, ref_rows, row_of, unit_words, y, s);
   if (st != SF_OK) return st;

@@ -1,4 +1,4 @@
-// sf_gemv_refine for batches of 8 to 16 rows on the tensor cores.
+// sf_gemv_refine for batches of 2 to 16 rows on the tensor cores.
 //
 //   y[b][i] = sum_j x[b][j] w_res[i][j] + sum_{j in S} x[b][j] s_{g(j),i} (q_f[i][j] - m_f)
 //
@@ -6,7 +6,10 @@
 // selection S is one set for the whole batch, rag-lover.com explainer of
 // StrataFlux, 解説).  With eight or more rows the resident part is a dense
 // contraction worth the tensor cores, and so is the refinement correction
-// once the union of the rows' selections is large.
+// once the union of the rows' selections is large.  Below eight rows the
+// MMA's unused columns cost nothing that matters: unpacking 2-3-bit codes
+// for CUDA-core FMAs is instruction-bound, one MMA per 16x16 codes is not,
+// and the bytes read are the same.
 //
 // Resident part on mma.m16n8k16 (f16 in, f32 accumulate), MMA rows = output
 // rows, MMA columns = batch rows (two n-tiles for more than eight):
@@ -484,7 +487,7 @@ namespace sf {
 bool gemv_tc_try(const sf_qweight* W, const uint16_t* x, int B, const int32_t* idx, const int32_t* n,
                  const uint32_t* ref_rows, const int32_t* row_of, int unit_words, float* y, cudaStream_t s,
                  sf_status* st) {
-  if (B < 8 || B > 16 || W->G % 128 != 0 || W->K % 128 != 0 || !aligned(W->res, 16) || !aligned(x, 16)) return false;
+  if (B < 2 || B > 16 || W->G % 128 != 0 || W->K % 128 != 0 || !aligned(W->res, 16) || !aligned(x, 16)) return false;
   if (B <= 8)
     *st = W->b_r == 2 ? launch_tc<2, 1>(W, x, B, idx, n, ref_rows, row_of, unit_words, y, s)
                       : launch_tc<3, 1>(W, x, B, idx, n, ref_rows, row_of, unit_words, y, s);

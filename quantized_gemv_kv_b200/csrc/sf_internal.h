@@ -84,7 +84,7 @@ sf_status cache_append_stage(sf_refine_cache* c, cudaStream_t stream, size_t wor
 sf_status cache_append_flush(sf_refine_cache* c, cudaStream_t stream, cudaStream_t side, size_t dst_off,
                              size_t dpitch, size_t width, int height);
 
-// Batch 8-16 GEMV with the resident part on the tensor cores (gemv_tc.cu).
+// Batch 2-16 GEMV on the tensor cores (gemv_tc.cu).
 // Returns false when the shape is outside that kernel's range (the caller
 // then runs the CUDA-core kernel); otherwise launches it and reports through
 // *st.

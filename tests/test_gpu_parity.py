@@ -210,6 +210,7 @@ def test_gemv_linear_512_preloaded_cache(sf):
 @pytest.mark.parametrize("N,K,G,b_r,b_f,B,pct", [
     (1024, 4096, 128, 3, 1, 1, 5), (1024, 4096, 128, 3, 1, 4, 5), (512, 4096, 128, 3, 1, 16, 5),
     (256, 14336, 128, 2, 2, 1, 3), (4096, 1024, 128, 2, 2, 2, 3), (96, 2048, 64, 2, 1, 7, 5),
+    (256, 2048, 64, 3, 1, 16, 5), (128, 1024, 32, 2, 2, 9, 5),
 ])
 def test_gemv_store(sf, N, K, G, b_r, b_f, B, pct):
     W = gen_weight(300 + N + K + B, N, K)
