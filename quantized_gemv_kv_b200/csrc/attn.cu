@@ -831,7 +831,7 @@ struct OutCfg {
   static constexpr size_t ulist_bytes = static_cast<size_t>(kSub) * 2;
   static constexpr size_t vref_bytes = static_cast<size_t>(kUCap) * kWordsPerRow * 4;
   static constexpr size_t smem = alpha_bytes + ring_bytes + ulist_bytes + vref_bytes;
-  static_assert(alpha_bytes >= static_cast<size_t>(kOW) * GRP * D * 4, "per-warp output tiles must fit the weight tile");
+  static_assert(alpha_bytes >= static_cast<size_t>(kOW) * 16 * 8 * NT * 8 * 4, "per-warp output tiles must fit the weight tile");
   static_assert(kSub / 32 <= kOutThreads, "the union scan takes a bitmask word per thread");
 };
 
@@ -964,16 +964,6 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
     for (int w = 0; w < 8; ++w)
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[nt][w][c] = 0.0f;
-  // head of each of this lane's accumulator columns (-1: padding column)
-  int colh[NT][2];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int n = nt * 8 + 2 * tig + c;
-      colh[nt][c] = n < GRP ? n : (n < 2 * GRP ? n - GRP : -1);
-    }
-
   for (int c0 = t0s; c0 < t1s; c0 += kSub) {
     const int n = min(t1s, c0 + kSub) - c0;
     const int ntile = (n + 15) >> 4;
@@ -1100,33 +1090,31 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
     __syncthreads();  // weights and the list are rewritten by the next sub-chunk
   }
 
-  // this warp's output tile ww[head][dim] (in units of the code part, which
-  // carries the factor 4^e of the dim's fragment position: uo enters as
-  // uo 4^e / 2^b_f) in the dead weight tile, written in three phases whose
-  // stores within a warp never collide (high columns, then remainder
-  // columns, then the refined corrections); summed over warps below
+  // this warp's output tile (in units of the code part, which carries the
+  // factor 4^e of the dim's fragment position: uo enters as uo 4^e / 2^b_f)
+  // in the dead weight tile: row (s, g8) for MMA s's rows g8 (s < 8) and
+  // g8 + 8 (s + 8), i.e. dims 16 g8 + s and 16 g8 + 8 + s, columns = the
+  // MMA's columns (head high parts, then remainders); a lane's two adjacent
+  // columns go in one 8-byte store, and a store instruction's 32 lanes
+  // cover 64 consecutive words (no bank conflict).  Summed over warps below.
+  constexpr int kCols = NT * 8;
+  auto tile_row = [](int dim) { return ((dim & 15) << 3) | (dim >> 4); };  // dim = 16 g8 + r -> r * 8 + g8
   __syncthreads();  // every warp is done with the weight tile
-  float* ww = reinterpret_cast<float*>(smem) + warp * GRP * D;
+  float* ww = reinterpret_cast<float*>(smem) + warp * 16 * 8 * kCols;
 #pragma unroll
-  for (int ph = 0; ph < 2; ++ph) {
+  for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int w = 0; w < 8; ++w)
 #pragma unroll
-      for (int w = 0; w < 8; ++w)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int n = nt * 8 + 2 * tig + (c & 1);
-          const int hh = colh[nt][c & 1];
-          if (hh < 0 || (n < GRP) != (ph == 0)) continue;
-          float* dst = &ww[hh * D + 16 * g8 + w + 8 * (c >> 1)];  // MMA w, row g8 (+ 8)
-          *dst = ph == 0 ? acc[nt][w][c] : *dst + acc[nt][w][c];
-        }
-    __syncwarp();
-  }
+      for (int hh = 0; hh < 2; ++hh)
+        *reinterpret_cast<float2*>(ww + ((w + 8 * hh) * 8 + g8) * kCols + nt * 8 + 2 * tig) =
+            make_float2(acc[nt][w][2 * hh], acc[nt][w][2 * hh + 1]);
+  __syncwarp();
 #pragma unroll
   for (int h = 0; h < GRP; ++h)
 #pragma unroll
-    for (int dd = 0; dd < 4; ++dd) ww[h * D + 4 * lane + dd] += (0.25f * vpos_mul(4 * lane + dd)) * uo[h][dd];
+    for (int dd = 0; dd < 4; ++dd)
+      ww[tile_row(4 * lane + dd) * kCols + h] += (0.25f * vpos_mul(4 * lane + dd)) * uo[h][dd];
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
     const float l = warp_sum(lsum[h]), cs = warp_sum(csum[h]), a = warp_sum(asum[h]);
@@ -1137,26 +1125,36 @@ attn_out_kernel(const uint16_t* __restrict__ q, const uint32_t* __restrict__ k_r
     }
   }
   __syncthreads();
+  if (tid < GRP) {  // the CTA's weight sums per head: L, the offset part Cs and sum(alpha) A
+    float L = 0.0f, Cs = 0.0f, A = 0.0f;
+    for (int w = 0; w < kOW; ++w) {
+      L += red2[w][tid];
+      Cs += red2[w][GRP + tid];
+      A += red2[w][2 * GRP + tid];
+    }
+    red2[0][tid] = L;
+    red2[0][GRP + tid] = Cs;
+    red2[0][2 * GRP + tid] = A;
+  }
+  __syncthreads();
   float* pg = part + static_cast<size_t>(g) * GRP * splits * (D + 2);
+  const float* wt = reinterpret_cast<const float*>(smem);
   for (int e = tid; e < GRP * (D + 2); e += kOutThreads) {
     const int h = e / (D + 2), j = e % (D + 2);
     float v;
     if (j == 0) {
       v = Msh[h];
+    } else if (j == 1) {
+      v = red2[0][h];
     } else {
-      float L = 0.0f, Cs = 0.0f, A = 0.0f;
-      for (int w = 0; w < kOW; ++w) {
-        L += red2[w][h];
-        Cs += red2[w][GRP + h];
-        A += red2[w][2 * GRP + h];
-      }
       // resident value s (2^b_f c + m_f - z): code part 4 (acc - 1024 A) 4^-e,
-      // offset part Cs
+      // offset part Cs; acc = the high and remainder columns of head h
+      const int r = tile_row(j - 2) * kCols;
       float o = 0.0f;
-      if (j >= 2)
-        for (int w = 0; w < kOW; ++w) o += reinterpret_cast<const float*>(smem)[(w * GRP + h) * D + j - 2];
-      const float f = j >= 2 ? vpos_inv(j - 2) : 1.0f;
-      v = j == 1 ? L : fmaf(4.0f * f, o, fmaf(-4096.0f * f, A, Cs));
+#pragma unroll
+      for (int w = 0; w < kOW; ++w) o += wt[w * 16 * 8 * kCols + r + h] + wt[w * 16 * 8 * kCols + r + GRP + h];
+      const float f = vpos_inv(j - 2);
+      v = fmaf(4.0f * f, o, fmaf(-4096.0f * f, red2[0][2 * GRP + h], red2[0][GRP + h]));
     }
     pg[(static_cast<size_t>(h) * splits + split) * (D + 2) + j] = v;
   }
