@@ -692,7 +692,8 @@ def qwen3_batch_leg(sf, torch, dist, dev, iters=20):
     """Qwen3-8B-shaped decode linear layers at 3+1 bits, group 128, batch 1,
     4 and 16: top 5% of channels per row, their union refined; one layer's
     seven GEMVs (batch 1: the integer tensor-core batch-1 path; 4 and 16:
-    the f16 tensor-core batch path) with the selection, graph-timed over a pool
+    the f16 tensor-core batch path) with the selection of each distinct
+    input (q/k/v share one, gate/up another), graph-timed over a pool
     of 8 seeded inputs per batch size.  "store": refinement bits read from
     HBM; "cache": a 25% LRU refinement cache per matrix stepped with the
     selection, its misses fetched from pinned host memory in the step (the
@@ -738,7 +739,8 @@ def qwen3_batch_leg(sf, torch, dist, dev, iters=20):
             for name, N, K in shapes:
                 pool, k, idx, n = bufs[K]
                 x = pool[i % 8]
-                sf.select_topk(x, k, idx, n)
+                if name in ("q", "o", "gate", "down"):  # k/v share q's input, up shares gate's
+                    sf.select_topk(x, k, idx, n)
                 if cached:
                     caches[name].prefetch(idx, n)
                 if B == 1:
@@ -770,7 +772,7 @@ def qwen3_batch_leg(sf, torch, dist, dev, iters=20):
         for c in caches.values():
             c.close()
     return {"workload": "Qwen3-8B decode linear layers (q/k/v/o 4096, gate/up/down 12288), 3+1 bits, group 128, "
-                        "top 5% per row, union refined; one layer's seven GEMVs with the selection",
+                        "top 5% per row, union refined; one layer's seven GEMVs with the selection of each input",
             **out}
 
 
