@@ -412,9 +412,11 @@ typedef struct sf_gemv_job {
  * Constraints: b_r in {2, 3}, b_f in {1, 2}, b_r + b_f <= 4, G == 128, all
  * jobs share K, G and bit widths; N % 16 == 0; K a multiple of 256 whose
  * K/256 slices split into at most 16 warps of one or two slices, in one or
- * two K halves (4096 and 14336 qualify; with two halves the partial sums are
- * added onto zeroed outputs, an order-independent fp32 addition); weight
- * arrays 16-byte aligned; 3-bit codes given as res_b1.  SF_EINVAL otherwise.
+ * two K halves (4096 and 14336 qualify; two halves run as the two thread
+ * blocks of a cluster, which add their partial sums through distributed
+ * shared memory: y = half 0 + half 1, one fp32 addition, and y needs no
+ * zeroing); weight arrays 16-byte aligned; 3-bit codes given as res_b1.
+ * SF_EINVAL otherwise.
  * Accuracy: as sf_gemv_refine, given that within every 128-channel group
  * the channels that matter are within 2^14 of the group's largest |x|: x is
  * taken in fixed point relative to that maximum, with an absolute error of
@@ -423,6 +425,48 @@ typedef struct sf_gemv_job {
  */
 sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, const uint16_t* x, const int32_t* idx,
                                 const int32_t* n, sf_stream_t stream);
+
+/* The producer of a batch-1 GEMV's input row when the GEMV launch computes
+ * the row itself (sf_gemv_refine_batch1_produce).  Ops: */
+enum { SF_PRODUCE_NORM = 0, SF_PRODUCE_ROUND = 1, SF_PRODUCE_SILU_MUL = 2 };
+typedef struct sf_gemv_producer {
+  int op;             /* SF_PRODUCE_* */
+  int k;              /* channels of the row to select (0: none) */
+  float eps;          /* SF_PRODUCE_NORM: the RMSNorm epsilon, >= 0 */
+  const float* x;     /* fp32 [K], device: NORM the residual, ROUND the row, SILU_MUL the gate g */
+  const float* delta; /* NORM: added to x first (fp32 [K]); may be NULL */
+  const float* w;     /* NORM: the RMSNorm weights, fp32 [K] */
+  const float* u;     /* SILU_MUL: the up projection, fp32 [K] */
+  float* x_out;       /* NORM: receives x + delta (fp32 [K]); may be NULL; must not overlap x or delta */
+  uint16_t* y;        /* out: the bf16 row [K], 16-byte aligned */
+  int32_t* idx;       /* out: its selection, ascending, room for k entries */
+  int32_t* n;         /* out: the selection's length (-1: the row holds a NaN or Inf) */
+} sf_gemv_producer;
+
+/*
+ * sf_gemv_refine_batch1_produce -- sf_gemv_refine_batch1 whose input row and
+ * selection are made inside the launch: the same results, bit for bit, as
+ * the producer's stand-alone call followed by sf_gemv_refine_batch1(jobs,
+ * count, p->y, p->idx, p->n):
+ *   SF_PRODUCE_NORM     -- sf_norm_select(x, delta, w, K, eps, y, k, idx, n,
+ *                          NULL) with the updated residual written to x_out
+ *                          instead of in place (x is not modified);
+ *   SF_PRODUCE_ROUND    -- sf_round_select(x, K, y, k, idx, n, NULL);
+ *   SF_PRODUCE_SILU_MUL -- sf_silu_mul_select(x, u, K, y, k, idx, n, NULL).
+ * Every thread block computes the row and its selection (the explainer of
+ * StrataFlux, 解説: refinement where the input activation is large) while
+ * its first weight codes stream in, so no one-block producer launch precedes
+ * the GEMV; y, idx and n are written for later readers (a cache prefetch
+ * after the launch, for instance).  Constraints: those of
+ * sf_gemv_refine_batch1; K <= 32768; 0 <= k <= K and k within the launch's
+ * scratch (several thousand entries at the Llama shapes; SF_EINVAL beyond);
+ * caches, if any, in the deadline reading (a blocking prefetch needs the
+ * selection before the launch).  With sf_gemv_set_launch_overlap on, the
+ * launch may start while the previous kernel runs and reads x, delta, w and u
+ * only after that kernel has completed.
+ */
+sf_status sf_gemv_refine_batch1_produce(const sf_gemv_job* jobs, int count, const sf_gemv_producer* p,
+                                        sf_stream_t stream);
 
 /*
  * sf_gemv_set_launch_overlap -- on != 0: sf_gemv_refine_batch1 launches with
@@ -433,8 +477,7 @@ sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, const uint16
  *   zero points before it has finished; x, the selection and the refinement
  *   rows are read only after it has completed.  The caller guarantees that
  *   no kernel that may still be running when the GEMV starts writes those
- *   weight arrays.  Launches that first zero y (two K halves) are never
- *   overlapped.  Process-wide; default off.
+ *   weight arrays.  Process-wide; default off.
  */
 sf_status sf_gemv_set_launch_overlap(int on);
 

@@ -59,6 +59,14 @@ class _GemvJob(ctypes.Structure):
     _fields_ = [("W", ctypes.POINTER(_QWeight)), ("cache", _p), ("use_ref_store", _i), ("y", _p), ("res_b1", _p)]
 
 
+class _GemvProducer(ctypes.Structure):
+    _fields_ = [("op", _i), ("k", _i), ("eps", ctypes.c_float), ("x", _p), ("delta", _p), ("w", _p), ("u", _p),
+                ("x_out", _p), ("y", _p), ("idx", _p), ("n", _p)]
+
+
+PRODUCE_NORM, PRODUCE_ROUND, PRODUCE_SILU_MUL = 0, 1, 2
+
+
 class _SelectJob(ctypes.Structure):
     _fields_ = [("x", _p), ("K", _i), ("k", _i), ("idx_out", _p), ("n_out", _p), ("act", _p)]
 
@@ -98,6 +106,7 @@ _SIGS = {
     "sf_act_prepare": ([_p, _i, _p, _p], _i),
     "sf_select_topk_act_many": ([_p, _i, _p], _i),
     "sf_gemv_refine_batch1": ([_p, _i, _p, _p, _p, _p], _i),
+    "sf_gemv_refine_batch1_produce": ([_p, _i, _p, _p], _i),
     "sf_gemv_pack_batch1": ([_p, _i, _i, _i, _p, _p], _i),
     "sf_attn_workspace_size": ([_i, _i, _i, _i, _i, ctypes.POINTER(_sz)], _i),
     "sf_attn_decode_refine": ([_p, _i, _i, _i, _i, ctypes.POINTER(_QKV), _i, _p, _p, _p, _p, _sz, _p], _i),
@@ -522,6 +531,22 @@ class Batch1Jobs:
         """x: the bf16 row; (idx, n): its selection (None: nothing selected)."""
         _check(_lib.sf_gemv_refine_batch1(ctypes.cast(self._arr, _p), self.count, _ptr(x), _ptr(idx), _ptr(n),
                                           _stream(stream)))
+
+    def run_produce(self, op: int, x: torch.Tensor, y: torch.Tensor, k: int, idx: torch.Tensor, n: torch.Tensor,
+                    delta: torch.Tensor | None = None, w: torch.Tensor | None = None, u: torch.Tensor | None = None,
+                    x_out: torch.Tensor | None = None, eps: float = 1e-5,
+                    stream: torch.cuda.Stream | None = None) -> None:
+        """``sf_gemv_refine_batch1_produce``: the input row made inside the
+        launch by ``op`` (PRODUCE_NORM: bf16(RMSNorm(x + delta) w), x + delta
+        to x_out; PRODUCE_ROUND: bf16(x); PRODUCE_SILU_MUL: bf16(silu(x) u)),
+        written to y with its top-k selection (idx, n), then the GEMVs."""
+        _dev(x, "x")
+        if idx.dtype != torch.int32 or idx.numel() < max(k, 1) or n.dtype != torch.int32:
+            raise ValueError("idx and n must be int32, idx with room for k entries")
+        pr = _GemvProducer(op, k, eps, _ptr(x), _ptr(delta), _ptr(w), _ptr(u), _ptr(x_out), _ptr(y), _ptr(idx),
+                           _ptr(n))
+        pp = ctypes.cast(ctypes.pointer(pr), _p)
+        _check(_lib.sf_gemv_refine_batch1_produce(ctypes.cast(self._arr, _p), self.count, pp, _stream(stream)))
 
 
 _gemv_overlap = False

@@ -10,33 +10,16 @@
 // query and key heads in one launch.
 #include <cuda_bf16.h>
 
+#include "produce.cuh"
 #include "select_row.cuh"
 #include "sf_internal.h"
 
 namespace {
 
-constexpr int kThreads = 1024;
+constexpr int kThreads = sfd::kNormVThreads;  // the RMSNorm sum order is that of 1024 threads
 
-__device__ __forceinline__ uint16_t to_bf16(double v) { return __bfloat16_as_ushort(__double2bfloat16(v)); }
-
-// bf16(silu(g) u) rounded once from the exact value.  The fp32 evaluation
-// r = fl(fl(g / fl(1 + expf(-g))) u) is within 7 * 2^-24 |r| of the exact
-// value (expf within 2 ulp, CUDA math API accuracy table; four correctly
-// rounded operations), i.e. within 16 steps of r's fp32 bit pattern even
-// across a binade.  RNE to bf16 changes only at the midpoints (low 16 bits
-// 0x8000), so when r's low half lies farther than 16 from 0x8000 the exact
-// value rounds as r does; otherwise (and for non-normal or huge r) the value
-// is recomputed in fp64 and rounded once.
-__device__ __forceinline__ uint16_t silu_mul_bf16(float g, float u) {
-  const float e = expf(-g);
-  const float r = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, e)), u);
-  const uint32_t b = __float_as_uint(r) & 0x7FFFFFFFu;
-  const int low = static_cast<int>(b & 0xFFFFu);
-  if (isfinite(e) && b >= 0x00800000u && b < 0x7E800000u && (low < 0x8000 - 16 || low > 0x8000 + 16))
-    return __bfloat16_as_ushort(__float2bfloat16_rn(r));
-  const double gv = g;
-  return to_bf16(gv / (1.0 + exp(-gv)) * static_cast<double>(u));
-}
+using sfd::silu_mul_bf16;
+using sfd::to_bf16;
 
 // Writes the producer's row to xs (shared) and y (global), then selects.
 enum Producer { kNorm = 0, kRound = 1, kSilu = 2 };

@@ -43,12 +43,20 @@
 //               the high bit of channel 16 (8 slot + 2 t + h) + 4 b + j.
 // A fragment byte is then ((w >> 2j) & 0x03030303) | (high bit moved to bit
 // 2 of each byte): two shifts and two logic operations per register.
+#include <cooperative_groups.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include <algorithm>
 #include <atomic>
+#include <map>
+#include <mutex>
+#include <type_traits>
+#include <utility>
 
 #include "act.cuh"  // bf16_exponent, bf16_fixed
+#include "produce.cuh"
+#include "select_row.cuh"
 #include "sf_internal.h"
 
 namespace {
@@ -72,9 +80,28 @@ struct MJob {
   int N, unit_words, tile_begin;
 };
 
+// The input row made inside the launch (sf_gemv_refine_batch1_produce): every
+// CTA computes the row and its selection itself, in the ring stage that the
+// weight stream does not use before the main loop.
+enum ProdOp { kProdNone = -1, kProdNorm = 0, kProdRound = 1, kProdSilu = 2 };
+
+struct MProd {
+  int op, k, hrows;  // hrows: histogram rows of the selection (warps share them)
+  float eps;
+  const float* x;      // kProdNorm: the residual; kProdRound: the row; kProdSilu: the gate
+  const float* delta;  // kProdNorm: added to x first (may be null)
+  const float* w;      // kProdNorm: RMSNorm weights
+  const float* u;      // kProdSilu: the up projection
+  float* x_out;        // kProdNorm: x + delta, written by CTA 0 (may be null)
+  uint16_t* y;         // the bf16 row: written by every CTA (identical values)
+  int32_t* idx;        // its selection and length: likewise
+  int32_t* n;
+};
+
 struct MArgs {
   MJob job[kMaxJobs];
-  const uint16_t* x;
+  MProd prod;
+  const uint16_t* x;     // the row (with a producer: prod.y, read back by the fp32 correction)
   const int32_t* idx;    // the selection: ascending channels (nullptr: none)
   const int32_t* n_sel;  // its length (negative counts as 0)
   int njobs, K, ksplit;
@@ -159,6 +186,136 @@ __device__ __forceinline__ void qf_frag(uint32_t wa, uint32_t wb, int g8, int of
   }
 }
 
+// The producer's row into xs (bf16 bits), with the arithmetic of
+// produce_select_kernel (decode_fused.cu): kProdNorm y = bf16(RMSNorm(x +
+// delta) w) (fp32 add, fp64 sum of squares in the order of 1024 threads,
+// fp64 scaling, one rounding), kProdRound y = bf16(x), kProdSilu y =
+// bf16(silu(x) u).  A thread's entries are i = tid + j blockDim.x, loaded
+// kProdBatch at a time with every load in flight (the weight stream keeps
+// the memory system busy, so each round trip is long).  vbuf (vcap floats of
+// scratch) holds x + delta for the fp64 sum when the row fits (else the sum
+// re-reads x and delta).  Every CTA writes y to global memory (the same
+// values) and CTA 0 the updated residual.  Ends with a barrier.
+constexpr int kProdBatch = 12;
+
+__device__ void produce_row(const MProd& P, int K, uint16_t* xs, float* vbuf, int vcap, double* part,
+                            double* inv_sh) {
+  const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
+  if (P.op == kProdNorm) {
+    const bool keep = K <= vcap;
+    // one load round for x, delta and w when a thread's entries fit one batch
+    const bool one = keep && K <= kProdBatch * nthr;
+    const bool cta0 = blockIdx.x == 0 && P.x_out != nullptr;
+    float wv[kProdBatch];
+    if (keep) {
+      for (int i0 = 0; i0 < K; i0 += kProdBatch * nthr) {
+        float xv[kProdBatch], dv[kProdBatch];
+#pragma unroll
+        for (int j = 0; j < kProdBatch; ++j) {
+          const int i = i0 + tid + j * nthr;
+          xv[j] = i < K ? P.x[i] : 0.0f;
+          dv[j] = i < K && P.delta ? P.delta[i] : 0.0f;
+          wv[j] = one && i < K ? P.w[i] : 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < kProdBatch; ++j) {
+          const int i = i0 + tid + j * nthr;
+          if (i < K) {
+            const float v = P.delta ? __fadd_rn(xv[j], dv[j]) : xv[j];
+            vbuf[i] = v;
+            if (cta0) P.x_out[i] = v;
+          }
+        }
+      }
+      __syncthreads();
+    }
+    // virtual warp vw (threads 32 vw .. 32 vw + 31 of the 1024) is taken by
+    // warp vw % nw, whose lanes coincide with the virtual lanes
+    for (int vw = warp; vw < 32; vw += nw) {
+      const int vt = 32 * vw + lane;
+      double ss = 0.0;
+      for (int i = vt; i < K; i += sfd::kNormVThreads) {
+        float v;
+        if (keep) {
+          v = vbuf[i];
+        } else {
+          v = P.x[i];
+          if (P.delta) v = __fadd_rn(v, P.delta[i]);
+        }
+        ss = fma(static_cast<double>(v), static_cast<double>(v), ss);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) part[vw] = ss;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      double t = 0.0;
+      for (int i = 0; i < sfd::kNormVThreads / 32; ++i) t += part[i];
+      *inv_sh = 1.0 / sqrt(t / K + static_cast<double>(P.eps));
+    }
+    __syncthreads();
+    const double inv = *inv_sh;
+    for (int i0 = 0; i0 < K; i0 += kProdBatch * nthr) {
+      float xv[kProdBatch], dv[kProdBatch];
+      if (!one) {
+#pragma unroll
+        for (int j = 0; j < kProdBatch; ++j) {
+          const int i = i0 + tid + j * nthr;
+          wv[j] = i < K ? P.w[i] : 0.0f;
+          if (!keep) {
+            xv[j] = i < K ? P.x[i] : 0.0f;
+            dv[j] = i < K && P.delta ? P.delta[i] : 0.0f;
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kProdBatch; ++j) {
+        const int i = i0 + tid + j * nthr;
+        if (i < K) {
+          float v;
+          if (keep) {
+            v = vbuf[i];
+          } else {
+            v = P.delta ? __fadd_rn(xv[j], dv[j]) : xv[j];
+            if (cta0) P.x_out[i] = v;
+          }
+          const uint16_t y = sfd::to_bf16(static_cast<double>(v) * inv * static_cast<double>(wv[j]));
+          xs[i] = y;
+          P.y[i] = y;
+        }
+      }
+    }
+  } else {
+    const bool silu = P.op == kProdSilu;
+    for (int i0 = 0; i0 < K; i0 += kProdBatch * nthr) {
+      float av[kProdBatch], uv[kProdBatch];
+#pragma unroll
+      for (int j = 0; j < kProdBatch; ++j) {
+        const int i = i0 + tid + j * nthr;
+        av[j] = i < K ? P.x[i] : 0.0f;
+        uv[j] = i < K && silu ? P.u[i] : 0.0f;
+      }
+#pragma unroll
+      for (int j = 0; j < kProdBatch; ++j) {
+        const int i = i0 + tid + j * nthr;
+        if (i < K) {
+          const uint16_t y = silu ? sfd::silu_mul_bf16(av[j], uv[j])
+                                  : __bfloat16_as_ushort(__float2bfloat16_rn(av[j]));
+          xs[i] = y;
+          P.y[i] = y;
+        }
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// Words of the producer's scratch (the last ring stage of every warp) taken
+// before the selection list: the row, the histogram rows, scan and info.
+__host__ __device__ constexpr int prod_row_words(int K) { return (K / 2 + 3) & ~3; }
+__host__ __device__ constexpr int prod_fixed_words(int K, int hrows) { return prod_row_words(K) + hrows * 256 + 48; }
+
 template <int SPW, int BR>
 struct MCfg {
   static constexpr int kCodeWords = 128 * BR;              // 16 rows x 8 BR words
@@ -176,7 +333,9 @@ struct MCfg {
   }
 };
 
-template <int SPW, int BF, int BR>
+// PROD: the launch makes its own input row and selection (a.prod); the
+// plain instantiation reads them from a.x, a.idx, a.n_sel.
+template <int SPW, int BF, int BR, bool PROD>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1)
 gemv_mma_kernel(const __grid_constant__ MArgs a) {
   using C = MCfg<SPW, BR>;
@@ -186,10 +345,15 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
   const int W = blockDim.x >> 5;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, tig = lane & 3;
   const int ks = blockIdx.x % a.ksplit, crow = blockIdx.x / a.ksplit, ncta = gridDim.x / a.ksplit;
-  uint32_t* ring = sm + warp * kStages * SW;
+  // ring stage s of warp w at sm + (s W + w) SW: the last stage of all warps
+  // is one contiguous block, the producer's scratch until the main loop
+  auto stage_base = [&](int st) { return sm + (st * W + warp) * SW; };
   uint16_t* mylist = reinterpret_cast<uint16_t*>(sm + W * kStages * SW) + warp * SPW * kCorrList;  // [SPW][32]
   float* red = reinterpret_cast<float*>(sm + W * kStages * SW + W * SPW * kCorrList / 2);
 
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  const bool pair = a.ksplit > 1;  // launched as clusters of the two K halves
   const int slice0 = (ks * W + warp) * SPW;
   const int myslot = tig >> 1, myrow = g8 + 8 * (tig & 1);
   const bool even = (tig & 1) == 0;
@@ -247,7 +411,7 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
       ++c_jb;
       c_seek();
     }
-    uint32_t* stage = ring + (i % kStages) * SW;
+    uint32_t* stage = stage_base(i % kStages);
 #pragma unroll
     for (int sp = 0; sp < SPW; ++sp) {
       uint32_t* base = stage + sp * kSliceWords;
@@ -287,7 +451,7 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
     }
     if (r_has) {
       const int woff = ((r_t - r_tb) * kRows * BF) >> 5;
-      uint32_t* stage = ring + (i % kStages) * SW;
+      uint32_t* stage = stage_base(i % kStages);
 #pragma unroll
       for (int sp = 0; sp < SPW; ++sp)
         if (lane < ntc[sp]) cp_async4(stage + sp * kSliceWords + kRF + lane, r_row[sp] + woff);
@@ -307,8 +471,34 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
   // serialization, the kernel may have started before the producer of x and
   // the selection finished: the code copies above need nothing it writes.
   pdl_wait_gemv();
-  int n_all = a.idx != nullptr ? *a.n_sel : 0;
-  n_all = n_all < 0 ? 0 : n_all;
+  constexpr bool produce = PROD;
+  const uint16_t* xrow = a.x;  // the row and its selection for the setup below
+  const int32_t* sel = a.idx;
+  int n_all;
+  if constexpr (PROD) {
+    // the row and its selection, computed by this CTA in the last ring stage
+    __shared__ double part[sfd::kNormVThreads / 32];
+    __shared__ double inv_sh;
+    uint32_t* scr = sm + (kStages - 1) * W * SW;
+    uint16_t* xs = reinterpret_cast<uint16_t*>(scr);
+    int* whist = reinterpret_cast<int*>(scr + prod_row_words(a.K));
+    int* sscan = whist + a.prod.hrows * 256;
+    int* info = sscan + 40;
+    int32_t* list = reinterpret_cast<int32_t*>(scr + prod_fixed_words(a.K, a.prod.hrows));
+    // x + delta kept between the producer's sweeps in the rest of the scratch
+    produce_row(a.prod, a.K, xs, reinterpret_cast<float*>(whist), W * SW - prod_row_words(a.K), part, &inv_sh);
+    sfd::select_row_cta(xs, a.K, a.prod.k, list, whist, a.prod.hrows, sscan, info, nullptr);
+    // every CTA writes the same selection; the fp32 correction reads it back
+    const int taken = info[6];
+    for (int i = tid; i < taken; i += blockDim.x) a.prod.idx[i] = list[i];
+    if (tid == 0) *a.prod.n = info[5];
+    n_all = info[5] < 0 ? 0 : info[5];
+    xrow = xs;
+    sel = list;
+  } else {
+    n_all = a.idx != nullptr ? *a.n_sel : 0;
+    n_all = n_all < 0 ? 0 : n_all;
+  }
 #pragma unroll
   for (int sp = 0; sp < SPW; ++sp) {
     const int slice = slice0 + sp;
@@ -319,7 +509,7 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
       // (slot_b, t) share those channels: lane plane q converts channels
       // 8q .. 8q + 7 and the lanes swap digit bytes by shuffles.
       const int bn = lane >> 2, slot_b = bn >> 2, plane = bn & 3;
-      const uint4 v = *reinterpret_cast<const uint4*>(a.x + 256 * static_cast<size_t>(slice) + 128 * slot_b +
+      const uint4 v = *reinterpret_cast<const uint4*>(xrow + 256 * static_cast<size_t>(slice) + 128 * slot_b +
                                                      32 * tig + 8 * plane);
       const uint32_t xw[4] = {v.x, v.y, v.z, v.w};
       // the group's largest |x| (15-bit magnitude keys order as |x| does):
@@ -399,7 +589,7 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
       int c_lo = 0, c_hi = 0;
       if (step > 32) {  // more than 1024 selected: count by a plain sweep
         for (int i = lane; i < n_all; i += 32) {
-          const int w = a.idx[i];
+          const int w = sel[i];
           c_lo += w < lo;
           c_hi += w < hi;
         }
@@ -410,26 +600,26 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
         }
       } else if (n_all > 0) {
         const int p1 = min(n_all - 1, lane * step);
-        const int v1 = a.idx[p1];
+        const int v1 = sel[p1];
         const bool in1 = lane * step < n_all;
         const int seg_lo = __popc(__ballot_sync(0xffffffffu, in1 && v1 < lo));  // segments entirely below lo
         const int seg_hi = __popc(__ballot_sync(0xffffffffu, in1 && v1 < hi));
         // entries before segment seg - 1 are all below the bound; search it
         const int b_lo = max(seg_lo - 1, 0) * step, b_hi = max(seg_hi - 1, 0) * step;
         const bool ok_lo = lane < step && b_lo + lane < n_all, ok_hi = lane < step && b_hi + lane < n_all;
-        const int w_lo = ok_lo ? a.idx[b_lo + lane] : 0x7FFFFFFF;
-        const int w_hi = ok_hi ? a.idx[b_hi + lane] : 0x7FFFFFFF;
+        const int w_lo = ok_lo ? sel[b_lo + lane] : 0x7FFFFFFF;
+        const int w_hi = ok_hi ? sel[b_hi + lane] : 0x7FFFFFFF;
         c_lo = b_lo + __popc(__ballot_sync(0xffffffffu, ok_lo && w_lo < lo));
         c_hi = b_hi + __popc(__ballot_sync(0xffffffffu, ok_hi && w_hi < hi));
       }
       psl[sp] = c_lo;
       nsl[sp] = c_hi - c_lo;
-      if (lane < min(nsl[sp], kCorrList)) mylist[sp * kCorrList + lane] = static_cast<uint16_t>(a.idx[c_lo + lane] - lo);
+      if (lane < min(nsl[sp], kCorrList)) mylist[sp * kCorrList + lane] = static_cast<uint16_t>(sel[c_lo + lane] - lo);
     }
     __syncwarp();
     int nl = min(nsl[sp], kCorrList);
     float xv = 0.0f;
-    if (lane < nl) xv = sfd::bf16_bits_to_float(a.x[256 * slice + mylist[sp * kCorrList + lane]]);
+    if (lane < nl) xv = sfd::bf16_bits_to_float(xrow[256 * slice + mylist[sp * kCorrList + lane]]);
     // a listed |x| at or above 2^15 would overflow the f16 split: the whole
     // slice is then corrected by the fp32 loop
     if (__any_sync(0xffffffffu, !(fabsf(xv) < kCorrXMax))) nl = 0;
@@ -446,6 +636,7 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
     hl_l[sp] = hl;
     grp_l[sp] = grp;
   }
+  if constexpr (PROD) __syncthreads();  // every warp is done with the scratch before the main loop refills it
   // the correction MMA's B fragments and offset constant for the job the
   // compute cursor is in: a job reading a cache in the deadline reading drops
   // the listed channels not cached (their x becomes 0)
@@ -521,7 +712,7 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
     float v = 0.0f;
 #pragma unroll
     for (int sp = 0; sp < SPW; ++sp) {
-      const uint32_t* base = ring + st * SW + sp * kSliceWords;
+      const uint32_t* base = stage_base(st) + sp * kSliceWords;
       // (low) code words: rows g8 and g8 + 8, words 2 tig, 2 tig + 1 of each group
       const uint2 r0a = *reinterpret_cast<const uint2*>(base + code_off<BR>(g8, tig >> 1) + 2 * (tig & 1));
       const uint2 r0b = *reinterpret_cast<const uint2*>(base + code_off<BR>(g8, 2 + (tig >> 1)) + 2 * (tig & 1));
@@ -609,19 +800,30 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
     v += __shfl_xor_sync(0xffffffffu, v, 2);
     if (tig < 2) red[((i % kRedTiles) * W + warp) * kRows + myrow] = v;
     if (i % kRedTiles == kRedTiles - 1 || i == my_tiles - 1) {
-      __syncthreads();
+      // with two K halves the CTAs of a cluster pair hold the same tiles:
+      // each writes half of the rows, summing both CTAs' warp partials
+      // through distributed shared memory (half 0's sum plus half 1's)
+      if (pair) cl.sync();
+      else __syncthreads();
       const int i0 = i - i % kRedTiles, nt = i - i0 + 1;
-      for (int e = tid; e < nt * kRows; e += blockDim.x) {
-        const int ti = e / kRows, rr = e % kRows;
+      const int rows = pair ? kRows / 2 : kRows, r0 = ks * rows;
+      const float* red0 = pair ? cl.map_shared_rank(red, 0) : red;
+      const float* red1 = pair ? cl.map_shared_rank(red, 1) : red;
+      for (int e = tid; e < nt * rows; e += blockDim.x) {
+        const int ti = e / rows, rr = r0 + e % rows;
         float acc = 0.0f;
-        for (int w = 0; w < W; ++w) acc += red[(ti * W + w) * kRows + rr];
+        for (int w = 0; w < W; ++w) acc += red0[(ti * W + w) * kRows + rr];
+        if (pair) {
+          float acc1 = 0.0f;
+          for (int w = 0; w < W; ++w) acc1 += red1[(ti * W + w) * kRows + rr];
+          acc += acc1;
+        }
         const int tt = t_begin + i0 + ti;
         const MJob& Jt = a.job[job_of(a, tt)];
-        float* dst = Jt.y + (tt - Jt.tile_begin) * kRows + rr;
-        if (a.ksplit > 1) atomicAdd(dst, acc);
-        else *dst = acc;
+        Jt.y[(tt - Jt.tile_begin) * kRows + rr] = acc;
       }
-      __syncthreads();
+      if (pair) cl.sync();  // the partner has read this CTA's partials
+      else __syncthreads();
     }
   }
   cp_async_wait<0>();
@@ -694,44 +896,119 @@ extern "C" sf_status sf_gemv_pack_batch1(const uint32_t* res, int N, int K, int 
   return sf::check_launch("pack_res3_kernel");
 }
 
-extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, const uint16_t* x, const int32_t* idx,
-                                           const int32_t* n, sf_stream_t stream) {
-  SF_REQUIRE(jobs && x, "sf_gemv_refine_batch1: null pointer");
-  SF_REQUIRE((idx == nullptr) == (n == nullptr), "sf_gemv_refine_batch1: idx and n go together");
-  SF_REQUIRE(count >= 1 && count <= kMaxJobs, "sf_gemv_refine_batch1: count must be in [1, %d]", kMaxJobs);
-  SF_REQUIRE(sf::aligned(x, 16), "sf_gemv_refine_batch1: x must be 16-byte aligned");
+namespace {
+
+// Clusters of two K halves that can be resident at once (cached per kernel
+// and shared-memory size): the grid never holds more pairs than that, so no
+// pair waits for a second wave.
+int max_pairs(const void* kern, size_t smem, int block) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, size_t>, int> known;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(kern, smem);
+  const auto it = known.find(key);
+  if (it != known.end()) return it->second;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2 * sf::sm_count());
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    n = sf::sm_count() / 2;
+  }
+  known[key] = n;
+  return n;
+}
+
+sf_status run_batch1(const char* what, const sf_gemv_job* jobs, int count, const uint16_t* x, const int32_t* idx,
+                     const int32_t* n, const sf_gemv_producer* p, cudaStream_t s) {
+  SF_REQUIRE(jobs, "%s: null pointer", what);
+  SF_REQUIRE(count >= 1 && count <= kMaxJobs, "%s: count must be in [1, %d]", what, kMaxJobs);
   const sf_qweight* W0 = jobs[0].W;
-  SF_REQUIRE(W0, "sf_gemv_refine_batch1: null weight");
+  SF_REQUIRE(W0, "%s: null weight", what);
   const int K = W0->K, G = W0->G, b_f = W0->b_f, b_r = W0->b_r;
-  SF_REQUIRE(b_r == 2 || b_r == 3, "sf_gemv_refine_batch1: b_r must be 2 or 3");
-  SF_REQUIRE(b_f == 1 || b_f == 2, "sf_gemv_refine_batch1: b_f must be 1 or 2");
-  SF_REQUIRE(b_r + b_f <= 4, "sf_gemv_refine_batch1: b_r + b_f must be at most 4");
-  SF_REQUIRE(G == 128, "sf_gemv_refine_batch1: group size must be 128 (the prepared activations' group)");
-  SF_REQUIRE(K >= 256 && K % 256 == 0, "sf_gemv_refine_batch1: K must be a positive multiple of 256");
+  SF_REQUIRE(b_r == 2 || b_r == 3, "%s: b_r must be 2 or 3", what);
+  SF_REQUIRE(b_f == 1 || b_f == 2, "%s: b_f must be 1 or 2", what);
+  SF_REQUIRE(b_r + b_f <= 4, "%s: b_r + b_f must be at most 4", what);
+  SF_REQUIRE(G == 128, "%s: group size must be 128 (the prepared activations' group)", what);
+  SF_REQUIRE(K >= 256 && K % 256 == 0, "%s: K must be a positive multiple of 256", what);
   int spw = 0, ksplit = 0;
   SF_REQUIRE(pick_split(K / 256, &spw, &ksplit),
-             "sf_gemv_refine_batch1: K/256 must split into at most 16 warps of 1 or 2 slices, in 1 or 2 halves");
-  cudaStream_t s = sf::as_cuda(stream);
+             "%s: K/256 must split into at most 16 warps of 1 or 2 slices, in 1 or 2 halves", what);
+  const int warps = K / 256 / (spw * ksplit);
   MArgs a{};
   a.njobs = count;
   a.K = K;
   a.ksplit = ksplit;
-  a.x = x;
-  a.idx = idx;
-  a.n_sel = n;
+  a.prod.op = kProdNone;
+  if (p == nullptr) {
+    SF_REQUIRE(x, "%s: null pointer", what);
+    SF_REQUIRE((idx == nullptr) == (n == nullptr), "%s: idx and n go together", what);
+    SF_REQUIRE(sf::aligned(x, 16), "%s: x must be 16-byte aligned", what);
+    a.x = x;
+    a.idx = idx;
+    a.n_sel = n;
+  } else {
+    SF_REQUIRE(p->op == SF_PRODUCE_NORM || p->op == SF_PRODUCE_ROUND || p->op == SF_PRODUCE_SILU_MUL,
+               "%s: unknown producer op %d", what, p->op);
+    SF_REQUIRE(p->x && p->y && p->idx && p->n, "%s: null producer pointer", what);
+    SF_REQUIRE(p->op != SF_PRODUCE_NORM || p->w, "%s: SF_PRODUCE_NORM needs w", what);
+    SF_REQUIRE(p->op != SF_PRODUCE_SILU_MUL || p->u, "%s: SF_PRODUCE_SILU_MUL needs u", what);
+    SF_REQUIRE(p->op != SF_PRODUCE_NORM || p->eps >= 0.0f, "%s: eps must be >= 0", what);
+    SF_REQUIRE(sf::aligned(p->y, 16), "%s: y must be 16-byte aligned", what);
+    SF_REQUIRE(K <= sfd::kSelRowMaxK, "%s: K must be at most %d with a producer", what, sfd::kSelRowMaxK);
+    // the selection list shares the last ring stage with the row and the histograms
+    const size_t stage_words = static_cast<size_t>(warps) * (b_r == 2 ? (spw == 1 ? MCfg<1, 2>::SW : MCfg<2, 2>::SW)
+                                                                      : (spw == 1 ? MCfg<1, 3>::SW : MCfg<2, 3>::SW));
+    // histogram rows: one per warp while the list still fits, else shared
+    int hrows = warps;
+    auto cap = [&](int h) { return static_cast<long long>(stage_words) - prod_fixed_words(K, h); };
+    while (hrows > 1 && cap(hrows) < p->k) hrows = (hrows + 1) / 2;
+    SF_REQUIRE(p->k >= 0 && p->k <= K && p->k <= cap(hrows), "%s: k must be in [0, min(K, %lld)]", what,
+               std::max(0LL, std::min(static_cast<long long>(K), cap(hrows))));
+    a.prod.hrows = hrows;
+    if (p->op == SF_PRODUCE_NORM && p->x_out) {
+      auto overlaps = [&](const float* q) {
+        return q != nullptr && p->x_out < q + K && q < p->x_out + K;
+      };
+      SF_REQUIRE(!overlaps(p->x) && !overlaps(p->delta), "%s: x_out must not overlap x or delta", what);
+    }
+    a.prod.op = p->op;
+    a.prod.k = p->k;
+    a.prod.eps = p->eps;
+    a.prod.x = p->x;
+    a.prod.delta = p->op == SF_PRODUCE_NORM ? p->delta : nullptr;
+    a.prod.w = p->w;
+    a.prod.u = p->u;
+    a.prod.x_out = p->op == SF_PRODUCE_NORM ? p->x_out : nullptr;
+    a.prod.y = p->y;
+    a.prod.idx = p->idx;
+    a.prod.n = p->n;
+    a.x = p->y;
+    a.idx = p->idx;
+    a.n_sel = p->n;
+  }
   int row_tiles = 0;
   for (int i = 0; i < count; ++i) {
     const sf_qweight* W = jobs[i].W;
-    SF_REQUIRE(W && W->scale && W->zero && jobs[i].y, "sf_gemv_refine_batch1: job %d incomplete", i);
+    SF_REQUIRE(W && W->scale && W->zero && jobs[i].y, "%s: job %d incomplete", what, i);
     SF_REQUIRE(W->K == K && W->G == G && W->b_f == b_f && W->b_r == b_r,
-               "sf_gemv_refine_batch1: jobs must share K, G and bit widths");
+               "%s: jobs must share K, G and bit widths", what);
     const uint32_t* res = jobs[i].res_b1 ? jobs[i].res_b1 : W->res;
-    SF_REQUIRE(res, "sf_gemv_refine_batch1: job %d has no resident codes", i);
+    SF_REQUIRE(res, "%s: job %d has no resident codes", what, i);
     SF_REQUIRE(b_r == 2 || jobs[i].res_b1,
-               "sf_gemv_refine_batch1: 3-bit codes must be given in the batch-1 layout (res_b1, sf_gemv_pack_batch1)");
-    SF_REQUIRE(W->N >= kRows && W->N % kRows == 0, "sf_gemv_refine_batch1: N must be a multiple of %d", kRows);
+               "%s: 3-bit codes must be given in the batch-1 layout (res_b1, sf_gemv_pack_batch1)", what);
+    SF_REQUIRE(W->N >= kRows && W->N % kRows == 0, "%s: N must be a multiple of %d", what, kRows);
     SF_REQUIRE(sf::aligned(res, 16) && sf::aligned(W->scale, 16) && sf::aligned(W->zero, 16),
-               "sf_gemv_refine_batch1: weight arrays must be 16-byte aligned");
+               "%s: weight arrays must be 16-byte aligned", what);
     MJob& J = a.job[i];
     J.res = res;
     J.scale = W->scale;
@@ -744,56 +1021,74 @@ extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, c
     if (jobs[i].cache) {
       sf::CacheView v{};
       const bool deadline = sf::cache_deadline(jobs[i].cache);
+      SF_REQUIRE(deadline || p == nullptr,
+                 "%s: a producer needs caches in the deadline reading (a blocking prefetch needs the selection "
+                 "before the launch)", what);
       const sf_status st = deadline ? sf::cache_view_for_reader(jobs[i].cache, s, &v)
                                     : sf::cache_view_for_gemv(jobs[i].cache, s, &v);
       if (st != SF_OK) return st;
-      SF_REQUIRE(v.unit_words == J.unit_words, "sf_gemv_refine_batch1: cache unit size does not match N*b_f/8");
-      SF_REQUIRE(!deadline || v.num_units == K, "sf_gemv_refine_batch1: a deadline cache must have K units");
+      SF_REQUIRE(v.unit_words == J.unit_words, "%s: cache unit size does not match N*b_f/8", what);
+      SF_REQUIRE(!deadline || v.num_units == K, "%s: a deadline cache must have K units", what);
       J.ref_rows = v.rows;
       J.row_of = deadline ? nullptr : v.row_of;
       J.unit_slot = deadline ? v.unit_slot : nullptr;
     } else if (jobs[i].use_ref_store) {
-      SF_REQUIRE(W->ref, "sf_gemv_refine_batch1: use_ref_store without W->ref");
+      SF_REQUIRE(W->ref, "%s: use_ref_store without W->ref", what);
       J.ref_rows = W->ref;
       J.row_of = nullptr;
     }
-    if (ksplit > 1) SF_CHECK_CUDA(cudaMemsetAsync(jobs[i].y, 0, sizeof(float) * W->N, s));
   }
-  const int warps = K / 256 / (spw * ksplit);
   const int sms = sf::sm_count();
-  const int nrow_cta = std::max(1, std::min(row_tiles, std::max(1, sms / ksplit)));
-  const dim3 grid(nrow_cta * ksplit), block(32 * warps);
   auto launch = [&](auto kern, size_t smem) -> sf_status {
     SF_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+    // row blocks (pairs with two K halves) with work only: ceil(tiles / per)
+    // blocks of per = ceil(tiles / cap) tiles, so no block idles and the SMs
+    // left over stay free (for a producer that the launch overlaps)
+    int cap = std::max(1, sms / ksplit);
+    if (ksplit > 1) cap = std::max(1, std::min(cap, max_pairs(reinterpret_cast<const void*>(kern), smem, 32 * warps)));
+    const int per = (row_tiles + cap - 1) / cap;
+    const int nrow_cta = (row_tiles + per - 1) / per;
     // programmatic stream serialization: the CTAs may start streaming codes
-    // while the previous kernel (typically the one-CTA producer of x) runs;
-    // not when memsets of y were just enqueued (ksplit > 1)
+    // while the previous kernel (typically the producer of x) runs
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
+    cfg.gridDim = dim3(nrow_cta * ksplit);
+    cfg.blockDim = dim3(32 * warps);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (g_gemv_overlap.load(std::memory_order_relaxed)) {
+      attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[na].val.programmaticStreamSerializationAllowed = 1;
+      ++na;
+    }
+    if (ksplit > 1) {  // the two K halves of a row block form a cluster
+      attr[na].id = cudaLaunchAttributeClusterDimension;
+      attr[na].val.clusterDim.x = 2;
+      attr[na].val.clusterDim.y = 1;
+      attr[na].val.clusterDim.z = 1;
+      ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = (ksplit > 1 || !g_gemv_overlap.load(std::memory_order_relaxed)) ? 0 : 1;
+    cfg.numAttrs = na;
     SF_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kern, a));
     return sf::check_launch("gemv_mma_kernel");
   };
-  sf_status st;
-  if (b_r == 2) {
-    if (spw == 1) {
-      const size_t smem = MCfg<1, 2>::smem_bytes(warps);
-      st = b_f == 2 ? launch(gemv_mma_kernel<1, 2, 2>, smem) : launch(gemv_mma_kernel<1, 1, 2>, smem);
-    } else {
+  auto dispatch = [&](auto prod) -> sf_status {
+    constexpr bool P = decltype(prod)::value;
+    if (b_r == 2) {
+      if (spw == 1) {
+        const size_t smem = MCfg<1, 2>::smem_bytes(warps);
+        return b_f == 2 ? launch(gemv_mma_kernel<1, 2, 2, P>, smem) : launch(gemv_mma_kernel<1, 1, 2, P>, smem);
+      }
       const size_t smem = MCfg<2, 2>::smem_bytes(warps);
-      st = b_f == 2 ? launch(gemv_mma_kernel<2, 2, 2>, smem) : launch(gemv_mma_kernel<2, 1, 2>, smem);
+      return b_f == 2 ? launch(gemv_mma_kernel<2, 2, 2, P>, smem) : launch(gemv_mma_kernel<2, 1, 2, P>, smem);
     }
-  } else {  // b_r == 3, b_f == 1
-    st = spw == 1 ? launch(gemv_mma_kernel<1, 1, 3>, MCfg<1, 3>::smem_bytes(warps))
-                  : launch(gemv_mma_kernel<2, 1, 3>, MCfg<2, 3>::smem_bytes(warps));
-  }
+    // b_r == 3, b_f == 1
+    return spw == 1 ? launch(gemv_mma_kernel<1, 1, 3, P>, MCfg<1, 3>::smem_bytes(warps))
+                    : launch(gemv_mma_kernel<2, 1, 3, P>, MCfg<2, 3>::smem_bytes(warps));
+  };
+  const sf_status st = p != nullptr ? dispatch(std::true_type{}) : dispatch(std::false_type{});
   if (st != SF_OK) return st;
   for (int i = 0; i < count; ++i)
     if (jobs[i].cache) {
@@ -801,6 +1096,20 @@ extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, c
       if (m != SF_OK) return m;
     }
   return SF_OK;
+}
+
+}  // namespace
+
+extern "C" sf_status sf_gemv_refine_batch1(const sf_gemv_job* jobs, int count, const uint16_t* x, const int32_t* idx,
+                                           const int32_t* n, sf_stream_t stream) {
+  return run_batch1("sf_gemv_refine_batch1", jobs, count, x, idx, n, nullptr, sf::as_cuda(stream));
+}
+
+extern "C" sf_status sf_gemv_refine_batch1_produce(const sf_gemv_job* jobs, int count, const sf_gemv_producer* p,
+                                                   sf_stream_t stream) {
+  SF_REQUIRE(p, "sf_gemv_refine_batch1_produce: null producer");
+  return run_batch1("sf_gemv_refine_batch1_produce", jobs, count, nullptr, nullptr, nullptr, p,
+                    sf::as_cuda(stream));
 }
 
 extern "C" sf_status sf_gemv_set_launch_overlap(int on) {

@@ -247,8 +247,8 @@ __device__ __forceinline__ uint64_t splitmix64(uint64_t z) {
 __global__ void __launch_bounds__(kThreads)
 select_random_kernel(int K, int k, uint64_t seed, uint64_t step, int32_t* __restrict__ idx, int32_t* __restrict__ n) {
   extern __shared__ __align__(16) uint8_t smem[];
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [K]
-  uint8_t* flags = smem + 2 * K;                     // [K]
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [K], padded to sel_row_bytes(K)
+  uint8_t* flags = smem + sfd::sel_row_bytes(K);     // [K]
   const uint64_t base = seed + static_cast<uint64_t>(K) * step;
   for (int j = threadIdx.x; j < K; j += kThreads)
     xs[j] = static_cast<uint16_t>((splitmix64(base + static_cast<uint64_t>(j)) >> 49) % 0x7F80u);
@@ -270,8 +270,8 @@ select_union_cluster_kernel(const uint16_t* __restrict__ x, int K, int k, int32_
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
   extern __shared__ __align__(16) uint8_t smem[];
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [K]
-  uint8_t* flags = smem + 2 * K;                     // [K]
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);  // [K], padded to sel_row_bytes(K)
+  uint8_t* flags = smem + sfd::sel_row_bytes(K);     // [K]
   __shared__ uint32_t mask[kUnionMaxWords];          // rank 0's: the union
   __shared__ int nrow, bad_any, scan_scratch[33];
   const int b = static_cast<int>(cl.block_rank()), tid = threadIdx.x;
@@ -322,7 +322,7 @@ extern "C" sf_status sf_select_random(int K, int k, uint64_t seed, uint64_t step
                                       sf_stream_t stream) {
   SF_REQUIRE(idx_out && n_out, "sf_select_random: null pointer");
   SF_REQUIRE(K >= 1 && K <= 32768 && k >= 0 && k <= K, "sf_select_random: need 1 <= K <= 32768, 0 <= k <= K");
-  const size_t smem = 3 * static_cast<size_t>(K);
+  const size_t smem = sfd::sel_row_bytes(K) + static_cast<size_t>(K);
   SF_CHECK_CUDA(cudaFuncSetAttribute(select_random_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(smem)));
   select_random_kernel<<<1, kThreads, smem, sf::as_cuda(stream)>>>(K, k, seed, step, idx_out, n_out);
@@ -337,7 +337,7 @@ extern "C" sf_status sf_select_topk(const uint16_t* x, int B, int K, int k, int3
   SF_REQUIRE(k >= 0 && k <= K, "sf_select_topk: k must be in [0, K]");
   if (B >= 2 && K <= kActMaxK && k >= 1) {
     // one CTA per row, the union through a thread-block cluster
-    const size_t smem = 3 * static_cast<size_t>(K);
+    const size_t smem = sfd::sel_row_bytes(K) + static_cast<size_t>(K);
     SF_CHECK_CUDA(cudaFuncSetAttribute(select_union_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem)));
     SF_CHECK_CUDA(cudaFuncSetAttribute(select_union_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));

@@ -50,9 +50,10 @@ from fractions import Fraction
 
 import torch
 
-from . import (QKV, Batch1Jobs, RefineCache, RefineGroup, act_bytes, attn_decode_refine, attn_union_units,
-               attn_workspace_size, gemv_set_launch_overlap, kv_append, kv_append_pair_cached, norm_select, pack_batch1, quantize_nested, rope_qk,
-               round_select, silu_mul_select)
+from . import (PRODUCE_NORM, PRODUCE_ROUND, PRODUCE_SILU_MUL, QKV, Batch1Jobs, RefineCache, RefineGroup, act_bytes,
+               attn_decode_refine, attn_union_units, attn_workspace_size, gemv_set_launch_overlap, kv_append,
+               kv_append_pair_cached, norm_select, pack_batch1, quantize_nested, rope_qk, round_select,
+               silu_mul_select)
 
 MATS = ("q", "k", "v", "o", "gate", "up", "down")
 
@@ -120,7 +121,7 @@ class DecodeModel:
     def __init__(self, shape: Shape, weight, norm, kv, capacity: int, p: Fraction = Fraction(3, 100),
                  p_tok: Fraction = Fraction(1, 100), weight_cache_pct=None, kv_cache_pct=None,
                  kv_budget: int | None = None, weight_deadline: bool = False, fetch_lead: bool = False,
-                 record: bool = False, device=None):
+                 record: bool = False, fused_producers: bool = False, device=None):
         self.s = shape
         self.dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
         self.p, self.p_tok = Fraction(p), Fraction(p_tok)
@@ -128,6 +129,10 @@ class DecodeModel:
         self.record = record
         self.deadline = weight_deadline and weight_cache_pct is not None
         self.lead = fetch_lead and self.deadline
+        # fused_producers: each GEMV makes its own input row and selection in
+        # its launch (sf_gemv_refine_batch1_produce); not with a blocking
+        # cache prefetch, which needs the selection before the launch
+        self.fused = fused_producers and (weight_cache_pct is None or self.deadline)
         H, F, d = shape.hidden, shape.mlp, shape.head_dim
         Hq, Hkv = shape.n_q, shape.n_kv
         dev = self.dev
@@ -199,7 +204,11 @@ class DecodeModel:
         H, F, d, Hq, Hkv = s.hidden, s.mlp, s.head_dim, s.n_q, s.n_kv
         bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
         nl = s.layers
-        self.x = torch.zeros(H, dtype=f32, device=dev)          # the residual stream
+        # the residual stream, in two buffers: a launch that updates it reads
+        # one and writes the other (its thread blocks read the old value)
+        self.xr = torch.zeros((2, H), dtype=f32, device=dev)
+        self.cur = 0
+        self.read_evt = [None, None]
         self.x_in = torch.zeros(H, dtype=f32, device=dev)       # the step's input embedding
         self.buf = {}
         for slot in ("attn_in", "attn_out", "mlp_in", "mlp_mid"):
@@ -263,6 +272,11 @@ class DecodeModel:
             ph = self.pred["head"]
             self.head_pgroup = RefineGroup([(self.head.cache, ph["idx"][0], ph["n"][0])])
 
+    @property
+    def x(self) -> torch.Tensor:
+        """The residual stream as it stands."""
+        return self.xr[self.cur]
+
     # ---- the step -----------------------------------------------------------------------
 
     def _sel(self, l, slot, refine):
@@ -289,13 +303,58 @@ class DecodeModel:
         else:
             (self.jobs0[l][slot] if l >= 0 else self.head_job0).run(x)
 
+    def _produce_linear(self, l, slot, refine, main, op, x, **kw):
+        """The GEMVs of `slot` with their input row made in the same launch by
+        ``op`` (sf_gemv_refine_batch1_produce); the caches' step for later
+        steps follows on the side stream (deadline reading).  For
+        PRODUCE_NORM the residual x + delta goes to the other residual
+        buffer, which becomes the current one."""
+        b = self.buf[slot]
+        li = max(l, 0)
+        k = self.k_in[slot] if refine else 0
+        jobs = (self.jobs[l][slot] if l >= 0 else self.head_job) if refine else \
+            (self.jobs0[l][slot] if l >= 0 else self.head_job0)
+        y = b["x"][l] if l >= 0 else b["x"][0]
+        if op == PRODUCE_NORM:
+            kw["x_out"] = self.xr[1 - self.cur]
+        jobs.run_produce(op, x, y, k, b["idx"][li], b["n"][li], eps=self.s.eps, **kw)
+        if op == PRODUCE_NORM:
+            self.cur ^= 1
+        if refine:
+            grp = self.wgroups[l].get(slot) if l >= 0 else self.head_group
+            if grp is not None:
+                grp.prefetch(main, self.side)   # for later steps; nothing waits within this one
+
+    def _norm_linear(self, l, slot, norm_w, delta, refine, main, predict=None):
+        """x += delta, RMSNorm, the selection, the GEMVs of `slot`; predict()
+        runs once the updated residual is enqueued (before the GEMV launch
+        when the producer is a launch of its own).  The residual buffer
+        written (the other one when fused, else the current) must first have
+        been read by any prediction that reads it."""
+        target = 1 - self.cur if self.fused else self.cur
+        if self.read_evt[target] is not None:
+            main.wait_event(self.read_evt[target])
+            self.read_evt[target] = None
+        if self.fused:
+            self._produce_linear(l, slot, refine, main, PRODUCE_NORM, self.x, delta=delta, w=norm_w)
+            if predict is not None:
+                predict()
+        else:
+            b = self.buf[slot]
+            norm_select(self.x, norm_w, b["x"][l] if l >= 0 else b["x"], eps=self.s.eps, delta=delta,
+                        **self._sel(l, slot, refine))
+            if predict is not None:
+                predict()
+            self._linear(l, slot, refine, main)
+
     def _predict(self, l, slot, norm_w, main):
         """Fetch lead: select the channels the input of `slot` (layer l; the LM
         head for l < 0) will have, from the residual stream as it is now
         (RMSNorm of the current residual with that input's norm weights), and
         step those matrices' caches with the prediction, on the side stream,
         while the main stream goes on.  The main stream waits for the
-        prediction's read of the residual before it changes the residual."""
+        prediction's read of the residual buffer before it next writes that
+        buffer."""
         pr = self.pred[slot]
         li = max(l, 0)
         self.side.wait_stream(main)
@@ -306,7 +365,7 @@ class DecodeModel:
             ev.record(self.side)
         grp = self.pgroups[l][slot] if l >= 0 else self.head_pgroup
         grp.prefetch(self.side, self.side)
-        return ev
+        self.read_evt[self.cur] = ev
 
     def step(self, T: int, refine: bool = True) -> None:
         """One decode step of the token at position T (T tokens already in
@@ -331,19 +390,16 @@ class DecodeModel:
         side_used = refine and any(self.wgroups) or (refine and self.head_group is not None)
         kv_used = False
         lead = refine and self.lead
+        self.cur = 0
+        self.read_evt = [None, None]  # per residual buffer: the last prediction that reads it
         self.x.copy_(self.x_in)
         prev = None
-        read_done = None  # the last prediction's read of the residual
         for l, L in enumerate(self.layers):
-            if read_done is not None:
-                main.wait_event(read_done)
-            norm_select(self.x, L["norm1"], self.buf["attn_in"]["x"][l], eps=s.eps, delta=prev,
-                        **self._sel(l, "attn_in", refine))
-            if lead:  # gate/up of this layer, from the residual before the attention
-                read_done = self._predict(l, "mlp_in", L["norm2"], main)
+            # lead: gate/up of this layer, predicted from the residual before the attention
+            self._norm_linear(l, "attn_in", L["norm1"], prev, refine, main,
+                              predict=(lambda: self._predict(l, "mlp_in", L["norm2"], main)) if lead else None)
             if self.record:
                 self.x_hist[l].copy_(self.x)
-            self._linear(l, "attn_in", refine, main)
             q, k, v = L["q"].y.view(Hq, d), L["k"].y.view(Hkv, d), L["v"].y.view(Hkv, d)
             if self.record:
                 self.qkv_raw[l, :Hq * d].copy_(L["q"].y)
@@ -370,30 +426,29 @@ class DecodeModel:
                                  self.n_units[l], stream=self.side_kv)
                 L["kv_cache"].prefetch(self.units[l], self.n_units[l], self.side_kv, self.side_kv)
                 kv_used = True
-            round_select(self.att[l].view(-1), self.buf["attn_out"]["x"][l], **self._sel(l, "attn_out", refine))
-            self._linear(l, "attn_out", refine, main)
-            if read_done is not None:
-                main.wait_event(read_done)
-            norm_select(self.x, L["norm2"], self.buf["mlp_in"]["x"][l], eps=s.eps, delta=L["o"].y,
-                        **self._sel(l, "mlp_in", refine))
-            read_done = None
-            if lead:  # the next layer's q/k/v (or the LM head), from the residual after the attention
-                nxt = self.layers[l + 1]["norm1"] if l + 1 < s.layers else self.final_norm
-                read_done = self._predict(l + 1 if l + 1 < s.layers else -1, "attn_in" if l + 1 < s.layers else "head",
-                                          nxt, main)
+            if self.fused:
+                self._produce_linear(l, "attn_out", refine, main, PRODUCE_ROUND, self.att[l].view(-1))
+            else:
+                round_select(self.att[l].view(-1), self.buf["attn_out"]["x"][l], **self._sel(l, "attn_out", refine))
+                self._linear(l, "attn_out", refine, main)
+            # lead: the next layer's q/k/v (or the LM head), from the residual after the attention
+            last = l + 1 == s.layers
+            nxt = self.final_norm if last else self.layers[l + 1]["norm1"]
+            self._norm_linear(l, "mlp_in", L["norm2"], L["o"].y, refine, main,
+                              predict=(lambda: self._predict(-1 if last else l + 1, "head" if last else "attn_in",
+                                                             nxt, main)) if lead else None)
             if self.record:
                 self.h_hist[l].copy_(self.x)
-            self._linear(l, "mlp_in", refine, main)
-            silu_mul_select(L["gate"].y, L["up"].y, self.buf["mlp_mid"]["x"][l], **self._sel(l, "mlp_mid", refine))
-            self._linear(l, "mlp_mid", refine, main)
+            if self.fused:
+                self._produce_linear(l, "mlp_mid", refine, main, PRODUCE_SILU_MUL, L["gate"].y, u=L["up"].y)
+            else:
+                silu_mul_select(L["gate"].y, L["up"].y, self.buf["mlp_mid"]["x"][l],
+                                **self._sel(l, "mlp_mid", refine))
+                self._linear(l, "mlp_mid", refine, main)
             prev = L["down"].y
-        if read_done is not None:
-            main.wait_event(read_done)
-        norm_select(self.x, self.final_norm, self.buf["head"]["x"][0], eps=s.eps, delta=prev,
-                    **self._sel(-1, "head", refine))
+        self._norm_linear(-1, "head", self.final_norm, prev, refine, main)
         if self.record:
             self.x_hist[s.layers].copy_(self.x)
-        self._linear(-1, "head", refine, main)
         # every fetch of the step (the KV caches' misses for later steps
         # included) completes within the step
         if side_used:

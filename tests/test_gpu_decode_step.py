@@ -211,12 +211,14 @@ def _embedding(seed):
     return (bits.astype(np.uint32) << 16).view(np.float32)
 
 
-def test_decode_step_store_mode_against_oracle(sf):
+@pytest.mark.parametrize("fused", [False, True])
+def test_decode_step_store_mode_against_oracle(sf, fused):
     """Refinement stores in device memory: the teacher-forced checks of one
     step, the logits of the whole step against oracle.decode.decode_step, and
-    a graph replay that reproduces the eager step bit for bit."""
+    a graph replay that reproduces the eager step bit for bit; with the input
+    rows made by stand-alone producers or inside the GEMV launches."""
     host = _host_model()
-    m = _build(sf, host)
+    m = _build(sf, host, fused_producers=fused)
     olayers, ohead, ofinal, okv = _oracle_model(host)
     x0 = _embedding(7000)
     m.x_in.copy_(torch.from_numpy(x0))
@@ -248,8 +250,9 @@ def test_decode_step_store_mode_against_oracle(sf):
     m.close()
 
 
-@pytest.mark.parametrize("deadline,lead", [(False, False), (True, False), (True, True)])
-def test_decode_step_cache_mode_against_oracle(sf, deadline, lead):
+@pytest.mark.parametrize("deadline,lead,fused", [(False, False, False), (True, False, False), (True, True, False),
+                                                 (True, True, True)])
+def test_decode_step_cache_mode_against_oracle(sf, deadline, lead, fused):
     """Weight refinements behind 25% LRU caches and K/V refinements behind a
     20% KV refinement cache per layer with a fetch budget, over three decode
     steps at positions T0, T0+1, T0+2: every op of every step, the attention
@@ -258,11 +261,12 @@ def test_decode_step_cache_mode_against_oracle(sf, deadline, lead):
     the deadline reading the GEMVs refine only the selected columns cached
     when the step starts (and never wait for a fetch); with fetch lead the
     q/k/v, gate/up and LM-head caches are first stepped with the channels
-    predicted from the residual stream a block ahead."""
+    predicted from the residual stream a block ahead.  ``fused``: the GEMVs
+    make their input rows and selections in their own launches."""
     host = _host_model()
     budget = 12                                   # per KV head and step
     m = _build(sf, host, weight_cache_pct=25, kv_cache_pct=20, kv_budget=budget, weight_deadline=deadline,
-               fetch_lead=lead)
+               fetch_lead=lead, fused_producers=fused)
     olayers, ohead, ofinal, okv = _oracle_model(host)
     # oracle LRUs: q (attn_in), o, gate (mlp_in), down, head; the KV caches
     worcs = {slot: [ocache.LRUCache(K, od.count_half_up(Fraction(25, 100), K)) for _ in range(NL)]
