@@ -904,7 +904,10 @@ def run_sf(args, rank, world, local_rank, dist):
     outl = ds.outlier_channels(5000, H, count_fraction(OUTLIER_PCT, H), dev)
     pool = torch.stack([ds.activations(2000 + i, 1, H, outl, OUTLIER_SCALE, dev)[0].float()
                         for i in range(n_total)])
-    cap_stream = torch.cuda.Stream(device=dev)
+    # the step's own stream above the side streams' priority (theirs is the
+    # default, the lowest): when SMs free up, the critical path's blocks go
+    # first (measured: 7.39 -> 7.33 ms per step at 128K)
+    cap_stream = torch.cuda.Stream(device=dev, priority=-1)
     # one eager step (cold caches fill), then the step as one graph
     model.x_in.copy_(pool[0])
     with torch.cuda.stream(cap_stream):

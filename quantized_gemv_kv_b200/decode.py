@@ -142,6 +142,8 @@ class DecodeModel:
         self.K_in = {"attn_in": H, "attn_out": Hq * d, "mlp_in": H, "mlp_mid": F, "head": H}
         slot_of = {"q": "attn_in", "k": "attn_in", "v": "attn_in", "o": "attn_out", "gate": "mlp_in",
                    "up": "mlp_in", "down": "mlp_mid"}
+        # side streams at the default (lowest) priority: a step run on a
+        # higher-priority stream keeps its critical path ahead of them
         self.side = torch.cuda.Stream(device=dev)      # weight caches' steps and gathers
         self.side_kv = torch.cuda.Stream(device=dev)   # the KV caches' bookkeeping and gathers
         self.layers = []
