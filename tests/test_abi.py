@@ -134,3 +134,33 @@ def test_attention_binding_refuses_bad_output_buffers_before_any_call(sf):
     # well-formed buffers still stop at the device check on a CPU tensor
     with pytest.raises(ValueError, match="CUDA"):
         sf.attn_decode_refine_noalloc(q, kv, Hkv, 64, k, out, sel, sel_n)
+
+
+def test_host_validation_gemv_produce(sf):
+    """sf_gemv_refine_batch1_produce checks its producer on the host, before
+    any device work: the op, its pointers, y's alignment, the selection's
+    room in the launch's scratch, and an updated residual that overlaps x."""
+    L = sf._lib
+    qw = sf._QWeight(256, 256, 256, 256, 64, 4096, 128, 2, 2)
+    job = sf._GemvJob(ctypes.pointer(qw), None, 1, 256, None)
+    jp = ctypes.cast(ctypes.pointer(job), ctypes.c_void_p)
+
+    def call(op=sf.PRODUCE_ROUND, k=10, x=4096, w=None, u=None, x_out=None, y=8192):
+        pr = sf._GemvProducer(op, k, 1e-5, x, None, w, u, x_out, y, 256, 256)
+        return L.sf_gemv_refine_batch1_produce(jp, 1, ctypes.cast(ctypes.pointer(pr), ctypes.c_void_p), None)
+
+    assert L.sf_gemv_refine_batch1_produce(jp, 1, None, None) == sf.SF_EINVAL
+    assert call(op=7) == sf.SF_EINVAL
+    assert "unknown producer op" in _err(sf)
+    assert call(op=sf.PRODUCE_NORM) == sf.SF_EINVAL
+    assert "needs w" in _err(sf)
+    assert call(op=sf.PRODUCE_SILU_MUL) == sf.SF_EINVAL
+    assert "needs u" in _err(sf)
+    assert call(y=8194) == sf.SF_EINVAL
+    assert "aligned" in _err(sf)
+    # 2-bit codes at K = 4096: the whole row is more than the scratch holds
+    assert call(k=4096) == sf.SF_EINVAL
+    assert "k must be" in _err(sf)
+    assert call(k=-1) == sf.SF_EINVAL
+    assert call(op=sf.PRODUCE_NORM, w=4096, x_out=4096 + 4 * 100) == sf.SF_EINVAL
+    assert "x_out" in _err(sf)
