@@ -723,6 +723,24 @@ sf_status sf_kv_append_pair_cached(const float* k_src, const float* v_src, int H
                                    uint32_t* v_res, uint16_t* v_scale, uint16_t* v_zero, sf_refine_cache* ref_cache,
                                    sf_stream_t stream, sf_stream_t side);
 
+/*
+ * sf_rope_kv_append_pair_cached -- sf_rope_qk(q, Hq, k, Hkv, d, pos, theta,
+ *   q_bf16) followed by sf_kv_append_pair_cached of the rotated k and of v,
+ *   in one launch with the same results bit for bit: the key rows are
+ *   rotated in registers before they are quantized (and written back to k),
+ *   while other blocks of the launch rotate the query heads (q in place,
+ *   q_bf16 when it is not NULL).  The rotation and the append are the steps
+ *   of a decode step between the q/k/v projections and the attention (RoPE
+ *   of the new token, then its K/V rows appended; the attention reads both).
+ *   Constraints: those of sf_rope_qk and sf_kv_append_pair_cached, with d a
+ *   multiple of 64 (the thread that holds dim i also holds i + d/2).
+ */
+sf_status sf_rope_kv_append_pair_cached(float* q, int Hq, uint16_t* q_bf16, float* k, const float* v, int Hkv, int d,
+                                        int pos, double theta, int row_stride, int t, int b_r, int b_f,
+                                        uint32_t* k_res, uint16_t* k_scale, uint16_t* k_zero, uint32_t* v_res,
+                                        uint16_t* v_scale, uint16_t* v_zero, sf_refine_cache* ref_cache,
+                                        sf_stream_t stream, sf_stream_t side);
+
 #ifdef __cplusplus
 }
 #endif

@@ -125,6 +125,8 @@ _SIGS = {
     "sf_kv_append_cached": ([_p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _i, _p], _i),
     "sf_gemv_set_launch_overlap": ([_i], _i),
     "sf_kv_append_pair_cached": ([_p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p], _i),
+    "sf_rope_kv_append_pair_cached": ([_p, _i, _p, _p, _p, _i, _i, _i, ctypes.c_double, _i, _i, _i, _i, _p, _p, _p,
+                                       _p, _p, _p, _p, _p, _p], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -687,6 +689,30 @@ def kv_append_pair_cached(k_src: torch.Tensor, v_src: torch.Tensor, kq: "QWeight
     _check(_lib.sf_kv_append_pair_cached(_ptr(k_src), _ptr(v_src), Hkv, d, row_stride, t, b_r, b_f, _ptr(kq.res),
                                          _ptr(kq.scale), _ptr(kq.zero), _ptr(vq.res), _ptr(vq.scale), _ptr(vq.zero),
                                          cache.handle, st, _stream(side) if side is not None else st))
+
+
+def rope_kv_append_pair_cached(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kq: "QWeight", vq: "QWeight",
+                               cache: RefineCache, row_stride: int, t: int, pos: int, b_r: int = 2, b_f: int = 2,
+                               theta: float = 500000.0, q_bf16: torch.Tensor | None = None,
+                               stream: torch.cuda.Stream | None = None, side: torch.cuda.Stream | None = None) -> None:
+    """``sf_rope_kv_append_pair_cached``: RoPE of q [Hq][d] (in place, and as
+    bf16 to q_bf16) and k [Hkv][d] to position pos, then the rotated key and
+    the value rows of token t appended, in one launch."""
+    for name, a in (("q", q), ("k", k), ("v", v)):
+        _dev(a, name)
+        if a.dtype != torch.float32 or a.dim() != 2:
+            raise ValueError(f"{name} must be a 2-D float32 tensor")
+    if v.shape != k.shape or q.shape[1] != k.shape[1]:
+        raise ValueError("k and v must have one shape, and q the same head dim")
+    if q_bf16 is not None and (q_bf16.dtype != torch.bfloat16 or q_bf16.numel() != q.numel()):
+        raise ValueError("q_bf16 must be bfloat16 with q's size")
+    Hq, d = q.shape
+    Hkv = k.shape[0]
+    st = _stream(stream)
+    _check(_lib.sf_rope_kv_append_pair_cached(_ptr(q), Hq, _ptr(q_bf16), _ptr(k), _ptr(v), Hkv, d, pos, theta,
+                                              row_stride, t, b_r, b_f, _ptr(kq.res), _ptr(kq.scale), _ptr(kq.zero),
+                                              _ptr(vq.res), _ptr(vq.scale), _ptr(vq.zero), cache.handle, st,
+                                              _stream(side) if side is not None else st))
 
 
 def norm_select(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor, k: int, idx: torch.Tensor, n: torch.Tensor,

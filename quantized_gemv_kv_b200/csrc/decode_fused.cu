@@ -163,11 +163,8 @@ __global__ void rope_qk_kernel(float* __restrict__ q, int Hq, float* __restrict_
   if (i >= half) return;
   const bool is_q = static_cast<int>(blockIdx.x) < Hq;
   float* xh = is_q ? q + static_cast<size_t>(blockIdx.x) * d : kk + static_cast<size_t>(blockIdx.x - Hq) * d;
-  const double ang = static_cast<double>(pos) * pow(theta, -2.0 * i / d);
-  double s, c;
-  sincos(ang, &s, &c);
-  const double lo = xh[i], hi = xh[i + half];
-  const double rlo = lo * c - hi * s, rhi = hi * c + lo * s;
+  double rlo, rhi;
+  sfd::rope_pair(xh[i], xh[i + half], i, d, pos, theta, rlo, rhi);
   xh[i] = static_cast<float>(rlo);
   xh[i + half] = static_cast<float>(rhi);
   if (is_q && q_bf16) {

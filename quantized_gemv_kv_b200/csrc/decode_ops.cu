@@ -8,9 +8,12 @@
 // rounded once (to fp32 for the fp32 outputs, to bf16 with ties to even for
 // the GEMV and attention inputs), so the results sit within one rounding of
 // the exact values.
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "produce.cuh"
 #include "sf_internal.h"
 
 namespace {
@@ -57,12 +60,9 @@ add_rmsnorm_kernel(float* __restrict__ x, const float* __restrict__ delta, const
 __global__ void rope_kernel(float* __restrict__ x, int d, int pos, double theta, uint16_t* __restrict__ y) {
   const int half = d >> 1, i = threadIdx.x;
   if (i >= half) return;
-  const double ang = static_cast<double>(pos) * pow(theta, -2.0 * i / d);
-  double s, c;
-  sincos(ang, &s, &c);
   float* xh = x + static_cast<size_t>(blockIdx.x) * d;
-  const double lo = xh[i], hi = xh[i + half];
-  const double rlo = lo * c - hi * s, rhi = hi * c + lo * s;
+  double rlo, rhi;
+  sfd::rope_pair(xh[i], xh[i + half], i, d, pos, theta, rlo, rhi);
   xh[i] = static_cast<float>(rlo);
   xh[i + half] = static_cast<float>(rhi);
   if (y) {
@@ -93,21 +93,45 @@ constexpr int kAppendMaxD = 512;
 // g * row_stride + t: resident and refinement bitstreams (row-major, little
 // endian), fp16 scale and zero.  The refinement words go to ref_row and, when
 // crow is not null (the unit is cached), to crow as well, so a cached copy
-// never goes stale.
+// never goes stale.  With rope_pos >= 0 the row is first rotated to that
+// position (sfd::rope_pair, each value rounded to fp32 once, d a multiple of
+// 64 so that a lane holds both dims of its pairs) and written back to rot_out.
+// PER: d / 32 known at compile time (the row stays in registers), 0: any d.
+template <int PER>
 __device__ void append_row(const float* __restrict__ row, int d, int b_r, int b_f, size_t r, uint32_t* __restrict__ res,
                            uint16_t* __restrict__ scale, uint16_t* __restrict__ zero, uint32_t* __restrict__ ref_row,
-                           uint32_t* __restrict__ crow, uint8_t* codes) {
+                           uint32_t* __restrict__ crow, uint8_t* codes, int rope_pos = -1, double theta = 0.0,
+                           float* rot_out = nullptr) {
+  constexpr int kMax = PER > 0 ? PER : kAppendMaxD / 32;
   const int lane = threadIdx.x & 31;
   const int b = b_r + b_f;
   const float qmax = static_cast<float>((1 << b) - 1);
-  const int per_lane = d >> 5;
-  float v[kAppendMaxD / 32];
-  float lo = INFINITY, hi = -INFINITY;
-  for (int m = 0; m < per_lane; ++m) {
-    v[m] = row[lane + 32 * m];
-    lo = fminf(lo, v[m]);
-    hi = fmaxf(hi, v[m]);
+  const int per_lane = PER > 0 ? PER : d >> 5;
+  float v[kMax];
+#pragma unroll
+  for (int m = 0; m < kMax; ++m)
+    if (m < per_lane) v[m] = row[lane + 32 * m];
+  if (rope_pos >= 0) {
+    const int hm = per_lane >> 1;  // dim lane + 32 m pairs with dim lane + 32 (m + hm)
+#pragma unroll
+    for (int m = 0; m < kMax / 2; ++m)
+      if (m < hm) {
+        double rlo, rhi;
+        sfd::rope_pair(v[m], v[m + hm], lane + 32 * m, d, rope_pos, theta, rlo, rhi);
+        v[m] = static_cast<float>(rlo);
+        v[m + hm] = static_cast<float>(rhi);
+      }
+#pragma unroll
+    for (int m = 0; m < kMax; ++m)
+      if (m < per_lane) rot_out[lane + 32 * m] = v[m];
   }
+  float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+  for (int m = 0; m < kMax; ++m)
+    if (m < per_lane) {
+      lo = fminf(lo, v[m]);
+      hi = fmaxf(hi, v[m]);
+    }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
@@ -125,11 +149,13 @@ __device__ void append_row(const float* __restrict__ row, int d, int b_r, int b_
     scale[r] = __half_as_ushort(s16);
     zero[r] = __half_as_ushort(__int2half_rn(zi));
   }
-  for (int m = 0; m < per_lane; ++m) {
-    float qf = rintf(__fdiv_rn(v[m], sf)) + static_cast<float>(zi);
-    qf = fminf(fmaxf(qf, 0.0f), qmax);
-    codes[lane + 32 * m] = static_cast<uint8_t>(static_cast<int>(qf));
-  }
+#pragma unroll
+  for (int m = 0; m < kMax; ++m)
+    if (m < per_lane) {
+      float qf = rintf(__fdiv_rn(v[m], sf)) + static_cast<float>(zi);
+      qf = fminf(fmaxf(qf, 0.0f), qmax);
+      codes[lane + 32 * m] = static_cast<uint8_t>(static_cast<int>(qf));
+    }
   __syncwarp();
   const uint32_t rmask = (1u << b_r) - 1u, fmask = (1u << b_f) - 1u;
   const int rw = d * b_r / 32, fw = d * b_f / 32;
@@ -169,8 +195,12 @@ __global__ void kv_append_kernel(const float* __restrict__ src, int Hkv, int d, 
     const int slot = unit_slot[r];
     if (slot >= 0) crow = crows + static_cast<size_t>(slot) * ref_pitch + ref_off;
   }
-  append_row(src + static_cast<size_t>(g) * d, d, b_r, b_f, r, res, scale, zero, ref + r * ref_pitch + ref_off, crow,
-             codes[warp]);
+  if (d == 128)
+    append_row<4>(src + static_cast<size_t>(g) * d, d, b_r, b_f, r, res, scale, zero, ref + r * ref_pitch + ref_off,
+                  crow, codes[warp]);
+  else
+    append_row<0>(src + static_cast<size_t>(g) * d, d, b_r, b_f, r, res, scale, zero, ref + r * ref_pitch + ref_off,
+                  crow, codes[warp]);
 }
 
 // The key and value rows of token t in one launch (blockIdx.y: 0 keys, 1
@@ -186,19 +216,52 @@ struct AppendPair {
   const int32_t* unit_slot;
   uint32_t* crows;
   int Hkv, d, row_stride, t, b_r, b_f;
+  // RoPE to position rope_pos (< 0: none) of the keys, rotated in place in
+  // src[0] before they are quantized, and of the Hq query heads in q (in
+  // place, and as bf16 to q_bf16 when it is not null), by blockIdx.y == 2
+  int rope_pos, Hq;
+  double theta;
+  float* k_rot;
+  float* q;
+  uint16_t* q_bf16;
 };
 
 __global__ void kv_append_pair_kernel(const __grid_constant__ AppendPair A) {
   __shared__ uint8_t codes[4][kAppendMaxD];
-  const int warp = threadIdx.x >> 5, part = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, part = blockIdx.y;
   const int g = blockIdx.x * 4 + warp;
+  if (part == 2) {  // a warp per query head
+    if (g >= A.Hq) return;  // uniform over the warp
+    float* xh = A.q + static_cast<size_t>(g) * A.d;
+    const int half = A.d >> 1;
+    for (int i = lane; i < half; i += 32) {
+      double rlo, rhi;
+      sfd::rope_pair(xh[i], xh[i + half], i, A.d, A.rope_pos, A.theta, rlo, rhi);
+      xh[i] = static_cast<float>(rlo);
+      xh[i + half] = static_cast<float>(rhi);
+      if (A.q_bf16 != nullptr) {
+        uint16_t* yh = A.q_bf16 + static_cast<size_t>(g) * A.d;
+        yh[i] = sfd::to_bf16(rlo);
+        yh[i + half] = sfd::to_bf16(rhi);
+      }
+    }
+    return;
+  }
   if (g >= A.Hkv) return;  // uniform over the warp
   const int fw = A.d * A.b_f / 32;
   const size_t r = static_cast<size_t>(g) * A.row_stride + A.t;
   const int slot = A.unit_slot[r];
   uint32_t* crow = slot >= 0 ? A.crows + static_cast<size_t>(slot) * 2 * fw + part * fw : nullptr;
-  append_row(A.src[part] + static_cast<size_t>(g) * A.d, A.d, A.b_r, A.b_f, r, A.res[part], A.scale[part],
-             A.zero[part], A.stage + static_cast<size_t>(g) * 2 * fw + part * fw, crow, codes[warp]);
+  const bool rot = part == 0 && A.rope_pos >= 0;
+  const float* row = A.src[part] + static_cast<size_t>(g) * A.d;
+  uint32_t* stage = A.stage + static_cast<size_t>(g) * 2 * fw + part * fw;
+  float* rot_out = rot ? A.k_rot + static_cast<size_t>(g) * A.d : nullptr;
+  if (A.d == 128)
+    append_row<4>(row, A.d, A.b_r, A.b_f, r, A.res[part], A.scale[part], A.zero[part], stage, crow, codes[warp],
+                  rot ? A.rope_pos : -1, A.theta, rot_out);
+  else
+    append_row<0>(row, A.d, A.b_r, A.b_f, r, A.res[part], A.scale[part], A.zero[part], stage, crow, codes[warp],
+                  rot ? A.rope_pos : -1, A.theta, rot_out);
 }
 
 }  // namespace
@@ -251,28 +314,34 @@ extern "C" sf_status sf_kv_append(const float* src, int Hkv, int d, int row_stri
   return sf::check_launch("kv_append_kernel");
 }
 
-extern "C" sf_status sf_kv_append_pair_cached(const float* k_src, const float* v_src, int Hkv, int d, int row_stride,
-                                              int t, int b_r, int b_f, uint32_t* k_res, uint16_t* k_scale,
-                                              uint16_t* k_zero, uint32_t* v_res, uint16_t* v_scale, uint16_t* v_zero,
-                                              sf_refine_cache* ref_cache, sf_stream_t stream, sf_stream_t side) {
+namespace {
+
+// The pair append, with RoPE of q and k in the same launch when q is given.
+sf_status append_pair(const char* what, float* q, int Hq, uint16_t* q_bf16, int pos, double theta, const float* k_src,
+                      const float* v_src, int Hkv, int d, int row_stride, int t, int b_r, int b_f, uint32_t* k_res,
+                      uint16_t* k_scale, uint16_t* k_zero, uint32_t* v_res, uint16_t* v_scale, uint16_t* v_zero,
+                      sf_refine_cache* ref_cache, sf_stream_t stream, sf_stream_t side) {
   SF_REQUIRE(k_src && v_src && k_res && k_scale && k_zero && v_res && v_scale && v_zero && ref_cache,
-             "sf_kv_append_pair_cached: null pointer");
-  SF_REQUIRE(Hkv >= 1, "sf_kv_append_pair_cached: Hkv must be >= 1");
-  SF_REQUIRE(d >= 32 && d % 32 == 0 && d <= kAppendMaxD,
-             "sf_kv_append_pair_cached: d must be a multiple of 32 in [32, %d]", kAppendMaxD);
-  SF_REQUIRE(b_r == 2 || b_r == 3, "sf_kv_append_pair_cached: b_r must be 2 or 3");
-  SF_REQUIRE(b_f == 1 || b_f == 2, "sf_kv_append_pair_cached: b_f must be 1 or 2");
-  SF_REQUIRE(b_r + b_f <= 4, "sf_kv_append_pair_cached: b_r + b_f must be <= 4");
-  SF_REQUIRE(row_stride >= 1 && t >= 0 && t < row_stride, "sf_kv_append_pair_cached: need 0 <= t < row_stride");
+             "%s: null pointer", what);
+  SF_REQUIRE(Hkv >= 1, "%s: Hkv must be >= 1", what);
+  SF_REQUIRE(d >= 32 && d % 32 == 0 && d <= kAppendMaxD, "%s: d must be a multiple of 32 in [32, %d]", what,
+             kAppendMaxD);
+  SF_REQUIRE(b_r == 2 || b_r == 3, "%s: b_r must be 2 or 3", what);
+  SF_REQUIRE(b_f == 1 || b_f == 2, "%s: b_f must be 1 or 2", what);
+  SF_REQUIRE(b_r + b_f <= 4, "%s: b_r + b_f must be <= 4", what);
+  SF_REQUIRE(row_stride >= 1 && t >= 0 && t < row_stride, "%s: need 0 <= t < row_stride", what);
+  if (q != nullptr) {
+    SF_REQUIRE(Hq >= 1 && d % 64 == 0, "%s: need Hq >= 1 and d a multiple of 64 for the rotation", what);
+    SF_REQUIRE(pos >= 0 && theta > 0.0, "%s: need pos >= 0 and theta > 0", what);
+  }
   cudaStream_t s = sf::as_cuda(stream);
   sf::CacheWriteView w{};
   sf_status st = sf::cache_view_for_writer(ref_cache, s, &w);
   if (st != SF_OK) return st;
   const int fw = d * b_f / 32;
-  SF_REQUIRE(w.unit_words == 2 * fw, "sf_kv_append_pair_cached: the cache's units must be %d bytes (K then V words)",
-             8 * fw);
+  SF_REQUIRE(w.unit_words == 2 * fw, "%s: the cache's units must be %d bytes (K then V words)", what, 8 * fw);
   SF_REQUIRE(static_cast<long long>(w.num_units) >= static_cast<long long>(Hkv) * row_stride,
-             "sf_kv_append_pair_cached: the cache has fewer units than Hkv * row_stride");
+             "%s: the cache has fewer units than Hkv * row_stride", what);
   uint32_t* stage = nullptr;
   st = sf::cache_append_stage(ref_cache, s, static_cast<size_t>(Hkv) * 2 * fw, &stage);
   if (st != SF_OK) return st;
@@ -294,7 +363,14 @@ extern "C" sf_status sf_kv_append_pair_cached(const float* k_src, const float* v
   A.t = t;
   A.b_r = b_r;
   A.b_f = b_f;
-  kv_append_pair_kernel<<<dim3((Hkv + 3) / 4, 2), 128, 0, s>>>(A);
+  A.rope_pos = q != nullptr ? pos : -1;
+  A.Hq = q != nullptr ? Hq : 0;
+  A.theta = theta;
+  A.k_rot = const_cast<float*>(k_src);
+  A.q = q;
+  A.q_bf16 = q_bf16;
+  const int gx = std::max((Hkv + 3) / 4, (A.Hq + 3) / 4);
+  kv_append_pair_kernel<<<dim3(gx, q != nullptr ? 3 : 2), 128, 0, s>>>(A);
   st = sf::check_launch("kv_append_pair_kernel");
   if (st != SF_OK) return st;
   st = sf::cache_mark_used(ref_cache, s);
@@ -302,6 +378,27 @@ extern "C" sf_status sf_kv_append_pair_cached(const float* k_src, const float* v
   // rows g * row_stride + t of the master, one per KV head
   return sf::cache_append_flush(ref_cache, s, sf::as_cuda(side), static_cast<size_t>(t) * 2 * fw * 4,
                                 static_cast<size_t>(row_stride) * 2 * fw * 4, static_cast<size_t>(2 * fw) * 4, Hkv);
+}
+
+}  // namespace
+
+extern "C" sf_status sf_kv_append_pair_cached(const float* k_src, const float* v_src, int Hkv, int d, int row_stride,
+                                              int t, int b_r, int b_f, uint32_t* k_res, uint16_t* k_scale,
+                                              uint16_t* k_zero, uint32_t* v_res, uint16_t* v_scale, uint16_t* v_zero,
+                                              sf_refine_cache* ref_cache, sf_stream_t stream, sf_stream_t side) {
+  return append_pair("sf_kv_append_pair_cached", nullptr, 0, nullptr, 0, 0.0, k_src, v_src, Hkv, d, row_stride, t,
+                     b_r, b_f, k_res, k_scale, k_zero, v_res, v_scale, v_zero, ref_cache, stream, side);
+}
+
+extern "C" sf_status sf_rope_kv_append_pair_cached(float* q, int Hq, uint16_t* q_bf16, float* k, const float* v,
+                                                   int Hkv, int d, int pos, double theta, int row_stride, int t,
+                                                   int b_r, int b_f, uint32_t* k_res, uint16_t* k_scale,
+                                                   uint16_t* k_zero, uint32_t* v_res, uint16_t* v_scale,
+                                                   uint16_t* v_zero, sf_refine_cache* ref_cache, sf_stream_t stream,
+                                                   sf_stream_t side) {
+  SF_REQUIRE(q, "sf_rope_kv_append_pair_cached: null pointer");
+  return append_pair("sf_rope_kv_append_pair_cached", q, Hq, q_bf16, pos, theta, k, v, Hkv, d, row_stride, t, b_r,
+                     b_f, k_res, k_scale, k_zero, v_res, v_scale, v_zero, ref_cache, stream, side);
 }
 
 extern "C" sf_status sf_kv_append_cached(const float* src, int Hkv, int d, int row_stride, int t, int b_r, int b_f,

@@ -809,15 +809,22 @@ gemv_mma_kernel(const __grid_constant__ MArgs a) {
       const int rows = pair ? kRows / 2 : kRows, r0 = ks * rows;
       const float* red0 = pair ? cl.map_shared_rank(red, 0) : red;
       const float* red1 = pair ? cl.map_shared_rank(red, 1) : red;
+      // every partial of a row is loaded before the sum (the partner's are
+      // remote loads), then added in warp order
+      auto sum_warps = [&](const float* rd, int ti, int rr) {
+        float t[kMaxWarps];
+#pragma unroll
+        for (int w = 0; w < kMaxWarps; ++w) t[w] = w < W ? rd[(ti * W + w) * kRows + rr] : 0.0f;
+        float acc = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kMaxWarps; ++w)
+          if (w < W) acc += t[w];
+        return acc;
+      };
       for (int e = tid; e < nt * rows; e += blockDim.x) {
         const int ti = e / rows, rr = r0 + e % rows;
-        float acc = 0.0f;
-        for (int w = 0; w < W; ++w) acc += red0[(ti * W + w) * kRows + rr];
-        if (pair) {
-          float acc1 = 0.0f;
-          for (int w = 0; w < W; ++w) acc1 += red1[(ti * W + w) * kRows + rr];
-          acc += acc1;
-        }
+        float acc = sum_warps(red0, ti, rr);
+        if (pair) acc += sum_warps(red1, ti, rr);
         const int tt = t_begin + i0 + ti;
         const MJob& Jt = a.job[job_of(a, tt)];
         Jt.y[(tt - Jt.tile_begin) * kRows + rr] = acc;

@@ -38,4 +38,17 @@ __device__ __forceinline__ uint16_t silu_mul_bf16(float g, float u) {
 // order, so every kernel that normalises a row gets the same bits.
 constexpr int kNormVThreads = 1024;
 
+// RoPE of the pair (i, i + d/2) of one head at position pos: the angle
+// pos theta^(-2i/d), its sine and cosine and the rotation in fp64 (each
+// result rounded once by the caller).  Shared by every kernel that rotates,
+// so a key rotated inside the K/V append equals one rotated on its own.
+__device__ __forceinline__ void rope_pair(double lo, double hi, int i, int d, int pos, double theta, double& rlo,
+                                          double& rhi) {
+  const double ang = static_cast<double>(pos) * pow(theta, -2.0 * i / d);
+  double s, c;
+  sincos(ang, &s, &c);
+  rlo = lo * c - hi * s;
+  rhi = hi * c + lo * s;
+}
+
 }  // namespace sfd

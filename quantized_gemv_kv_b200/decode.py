@@ -13,7 +13,9 @@ memory with 3-bit weights and 2-bit KV).  Per layer, batch 1:
                                           sf_gemv_refine_batch1
   q, k rotated to position T              sf_rope_qk (q also as bf16)
   k, v quantized, appended as token T     sf_kv_append (with a KV refinement
-                                          cache: sf_kv_append_pair_cached)
+                                          cache, both rows and the rotation
+                                          in one launch:
+                                          sf_rope_kv_append_pair_cached)
   a = refined attention over T + 1        sf_attn_decode_refine (+ the KV
                                           refinement cache's prefetch)
   h = x + o(bf16(a))                      sf_round_select, GEMV, sf_norm_select
@@ -52,7 +54,7 @@ import torch
 
 from . import (PRODUCE_NORM, PRODUCE_ROUND, PRODUCE_SILU_MUL, QKV, Batch1Jobs, RefineCache, RefineGroup, act_bytes,
                attn_decode_refine, attn_union_units, attn_workspace_size, gemv_set_launch_overlap, kv_append,
-               kv_append_pair_cached, norm_select, pack_batch1, quantize_nested, rope_qk, round_select,
+               norm_select, pack_batch1, quantize_nested, rope_kv_append_pair_cached, rope_qk, round_select,
                silu_mul_select)
 
 MATS = ("q", "k", "v", "o", "gate", "up", "down")
@@ -407,17 +409,18 @@ class DecodeModel:
                 self.qkv_raw[l, :Hq * d].copy_(L["q"].y)
                 self.qkv_raw[l, Hq * d:(Hq + Hkv) * d].copy_(L["k"].y)
                 self.qkv_raw[l, (Hq + Hkv) * d:].copy_(L["v"].y)
-            rope_qk(q, k, T, s.theta, q_bf16=self.q_bf[l])
-            if self.record:
-                self.k_rot[l].copy_(k)
             kq, vq = L["kv"].k, L["kv"].v
             if L["kv_cache"] is None:
+                rope_qk(q, k, T, s.theta, q_bf16=self.q_bf[l])
                 kv_append(k, kq.res, kq.ref, kq.scale, kq.zero, self.S, T, b_r, b_f)
                 kv_append(v, vq.res, vq.ref, vq.scale, vq.zero, self.S, T, b_r, b_f)
-            else:  # the new token's refinement bits go to the host master (and a cached copy); the
-                # master's copy runs on the KV side stream, ahead of that stream's prefetch
-                kv_append_pair_cached(k, v, kq, vq, L["kv_cache"], self.S, T, b_r, b_f, stream=main, side=self.side_kv)
+            else:  # RoPE and the append in one launch; the new token's refinement bits go to the
+                # host master (and a cached copy), the master's copy on the KV side stream
+                rope_kv_append_pair_cached(q, k, v, kq, vq, L["kv_cache"], self.S, T, T, b_r, b_f, theta=s.theta,
+                                           q_bf16=self.q_bf[l], stream=main, side=self.side_kv)
                 kv_used = True
+            if self.record:
+                self.k_rot[l].copy_(k)
             attn_decode_refine(self.q_bf[l], L["kv"], Hkv, T + 1, k_tok, workspace=self.ws, out=self.att[l],
                                sel_out=self.sel[l], sel_n=self.sel_n[l])
             if L["kv_cache"] is not None and refine and k_tok > 0:

@@ -181,3 +181,52 @@ def test_kv_append_pair_cached(sf, t, b_f):
     keep[t] = False
     assert np.all(master.numpy().reshape(Hkv, S, unit)[:, keep] == 0xA5)
     cache.close()
+
+
+@pytest.mark.parametrize("t,pos", [(0, 0), (17, 131071), (63, 5)])
+def test_rope_kv_append_pair_cached_equals_separate(sf, t, pos):
+    """RoPE of q and k and the append of the rotated key and value rows in one
+    launch equal sf_rope_qk followed by sf_kv_append_pair_cached, bit for bit:
+    q, its bf16 copy, the rotated k, the resident codes, scales and zeros and
+    the refinement words in the host master."""
+    Hq, Hkv, d, S, b_r, b_f = 32, 8, 128, 64, 2, 2
+    rng = np.random.default_rng(1300 + t)
+    q0 = (rng.standard_normal((Hq, d)) * 3).astype(np.float32)
+    k0 = (rng.standard_normal((Hkv, d)) * 3).astype(np.float32)
+    v0 = (rng.standard_normal((Hkv, d)) * 3).astype(np.float32)
+    fw = d * b_f // 32
+    unit = 2 * fw * 4
+
+    class _Q:  # the views the binding reads
+        def __init__(self, res, scale, zero):
+            self.res, self.scale, self.zero = res, scale, zero
+
+    outs = []
+    for fused in (False, True):
+        master = torch.full((Hkv * S * unit,), 0xA5, dtype=torch.uint8).pin_memory()
+        cache = sf.RefineCache(Hkv * S, unit, 8, 8, master)
+        cache.preload(torch.tensor([3 * S + t], dtype=torch.int32, device="cuda"))
+        rows = Hkv * S
+        kq = _Q(torch.zeros((rows, d * b_r // 32), dtype=torch.int32, device="cuda"),
+                torch.zeros((rows,), dtype=torch.float16, device="cuda"),
+                torch.zeros((rows,), dtype=torch.float16, device="cuda"))
+        vq = _Q(torch.zeros((rows, d * b_r // 32), dtype=torch.int32, device="cuda"),
+                torch.zeros((rows,), dtype=torch.float16, device="cuda"),
+                torch.zeros((rows,), dtype=torch.float16, device="cuda"))
+        q, k, v = dev(q0), dev(k0), dev(v0)
+        qb = torch.zeros((Hq, d), dtype=torch.bfloat16, device="cuda")
+        side = torch.cuda.Stream()
+        if fused:
+            sf.rope_kv_append_pair_cached(q, k, v, kq, vq, cache, S, t, pos, b_r, b_f, q_bf16=qb, side=side)
+        else:
+            sf.rope_qk(q, k, pos, q_bf16=qb)
+            sf.kv_append_pair_cached(k, v, kq, vq, cache, S, t, b_r, b_f, side=side)
+        side.synchronize()
+        torch.cuda.synchronize()
+        outs.append([q.cpu(), qb.view(torch.int16).cpu(), k.cpu()] +
+                    [a.cpu().view(torch.int16) if a.dtype == torch.float16 else a.cpu()
+                     for a in (kq.res, kq.scale, kq.zero, vq.res, vq.scale, vq.zero)] + [master.clone()])
+        cache.close()
+    for a, b in zip(*outs):
+        assert torch.equal(a.view(torch.int32) if a.dtype == torch.float32 else a,
+                           b.view(torch.int32) if b.dtype == torch.float32 else b)
