@@ -44,6 +44,9 @@ SLOTS = (("attn_in", 4096), ("attn_out", 4096), ("mlp_in", 4096), ("mlp_mid", 14
 G, B_R, B_F = 128, 2, 2
 HQ, HKV, D = 32, 8, 128
 TOPK_PCT, CACHE_PCT, OUTLIER_PCT, OUTLIER_SCALE = 3, 10, "1/2", 30.0
+# the headline metric; both arms (this library, and the oracle as the
+# reference) report it under this name
+METRIC = "effective HBM GB/s (refined low-bit decode step) and tokens/s at 128K"
 TOK_PCT = 1
 
 
@@ -504,6 +507,22 @@ def cpu_model():
     return "unknown"
 
 
+def step_config(args) -> dict:
+    """The headline workload, as both arms report it in ``config``."""
+    return {"workload": workload_step(args.context), "model_shape": "Llama-3.1-8B (32 layers, LM head 128256)",
+            "context": args.context, "layers": args.layers, "batch": 1,
+            "weights": "3-bit resident + 1-bit refinement, group 128", "kv": "2-bit + 2-bit, per token-head",
+            "topk_channels": "3% of each GEMV input",
+            "weight_cache": "10% LRU per matrix, " + ("deadline reading (misses fetched for later steps)"
+                                                       if args.weight_deadline else "every GEMV waits for its misses")
+            + ("; fetch lead: q/k/v, gate/up and LM-head channels predicted from the residual stream "
+               "a block ahead and prefetched" if args.fetch_lead and args.weight_deadline else ""),
+            "topk_tokens": "1% per query head",
+            "kv_cache": (f"{args.kv_cache_pct}% of token-heads, one LRU per KV head, budget {args.kv_budget} per "
+                         "head and step" if args.kv_cache_pct >= 0 else "store in HBM"),
+            "position": "the step decodes position T = context - 1 every time (rewriting that row)"}
+
+
 def run_reference(args, rank):
     """The CPU oracle as the reference arm (rank 0 only), on the headline's
     workload: each step one bounded item of the full decode step."""
@@ -523,11 +542,11 @@ def run_reference(args, rank):
               f"linear layers (3+1 bits: selection, LRU step, refined GEMV) or the refined attention of one KV "
               f"head over 16384 tokens; CPU {cpu_model()}")
     line = {
-        "impl": "reference", "metric": "effective HBM GB/s (refined low-bit decode step)", "value": gbs,
+        "impl": "reference", "metric": METRIC, "value": gbs,
         "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * t_tot / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy draws)",
-        "config": {"workload": workload_step(T), "context": T, "layers": args.layers, "batch": 1},
+        "config": step_config(args),
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -1069,25 +1088,12 @@ def run_sf(args, rank, world, local_rank, dist):
     hits, miss = w1["hits"] - w0["hits"], w1["misses"] - w0["misses"]
     khits, kmisses = k1["hits"] - k0["hits"], k1["misses"] - k0["misses"]
     line = {
-        "metric": "effective HBM GB/s (refined low-bit decode step) and tokens/s at 128K", "value": value,
+        "metric": METRIC, "value": value,
         "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded on-device draws; random-init weights and initial context)",
-        "config": {"workload": workload_step(args.context), "model_shape": "Llama-3.1-8B (32 layers, LM head 128256)",
-                   "context": args.context, "layers": args.layers, "batch": 1,
-                   "weights": "3-bit resident + 1-bit refinement, group 128", "kv": "2-bit + 2-bit, per token-head",
-                   "topk_channels": "3% of each GEMV input",
-                   "weight_cache": "10% LRU per matrix, " + ("deadline reading (misses fetched for later steps)"
-                                                              if args.weight_deadline else
-                                                              "every GEMV waits for its misses")
-                   + ("; fetch lead: q/k/v, gate/up and LM-head channels predicted from the residual stream "
-                      "a block ahead and prefetched" if args.fetch_lead and args.weight_deadline else ""),
-                   "topk_tokens": "1% per query head", "kv_cache": (f"{args.kv_cache_pct}% of token-heads, "
-                                                                    f"one LRU per KV head, budget {args.kv_budget} per head and step"
-                                                                    if args.kv_cache_pct >= 0 else "store in HBM"),
-                   "position": "the step decodes position T = context - 1 every time (rewriting that row)",
-                   "l2": "working set > L2, no flush", "parallelism": f"replicas x{world}",
-                   "graph": "CUDA graph per step"},
+        "config": dict(step_config(args), **{"l2": "working set > L2, no flush",
+                                             "parallelism": f"replicas x{world}", "graph": "CUDA graph per step"}),
         "tokens_per_s": world * 1e3 / ms_step,
         "bytes_per_step": nbytes,
         "gpu_memory_gb": (free0 - free1) / 1e9,
