@@ -109,6 +109,11 @@ def parse():
 # the kernel has changed since its last capture.
 ATTN_TRAFFIC_32K = 21377792          # attn_fused_kernel<4>, Hq 32, Hkv 8, T 32768, k 1%
 GEMV_TRAFFIC_PER_LAUNCH = None       # gemv_mma_kernel (changed since its capture)
+# the attention pipeline's four launches of one call (score, listing, ranking,
+# output) at Hq 32, Hkv 8, T 131072, k 1%, from the one-layer step's launch
+# list; ncu flushes the caches between launches, so each reader of the fp32
+# scores counts them from DRAM (in the step they stay in L2)
+ATTN_TRAFFIC_128K = 118992128
 
 
 def gemv_bytes(N, K, k_sel, b_r=B_R, b_f=B_F):
@@ -991,7 +996,9 @@ def run_sf(args, rank, world, local_rank, dist):
         roofline = {"bound": "hbm", "kernel": "attention pipeline (attn_score_mma, attn_compact, attn_select, "
                                               "attn_out)",
                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                    "traffic": None, "peak_source": peak_src, "launch_us": t_attn * 1e6,
+                    "traffic": ATTN_TRAFFIC_128K if (T + 1 == 131072 and model.s.n_q == 32 and model.s.n_kv == 8)
+                    else None,
+                    "peak_source": peak_src, "launch_us": t_attn * 1e6,
                     "bytes_per_launch": attn_b / L}
         del ga
         # the GEMVs of the step (four launches per layer and the LM head), in one graph
