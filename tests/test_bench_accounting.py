@@ -74,3 +74,18 @@ def test_bench_defaults(monkeypatch):
     monkeypatch.setattr("sys.argv", ["bench.py", "--impl", "reference", "--steps", "2", "--warmup", "3"])
     a = bench.parse()
     assert (a.impl, a.steps, a.warmup) == ("reference", 2, 3)
+
+
+def test_both_arms_report_one_metric_and_workload(monkeypatch, capsys):
+    """The reference arm (the CPU oracle) prints the headline's metric name
+    and the same workload config as the library's arm; one step of it runs
+    here, on the host."""
+    import json
+    monkeypatch.setattr("sys.argv", ["bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0"])
+    a = bench.parse()
+    bench.run_reference(a, 0)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["metric"] == bench.METRIC
+    assert line["config"] == bench.step_config(a)
+    assert line["config"]["workload"] == "llama31_8b_decode_step_128k"
+    assert line["impl"] == "reference" and line["e2e"]["h2d_bytes_per_step"] == 0
