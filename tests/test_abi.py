@@ -164,3 +164,29 @@ def test_host_validation_gemv_produce(sf):
     assert call(k=-1) == sf.SF_EINVAL
     assert call(op=sf.PRODUCE_NORM, w=4096, x_out=4096 + 4 * 100) == sf.SF_EINVAL
     assert "x_out" in _err(sf)
+
+
+def test_host_validation_rope_kv_append(sf):
+    """sf_rope_kv_append_pair_cached refuses, on the host and before it
+    touches the cache: a head dim that is not a multiple of 64 (a lane must
+    hold both dims of its pairs), a negative position, theta <= 0, no query
+    heads, and the append's own bad sizes."""
+    L = sf._lib
+    p = ctypes.c_void_p(256)
+    good = dict(Hq=32, Hkv=8, d=128, pos=5, theta=500000.0, S=64, t=3, b_r=2, b_f=2)
+
+    def call(**kw):
+        a = dict(good, **kw)
+        return L.sf_rope_kv_append_pair_cached(p, a["Hq"], None, p, p, a["Hkv"], a["d"], a["pos"],
+                                               ctypes.c_double(a["theta"]), a["S"], a["t"], a["b_r"], a["b_f"],
+                                               p, p, p, p, p, p, p, None, None)
+
+    assert call(d=96) == sf.SF_EINVAL
+    assert "multiple of 64" in _err(sf)
+    assert call(pos=-1) == sf.SF_EINVAL
+    assert call(theta=0.0) == sf.SF_EINVAL
+    assert call(Hq=0) == sf.SF_EINVAL
+    assert call(t=64) == sf.SF_EINVAL
+    assert call(b_r=3, b_f=2) == sf.SF_EINVAL
+    assert L.sf_rope_kv_append_pair_cached(None, 32, None, p, p, 8, 128, 5, ctypes.c_double(1e4), 64, 3, 2, 2,
+                                           p, p, p, p, p, p, p, None, None) == sf.SF_EINVAL
